@@ -1,0 +1,123 @@
+/*
+ * nc_oracle.h -- CPU oracle for the nanochat base-pretraining step.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and the
+ * cpu_baseline / reference legs of bench.py may load this library.  The
+ * product path (pretraining_step_b200/) never links, imports or calls it,
+ * and shares no code, header, table or constant generator with it.
+ *
+ * What it computes: a plain, slow, double-precision restatement of
+ *   - the pre-norm decoder described in the dev.to guide "Como treinar seu
+ *     proprio ChatGPT por 50 dolares", section "1. Modelo GPT
+ *     (nanochat/gpt.py)": RoPE, QK normalisation, untied embedding and
+ *     lm_head, ReLU^2 MLP, causal softmax attention; with the widths that
+ *     --depth selects (section "Filosofia: Um Unico Seletor Para Controlar
+ *     Tudo": model_dim = 64*depth, head_dim 128, MLP 4*model_dim,
+ *     BPE vocabulary 32768 from the "O Que o nanochat Abrange" table);
+ *   - next-token cross-entropy and its gradient by hand-written reverse
+ *     mode;
+ *   - the Muon step of section "2. Otimizador Muon (nanochat/optim.py)":
+ *     momentum, Frobenius normalisation, five quintic Newton-Schulz steps
+ *     in the page's form A = X^T X, B = b*A + c*A*A, X = a*X + X*B, with
+ *     the constant coefficients (a, b, c) = (3.4445, -4.7750, 2.0315).
+ *
+ * Readings of points the pages leave open (each is listed with its reason
+ * in the design notes of the repository):
+ *   RMSNorm eps 1e-6 (also for QK-norm); norms before attention, before
+ *   the MLP and before lm_head; RoPE base 10000, half-split pairs (i, i+64),
+ *   rotation by +theta; QK-norm after RoPE; heads = d/128 (one head of
+ *   width d when d < 128); attention scale 1/sqrt(head_dim); loss = mean
+ *   over all B*T positions; heavy-ball momentum M <- mu*M + G; update
+ *   W <- W - lr*X with no shape scale and no weight decay.
+ *
+ * Parameter layout (the interface both sides follow, in this order):
+ *   0            wte     [V, d]        token embedding
+ *   1 + 6l + 0   wq_l    [d, d]
+ *   1 + 6l + 1   wk_l    [d, d]
+ *   1 + 6l + 2   wv_l    [d, d]
+ *   1 + 6l + 3   wo_l    [d, d]
+ *   1 + 6l + 4   wup_l   [4d, d]
+ *   1 + 6l + 5   wdown_l [d, 4d]
+ *   6L + 1       lm_head [V, d]
+ * Every matrix is row-major [out, in], so y = x * W^T.
+ *
+ * All functions return 0 on success and a negative value on a bad
+ * argument.  No function allocates memory the caller must free.
+ */
+#ifndef NC_ORACLE_H
+#define NC_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Model shape derived from depth (guide, "Filosofia" section).
+ * out[0..5] = {d, n_head, head_dim, mlp_dim, n_params_tensors, n_block_matrices}.
+ * Returns -1 if depth < 1, vocab < 1 or d is not a multiple of head_dim. */
+int oc_dims(int depth, int vocab, int64_t* out);
+
+/* Number of elements of parameter tensor `idx` (layout above), -1 if out of range. */
+int64_t oc_param_numel(int depth, int vocab, int idx);
+
+/* SplitMix64 mixing function (Steele, Lea & Flood, OOPSLA 2014), exposed
+ * so its published test values can be checked. */
+uint64_t oc_splitmix64(uint64_t x);
+
+/* Parameter initialisation from seed, drawing from a counter-based
+ * SplitMix64 stream and the Box-Muller transform.  Element i of tensor t
+ * takes the two words  splitmix64(key_t + 2i)  and  splitmix64(key_t + 2i + 1)
+ * with key_t = splitmix64(seed ^ splitmix64(t + 1)), uniform
+ * u = (word >> 11) * 2^-53, and  z = sqrt(-2 ln(1 - u1)) * cos(2 pi u2).
+ * Weight = z / sqrt(fan_in) (fan_in = in-features; 1 for wte).
+ * spec_zero != 0: wo, wdown and lm_head are zero (the specified init);
+ * spec_zero == 0: every tensor is random, lm_head with std 1/sqrt(d).
+ * params[i] points to caller-owned float storage of oc_param_numel(i). */
+int oc_init_params(int depth, int vocab, uint64_t seed, int spec_zero, float* const* params);
+
+/* Parameter-free RMSNorm over rows: y = x / sqrt(mean(x^2) + eps). rstd may be NULL. */
+int oc_rmsnorm(const double* x, int64_t rows, int cols, double eps, double* y, double* rstd);
+
+/* Rotary embedding of one head-row of width hd at position pos, in place. */
+int oc_rope_row(double* v, int hd, int64_t pos, double base);
+
+/* Causal attention over [B, T, H, hd] tensors (row-major, head-interleaved
+ * exactly like the [B*T, d] activations).  o is [B, T, H, hd]; lse [B, H, T]
+ * (natural log); probs, if not NULL, is [B, H, T, T] with zeros above the
+ * diagonal. */
+int oc_attention(const double* q, const double* k, const double* v, int B, int T, int H, int hd,
+                 double* o, double* lse, double* probs);
+
+/* One layer-free piece used by kernel-level checks: y = x * W^T for
+ * x [rows, k] and W [n, k]. */
+int oc_matmul_nt(const double* x, const double* w, int64_t rows, int64_t n, int64_t k, double* y);
+
+/* Whole-model forward (and backward when grads != NULL).
+ * tokens, targets: [B, T] int32 row-major.  params: layout above (float).
+ * loss: mean next-token cross-entropy (natural log).
+ * grads: same layout, double storage, OVERWRITTEN.
+ * logits: optional [B*T, V] output of the final layer.
+ * Returns -2 if a token or target is out of [0, V). */
+int oc_gpt_fwd_bwd(int depth, int vocab, const float* const* params, const int32_t* tokens,
+                   const int32_t* targets, int B, int T, double* loss, double* const* grads,
+                   double* logits);
+
+/* Newton-Schulz orthogonalisation of one matrix G [rows, cols]:
+ * X = G / (||G||_F + eps_norm), then `steps` iterations of the quintic in
+ * the page's right-hand form on the orientation whose Gram X^T X is the
+ * smaller one (a wide matrix is transposed first and the result transposed
+ * back).  out: [rows, cols]. */
+int oc_newton_schulz(const double* G, int rows, int cols, int steps, double a, double b, double c,
+                     double eps_norm, double* out);
+
+/* Muon update of one block matrix, in place:
+ *   M <- mu*M + G;  O = NS5(M);  W <- W - lr*O.
+ * W, M: [rows, cols] double; G: [rows, cols] double. */
+int oc_muon_update(double* W, double* M, const double* G, int rows, int cols, double lr, double mu);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NC_ORACLE_H */

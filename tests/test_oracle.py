@@ -1,0 +1,418 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: published
+test values, closed forms, invariants, finite differences, or a brute-force
+computation written independently here.  A plausible slip in the oracle (a
+dropped term, a sign, a swapped index or operand) fails at least one.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from pretraining_step_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+V_SMALL = 64
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ------------------------------------------------------------------ RNG, shapes
+def test_splitmix64_published_values():
+    g = _golden("splitmix64.json")
+    for s, o in zip(g["inputs_state_before_step"], g["outputs"]):
+        assert oracle.splitmix64(int(s, 16)) == int(o, 16)
+        assert int(inputs.splitmix64(np.uint64(int(s, 16)))) == int(o, 16)
+
+
+@pytest.mark.parametrize("depth", [4, 12, 20, 26])
+def test_shapes_from_depth(depth):
+    g = _golden("model_pins.json")["depth%d" % depth]
+    s = oracle.dims(depth)
+    assert (s["d"], s["n_head"], s["mlp"], s["head_dim"]) == (g["d"], g["n_head"], g["mlp"], 128)
+    block = sum(oracle.param_numel(depth, i) for i in range(1, 6 * depth + 1))
+    assert block == g["block_params"]
+    if "lm_head_params" in g:
+        assert oracle.param_numel(depth, 6 * depth + 1) == g["lm_head_params"]
+        assert oracle.param_numel(depth, 0) == g["wte_params"]
+
+
+def test_depth_one_has_one_head_of_width_64():
+    s = oracle.dims(1)
+    assert (s["d"], s["n_head"], s["head_dim"]) == (64, 1, 64)
+    with pytest.raises(ValueError):
+        oracle.dims(3)  # d = 192 is not a whole number of 128-wide heads
+
+
+def test_init_statistics_and_zero_pattern():
+    depth = 4
+    P = oracle.init_params(depth, 32768, seed=7, spec_zero=True)
+    shapes = oracle.param_shapes(depth)
+    assert [p.shape for p in P] == shapes
+    for i, p in enumerate(P):
+        if i == len(P) - 1 or (i > 0 and (i - 1) % 6 in (3, 5)):
+            assert not p.any(), "out-projections and lm_head start at zero"
+            continue
+        fan_in = 1 if i == 0 else shapes[i][1]
+        std = fan_in ** -0.5
+        x = p.astype(np.float64) / std
+        n = x.size
+        assert abs(x.mean()) < 5 / math.sqrt(n)
+        assert abs(x.std() - 1) < 6 / math.sqrt(2 * n)
+    # Box-Muller normals: kurtosis 3 and symmetric tails on the big table.
+    x = P[0].astype(np.float64).ravel()
+    k = np.mean(x ** 4) / np.mean(x ** 2) ** 2
+    assert abs(k - 3) < 0.02
+    assert abs(np.mean(x > 1.0) - 0.158655) < 2e-3
+    # Deterministic and seed-dependent.
+    Q = oracle.init_params(depth, 32768, seed=7, spec_zero=True)
+    R = oracle.init_params(depth, 32768, seed=8, spec_zero=True)
+    assert np.array_equal(P[1], Q[1]) and not np.array_equal(P[1], R[1])
+    A = oracle.init_params(depth, 32768, seed=7, spec_zero=False)
+    assert np.array_equal(A[1], P[1]) and A[4].any() and A[-1].any()
+    assert abs(A[-1].std() * math.sqrt(256) - 1) < 0.01
+
+
+# ------------------------------------------------------------------ RMSNorm, RoPE
+def test_rmsnorm_closed_form():
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal((5, 96)) * np.array([[1e-4], [0.1], [1], [10], [1e3]])
+    y, r = oracle.rmsnorm(x)
+    m = np.mean(x * x, axis=1)
+    # mean(y^2) = m / (m + eps) exactly, and y is x scaled per row.
+    np.testing.assert_allclose(np.mean(y * y, axis=1), m / (m + 1e-6), rtol=1e-12)
+    np.testing.assert_allclose(y / x, np.broadcast_to(r[:, None], x.shape), rtol=1e-12)
+    z, _ = oracle.rmsnorm(np.zeros((1, 8)))
+    assert not z.any()
+
+
+def test_rope_two_dim_rotation_is_by_pos_radians():
+    for p in [0, 1, 2, 7, 1000]:
+        v = oracle.rope_row(np.array([1.0, 0.0]), p)
+        np.testing.assert_allclose(v, [math.cos(p), math.sin(p)], atol=1e-15)
+
+
+def test_rope_pairing_and_frequency():
+    hd, p, i = 128, 37, 5
+    e = np.zeros(hd)
+    e[i] = 1.0
+    v = oracle.rope_row(e, p)
+    th = p * 10000.0 ** (-2.0 * i / hd)
+    expect = np.zeros(hd)
+    expect[i], expect[i + 64] = math.cos(th), math.sin(th)
+    np.testing.assert_allclose(v, expect, atol=1e-14)
+
+
+def test_rope_norm_and_relative_position():
+    rng = np.random.default_rng(1)
+    q, k = rng.standard_normal(128), rng.standard_normal(128)
+    assert np.array_equal(oracle.rope_row(q, 0), q)
+    for m, n in [(5, 2), (100, 3), (2047, 2000)]:
+        qm = oracle.rope_row(q, m)
+        assert abs(np.linalg.norm(qm) - np.linalg.norm(q)) < 1e-12
+        a = qm @ oracle.rope_row(k, n)
+        b = oracle.rope_row(q, m + 11) @ oracle.rope_row(k, n + 11)
+        assert abs(a - b) < 1e-11
+
+
+# ------------------------------------------------------------------ attention
+def _brute_attention(q, k, v):
+    B, T, H, hd = q.shape
+    o = np.zeros_like(q)
+    lse = np.zeros((B, H, T))
+    for b in range(B):
+        for h in range(H):
+            s = q[b, :, h, :] @ k[b, :, h, :].T / math.sqrt(hd)
+            s = np.where(np.tril(np.ones((T, T))) > 0, s, -np.inf)
+            mx = s.max(axis=1, keepdims=True)
+            e = np.exp(s - mx)
+            lse[b, h] = (mx[:, 0] + np.log(e.sum(axis=1)))
+            o[b, :, h, :] = (e / e.sum(axis=1, keepdims=True)) @ v[b, :, h, :]
+    return o, lse
+
+
+def test_attention_against_brute_force_and_row_sums():
+    rng = np.random.default_rng(2)
+    q, k, v = (rng.standard_normal((2, 9, 3, 16)) for _ in range(3))
+    o, lse, P = oracle.attention(q, k, v, want_probs=True)
+    ob, lb = _brute_attention(q, k, v)
+    np.testing.assert_allclose(o, ob, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse, lb, rtol=1e-12)
+    np.testing.assert_allclose(P.sum(axis=-1), 1.0, rtol=1e-13)
+    assert not np.triu(P, k=1).any()
+
+
+def test_attention_special_cases():
+    rng = np.random.default_rng(3)
+    v = rng.standard_normal((1, 6, 2, 8))
+    # T = 1: the only key is the query's own position, so o = v.
+    o1, lse1, _ = oracle.attention(v[:, :1], v[:, :1] * 2, v[:, :1])
+    np.testing.assert_allclose(o1, v[:, :1], rtol=1e-14)
+    # q = 0: uniform weights over the causal prefix, o_t = mean(v_0..t), lse = ln(t+1).
+    o, lse, _ = oracle.attention(np.zeros_like(v), rng.standard_normal(v.shape), v)
+    expect = np.cumsum(v, axis=1) / np.arange(1, 7)[None, :, None, None]
+    np.testing.assert_allclose(o, expect, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(lse[0, 0], np.log(np.arange(1, 7)), rtol=1e-14)
+
+
+# ------------------------------------------------------------------ whole model
+def test_loss_at_spec_init_is_ln_vocab_and_gradients_closed_form():
+    depth, B, T = 2, 2, 16
+    g = _golden("model_pins.json")
+    P = oracle.init_params(depth, 32768, seed=3, spec_zero=True)
+    tok, tgt = inputs.token_batch(5, B, T)
+    loss, G, _ = oracle.gpt_fwd_bwd(depth, P, tok, tgt)
+    assert abs(loss - g["ln_vocab"]) < 1e-12
+    assert abs(loss - 15 * math.log(2)) < 1e-12
+    for i in range(len(G) - 1):
+        assert not G[i].any(), "every gradient except lm_head's is exactly zero"
+    # dW_lm = sum_n (1/V - onehot(target_n))^T rms(E[token_n]) / N
+    N, V = B * T, 32768
+    x = P[0][tok.ravel()].astype(np.float64)
+    xf = x / np.sqrt(np.mean(x * x, axis=1, keepdims=True) + 1e-6)
+    expect = np.tile(xf.sum(axis=0) / (V * N), (V, 1))
+    np.subtract.at(expect, tgt.ravel(), xf / N)
+    np.testing.assert_allclose(G[-1], expect, rtol=1e-10, atol=1e-15)
+
+
+def test_loss_near_ln_vocab_with_small_head():
+    depth = 2
+    P = inputs.random_params(depth, seed=4, head_std=1e-4)
+    tok, tgt = inputs.token_batch(6, 1, 32)
+    loss, _, _ = oracle.gpt_fwd_bwd(depth, P, tok, tgt, grads=False)
+    assert abs(loss - math.log(32768)) < 5e-3
+
+
+def test_causality_exact():
+    depth, T, t0 = 2, 10, 6
+    P = inputs.random_params(depth, seed=5, vocab=V_SMALL)
+    tok, tgt = inputs.token_batch(7, 1, T, vocab=V_SMALL)
+    _, _, z0 = oracle.gpt_fwd_bwd(depth, P, tok, tgt, vocab=V_SMALL, grads=False, want_logits=True)
+    tok2 = tok.copy()
+    tok2[0, t0] = (tok2[0, t0] + 1) % V_SMALL
+    _, _, z1 = oracle.gpt_fwd_bwd(depth, P, tok2, tgt, vocab=V_SMALL, grads=False,
+                                  want_logits=True)
+    assert np.array_equal(z0[:t0], z1[:t0]), "positions before t0 must not see token t0"
+    assert not np.allclose(z0[t0:], z1[t0:])
+
+
+def test_accumulation_invariant():
+    """One batch of B rows gives the mean of the gradients of its rows (the
+    single-GPU gradient-accumulation equivalence the pages describe)."""
+    depth, B, T = 1, 4, 8
+    P = inputs.random_params(depth, seed=8, vocab=V_SMALL)
+    tok, tgt = inputs.token_batch(9, B, T, vocab=V_SMALL)
+    loss, G, _ = oracle.gpt_fwd_bwd(depth, P, tok, tgt, vocab=V_SMALL)
+    acc = [np.zeros_like(g) for g in G]
+    tot = 0.0
+    for b in range(B):
+        lb, Gb, _ = oracle.gpt_fwd_bwd(depth, P, tok[b:b + 1], tgt[b:b + 1], vocab=V_SMALL)
+        tot += lb / B
+        for a, g in zip(acc, Gb):
+            a += g / B
+    assert abs(loss - tot) < 1e-12
+    for a, g in zip(acc, G):
+        np.testing.assert_allclose(g, a, rtol=1e-9, atol=1e-13)
+
+
+@pytest.mark.parametrize("depth", [1, 2])
+def test_gradients_central_finite_differences(depth):
+    """Central differences on a depth-1 (one 64-wide head) and a depth-2 (one
+    128-wide head) model at T = 8 and a 64-entry vocabulary, every tensor."""
+    T = 8
+    P = inputs.random_params(depth, seed=10 + depth, vocab=V_SMALL, head_std=0.5)
+    tok, tgt = inputs.token_batch(11, 1, T, vocab=V_SMALL)
+    _, G, _ = oracle.gpt_fwd_bwd(depth, P, tok, tgt, vocab=V_SMALL)
+    rng = np.random.default_rng(12)
+    h = 2.0 ** -12
+    for ti, (p, g) in enumerate(zip(P, G)):
+        scale = np.abs(g).max()
+        assert scale > 0, "tensor %d has an all-zero gradient" % ti
+        # Pick the largest-gradient coordinate plus random ones.
+        picks = [np.unravel_index(np.argmax(np.abs(g)), g.shape)]
+        picks += [tuple(rng.integers(0, s) for s in g.shape) for _ in range(3)]
+        if ti == 0:
+            picks = [(int(tok[0, j]), int(rng.integers(0, p.shape[1]))) for j in range(3)]
+            picks.append(np.unravel_index(np.argmax(np.abs(g)), g.shape))
+        for idx in picks:
+            w0 = p[idx]
+            Pp = [q.copy() for q in P]
+            Pm = [q.copy() for q in P]
+            Pp[ti][idx] = np.float32(w0 + h)
+            Pm[ti][idx] = np.float32(w0 - h)
+            lp, _, _ = oracle.gpt_fwd_bwd(depth, Pp, tok, tgt, vocab=V_SMALL, grads=False)
+            lm, _, _ = oracle.gpt_fwd_bwd(depth, Pm, tok, tgt, vocab=V_SMALL, grads=False)
+            fd = (lp - lm) / (float(Pp[ti][idx]) - float(Pm[ti][idx]))
+            assert abs(fd - g[idx]) <= 2e-5 * scale + 1e-9, (ti, idx, fd, g[idx], scale)
+
+
+# ------------------------------------------------------------------ Newton-Schulz, Muon
+def _f(x, a=3.4445, b=-4.7750, c=2.0315):
+    return a * x + b * x ** 3 + c * x ** 5
+
+
+def _orth(rng, n):
+    q, r = np.linalg.qr(rng.standard_normal((n, n)))
+    return q * np.sign(np.diag(r))
+
+
+@pytest.mark.parametrize("shape", [(24, 24), (16, 40), (40, 16)])
+def test_newton_schulz_acts_on_singular_values_by_the_quintic(shape):
+    m, n = shape
+    k = min(m, n)
+    rng = np.random.default_rng(13)
+    U, Vt = _orth(rng, m)[:, :k], _orth(rng, n)[:k, :]
+    sig = np.geomspace(1.0, 0.01, k)
+    G = (U * sig) @ Vt
+    out = oracle.newton_schulz(G)
+    s = sig / (np.linalg.norm(sig) + 1e-7)
+    for _ in range(5):
+        s = _f(s)
+    np.testing.assert_allclose(out, (U * s) @ Vt, rtol=0, atol=1e-12)
+
+
+def test_newton_schulz_left_and_right_forms_agree():
+    rng = np.random.default_rng(14)
+    for m, n in [(12, 30), (30, 12)]:
+        G = rng.standard_normal((m, n))
+        X = G / (np.linalg.norm(G) + 1e-7)
+        for _ in range(5):
+            A = X @ X.T
+            B = -4.7750 * A + 2.0315 * (A @ A)
+            X = 3.4445 * X + B @ X
+        np.testing.assert_allclose(oracle.newton_schulz(G), X, rtol=0, atol=1e-12)
+
+
+def test_newton_schulz_singular_values_in_band():
+    G = inputs.normal_stack(15, 1, 64, 256, bf16_exact=False)[0]
+    s = np.linalg.svd(oracle.newton_schulz(G), compute_uv=False)
+    assert s.min() > 0.6 and s.max() < 1.21
+
+
+def test_muon_update_momentum_and_apply():
+    rng = np.random.default_rng(16)
+    W, M, G = (rng.standard_normal((20, 48)) for _ in range(3))
+    lr, mu = 0.02, 0.95
+    W1, M1 = oracle.muon_update(W, M, G, lr, mu)
+    np.testing.assert_array_equal(M1, mu * M + G)
+    np.testing.assert_allclose((W - W1) / lr, oracle.newton_schulz(mu * M + G), atol=1e-10)
+
+
+# ------------------------------------------------------------------ forward composition
+def _rms(x):
+    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + 1e-6)
+
+
+def _logits(depth, P, tok, tgt):
+    _, _, z = oracle.gpt_fwd_bwd(depth, P, tok, tgt, vocab=V_SMALL, grads=False, want_logits=True)
+    return z
+
+
+def test_forward_attention_branch_closed_form():
+    """q = k = 0 (zero Wq, Wk) makes attention uniform over the causal prefix
+    and a zero W_up silences the MLP, so one layer reduces to
+    z = rms(x0 + cummean(rms(x0) Wv^T) Wo^T) Wlm^T with x0 = E[tok]."""
+    depth, T = 1, 7
+    P = inputs.random_params(depth, seed=20, vocab=V_SMALL, head_std=0.5)
+    P[1][:] = 0
+    P[2][:] = 0
+    P[5][:] = 0
+    tok, tgt = inputs.token_batch(21, 1, T, vocab=V_SMALL)
+    x0 = P[0][tok[0]].astype(np.float64)
+    v = _rms(x0) @ P[3].astype(np.float64).T
+    o = np.cumsum(v, axis=0) / np.arange(1, T + 1)[:, None]
+    x1 = x0 + o @ P[4].astype(np.float64).T
+    z = _rms(x1) @ P[-1].astype(np.float64).T
+    np.testing.assert_allclose(_logits(depth, P, tok, tgt), z, rtol=1e-11, atol=1e-12)
+
+
+def test_forward_mlp_branch_closed_form():
+    """A zero Wo silences attention, so one layer is
+    z = rms(x0 + relu(rms(x0) Wup^T)^2 Wdown^T) Wlm^T."""
+    depth, T = 1, 5
+    P = inputs.random_params(depth, seed=22, vocab=V_SMALL, head_std=0.5)
+    P[4][:] = 0
+    tok, tgt = inputs.token_batch(23, 1, T, vocab=V_SMALL)
+    x0 = P[0][tok[0]].astype(np.float64)
+    a = np.maximum(_rms(x0) @ P[5].astype(np.float64).T, 0) ** 2
+    x1 = x0 + a @ P[6].astype(np.float64).T
+    z = _rms(x1) @ P[-1].astype(np.float64).T
+    np.testing.assert_allclose(_logits(depth, P, tok, tgt), z, rtol=1e-11, atol=1e-12)
+
+
+def test_forward_two_positions_brute_force():
+    """T = 2, one head, MLP off: the second position mixes two values with
+    weights softmax(q1.k0, q1.k1)/sqrt(hd) after RoPE (positions 0, 1) and
+    QK-norm; written out here from the definitions."""
+    depth = 1
+    P = inputs.random_params(depth, seed=24, vocab=V_SMALL, head_std=0.5)
+    P[5][:] = 0
+    tok, tgt = inputs.token_batch(25, 1, 2, vocab=V_SMALL)
+    Wq, Wk, Wv, Wo = (P[i].astype(np.float64) for i in (1, 2, 3, 4))
+    x0 = P[0][tok[0]].astype(np.float64)
+    h = _rms(x0)
+    q, k, v = h @ Wq.T, h @ Wk.T, h @ Wv.T
+
+    def rot(u, pos):  # pairs (i, i + 32) of a 64-wide head, theta_i = pos * 10000^(-i/32)
+        th = pos * 10000.0 ** (-np.arange(32) / 32.0)
+        a, b = u[:32], u[32:]
+        return np.concatenate([a * np.cos(th) - b * np.sin(th), a * np.sin(th) + b * np.cos(th)])
+
+    qh = [_rms(rot(q[t], t)) for t in range(2)]
+    kh = [_rms(rot(k[t], t)) for t in range(2)]
+    s = np.array([qh[1] @ kh[0], qh[1] @ kh[1]]) / 8.0
+    w = np.exp(s - s.max())
+    w /= w.sum()
+    o = np.stack([v[0], w[0] * v[0] + w[1] * v[1]])
+    z = _rms(x0 + o @ Wo.T) @ P[-1].astype(np.float64).T
+    np.testing.assert_allclose(_logits(depth, P, tok, tgt), z, rtol=1e-11, atol=1e-12)
+
+
+def test_qk_norm_makes_loss_invariant_to_q_k_scale():
+    depth, T = 2, 9
+    P = inputs.random_params(depth, seed=26, vocab=V_SMALL, head_std=0.5)
+    tok, tgt = inputs.token_batch(27, 1, T, vocab=V_SMALL)
+    # Large q and k make the eps inside the norm negligible (relative 1e-10).
+    for i in (1, 2, 7, 8):
+        P[i] *= 100.0
+    l0, _, _ = oracle.gpt_fwd_bwd(depth, P, tok, tgt, vocab=V_SMALL, grads=False)
+    Q = [p.copy() for p in P]
+    Q[1] *= 4.0  # wq of layer 0
+    Q[8] *= 0.5  # wk of layer 1
+    l1, _, _ = oracle.gpt_fwd_bwd(depth, Q, tok, tgt, vocab=V_SMALL, grads=False)
+    assert abs(l0 - l1) < 1e-9
+    Q[3] *= 4.0  # wv is not normalised
+    l2, _, _ = oracle.gpt_fwd_bwd(depth, Q, tok, tgt, vocab=V_SMALL, grads=False)
+    assert abs(l0 - l2) > 1e-4
+
+
+def test_head_and_hidden_permutations_leave_loss_unchanged():
+    depth, T = 4, 6  # d = 256: two heads of 128
+    P = inputs.random_params(depth, seed=28, vocab=V_SMALL, head_std=0.5)
+    tok, tgt = inputs.token_batch(29, 1, T, vocab=V_SMALL)
+    l0, _, _ = oracle.gpt_fwd_bwd(depth, P, tok, tgt, vocab=V_SMALL, grads=False)
+    Q = [p.copy() for p in P]
+    perm_heads = np.concatenate([np.arange(128, 256), np.arange(0, 128)])
+    perm_hidden = np.random.default_rng(30).permutation(1024)
+    for l in range(depth):
+        b = 1 + 6 * l
+        for j in range(3):
+            Q[b + j] = Q[b + j][perm_heads]
+        Q[b + 3] = Q[b + 3][:, perm_heads]
+        Q[b + 4] = Q[b + 4][perm_hidden]
+        Q[b + 5] = Q[b + 5][:, perm_hidden]
+    l1, _, _ = oracle.gpt_fwd_bwd(depth, Q, tok, tgt, vocab=V_SMALL, grads=False)
+    assert abs(l0 - l1) < 1e-10
+    # Mixing a head's halves is not a symmetry: RoPE pairs i with i + 64.
+    R = [p.copy() for p in P]
+    swap = np.concatenate([np.arange(64, 128), np.arange(0, 64), np.arange(128, 256)])
+    R[1], R[2] = R[1][swap], R[2][swap]
+    l2, _, _ = oracle.gpt_fwd_bwd(depth, R, tok, tgt, vocab=V_SMALL, grads=False)
+    assert abs(l0 - l2) > 1e-6
