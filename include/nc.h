@@ -1,0 +1,252 @@
+/*
+ * nc.h -- C ABI of the B200 (sm_100a) nanochat base-pretraining step.
+ *
+ * The step is the one the dev.to guide "Como treinar seu proprio ChatGPT
+ * por 50 dolares" describes for scripts.base_train: forward and backward
+ * of the depth-parametrised GPT of its section "1. Modelo GPT
+ * (nanochat/gpt.py)" under next-token cross-entropy, then the Muon update
+ * of the 2-D block matrices of its section "2. Otimizador Muon
+ * (nanochat/optim.py)".  --depth selects every shape (section "Filosofia:
+ * Um Unico Seletor Para Controlar Tudo"): d = 64*depth, head_dim 128
+ * (one head of width d when d < 128), MLP width 4d; the BPE vocabulary
+ * has 32768 entries (table "O Que o nanochat Abrange").
+ *
+ * Conventions shared by every entry point:
+ *   - Every call returns nc_status; nothing throws or aborts across the ABI.
+ *     On failure nc_last_error() returns a thread-local message.
+ *   - Work is enqueued on the handle's CUDA stream (nc_set_stream; default:
+ *     the legacy default stream).  Calls return before the GPU finishes
+ *     unless stated otherwise.
+ *   - Objects (nc_params, nc_grads) are owned by the library and released
+ *     with the matching *_free.  Pointers passed in are borrowed.
+ *   - "host or device" pointer arguments are classified with
+ *     cudaPointerGetAttributes; host memory is copied in or out on the
+ *     handle's stream.
+ *   - Bounded device waits: a kernel that waits too long on an mbarrier
+ *     records NC_ERR_TIMEOUT in a device status word instead of hanging;
+ *     the next synchronising call returns it and the handle is poisoned.
+ *   - Matrices are row-major [out, in] (y = x W^T).  bf16 is IEEE bfloat16
+ *     with round-to-nearest-even; accumulation is fp32.
+ */
+#ifndef NC_H
+#define NC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NC_OK = 0,
+  NC_ERR_INVALID_ARG = 1, /* bad size, null pointer, unsupported shape      */
+  NC_ERR_OOM = 2,         /* device allocation failed                       */
+  NC_ERR_CUDA = 3,        /* a CUDA runtime call failed                     */
+  NC_ERR_TOKEN_RANGE = 4, /* a token or target id outside [0, vocab)        */
+  NC_ERR_TIMEOUT = 5,     /* a bounded device wait expired; handle poisoned */
+  NC_ERR_UNSUPPORTED = 6  /* valid request this build does not implement    */
+} nc_status;
+
+typedef enum { NC_F32 = 0, NC_BF16 = 1, NC_I32 = 2 } nc_dtype;
+
+typedef struct nc_params nc_params;
+typedef struct nc_grads nc_grads;
+
+/* One parameter or gradient tensor.  data: device pointer of the fp32
+ * storage (parameters: the fp32 master; gradients: the fp32 gradient).
+ * data_bf16: device pointer of the bf16 working copy the kernels read
+ * (NULL for the embedding, which is gathered from the fp32 master). */
+typedef struct {
+  char name[32];
+  int ndim;
+  int64_t shape[2];
+  nc_dtype dtype;
+  void* data;
+  void* data_bf16;
+} nc_tensor_desc;
+
+/* ------------------------------------------------------------------ model */
+
+/* Flags of nc_gpt_init_ex. */
+#define NC_INIT_SPEC 0        /* out-projections (wo, wdown) and lm_head zero */
+#define NC_INIT_ALL_RANDOM 1  /* every tensor random; lm_head std 1/sqrt(d)   */
+
+/* Create a model of the given depth on the current CUDA device and draw its
+ * weights from seed: N(0, 1/fan_in) for every matrix (std 1 for the
+ * embedding), out-projections and lm_head zero (guide, section "1. Modelo
+ * GPT"; the zero out-projections as the workload fixes them).  Normals come
+ * from a counter-based SplitMix64 stream and Box-Muller: element i of
+ * tensor t uses splitmix64(key_t + 2i) and splitmix64(key_t + 2i + 1),
+ * key_t = splitmix64(seed ^ splitmix64(t + 1)).
+ * depth: an even number in [2, 64] (head_dim 128; depth 1, whose single
+ * head is 64 wide, returns NC_ERR_UNSUPPORTED in this build);
+ * vocab: [8, 32768], multiple of 8.
+ * Parameters, Muon momentum (zero) and bf16 copies are allocated here;
+ * activations are allocated by the first nc_gpt_fwd_bwd of a given B*T.
+ * Synchronises the device before returning.
+ * Errors: NC_ERR_INVALID_ARG (depth/vocab), NC_ERR_OOM, NC_ERR_CUDA. */
+nc_status nc_gpt_init(int depth, int vocab, uint64_t seed, nc_params** out);
+nc_status nc_gpt_init_ex(int depth, int vocab, uint64_t seed, int flags, nc_params** out);
+void nc_params_free(nc_params* p);
+
+/* Stream all later work of this handle is enqueued on (a cudaStream_t). */
+nc_status nc_set_stream(nc_params* p, void* cuda_stream);
+
+/* Number of parameter tensors (6*depth + 2) and their descriptors, in the
+ * order: wte [V,d]; per layer wq, wk, wv, wo [d,d], wup [4d,d],
+ * wdown [d,4d]; lm_head [V,d].  wq, wk, wv of a layer are adjacent in
+ * memory (one [3d, d] matrix). */
+int nc_num_tensors(const nc_params* p);
+nc_status nc_tensor_info(const nc_params* p, int idx, nc_tensor_desc* out);
+
+/* Re-derive every bf16 working copy from the fp32 masters (call after
+ * writing masters through nc_tensor_info pointers). */
+nc_status nc_params_sync(nc_params* p);
+
+/* Copy the fp32 master of parameter idx in from `src` or out to `dst`
+ * (host or device pointer, shape[0]*shape[1] floats); writing also
+ * refreshes that tensor's bf16 copy.  Both synchronise the stream.
+ * Errors: NC_ERR_INVALID_ARG (index, null), NC_ERR_CUDA. */
+nc_status nc_tensor_write(nc_params* p, int idx, const float* src);
+nc_status nc_tensor_read(const nc_params* p, int idx, float* dst);
+
+/* Muon momentum buffer of block matrix idx (1 <= idx <= 6*depth), fp32,
+ * copied out to `dst` (host or device).  Synchronises. */
+nc_status nc_momentum_read(const nc_params* p, int idx, float* dst);
+
+/* Gradient buffers (fp32, one per parameter tensor, same order). */
+nc_status nc_grads_create(const nc_params* p, nc_grads** out);
+void nc_grads_free(nc_grads* g);
+nc_status nc_grad_info(const nc_grads* g, int idx, nc_tensor_desc* out);
+/* Copy gradient idx out to `dst` / in from `src` (host or device, fp32).
+ * Writing lets a caller run nc_muon_step on gradients it computed itself.
+ * Both synchronise. */
+nc_status nc_grad_read(const nc_grads* g, int idx, float* dst);
+nc_status nc_grad_write(nc_grads* g, int idx, const float* src);
+
+/* Forward + backward of the whole model on one batch.
+ * tokens, targets: [B, T] int32 row-major, host or device; ids in
+ * [0, vocab).  loss_host: host float, receives the mean next-token
+ * cross-entropy (natural log) over all B*T positions; this call
+ * synchronises the stream to deliver it.  Every gradient in g is
+ * OVERWRITTEN (not accumulated).  T must be >= 1 and B*T <= 2^24;
+ * activations for B*T tokens are (re)allocated on first use.
+ * Errors: NC_ERR_INVALID_ARG, NC_ERR_TOKEN_RANGE (ids are clamped for the
+ * reads, so nothing is read out of bounds), NC_ERR_OOM, NC_ERR_TIMEOUT,
+ * NC_ERR_CUDA. */
+nc_status nc_gpt_fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, int B,
+                         int T, float* loss_host, nc_grads* g);
+
+/* Same, without the synchronisation: the loss is written to loss_dev
+ * (device float) and errors found on the device surface at the next
+ * synchronising call (nc_sync). */
+nc_status nc_gpt_fwd_bwd_async(nc_params* p, const int32_t* tokens, const int32_t* targets, int B,
+                               int T, float* loss_dev, nc_grads* g);
+
+/* Muon step on the 6*depth block matrices (guide, section "2. Otimizador
+ * Muon"): M <- momentum*M + G; X = M / (||M||_F + 1e-7), transposed to
+ * rows <= cols; five Newton-Schulz steps A = X X^T, B = b A + c A A,
+ * X = a X + B X with (a, b, c) = (3.4445, -4.7750, 2.0315) in bf16 with
+ * fp32 accumulation; W <- W - lr * X (transposed back).  The embedding and
+ * lm_head are not touched (the guide gives them to AdamW).  Asynchronous. */
+nc_status nc_muon_step(nc_params* p, const nc_grads* g, float lr, float momentum);
+
+/* Wait for the handle's stream; returns the first device-side error. */
+nc_status nc_sync(nc_params* p);
+
+/* ------------------------------------------------------------------ ops
+ * Single kernels of the step, for kernel-level checks and the
+ * Newton-Schulz sweep.  All pointers are device pointers; all calls are
+ * asynchronous on `stream` (a cudaStream_t, NULL = legacy default). */
+
+/* Epilogues of the GEMM engine. */
+typedef enum {
+  NC_EPI_STORE_BF16 = 0, /* D(bf16) = alpha*acc                               */
+  NC_EPI_STORE_F32 = 1,  /* D(f32)  = alpha*acc                               */
+  NC_EPI_RESID_F32 = 2,  /* D(f32)  = aux(f32) + alpha*acc       (residual)   */
+  NC_EPI_RELU2 = 3,      /* D(bf16) = max(alpha*acc, 0)^2        (ReLU^2)     */
+  NC_EPI_RELU2_BWD = 4,  /* D(bf16) = 2*sqrt(aux(bf16))*alpha*acc (aux = relu(u)^2) */
+  NC_EPI_AXPBY_BF16 = 5, /* D(bf16) = alpha*acc + beta*aux(bf16)              */
+  NC_EPI_ACC_F32 = 6     /* D(f32) += alpha*acc                  (atomic)     */
+} nc_epilogue;
+
+/* Batched GEMM on the tcgen05 tensor cores, D[b] = epi(op(A[b]) op(B[b])^T):
+ *   acc[m, n] = sum_k A(m, k) * B(n, k)
+ * A(m, k) = a_kmajor ? A[m*lda + k] : A[k*lda + m]      (bf16)
+ * B(n, k) = b_kmajor ? B[n*ldb + k] : B[k*ldb + n]      (bf16)
+ * D[m*ldd + n]; aux[m*ldaux + n]; batch strides in elements.
+ * lda, ldb, ldd, ldaux and the batch strides must be multiples of 8
+ * elements, A, B 16-byte aligned.  M, N, K >= 1.  split_k >= 1 splits the
+ * K loop across CTAs (epilogue must be NC_EPI_ACC_F32 when split_k > 1). */
+typedef struct {
+  int M, N, K, batch;
+  const void* A;
+  int64_t lda, stride_a;
+  int a_kmajor;
+  const void* B;
+  int64_t ldb, stride_b;
+  int b_kmajor;
+  void* D;
+  int64_t ldd, stride_d;
+  const void* aux;
+  int64_t ldaux, stride_aux;
+  nc_epilogue epi;
+  float alpha, beta;
+  int split_k;
+} nc_gemm_desc;
+nc_status nc_op_gemm(const nc_gemm_desc* desc, void* stream);
+
+/* Parameter-free RMSNorm: y(bf16) = x(f32) / sqrt(mean(x^2) + 1e-6); rstd(f32). */
+nc_status nc_op_rmsnorm(const float* x, int64_t rows, int cols, void* y_bf16, float* rstd,
+                        void* stream);
+
+/* Causal attention forward on q, k, v (bf16, [B, T, H, 128] rows of stride
+ * ld elements, i.e. slices of the fused [B*T, 3d] qkv activation):
+ * o(bf16) [B, T, H, 128] with row stride ldo; lse (f32, natural log)
+ * [B, H, T].  Scale 1/sqrt(128). */
+nc_status nc_op_attention_fwd(const void* q, const void* k, const void* v, int64_t ld, void* o,
+                              int64_t ldo, float* lse, int B, int T, int H, void* stream);
+
+/* Causal attention backward: from dO (bf16, stride ldo) and the forward's
+ * O, lse: dq (f32, [B,T,H,128] dense, OVERWRITTEN), dk, dv (bf16, stride
+ * ldg).  delta_scratch: f32 [B, H, T] workspace. */
+nc_status nc_op_attention_bwd(const void* q, const void* k, const void* v, int64_t ld,
+                              const void* o, const void* dout, int64_t ldo, const float* lse,
+                              float* dq, void* dk, void* dv, int64_t ldg, float* delta_scratch,
+                              int B, int T, int H, void* stream);
+
+/* Newton-Schulz orthogonalisation of `count` matrices [rows, cols] (bf16
+ * in and out, dense, batch stride rows*cols): Frobenius normalisation
+ * (eps 1e-7) then `steps` quintic steps with the coefficients above, on the
+ * wide orientation (a tall stack is transposed in and out).  scratch:
+ * device workspace of nc_newton_schulz_scratch_bytes() bytes. */
+size_t nc_newton_schulz_scratch_bytes(int count, int rows, int cols);
+nc_status nc_op_newton_schulz(const void* x_bf16, void* out_bf16, int count, int rows, int cols,
+                              int steps, void* scratch, void* stream);
+
+/* ------------------------------------------------------------------ profiling
+ * Per-kernel-class device timing with CUDA events recorded on the launch
+ * stream around every launch while enabled. */
+typedef struct {
+  char name[32];
+  int launches;
+  double total_ms;
+  double flops;  /* algorithmic FLOPs of those launches (tensor kernels) */
+  double bytes;  /* algorithmic HBM bytes of those launches (memory kernels) */
+} nc_kernel_stat;
+nc_status nc_profile_enable(nc_params* p, int on);
+/* Collects (synchronising) and resets the statistics; *n = classes written. */
+nc_status nc_profile_read(nc_params* p, nc_kernel_stat* out, int max, int* n);
+
+/* Kernels launched by this handle since creation (all classes). */
+int64_t nc_launch_count(const nc_params* p);
+
+const char* nc_last_error(void);
+const char* nc_status_string(nc_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NC_H */

@@ -37,6 +37,7 @@ def lib():
         L.oc_rmsnorm.argtypes = [dp, ctypes.c_int64, ctypes.c_int, ctypes.c_double, dp, dp]
         L.oc_rope_row.argtypes = [dp, ctypes.c_int, ctypes.c_int64, ctypes.c_double]
         L.oc_attention.argtypes = [dp, dp, dp] + [ctypes.c_int] * 4 + [dp, dp, dp]
+        L.oc_attention_bwd.argtypes = [dp, dp, dp, dp, dp] + [ctypes.c_int] * 4 + [dp, dp, dp]
         L.oc_matmul_nt.argtypes = [dp, dp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, dp]
         L.oc_gpt_fwd_bwd.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
                                      ctypes.c_void_p, ctypes.c_int, ctypes.c_int, dp,
@@ -116,6 +117,16 @@ def attention(q, k, v, want_probs=False):
     pp = _dp(probs) if want_probs else ctypes.cast(None, ctypes.POINTER(ctypes.c_double))
     assert lib().oc_attention(_dp(q), _dp(k), _dp(v), B, T, H, hd, _dp(o), _dp(lse), pp) == 0
     return o, lse, probs
+
+
+def attention_bwd(q, k, v, lse, dout):
+    """Gradients (dq, dk, dv) of causal attention, layout [B, T, H, hd]."""
+    q, k, v, lse, dout = _f64(q), _f64(k), _f64(v), _f64(lse), _f64(dout)
+    B, T, H, hd = q.shape
+    dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+    assert lib().oc_attention_bwd(_dp(q), _dp(k), _dp(v), _dp(lse), _dp(dout), B, T, H, hd,
+                                  _dp(dq), _dp(dk), _dp(dv)) == 0
+    return dq, dk, dv
 
 
 def matmul_nt(x, w):

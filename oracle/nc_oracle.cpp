@@ -361,6 +361,15 @@ int oc_attention(const double* q, const double* k, const double* v, int B, int T
   return 0;
 }
 
+int oc_attention_bwd(const double* q, const double* k, const double* v, const double* lse,
+                     const double* dout, int B, int T, int H, int hd, double* dq, double* dk,
+                     double* dv) {
+  if (!q || !k || !v || !lse || !dout || !dq || !dk || !dv || B < 0 || T < 0 || H < 1 || hd < 1)
+    return -1;
+  attention_bwd(q, k, v, lse, dout, B, T, H, hd, dq, dk, dv);
+  return 0;
+}
+
 int oc_matmul_nt(const double* x, const double* w, int64_t rows, int64_t n, int64_t k, double* y) {
   if (!x || !w || !y || rows < 0 || n < 0 || k < 0) return -1;
   mm_nt(x, w, rows, n, k, y);

@@ -89,6 +89,12 @@ int oc_rope_row(double* v, int hd, int64_t pos, double base);
 int oc_attention(const double* q, const double* k, const double* v, int B, int T, int H, int hd,
                  double* o, double* lse, double* probs);
 
+/* Reverse mode of oc_attention: from dout [B, T, H, hd] and the forward's
+ * lse, the gradients dq, dk, dv (same layout), OVERWRITTEN. */
+int oc_attention_bwd(const double* q, const double* k, const double* v, const double* lse,
+                     const double* dout, int B, int T, int H, int hd, double* dq, double* dk,
+                     double* dv);
+
 /* One layer-free piece used by kernel-level checks: y = x * W^T for
  * x [rows, k] and W [n, k]. */
 int oc_matmul_nt(const double* x, const double* w, int64_t rows, int64_t n, int64_t k, double* y);

@@ -1,0 +1,304 @@
+"""ctypes binding of libnc_b200.so (the C ABI in include/nc.h).
+
+Argument marshalling only: every step of the computation runs in the
+library's CUDA kernels.  Device buffers may be torch CUDA tensors (their
+data_ptr() is passed) or raw integer device pointers; host buffers are
+numpy arrays.  There is no CPU fallback: if the shared library is missing
+or fails to load, every entry point raises.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnc_b200.so")
+
+NC_OK, NC_ERR_INVALID_ARG, NC_ERR_OOM, NC_ERR_CUDA, NC_ERR_TOKEN_RANGE, NC_ERR_TIMEOUT, \
+    NC_ERR_UNSUPPORTED = range(7)
+NC_INIT_SPEC, NC_INIT_ALL_RANDOM = 0, 1
+(EPI_STORE_BF16, EPI_STORE_F32, EPI_RESID_F32, EPI_RELU2, EPI_RELU2_BWD, EPI_AXPBY_BF16,
+ EPI_ACC_F32) = range(7)
+
+
+class NcError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__("nc status %d: %s" % (status, msg))
+        self.status = status
+
+
+class TensorDesc(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("ndim", ctypes.c_int),
+                ("shape", ctypes.c_int64 * 2), ("dtype", ctypes.c_int),
+                ("data", ctypes.c_void_p), ("data_bf16", ctypes.c_void_p)]
+
+
+class GemmDesc(ctypes.Structure):
+    _fields_ = [("M", ctypes.c_int), ("N", ctypes.c_int), ("K", ctypes.c_int),
+                ("batch", ctypes.c_int),
+                ("A", ctypes.c_void_p), ("lda", ctypes.c_int64), ("stride_a", ctypes.c_int64),
+                ("a_kmajor", ctypes.c_int),
+                ("B", ctypes.c_void_p), ("ldb", ctypes.c_int64), ("stride_b", ctypes.c_int64),
+                ("b_kmajor", ctypes.c_int),
+                ("D", ctypes.c_void_p), ("ldd", ctypes.c_int64), ("stride_d", ctypes.c_int64),
+                ("aux", ctypes.c_void_p), ("ldaux", ctypes.c_int64),
+                ("stride_aux", ctypes.c_int64),
+                ("epi", ctypes.c_int), ("alpha", ctypes.c_float), ("beta", ctypes.c_float),
+                ("split_k", ctypes.c_int)]
+
+
+class KernelStat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int),
+                ("total_ms", ctypes.c_double), ("flops", ctypes.c_double),
+                ("bytes", ctypes.c_double)]
+
+
+_lib = None
+vp = ctypes.c_void_p
+i64 = ctypes.c_int64
+ci = ctypes.c_int
+cf = ctypes.c_float
+
+
+def lib():
+    """Load the library (raises if it was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError("libnc_b200.so is missing: run pretraining_step_b200/build.py "
+                           "(there is no fallback path)")
+    L = ctypes.CDLL(LIB_PATH)
+    sig = {
+        "nc_gpt_init": (ci, [ci, ci, ctypes.c_uint64, ctypes.POINTER(vp)]),
+        "nc_gpt_init_ex": (ci, [ci, ci, ctypes.c_uint64, ci, ctypes.POINTER(vp)]),
+        "nc_params_free": (None, [vp]),
+        "nc_set_stream": (ci, [vp, vp]),
+        "nc_num_tensors": (ci, [vp]),
+        "nc_tensor_info": (ci, [vp, ci, ctypes.POINTER(TensorDesc)]),
+        "nc_tensor_write": (ci, [vp, ci, vp]),
+        "nc_tensor_read": (ci, [vp, ci, vp]),
+        "nc_momentum_read": (ci, [vp, ci, vp]),
+        "nc_params_sync": (ci, [vp]),
+        "nc_grads_create": (ci, [vp, ctypes.POINTER(vp)]),
+        "nc_grads_free": (None, [vp]),
+        "nc_grad_info": (ci, [vp, ci, ctypes.POINTER(TensorDesc)]),
+        "nc_grad_read": (ci, [vp, ci, vp]),
+        "nc_grad_write": (ci, [vp, ci, vp]),
+        "nc_gpt_fwd_bwd": (ci, [vp, vp, vp, ci, ci, ctypes.POINTER(cf), vp]),
+        "nc_gpt_fwd_bwd_async": (ci, [vp, vp, vp, ci, ci, vp, vp]),
+        "nc_muon_step": (ci, [vp, vp, cf, cf]),
+        "nc_sync": (ci, [vp]),
+        "nc_op_gemm": (ci, [ctypes.POINTER(GemmDesc), vp]),
+        "nc_op_rmsnorm": (ci, [vp, i64, ci, vp, vp, vp]),
+        "nc_op_attention_fwd": (ci, [vp, vp, vp, i64, vp, i64, vp, ci, ci, ci, vp]),
+        "nc_op_attention_bwd": (ci, [vp, vp, vp, i64, vp, vp, i64, vp, vp, vp, vp, i64, vp,
+                                     ci, ci, ci, vp]),
+        "nc_newton_schulz_scratch_bytes": (ctypes.c_size_t, [ci, ci, ci]),
+        "nc_op_newton_schulz": (ci, [vp, vp, ci, ci, ci, ci, vp, vp]),
+        "nc_profile_enable": (ci, [vp, ci]),
+        "nc_profile_read": (ci, [vp, ctypes.POINTER(KernelStat), ci, ctypes.POINTER(ci)]),
+        "nc_launch_count": (i64, [vp]),
+        "nc_last_error": (ctypes.c_char_p, []),
+        "nc_status_string": (ctypes.c_char_p, [ci]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = L
+    return L
+
+
+def _check(status):
+    if status != NC_OK:
+        raise NcError(status, lib().nc_last_error().decode())
+
+
+def _ptr(x):
+    """Device pointer of a torch tensor, an int, or None."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if isinstance(x, np.ndarray):
+        return x.ctypes.data
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+# ------------------------------------------------------------------ model
+class GPT:
+    """One model (nc_params) and its gradients (nc_grads)."""
+
+    def __init__(self, depth, vocab=32768, seed=0, all_random=False, stream=None):
+        h = vp()
+        _check(lib().nc_gpt_init_ex(depth, vocab, seed,
+                                    NC_INIT_ALL_RANDOM if all_random else NC_INIT_SPEC,
+                                    ctypes.byref(h)))
+        self.h = h
+        g = vp()
+        st = lib().nc_grads_create(self.h, ctypes.byref(g))
+        if st != NC_OK:
+            lib().nc_params_free(self.h)
+            _check(st)
+        self.g = g
+        self.depth, self.vocab = depth, vocab
+        if stream is not None:
+            self.set_stream(stream)
+
+    def close(self):
+        if getattr(self, "g", None):
+            lib().nc_grads_free(self.g)
+            self.g = None
+        if getattr(self, "h", None):
+            lib().nc_params_free(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def set_stream(self, stream):
+        _check(lib().nc_set_stream(self.h, _stream(stream)))
+
+    def num_tensors(self):
+        return lib().nc_num_tensors(self.h)
+
+    def tensor_info(self, idx):
+        t = TensorDesc()
+        _check(lib().nc_tensor_info(self.h, idx, ctypes.byref(t)))
+        return t
+
+    def shapes(self):
+        return [tuple(self.tensor_info(i).shape) for i in range(self.num_tensors())]
+
+    def write(self, idx, arr):
+        a = np.ascontiguousarray(arr, dtype=np.float32)
+        assert a.shape == tuple(self.tensor_info(idx).shape)
+        _check(lib().nc_tensor_write(self.h, idx, a.ctypes.data))
+
+    def read(self, idx):
+        t = self.tensor_info(idx)
+        out = np.empty(tuple(t.shape), dtype=np.float32)
+        _check(lib().nc_tensor_read(self.h, idx, out.ctypes.data))
+        return out
+
+    def load(self, params):
+        for i, p in enumerate(params):
+            self.write(i, p)
+
+    def params(self):
+        return [self.read(i) for i in range(self.num_tensors())]
+
+    def grad(self, idx):
+        t = self.tensor_info(idx)
+        out = np.empty(tuple(t.shape), dtype=np.float32)
+        _check(lib().nc_grad_read(self.g, idx, out.ctypes.data))
+        return out
+
+    def write_grad(self, idx, arr):
+        a = np.ascontiguousarray(arr, dtype=np.float32)
+        assert a.shape == tuple(self.tensor_info(idx).shape)
+        _check(lib().nc_grad_write(self.g, idx, a.ctypes.data))
+
+    def grads(self):
+        return [self.grad(i) for i in range(self.num_tensors())]
+
+    def momentum(self, idx):
+        t = self.tensor_info(idx)
+        out = np.empty(tuple(t.shape), dtype=np.float32)
+        _check(lib().nc_momentum_read(self.h, idx, out.ctypes.data))
+        return out
+
+    def fwd_bwd(self, tokens, targets):
+        """tokens/targets: numpy int32 [B, T] (host) or torch int32 CUDA tensors."""
+        if isinstance(tokens, np.ndarray):
+            tokens = np.ascontiguousarray(tokens, dtype=np.int32)
+            targets = np.ascontiguousarray(targets, dtype=np.int32)
+        B, T = tokens.shape
+        loss = cf(0)
+        _check(lib().nc_gpt_fwd_bwd(self.h, _ptr(tokens), _ptr(targets), B, T,
+                                    ctypes.byref(loss), self.g))
+        return loss.value
+
+    def fwd_bwd_async(self, tokens, targets, loss_dev):
+        B, T = tokens.shape
+        _check(lib().nc_gpt_fwd_bwd_async(self.h, _ptr(tokens), _ptr(targets), B, T,
+                                          _ptr(loss_dev), self.g))
+
+    def muon_step(self, lr, momentum):
+        _check(lib().nc_muon_step(self.h, self.g, lr, momentum))
+
+    def sync(self):
+        _check(lib().nc_sync(self.h))
+
+    def profile(self, on=True):
+        _check(lib().nc_profile_enable(self.h, 1 if on else 0))
+
+    def profile_read(self):
+        arr = (KernelStat * 64)()
+        n = ci(0)
+        _check(lib().nc_profile_read(self.h, arr, 64, ctypes.byref(n)))
+        return {arr[i].name.decode(): dict(launches=arr[i].launches, ms=arr[i].total_ms,
+                                           flops=arr[i].flops, bytes=arr[i].bytes)
+                for i in range(n.value)}
+
+    def launch_count(self):
+        return int(lib().nc_launch_count(self.h))
+
+
+# ------------------------------------------------------------------ ops
+def gemm(M, N, K, A, B, D, *, lda=None, ldb=None, ldd=None, a_kmajor=True, b_kmajor=True,
+         batch=1, stride_a=0, stride_b=0, stride_d=0, epi=EPI_STORE_BF16, aux=None, ldaux=0,
+         stride_aux=0, alpha=1.0, beta=0.0, split_k=1, stream=None):
+    d = GemmDesc()
+    d.M, d.N, d.K, d.batch = M, N, K, batch
+    d.A, d.B, d.D, d.aux = _ptr(A), _ptr(B), _ptr(D), _ptr(aux)
+    d.lda = lda if lda is not None else (K if a_kmajor else M)
+    d.ldb = ldb if ldb is not None else (K if b_kmajor else N)
+    d.ldd = ldd if ldd is not None else N
+    d.stride_a, d.stride_b, d.stride_d = stride_a, stride_b, stride_d
+    d.a_kmajor, d.b_kmajor = int(bool(a_kmajor)), int(bool(b_kmajor))
+    d.ldaux = ldaux if ldaux else d.ldd
+    d.stride_aux = stride_aux
+    d.epi, d.alpha, d.beta, d.split_k = epi, alpha, beta, split_k
+    _check(lib().nc_op_gemm(ctypes.byref(d), _stream(stream)))
+
+
+def rmsnorm(x, y, rstd, rows, cols, stream=None):
+    _check(lib().nc_op_rmsnorm(_ptr(x), rows, cols, _ptr(y), _ptr(rstd), _stream(stream)))
+
+
+def attention_fwd(q, k, v, ld, o, ldo, lse, B, T, H, stream=None):
+    _check(lib().nc_op_attention_fwd(_ptr(q), _ptr(k), _ptr(v), ld, _ptr(o), ldo, _ptr(lse),
+                                     B, T, H, _stream(stream)))
+
+
+def attention_bwd(q, k, v, ld, o, dout, ldo, lse, dq, dk, dv, ldg, delta, B, T, H,
+                  stream=None):
+    _check(lib().nc_op_attention_bwd(_ptr(q), _ptr(k), _ptr(v), ld, _ptr(o), _ptr(dout), ldo,
+                                     _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), ldg, _ptr(delta),
+                                     B, T, H, _stream(stream)))
+
+
+def newton_schulz_scratch_bytes(count, rows, cols):
+    return int(lib().nc_newton_schulz_scratch_bytes(count, rows, cols))
+
+
+def newton_schulz(x, out, count, rows, cols, steps, scratch, stream=None):
+    _check(lib().nc_op_newton_schulz(_ptr(x), _ptr(out), count, rows, cols, steps,
+                                     _ptr(scratch), _stream(stream)))
+
+
+def status_string(s):
+    return lib().nc_status_string(s).decode()

@@ -1,0 +1,674 @@
+// elementwise.cu -- the memory-bound kernels of the step: embedding gather
+// and scatter-add, RMSNorm forward/backward, RoPE + QK-norm forward/backward,
+// fused softmax cross-entropy (loss and logits gradient in one pass),
+// parameter init, bf16 refresh, and the Muon momentum / normalise / apply
+// passes.  One warp per row where a row reduction is needed (warp-shuffle
+// sums, fp32 statistics), 16-byte vector accesses where rows allow.
+
+#include "common.cuh"
+#include "internal.h"
+#include "kernels.h"
+
+namespace nc {
+namespace {
+
+constexpr float kNormEps = 1e-6f;
+
+// ------------------------------------------------------------------ embedding
+__global__ void embed_gather_kernel(const int32_t* __restrict__ tok, int64_t n, const float* __restrict__ E,
+                                    int V, int d, float* __restrict__ x, int* status) {
+  const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= n) return;
+  int id = tok[w];
+  if (id < 0 || id >= V) {
+    if (lane == 0) atomicExch(status, kDevTokenRange);
+    id = id < 0 ? 0 : V - 1;
+  }
+  const float4* src = reinterpret_cast<const float4*>(E + (int64_t)id * d);
+  float4* dst = reinterpret_cast<float4*>(x + w * d);
+  for (int i = lane; i < d / 4; i += 32) dst[i] = src[i];
+}
+
+__global__ void embed_scatter_kernel(const int32_t* __restrict__ tok, int64_t n, const float* __restrict__ dx,
+                                     int V, int d, float* __restrict__ dE) {
+  const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= n) return;
+  int id = tok[w];
+  id = id < 0 ? 0 : (id >= V ? V - 1 : id);
+  const float4* src = reinterpret_cast<const float4*>(dx + w * d);
+  float* dst = dE + (int64_t)id * d;
+  for (int i = lane; i < d / 4; i += 32) {
+    const float4 g = src[i];
+    atomicAdd(dst + 4 * i + 0, g.x);
+    atomicAdd(dst + 4 * i + 1, g.y);
+    atomicAdd(dst + 4 * i + 2, g.z);
+    atomicAdd(dst + 4 * i + 3, g.w);
+  }
+}
+
+// ------------------------------------------------------------------ RMSNorm
+// y = x / sqrt(mean(x^2) + eps) as bf16, rstd saved; one warp per row.
+__global__ void rmsnorm_fwd_kernel(const float* __restrict__ x, int64_t rows, int d,
+                                   __nv_bfloat16* __restrict__ y, float* __restrict__ rstd) {
+  const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const float4* xr = reinterpret_cast<const float4*>(x + r * d);
+  float ss = 0.f;
+  for (int i = lane; i < d / 4; i += 32) {
+    const float4 v = xr[i];
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  ss = warp_sum(ss);
+  const float rs = rsqrtf(ss / d + kNormEps);
+  uint2* yr = reinterpret_cast<uint2*>(y + r * d);
+  for (int i = lane; i < d / 4; i += 32) {
+    const float4 v = xr[i];
+    uint2 u;
+    u.x = pack_bf16x2(v.x * rs, v.y * rs);
+    u.y = pack_bf16x2(v.z * rs, v.w * rs);
+    yr[i] = u;
+  }
+  if (lane == 0 && rstd) rstd[r] = rs;
+}
+
+// dx = dres + r * (dh - y * mean(dh * y)), y = x * r; fp32 out and a bf16 copy.
+__global__ void rmsnorm_bwd_kernel(const __nv_bfloat16* __restrict__ dh, const float* __restrict__ x,
+                                   const float* __restrict__ rstd, const float* __restrict__ dres,
+                                   int64_t rows, int d, float* __restrict__ dx,
+                                   __nv_bfloat16* __restrict__ dx_bf16) {
+  const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const float rs = rstd[r];
+  const float4* xr = reinterpret_cast<const float4*>(x + r * d);
+  const uint2* gr = reinterpret_cast<const uint2*>(dh + r * d);
+  float dot = 0.f;
+  for (int i = lane; i < d / 4; i += 32) {
+    const float4 v = xr[i];
+    const uint2 u = gr[i];
+    const float2 g0 = unpack_bf16x2(u.x), g1 = unpack_bf16x2(u.y);
+    dot += g0.x * v.x + g0.y * v.y + g1.x * v.z + g1.y * v.w;
+  }
+  dot = warp_sum(dot) * rs;
+  const float m = dot / d;
+  const float4* rr = dres ? reinterpret_cast<const float4*>(dres + r * d) : nullptr;
+  float4* o = reinterpret_cast<float4*>(dx + r * d);
+  uint2* ob = dx_bf16 ? reinterpret_cast<uint2*>(dx_bf16 + r * d) : nullptr;
+  for (int i = lane; i < d / 4; i += 32) {
+    const float4 v = xr[i];
+    const uint2 u = gr[i];
+    const float2 g0 = unpack_bf16x2(u.x), g1 = unpack_bf16x2(u.y);
+    float4 res = rr ? rr[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    res.x += rs * (g0.x - v.x * rs * m);
+    res.y += rs * (g0.y - v.y * rs * m);
+    res.z += rs * (g1.x - v.z * rs * m);
+    res.w += rs * (g1.y - v.w * rs * m);
+    o[i] = res;
+    if (ob) {
+      uint2 w;
+      w.x = pack_bf16x2(res.x, res.y);
+      w.y = pack_bf16x2(res.z, res.w);
+      ob[i] = w;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ RoPE + QK-norm
+// cos/sin table [T][hd/2]: theta_i(pos) = pos * 10000^(-2i/hd), in double.
+__global__ void rope_table_kernel(float2* tab, int T, int hd) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int half = hd / 2;
+  if (i >= (int64_t)T * half) return;
+  const int pos = (int)(i / half), j = (int)(i % half);
+  const double th = (double)pos * pow(10000.0, -2.0 * j / hd);
+  tab[i] = make_float2((float)cos(th), (float)sin(th));
+}
+
+// In place on the q and k slices of qkv [n, ld]: rotate pairs (i, i + hd/2),
+// then RMS-normalise each head; rstd [n, H] per slice.  One warp per
+// (token, head, q|k).
+__global__ void rope_qknorm_fwd_kernel(__nv_bfloat16* __restrict__ qkv, int64_t ld, int64_t n,
+                                       int T, int H, int hd, const float2* __restrict__ tab,
+                                       float* __restrict__ rstd_q, float* __restrict__ rstd_k) {
+  const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= n * H * 2) return;
+  const int which = (int)(w & 1);
+  const int64_t th = w >> 1;
+  const int h = (int)(th % H);
+  const int64_t tok = th / H;
+  const int pos = (int)(tok % T);
+  const int half = hd / 2;
+  __nv_bfloat16* p = qkv + tok * ld + (int64_t)which * H * hd + (int64_t)h * hd;
+  float a[2], b[2];
+  float ss = 0.f;
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int i = lane + 32 * u;
+    a[u] = b[u] = 0.f;
+    if (i < half) {
+      const float2 cs = tab[(int64_t)pos * half + i];
+      const float x0 = bf2f(p[i]), x1 = bf2f(p[i + half]);
+      a[u] = x0 * cs.x - x1 * cs.y;
+      b[u] = x0 * cs.y + x1 * cs.x;
+      ss += a[u] * a[u] + b[u] * b[u];
+    }
+  }
+  ss = warp_sum(ss);
+  const float rs = rsqrtf(ss / hd + kNormEps);
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int i = lane + 32 * u;
+    if (i < half) {
+      p[i] = f2bf(a[u] * rs);
+      p[i + half] = f2bf(b[u] * rs);
+    }
+  }
+  if (lane == 0) (which ? rstd_k : rstd_q)[tok * H + h] = rs;
+}
+
+// Backward of the above for one slice: g = dL/dyhat (f32 dense [n, H*hd] for
+// q, or bf16 with stride ldg for k), yhat the saved normalised output.
+//   dr = r * (g - yhat * mean(g * yhat));   dx = R(-theta) dr.
+// Writes bf16 into out (stride ld_out).
+__global__ void rope_qknorm_bwd_kernel(const float* __restrict__ gf, const __nv_bfloat16* __restrict__ gb,
+                                       int64_t ldg, const __nv_bfloat16* __restrict__ yhat,
+                                       int64_t ldy, const float* __restrict__ rstd, int64_t n,
+                                       int T, int H, int hd, const float2* __restrict__ tab,
+                                       __nv_bfloat16* __restrict__ out, int64_t ld_out) {
+  const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (w >= n * H) return;
+  const int h = (int)(w % H);
+  const int64_t tok = w / H;
+  const int pos = (int)(tok % T);
+  const int half = hd / 2;
+  const __nv_bfloat16* y = yhat + tok * ldy + (int64_t)h * hd;
+  float g0[2], g1[2], y0[2], y1[2];
+  float dot = 0.f;
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int i = lane + 32 * u;
+    g0[u] = g1[u] = y0[u] = y1[u] = 0.f;
+    if (i < half) {
+      if (gf) {
+        const float* gp = gf + tok * ((int64_t)H * hd) + (int64_t)h * hd;
+        g0[u] = gp[i];
+        g1[u] = gp[i + half];
+      } else {
+        const __nv_bfloat16* gp = gb + tok * ldg + (int64_t)h * hd;
+        g0[u] = bf2f(gp[i]);
+        g1[u] = bf2f(gp[i + half]);
+      }
+      y0[u] = bf2f(y[i]);
+      y1[u] = bf2f(y[i + half]);
+      dot += g0[u] * y0[u] + g1[u] * y1[u];
+    }
+  }
+  dot = warp_sum(dot);
+  const float rs = rstd[tok * H + h];
+  const float m = dot / hd;
+  __nv_bfloat16* o = out + tok * ld_out + (int64_t)h * hd;
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int i = lane + 32 * u;
+    if (i < half) {
+      const float d0 = rs * (g0[u] - y0[u] * m), d1 = rs * (g1[u] - y1[u] * m);
+      const float2 cs = tab[(int64_t)pos * half + i];
+      o[i] = f2bf(d0 * cs.x + d1 * cs.y);
+      o[i + half] = f2bf(-d0 * cs.y + d1 * cs.x);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ cross-entropy
+// One CTA (256 threads) per row of logits z[n, V] (bf16, V <= 32768, V % 8 == 0):
+// loss_row = lse(z) - z[target];  z <- (softmax(z) - onehot(target)) * inv_n
+// in place.  The row stays in registers between the two reductions.
+constexpr int kCeThreads = 256;
+constexpr int kCeChunks = 16;  // 16 x 8 bf16 per thread -> V <= 32768
+
+__global__ void __launch_bounds__(kCeThreads) ce_fwd_bwd_kernel(__nv_bfloat16* __restrict__ z,
+                                                                const int32_t* __restrict__ tgt,
+                                                                int V, float inv_n,
+                                                                float* __restrict__ loss_rows,
+                                                                int* status) {
+  __shared__ float red[kCeThreads / 32];
+  __shared__ float s_bcast;
+  __shared__ float s_zt;
+  const int64_t row = blockIdx.x;
+  uint4* zr = reinterpret_cast<uint4*>(z + row * (int64_t)V);
+  const int nchunk = V / 8;
+  int t = tgt[row];
+  if (t < 0 || t >= V) {
+    if (threadIdx.x == 0) atomicExch(status, kDevTokenRange);
+    t = t < 0 ? 0 : V - 1;
+  }
+  if (threadIdx.x == 0) s_zt = bf2f(z[row * (int64_t)V + t]);
+  uint4 buf[kCeChunks];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < kCeChunks; ++c) {
+    const int idx = threadIdx.x + c * kCeThreads;
+    if (idx < nchunk) {
+      buf[c] = zr[idx];
+      const uint32_t* u = reinterpret_cast<const uint32_t*>(&buf[c]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = unpack_bf16x2(u[j]);
+        mx = fmaxf(mx, fmaxf(f.x, f.y));
+      }
+    }
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  mx = warp_max(mx);
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = red[0];
+    for (int i = 1; i < kCeThreads / 32; ++i) m = fmaxf(m, red[i]);
+    s_bcast = m;
+  }
+  __syncthreads();
+  mx = s_bcast;
+  float se = 0.f;
+#pragma unroll
+  for (int c = 0; c < kCeChunks; ++c) {
+    const int idx = threadIdx.x + c * kCeThreads;
+    if (idx < nchunk) {
+      const uint32_t* u = reinterpret_cast<const uint32_t*>(&buf[c]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = unpack_bf16x2(u[j]);
+        se += __expf(f.x - mx) + __expf(f.y - mx);
+      }
+    }
+  }
+  se = warp_sum(se);
+  __syncthreads();
+  if (lane == 0) red[warp] = se;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float s = 0.f;
+    for (int i = 0; i < kCeThreads / 32; ++i) s += red[i];
+    const float lse = mx + logf(s);
+    s_bcast = lse;
+    loss_rows[row] = lse - s_zt;
+  }
+  __syncthreads();
+  const float lse = s_bcast;
+#pragma unroll
+  for (int c = 0; c < kCeChunks; ++c) {
+    const int idx = threadIdx.x + c * kCeThreads;
+    if (idx < nchunk) {
+      const uint32_t* u = reinterpret_cast<const uint32_t*>(&buf[c]);
+      uint4 o;
+      uint32_t* ou = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = unpack_bf16x2(u[j]);
+        const int col = idx * 8 + 2 * j;
+        float p0 = __expf(f.x - lse) - (col == t ? 1.f : 0.f);
+        float p1 = __expf(f.y - lse) - (col + 1 == t ? 1.f : 0.f);
+        ou[j] = pack_bf16x2(p0 * inv_n, p1 * inv_n);
+      }
+      zr[idx] = o;
+    }
+  }
+}
+
+// Deterministic mean of per-row losses (one CTA).
+__global__ void mean_kernel(const float* __restrict__ v, int64_t n, float* out) {
+  __shared__ double red[256];
+  double s = 0;
+  for (int64_t i = threadIdx.x; i < n; i += 256) s += v[i];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int o = 128; o > 0; o >>= 1) {
+    if (threadIdx.x < o) red[threadIdx.x] += red[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *out = (float)(red[0] / (double)n);
+}
+
+// ------------------------------------------------------------------ init
+__device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
+  uint64_t z = x + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// Normal draws by Box-Muller from a counter-based SplitMix64 stream.
+__global__ void init_normal_kernel(float* __restrict__ out, int64_t n, uint64_t key, float stdv) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const uint64_t w1 = splitmix64(key + 2 * (uint64_t)i);
+    const uint64_t w2 = splitmix64(key + 2 * (uint64_t)i + 1);
+    const double u1 = (double)(w1 >> 11) * 0x1.0p-53;
+    const double u2 = (double)(w2 >> 11) * 0x1.0p-53;
+    const double z = sqrt(-2.0 * log(1.0 - u1)) * cos(6.283185307179586476925286766559 * u2);
+    out[i] = (float)(z * stdv);
+  }
+}
+
+__global__ void f32_to_bf16_kernel(const float* __restrict__ in, __nv_bfloat16* __restrict__ out,
+                                   int64_t n) {
+  const int64_t i4 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+  const int64_t base = i4 * 4;
+  if (base + 3 < n) {
+    const float4 v = reinterpret_cast<const float4*>(in)[i4];
+    uint2 u;
+    u.x = pack_bf16x2(v.x, v.y);
+    u.y = pack_bf16x2(v.z, v.w);
+    reinterpret_cast<uint2*>(out)[i4] = u;
+  } else {
+    for (int64_t i = base; i < n; ++i) out[i] = f2bf(in[i]);
+  }
+}
+
+// ------------------------------------------------------------------ Muon
+// Block matrices of layer l live at l * 12 d^2: wq, wk, wv, wo (d x d) at
+// j * d^2, wup (4d x d) at 4 d^2, wdown (d x 4d) at 8 d^2.
+__device__ __forceinline__ void mat_of(int64_t d, int j, int64_t* off, int64_t* size) {
+  const int64_t d2 = d * d;
+  *off = j < 4 ? j * d2 : (j == 4 ? 4 * d2 : 8 * d2);
+  *size = j < 4 ? d2 : 4 * d2;
+}
+
+// M <- mu*M + G over matrix (blockIdx.y = l*6 + j); sumsq[l*6 + j] += ||M||^2.
+__global__ void muon_momentum_kernel(float* __restrict__ M, const float* __restrict__ G, int d,
+                                     float mu, float* __restrict__ sumsq) {
+  const int mat = blockIdx.y;
+  const int l = mat / 6, j = mat % 6;
+  int64_t off, size;
+  mat_of(d, j, &off, &size);
+  off += (int64_t)l * 12 * d * d;
+  float4* m4 = reinterpret_cast<float4*>(M + off);
+  const float4* g4 = reinterpret_cast<const float4*>(G + off);
+  float ss = 0.f;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < size / 4;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float4 m = m4[i];
+    const float4 g = g4[i];
+    m.x = mu * m.x + g.x;
+    m.y = mu * m.y + g.y;
+    m.z = mu * m.z + g.z;
+    m.w = mu * m.w + g.w;
+    m4[i] = m;
+    ss += m.x * m.x + m.y * m.y + m.z * m.z + m.w * m.w;
+  }
+  __shared__ float red[8];
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float s = 0.f;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) s += red[i];
+    atomicAdd(sumsq + mat, s);
+  }
+}
+
+// X = bf16(M / (||M|| + eps)), optionally transposed, 32 x 32 tiles.
+// src matrix (rows x cols, fp32) of layer blockIdx.z at src + z*src_stride;
+// dst (bf16) at dst + z*dst_stride; norm index = z*6 + j.
+__global__ void muon_prep_kernel(const float* __restrict__ src, int64_t src_stride, int rows,
+                                 int cols, int transpose, __nv_bfloat16* __restrict__ dst,
+                                 int64_t dst_stride, const float* __restrict__ sumsq, int j,
+                                 float eps) {
+  __shared__ float tile[32][33];
+  const int z = blockIdx.z;
+  const float inv = 1.f / (sqrtf(sumsq[z * 6 + j]) + eps);
+  const float* s = src + z * src_stride;
+  __nv_bfloat16* dd = dst + z * dst_stride;
+  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    tile[i][threadIdx.x] = (r < rows && c < cols) ? s[(int64_t)r * cols + c] * inv : 0.f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    if (!transpose) {
+      const int r = r0 + i, c = c0 + threadIdx.x;
+      if (r < rows && c < cols) dd[(int64_t)r * cols + c] = f2bf(tile[i][threadIdx.x]);
+    } else {
+      const int r = c0 + i, c = r0 + threadIdx.x;  // dst is cols x rows
+      if (r < cols && c < rows) dd[(int64_t)r * rows + c] = f2bf(tile[threadIdx.x][i]);
+    }
+  }
+}
+
+// W <- W - lr * X^(T), bf16 copy refreshed.  W (rows x cols) per layer z.
+__global__ void muon_apply_kernel(float* __restrict__ W, __nv_bfloat16* __restrict__ Wb,
+                                  int64_t w_stride, int rows, int cols, int transpose,
+                                  const __nv_bfloat16* __restrict__ X, int64_t x_stride,
+                                  float lr) {
+  __shared__ float tile[32][33];
+  const int z = blockIdx.z;
+  float* w = W + z * w_stride;
+  __nv_bfloat16* wb = Wb + z * w_stride;
+  const __nv_bfloat16* x = X + z * x_stride;
+  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+  if (transpose) {
+    // X is cols x rows: stage X[c0.., r0..] then read it transposed.
+    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+      const int xr = c0 + i, xc = r0 + threadIdx.x;
+      tile[i][threadIdx.x] = (xr < cols && xc < rows) ? bf2f(x[(int64_t)xr * rows + xc]) : 0.f;
+    }
+    __syncthreads();
+  }
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < rows && c < cols) {
+      const float u = transpose ? tile[threadIdx.x][i] : bf2f(x[(int64_t)r * cols + c]);
+      const float nw = w[(int64_t)r * cols + c] - lr * u;
+      w[(int64_t)r * cols + c] = nw;
+      wb[(int64_t)r * cols + c] = f2bf(nw);
+    }
+  }
+}
+
+// Frobenius norms of a bf16 stack (count matrices of n elements) for the
+// standalone Newton-Schulz op.
+__global__ void sumsq_bf16_kernel(const __nv_bfloat16* __restrict__ x, int64_t n, float* out) {
+  const __nv_bfloat16* p = x + (int64_t)blockIdx.y * n;
+  float ss = 0.f;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float v = bf2f(p[i]);
+    ss += v * v;
+  }
+  __shared__ float red[8];
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float s = 0.f;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) s += red[i];
+    atomicAdd(out + blockIdx.y, s);
+  }
+}
+
+// y = bf16(x * inv_norm) (optionally transposed), per matrix blockIdx.z.
+__global__ void scale_bf16_kernel(const __nv_bfloat16* __restrict__ x, int rows, int cols,
+                                  int transpose, const float* __restrict__ sumsq, float eps,
+                                  __nv_bfloat16* __restrict__ y) {
+  __shared__ float tile[32][33];
+  const int z = blockIdx.z;
+  const int64_t n = (int64_t)rows * cols;
+  const float inv = sumsq ? 1.f / (sqrtf(sumsq[z]) + eps) : 1.f;
+  const __nv_bfloat16* s = x + z * n;
+  __nv_bfloat16* dd = y + z * n;
+  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int r = r0 + i, c = c0 + threadIdx.x;
+    tile[i][threadIdx.x] = (r < rows && c < cols) ? bf2f(s[(int64_t)r * cols + c]) * inv : 0.f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    if (!transpose) {
+      const int r = r0 + i, c = c0 + threadIdx.x;
+      if (r < rows && c < cols) dd[(int64_t)r * cols + c] = f2bf(tile[i][threadIdx.x]);
+    } else {
+      const int r = c0 + i, c = r0 + threadIdx.x;
+      if (r < cols && c < rows) dd[(int64_t)r * rows + c] = f2bf(tile[threadIdx.x][i]);
+    }
+  }
+}
+
+inline unsigned blocks_for(int64_t threads, int per_block) {
+  return (unsigned)((threads + per_block - 1) / per_block);
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ launchers
+nc_status embed_gather(const int32_t* tok, int64_t n, const float* E, int V, int d, float* x,
+                       int* status, cudaStream_t s, Profiler* prof) {
+  Probe probe(prof, s, "embed_gather", 0.0, n * (8.0 * d + 4.0));
+  embed_gather_kernel<<<blocks_for(n * 32, 256), 256, 0, s>>>(tok, n, E, V, d, x, status);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+nc_status embed_scatter(const int32_t* tok, int64_t n, const float* dx, int V, int d, float* dE,
+                        cudaStream_t s, Profiler* prof) {
+  Probe probe(prof, s, "embed_scatter", 0.0, n * (8.0 * d + 4.0));
+  embed_scatter_kernel<<<blocks_for(n * 32, 256), 256, 0, s>>>(tok, n, dx, V, d, dE);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+nc_status rmsnorm_fwd(const float* x, int64_t rows, int d, void* y, float* rstd, cudaStream_t s,
+                      Profiler* prof) {
+  if (d % 4) return fail(NC_ERR_INVALID_ARG, "rmsnorm: width must be a multiple of 4");
+  Probe probe(prof, s, "rmsnorm_fwd", 0.0, rows * (6.0 * d + 4.0));
+  rmsnorm_fwd_kernel<<<blocks_for(rows * 32, 256), 256, 0, s>>>(x, rows, d, (__nv_bfloat16*)y,
+                                                                 rstd);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+nc_status rmsnorm_bwd(const void* dh, const float* x, const float* rstd, const float* dres,
+                      int64_t rows, int d, float* dx, void* dx_bf16, cudaStream_t s,
+                      Profiler* prof) {
+  Probe probe(prof, s, "rmsnorm_bwd", 0.0,
+              rows * ((2.0 + 4.0 + (dres ? 4.0 : 0.0) + 4.0 + (dx_bf16 ? 2.0 : 0.0)) * d + 4.0));
+  rmsnorm_bwd_kernel<<<blocks_for(rows * 32, 256), 256, 0, s>>>(
+      (const __nv_bfloat16*)dh, x, rstd, dres, rows, d, dx, (__nv_bfloat16*)dx_bf16);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+nc_status rope_table(float2* tab, int T, int hd, cudaStream_t s) {
+  rope_table_kernel<<<blocks_for((int64_t)T * hd / 2, 256), 256, 0, s>>>(tab, T, hd);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+nc_status rope_qknorm_fwd(void* qkv, int64_t ld, int64_t n, int T, int H, int hd,
+                          const float2* tab, float* rstd_q, float* rstd_k, cudaStream_t s,
+                          Profiler* prof) {
+  Probe probe(prof, s, "rope_qknorm_fwd", 0.0, n * H * (2.0 * hd * 2 * 2 + 8.0));
+  rope_qknorm_fwd_kernel<<<blocks_for(n * H * 2 * 32, 256), 256, 0, s>>>(
+      (__nv_bfloat16*)qkv, ld, n, T, H, hd, tab, rstd_q, rstd_k);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+nc_status rope_qknorm_bwd(const float* gf, const void* gb, int64_t ldg, const void* yhat,
+                          int64_t ldy, const float* rstd, int64_t n, int T, int H, int hd,
+                          const float2* tab, void* out, int64_t ld_out, cudaStream_t s,
+                          Profiler* prof) {
+  Probe probe(prof, s, "rope_qknorm_bwd", 0.0, n * H * (hd * ((gf ? 4.0 : 2.0) + 2.0 + 2.0) + 4.0));
+  rope_qknorm_bwd_kernel<<<blocks_for(n * H * 32, 256), 256, 0, s>>>(
+      gf, (const __nv_bfloat16*)gb, ldg, (const __nv_bfloat16*)yhat, ldy, rstd, n, T, H, hd, tab,
+      (__nv_bfloat16*)out, ld_out);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+nc_status ce_fwd_bwd(void* z, const int32_t* tgt, int64_t n, int V, float* loss_rows,
+                     float* loss_out, int* status, cudaStream_t s, Profiler* prof) {
+  if (V % 8 || V > kCeThreads * kCeChunks * 8)
+    return fail(NC_ERR_UNSUPPORTED, "cross-entropy: vocab must be a multiple of 8 and <= 32768");
+  if (n >= (1ll << 31)) return fail(NC_ERR_INVALID_ARG, "cross-entropy: too many rows");
+  {
+    Probe probe(prof, s, "ce_fwd_bwd", 0.0, n * (4.0 * V + 8.0));
+    ce_fwd_bwd_kernel<<<(unsigned)n, kCeThreads, 0, s>>>((__nv_bfloat16*)z, tgt, V,
+                                                          1.0f / (float)n, loss_rows, status);
+    NC_CUDA_TRY(cudaGetLastError());
+  }
+  mean_kernel<<<1, 256, 0, s>>>(loss_rows, n, loss_out);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+nc_status init_normal(float* out, int64_t n, uint64_t key, float stdv, cudaStream_t s) {
+  const unsigned grid = (unsigned)std::min<int64_t>(blocks_for(n, 256), 148 * 16);
+  init_normal_kernel<<<grid, 256, 0, s>>>(out, n, key, stdv);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+nc_status f32_to_bf16(const float* in, void* out, int64_t n, cudaStream_t s, Profiler* prof) {
+  Probe probe(prof, s, "f32_to_bf16", 0.0, n * 6.0);
+  f32_to_bf16_kernel<<<blocks_for((n + 3) / 4, 256), 256, 0, s>>>(in, (__nv_bfloat16*)out, n);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+nc_status muon_momentum(float* M, const float* G, int L, int d, float mu, float* sumsq,
+                        cudaStream_t s, Profiler* prof) {
+  Probe probe(prof, s, "muon_momentum", 0.0, 12.0 * L * (double)d * d * 12.0);
+  dim3 grid(64, 6 * L);
+  muon_momentum_kernel<<<grid, 256, 0, s>>>(M, G, d, mu, sumsq);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+nc_status muon_prep(const float* src, int64_t src_stride, int rows, int cols, int transpose,
+                    void* dst, int64_t dst_stride, const float* sumsq, int j, int L,
+                    cudaStream_t s, Profiler* prof) {
+  Probe probe(prof, s, "muon_prep", 0.0, (double)L * rows * cols * 6.0);
+  dim3 grid((cols + 31) / 32, (rows + 31) / 32, L);
+  muon_prep_kernel<<<grid, dim3(32, 8), 0, s>>>(src, src_stride, rows, cols, transpose,
+                                                (__nv_bfloat16*)dst, dst_stride, sumsq, j, 1e-7f);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+nc_status muon_apply(float* W, void* Wb, int64_t w_stride, int rows, int cols, int transpose,
+                     const void* X, int64_t x_stride, float lr, int L, cudaStream_t s,
+                     Profiler* prof) {
+  Probe probe(prof, s, "muon_apply", 0.0, (double)L * rows * cols * 12.0);
+  dim3 grid((cols + 31) / 32, (rows + 31) / 32, L);
+  muon_apply_kernel<<<grid, dim3(32, 8), 0, s>>>(W, (__nv_bfloat16*)Wb, w_stride, rows, cols,
+                                                 transpose, (const __nv_bfloat16*)X, x_stride, lr);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+nc_status sumsq_bf16(const void* x, int64_t n, int count, float* out, cudaStream_t s,
+                     Profiler* prof) {
+  Probe probe(prof, s, "ns_sumsq", 0.0, (double)count * n * 2.0);
+  dim3 grid((unsigned)std::min<int64_t>(blocks_for(n, 256), 64), count);
+  sumsq_bf16_kernel<<<grid, 256, 0, s>>>((const __nv_bfloat16*)x, n, out);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+nc_status scale_bf16(const void* x, int rows, int cols, int transpose, const float* sumsq,
+                     float eps, void* y, int count, cudaStream_t s, Profiler* prof) {
+  Probe probe(prof, s, "ns_scale", 0.0, (double)count * rows * cols * 4.0);
+  dim3 grid((cols + 31) / 32, (rows + 31) / 32, count);
+  scale_bf16_kernel<<<grid, dim3(32, 8), 0, s>>>((const __nv_bfloat16*)x, rows, cols, transpose,
+                                                 sumsq, eps, (__nv_bfloat16*)y);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+}  // namespace nc

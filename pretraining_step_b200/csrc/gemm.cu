@@ -1,0 +1,526 @@
+// gemm.cu -- the tcgen05 GEMM engine (sm_100a).
+//
+// One persistent CTA per SM walks a list of 128 x BN output tiles.  Warp
+// roles inside the CTA (192 threads):
+//   warp 0      TMA producer: streams 64-wide K slices of A and B into a
+//               STAGES-deep shared-memory ring (128-byte swizzle), one
+//               mbarrier pair (full / empty) per slot;
+//   warp 1      allocates TMEM; one elected thread issues tcgen05.mma
+//               (M = 128, N = BN, K = 16) into a TMEM accumulator and
+//               releases ring slots and accumulators with tcgen05.commit;
+//   warps 2..5  epilogue: tcgen05.ld the accumulator (each thread owns one
+//               row), apply the fused epilogue, store to global memory.
+// The accumulator is double-buffered in TMEM (2 x BN columns), so the
+// epilogue of tile i overlaps the main loop of tile i + 1.
+// Operands may be K-major or MN-major (transposed) independently, which
+// covers y = x W^T, dx = dy W and dW = dy^T x without transposes.
+// Every mbarrier wait is bounded (see tc.cuh); a timeout sets the device
+// status word and every role drains and exits.
+
+#include <algorithm>
+#include <mutex>
+
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace nc {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int kThreads = 192;
+
+template <int BN>
+struct Cfg {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+};
+
+struct Args {
+  int M, N, K, batch;
+  int tiles_m, tiles_n, split_k, kb_per_split, num_kb;
+  int a_mn, b_mn;
+  int epi;
+  float alpha, beta;
+  void* D;
+  int64_t ldd, stride_d;
+  const void* aux;
+  int64_t ldaux, stride_aux;
+  int* status;
+};
+
+struct TileCoord {
+  int b, mb, nb, kb0, kb1;
+};
+
+__device__ __forceinline__ TileCoord decode(const Args& p, int t) {
+  TileCoord c;
+  c.nb = t % p.tiles_n;
+  t /= p.tiles_n;
+  c.mb = t % p.tiles_m;
+  t /= p.tiles_m;
+  const int ks = t % p.split_k;
+  c.b = t / p.split_k;
+  c.kb0 = ks * p.kb_per_split;
+  c.kb1 = min(c.kb0 + p.kb_per_split, p.num_kb);
+  return c;
+}
+
+// Plain bounded wait used while draining after an abort.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  while (!tc::mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > kWaitTimeoutNs) return;
+  }
+}
+
+// ------------------------------------------------------------------ epilogue
+__device__ __forceinline__ void store_row_chunk(const Args& p, int b, int row, int col0,
+                                                const float (&v)[32]) {
+  const int nvalid = min(32, p.N - col0);
+  const bool full = (nvalid == 32);
+  switch (p.epi) {
+    case NC_EPI_STORE_BF16:
+    case NC_EPI_RELU2: {
+      __nv_bfloat16* D = (__nv_bfloat16*)p.D + (int64_t)b * p.stride_d + (int64_t)row * p.ldd + col0;
+      float w[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        float x = v[j] * p.alpha;
+        if (p.epi == NC_EPI_RELU2) {
+          x = fmaxf(x, 0.f);
+          x = x * x;
+        }
+        w[j] = x;
+      }
+      if (full) {
+        uint4* d4 = reinterpret_cast<uint4*>(D);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint4 u;
+          u.x = pack_bf16x2(w[8 * j + 0], w[8 * j + 1]);
+          u.y = pack_bf16x2(w[8 * j + 2], w[8 * j + 3]);
+          u.z = pack_bf16x2(w[8 * j + 4], w[8 * j + 5]);
+          u.w = pack_bf16x2(w[8 * j + 6], w[8 * j + 7]);
+          d4[j] = u;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < nvalid) D[j] = f2bf(w[j]);
+      }
+      break;
+    }
+    case NC_EPI_STORE_F32:
+    case NC_EPI_RESID_F32: {
+      float* D = (float*)p.D + (int64_t)b * p.stride_d + (int64_t)row * p.ldd + col0;
+      const float* R = p.epi == NC_EPI_RESID_F32
+                           ? (const float*)p.aux + (int64_t)b * p.stride_aux +
+                                 (int64_t)row * p.ldaux + col0
+                           : nullptr;
+      if (full) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float4 o = make_float4(v[4 * j] * p.alpha, v[4 * j + 1] * p.alpha,
+                                 v[4 * j + 2] * p.alpha, v[4 * j + 3] * p.alpha);
+          if (R) {
+            const float4 r = reinterpret_cast<const float4*>(R)[j];
+            o.x += r.x;
+            o.y += r.y;
+            o.z += r.z;
+            o.w += r.w;
+          }
+          reinterpret_cast<float4*>(D)[j] = o;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < nvalid) D[j] = v[j] * p.alpha + (R ? R[j] : 0.f);
+      }
+      break;
+    }
+    case NC_EPI_RELU2_BWD:
+    case NC_EPI_AXPBY_BF16: {
+      __nv_bfloat16* D = (__nv_bfloat16*)p.D + (int64_t)b * p.stride_d + (int64_t)row * p.ldd + col0;
+      const __nv_bfloat16* X = (const __nv_bfloat16*)p.aux + (int64_t)b * p.stride_aux +
+                               (int64_t)row * p.ldaux + col0;
+      float x[32];
+      if (full) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint4 u = reinterpret_cast<const uint4*>(X)[j];
+          float2 f;
+          f = unpack_bf16x2(u.x); x[8 * j + 0] = f.x; x[8 * j + 1] = f.y;
+          f = unpack_bf16x2(u.y); x[8 * j + 2] = f.x; x[8 * j + 3] = f.y;
+          f = unpack_bf16x2(u.z); x[8 * j + 4] = f.x; x[8 * j + 5] = f.y;
+          f = unpack_bf16x2(u.w); x[8 * j + 6] = f.x; x[8 * j + 7] = f.y;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] = j < nvalid ? bf2f(X[j]) : 0.f;
+      }
+      float w[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (p.epi == NC_EPI_RELU2_BWD)
+          w[j] = 2.f * sqrtf(fmaxf(x[j], 0.f)) * (v[j] * p.alpha);
+        else
+          w[j] = v[j] * p.alpha + p.beta * x[j];
+      }
+      if (full) {
+        uint4* d4 = reinterpret_cast<uint4*>(D);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint4 u;
+          u.x = pack_bf16x2(w[8 * j + 0], w[8 * j + 1]);
+          u.y = pack_bf16x2(w[8 * j + 2], w[8 * j + 3]);
+          u.z = pack_bf16x2(w[8 * j + 4], w[8 * j + 5]);
+          u.w = pack_bf16x2(w[8 * j + 6], w[8 * j + 7]);
+          d4[j] = u;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < nvalid) D[j] = f2bf(w[j]);
+      }
+      break;
+    }
+    case NC_EPI_ACC_F32: {
+      float* D = (float*)p.D + (int64_t)b * p.stride_d + (int64_t)row * p.ldd + col0;
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (j < nvalid) atomicAdd(D + j, v[j] * p.alpha);
+      break;
+    }
+    default:
+      break;
+  }
+}
+
+// ------------------------------------------------------------------ kernel
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const Args p) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* tfull = empty + C::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drained = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&tfull[i], 1);
+      tc::mbar_init(&tempty[i], 128);
+    }
+    tc::mbar_init(drained, 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int total = p.tiles_m * p.tiles_n * p.split_k * p.batch;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tc::tma_prefetch_desc(&tmA);
+      tc::tma_prefetch_desc(&tmB);
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const TileCoord c = decode(p, t);
+        for (int kb = c.kb0; kb < c.kb1; ++kb) {
+          if (!tc::mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc::mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          uint8_t* a_dst = smem + stage * C::STAGE_BYTES;
+          uint8_t* b_dst = a_dst + C::A_BYTES;
+          const int k0 = kb * BK;
+          if (!p.a_mn) {
+            tc::tma_load_3d(a_dst, &tmA, &full[stage], k0, c.mb * BM, c.b);
+          } else {
+            tc::tma_load_3d(a_dst, &tmA, &full[stage], c.mb * BM, k0, c.b);
+            tc::tma_load_3d(a_dst + 8192, &tmA, &full[stage], c.mb * BM + 64, k0, c.b);
+          }
+          if (!p.b_mn) {
+            tc::tma_load_3d(b_dst, &tmB, &full[stage], k0, c.nb * BN, c.b);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tc::tma_load_3d(b_dst + j * 8192, &tmB, &full[stage], c.nb * BN + 64 * j, k0, c.b);
+          }
+          ++issued;
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // Let the copies already in flight land before the CTA exits.
+        int s = stage;
+        uint32_t ph = phase;
+        for (int i = 0; i < min(issued, C::STAGES); ++i) {
+          if (--s < 0) {
+            s = C::STAGES - 1;
+            ph ^= 1;
+          }
+          drain_wait(&full[s], ph);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_bf16_f32(BM, BN, p.a_mn, p.b_mn);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const TileCoord c = decode(p, t);
+        if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = c.kb0; kb < c.kb1; ++kb) {
+          if (!tc::mbar_wait(&full[stage], phase, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc::tc_fence_after();
+          const uint32_t a_base = tc::smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t b_base = a_base + C::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = p.a_mn ? tc::smem_desc_sw128(a_base + kk * 2048, 8192, 1024)
+                                       : tc::smem_desc_sw128(a_base + kk * 32, 16, 1024);
+            const uint64_t bd = p.b_mn ? tc::smem_desc_sw128(b_base + kk * 2048, 8192, 1024)
+                                       : tc::smem_desc_sw128(b_base + kk * 32, 16, 1024);
+            tc::umma_bf16_ss(d_tmem, ad, bd, idesc, (kb > c.kb0 || kk > 0) ? 1u : 0u);
+          }
+          tc::umma_commit(&empty[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        tc::umma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+      // Wait for every issued MMA before TMEM is released.
+      tc::umma_commit(drained);
+      drain_wait(drained, 0);
+    }
+  } else {
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row_in_tile = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      const TileCoord c = decode(p, t);
+      if (!tc::mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status)) break;
+      tc::tc_fence_after();
+      const int row = c.mb * BM + row_in_tile;
+#pragma unroll 1
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        uint32_t r[32];
+        tc::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + ch * 32, r);
+        tc::tmem_ld_wait();
+        const int col0 = c.nb * BN + ch * 32;
+        if (row < p.M && col0 < p.N) {
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          store_row_chunk(p, c.b, row, col0, v);
+        }
+      }
+      tc::tc_fence_before();
+      tc::mbar_arrive(&tempty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 3-D bf16 tensor map {inner, outer, batch}, row stride ld and batch stride
+// in elements, box {64, box_outer, 1}, 128-byte swizzle, zero fill.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t batch,
+              int64_t ld, int64_t bstride, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, outer, batch};
+  cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)(batch > 1 ? bstride : ld * outer) * 2};
+  cuuint32_t box[3] = {64, box_outer, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN>
+nc_status launch_bn(const nc_gemm_desc& d, int split, int* status, cudaStream_t s,
+                    Profiler* prof) {
+  using C = Cfg<BN>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    NC_CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+    attr_set = true;
+  }
+  CUtensorMap ta, tb;
+  const bool ok_a = d.a_kmajor ? make_map(&ta, d.A, d.K, d.M, d.batch, d.lda, d.stride_a, BM)
+                               : make_map(&ta, d.A, d.M, d.K, d.batch, d.lda, d.stride_a, 64);
+  const bool ok_b = d.b_kmajor ? make_map(&tb, d.B, d.K, d.N, d.batch, d.ldb, d.stride_b, BN)
+                               : make_map(&tb, d.B, d.N, d.K, d.batch, d.ldb, d.stride_b, 64);
+  if (!ok_a || !ok_b) return fail(NC_ERR_INVALID_ARG, "gemm: cuTensorMapEncodeTiled rejected an operand");
+
+  Args a;
+  a.M = d.M;
+  a.N = d.N;
+  a.K = d.K;
+  a.batch = d.batch;
+  a.tiles_m = (d.M + BM - 1) / BM;
+  a.tiles_n = (d.N + BN - 1) / BN;
+  a.num_kb = (d.K + BK - 1) / BK;
+  a.kb_per_split = (a.num_kb + split - 1) / split;
+  a.split_k = (a.num_kb + a.kb_per_split - 1) / a.kb_per_split;
+  a.a_mn = d.a_kmajor ? 0 : 1;
+  a.b_mn = d.b_kmajor ? 0 : 1;
+  a.epi = d.epi;
+  a.alpha = d.alpha;
+  a.beta = d.beta;
+  a.D = d.D;
+  a.ldd = d.ldd;
+  a.stride_d = d.stride_d;
+  a.aux = d.aux;
+  a.ldaux = d.ldaux;
+  a.stride_aux = d.stride_aux;
+  a.status = status;
+  const int64_t total = (int64_t)a.tiles_m * a.tiles_n * a.split_k * a.batch;
+  if (total >= (1ll << 31)) return fail(NC_ERR_INVALID_ARG, "gemm: too many tiles");
+  const int grid = (int)std::min<int64_t>(total, num_sms());
+  const double flops = 2.0 * d.M * (double)d.N * d.K * d.batch;
+  Probe probe(prof, s, "gemm_tc", flops, 0.0);
+  gemm_tc_kernel<BN><<<grid, kThreads, C::SMEM_BYTES, s>>>(ta, tb, a);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+// Smallest split that keeps the last wave at least 85% full (or 16).
+int auto_split(int64_t tiles, int num_kb) {
+  const int sms = num_sms();
+  int best = 1;
+  double best_eff = 0;
+  for (int s = 1; s <= 16; ++s) {
+    if (s > 1 && num_kb / s < 8) break;
+    const int64_t t = tiles * s;
+    const double eff = (double)t / (double)(((t + sms - 1) / sms) * sms);
+    if (eff > best_eff + 0.02) {
+      best_eff = eff;
+      best = s;
+    }
+    if (eff >= 0.85) break;
+  }
+  return best;
+}
+
+}  // namespace
+
+nc_status gemm_launch(const GemmLaunch& g, cudaStream_t s, Profiler* prof) {
+  const nc_gemm_desc& d = g.d;
+  if (d.M < 1 || d.N < 1 || d.K < 1 || d.batch < 1 || !d.A || !d.B || !d.D)
+    return fail(NC_ERR_INVALID_ARG, "gemm: empty shape or null operand");
+  auto aligned = [](int64_t v) { return v % 8 == 0; };
+  if (!aligned(d.lda) || !aligned(d.ldb) || (d.batch > 1 && (!aligned(d.stride_a) || !aligned(d.stride_b))))
+    return fail(NC_ERR_INVALID_ARG, "gemm: leading dimensions and batch strides must be multiples of 8");
+  if ((reinterpret_cast<uintptr_t>(d.A) | reinterpret_cast<uintptr_t>(d.B)) & 15)
+    return fail(NC_ERR_INVALID_ARG, "gemm: operands must be 16-byte aligned");
+  const bool needs_aux = d.epi == NC_EPI_RESID_F32 || d.epi == NC_EPI_RELU2_BWD ||
+                         d.epi == NC_EPI_AXPBY_BF16;
+  if (needs_aux && (!d.aux || !aligned(d.ldaux)))
+    return fail(NC_ERR_INVALID_ARG, "gemm: epilogue needs an aux operand with ld multiple of 8");
+  if (!aligned(d.ldd) || (reinterpret_cast<uintptr_t>(d.D) & 15) ||
+      (needs_aux && (reinterpret_cast<uintptr_t>(d.aux) & 15)))
+    return fail(NC_ERR_INVALID_ARG, "gemm: output / aux must be 16-byte aligned rows");
+  if (d.epi < NC_EPI_STORE_BF16 || d.epi > NC_EPI_ACC_F32)
+    return fail(NC_ERR_INVALID_ARG, "gemm: unknown epilogue");
+  int split = d.split_k;
+  if (split != 1 && d.epi != NC_EPI_ACC_F32)
+    return fail(NC_ERR_INVALID_ARG, "gemm: split_k > 1 needs the accumulate epilogue");
+  // N tile: 256 unless 128 wastes less of the last column tile.
+  const int waste256 = ((d.N + 255) / 256) * 256 - d.N;
+  const int waste128 = ((d.N + 127) / 128) * 128 - d.N;
+  const bool bn256 = d.N > 128 && waste256 <= waste128;
+  const int bn = bn256 ? 256 : 128;
+  const int num_kb = (d.K + BK - 1) / BK;
+  if (split <= 0) {
+    const int64_t tiles = (int64_t)((d.M + BM - 1) / BM) * ((d.N + bn - 1) / bn) * d.batch;
+    split = auto_split(tiles, num_kb);
+  }
+  if (split > num_kb) split = num_kb;
+  return bn256 ? launch_bn<256>(d, split, g.status, s, prof)
+               : launch_bn<128>(d, split, g.status, s, prof);
+}
+
+}  // namespace nc

@@ -1,0 +1,49 @@
+// internal.h -- host-side interfaces between the translation units of the
+// step library (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "../../include/nc.h"
+
+namespace nc {
+
+// Thread-local error message behind nc_last_error().
+void set_error(const std::string& msg);
+nc_status fail(nc_status s, const std::string& msg);
+nc_status cuda_fail(cudaError_t e, const char* what);
+
+#define NC_CUDA_TRY(expr)                                     \
+  do {                                                        \
+    cudaError_t _e = (expr);                                  \
+    if (_e != cudaSuccess) return ::nc::cuda_fail(_e, #expr); \
+  } while (0)
+
+#define NC_TRY(expr)                   \
+  do {                                 \
+    nc_status _s = (expr);             \
+    if (_s != NC_OK) return _s;        \
+  } while (0)
+
+int num_sms();
+
+// Per-kernel-class timing (profile.cpp).  Every launch site wraps its launch
+// in a Probe; with profiling off it only counts the launch.
+struct Profiler;
+struct Probe {
+  Probe(Profiler* prof, cudaStream_t s, const char* name, double flops, double bytes);
+  ~Probe();
+  Profiler* prof;
+  cudaStream_t stream;
+  int slot;
+};
+Profiler* profiler_create();
+void profiler_destroy(Profiler*);
+void profiler_enable(Profiler*, bool on);
+nc_status profiler_read(Profiler*, nc_kernel_stat* out, int max, int* n);
+int64_t profiler_launches(const Profiler*);
+
+}  // namespace nc

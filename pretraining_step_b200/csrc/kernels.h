@@ -1,0 +1,67 @@
+// kernels.h -- launchers of the device kernels (host side).  Pointers are
+// device pointers; bf16 tensors are passed as void*.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "internal.h"
+
+namespace nc {
+
+struct GemmLaunch {
+  nc_gemm_desc d;
+  int* status;  // device status word (may be null)
+};
+// d.split_k == 0 selects the split automatically (NC_EPI_ACC_F32 only).
+nc_status gemm_launch(const GemmLaunch& g, cudaStream_t s, Profiler* prof);
+
+nc_status attention_fwd(const void* q, const void* k, const void* v, int64_t ld, void* o,
+                        int64_t ldo, float* lse, int B, int T, int H, cudaStream_t s,
+                        Profiler* prof);
+nc_status attention_bwd(const void* q, const void* k, const void* v, int64_t ld, const void* o,
+                        const void* dout, int64_t ldo, const float* lse, float* dq, void* dk,
+                        void* dv, int64_t ldg, float* delta, int B, int T, int H, cudaStream_t s,
+                        Profiler* prof);
+
+nc_status embed_gather(const int32_t* tok, int64_t n, const float* E, int V, int d, float* x,
+                       int* status, cudaStream_t s, Profiler* prof);
+nc_status embed_scatter(const int32_t* tok, int64_t n, const float* dx, int V, int d, float* dE,
+                        cudaStream_t s, Profiler* prof);
+nc_status rmsnorm_fwd(const float* x, int64_t rows, int d, void* y, float* rstd, cudaStream_t s,
+                      Profiler* prof);
+nc_status rmsnorm_bwd(const void* dh, const float* x, const float* rstd, const float* dres,
+                      int64_t rows, int d, float* dx, void* dx_bf16, cudaStream_t s,
+                      Profiler* prof);
+nc_status rope_table(float2* tab, int T, int hd, cudaStream_t s);
+nc_status rope_qknorm_fwd(void* qkv, int64_t ld, int64_t n, int T, int H, int hd,
+                          const float2* tab, float* rstd_q, float* rstd_k, cudaStream_t s,
+                          Profiler* prof);
+nc_status rope_qknorm_bwd(const float* gf, const void* gb, int64_t ldg, const void* yhat,
+                          int64_t ldy, const float* rstd, int64_t n, int T, int H, int hd,
+                          const float2* tab, void* out, int64_t ld_out, cudaStream_t s,
+                          Profiler* prof);
+nc_status ce_fwd_bwd(void* z, const int32_t* tgt, int64_t n, int V, float* loss_rows,
+                     float* loss_out, int* status, cudaStream_t s, Profiler* prof);
+nc_status init_normal(float* out, int64_t n, uint64_t key, float stdv, cudaStream_t s);
+nc_status f32_to_bf16(const float* in, void* out, int64_t n, cudaStream_t s, Profiler* prof);
+nc_status muon_momentum(float* M, const float* G, int L, int d, float mu, float* sumsq,
+                        cudaStream_t s, Profiler* prof);
+nc_status muon_prep(const float* src, int64_t src_stride, int rows, int cols, int transpose,
+                    void* dst, int64_t dst_stride, const float* sumsq, int j, int L,
+                    cudaStream_t s, Profiler* prof);
+nc_status muon_apply(float* W, void* Wb, int64_t w_stride, int rows, int cols, int transpose,
+                     const void* X, int64_t x_stride, float lr, int L, cudaStream_t s,
+                     Profiler* prof);
+nc_status sumsq_bf16(const void* x, int64_t n, int count, float* out, cudaStream_t s,
+                     Profiler* prof);
+nc_status scale_bf16(const void* x, int rows, int cols, int transpose, const float* sumsq,
+                     float eps, void* y, int count, cudaStream_t s, Profiler* prof);
+
+// Newton-Schulz on a wide bf16 stack X[count][m][n] (m <= n), in place in
+// x0 (result lands back in x0); ws: 2*count*m*m + count*m*n bf16 elements.
+nc_status newton_schulz_wide(void* x0, int count, int m, int n, int steps, void* ws,
+                             int* status, cudaStream_t s, Profiler* prof);
+
+}  // namespace nc

@@ -1,0 +1,775 @@
+// step.cu -- the step driver behind the C ABI: parameter / gradient /
+// activation storage, the forward + backward sequence of the depth-L GPT,
+// the Muon step, and the op-level entry points.
+//
+// Model (dev.to guide "Como treinar seu proprio ChatGPT por 50 dolares",
+// section "1. Modelo GPT"):  x0 = wte[tok];  per layer
+//   h1 = rms(x);  [q k v] = h1 [wq wk wv]^T;  q, k <- rms_head(rope(.));
+//   o = causal_attention(q, k, v);  x <- x + o wo^T;
+//   h2 = rms(x);  a = relu(h2 wup^T)^2;  x <- x + a wdown^T;
+// then z = rms(x) lm_head^T and loss = mean(lse(z) - z[target]).
+// Residual stream and every row statistic are fp32; GEMM operands are bf16
+// with fp32 accumulation in TMEM.
+//
+// Memory layout in HBM (one allocation per role):
+//   wte [V,d] f32;  blocks [L][12 d^2] f32 masters + bf16 copies, layer l at
+//   l*12d^2: wq | wk | wv (one [3d,d] matrix) | wo | wup [4d,d] | wdown [d,4d];
+//   lm_head [V,d] f32 + bf16;  Muon momentum like blocks (f32).
+//   Activations per B*T tokens: x_0..x_L and the mid-layer residuals (f32),
+//   h1, h2, qkv, o, a (bf16), row statistics (f32), logits [N,V] bf16
+//   (overwritten in place by their gradient), backward scratch.
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <utility>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nc {
+
+// ------------------------------------------------------------------ errors
+static thread_local std::string g_last_error;
+void set_error(const std::string& msg) { g_last_error = msg; }
+nc_status fail(nc_status s, const std::string& msg) {
+  g_last_error = msg;
+  return s;
+}
+nc_status cuda_fail(cudaError_t e, const char* what) {
+  g_last_error = std::string(what) + ": " + cudaGetErrorString(e);
+  return e == cudaErrorMemoryAllocation ? NC_ERR_OOM : NC_ERR_CUDA;
+}
+
+int num_sms() {
+  static int n = 0;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+  });
+  return n;
+}
+
+namespace {
+
+typedef __nv_bfloat16 bf16;
+
+// Bump allocator over one cudaMalloc.
+struct Arena {
+  char* base = nullptr;
+  size_t size = 0, used = 0;
+  template <class T>
+  T* take(int64_t n) {
+    const size_t bytes = ((size_t)n * sizeof(T) + 255) & ~size_t(255);
+    T* p = reinterpret_cast<T*>(base + used);
+    used += bytes;
+    return p;
+  }
+};
+
+struct Acts {
+  int64_t N = 0;
+  int B = 0, T = 0;
+  void* mem = nullptr;
+  int32_t *tok = nullptr, *tgt = nullptr;
+  std::vector<float*> x, xmid, r1, r2, rq, rk, lse;
+  std::vector<bf16*> h1, h2, qkv, o, a;
+  bf16 *hf = nullptr, *logits = nullptr, *dxb = nullptr, *dh = nullptr, *du = nullptr,
+       *dqkv = nullptr;
+  float *rf = nullptr, *loss_rows = nullptr, *loss = nullptr, *dx0 = nullptr, *dx1 = nullptr,
+        *dq = nullptr, *delta = nullptr;
+};
+
+}  // namespace
+}  // namespace nc
+
+struct nc_params {
+  int depth = 0, vocab = 0, d = 0, H = 0, hd = 0, F = 0;
+  cudaStream_t stream = nullptr;
+  nc::Profiler* prof = nullptr;
+  int* status = nullptr;  // device status word
+  bool poisoned = false;
+  void* pmem = nullptr;
+  float *wte = nullptr, *blocks = nullptr, *lm = nullptr, *mom = nullptr;
+  nc::bf16 *blocks_b = nullptr, *lm_b = nullptr;
+  // Muon
+  float* sumsq = nullptr;
+  nc::bf16 *xsq = nullptr, *xw = nullptr, *nsws = nullptr;
+  // RoPE table
+  float2* rope = nullptr;
+  int rope_T = 0;
+  nc::Acts act;
+  // pinned host staging for loss + status
+  float* h_loss = nullptr;
+  int* h_status = nullptr;
+};
+
+struct nc_grads {
+  const nc_params* p = nullptr;
+  void* mem = nullptr;
+  float *wte = nullptr, *blocks = nullptr, *lm = nullptr;
+};
+
+namespace nc {
+namespace {
+
+int64_t block_elems(const nc_params* p) { return 12ll * p->depth * p->d * p->d; }
+
+// Offset and shape of parameter tensor idx (interface order).
+void tensor_layout(const nc_params* p, int idx, int64_t* off, int64_t* rows, int64_t* cols,
+                   const char** name, int* layer) {
+  const int64_t d = p->d, d2 = d * d;
+  const int n = 6 * p->depth + 2;
+  *layer = -1;
+  if (idx == 0) {
+    *off = 0; *rows = p->vocab; *cols = d; *name = "wte";
+  } else if (idx == n - 1) {
+    *off = 0; *rows = p->vocab; *cols = d; *name = "lm_head";
+  } else {
+    const int l = (idx - 1) / 6, j = (idx - 1) % 6;
+    static const char* names[6] = {"wq", "wk", "wv", "wo", "wup", "wdown"};
+    *layer = l;
+    *name = names[j];
+    *off = l * 12 * d2 + (j < 4 ? j * d2 : (j == 4 ? 4 * d2 : 8 * d2));
+    *rows = (j == 4) ? 4 * d : d;
+    *cols = (j == 5) ? 4 * d : d;
+  }
+}
+
+nc_status check_status(nc_params* p) {
+  // Called after a synchronisation that copied the status word.
+  const int st = *p->h_status;
+  if (st == kDevOk) return NC_OK;
+  if (st == kDevTimeout) {
+    p->poisoned = true;
+    return fail(NC_ERR_TIMEOUT, "a device wait timed out; the handle is poisoned");
+  }
+  if (st == kDevTokenRange) return fail(NC_ERR_TOKEN_RANGE, "token or target id out of [0, vocab)");
+  return fail(NC_ERR_CUDA, "unknown device status");
+}
+
+nc_status sync_and_check(nc_params* p, const float* loss_dev) {
+  if (loss_dev)
+    NC_CUDA_TRY(cudaMemcpyAsync(p->h_loss, loss_dev, sizeof(float), cudaMemcpyDeviceToHost,
+                                p->stream));
+  NC_CUDA_TRY(cudaMemcpyAsync(p->h_status, p->status, sizeof(int), cudaMemcpyDeviceToHost,
+                              p->stream));
+  NC_CUDA_TRY(cudaStreamSynchronize(p->stream));
+  nc_status s = check_status(p);
+  if (*p->h_status == kDevTokenRange) {
+    NC_CUDA_TRY(cudaMemsetAsync(p->status, 0, sizeof(int), p->stream));
+    NC_CUDA_TRY(cudaStreamSynchronize(p->stream));
+  }
+  return s;
+}
+
+nc_status ensure_rope(nc_params* p, int T) {
+  if (p->rope_T >= T) return NC_OK;
+  int newT = std::max(T, 2048);
+  if (p->rope) cudaFree(p->rope);
+  p->rope = nullptr;
+  NC_CUDA_TRY(cudaMalloc(&p->rope, sizeof(float2) * (size_t)newT * (p->hd / 2)));
+  NC_TRY(rope_table(p->rope, newT, p->hd, p->stream));
+  p->rope_T = newT;
+  return NC_OK;
+}
+
+nc_status ensure_acts(nc_params* p, int B, int T) {
+  Acts& a = p->act;
+  const int64_t N = (int64_t)B * T;
+  if (a.mem && a.N == N && a.B == B && a.T == T) return NC_OK;
+  if (a.mem) {
+    NC_CUDA_TRY(cudaStreamSynchronize(p->stream));
+    cudaFree(a.mem);
+    a = Acts();
+  }
+  const int L = p->depth;
+  const int64_t d = p->d, F = p->F, V = p->vocab, H = p->H;
+  // Sizes in bytes, each rounded to 256.
+  auto r = [](int64_t bytes) { return (bytes + 255) & ~int64_t(255); };
+  int64_t total = 0;
+  total += 2 * r(4 * N);                                     // tok, tgt
+  total += (L + 1) * r(4 * N * d) + L * r(4 * N * d);        // x, xmid
+  total += 2 * L * r(4 * N) + 2 * L * r(4 * N * H);          // r1 r2 rq rk
+  total += L * r(4 * N * H);                                 // lse [B,H,T]
+  total += 2 * L * r(2 * N * d) + L * r(2 * N * 3 * d) + L * r(2 * N * d) + L * r(2 * N * F);
+  total += r(2 * N * d) + r(4 * N) + r(2 * N * V) + r(4 * N) + r(4);  // hf rf logits loss
+  total += 2 * r(4 * N * d) + 2 * r(2 * N * d) + r(2 * N * F) + r(2 * N * 3 * d) +
+           r(4 * N * d) + r(4 * N * H);                      // backward scratch
+  void* mem = nullptr;
+  cudaError_t e = cudaMalloc(&mem, (size_t)total);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(NC_ERR_OOM, "activation allocation of " + std::to_string(total >> 20) + " MiB failed");
+  }
+  Arena ar{static_cast<char*>(mem), (size_t)total, 0};
+  a.mem = mem;
+  a.N = N;
+  a.B = B;
+  a.T = T;
+  a.tok = ar.take<int32_t>(N);
+  a.tgt = ar.take<int32_t>(N);
+  for (int l = 0; l <= L; ++l) a.x.push_back(ar.take<float>(N * d));
+  for (int l = 0; l < L; ++l) {
+    a.xmid.push_back(ar.take<float>(N * d));
+    a.r1.push_back(ar.take<float>(N));
+    a.r2.push_back(ar.take<float>(N));
+    a.rq.push_back(ar.take<float>(N * H));
+    a.rk.push_back(ar.take<float>(N * H));
+    a.lse.push_back(ar.take<float>(N * H));
+    a.h1.push_back(ar.take<bf16>(N * d));
+    a.h2.push_back(ar.take<bf16>(N * d));
+    a.qkv.push_back(ar.take<bf16>(N * 3 * d));
+    a.o.push_back(ar.take<bf16>(N * d));
+    a.a.push_back(ar.take<bf16>(N * F));
+  }
+  a.hf = ar.take<bf16>(N * d);
+  a.rf = ar.take<float>(N);
+  a.logits = ar.take<bf16>(N * V);
+  a.loss_rows = ar.take<float>(N);
+  a.loss = ar.take<float>(1);
+  a.dx0 = ar.take<float>(N * d);
+  a.dx1 = ar.take<float>(N * d);
+  a.dxb = ar.take<bf16>(N * d);
+  a.dh = ar.take<bf16>(N * d);
+  a.du = ar.take<bf16>(N * F);
+  a.dqkv = ar.take<bf16>(N * 3 * d);
+  a.dq = ar.take<float>(N * d);
+  a.delta = ar.take<float>(N * H);
+  if (ar.used > ar.size) return fail(NC_ERR_CUDA, "activation arena overflow");
+  return NC_OK;
+}
+
+bool is_device_ptr(const void* ptr) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, ptr) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
+}
+
+// y[M,N] = epi(x[M,K] W[N,K]^T): the forward projection.
+nc_status proj(nc_params* p, const bf16* x, int64_t M, int64_t K, const bf16* W, int64_t Nout,
+               void* D, int64_t ldd, nc_epilogue epi, const void* aux, int64_t ldaux) {
+  GemmLaunch g{};
+  g.status = p->status;
+  g.d.M = (int)M; g.d.N = (int)Nout; g.d.K = (int)K; g.d.batch = 1;
+  g.d.A = x; g.d.lda = K; g.d.a_kmajor = 1;
+  g.d.B = W; g.d.ldb = K; g.d.b_kmajor = 1;
+  g.d.D = D; g.d.ldd = ldd;
+  g.d.aux = aux; g.d.ldaux = ldaux;
+  g.d.epi = epi; g.d.alpha = 1.f; g.d.split_k = 1;
+  return gemm_launch(g, p->stream, p->prof);
+}
+
+// dx[M,N] = epi(dy[M,K] W[K,N]): the input gradient of a projection.
+nc_status proj_dx(nc_params* p, const bf16* dy, int64_t M, int64_t K, const bf16* W, int64_t Nout,
+                  void* D, int64_t ldd, nc_epilogue epi, const void* aux, int64_t ldaux) {
+  GemmLaunch g{};
+  g.status = p->status;
+  g.d.M = (int)M; g.d.N = (int)Nout; g.d.K = (int)K; g.d.batch = 1;
+  g.d.A = dy; g.d.lda = K; g.d.a_kmajor = 1;
+  g.d.B = W; g.d.ldb = Nout; g.d.b_kmajor = 0;
+  g.d.D = D; g.d.ldd = ldd;
+  g.d.aux = aux; g.d.ldaux = ldaux;
+  g.d.epi = epi; g.d.alpha = 1.f; g.d.split_k = 1;
+  return gemm_launch(g, p->stream, p->prof);
+}
+
+// dW[Mo,No] = dy[Ntok,Mo]^T x[Ntok,No] into a zeroed fp32 gradient.
+nc_status proj_dw(nc_params* p, const bf16* dy, int64_t ldy, int64_t Mo, const bf16* x,
+                  int64_t ldx, int64_t No, int64_t Ntok, float* dW) {
+  GemmLaunch g{};
+  g.status = p->status;
+  g.d.M = (int)Mo; g.d.N = (int)No; g.d.K = (int)Ntok; g.d.batch = 1;
+  g.d.A = dy; g.d.lda = ldy; g.d.a_kmajor = 0;
+  g.d.B = x; g.d.ldb = ldx; g.d.b_kmajor = 0;
+  g.d.D = dW; g.d.ldd = No;
+  g.d.epi = NC_EPI_ACC_F32; g.d.alpha = 1.f; g.d.split_k = 0;  // automatic split
+  return gemm_launch(g, p->stream, p->prof);
+}
+
+nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, int B, int T,
+                  float* loss_dev, nc_grads* g) {
+  if (p->poisoned) return fail(NC_ERR_TIMEOUT, "handle poisoned by an earlier device timeout");
+  if (!tokens || !targets || !g || g->p != p || B < 1 || T < 1 || (int64_t)B * T > (1 << 24))
+    return fail(NC_ERR_INVALID_ARG, "fwd_bwd: bad arguments");
+  NC_TRY(ensure_acts(p, B, T));
+  NC_TRY(ensure_rope(p, T));
+  Acts& a = p->act;
+  cudaStream_t s = p->stream;
+  Profiler* pr = p->prof;
+  const int L = p->depth, H = p->H, hd = p->hd, V = p->vocab;
+  const int64_t N = (int64_t)B * T, d = p->d, F = p->F, d2 = d * d;
+
+  const int32_t* tok = tokens;
+  const int32_t* tgt = targets;
+  if (!is_device_ptr(tokens)) {
+    NC_CUDA_TRY(cudaMemcpyAsync(a.tok, tokens, 4 * N, cudaMemcpyHostToDevice, s));
+    tok = a.tok;
+  }
+  if (!is_device_ptr(targets)) {
+    NC_CUDA_TRY(cudaMemcpyAsync(a.tgt, targets, 4 * N, cudaMemcpyHostToDevice, s));
+    tgt = a.tgt;
+  }
+  NC_CUDA_TRY(cudaMemsetAsync(g->mem, 0, sizeof(float) * (2 * (int64_t)V * d + block_elems(p)), s));
+
+  // ---------------- forward
+  NC_TRY(embed_gather(tok, N, p->wte, V, (int)d, a.x[0], p->status, s, pr));
+  for (int l = 0; l < L; ++l) {
+    const bf16* W = p->blocks_b + l * 12 * d2;
+    NC_TRY(rmsnorm_fwd(a.x[l], N, (int)d, a.h1[l], a.r1[l], s, pr));
+    NC_TRY(proj(p, a.h1[l], N, d, W, 3 * d, a.qkv[l], 3 * d, NC_EPI_STORE_BF16, nullptr, 0));
+    NC_TRY(rope_qknorm_fwd(a.qkv[l], 3 * d, N, T, H, hd, p->rope, a.rq[l], a.rk[l], s, pr));
+    NC_TRY(attention_fwd(a.qkv[l], a.qkv[l] + d, a.qkv[l] + 2 * d, 3 * d, a.o[l], d, a.lse[l], B,
+                         T, H, s, pr));
+    NC_TRY(proj(p, a.o[l], N, d, W + 3 * d2, d, a.xmid[l], d, NC_EPI_RESID_F32, a.x[l], d));
+    NC_TRY(rmsnorm_fwd(a.xmid[l], N, (int)d, a.h2[l], a.r2[l], s, pr));
+    NC_TRY(proj(p, a.h2[l], N, d, W + 4 * d2, F, a.a[l], F, NC_EPI_RELU2, nullptr, 0));
+    NC_TRY(proj(p, a.a[l], N, F, W + 8 * d2, d, a.x[l + 1], d, NC_EPI_RESID_F32, a.xmid[l], d));
+  }
+  NC_TRY(rmsnorm_fwd(a.x[L], N, (int)d, a.hf, a.rf, s, pr));
+  NC_TRY(proj(p, a.hf, N, d, p->lm_b, V, a.logits, V, NC_EPI_STORE_BF16, nullptr, 0));
+  NC_TRY(ce_fwd_bwd(a.logits, tgt, N, V, a.loss_rows, loss_dev ? loss_dev : a.loss, p->status, s,
+                    pr));
+
+  // ---------------- backward (a.logits now holds dz)
+  NC_TRY(proj_dw(p, a.logits, V, V, a.hf, d, d, N, g->lm));
+  NC_TRY(proj_dx(p, a.logits, N, V, p->lm_b, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0));
+  float* dx = a.dx0;
+  float* dxn = a.dx1;
+  NC_TRY(rmsnorm_bwd(a.dh, a.x[L], a.rf, nullptr, N, (int)d, dx, a.dxb, s, pr));
+  for (int l = L - 1; l >= 0; --l) {
+    const bf16* W = p->blocks_b + l * 12 * d2;
+    float* G = g->blocks + l * 12 * d2;
+    // MLP: x_out = xmid + a wdown^T, a = relu(h2 wup^T)^2
+    NC_TRY(proj_dw(p, a.dxb, d, d, a.a[l], F, F, N, G + 8 * d2));
+    NC_TRY(proj_dx(p, a.dxb, N, d, W + 8 * d2, F, a.du, F, NC_EPI_RELU2_BWD, a.a[l], F));
+    NC_TRY(proj_dw(p, a.du, F, F, a.h2[l], d, d, N, G + 4 * d2));
+    NC_TRY(proj_dx(p, a.du, N, F, W + 4 * d2, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0));
+    NC_TRY(rmsnorm_bwd(a.dh, a.xmid[l], a.r2[l], dx, N, (int)d, dxn, a.dxb, s, pr));
+    std::swap(dx, dxn);
+    // Attention: xmid = x + o wo^T
+    NC_TRY(proj_dw(p, a.dxb, d, d, a.o[l], d, d, N, G + 3 * d2));
+    NC_TRY(proj_dx(p, a.dxb, N, d, W + 3 * d2, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0));
+    NC_TRY(attention_bwd(a.qkv[l], a.qkv[l] + d, a.qkv[l] + 2 * d, 3 * d, a.o[l], a.dh, d,
+                         a.lse[l], a.dq, a.dqkv + d, a.dqkv + 2 * d, 3 * d, a.delta, B, T, H, s,
+                         pr));
+    NC_TRY(rope_qknorm_bwd(a.dq, nullptr, 0, a.qkv[l], 3 * d, a.rq[l], N, T, H, hd, p->rope,
+                           a.dqkv, 3 * d, s, pr));
+    NC_TRY(rope_qknorm_bwd(nullptr, a.dqkv + d, 3 * d, a.qkv[l] + d, 3 * d, a.rk[l], N, T, H, hd,
+                           p->rope, a.dqkv + d, 3 * d, s, pr));
+    NC_TRY(proj_dw(p, a.dqkv, 3 * d, 3 * d, a.h1[l], d, d, N, G));
+    NC_TRY(proj_dx(p, a.dqkv, N, 3 * d, W, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0));
+    NC_TRY(rmsnorm_bwd(a.dh, a.x[l], a.r1[l], dx, N, (int)d, dxn, a.dxb, s, pr));
+    std::swap(dx, dxn);
+  }
+  NC_TRY(embed_scatter(tok, N, dx, V, (int)d, g->wte, s, pr));
+  return NC_OK;
+}
+
+nc_status muon(nc_params* p, const nc_grads* g, float lr, float mu) {
+  if (p->poisoned) return fail(NC_ERR_TIMEOUT, "handle poisoned by an earlier device timeout");
+  if (!g || g->p != p) return fail(NC_ERR_INVALID_ARG, "muon: gradients of another model");
+  cudaStream_t s = p->stream;
+  Profiler* pr = p->prof;
+  const int L = p->depth;
+  const int64_t d = p->d, d2 = d * d;
+  NC_CUDA_TRY(cudaMemsetAsync(p->sumsq, 0, sizeof(float) * 6 * L, s));
+  NC_TRY(muon_momentum(p->mom, g->blocks, L, (int)d, mu, p->sumsq, s, pr));
+  for (int j = 0; j < 4; ++j)
+    NC_TRY(muon_prep(p->mom + j * d2, 12 * d2, (int)d, (int)d, 0, p->xsq + j * d2, 4 * d2,
+                     p->sumsq, j, L, s, pr));
+  NC_TRY(muon_prep(p->mom + 4 * d2, 12 * d2, (int)(4 * d), (int)d, 1, p->xw, 8 * d2, p->sumsq, 4,
+                   L, s, pr));
+  NC_TRY(muon_prep(p->mom + 8 * d2, 12 * d2, (int)d, (int)(4 * d), 0, p->xw + 4 * d2, 8 * d2,
+                   p->sumsq, 5, L, s, pr));
+  NC_TRY(newton_schulz_wide(p->xsq, 4 * L, (int)d, (int)d, 5, p->nsws, p->status, s, pr));
+  NC_TRY(newton_schulz_wide(p->xw, 2 * L, (int)d, (int)(4 * d), 5, p->nsws, p->status, s, pr));
+  for (int j = 0; j < 4; ++j)
+    NC_TRY(muon_apply(p->blocks + j * d2, p->blocks_b + j * d2, 12 * d2, (int)d, (int)d, 0,
+                      p->xsq + j * d2, 4 * d2, lr, L, s, pr));
+  NC_TRY(muon_apply(p->blocks + 4 * d2, p->blocks_b + 4 * d2, 12 * d2, (int)(4 * d), (int)d, 1,
+                    p->xw, 8 * d2, lr, L, s, pr));
+  NC_TRY(muon_apply(p->blocks + 8 * d2, p->blocks_b + 8 * d2, 12 * d2, (int)d, (int)(4 * d), 0,
+                    p->xw + 4 * d2, 8 * d2, lr, L, s, pr));
+  return NC_OK;
+}
+
+nc_status sync_bf16(nc_params* p) {
+  NC_TRY(f32_to_bf16(p->blocks, p->blocks_b, block_elems(p), p->stream, p->prof));
+  NC_TRY(f32_to_bf16(p->lm, p->lm_b, (int64_t)p->vocab * p->d, p->stream, p->prof));
+  return NC_OK;
+}
+
+uint64_t splitmix64_host(uint64_t x) {
+  uint64_t z = x + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+nc_status init_model(nc_params* p, uint64_t seed, int flags) {
+  const int n = 6 * p->depth + 2;
+  for (int t = 0; t < n; ++t) {
+    int64_t off, rows, cols;
+    const char* name;
+    int layer;
+    tensor_layout(p, t, &off, &rows, &cols, &name, &layer);
+    float* base = (t == 0) ? p->wte : (t == n - 1 ? p->lm : p->blocks);
+    float* dst = base + off;
+    const int64_t numel = rows * cols;
+    const bool out_proj = (layer >= 0) && ((t - 1) % 6 == 3 || (t - 1) % 6 == 5);
+    const bool head = (t == n - 1);
+    if (flags == NC_INIT_SPEC && (out_proj || head)) {
+      NC_CUDA_TRY(cudaMemsetAsync(dst, 0, sizeof(float) * numel, p->stream));
+      continue;
+    }
+    const double fan_in = (t == 0) ? 1.0 : (double)cols;
+    const uint64_t key = splitmix64_host(seed ^ splitmix64_host((uint64_t)t + 1));
+    NC_TRY(init_normal(dst, numel, key, (float)(1.0 / std::sqrt(fan_in)), p->stream));
+  }
+  return sync_bf16(p);
+}
+
+}  // namespace
+}  // namespace nc
+
+// ==================================================================== C ABI
+using namespace nc;
+
+extern "C" {
+
+const char* nc_last_error(void) { return g_last_error.c_str(); }
+
+const char* nc_status_string(nc_status s) {
+  switch (s) {
+    case NC_OK: return "ok";
+    case NC_ERR_INVALID_ARG: return "invalid argument";
+    case NC_ERR_OOM: return "out of device memory";
+    case NC_ERR_CUDA: return "CUDA error";
+    case NC_ERR_TOKEN_RANGE: return "token id out of range";
+    case NC_ERR_TIMEOUT: return "device wait timed out";
+    case NC_ERR_UNSUPPORTED: return "unsupported";
+  }
+  return "unknown";
+}
+
+nc_status nc_gpt_init_ex(int depth, int vocab, uint64_t seed, int flags, nc_params** out) {
+  if (!out) return fail(NC_ERR_INVALID_ARG, "init: null output");
+  *out = nullptr;
+  if (depth < 1 || depth > 64 || vocab < 8 || vocab > 32768 || vocab % 8 ||
+      (flags != NC_INIT_SPEC && flags != NC_INIT_ALL_RANDOM))
+    return fail(NC_ERR_INVALID_ARG, "init: depth in [1, 64], vocab in [8, 32768] (multiple of 8)");
+  if (depth % 2)
+    return fail(NC_ERR_UNSUPPORTED, "init: odd depth gives a head width other than 128");
+  nc_params* p = new nc_params();
+  p->depth = depth;
+  p->vocab = vocab;
+  p->d = 64 * depth;
+  p->hd = 128;
+  p->H = p->d / 128;
+  p->F = 4 * p->d;
+  p->prof = profiler_create();
+  const int64_t d = p->d, V = vocab, be = block_elems(p);
+  const int64_t sq = 4ll * depth * d * d, wide = 8ll * depth * d * d, ws = 12ll * depth * d * d;
+  auto r = [](int64_t bytes) { return (bytes + 255) & ~int64_t(255); };
+  const int64_t total = r(4 * V * d) * 2 + r(4 * be) * 2 + r(2 * be) + r(2 * V * d) +
+                        r(4 * 6 * depth) + r(2 * sq) + r(2 * wide) + r(2 * ws) + r(4);
+  cudaError_t e = cudaMalloc(&p->pmem, (size_t)total);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    profiler_destroy(p->prof);
+    delete p;
+    return fail(NC_ERR_OOM, "parameter allocation failed");
+  }
+  Arena ar{static_cast<char*>(p->pmem), (size_t)total, 0};
+  p->wte = ar.take<float>(V * d);
+  p->lm = ar.take<float>(V * d);
+  p->blocks = ar.take<float>(be);
+  p->mom = ar.take<float>(be);
+  p->blocks_b = ar.take<bf16>(be);
+  p->lm_b = ar.take<bf16>(V * d);
+  p->sumsq = ar.take<float>(6 * depth);
+  p->xsq = ar.take<bf16>(sq);
+  p->xw = ar.take<bf16>(wide);
+  p->nsws = ar.take<bf16>(ws);
+  p->status = ar.take<int>(1);
+  nc_status st = NC_OK;
+  if (cudaMallocHost(&p->h_loss, sizeof(float)) != cudaSuccess ||
+      cudaMallocHost(&p->h_status, sizeof(int)) != cudaSuccess)
+    st = fail(NC_ERR_OOM, "pinned host allocation failed");
+  if (st == NC_OK && cudaMemsetAsync(p->mom, 0, sizeof(float) * be, p->stream) != cudaSuccess)
+    st = fail(NC_ERR_CUDA, "momentum clear failed");
+  if (st == NC_OK && cudaMemsetAsync(p->status, 0, sizeof(int), p->stream) != cudaSuccess)
+    st = fail(NC_ERR_CUDA, "status clear failed");
+  if (st == NC_OK) st = init_model(p, seed, flags);
+  if (st == NC_OK && cudaStreamSynchronize(p->stream) != cudaSuccess)
+    st = fail(NC_ERR_CUDA, "init synchronisation failed");
+  if (st != NC_OK) {
+    nc_params_free(p);
+    return st;
+  }
+  *out = p;
+  return NC_OK;
+}
+
+nc_status nc_gpt_init(int depth, int vocab, uint64_t seed, nc_params** out) {
+  return nc_gpt_init_ex(depth, vocab, seed, NC_INIT_SPEC, out);
+}
+
+void nc_params_free(nc_params* p) {
+  if (!p) return;
+  if (p->stream) cudaStreamSynchronize(p->stream);
+  else cudaDeviceSynchronize();
+  if (p->act.mem) cudaFree(p->act.mem);
+  if (p->rope) cudaFree(p->rope);
+  if (p->pmem) cudaFree(p->pmem);
+  if (p->h_loss) cudaFreeHost(p->h_loss);
+  if (p->h_status) cudaFreeHost(p->h_status);
+  profiler_destroy(p->prof);
+  delete p;
+}
+
+nc_status nc_set_stream(nc_params* p, void* stream) {
+  if (!p) return fail(NC_ERR_INVALID_ARG, "set_stream: null handle");
+  p->stream = static_cast<cudaStream_t>(stream);
+  return NC_OK;
+}
+
+int nc_num_tensors(const nc_params* p) { return p ? 6 * p->depth + 2 : 0; }
+
+nc_status nc_tensor_info(const nc_params* p, int idx, nc_tensor_desc* out) {
+  if (!p || !out || idx < 0 || idx >= nc_num_tensors(p))
+    return fail(NC_ERR_INVALID_ARG, "tensor_info: bad index");
+  int64_t off, rows, cols;
+  const char* name;
+  int layer;
+  tensor_layout(p, idx, &off, &rows, &cols, &name, &layer);
+  std::memset(out, 0, sizeof(*out));
+  if (layer >= 0) std::snprintf(out->name, sizeof(out->name), "h%d.%s", layer, name);
+  else std::snprintf(out->name, sizeof(out->name), "%s", name);
+  out->ndim = 2;
+  out->shape[0] = rows;
+  out->shape[1] = cols;
+  out->dtype = NC_F32;
+  const int n = nc_num_tensors(p);
+  if (idx == 0) {
+    out->data = p->wte;
+    out->data_bf16 = nullptr;
+  } else if (idx == n - 1) {
+    out->data = p->lm;
+    out->data_bf16 = p->lm_b;
+  } else {
+    out->data = p->blocks + off;
+    out->data_bf16 = p->blocks_b + off;
+  }
+  return NC_OK;
+}
+
+nc_status nc_params_sync(nc_params* p) {
+  if (!p) return fail(NC_ERR_INVALID_ARG, "params_sync: null handle");
+  return sync_bf16(p);
+}
+
+nc_status nc_tensor_write(nc_params* p, int idx, const float* src) {
+  nc_tensor_desc t;
+  NC_TRY(nc_tensor_info(p, idx, &t));
+  if (!src) return fail(NC_ERR_INVALID_ARG, "tensor_write: null source");
+  const int64_t n = t.shape[0] * t.shape[1];
+  NC_CUDA_TRY(cudaMemcpyAsync(t.data, src, sizeof(float) * n, cudaMemcpyDefault, p->stream));
+  if (t.data_bf16)
+    NC_TRY(f32_to_bf16(static_cast<float*>(t.data), t.data_bf16, n, p->stream, nullptr));
+  NC_CUDA_TRY(cudaStreamSynchronize(p->stream));
+  return NC_OK;
+}
+
+nc_status nc_tensor_read(const nc_params* p, int idx, float* dst) {
+  nc_tensor_desc t;
+  NC_TRY(nc_tensor_info(p, idx, &t));
+  if (!dst) return fail(NC_ERR_INVALID_ARG, "tensor_read: null destination");
+  NC_CUDA_TRY(cudaMemcpyAsync(dst, t.data, sizeof(float) * t.shape[0] * t.shape[1],
+                              cudaMemcpyDefault, p->stream));
+  NC_CUDA_TRY(cudaStreamSynchronize(p->stream));
+  return NC_OK;
+}
+
+nc_status nc_momentum_read(const nc_params* p, int idx, float* dst) {
+  if (!p || !dst || idx < 1 || idx > 6 * p->depth)
+    return fail(NC_ERR_INVALID_ARG, "momentum_read: bad index");
+  int64_t off, rows, cols;
+  const char* name;
+  int layer;
+  tensor_layout(p, idx, &off, &rows, &cols, &name, &layer);
+  NC_CUDA_TRY(cudaMemcpyAsync(dst, p->mom + off, sizeof(float) * rows * cols, cudaMemcpyDefault,
+                              p->stream));
+  NC_CUDA_TRY(cudaStreamSynchronize(p->stream));
+  return NC_OK;
+}
+
+nc_status nc_grads_create(const nc_params* p, nc_grads** out) {
+  if (!p || !out) return fail(NC_ERR_INVALID_ARG, "grads_create: null argument");
+  nc_grads* g = new nc_grads();
+  g->p = p;
+  const int64_t vd = (int64_t)p->vocab * p->d, be = block_elems(p);
+  cudaError_t e = cudaMalloc(&g->mem, sizeof(float) * (2 * vd + be));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    delete g;
+    return fail(NC_ERR_OOM, "gradient allocation failed");
+  }
+  g->wte = static_cast<float*>(g->mem);
+  g->lm = g->wte + vd;
+  g->blocks = g->lm + vd;
+  *out = g;
+  return NC_OK;
+}
+
+void nc_grads_free(nc_grads* g) {
+  if (!g) return;
+  cudaDeviceSynchronize();
+  if (g->mem) cudaFree(g->mem);
+  delete g;
+}
+
+nc_status nc_grad_info(const nc_grads* g, int idx, nc_tensor_desc* out) {
+  if (!g) return fail(NC_ERR_INVALID_ARG, "grad_info: null handle");
+  NC_TRY(nc_tensor_info(g->p, idx, out));
+  int64_t off, rows, cols;
+  const char* name;
+  int layer;
+  tensor_layout(g->p, idx, &off, &rows, &cols, &name, &layer);
+  const int n = nc_num_tensors(g->p);
+  out->data = idx == 0 ? g->wte : (idx == n - 1 ? g->lm : g->blocks + off);
+  out->data_bf16 = nullptr;
+  return NC_OK;
+}
+
+nc_status nc_grad_read(const nc_grads* g, int idx, float* dst) {
+  nc_tensor_desc t;
+  NC_TRY(nc_grad_info(g, idx, &t));
+  if (!dst) return fail(NC_ERR_INVALID_ARG, "grad_read: null destination");
+  NC_CUDA_TRY(cudaMemcpyAsync(dst, t.data, sizeof(float) * t.shape[0] * t.shape[1],
+                              cudaMemcpyDefault, g->p->stream));
+  NC_CUDA_TRY(cudaStreamSynchronize(g->p->stream));
+  return NC_OK;
+}
+
+nc_status nc_grad_write(nc_grads* g, int idx, const float* src) {
+  nc_tensor_desc t;
+  NC_TRY(nc_grad_info(g, idx, &t));
+  if (!src) return fail(NC_ERR_INVALID_ARG, "grad_write: null source");
+  NC_CUDA_TRY(cudaMemcpyAsync(t.data, src, sizeof(float) * t.shape[0] * t.shape[1],
+                              cudaMemcpyDefault, g->p->stream));
+  NC_CUDA_TRY(cudaStreamSynchronize(g->p->stream));
+  return NC_OK;
+}
+
+nc_status nc_gpt_fwd_bwd_async(nc_params* p, const int32_t* tokens, const int32_t* targets, int B,
+                               int T, float* loss_dev, nc_grads* g) {
+  if (!p) return fail(NC_ERR_INVALID_ARG, "fwd_bwd: null handle");
+  return fwd_bwd(p, tokens, targets, B, T, loss_dev, g);
+}
+
+nc_status nc_gpt_fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, int B,
+                         int T, float* loss_host, nc_grads* g) {
+  if (!p || !loss_host) return fail(NC_ERR_INVALID_ARG, "fwd_bwd: null argument");
+  NC_TRY(fwd_bwd(p, tokens, targets, B, T, nullptr, g));
+  NC_TRY(sync_and_check(p, p->act.loss));
+  *loss_host = *p->h_loss;
+  return NC_OK;
+}
+
+nc_status nc_muon_step(nc_params* p, const nc_grads* g, float lr, float momentum) {
+  if (!p) return fail(NC_ERR_INVALID_ARG, "muon: null handle");
+  return muon(p, g, lr, momentum);
+}
+
+nc_status nc_sync(nc_params* p) {
+  if (!p) return fail(NC_ERR_INVALID_ARG, "sync: null handle");
+  return sync_and_check(p, nullptr);
+}
+
+nc_status nc_profile_enable(nc_params* p, int on) {
+  if (!p) return fail(NC_ERR_INVALID_ARG, "profile: null handle");
+  profiler_enable(p->prof, on != 0);
+  return NC_OK;
+}
+
+nc_status nc_profile_read(nc_params* p, nc_kernel_stat* out, int max, int* n) {
+  if (!p || !out || max < 0) return fail(NC_ERR_INVALID_ARG, "profile: bad arguments");
+  return profiler_read(p->prof, out, max, n);
+}
+
+int64_t nc_launch_count(const nc_params* p) { return p ? profiler_launches(p->prof) : 0; }
+
+// ------------------------------------------------------------------ ops
+nc_status nc_op_gemm(const nc_gemm_desc* desc, void* stream) {
+  if (!desc) return fail(NC_ERR_INVALID_ARG, "gemm: null descriptor");
+  GemmLaunch g{};
+  g.d = *desc;
+  g.status = nullptr;
+  if (g.d.split_k < 0) return fail(NC_ERR_INVALID_ARG, "gemm: split_k < 0");
+  if (g.d.split_k == 0) g.d.split_k = 1;
+  return gemm_launch(g, static_cast<cudaStream_t>(stream), nullptr);
+}
+
+nc_status nc_op_rmsnorm(const float* x, int64_t rows, int cols, void* y_bf16, float* rstd,
+                        void* stream) {
+  if (!x || !y_bf16 || rows < 0 || cols < 4) return fail(NC_ERR_INVALID_ARG, "rmsnorm: bad arguments");
+  if (rows == 0) return NC_OK;
+  return rmsnorm_fwd(x, rows, cols, y_bf16, rstd, static_cast<cudaStream_t>(stream), nullptr);
+}
+
+nc_status nc_op_attention_fwd(const void* q, const void* k, const void* v, int64_t ld, void* o,
+                              int64_t ldo, float* lse, int B, int T, int H, void* stream) {
+  return attention_fwd(q, k, v, ld, o, ldo, lse, B, T, H, static_cast<cudaStream_t>(stream),
+                       nullptr);
+}
+
+nc_status nc_op_attention_bwd(const void* q, const void* k, const void* v, int64_t ld,
+                              const void* o, const void* dout, int64_t ldo, const float* lse,
+                              float* dq, void* dk, void* dv, int64_t ldg, float* delta_scratch,
+                              int B, int T, int H, void* stream) {
+  return attention_bwd(q, k, v, ld, o, dout, ldo, lse, dq, dk, dv, ldg, delta_scratch, B, T, H,
+                       static_cast<cudaStream_t>(stream), nullptr);
+}
+
+size_t nc_newton_schulz_scratch_bytes(int count, int rows, int cols) {
+  if (count < 1 || rows < 1 || cols < 1) return 0;
+  const int64_t m = std::min(rows, cols), n = std::max(rows, cols);
+  // X (normalised, wide) + A + B + second X, then the fp32 norms.
+  return (size_t)(2 * (count * m * n) + 2 * (count * m * m)) * 2 + (size_t)count * 4 + 256;
+}
+
+nc_status nc_op_newton_schulz(const void* x_bf16, void* out_bf16, int count, int rows, int cols,
+                              int steps, void* scratch, void* stream) {
+  if (!x_bf16 || !out_bf16 || !scratch || count < 1 || rows < 1 || cols < 1 || steps < 0)
+    return fail(NC_ERR_INVALID_ARG, "newton_schulz: bad arguments");
+  if (((int64_t)rows * cols) % 8 || std::min(rows, cols) % 8)
+    return fail(NC_ERR_INVALID_ARG, "newton_schulz: dims must be multiples of 8");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int m = std::min(rows, cols), n = std::max(rows, cols);
+  const bool tall = rows > cols;
+  const int64_t mn = (int64_t)m * n;
+  bf16* X = static_cast<bf16*>(scratch);
+  bf16* ws = X + count * mn;  // A, B, second X
+  float* norms = reinterpret_cast<float*>(ws + count * mn + 2 * (int64_t)count * m * m);
+  NC_CUDA_TRY(cudaMemsetAsync(norms, 0, sizeof(float) * count, s));
+  NC_TRY(sumsq_bf16(x_bf16, mn, count, norms, s, nullptr));
+  NC_TRY(scale_bf16(x_bf16, rows, cols, tall ? 1 : 0, norms, 1e-7f, X, count, s, nullptr));
+  NC_TRY(newton_schulz_wide(X, count, m, n, steps, ws, nullptr, s, nullptr));
+  // Back to the caller's orientation (no scaling).
+  NC_TRY(scale_bf16(X, m, n, tall ? 1 : 0, nullptr, 0.f, out_bf16, count, s, nullptr));
+  return NC_OK;
+}
+
+}  // extern "C"

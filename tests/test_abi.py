@@ -1,0 +1,73 @@
+"""Host-side checks of the boundary (no GPU compute): the C-ABI library
+builds for sm_100a, loads, and exports every entry point include/nc.h
+declares; the binding refuses to run without the library; the seeded input
+generators behave as documented."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+from pretraining_step_b200 import binding, inputs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(nc_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    from pretraining_step_b200 import build
+    build.build()
+    L = binding.lib()
+    declared = _declared()
+    assert len(declared) >= 25
+    missing = [n for n in sorted(declared) if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_status_strings():
+    assert binding.status_string(binding.NC_OK) == "ok"
+    assert binding.status_string(binding.NC_ERR_TIMEOUT) == "device wait timed out"
+    assert binding.status_string(99) == "unknown"
+
+
+def test_oracle_is_not_linked_by_the_product():
+    import subprocess
+    from pretraining_step_b200 import build
+    out = subprocess.run(["nm", "-D", build.build()], capture_output=True, text=True).stdout
+    assert "oc_" not in " ".join(l.split()[-1] for l in out.splitlines() if " T " in l)
+    for dirpath, _, files in os.walk(os.path.join(ROOT, "pretraining_step_b200")):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in src and "nc_oracle" not in src, f
+
+
+def test_token_generator_range_and_shift():
+    tok, tgt = inputs.token_batch(20, 4, 64)
+    assert tok.dtype == np.int32 and tok.shape == (4, 64)
+    assert tok.min() >= 0 and tok.max() < 32768
+    assert np.array_equal(tok[:, 1:], tgt[:, :-1])
+    a, _ = inputs.token_batch(20, 4, 64)
+    b, _ = inputs.token_batch(21, 4, 64)
+    assert np.array_equal(a, tok) and not np.array_equal(a, b)
+    # V = 32768: ids are the top 15 bits of the SplitMix64 word.
+    w = inputs.splitmix64(inputs.stream_key(20, inputs.STREAM_TOKENS) + np.uint64(0))
+    assert tok[0, 0] == int(w) >> 49
+    z, _ = inputs.zipf_token_batch(3, 8, 256)
+    assert z.min() >= 0 and z.max() < 32768 and np.mean(z == 0) > 0.05
+
+
+def test_bf16_rounding_is_exact_and_nearest_even():
+    x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -9, -2.5, 3.0e38], dtype=np.float32)
+    r = inputs.round_to_bf16(x)
+    assert r[0] == 1.0 and r[1] == 1.0 and r[2] == 1.0 + 2 ** -7 and r[3] == -2.5
+    assert np.all((r.view(np.uint32) & 0xFFFF) == 0)

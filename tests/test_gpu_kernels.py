@@ -1,0 +1,241 @@
+"""Kernel-level parity of the CUDA path (through the C ABI) with the oracle.
+
+Inputs come from the seeded generators (bf16-representable, so both sides
+see identical numbers); expected values from oracle/ only.
+Tolerances: bf16 outputs carry one bf16 rounding (relative 2^-9), so a
+relative Frobenius error of 5e-3 bounds them; fp32 outputs accumulate in
+fp32 over K <= 1280 products (relative ~1e-6), bound 2e-5.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from pretraining_step_b200 import binding as nc
+from pretraining_step_b200 import inputs
+
+from gpu_util import dev_bf16, dev_f32, host, rel_fro, torch
+
+pytestmark = pytest.mark.gpu
+
+
+# ------------------------------------------------------------------ GEMM
+@pytest.mark.parametrize("a_k,b_k", [(1, 1), (1, 0), (0, 1), (0, 0)])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 64), (200, 296, 136), (256, 128, 512),
+                                   (384, 384, 200), (64, 1280, 1280)])
+def test_gemm_layouts(a_k, b_k, M, N, K):
+    t = torch()
+    A = inputs.bf16_normal(1, (M, K))
+    B = inputs.bf16_normal(2, (N, K))
+    tA = dev_bf16(A if a_k else A.T)
+    tB = dev_bf16(B if b_k else B.T)
+    D = t.empty(M, N, dtype=t.bfloat16, device="cuda")
+    nc.gemm(M, N, K, tA, tB, D, a_kmajor=a_k, b_kmajor=b_k)
+    t.cuda.synchronize()
+    ref = oracle.matmul_nt(A, B)
+    assert rel_fro(host(D), ref) < 5e-3
+
+
+@pytest.mark.parametrize("a_k,b_k", [(1, 1), (0, 0)])
+def test_gemm_f32_store_and_alpha(a_k, b_k):
+    t = torch()
+    M, N, K = 256, 512, 320
+    A = inputs.bf16_normal(3, (M, K))
+    B = inputs.bf16_normal(4, (N, K))
+    D = t.empty(M, N, dtype=t.float32, device="cuda")
+    nc.gemm(M, N, K, dev_bf16(A if a_k else A.T), dev_bf16(B if b_k else B.T), D,
+            a_kmajor=a_k, b_kmajor=b_k, epi=nc.EPI_STORE_F32, alpha=0.5)
+    t.cuda.synchronize()
+    assert rel_fro(host(D), 0.5 * oracle.matmul_nt(A, B)) < 2e-5
+
+
+def test_gemm_residual_relu2_and_backward_epilogues():
+    t = torch()
+    M, N, K = 300, 384, 256
+    A = inputs.bf16_normal(5, (M, K))
+    B = inputs.bf16_normal(6, (N, K), std=0.1)
+    acc = oracle.matmul_nt(A, B)
+    R = np.random.default_rng(7).standard_normal((M, N)).astype(np.float32)
+    D = t.empty(M, N, dtype=t.float32, device="cuda")
+    nc.gemm(M, N, K, dev_bf16(A), dev_bf16(B), D, epi=nc.EPI_RESID_F32, aux=dev_f32(R))
+    t.cuda.synchronize()
+    assert rel_fro(host(D), R + acc) < 2e-5
+    # ReLU^2
+    D2 = t.empty(M, N, dtype=t.bfloat16, device="cuda")
+    nc.gemm(M, N, K, dev_bf16(A), dev_bf16(B), D2, epi=nc.EPI_RELU2)
+    t.cuda.synchronize()
+    assert rel_fro(host(D2), np.maximum(acc, 0) ** 2) < 5e-3
+    # 2 sqrt(a) * acc with a = relu(u)^2 >= 0
+    Aux = inputs.round_to_bf16(np.abs(np.random.default_rng(8).standard_normal((M, N)))
+                               .astype(np.float32))
+    D3 = t.empty(M, N, dtype=t.bfloat16, device="cuda")
+    nc.gemm(M, N, K, dev_bf16(A), dev_bf16(B), D3, epi=nc.EPI_RELU2_BWD, aux=dev_bf16(Aux))
+    t.cuda.synchronize()
+    assert rel_fro(host(D3), 2 * np.sqrt(Aux.astype(np.float64)) * acc) < 5e-3
+    # alpha*acc + beta*aux
+    D4 = t.empty(M, N, dtype=t.bfloat16, device="cuda")
+    nc.gemm(M, N, K, dev_bf16(A), dev_bf16(B), D4, epi=nc.EPI_AXPBY_BF16, aux=dev_bf16(Aux),
+            alpha=2.0315, beta=-4.775)
+    t.cuda.synchronize()
+    assert rel_fro(host(D4), 2.0315 * acc - 4.775 * Aux) < 5e-3
+
+
+@pytest.mark.parametrize("split", [1, 3, 7])
+def test_gemm_split_k_accumulates(split):
+    t = torch()
+    M, N, K = 256, 256, 2048
+    A = inputs.bf16_normal(9, (K, M))   # stored M-major, like dy^T
+    B = inputs.bf16_normal(10, (K, N))  # stored N-major, like x
+    D0 = np.random.default_rng(11).standard_normal((M, N)).astype(np.float32)
+    D = dev_f32(D0)
+    nc.gemm(M, N, K, dev_bf16(A), dev_bf16(B), D, a_kmajor=0, b_kmajor=0, epi=nc.EPI_ACC_F32,
+            split_k=split)
+    t.cuda.synchronize()
+    assert rel_fro(host(D), D0 + oracle.matmul_nt(A.T, B.T)) < 2e-5
+
+
+def test_gemm_batched_strided():
+    t = torch()
+    bt, M, N, K = 3, 136, 264, 192
+    A = inputs.bf16_normal(12, (bt, M, K))
+    B = inputs.bf16_normal(13, (bt, K, N))  # N-major per batch
+    D = t.empty(bt, M, N, dtype=t.bfloat16, device="cuda")
+    nc.gemm(M, N, K, dev_bf16(A), dev_bf16(B), D, b_kmajor=0, batch=bt, stride_a=M * K,
+            stride_b=K * N, stride_d=M * N)
+    t.cuda.synchronize()
+    for i in range(bt):
+        assert rel_fro(host(D[i]), oracle.matmul_nt(A[i], B[i].T)) < 5e-3
+
+
+def test_gemm_rejects_bad_arguments():
+    t = torch()
+    A = t.zeros(64, 60, dtype=t.bfloat16, device="cuda")
+    D = t.zeros(64, 64, dtype=t.bfloat16, device="cuda")
+    with pytest.raises(nc.NcError) as e:
+        nc.gemm(64, 64, 60, A, A, D, lda=60, ldb=60)  # 60 % 8 != 0
+    assert e.value.status == nc.NC_ERR_INVALID_ARG
+    with pytest.raises(nc.NcError):
+        nc.gemm(64, 64, 64, A, A, D, epi=nc.EPI_STORE_BF16, split_k=2)
+
+
+def test_gemm_full_size_sampled():
+    """The MLP-up shape of the depth-20 step (65536 x 5120 x 1280, the size
+    the step runs), checked on sampled rows and columns."""
+    t = torch()
+    M, N, K = 65536, 5120, 1280
+    A = inputs.bf16_normal(14, (M, K))
+    B = inputs.bf16_normal(15, (N, K), std=K ** -0.5)
+    D = t.empty(M, N, dtype=t.bfloat16, device="cuda")
+    nc.gemm(M, N, K, dev_bf16(A), dev_bf16(B), D, epi=nc.EPI_RELU2)
+    t.cuda.synchronize()
+    rng = np.random.default_rng(16)
+    rows = np.sort(rng.choice(M, 96, replace=False))
+    rows[-1] = M - 1
+    cols = np.sort(rng.choice(N, 96, replace=False))
+    ref = np.maximum(oracle.matmul_nt(A[rows], B[cols]), 0) ** 2
+    got = host(D[t.from_numpy(rows).cuda()][:, t.from_numpy(cols).cuda()])
+    assert rel_fro(got, ref) < 5e-3
+
+
+# ------------------------------------------------------------------ RMSNorm
+@pytest.mark.parametrize("rows,cols", [(1, 256), (37, 1280), (1000, 768)])
+def test_rmsnorm(rows, cols):
+    t = torch()
+    x = (np.random.default_rng(17).standard_normal((rows, cols)) * 3).astype(np.float32)
+    y = t.empty(rows, cols, dtype=t.bfloat16, device="cuda")
+    r = t.empty(rows, dtype=t.float32, device="cuda")
+    nc.rmsnorm(dev_f32(x), y, r, rows, cols)
+    t.cuda.synchronize()
+    yr, rr = oracle.rmsnorm(x)
+    assert rel_fro(host(y), yr) < 5e-3
+    np.testing.assert_allclose(host(r), rr, rtol=1e-5)
+
+
+# ------------------------------------------------------------------ attention
+def _attn_inputs(B, T, H, seed):
+    # q, k with unit RMS per head (as after QK-norm), v normal; fused [B*T, 3d] rows.
+    d = H * 128
+    qkv = inputs.bf16_normal(seed, (B * T, 3 * d))
+    return qkv
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 64, 1), (2, 200, 2), (1, 1, 1), (1, 577, 3)])
+def test_attention_forward(B, T, H):
+    t = torch()
+    d = H * 128
+    qkv = _attn_inputs(B, T, H, 18 + T)
+    q = qkv[:, :d].reshape(B, T, H, 128)
+    k = qkv[:, d:2 * d].reshape(B, T, H, 128)
+    v = qkv[:, 2 * d:].reshape(B, T, H, 128)
+    dq = dev_bf16(qkv)
+    o = t.empty(B * T, d, dtype=t.bfloat16, device="cuda")
+    lse = t.empty(B, H, T, dtype=t.float32, device="cuda")
+    nc.attention_fwd(dq, dq[:, d:], dq[:, 2 * d:], 3 * d, o, d, lse, B, T, H)
+    t.cuda.synchronize()
+    oref, lref, _ = oracle.attention(q, k, v)
+    assert rel_fro(host(o), oref.reshape(B * T, d)) < 5e-3
+    np.testing.assert_allclose(host(lse), lref, rtol=2e-4, atol=2e-4)
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 64, 1), (2, 200, 2), (1, 333, 1)])
+def test_attention_backward(B, T, H):
+    t = torch()
+    d = H * 128
+    qkv = _attn_inputs(B, T, H, 40 + T)
+    q = qkv[:, :d].reshape(B, T, H, 128)
+    k = qkv[:, d:2 * d].reshape(B, T, H, 128)
+    v = qkv[:, 2 * d:].reshape(B, T, H, 128)
+    # The backward consumes the forward's O and lse; those come from the
+    # oracle here (rounded to bf16 like the saved activation).
+    oref, lref, _ = oracle.attention(q, k, v)
+    o_b = inputs.round_to_bf16(oref.reshape(B * T, d).astype(np.float32))
+    dout = inputs.bf16_normal(41 + T, (B * T, d))
+    dqkv = t.zeros(B * T, 3 * d, dtype=t.bfloat16, device="cuda")
+    dqf = t.empty(B * T, d, dtype=t.float32, device="cuda")
+    delta = t.empty(B, H, T, dtype=t.float32, device="cuda")
+    tq = dev_bf16(qkv)
+    nc.attention_bwd(tq, tq[:, d:], tq[:, 2 * d:], 3 * d, dev_bf16(o_b), dev_bf16(dout), d,
+                     dev_f32(lref.astype(np.float32)), dqf, dqkv[:, d:], dqkv[:, 2 * d:], 3 * d,
+                     delta, B, T, H)
+    t.cuda.synchronize()
+    rq, rk, rv = oracle.attention_bwd(q, k, v, lref, dout.reshape(B, T, H, 128))
+    assert rel_fro(host(dqf), rq.reshape(B * T, d)) < 1e-2
+    assert rel_fro(host(dqkv[:, d:2 * d]), rk.reshape(B * T, d)) < 1e-2
+    assert rel_fro(host(dqkv[:, 2 * d:]), rv.reshape(B * T, d)) < 1e-2
+
+
+def test_attention_full_length_sampled_heads():
+    """T = 2048 (the step's sequence length), one batch row, two heads."""
+    t = torch()
+    B, T, H = 1, 2048, 2
+    d = H * 128
+    qkv = _attn_inputs(B, T, H, 60)
+    dq = dev_bf16(qkv)
+    o = t.empty(B * T, d, dtype=t.bfloat16, device="cuda")
+    lse = t.empty(B, H, T, dtype=t.float32, device="cuda")
+    nc.attention_fwd(dq, dq[:, d:], dq[:, 2 * d:], 3 * d, o, d, lse, B, T, H)
+    t.cuda.synchronize()
+    q = qkv[:, :d].reshape(B, T, H, 128)
+    k = qkv[:, d:2 * d].reshape(B, T, H, 128)
+    v = qkv[:, 2 * d:].reshape(B, T, H, 128)
+    oref, lref, _ = oracle.attention(q, k, v)
+    assert rel_fro(host(o), oref.reshape(B * T, d)) < 5e-3
+    np.testing.assert_allclose(host(lse), lref, rtol=2e-4, atol=2e-4)
+
+
+# ------------------------------------------------------------------ Newton-Schulz
+@pytest.mark.parametrize("count,rows,cols", [(3, 256, 256), (2, 128, 512), (2, 512, 128)])
+def test_newton_schulz_op(count, rows, cols):
+    t = torch()
+    X = inputs.normal_stack(70 + rows, count, rows, cols)
+    out = t.empty(count, rows, cols, dtype=t.bfloat16, device="cuda")
+    scratch = t.empty(nc.newton_schulz_scratch_bytes(count, rows, cols), dtype=t.uint8,
+                      device="cuda")
+    nc.newton_schulz(dev_bf16(X), out, count, rows, cols, 5, scratch)
+    t.cuda.synchronize()
+    got = host(out)
+    for i in range(count):
+        ref = oracle.newton_schulz(X[i])
+        assert rel_fro(got[i], ref) < 2e-2
+        s = np.linalg.svd(got[i], compute_uv=False)
+        if rows != cols:  # wide/tall N(0,1): every normalised sigma is well above 2e-3
+            assert s.min() > 0.6 and s.max() < 1.22
