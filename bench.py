@@ -1,0 +1,428 @@
+"""Throughput of the depth-20 nanochat base-pretraining step on B200.
+
+One step = forward + backward of the depth-20 GPT (d 1280, 10 heads x 128,
+MLP 5120, vocab 32768) on B = 32 rows of T = 2048 synthetic token ids,
+followed by the Muon update of the 120 block matrices.  Weights are
+random-init (every matrix drawn, so no branch multiplies zeros); token ids
+are uniform SplitMix64 draws (the pages' web-text shards are not available).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+Prints one JSON line (rank 0).  `value` is device-timed whole-job tokens/s
+with inputs resident in HBM; `e2e` is the same metric through the C ABI
+with the token ids in pinned host memory, copied in every step, and the
+loss read back every step.  N > 1 runs N independent replicas (one process
+per GPU under torchrun): the step has no exchange.  --impl reference runs
+the CPU oracle on bounded samples of the same workload on the host cores.
+"""
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "train tokens/s and MFU (bf16 peak) at depth-20 GPT, 1×B200"
+DEPTH, B, T, V = 20, 32, 2048, 32768
+LR, MOMENTUM = 0.02, 0.95
+NOMINAL_BF16_TFLOPS = 2250.0
+
+
+def model_flops_per_token(depth=DEPTH, seq=T, vocab=V):
+    """Algorithmic training FLOPs per token: 6 * N_matmul + 6 * L * d * T
+    (causal attention counts the half of QK^T and PV it computes)."""
+    d = 64 * depth
+    n_mm = 12 * depth * d * d + vocab * d
+    return 6.0 * n_mm + 6.0 * depth * d * seq
+
+
+def ns_flops(depth=DEPTH):
+    """Newton-Schulz FLOPs of one Muon step (5 iterations, m <= n Gram form)."""
+    d = 64 * depth
+    sq = 2 * d ** 3 * 3                      # X X^T, A A, B X for d x d
+    wide = 2 * (d * d * 4 * d) * 2 + 2 * d ** 3  # X X^T and B X at n = 4d, A A at d
+    return 5.0 * (4 * depth * sq + 2 * depth * wide)
+
+
+def workload_name():
+    return ("depth-20 GPT (d 1280, 10x128 heads, MLP 5120, vocab 32768), bf16, B=32, T=2048: "
+            "forward + backward + Muon step")
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, \
+            "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", "nc_clocks_%d_%d.csv" % (os.getpid(), gpu_index))
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.QUERY,
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        load = [s for s in sm if s > 0.5 * mx] or sm
+        return {"sm_mhz": float(np.median(load)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle sample
+def cpu_oracle_sample(budget_s=20.0, per_step=False):
+    """Time the oracle on a bounded sample of the workload and convert to the
+    workload's tokens/s: forward+backward on a short row (cost per token) and
+    the Newton-Schulz of one matrix of each Muon shape (cost per matrix)."""
+    import oracle
+    from pretraining_step_b200 import inputs
+    oracle.lib()
+    P = inputs.random_params(DEPTH, seed=1)
+    t_tok = 16
+    tok, tgt = inputs.token_batch(2, 1, t_tok)
+    t0 = time.perf_counter()
+    oracle.gpt_fwd_bwd(DEPTH, P, tok, tgt)
+    fb = time.perf_counter() - t0
+    d = 64 * DEPTH
+    t0 = time.perf_counter()
+    oracle.newton_schulz(P[1])                  # one d x d matrix (of 80)
+    ns_sq = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.newton_schulz(P[5])                  # one 4d x d matrix (of 40)
+    ns_w = time.perf_counter() - t0
+    step_s = fb / t_tok * (B * T) + 4 * DEPTH * ns_sq + 2 * DEPTH * ns_w
+    return {
+        "value": (B * T) / step_s,
+        "unit": "tokens/s",
+        "cores": int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1)),
+        "kind": "oracle",
+        "sample": ("double-precision CPU oracle: forward+backward of depth 20 on 1 x %d tokens "
+                   "(%.1f s) scaled to 65536 tokens, plus Newton-Schulz of one 1280x1280 "
+                   "(%.1f s) and one 5120x1280 matrix (%.1f s) scaled to 80 + 40 matrices"
+                   % (t_tok, fb, ns_sq, ns_w)),
+        "sample_seconds": fb + ns_sq + ns_w,
+    }
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args, rank):
+    if rank != 0:
+        return 0
+    from pretraining_step_b200 import inputs
+    import oracle
+    oracle.lib()
+    P = inputs.random_params(DEPTH, seed=1)
+    t_tok = 8
+    times_fb, times_ns = [], {"sq": [], "w": []}
+    for step in range(args.warmup + args.steps):
+        tok, tgt = inputs.token_batch(100 + step, 1, t_tok)
+        t0 = time.perf_counter()
+        oracle.gpt_fwd_bwd(DEPTH, P, tok, tgt)
+        fb = time.perf_counter() - t0
+        which = "sq" if step % 2 == 0 else "w"
+        t0 = time.perf_counter()
+        oracle.newton_schulz(P[1] if which == "sq" else P[5])
+        ns = time.perf_counter() - t0
+        if step >= args.warmup:
+            times_fb.append(fb)
+            times_ns[which].append(ns)
+    fb_tok = float(np.mean(times_fb)) / t_tok
+    ns_sq = float(np.mean(times_ns["sq"])) if times_ns["sq"] else 0.0
+    ns_w = float(np.mean(times_ns["w"])) if times_ns["w"] else ns_sq * 4.5
+    step_s = fb_tok * B * T + 4 * DEPTH * ns_sq + 2 * DEPTH * ns_w
+    value = B * T / step_s
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_name(), "global_batch": B, "seq_len": T,
+                   "parallelism": "none (host cores)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": "each step: oracle forward+backward on 1 x %d tokens and "
+                                   "Newton-Schulz of one block matrix (alternating 1280x1280 / "
+                                   "5120x1280), scaled to the 65536-token step and 120 "
+                                   "matrices" % t_tok},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ native arm
+def run_native(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from pretraining_step_b200 import binding as nc
+    from pretraining_step_b200 import inputs
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.Stream(device=dev)
+    peaks, peak_kind = load_peaks()
+
+    m = nc.GPT(DEPTH, vocab=V, seed=1234 + rank, all_random=True, stream=stream)
+    # A few distinct batches, resident in HBM.
+    nbat = 4
+    toks, tgts = [], []
+    for i in range(nbat):
+        tk, tg = inputs.token_batch(20 + 97 * rank + i, B, T)
+        toks.append(torch.from_numpy(tk).to(dev))
+        tgts.append(torch.from_numpy(tg).to(dev))
+    loss_dev = torch.zeros(1, dtype=torch.float32, device=dev)
+    torch.cuda.synchronize()
+
+    def step(i):
+        m.fwd_bwd_async(toks[i % nbat], tgts[i % nbat], loss_dev)
+        m.muon_step(LR, MOMENTUM)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+        m.sync()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---- device-timed region (inputs resident)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    m.profile(True)
+    m.profile_read()  # reset
+    launches0 = m.launch_count()
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        e1.record(stream)
+    m.sync()
+    torch.cuda.synchronize()
+    barrier()
+    launches = m.launch_count() - launches0
+    ms = e0.elapsed_time(e1)
+    prof = m.profile_read()
+    m.profile(False)
+    clk = clocks.stop()
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    final_loss = float(loss_dev.item())
+
+    # ---- end-to-end through the C ABI with host buffers
+    pin_tok = [torch.from_numpy(inputs.token_batch(20 + 97 * rank + i, B, T)[0]).pin_memory()
+               for i in range(nbat)]
+    pin_tgt = [torch.from_numpy(inputs.token_batch(20 + 97 * rank + i, B, T)[1]).pin_memory()
+               for i in range(nbat)]
+    e2e_steps = max(3, args.steps // 2)
+    barrier()
+    torch.cuda.synchronize()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        f0.record(stream)
+        for i in range(e2e_steps):
+            tk = pin_tok[i % nbat]
+            tg = pin_tgt[i % nbat]
+            # Host pointers: nc_gpt_fwd_bwd copies them in and returns the loss.
+            m.fwd_bwd(tk.numpy(), tg.numpy())
+            m.muon_step(LR, MOMENTUM)
+        f1.record(stream)
+    m.sync()
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    m.close()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_sample()
+
+    if rank != 0:
+        return 0
+    tokens = args.steps * B * T * world
+    value = tokens / (ms_max / 1e3)
+    tflops = value * model_flops_per_token() / 1e12
+    # Dominant kernel: the tcgen05 GEMM (largest share of device time).
+    total_ms = sum(v["ms"] for v in prof.values()) or 1.0
+    kernels = {}
+    for name, v in sorted(prof.items(), key=lambda kv: -kv[1]["ms"]):
+        ent = {"launches": v["launches"], "ms": round(v["ms"], 3),
+               "share": round(v["ms"] / total_ms, 4)}
+        if v["flops"] > 0:
+            ach = v["flops"] / (v["ms"] / 1e3) / 1e12
+            ent.update(achieved_tflops=round(ach, 1),
+                       frac=round(ach / peaks["bf16_tflops_sustained"], 3))
+        elif v["bytes"] > 0:
+            ach = v["bytes"] / (v["ms"] / 1e3) / 1e9
+            ent.update(achieved_gbs=round(ach, 1), frac=round(ach / peaks["hbm_gbs"], 3))
+        kernels[name] = ent
+    g = prof.get("gemm_tc", {"flops": 0.0, "ms": 1.0, "launches": 1})
+    gemm_ach = g["flops"] / (g["ms"] / 1e3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic uniform token ids (SplitMix64), random-init weights",
+        "config": {"workload": workload_name(), "global_batch": B * world, "seq_len": T,
+                   "parallelism": "replicas" if world > 1 else "single-gpu",
+                   "l2": "working set (~55 GB of saved activations per step) far above the "
+                         "126 MB L2; no flush needed"},
+        "tflops": tflops,
+        "mfu": tflops / NOMINAL_BF16_TFLOPS,
+        "mfu_vs_measured_sustained": tflops / peaks["bf16_tflops_sustained"],
+        "flops_per_token": model_flops_per_token(),
+        "muon_ns_tflop_per_step": ns_flops() / 1e12,
+        "final_loss": final_loss,
+        "roofline": {"kernel": "gemm_tc", "bound": "tensor", "achieved": gemm_ach,
+                     "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": gemm_ach / peaks["bf16_tflops_sustained"], "traffic": None,
+                     "peak_source": peak_kind + " bf16_tflops_sustained"},
+        "kernels": kernels,
+        "gpu_launches": int(launches),
+        "e2e": {"value": e2e_steps * B * T * world / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": 2 * B * T * 4, "d2h_bytes_per_step": 8,
+                "steps": e2e_steps},
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ single-kernel modes
+def run_op(args):
+    """Time one kernel class alone (for tuning and ncu captures on a small
+    case): --op gemm --shape M,N,K[,a_kmajor,b_kmajor] or --op attn --shape B,T,H."""
+    import torch
+    from pretraining_step_b200 import binding as nc
+    peaks, peak_kind = load_peaks()
+    torch.manual_seed(0)
+    dims = [int(x) for x in args.shape.split(",")]
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    if args.op == "gemm":
+        M, N, K = dims[:3]
+        ak = dims[3] if len(dims) > 3 else 1
+        bk = dims[4] if len(dims) > 4 else 1
+        A = torch.randn(M * K, device="cuda").to(torch.bfloat16)
+        Bm = (torch.randn(N * K, device="cuda") * K ** -0.5).to(torch.bfloat16)
+        D = torch.empty(M * N, device="cuda", dtype=torch.bfloat16)
+        run = lambda: nc.gemm(M, N, K, A, Bm, D, a_kmajor=ak, b_kmajor=bk)
+        flops, nbytes = 2.0 * M * N * K, 2.0 * (M * K + N * K + M * N)
+    else:
+        Bb, T_, H = dims
+        d = H * 128
+        qkv = torch.randn(Bb * T_ * 3 * d, device="cuda").to(torch.bfloat16).view(Bb * T_, 3 * d)
+        o = torch.empty(Bb * T_, d, device="cuda", dtype=torch.bfloat16)
+        lse = torch.empty(Bb, H, T_, device="cuda", dtype=torch.float32)
+        run = lambda: nc.attention_fwd(qkv, qkv[:, d:], qkv[:, 2 * d:], 3 * d, o, d, lse, Bb,
+                                       T_, H)
+        flops, nbytes = 4.0 * Bb * H * 128 * T_ * (T_ + 1) / 2, 2.0 * Bb * T_ * 4 * d
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+    ev[0].record()
+    for _ in range(args.steps):
+        run()
+    ev[1].record()
+    torch.cuda.synchronize()
+    ms = ev[0].elapsed_time(ev[1]) / args.steps
+    tf = flops / (ms / 1e3) / 1e12
+    print(json.dumps({"op": args.op, "shape": dims, "ms_per_launch": ms, "tflops": tf,
+                      "frac_of_burst_peak": tf / peaks["bf16_tflops"],
+                      "peak_source": peak_kind, "algorithmic_bytes": nbytes}), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", choices=["gemm", "attn"], default=None,
+                    help="time one kernel class alone instead of the step")
+    ap.add_argument("--shape", default="16384,5120,1280")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+    if args.op:
+        return run_op(args)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        return run_native(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())
