@@ -216,6 +216,29 @@ nc_status nc_op_attention_bwd(const void* q, const void* k, const void* v, int64
                               float* dq, void* dk, void* dv, int64_t ldg, float* delta_scratch,
                               int B, int T, int H, void* stream);
 
+/* Causal attention backward like nc_op_attention_bwd, for callers that
+ * cannot allocate device memory (no cudaMalloc / cudaFree of their own, no
+ * workspace they can lend): a caller running while another component owns
+ * the whole device-memory budget, a path that must not risk the implicit
+ * device synchronisation cudaMalloc and cudaFree can cause, or a caller with
+ * nowhere to keep a workspace between calls.  The guide has no counterpart:
+ * this is a property of the library, not of the method.
+ * The D = rowsum(dO * O) scratch lives in a fixed 4 MiB array inside the
+ * library's device image (held on every device that loads the library until
+ * the process exits), so B * H * T must not exceed 1048576; larger sizes
+ * return NC_ERR_INVALID_ARG before anything is launched.  Nothing is
+ * allocated: no cudaMalloc, cudaFree or allocating library routine.
+ * The first call on each device looks up the array's device address (with
+ * that device current) and should come before any stream capture.
+ * Every call shares the array and it keeps the last call's contents (each
+ * call rewrites the entries it uses before reading them); calls that overlap
+ * on the GPU (different streams, or graphs running concurrently) race on it.
+ * Inputs, outputs and errors otherwise as nc_op_attention_bwd. */
+nc_status nc_op_attention_bwd_noalloc(const void* q, const void* k, const void* v, int64_t ld,
+                                      const void* o, const void* dout, int64_t ldo,
+                                      const float* lse, float* dq, void* dk, void* dv,
+                                      int64_t ldg, int B, int T, int H, void* stream);
+
 /* Newton-Schulz orthogonalisation of `count` matrices [rows, cols] (bf16
  * in and out, dense, batch stride rows*cols): Frobenius normalisation
  * (eps 1e-7) then `steps` quintic steps with the coefficients above, on the

@@ -94,6 +94,8 @@ def lib():
         "nc_op_attention_fwd": (ci, [vp, vp, vp, i64, vp, i64, vp, ci, ci, ci, vp]),
         "nc_op_attention_bwd": (ci, [vp, vp, vp, i64, vp, vp, i64, vp, vp, vp, vp, i64, vp,
                                      ci, ci, ci, vp]),
+        "nc_op_attention_bwd_noalloc": (ci, [vp, vp, vp, i64, vp, vp, i64, vp, vp, vp, vp,
+                                             i64, ci, ci, ci, vp]),
         "nc_newton_schulz_scratch_bytes": (ctypes.c_size_t, [ci, ci, ci]),
         "nc_op_newton_schulz": (ci, [vp, vp, ci, ci, ci, ci, vp, vp]),
         "nc_profile_enable": (ci, [vp, ci]),
@@ -289,6 +291,14 @@ def attention_bwd(q, k, v, ld, o, dout, ldo, lse, dq, dk, dv, ldg, delta, B, T, 
     _check(lib().nc_op_attention_bwd(_ptr(q), _ptr(k), _ptr(v), ld, _ptr(o), _ptr(dout), ldo,
                                      _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), ldg, _ptr(delta),
                                      B, T, H, _stream(stream)))
+
+
+def attention_bwd_noalloc(q, k, v, ld, o, dout, ldo, lse, dq, dk, dv, ldg, B, T, H,
+                          stream=None):
+    """Attention backward that allocates nothing (scratch inside the library)."""
+    _check(lib().nc_op_attention_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), ld, _ptr(o),
+                                             _ptr(dout), ldo, _ptr(lse), _ptr(dq), _ptr(dk),
+                                             _ptr(dv), ldg, B, T, H, _stream(stream)))
 
 
 def newton_schulz_scratch_bytes(count, rows, cols):

@@ -13,6 +13,8 @@
 // with D = rowsum(dO * O) from a separate pass.  Scale 1/sqrt(128) is folded
 // into S, dK and dQ.
 
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 #include "kernels.h"
@@ -494,4 +496,57 @@ nc_status attention_bwd(const void* q, const void* k, const void* v, int64_t ld,
   return NC_OK;
 }
 
+// ------------------------------------------------------------------ allocation-free backward
+// Scratch for the row sums D = rowsum(dO * O) of nc_op_attention_bwd_noalloc:
+// a fixed array in the library's device image, so that entry point needs no
+// allocation.  Every device that loads the library holds these 4 MiB until
+// the process exits.
+namespace {
+constexpr int64_t kNoAllocDeltaMax = int64_t(1) << 20;  // floats: B * H * T limit
+static __device__ __align__(256) float g_attn_delta_scratch[kNoAllocDeltaMax];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+float* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once
+// per device.  In host code the array's name only stands in for the symbol;
+// cudaGetSymbolAddress turns it into the address kernels may use.
+nc_status noalloc_scratch(float** out) {
+  int dev = 0;
+  NC_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(NC_ERR_UNSUPPORTED, "device index too large");
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_attn_delta_scratch);
+    if (e != cudaSuccess || !ptr) return cuda_fail(e, "cudaGetSymbolAddress(attention scratch)");
+    g_scratch_ptr[dev] = static_cast<float*>(ptr);
+  }
+  *out = g_scratch_ptr[dev];
+  return NC_OK;
+}
+}  // namespace
+
 }  // namespace nc
+
+extern "C" nc_status nc_op_attention_bwd_noalloc(const void* q, const void* k, const void* v,
+                                                 int64_t ld, const void* o, const void* dout,
+                                                 int64_t ldo, const float* lse, float* dq,
+                                                 void* dk, void* dv, int64_t ldg, int B, int T,
+                                                 int H, void* stream) {
+  using namespace nc;
+  if (B < 1 || T < 1 || H < 1)
+    return fail(NC_ERR_INVALID_ARG, "attention_bwd_noalloc: B, T and H must be positive");
+  if ((int64_t)B * H * T > kNoAllocDeltaMax)
+    return fail(NC_ERR_INVALID_ARG,
+                "attention_bwd_noalloc: B*H*T = " + std::to_string((int64_t)B * H * T) +
+                    " exceeds the built-in scratch of " + std::to_string(kNoAllocDeltaMax) +
+                    " rows; use nc_op_attention_bwd with a caller-provided buffer");
+  float* delta = nullptr;
+  NC_TRY(noalloc_scratch(&delta));
+  // The row-sum pass rewrites every entry it reads, so nothing from an
+  // earlier call leaks into this one and no clearing is needed.
+  return attention_bwd(q, k, v, ld, o, dout, ldo, lse, dq, dk, dv, ldg, delta, B, T, H,
+                       static_cast<cudaStream_t>(stream), nullptr);
+}
