@@ -1,10 +1,5 @@
-// attention.cu -- causal softmax attention, forward and backward, head_dim 128.
-//
-// Forward: one CTA (4 warps) per 64-query block of one (batch, head); each
-// warp owns 16 query rows.  K/V tiles of 64 keys stream through a
-// double-buffered cp.async shared-memory ring; S = Q K^T and O += P V run on
-// the tensor cores (mma.m16n8k16, bf16 in, fp32 accumulate) with an online
-// softmax in the exp2 domain.  Saves lse = m + ln(l) per row.
+// attention.cu -- causal softmax attention backward, head_dim 128 (the
+// forward is in attention_tc.cu).
 //
 // Backward: one CTA (8 warps) per 64-key block; loops over the query blocks
 // at or after it.  Recomputes P^T = exp(S^T - lse) from the saved lse,
@@ -72,162 +67,6 @@ __device__ __forceinline__ void load_tile(__nv_bfloat16* s, const __nv_bfloat16*
     const bool ok = (r0 + r) < T;
     const __nv_bfloat16* src = g + (int64_t)(ok ? r0 + r : 0) * ld + c;
     cp_async16(s + r * LDS + c, src, ok);
-  }
-}
-
-// ------------------------------------------------------------------ forward
-__global__ void __launch_bounds__(128) attn_fwd_kernel(const __nv_bfloat16* __restrict__ q,
-                                                       const __nv_bfloat16* __restrict__ k,
-                                                       const __nv_bfloat16* __restrict__ v,
-                                                       int64_t ld, __nv_bfloat16* __restrict__ o,
-                                                       int64_t ldo, float* __restrict__ lse,
-                                                       int T, int H) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem_raw);
-  __nv_bfloat16* sK = sQ + 64 * LDS;  // [2][64][LDS]
-  __nv_bfloat16* sV = sK + 2 * 64 * LDS;
-
-  const int nqb = (T + BQ - 1) / BQ;
-  const int qb = nqb - 1 - blockIdx.x;  // heaviest blocks first
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, t4 = lane & 3;
-
-  const int64_t base = (int64_t)b * T * ld + (int64_t)h * HD;
-  const __nv_bfloat16* qg = q + base;
-  const __nv_bfloat16* kg = k + base;
-  const __nv_bfloat16* vg = v + base;
-  const int q0 = qb * BQ;
-  const int nkb = qb + 1;  // causal: key blocks 0..qb
-
-  load_tile<128>(sQ, qg, ld, q0, T);
-  load_tile<128>(sK, kg, ld, 0, T);
-  load_tile<128>(sV, vg, ld, 0, T);
-  cp_commit();
-
-  uint32_t qf[8][4];
-  float oacc[16][4];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  const float sl2 = kLog2e * rsqrtf((float)HD);
-  const int qrow0 = q0 + warp * 16 + g, qrow1 = qrow0 + 8;
-
-  for (int kb = 0; kb < nkb; ++kb) {
-    const int buf = kb & 1;
-    if (kb + 1 < nkb) {
-      load_tile<128>(sK + (buf ^ 1) * 64 * LDS, kg, ld, (kb + 1) * BKV, T);
-      load_tile<128>(sV + (buf ^ 1) * 64 * LDS, vg, ld, (kb + 1) * BKV, T);
-      cp_commit();
-      cp_wait<1>();
-    } else {
-      cp_wait<0>();
-    }
-    __syncthreads();
-    if (kb == 0) {
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-        ldsm_x4(qf[ks], s_u32(sQ + (warp * 16 + (lane & 15)) * LDS + ks * 16 + (lane >> 4) * 8));
-    }
-    const __nv_bfloat16* cK = sK + buf * 64 * LDS;
-    const __nv_bfloat16* cV = sV + buf * 64 * LDS;
-
-    float s[8][4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-#pragma unroll
-      for (int np = 0; np < 4; ++np) {
-        uint32_t bb[4];
-        const int j = lane >> 3;
-        ldsm_x4(bb, s_u32(cK + ((np * 2 + (j >> 1)) * 8 + (lane & 7)) * LDS + ks * 16 + (j & 1) * 8));
-        mma16816(s[2 * np], qf[ks], bb[0], bb[1]);
-        mma16816(s[2 * np + 1], qf[ks], bb[2], bb[3]);
-      }
-    }
-    // Scale, causal / length mask, online softmax (exp2 domain).
-    const int k0 = kb * BKV;
-    float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-    for (int nb = 0; nb < 8; ++nb) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int kj = k0 + nb * 8 + 2 * t4 + e;
-        float a = s[nb][e] * sl2, c = s[nb][2 + e] * sl2;
-        if (kj > qrow0 || kj >= T) a = -INFINITY;
-        if (kj > qrow1 || kj >= T) c = -INFINITY;
-        s[nb][e] = a;
-        s[nb][2 + e] = c;
-        mx0 = fmaxf(mx0, a);
-        mx1 = fmaxf(mx1, c);
-      }
-    }
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-    const float mu0 = (mn0 == -INFINITY) ? 0.f : mn0;
-    const float mu1 = (mn1 == -INFINITY) ? 0.f : mn1;
-    const float c0 = exp2f(m0 - mu0), c1 = exp2f(m1 - mu1);
-    m0 = mn0;
-    m1 = mn1;
-    float rs0 = 0.f, rs1 = 0.f;
-    uint32_t pa[4][4];
-#pragma unroll
-    for (int nb = 0; nb < 8; ++nb) {
-      const float p0 = exp2f(s[nb][0] - mu0), p1 = exp2f(s[nb][1] - mu0);
-      const float p2 = exp2f(s[nb][2] - mu1), p3 = exp2f(s[nb][3] - mu1);
-      rs0 += p0 + p1;
-      rs1 += p2 + p3;
-      const int kk = nb >> 1, hi = nb & 1;
-      pa[kk][hi * 2 + 0] = pack_bf16x2(p0, p1);
-      pa[kk][hi * 2 + 1] = pack_bf16x2(p2, p3);
-    }
-    l0 = l0 * c0 + rs0;
-    l1 = l1 * c1 + rs1;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      oacc[i][0] *= c0;
-      oacc[i][1] *= c0;
-      oacc[i][2] *= c1;
-      oacc[i][3] *= c1;
-    }
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-#pragma unroll
-      for (int np = 0; np < 8; ++np) {
-        uint32_t bb[4];
-        const int j = lane >> 3;
-        ldsm_x4_t(bb, s_u32(cV + (kk * 16 + (j & 1) * 8 + (lane & 7)) * LDS + (np * 2 + (j >> 1)) * 8));
-        mma16816(oacc[2 * np], pa[kk], bb[0], bb[1]);
-        mma16816(oacc[2 * np + 1], pa[kk], bb[2], bb[3]);
-      }
-    }
-    __syncthreads();
-  }
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-  const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
-  __nv_bfloat16* og = o + (int64_t)b * T * ldo + (int64_t)h * HD;
-#pragma unroll
-  for (int nd = 0; nd < 16; ++nd) {
-    const int c = nd * 8 + 2 * t4;
-    if (qrow0 < T)
-      *reinterpret_cast<uint32_t*>(og + (int64_t)qrow0 * ldo + c) =
-          pack_bf16x2(oacc[nd][0] * inv0, oacc[nd][1] * inv0);
-    if (qrow1 < T)
-      *reinterpret_cast<uint32_t*>(og + (int64_t)qrow1 * ldo + c) =
-          pack_bf16x2(oacc[nd][2] * inv1, oacc[nd][3] * inv1);
-  }
-  if (t4 == 0) {
-    const float ln2 = 0.69314718055994531f;
-    float* lg = lse + ((int64_t)b * H + h) * T;
-    if (qrow0 < T) lg[qrow0] = (m0 + log2f(l0)) * ln2;
-    if (qrow1 < T) lg[qrow1] = (m1 + log2f(l1)) * ln2;
   }
 }
 
@@ -435,33 +274,9 @@ __global__ void __launch_bounds__(256) attn_bwd_kernel(
   }
 }
 
-constexpr int kFwdSmem = 5 * 64 * LDS * 2;
 constexpr int kBwdSmem = 4 * 64 * LDS * 2 + 2 * 64 * LDP * 2 + 2 * 64 * 4;
 
 }  // namespace
-
-nc_status attention_fwd(const void* q, const void* k, const void* v, int64_t ld, void* o,
-                        int64_t ldo, float* lse, int B, int T, int H, cudaStream_t s,
-                        Profiler* prof) {
-  if (B < 1 || T < 1 || H < 1 || !q || !k || !v || !o || !lse)
-    return fail(NC_ERR_INVALID_ARG, "attention_fwd: bad arguments");
-  if (ld % 8 || ldo % 8 || ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
-                             reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o)) & 15))
-    return fail(NC_ERR_INVALID_ARG, "attention_fwd: rows must be 16-byte aligned");
-  static bool attr = false;
-  if (!attr) {
-    NC_CUDA_TRY(cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFwdSmem));
-    attr = true;
-  }
-  const double flops = 4.0 * B * H * HD * ((double)T * (T + 1) / 2.0);  // causal QK^T + PV
-  Probe probe(prof, s, "attn_fwd", flops, 0.0);
-  dim3 grid((T + BQ - 1) / BQ, H, B);
-  attn_fwd_kernel<<<grid, 128, kFwdSmem, s>>>((const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
-                                              (const __nv_bfloat16*)v, ld, (__nv_bfloat16*)o, ldo,
-                                              lse, T, H);
-  NC_CUDA_TRY(cudaGetLastError());
-  return NC_OK;
-}
 
 nc_status attention_bwd(const void* q, const void* k, const void* v, int64_t ld, const void* o,
                         const void* dout, int64_t ldo, const float* lse, float* dq, void* dk,

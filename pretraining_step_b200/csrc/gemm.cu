@@ -18,7 +18,6 @@
 // status word and every role drains and exits.
 
 #include <algorithm>
-#include <mutex>
 
 #include "kernels.h"
 #include "tc.cuh"
@@ -383,41 +382,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------ host
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  });
-  return fn;
-}
-
-// 3-D bf16 tensor map {inner, outer, batch}, row stride ld and batch stride
-// in elements, box {64, box_outer, 1}, 128-byte swizzle, zero fill.
-bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t batch,
-              int64_t ld, int64_t bstride, uint32_t box_outer) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[3] = {inner, outer, batch};
-  cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)(batch > 1 ? bstride : ld * outer) * 2};
-  cuuint32_t box[3] = {64, box_outer, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 template <int BN>
 nc_status launch_bn(const nc_gemm_desc& d, int split, int* status, cudaStream_t s,
                     Profiler* prof) {
@@ -429,10 +393,10 @@ nc_status launch_bn(const nc_gemm_desc& d, int split, int* status, cudaStream_t 
     attr_set = true;
   }
   CUtensorMap ta, tb;
-  const bool ok_a = d.a_kmajor ? make_map(&ta, d.A, d.K, d.M, d.batch, d.lda, d.stride_a, BM)
-                               : make_map(&ta, d.A, d.M, d.K, d.batch, d.lda, d.stride_a, 64);
-  const bool ok_b = d.b_kmajor ? make_map(&tb, d.B, d.K, d.N, d.batch, d.ldb, d.stride_b, BN)
-                               : make_map(&tb, d.B, d.N, d.K, d.batch, d.ldb, d.stride_b, 64);
+  const bool ok_a = d.a_kmajor ? make_tmap_bf16_3d(&ta, d.A, d.K, d.M, d.batch, d.lda, d.stride_a, BM)
+                               : make_tmap_bf16_3d(&ta, d.A, d.M, d.K, d.batch, d.lda, d.stride_a, 64);
+  const bool ok_b = d.b_kmajor ? make_tmap_bf16_3d(&tb, d.B, d.K, d.N, d.batch, d.ldb, d.stride_b, BN)
+                               : make_tmap_bf16_3d(&tb, d.B, d.N, d.K, d.batch, d.ldb, d.stride_b, 64);
   if (!ok_a || !ok_b) return fail(NC_ERR_INVALID_ARG, "gemm: cuTensorMapEncodeTiled rejected an operand");
 
   Args a;

@@ -2,6 +2,7 @@
 // device pointers; bf16 tensors are passed as void*.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -9,6 +10,11 @@
 #include "internal.h"
 
 namespace nc {
+
+// 3-D bf16 TMA tensor map {inner, outer, batch} (element strides ld and
+// bstride), box {64, box_outer, 1}, 128-byte swizzle, zero fill out of range.
+bool make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                       uint64_t batch, int64_t ld, int64_t bstride, uint32_t box_outer);
 
 struct GemmLaunch {
   nc_gemm_desc d;
@@ -18,7 +24,7 @@ struct GemmLaunch {
 nc_status gemm_launch(const GemmLaunch& g, cudaStream_t s, Profiler* prof);
 
 nc_status attention_fwd(const void* q, const void* k, const void* v, int64_t ld, void* o,
-                        int64_t ldo, float* lse, int B, int T, int H, cudaStream_t s,
+                        int64_t ldo, float* lse, int B, int T, int H, int* status, cudaStream_t s,
                         Profiler* prof);
 nc_status attention_bwd(const void* q, const void* k, const void* v, int64_t ld, const void* o,
                         const void* dout, int64_t ldo, const float* lse, float* dq, void* dk,

@@ -330,7 +330,7 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
     NC_TRY(proj(p, a.h1[l], N, d, W, 3 * d, a.qkv[l], 3 * d, NC_EPI_STORE_BF16, nullptr, 0));
     NC_TRY(rope_qknorm_fwd(a.qkv[l], 3 * d, N, T, H, hd, p->rope, a.rq[l], a.rk[l], s, pr));
     NC_TRY(attention_fwd(a.qkv[l], a.qkv[l] + d, a.qkv[l] + 2 * d, 3 * d, a.o[l], d, a.lse[l], B,
-                         T, H, s, pr));
+                         T, H, p->status, s, pr));
     NC_TRY(proj(p, a.o[l], N, d, W + 3 * d2, d, a.xmid[l], d, NC_EPI_RESID_F32, a.x[l], d));
     NC_TRY(rmsnorm_fwd(a.xmid[l], N, (int)d, a.h2[l], a.r2[l], s, pr));
     NC_TRY(proj(p, a.h2[l], N, d, W + 4 * d2, F, a.a[l], F, NC_EPI_RELU2, nullptr, 0));
@@ -731,8 +731,8 @@ nc_status nc_op_rmsnorm(const float* x, int64_t rows, int cols, void* y_bf16, fl
 
 nc_status nc_op_attention_fwd(const void* q, const void* k, const void* v, int64_t ld, void* o,
                               int64_t ldo, float* lse, int B, int T, int H, void* stream) {
-  return attention_fwd(q, k, v, ld, o, ldo, lse, B, T, H, static_cast<cudaStream_t>(stream),
-                       nullptr);
+  return attention_fwd(q, k, v, ld, o, ldo, lse, B, T, H, nullptr,
+                       static_cast<cudaStream_t>(stream), nullptr);
 }
 
 nc_status nc_op_attention_bwd(const void* q, const void* k, const void* v, int64_t ld,
