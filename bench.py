@@ -373,9 +373,21 @@ def run_op(args):
         qkv = torch.randn(Bb * T_ * 3 * d, device="cuda").to(torch.bfloat16).view(Bb * T_, 3 * d)
         o = torch.empty(Bb * T_, d, device="cuda", dtype=torch.bfloat16)
         lse = torch.empty(Bb, H, T_, device="cuda", dtype=torch.float32)
-        run = lambda: nc.attention_fwd(qkv, qkv[:, d:], qkv[:, 2 * d:], 3 * d, o, d, lse, Bb,
+        fwd = lambda: nc.attention_fwd(qkv, qkv[:, d:], qkv[:, 2 * d:], 3 * d, o, d, lse, Bb,
                                        T_, H)
-        flops, nbytes = 4.0 * Bb * H * 128 * T_ * (T_ + 1) / 2, 2.0 * Bb * T_ * 4 * d
+        if args.op == "attn":
+            run = fwd
+            flops, nbytes = 4.0 * Bb * H * 128 * T_ * (T_ + 1) / 2, 2.0 * Bb * T_ * 4 * d
+        else:
+            fwd()
+            dout = torch.randn(Bb * T_, d, device="cuda").to(torch.bfloat16)
+            dq = torch.empty(Bb * T_, d, device="cuda", dtype=torch.float32)
+            dkv = torch.empty(Bb * T_, 2 * d, device="cuda", dtype=torch.bfloat16)
+            delta = torch.empty(Bb, H, T_, device="cuda", dtype=torch.float32)
+            run = lambda: nc.attention_bwd(qkv, qkv[:, d:], qkv[:, 2 * d:], 3 * d, o, dout, d,
+                                           lse, dq, dkv[:, :d], dkv[:, d:], 2 * d, delta, Bb, T_,
+                                           H)
+            flops, nbytes = 10.0 * Bb * H * 128 * T_ * (T_ + 1) / 2, 2.0 * Bb * T_ * 7 * d
     for _ in range(args.warmup):
         run()
     torch.cuda.synchronize()
@@ -399,7 +411,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["gemm", "attn"], default=None,
+    ap.add_argument("--op", choices=["gemm", "attn", "attn_bwd"], default=None,
                     help="time one kernel class alone instead of the step")
     ap.add_argument("--shape", default="16384,5120,1280")
     args = ap.parse_args()

@@ -31,16 +31,20 @@ namespace {
 
 constexpr int HD = 128;
 constexpr int BQ = 128;
-constexpr int BKV = 128;
+constexpr int BKV = 128;  // key tile of the backward
+constexpr int FKV = 64;   // key tile of the forward
 constexpr int kThreads = 192;
 constexpr int TILE = 128 * 128 * 2;  // one 128 x 128 bf16 tile: two 64-column swizzled boxes
+constexpr int KT = FKV * 128 * 2;    // forward K / V tile: [64 keys x 128 dims]
+constexpr int PTF = 128 * FKV * 2;   // forward P tile: [128 queries x 64 keys]
 constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + TILE;      // 2 stages
-constexpr int OFF_V = OFF_K + 2 * TILE;  // 2 stages
-constexpr int OFF_P = OFF_V + 2 * TILE;
-constexpr int OFF_BAR = OFF_P + TILE;
-constexpr int kSmem = OFF_BAR + 256 + 1024;
-constexpr uint32_t TM_S0 = 0, TM_O = 256, kTmemCols = 512;
+constexpr int OFF_K = OFF_Q + TILE;    // 2 stages
+constexpr int OFF_V = OFF_K + 2 * KT;  // 2 stages
+constexpr int OFF_P = OFF_V + 2 * KT;
+constexpr int OFF_BAR = OFF_P + PTF;
+constexpr int kSmem = OFF_BAR + 256 + 1024;  // 112 KB + barriers: two CTAs per SM
+constexpr uint32_t TM_S0 = 0, TM_O = 128, kFwdTmemCols = 256;
+constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.f;  // log2 units
 
 struct FwdArgs {
@@ -53,13 +57,21 @@ struct FwdArgs {
   int* status;
 };
 
+// 2^x by the MUFU instruction (ex2.approx, flush-to-zero): the softmax
+// arguments are <= 0 (or <= 8 with a stale maximum), far from its range limits.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = globaltimer();
   while (!tc::mbar_try_wait(bar, parity))
     if (globaltimer() - t0 > kWaitTimeoutNs) return;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const FwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -82,7 +94,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qb = a.nqb - 1 - (int)blockIdx.x;
   const int h = blockIdx.y, b = blockIdx.z;
-  const int n = qb + 1;  // causal: key tiles 0..qb (BQ == BKV)
+  const int n = min((qb + 1) * BQ, a.T + FKV - 1) / FKV;  // causal: key tiles up to the diagonal
 
   if (threadIdx.x == 0) {
     tc::mbar_init(q_full, 1);
@@ -101,7 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::fence_mbar_init();
   }
   if (warp == 1) {
-    tc::tmem_alloc(tmem_slot, kTmemCols);
+    tc::tmem_alloc(tmem_slot, kFwdTmemCols);
     tc::tmem_relinquish();
   }
   tc::tc_fence_before();
@@ -124,14 +136,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = j & 1;
         const uint32_t ph = (j >> 1) & 1;
         if (!tc::mbar_wait(&k_empty[s], ph ^ 1, abort_flag, a.status)) { ok = false; break; }
-        tc::mbar_arrive_expect_tx(&k_full[s], TILE);
-        tc::tma_load_3d(smem + OFF_K + s * TILE, &tk, &k_full[s], col0, j * BKV, b);
-        tc::tma_load_3d(smem + OFF_K + s * TILE + TILE / 2, &tk, &k_full[s], col0 + 64, j * BKV, b);
+        tc::mbar_arrive_expect_tx(&k_full[s], KT);
+        tc::tma_load_3d(smem + OFF_K + s * KT, &tk, &k_full[s], col0, j * FKV, b);
+        tc::tma_load_3d(smem + OFF_K + s * KT + KT / 2, &tk, &k_full[s], col0 + 64, j * FKV, b);
         ++issued_k;
         if (!tc::mbar_wait(&v_empty[s], ph ^ 1, abort_flag, a.status)) { ok = false; break; }
-        tc::mbar_arrive_expect_tx(&v_full[s], TILE);
-        tc::tma_load_3d(smem + OFF_V + s * TILE, &tv, &v_full[s], col0, j * BKV, b);
-        tc::tma_load_3d(smem + OFF_V + s * TILE + TILE / 2, &tv, &v_full[s], col0 + 64, j * BKV, b);
+        tc::mbar_arrive_expect_tx(&v_full[s], KT);
+        tc::tma_load_3d(smem + OFF_V + s * KT, &tv, &v_full[s], col0, j * FKV, b);
+        tc::tma_load_3d(smem + OFF_V + s * KT + KT / 2, &tv, &v_full[s], col0 + 64, j * FKV, b);
         ++issued_v;
       }
       if (!ok) {
@@ -143,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t id_s = tc::idesc_bf16_f32(128, 128, 0, 0);
+      const uint32_t id_s = tc::idesc_bf16_f32(128, FKV, 0, 0);
       const uint32_t id_pv = tc::idesc_bf16_f32(128, 128, 0, 1);
       const uint32_t q_addr = tc::smem_u32(smem + OFF_Q);
       const uint32_t p_addr = tc::smem_u32(smem + OFF_P);
@@ -158,12 +170,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc::tc_fence_after();
-          const uint32_t k_addr = tc::smem_u32(smem + OFF_K + s * TILE);
+          const uint32_t k_addr = tc::smem_u32(smem + OFF_K + s * KT);
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (TILE / 2) + (kk & 3) * 32;
-            tc::umma_bf16_ss(tmem + TM_S0 + s * 128, tc::smem_desc_sw128(q_addr + off, 16, 1024),
-                             tc::smem_desc_sw128(k_addr + off, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+            const uint32_t qo = (kk >> 2) * (TILE / 2) + (kk & 3) * 32;
+            const uint32_t ko = (kk >> 2) * (KT / 2) + (kk & 3) * 32;
+            tc::umma_bf16_ss(tmem + TM_S0 + s * FKV, tc::smem_desc_sw128(q_addr + qo, 16, 1024),
+                             tc::smem_desc_sw128(k_addr + ko, 16, 1024), id_s, kk > 0 ? 1u : 0u);
           }
           tc::umma_commit(&s_full[s]);
           tc::umma_commit(&k_empty[s]);
@@ -178,14 +191,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc::tc_fence_after();
-          const uint32_t v_addr = tc::smem_u32(smem + OFF_V + s * TILE);
+          const uint32_t v_addr = tc::smem_u32(smem + OFF_V + s * KT);
 #pragma unroll
-          for (int kk = 0; kk < BKV / 16; ++kk) {
-            const uint32_t poff = (kk >> 2) * (TILE / 2) + (kk & 3) * 32;
-            tc::umma_bf16_ss(tmem + TM_O, tc::smem_desc_sw128(p_addr + poff, 16, 1024),
-                             tc::smem_desc_sw128(v_addr + kk * 2048, TILE / 2, 1024), id_pv,
+          for (int kk = 0; kk < FKV / 16; ++kk)
+            tc::umma_bf16_ss(tmem + TM_O, tc::smem_desc_sw128(p_addr + kk * 32, 16, 1024),
+                             tc::smem_desc_sw128(v_addr + kk * 2048, KT / 2, 1024), id_pv,
                              (jj > 0 || kk > 0) ? 1u : 0u);
-          }
           tc::umma_commit(pv_done);
           tc::umma_commit(&v_empty[s]);
         }
@@ -207,18 +218,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = tc::mbar_wait(&s_full[s], ph, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc::tc_fence_after();
-      uint32_t r[4][32];
+      uint32_t r[2][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tc::tmem_ld_32x32b_x32(lane_base + TM_S0 + s * 128 + c * 32, r[c]);
+      for (int c = 0; c < 2; ++c) tc::tmem_ld_32x32b_x32(lane_base + TM_S0 + s * FKV + c * 32, r[c]);
       tc::tmem_ld_wait();
       tc::tc_fence_before();
       tc::mbar_arrive(&s_empty[s]);
       // Scale, mask, block maximum.
-      const int k0 = j * BKV;
-      const bool diag = (j == qb);
+      const int k0 = j * FKV;
+      const bool diag = (k0 + FKV > qb * BQ);
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < 2; ++c)
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           float x = __uint_as_float(r[c][i]) * a.sl2;
@@ -229,18 +240,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       float alpha = 1.f;
       if (mx > m_used + kRescaleThreshold) {
-        alpha = exp2f(m_used - mx);  // 0 on the first tile
+        alpha = ex2(m_used - mx);  // 0 on the first tile
         m_used = mx;
       }
       const float mu = (m_used == -INFINITY) ? 0.f : m_used;
       l *= alpha;
-      uint32_t pk[64];
+      uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < 2; ++c)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = exp2f(__uint_as_float(r[c][2 * i]) - mu);
-          const float p1 = exp2f(__uint_as_float(r[c][2 * i + 1]) - mu);
+          const float p0 = ex2(__uint_as_float(r[c][2 * i]) - mu);
+          const float p1 = ex2(__uint_as_float(r[c][2 * i + 1]) - mu);
           l += p0 + p1;
           pk[c * 16 + i] = pack_bf16x2(p0, p1);
         }
@@ -265,13 +276,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P row -> K-major swizzled tile: 16-byte unit u of key chunk ch sits at
       // row*128 + ((u ^ (row & 7)) * 16) inside the chunk.
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch)
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint32_t* q4 = &pk[ch * 32 + u * 4];
-          tc::st_shared_v4(p_row + ch * (TILE / 2) + ((u ^ (row & 7)) << 4), q4[0], q4[1], q4[2],
-                           q4[3]);
-        }
+      for (int u = 0; u < 8; ++u)
+        tc::st_shared_v4(p_row + ((u ^ (row & 7)) << 4), pk[4 * u], pk[4 * u + 1], pk[4 * u + 2],
+                         pk[4 * u + 3]);
       tc::fence_proxy_async_smem();
       tc::tc_fence_before();
       tc::mbar_arrive(p_full);
@@ -309,6 +316,330 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, kFwdTmemCols);
+  }
+}
+
+
+// ------------------------------------------------------------------ backward
+// One CTA per (128-key tile, head, batch row); loops over the 64-query tiles
+// at or after it.  320 threads:
+//   warp 0      TMA: K and V once, then Q_i and dO_i through a 2-stage ring;
+//   warp 1      MMA issue, per query tile i:
+//                 S^T  = K Q_i^T        TMEM [  0, 64)   M 128 keys, N 64
+//                 dP^T = V dO_i^T       TMEM [ 64,128)
+//                 dV  += P^T dO_i       TMEM [256,384)   N 128 (dO MN-major)
+//                 dK  += dS^T Q_i       TMEM [384,512)   N 128 (Q MN-major)
+//                 dQ^T = K^T dS^T       TMEM [128,192)   M 128 dims, N 64
+//               (K^T and dS^T are the same shared tiles read MN-major);
+//   warps 2..5  one key row each: P^T = exp(S^T/sqrt(d) - lse),
+//               dS^T = P^T (dP^T - D), both as bf16 into K-major shared
+//               tiles; at the end dK, dV rows to global memory;
+//   warps 6..9  one head-dim row each: dQ^T row -> fp32 atomic adds into dq
+//               (a warp covers 32 consecutive dims of one query: coalesced).
+constexpr int BQB = 64;                  // query tile of the backward
+constexpr int QT = BQB * 128 * 2;        // 16 KB: [64 rows x 128 dims]
+constexpr int PT = 128 * BQB * 2;        // 16 KB: [128 keys x 64 queries]
+constexpr int B_OFF_K = 0;
+constexpr int B_OFF_V = B_OFF_K + TILE;
+constexpr int B_OFF_Q = B_OFF_V + TILE;       // 2 stages
+constexpr int B_OFF_DO = B_OFF_Q + 2 * QT;    // 2 stages
+constexpr int B_OFF_P = B_OFF_DO + 2 * QT;
+constexpr int B_OFF_DS = B_OFF_P + PT;
+constexpr int B_OFF_LD = B_OFF_DS + PT;  // per stage: lse * log2(e) [64], D [64] (f32)
+constexpr int B_OFF_BAR = B_OFF_LD + 2 * 2 * BQB * 4;
+constexpr int kBwdSmem = B_OFF_BAR + 256 + 1024;
+constexpr int kBwdThreads = 320;
+constexpr uint32_t TB_S = 0, TB_DP = 64, TB_DQ = 128, TB_DV = 256, TB_DK = 384;
+
+struct BwdArgs {
+  int T, H, nkb, nqb;
+  float sl2, scale;
+  const float* lse;
+  const float* delta;
+  float* dq;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  int64_t ldg;
+  int* status;
+};
+
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                       const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
+                       const BwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + B_OFF_BAR);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* qd_full = bars + 1;    // [2]
+  uint64_t* qd_empty = bars + 3;   // [2]
+  uint64_t* sdp_full = bars + 5;
+  uint64_t* sdp_empty = bars + 6;
+  uint64_t* pds_full = bars + 7;
+  uint64_t* pds_empty = bars + 8;
+  uint64_t* dq_full = bars + 9;
+  uint64_t* dq_empty = bars + 10;
+  uint64_t* dkv_full = bars + 11;
+  uint64_t* drained = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int i0 = (kb * BKV) / BQB;
+  const int nblk = a.nqb - i0;  // query tiles at or after this key tile
+  const int col0 = h * HD;
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(kv_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&qd_full[i], 32);  // the TMA lane (with its bytes) + 32 lse/D loader lanes
+      tc::mbar_init(&qd_empty[i], 1);
+    }
+    tc::mbar_init(sdp_full, 1);
+    tc::mbar_init(sdp_empty, 128);
+    tc::mbar_init(pds_full, 128);
+    tc::mbar_init(pds_empty, 1);
+    tc::mbar_init(dq_full, 1);
+    tc::mbar_init(dq_empty, 128);
+    tc::mbar_init(dkv_full, 1);
+    tc::mbar_init(drained, 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // Lane 0 issues the TMA copies; all 32 lanes stage lse * log2(e) and D of
+    // the query tile into shared memory and arrive on the same barrier.
+    const float* lse_bh = a.lse + ((int64_t)b * a.H + h) * a.T;
+    const float* d_bh = a.delta + ((int64_t)b * a.H + h) * a.T;
+    if (lane == 0) {
+      tc::tma_prefetch_desc(&tq);
+      tc::tma_prefetch_desc(&tk);
+      tc::tma_prefetch_desc(&tv);
+      tc::tma_prefetch_desc(&tdo);
+      tc::mbar_arrive_expect_tx(kv_full, 2 * TILE);
+      for (int c = 0; c < 2; ++c) {
+        tc::tma_load_3d(smem + B_OFF_K + c * (TILE / 2), &tk, kv_full, col0 + 64 * c, kb * BKV, b);
+        tc::tma_load_3d(smem + B_OFF_V + c * (TILE / 2), &tv, kv_full, col0 + 64 * c, kb * BKV, b);
+      }
+    }
+    int issued = 0;
+    bool ok = true;
+    for (int t = 0; t < nblk; ++t) {
+      const int st = t & 1;
+      const uint32_t ph = (t >> 1) & 1;
+      bool w = true;
+      if (lane == 0) w = tc::mbar_wait(&qd_empty[st], ph ^ 1, abort_flag, a.status);
+      if (!__shfl_sync(0xffffffffu, (int)w, 0)) { ok = false; break; }
+      const int q0 = (i0 + t) * BQB;
+      float* ld = reinterpret_cast<float*>(smem + B_OFF_LD) + st * 2 * BQB;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int c = lane + 32 * u;
+        const int q = q0 + c;
+        ld[c] = q < a.T ? lse_bh[q] * 1.4426950408889634f : INFINITY;
+        ld[BQB + c] = q < a.T ? d_bh[q] : 0.f;
+      }
+      if (lane == 0) {
+        tc::mbar_arrive_expect_tx(&qd_full[st], 2 * QT);
+        for (int c = 0; c < 2; ++c) {
+          tc::tma_load_3d(smem + B_OFF_Q + st * QT + c * (QT / 2), &tq, &qd_full[st], col0 + 64 * c, q0, b);
+          tc::tma_load_3d(smem + B_OFF_DO + st * QT + c * (QT / 2), &tdo, &qd_full[st], col0 + 64 * c, q0, b);
+        }
+      } else {
+        tc::mbar_arrive(&qd_full[st]);
+      }
+      ++issued;
+    }
+    if (!ok && lane == 0) {
+      drain_wait(kv_full, 0);
+      for (int t = max(0, issued - 2); t < issued; ++t) drain_wait(&qd_full[t & 1], (t >> 1) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id_sdp = tc::idesc_bf16_f32(128, BQB, 0, 0);
+      const uint32_t id_acc = tc::idesc_bf16_f32(128, 128, 0, 1);
+      const uint32_t id_dq = tc::idesc_bf16_f32(128, BQB, 1, 1);
+      const uint32_t k_addr = tc::smem_u32(smem + B_OFF_K);
+      const uint32_t v_addr = tc::smem_u32(smem + B_OFF_V);
+      const uint32_t p_addr = tc::smem_u32(smem + B_OFF_P);
+      const uint32_t ds_addr = tc::smem_u32(smem + B_OFF_DS);
+      bool ok = tc::mbar_wait(kv_full, 0, abort_flag, a.status);
+      // S^T and dP^T of query tile t into TMEM once the tile has landed and the
+      // softmax warps have read the previous scores.
+      auto issue_sdp = [&](int t) -> bool {
+        const int st = t & 1;
+        if (!tc::mbar_wait(&qd_full[st], (t >> 1) & 1, abort_flag, a.status)) return false;
+        if (t > 0 && !tc::mbar_wait(sdp_empty, (t - 1) & 1, abort_flag, a.status)) return false;
+        tc::tc_fence_after();
+        const uint32_t q_addr = tc::smem_u32(smem + B_OFF_Q + st * QT);
+        const uint32_t do_addr = tc::smem_u32(smem + B_OFF_DO + st * QT);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t ao = (kk >> 2) * (TILE / 2) + (kk & 3) * 32;
+          const uint32_t bo = (kk >> 2) * (QT / 2) + (kk & 3) * 32;
+          tc::umma_bf16_ss(tmem + TB_S, tc::smem_desc_sw128(k_addr + ao, 16, 1024),
+                           tc::smem_desc_sw128(q_addr + bo, 16, 1024), id_sdp, kk > 0 ? 1u : 0u);
+          tc::umma_bf16_ss(tmem + TB_DP, tc::smem_desc_sw128(v_addr + ao, 16, 1024),
+                           tc::smem_desc_sw128(do_addr + bo, 16, 1024), id_sdp, kk > 0 ? 1u : 0u);
+        }
+        tc::umma_commit(sdp_full);
+        return true;
+      };
+      if (ok) ok = issue_sdp(0);
+      for (int t = 0; t < nblk && ok; ++t) {
+        const int st = t & 1;
+        if (t + 1 < nblk && !issue_sdp(t + 1)) { ok = false; break; }
+        if (!tc::mbar_wait(pds_full, t & 1, abort_flag, a.status) ||
+            !tc::mbar_wait(dq_empty, (t & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+        tc::tc_fence_after();
+        const uint32_t q_addr = tc::smem_u32(smem + B_OFF_Q + st * QT);
+        const uint32_t do_addr = tc::smem_u32(smem + B_OFF_DO + st * QT);
+#pragma unroll
+        for (int kk = 0; kk < BQB / 16; ++kk) {
+          const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+          tc::umma_bf16_ss(tmem + TB_DV, tc::smem_desc_sw128(p_addr + kk * 32, 16, 1024),
+                           tc::smem_desc_sw128(do_addr + kk * 2048, QT / 2, 1024), id_acc, acc);
+          tc::umma_bf16_ss(tmem + TB_DK, tc::smem_desc_sw128(ds_addr + kk * 32, 16, 1024),
+                           tc::smem_desc_sw128(q_addr + kk * 2048, QT / 2, 1024), id_acc, acc);
+        }
+#pragma unroll
+        for (int kk = 0; kk < BKV / 16; ++kk)
+          tc::umma_bf16_ss(tmem + TB_DQ, tc::smem_desc_sw128(k_addr + kk * 2048, TILE / 2, 1024),
+                           tc::smem_desc_sw128(ds_addr + kk * 2048, PT, 1024), id_dq,
+                           kk > 0 ? 1u : 0u);
+        tc::umma_commit(pds_empty);
+        tc::umma_commit(&qd_empty[st]);
+        tc::umma_commit(dq_full);
+      }
+      if (ok) tc::umma_commit(dkv_full);
+      tc::umma_commit(drained);
+      drain_wait(drained, 0);
+    }
+  } else if (warp < 6) {
+    // ---------------- P^T and dS^T, one key row per thread
+    const int qw = warp & 3;
+    const int row = qw * 32 + lane;
+    const int key = kb * BKV + row;
+    const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
+    const uint32_t p_row = tc::smem_u32(smem + B_OFF_P) + row * 128;
+    const uint32_t ds_row = tc::smem_u32(smem + B_OFF_DS) + row * 128;
+    bool ok = true;
+    for (int t = 0; t < nblk; ++t) {
+      const int q0 = (i0 + t) * BQB;
+      const float* ld = reinterpret_cast<const float*>(smem + B_OFF_LD) + (t & 1) * 2 * BQB;
+      ok = tc::mbar_wait(sdp_full, t & 1, abort_flag, a.status);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc::tc_fence_after();
+      uint32_t sv[64], dp[64];
+      tc::tmem_ld_32x32b_x32(lane_base + TB_S, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tc::tmem_ld_32x32b_x32(lane_base + TB_S + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tc::tmem_ld_32x32b_x32(lane_base + TB_DP, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+      tc::tmem_ld_32x32b_x32(lane_base + TB_DP + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+      tc::tmem_ld_wait();
+      tc::tc_fence_before();
+      tc::mbar_arrive(sdp_empty);
+      // The query tile's lse/D, staged by the TMA warp and published by the
+      // stage's qd_full barrier (already complete: the scores came from it).
+      ok = tc::mbar_wait(&qd_full[t & 1], (t >> 1) & 1, abort_flag, a.status);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      uint32_t pp[32], pd[32];
+      const bool edge = (q0 < key + 1) || (q0 + BQB > a.T) || (key >= a.T);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const int qa = q0 + 2 * c, qb2 = qa + 1;
+        float p0 = ex2(__uint_as_float(sv[2 * c]) * a.sl2 - ld[2 * c]);
+        float p1 = ex2(__uint_as_float(sv[2 * c + 1]) * a.sl2 - ld[2 * c + 1]);
+        if (edge) {
+          if (qa < key || qa >= a.T || key >= a.T) p0 = 0.f;
+          if (qb2 < key || qb2 >= a.T || key >= a.T) p1 = 0.f;
+        }
+        const float d0 = p0 * (__uint_as_float(dp[2 * c]) - ld[BQB + 2 * c]);
+        const float d1 = p1 * (__uint_as_float(dp[2 * c + 1]) - ld[BQB + 2 * c + 1]);
+        pp[c] = pack_bf16x2(p0, p1);
+        pd[c] = pack_bf16x2(d0, d1);
+      }
+      ok = tc::mbar_wait(pds_empty, (t & 1) ^ 1, abort_flag, a.status);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t sw = (uint32_t)((u ^ (row & 7)) << 4);
+        tc::st_shared_v4(p_row + sw, pp[4 * u], pp[4 * u + 1], pp[4 * u + 2], pp[4 * u + 3]);
+        tc::st_shared_v4(ds_row + sw, pd[4 * u], pd[4 * u + 1], pd[4 * u + 2], pd[4 * u + 3]);
+      }
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(pds_full);
+    }
+    if (ok) {
+      ok = tc::mbar_wait(dkv_full, 0, abort_flag, a.status);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      tc::tc_fence_after();
+      const int64_t grow = ((int64_t)b * a.T + key) * a.ldg + col0;
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t base = lane_base + (which ? TB_DK : TB_DV);
+        const float mul = which ? a.scale : 1.f;
+        __nv_bfloat16* dst = (which ? a.dk : a.dv) + grow;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tc::tmem_ld_32x32b_x32(base + c * 32, o);
+          tc::tmem_ld_wait();
+          if (key < a.T) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              uint4 v;
+              v.x = pack_bf16x2(__uint_as_float(o[8 * u + 0]) * mul, __uint_as_float(o[8 * u + 1]) * mul);
+              v.y = pack_bf16x2(__uint_as_float(o[8 * u + 2]) * mul, __uint_as_float(o[8 * u + 3]) * mul);
+              v.z = pack_bf16x2(__uint_as_float(o[8 * u + 4]) * mul, __uint_as_float(o[8 * u + 5]) * mul);
+              v.w = pack_bf16x2(__uint_as_float(o[8 * u + 6]) * mul, __uint_as_float(o[8 * u + 7]) * mul);
+              reinterpret_cast<uint4*>(dst + c * 32)[u] = v;
+            }
+          }
+        }
+      }
+    }
+  } else {
+    // ---------------- dQ^T rows: one head-dim per thread, atomics into dq
+    const int qw = warp & 3;
+    const int dim = qw * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
+    const int64_t dq_row = (int64_t)a.H * HD;
+    float* dq_bh = a.dq + (int64_t)b * a.T * dq_row + col0 + dim;
+    for (int t = 0; t < nblk; ++t) {
+      const int q0 = (i0 + t) * BQB;
+      bool ok = tc::mbar_wait(dq_full, t & 1, abort_flag, a.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc::tc_fence_after();
+      uint32_t v[64];
+      tc::tmem_ld_32x32b_x32(lane_base + TB_DQ, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      tc::tmem_ld_32x32b_x32(lane_base + TB_DQ + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+      tc::tmem_ld_wait();
+      tc::tc_fence_before();
+      tc::mbar_arrive(dq_empty);
+      float* dst = dq_bh + (int64_t)q0 * dq_row;
+#pragma unroll
+      for (int c = 0; c < BQB; ++c)
+        if (q0 + c < a.T) atomicAdd(dst + (int64_t)c * dq_row, __uint_as_float(v[c]) * a.scale);
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
     tc::tmem_dealloc(tmem, kTmemCols);
   }
 }
@@ -332,9 +663,10 @@ nc_status attention_fwd(const void* q, const void* k, const void* v, int64_t ld,
   }
   CUtensorMap mq, mk, mv;
   const uint64_t cols = (uint64_t)H * HD;
-  if (!make_tmap_bf16_3d(&mq, q, cols, T, B, ld, (int64_t)T * ld, 128) ||
-      !make_tmap_bf16_3d(&mk, k, cols, T, B, ld, (int64_t)T * ld, 128) ||
-      !make_tmap_bf16_3d(&mv, v, cols, T, B, ld, (int64_t)T * ld, 128))
+  // Box heights must match the tile sizes the kernel's byte counts assume.
+  if (!make_tmap_bf16_3d(&mq, q, cols, T, B, ld, (int64_t)T * ld, BQ) ||
+      !make_tmap_bf16_3d(&mk, k, cols, T, B, ld, (int64_t)T * ld, FKV) ||
+      !make_tmap_bf16_3d(&mv, v, cols, T, B, ld, (int64_t)T * ld, FKV))
     return fail(NC_ERR_INVALID_ARG, "attention_fwd: cuTensorMapEncodeTiled rejected q/k/v");
   FwdArgs a;
   a.T = T;
@@ -349,6 +681,51 @@ nc_status attention_fwd(const void* q, const void* k, const void* v, int64_t ld,
   Probe probe(prof, s, "attn_fwd", flops, 0.0);
   dim3 grid(a.nqb, H, B);
   attn_fwd_tc_kernel<<<grid, kThreads, kSmem, s>>>(mq, mk, mv, a);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+
+nc_status attention_bwd_tc(const void* q, const void* k, const void* v, int64_t ld,
+                           const void* dout, int64_t ldo, const float* lse, const float* delta,
+                           float* dq, void* dk, void* dv, int64_t ldg, int B, int T, int H,
+                           int* status, cudaStream_t s, Profiler* prof) {
+  static bool attr = false;
+  if (!attr) {
+    NC_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc_kernel,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdSmem));
+    attr = true;
+  }
+  if (ld % 8 || ldo % 8 || ldg % 8 ||
+      ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+        reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(dout) |
+        reinterpret_cast<uintptr_t>(dk) | reinterpret_cast<uintptr_t>(dv)) & 15))
+    return fail(NC_ERR_INVALID_ARG, "attention_bwd: rows must be 16-byte aligned");
+  CUtensorMap mq, mk, mv, mdo;
+  const uint64_t cols = (uint64_t)H * HD;
+  if (!make_tmap_bf16_3d(&mq, q, cols, T, B, ld, (int64_t)T * ld, BQB) ||
+      !make_tmap_bf16_3d(&mk, k, cols, T, B, ld, (int64_t)T * ld, BKV) ||
+      !make_tmap_bf16_3d(&mv, v, cols, T, B, ld, (int64_t)T * ld, BKV) ||
+      !make_tmap_bf16_3d(&mdo, dout, cols, T, B, ldo, (int64_t)T * ldo, BQB))
+    return fail(NC_ERR_INVALID_ARG, "attention_bwd: cuTensorMapEncodeTiled rejected an operand");
+  BwdArgs a;
+  a.T = T;
+  a.H = H;
+  a.nkb = (T + BKV - 1) / BKV;
+  a.nqb = (T + BQB - 1) / BQB;
+  a.scale = (float)(1.0 / std::sqrt((double)HD));
+  a.sl2 = (float)(1.4426950408889634 / std::sqrt((double)HD));
+  a.lse = lse;
+  a.delta = delta;
+  a.dq = dq;
+  a.dk = static_cast<__nv_bfloat16*>(dk);
+  a.dv = static_cast<__nv_bfloat16*>(dv);
+  a.ldg = ldg;
+  a.status = status;
+  const double flops = 10.0 * B * H * HD * ((double)T * (T + 1) / 2.0);
+  Probe probe(prof, s, "attn_bwd", flops, 0.0);
+  dim3 grid(a.nkb, H, B);
+  attn_bwd_tc_kernel<<<grid, kBwdThreads, kBwdSmem, s>>>(mq, mk, mv, mdo, a);
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }

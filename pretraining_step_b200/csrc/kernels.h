@@ -28,8 +28,13 @@ nc_status attention_fwd(const void* q, const void* k, const void* v, int64_t ld,
                         Profiler* prof);
 nc_status attention_bwd(const void* q, const void* k, const void* v, int64_t ld, const void* o,
                         const void* dout, int64_t ldo, const float* lse, float* dq, void* dk,
-                        void* dv, int64_t ldg, float* delta, int B, int T, int H, cudaStream_t s,
-                        Profiler* prof);
+                        void* dv, int64_t ldg, float* delta, int B, int T, int H, int* status,
+                        cudaStream_t s, Profiler* prof);
+// The tcgen05 backward proper (delta = rowsum(dO * O) precomputed, dq zeroed).
+nc_status attention_bwd_tc(const void* q, const void* k, const void* v, int64_t ld,
+                           const void* dout, int64_t ldo, const float* lse, const float* delta,
+                           float* dq, void* dk, void* dv, int64_t ldg, int B, int T, int H,
+                           int* status, cudaStream_t s, Profiler* prof);
 
 nc_status embed_gather(const int32_t* tok, int64_t n, const float* E, int V, int d, float* x,
                        int* status, cudaStream_t s, Profiler* prof);

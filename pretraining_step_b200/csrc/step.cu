@@ -361,8 +361,8 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
     NC_TRY(proj_dw(p, a.dxb, d, d, a.o[l], d, d, N, G + 3 * d2));
     NC_TRY(proj_dx(p, a.dxb, N, d, W + 3 * d2, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0));
     NC_TRY(attention_bwd(a.qkv[l], a.qkv[l] + d, a.qkv[l] + 2 * d, 3 * d, a.o[l], a.dh, d,
-                         a.lse[l], a.dq, a.dqkv + d, a.dqkv + 2 * d, 3 * d, a.delta, B, T, H, s,
-                         pr));
+                         a.lse[l], a.dq, a.dqkv + d, a.dqkv + 2 * d, 3 * d, a.delta, B, T, H,
+                         p->status, s, pr));
     NC_TRY(rope_qknorm_bwd(a.dq, nullptr, 0, a.qkv[l], 3 * d, a.rq[l], N, T, H, hd, p->rope,
                            a.dqkv, 3 * d, s, pr));
     NC_TRY(rope_qknorm_bwd(nullptr, a.dqkv + d, 3 * d, a.qkv[l] + d, 3 * d, a.rk[l], N, T, H, hd,
@@ -740,7 +740,7 @@ nc_status nc_op_attention_bwd(const void* q, const void* k, const void* v, int64
                               float* dq, void* dk, void* dv, int64_t ldg, float* delta_scratch,
                               int B, int T, int H, void* stream) {
   return attention_bwd(q, k, v, ld, o, dout, ldo, lse, dq, dk, dv, ldg, delta_scratch, B, T, H,
-                       static_cast<cudaStream_t>(stream), nullptr);
+                       nullptr, static_cast<cudaStream_t>(stream), nullptr);
 }
 
 size_t nc_newton_schulz_scratch_bytes(int count, int rows, int cols) {
