@@ -127,11 +127,13 @@ __global__ void rope_table_kernel(float2* tab, int T, int hd) {
   tab[i] = make_float2((float)cos(th), (float)sin(th));
 }
 
-// In place on the q and k slices of qkv [n, ld]: rotate pairs (i, i + hd/2),
-// then RMS-normalise each head; rstd [n, H] per slice.  One warp per
-// (token, head, q|k).
+// In place on the q and k slices of qkv [n, ld] (head_dim 128): rotate pairs
+// (i, i + 64), then RMS-normalise each head; rstd [n, H] per slice.  One warp
+// per (token, head, q|k): lane l holds dims 4(l % 16) .. +3 of half l / 16, so
+// its rotation partner sits 16 lanes away (one shuffle), and every access is
+// an 8-byte vector.
 __global__ void rope_qknorm_fwd_kernel(__nv_bfloat16* __restrict__ qkv, int64_t ld, int64_t n,
-                                       int T, int H, int hd, const float2* __restrict__ tab,
+                                       int T, int H, const float2* __restrict__ tab,
                                        float* __restrict__ rstd_q, float* __restrict__ rstd_k) {
   const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -141,97 +143,99 @@ __global__ void rope_qknorm_fwd_kernel(__nv_bfloat16* __restrict__ qkv, int64_t 
   const int h = (int)(th % H);
   const int64_t tok = th / H;
   const int pos = (int)(tok % T);
-  const int half = hd / 2;
-  __nv_bfloat16* p = qkv + tok * ld + (int64_t)which * H * hd + (int64_t)h * hd;
-  float a[2], b[2];
+  const int half = lane >> 4, j = lane & 15;
+  uint2* p = reinterpret_cast<uint2*>(qkv + tok * ld + (int64_t)which * H * 128 + (int64_t)h * 128 +
+                                      half * 64 + 4 * j);
+  const uint2 xv = *p;
+  uint2 yv;
+  yv.x = __shfl_xor_sync(0xffffffffu, xv.x, 16);
+  yv.y = __shfl_xor_sync(0xffffffffu, xv.y, 16);
+  const float4* t4 = reinterpret_cast<const float4*>(tab + (int64_t)pos * 64 + 4 * j);
+  const float4 cs01 = t4[0], cs23 = t4[1];
+  const float c[4] = {cs01.x, cs01.z, cs23.x, cs23.z};
+  const float sn[4] = {cs01.y, cs01.w, cs23.y, cs23.w};
+  const float2 x01 = unpack_bf16x2(xv.x), x23 = unpack_bf16x2(xv.y);
+  const float2 y01 = unpack_bf16x2(yv.x), y23 = unpack_bf16x2(yv.y);
+  const float x[4] = {x01.x, x01.y, x23.x, x23.y};
+  const float y[4] = {y01.x, y01.y, y23.x, y23.y};
+  float o[4];
   float ss = 0.f;
 #pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int i = lane + 32 * u;
-    a[u] = b[u] = 0.f;
-    if (i < half) {
-      const float2 cs = tab[(int64_t)pos * half + i];
-      const float x0 = bf2f(p[i]), x1 = bf2f(p[i + half]);
-      a[u] = x0 * cs.x - x1 * cs.y;
-      b[u] = x0 * cs.y + x1 * cs.x;
-      ss += a[u] * a[u] + b[u] * b[u];
-    }
+  for (int e = 0; e < 4; ++e) {
+    // first half: x_i c - x_{i+64} s;  second half: x_i s + x_{i+64} c
+    o[e] = half == 0 ? x[e] * c[e] - y[e] * sn[e] : y[e] * sn[e] + x[e] * c[e];
+    ss += o[e] * o[e];
   }
   ss = warp_sum(ss);
-  const float rs = rsqrtf(ss / hd + kNormEps);
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int i = lane + 32 * u;
-    if (i < half) {
-      p[i] = f2bf(a[u] * rs);
-      p[i + half] = f2bf(b[u] * rs);
-    }
-  }
+  const float rs = rsqrtf(ss / 128.f + kNormEps);
+  uint2 ov;
+  ov.x = pack_bf16x2(o[0] * rs, o[1] * rs);
+  ov.y = pack_bf16x2(o[2] * rs, o[3] * rs);
+  *p = ov;
   if (lane == 0) (which ? rstd_k : rstd_q)[tok * H + h] = rs;
 }
 
-// Backward of the above for one slice: g = dL/dyhat (f32 dense [n, H*hd] for
+// Backward of the above for one slice: g = dL/dyhat (f32 dense [n, H*128] for
 // q, or bf16 with stride ldg for k), yhat the saved normalised output.
 //   dr = r * (g - yhat * mean(g * yhat));   dx = R(-theta) dr.
-// Writes bf16 into out (stride ld_out).
-__global__ void rope_qknorm_bwd_kernel(const float* __restrict__ gf, const __nv_bfloat16* __restrict__ gb,
+// Writes bf16 into out (stride ld_out); may run in place on the k slice.
+__global__ void rope_qknorm_bwd_kernel(const float* __restrict__ gf, const __nv_bfloat16* gb,
                                        int64_t ldg, const __nv_bfloat16* __restrict__ yhat,
                                        int64_t ldy, const float* __restrict__ rstd, int64_t n,
-                                       int T, int H, int hd, const float2* __restrict__ tab,
-                                       __nv_bfloat16* __restrict__ out, int64_t ld_out) {
+                                       int T, int H, const float2* __restrict__ tab,
+                                       __nv_bfloat16* out, int64_t ld_out) {
   const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (w >= n * H) return;
   const int h = (int)(w % H);
   const int64_t tok = w / H;
   const int pos = (int)(tok % T);
-  const int half = hd / 2;
-  const __nv_bfloat16* y = yhat + tok * ldy + (int64_t)h * hd;
-  float g0[2], g1[2], y0[2], y1[2];
-  float dot = 0.f;
-#pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int i = lane + 32 * u;
-    g0[u] = g1[u] = y0[u] = y1[u] = 0.f;
-    if (i < half) {
-      if (gf) {
-        const float* gp = gf + tok * ((int64_t)H * hd) + (int64_t)h * hd;
-        g0[u] = gp[i];
-        g1[u] = gp[i + half];
-      } else {
-        const __nv_bfloat16* gp = gb + tok * ldg + (int64_t)h * hd;
-        g0[u] = bf2f(gp[i]);
-        g1[u] = bf2f(gp[i + half]);
-      }
-      y0[u] = bf2f(y[i]);
-      y1[u] = bf2f(y[i + half]);
-      dot += g0[u] * y0[u] + g1[u] * y1[u];
-    }
+  const int half = lane >> 4, j = lane & 15;
+  const int col = h * 128 + half * 64 + 4 * j;
+  float g[4];
+  if (gf) {
+    const float4 v = *reinterpret_cast<const float4*>(gf + tok * ((int64_t)H * 128) + col);
+    g[0] = v.x; g[1] = v.y; g[2] = v.z; g[3] = v.w;
+  } else {
+    const uint2 v = *reinterpret_cast<const uint2*>(gb + tok * ldg + col);
+    const float2 a0 = unpack_bf16x2(v.x), a1 = unpack_bf16x2(v.y);
+    g[0] = a0.x; g[1] = a0.y; g[2] = a1.x; g[3] = a1.y;
   }
+  const uint2 yv = *reinterpret_cast<const uint2*>(yhat + tok * ldy + col);
+  const float2 y01 = unpack_bf16x2(yv.x), y23 = unpack_bf16x2(yv.y);
+  const float y[4] = {y01.x, y01.y, y23.x, y23.y};
+  float dot = g[0] * y[0] + g[1] * y[1] + g[2] * y[2] + g[3] * y[3];
   dot = warp_sum(dot);
   const float rs = rstd[tok * H + h];
-  const float m = dot / hd;
-  __nv_bfloat16* o = out + tok * ld_out + (int64_t)h * hd;
+  const float m = dot / 128.f;
+  float dr[4], pr[4];
 #pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int i = lane + 32 * u;
-    if (i < half) {
-      const float d0 = rs * (g0[u] - y0[u] * m), d1 = rs * (g1[u] - y1[u] * m);
-      const float2 cs = tab[(int64_t)pos * half + i];
-      o[i] = f2bf(d0 * cs.x + d1 * cs.y);
-      o[i + half] = f2bf(-d0 * cs.y + d1 * cs.x);
-    }
-  }
+  for (int e = 0; e < 4; ++e) dr[e] = rs * (g[e] - y[e] * m);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) pr[e] = __shfl_xor_sync(0xffffffffu, dr[e], 16);
+  const float4* t4 = reinterpret_cast<const float4*>(tab + (int64_t)pos * 64 + 4 * j);
+  const float4 cs01 = t4[0], cs23 = t4[1];
+  const float c[4] = {cs01.x, cs01.z, cs23.x, cs23.z};
+  const float sn[4] = {cs01.y, cs01.w, cs23.y, cs23.w};
+  float o[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    // first half: dr_i c + dr_{i+64} s;  second half: -dr_i s + dr_{i+64} c
+    o[e] = half == 0 ? dr[e] * c[e] + pr[e] * sn[e] : dr[e] * c[e] - pr[e] * sn[e];
+  uint2 ov;
+  ov.x = pack_bf16x2(o[0], o[1]);
+  ov.y = pack_bf16x2(o[2], o[3]);
+  *reinterpret_cast<uint2*>(out + tok * ld_out + col) = ov;
 }
 
 // ------------------------------------------------------------------ cross-entropy
-// One CTA (256 threads) per row of logits z[n, V] (bf16, V <= 32768, V % 8 == 0):
+// One CTA (512 threads) per row of logits z[n, V] (bf16, V <= 32768, V % 8 == 0):
 // loss_row = lse(z) - z[target];  z <- (softmax(z) - onehot(target)) * inv_n
 // in place.  The row stays in registers between the two reductions.
-constexpr int kCeThreads = 256;
-constexpr int kCeChunks = 16;  // 16 x 8 bf16 per thread -> V <= 32768
+constexpr int kCeThreads = 512;
+constexpr int kCeChunks = 8;  // 8 x 8 bf16 per thread -> V <= 32768
 
-__global__ void __launch_bounds__(kCeThreads) ce_fwd_bwd_kernel(__nv_bfloat16* __restrict__ z,
+__global__ void __launch_bounds__(kCeThreads, 2) ce_fwd_bwd_kernel(__nv_bfloat16* __restrict__ z,
                                                                 const int32_t* __restrict__ tgt,
                                                                 int V, float inv_n,
                                                                 float* __restrict__ loss_rows,
@@ -573,8 +577,9 @@ nc_status rope_qknorm_fwd(void* qkv, int64_t ld, int64_t n, int T, int H, int hd
                           const float2* tab, float* rstd_q, float* rstd_k, cudaStream_t s,
                           Profiler* prof) {
   Probe probe(prof, s, "rope_qknorm_fwd", 0.0, n * H * (2.0 * hd * 2 * 2 + 8.0));
+  if (hd != 128) return fail(NC_ERR_UNSUPPORTED, "rope_qknorm: head_dim must be 128");
   rope_qknorm_fwd_kernel<<<blocks_for(n * H * 2 * 32, 256), 256, 0, s>>>(
-      (__nv_bfloat16*)qkv, ld, n, T, H, hd, tab, rstd_q, rstd_k);
+      (__nv_bfloat16*)qkv, ld, n, T, H, tab, rstd_q, rstd_k);
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }
@@ -584,8 +589,9 @@ nc_status rope_qknorm_bwd(const float* gf, const void* gb, int64_t ldg, const vo
                           const float2* tab, void* out, int64_t ld_out, cudaStream_t s,
                           Profiler* prof) {
   Probe probe(prof, s, "rope_qknorm_bwd", 0.0, n * H * (hd * ((gf ? 4.0 : 2.0) + 2.0 + 2.0) + 4.0));
+  if (hd != 128) return fail(NC_ERR_UNSUPPORTED, "rope_qknorm: head_dim must be 128");
   rope_qknorm_bwd_kernel<<<blocks_for(n * H * 32, 256), 256, 0, s>>>(
-      gf, (const __nv_bfloat16*)gb, ldg, (const __nv_bfloat16*)yhat, ldy, rstd, n, T, H, hd, tab,
+      gf, (const __nv_bfloat16*)gb, ldg, (const __nv_bfloat16*)yhat, ldy, rstd, n, T, H, tab,
       (__nv_bfloat16*)out, ld_out);
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;

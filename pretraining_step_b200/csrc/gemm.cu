@@ -27,7 +27,8 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // TMA warp, MMA warp, 8 epilogue warps
+constexpr int kEpiThreads = 256;
 
 template <int BN>
 struct Cfg {
@@ -79,118 +80,116 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // ------------------------------------------------------------------ epilogue
-__device__ __forceinline__ void store_row_chunk(const Args& p, int b, int row, int col0,
-                                                const float (&v)[32]) {
+__device__ __forceinline__ bool epi_has_aux(int epi) {
+  return epi == NC_EPI_RESID_F32 || epi == NC_EPI_RELU2_BWD || epi == NC_EPI_AXPBY_BF16;
+}
+
+// The aux operand of one 32-column chunk of one row, as floats (0 past N).
+__device__ __forceinline__ void load_aux(const Args& p, int b, int row, int col0,
+                                         float (&x)[32]) {
   const int nvalid = min(32, p.N - col0);
-  const bool full = (nvalid == 32);
+  if (p.epi == NC_EPI_RESID_F32) {
+    const float* R = (const float*)p.aux + (int64_t)b * p.stride_aux + (int64_t)row * p.ldaux + col0;
+    if (nvalid == 32) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float4 r = reinterpret_cast<const float4*>(R)[j];
+        x[4 * j] = r.x; x[4 * j + 1] = r.y; x[4 * j + 2] = r.z; x[4 * j + 3] = r.w;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) x[j] = j < nvalid ? R[j] : 0.f;
+    }
+  } else {
+    const __nv_bfloat16* X = (const __nv_bfloat16*)p.aux + (int64_t)b * p.stride_aux +
+                             (int64_t)row * p.ldaux + col0;
+    if (nvalid == 32) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 u = reinterpret_cast<const uint4*>(X)[j];
+        float2 f;
+        f = unpack_bf16x2(u.x); x[8 * j + 0] = f.x; x[8 * j + 1] = f.y;
+        f = unpack_bf16x2(u.y); x[8 * j + 2] = f.x; x[8 * j + 3] = f.y;
+        f = unpack_bf16x2(u.z); x[8 * j + 4] = f.x; x[8 * j + 5] = f.y;
+        f = unpack_bf16x2(u.w); x[8 * j + 6] = f.x; x[8 * j + 7] = f.y;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) x[j] = j < nvalid ? bf2f(X[j]) : 0.f;
+    }
+  }
+}
+
+__device__ __forceinline__ void store_bf16_chunk(__nv_bfloat16* D, int nvalid, const float (&w)[32]) {
+  if (nvalid == 32) {
+    uint4* d4 = reinterpret_cast<uint4*>(D);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint4 u;
+      u.x = pack_bf16x2(w[8 * j + 0], w[8 * j + 1]);
+      u.y = pack_bf16x2(w[8 * j + 2], w[8 * j + 3]);
+      u.z = pack_bf16x2(w[8 * j + 4], w[8 * j + 5]);
+      u.w = pack_bf16x2(w[8 * j + 6], w[8 * j + 7]);
+      d4[j] = u;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < nvalid) D[j] = f2bf(w[j]);
+  }
+}
+
+// Apply the epilogue to one 32-column chunk (v = accumulator, x = aux) and store.
+__device__ __forceinline__ void store_row_chunk(const Args& p, int b, int row, int col0,
+                                                const float (&v)[32], const float (&x)[32]) {
+  const int nvalid = min(32, p.N - col0);
+  const int64_t off = (int64_t)b * p.stride_d + (int64_t)row * p.ldd + col0;
+  float w[32];
   switch (p.epi) {
     case NC_EPI_STORE_BF16:
-    case NC_EPI_RELU2: {
-      __nv_bfloat16* D = (__nv_bfloat16*)p.D + (int64_t)b * p.stride_d + (int64_t)row * p.ldd + col0;
-      float w[32];
+    case NC_EPI_RELU2:
+    case NC_EPI_RELU2_BWD:
+    case NC_EPI_AXPBY_BF16: {
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        float x = v[j] * p.alpha;
+        const float a = v[j] * p.alpha;
         if (p.epi == NC_EPI_RELU2) {
-          x = fmaxf(x, 0.f);
-          x = x * x;
+          const float r = fmaxf(a, 0.f);
+          w[j] = r * r;
+        } else if (p.epi == NC_EPI_RELU2_BWD) {
+          w[j] = 2.f * sqrtf(fmaxf(x[j], 0.f)) * a;
+        } else if (p.epi == NC_EPI_AXPBY_BF16) {
+          w[j] = a + p.beta * x[j];
+        } else {
+          w[j] = a;
         }
-        w[j] = x;
       }
-      if (full) {
-        uint4* d4 = reinterpret_cast<uint4*>(D);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint4 u;
-          u.x = pack_bf16x2(w[8 * j + 0], w[8 * j + 1]);
-          u.y = pack_bf16x2(w[8 * j + 2], w[8 * j + 3]);
-          u.z = pack_bf16x2(w[8 * j + 4], w[8 * j + 5]);
-          u.w = pack_bf16x2(w[8 * j + 6], w[8 * j + 7]);
-          d4[j] = u;
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (j < nvalid) D[j] = f2bf(w[j]);
-      }
+      store_bf16_chunk((__nv_bfloat16*)p.D + off, nvalid, w);
       break;
     }
     case NC_EPI_STORE_F32:
     case NC_EPI_RESID_F32: {
-      float* D = (float*)p.D + (int64_t)b * p.stride_d + (int64_t)row * p.ldd + col0;
-      const float* R = p.epi == NC_EPI_RESID_F32
-                           ? (const float*)p.aux + (int64_t)b * p.stride_aux +
-                                 (int64_t)row * p.ldaux + col0
-                           : nullptr;
-      if (full) {
+      float* D = (float*)p.D + off;
+      const bool resid = p.epi == NC_EPI_RESID_F32;
+      if (nvalid == 32) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           float4 o = make_float4(v[4 * j] * p.alpha, v[4 * j + 1] * p.alpha,
                                  v[4 * j + 2] * p.alpha, v[4 * j + 3] * p.alpha);
-          if (R) {
-            const float4 r = reinterpret_cast<const float4*>(R)[j];
-            o.x += r.x;
-            o.y += r.y;
-            o.z += r.z;
-            o.w += r.w;
+          if (resid) {
+            o.x += x[4 * j]; o.y += x[4 * j + 1]; o.z += x[4 * j + 2]; o.w += x[4 * j + 3];
           }
           reinterpret_cast<float4*>(D)[j] = o;
         }
       } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          if (j < nvalid) D[j] = v[j] * p.alpha + (R ? R[j] : 0.f);
-      }
-      break;
-    }
-    case NC_EPI_RELU2_BWD:
-    case NC_EPI_AXPBY_BF16: {
-      __nv_bfloat16* D = (__nv_bfloat16*)p.D + (int64_t)b * p.stride_d + (int64_t)row * p.ldd + col0;
-      const __nv_bfloat16* X = (const __nv_bfloat16*)p.aux + (int64_t)b * p.stride_aux +
-                               (int64_t)row * p.ldaux + col0;
-      float x[32];
-      if (full) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint4 u = reinterpret_cast<const uint4*>(X)[j];
-          float2 f;
-          f = unpack_bf16x2(u.x); x[8 * j + 0] = f.x; x[8 * j + 1] = f.y;
-          f = unpack_bf16x2(u.y); x[8 * j + 2] = f.x; x[8 * j + 3] = f.y;
-          f = unpack_bf16x2(u.z); x[8 * j + 4] = f.x; x[8 * j + 5] = f.y;
-          f = unpack_bf16x2(u.w); x[8 * j + 6] = f.x; x[8 * j + 7] = f.y;
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) x[j] = j < nvalid ? bf2f(X[j]) : 0.f;
-      }
-      float w[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        if (p.epi == NC_EPI_RELU2_BWD)
-          w[j] = 2.f * sqrtf(fmaxf(x[j], 0.f)) * (v[j] * p.alpha);
-        else
-          w[j] = v[j] * p.alpha + p.beta * x[j];
-      }
-      if (full) {
-        uint4* d4 = reinterpret_cast<uint4*>(D);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint4 u;
-          u.x = pack_bf16x2(w[8 * j + 0], w[8 * j + 1]);
-          u.y = pack_bf16x2(w[8 * j + 2], w[8 * j + 3]);
-          u.z = pack_bf16x2(w[8 * j + 4], w[8 * j + 5]);
-          u.w = pack_bf16x2(w[8 * j + 6], w[8 * j + 7]);
-          d4[j] = u;
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (j < nvalid) D[j] = f2bf(w[j]);
+          if (j < nvalid) D[j] = v[j] * p.alpha + (resid ? x[j] : 0.f);
       }
       break;
     }
     case NC_EPI_ACC_F32: {
-      float* D = (float*)p.D + (int64_t)b * p.stride_d + (int64_t)row * p.ldd + col0;
+      float* D = (float*)p.D + off;
 #pragma unroll
       for (int j = 0; j < 32; ++j)
         if (j < nvalid) atomicAdd(D + j, v[j] * p.alpha);
@@ -228,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&tfull[i], 1);
-      tc::mbar_init(&tempty[i], 128);
+      tc::mbar_init(&tempty[i], kEpiThreads);
     }
     tc::mbar_init(drained, 1);
     *abort_flag = 0;
@@ -345,26 +344,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       drain_wait(drained, 0);
     }
   } else {
+    // Two epilogue warps per TMEM lane quarter, each taking half the columns.
     const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;
+    constexpr int CH = BN / 32 / 2;  // 32-column chunks per warp
     const int row_in_tile = q * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       const TileCoord c = decode(p, t);
-      if (!tc::mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status)) break;
+      bool ok = tc::mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
       tc::tc_fence_after();
       const int row = c.mb * BM + row_in_tile;
-#pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch) {
+      const bool aux = epi_has_aux(p.epi);
+      // The aux chunk is loaded one chunk ahead so its HBM latency overlaps
+      // the current chunk's TMEM load, arithmetic and stores.
+      float xa[32], xb[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) xa[j] = xb[j] = 0.f;
+      {
+        const int col0 = c.nb * BN + half * CH * 32;
+        if (aux && row < p.M && col0 < p.N) load_aux(p, c.b, row, col0, xa);
+      }
+#pragma unroll
+      for (int k = 0; k < CH; ++k) {
+        const int ch = half * CH + k;
         uint32_t r[32];
         tc::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + ch * 32, r);
-        tc::tmem_ld_wait();
         const int col0 = c.nb * BN + ch * 32;
+        float(&cur)[32] = (k & 1) ? xb : xa;
+        float(&nxt)[32] = (k & 1) ? xa : xb;
+        if (aux && k + 1 < CH && row < p.M && col0 + 32 < p.N) load_aux(p, c.b, row, col0 + 32, nxt);
+        tc::tmem_ld_wait();
         if (row < p.M && col0 < p.N) {
           float v[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          store_row_chunk(p, c.b, row, col0, v);
+          store_row_chunk(p, c.b, row, col0, v, cur);
         }
       }
       tc::tc_fence_before();
@@ -383,8 +400,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------------ host
 template <int BN>
-nc_status launch_bn(const nc_gemm_desc& d, int split, int* status, cudaStream_t s,
-                    Profiler* prof) {
+nc_status launch_bn(const nc_gemm_desc& d, int split, int* status, const char* tag,
+                    cudaStream_t s, Profiler* prof) {
   using C = Cfg<BN>;
   static bool attr_set = false;
   if (!attr_set) {
@@ -425,7 +442,7 @@ nc_status launch_bn(const nc_gemm_desc& d, int split, int* status, cudaStream_t 
   if (total >= (1ll << 31)) return fail(NC_ERR_INVALID_ARG, "gemm: too many tiles");
   const int grid = (int)std::min<int64_t>(total, num_sms());
   const double flops = 2.0 * d.M * (double)d.N * d.K * d.batch;
-  Probe probe(prof, s, "gemm_tc", flops, 0.0);
+  Probe probe(prof, s, tag, flops, 0.0);
   gemm_tc_kernel<BN><<<grid, kThreads, C::SMEM_BYTES, s>>>(ta, tb, a);
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
@@ -483,8 +500,8 @@ nc_status gemm_launch(const GemmLaunch& g, cudaStream_t s, Profiler* prof) {
     split = auto_split(tiles, num_kb);
   }
   if (split > num_kb) split = num_kb;
-  return bn256 ? launch_bn<256>(d, split, g.status, s, prof)
-               : launch_bn<128>(d, split, g.status, s, prof);
+  return bn256 ? launch_bn<256>(d, split, g.status, g.tag, s, prof)
+               : launch_bn<128>(d, split, g.status, g.tag, s, prof);
 }
 
 }  // namespace nc

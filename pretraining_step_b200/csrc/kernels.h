@@ -18,7 +18,8 @@ bool make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_
 
 struct GemmLaunch {
   nc_gemm_desc d;
-  int* status;  // device status word (may be null)
+  int* status;             // device status word (may be null)
+  const char* tag = "gemm_tc";  // profiler class
 };
 // d.split_k == 0 selects the split automatically (NC_EPI_ACC_F32 only).
 nc_status gemm_launch(const GemmLaunch& g, cudaStream_t s, Profiler* prof);

@@ -34,6 +34,7 @@ nc_status newton_schulz_wide(void* x0, int count, int m, int n, int steps, void*
   for (int it = 0; it < steps; ++it) {
     GemmLaunch g{};
     g.status = status;
+    g.tag = "gemm_ns";
     // A = X X^T
     g.d = nc_gemm_desc{};
     g.d.M = m; g.d.N = m; g.d.K = n; g.d.batch = count;

@@ -258,9 +258,11 @@ bool is_device_ptr(const void* ptr) {
 
 // y[M,N] = epi(x[M,K] W[N,K]^T): the forward projection.
 nc_status proj(nc_params* p, const bf16* x, int64_t M, int64_t K, const bf16* W, int64_t Nout,
-               void* D, int64_t ldd, nc_epilogue epi, const void* aux, int64_t ldaux) {
+               void* D, int64_t ldd, nc_epilogue epi, const void* aux, int64_t ldaux,
+               const char* tag = "gemm_fwd") {
   GemmLaunch g{};
   g.status = p->status;
+  g.tag = tag;
   g.d.M = (int)M; g.d.N = (int)Nout; g.d.K = (int)K; g.d.batch = 1;
   g.d.A = x; g.d.lda = K; g.d.a_kmajor = 1;
   g.d.B = W; g.d.ldb = K; g.d.b_kmajor = 1;
@@ -272,9 +274,11 @@ nc_status proj(nc_params* p, const bf16* x, int64_t M, int64_t K, const bf16* W,
 
 // dx[M,N] = epi(dy[M,K] W[K,N]): the input gradient of a projection.
 nc_status proj_dx(nc_params* p, const bf16* dy, int64_t M, int64_t K, const bf16* W, int64_t Nout,
-                  void* D, int64_t ldd, nc_epilogue epi, const void* aux, int64_t ldaux) {
+                  void* D, int64_t ldd, nc_epilogue epi, const void* aux, int64_t ldaux,
+                  const char* tag = "gemm_dgrad") {
   GemmLaunch g{};
   g.status = p->status;
+  g.tag = tag;
   g.d.M = (int)M; g.d.N = (int)Nout; g.d.K = (int)K; g.d.batch = 1;
   g.d.A = dy; g.d.lda = K; g.d.a_kmajor = 1;
   g.d.B = W; g.d.ldb = Nout; g.d.b_kmajor = 0;
@@ -286,9 +290,11 @@ nc_status proj_dx(nc_params* p, const bf16* dy, int64_t M, int64_t K, const bf16
 
 // dW[Mo,No] = dy[Ntok,Mo]^T x[Ntok,No] into a zeroed fp32 gradient.
 nc_status proj_dw(nc_params* p, const bf16* dy, int64_t ldy, int64_t Mo, const bf16* x,
-                  int64_t ldx, int64_t No, int64_t Ntok, float* dW) {
+                  int64_t ldx, int64_t No, int64_t Ntok, float* dW,
+                  const char* tag = "gemm_wgrad") {
   GemmLaunch g{};
   g.status = p->status;
+  g.tag = tag;
   g.d.M = (int)Mo; g.d.N = (int)No; g.d.K = (int)Ntok; g.d.batch = 1;
   g.d.A = dy; g.d.lda = ldy; g.d.a_kmajor = 0;
   g.d.B = x; g.d.ldb = ldx; g.d.b_kmajor = 0;
@@ -337,13 +343,15 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
     NC_TRY(proj(p, a.a[l], N, F, W + 8 * d2, d, a.x[l + 1], d, NC_EPI_RESID_F32, a.xmid[l], d));
   }
   NC_TRY(rmsnorm_fwd(a.x[L], N, (int)d, a.hf, a.rf, s, pr));
-  NC_TRY(proj(p, a.hf, N, d, p->lm_b, V, a.logits, V, NC_EPI_STORE_BF16, nullptr, 0));
+  NC_TRY(proj(p, a.hf, N, d, p->lm_b, V, a.logits, V, NC_EPI_STORE_BF16, nullptr, 0,
+              "gemm_lmhead"));
   NC_TRY(ce_fwd_bwd(a.logits, tgt, N, V, a.loss_rows, loss_dev ? loss_dev : a.loss, p->status, s,
                     pr));
 
   // ---------------- backward (a.logits now holds dz)
-  NC_TRY(proj_dw(p, a.logits, V, V, a.hf, d, d, N, g->lm));
-  NC_TRY(proj_dx(p, a.logits, N, V, p->lm_b, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0));
+  NC_TRY(proj_dw(p, a.logits, V, V, a.hf, d, d, N, g->lm, "gemm_lmhead"));
+  NC_TRY(proj_dx(p, a.logits, N, V, p->lm_b, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0,
+                 "gemm_lmhead"));
   float* dx = a.dx0;
   float* dxn = a.dx1;
   NC_TRY(rmsnorm_bwd(a.dh, a.x[L], a.rf, nullptr, N, (int)d, dx, a.dxb, s, pr));

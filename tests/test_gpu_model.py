@@ -189,7 +189,9 @@ def test_profiler_counts_launches():
     m.profile(True)
     m.fwd_bwd(tok, tgt)
     stats = m.profile_read()
-    assert stats["gemm_tc"]["launches"] == 12 * depth + 3  # 4 fwd + 8 bwd per layer, 3 for lm_head
+    n_gemm = sum(v["launches"] for k, v in stats.items() if k.startswith("gemm_"))
+    assert n_gemm == 12 * depth + 3  # 4 fwd + 8 bwd per layer, 3 for lm_head
+    assert stats["gemm_wgrad"]["launches"] == 4 * depth  # wqkv, wo, wup, wdown per layer
     assert stats["attn_fwd"]["launches"] == depth
     assert all(v["ms"] > 0 for v in stats.values())
     m.close()
