@@ -542,33 +542,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = tc::mbar_wait(sdp_full, t & 1, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc::tc_fence_after();
-      uint32_t sv[64], dp[64];
-      tc::tmem_ld_32x32b_x32(lane_base + TB_S, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-      tc::tmem_ld_32x32b_x32(lane_base + TB_S + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-      tc::tmem_ld_32x32b_x32(lane_base + TB_DP, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
-      tc::tmem_ld_32x32b_x32(lane_base + TB_DP + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
-      tc::tmem_ld_wait();
-      tc::tc_fence_before();
-      tc::mbar_arrive(sdp_empty);
       // The query tile's lse/D, staged by the TMA warp and published by the
       // stage's qd_full barrier (already complete: the scores came from it).
       ok = tc::mbar_wait(&qd_full[t & 1], (t >> 1) & 1, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      // S^T and dP^T rows in four 16-column chunks, read before the buffers
+      // are handed back; P^T / dS^T packed to bf16.
       uint32_t pp[32], pd[32];
-      const bool edge = (q0 < key + 1) || (q0 + BQB > a.T) || (key >= a.T);
+      {
+        uint32_t sv[64], dp[64];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const int qa = q0 + 2 * c, qb2 = qa + 1;
-        float p0 = ex2(__uint_as_float(sv[2 * c]) * a.sl2 - ld[2 * c]);
-        float p1 = ex2(__uint_as_float(sv[2 * c + 1]) * a.sl2 - ld[2 * c + 1]);
-        if (edge) {
-          if (qa < key || qa >= a.T || key >= a.T) p0 = 0.f;
-          if (qb2 < key || qb2 >= a.T || key >= a.T) p1 = 0.f;
+        for (int c = 0; c < 4; ++c) {
+          tc::tmem_ld_32x32b_x16(lane_base + TB_S + 16 * c, *reinterpret_cast<uint32_t(*)[16]>(&sv[16 * c]));
+          tc::tmem_ld_32x32b_x16(lane_base + TB_DP + 16 * c, *reinterpret_cast<uint32_t(*)[16]>(&dp[16 * c]));
         }
-        const float d0 = p0 * (__uint_as_float(dp[2 * c]) - ld[BQB + 2 * c]);
-        const float d1 = p1 * (__uint_as_float(dp[2 * c + 1]) - ld[BQB + 2 * c + 1]);
-        pp[c] = pack_bf16x2(p0, p1);
-        pd[c] = pack_bf16x2(d0, d1);
+        tc::tmem_ld_wait();
+        tc::tc_fence_before();
+        tc::mbar_arrive(sdp_empty);
+        const bool edge = (q0 < key + 1) || (q0 + BQB > a.T) || (key >= a.T);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          float p0 = ex2(__uint_as_float(sv[2 * c]) * a.sl2 - ld[2 * c]);
+          float p1 = ex2(__uint_as_float(sv[2 * c + 1]) * a.sl2 - ld[2 * c + 1]);
+          if (edge) {
+            const int qa = q0 + 2 * c, qb2 = qa + 1;
+            if (qa < key || qa >= a.T || key >= a.T) p0 = 0.f;
+            if (qb2 < key || qb2 >= a.T || key >= a.T) p1 = 0.f;
+          }
+          const float d0 = p0 * (__uint_as_float(dp[2 * c]) - ld[BQB + 2 * c]);
+          const float d1 = p1 * (__uint_as_float(dp[2 * c + 1]) - ld[BQB + 2 * c + 1]);
+          pp[c] = pack_bf16x2(p0, p1);
+          pd[c] = pack_bf16x2(d0, d1);
+        }
       }
       ok = tc::mbar_wait(pds_empty, (t & 1) ^ 1, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
@@ -624,16 +629,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       bool ok = tc::mbar_wait(dq_full, t & 1, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc::tc_fence_after();
-      uint32_t v[64];
-      tc::tmem_ld_32x32b_x32(lane_base + TB_DQ, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-      tc::tmem_ld_32x32b_x32(lane_base + TB_DQ + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-      tc::tmem_ld_wait();
-      tc::tc_fence_before();
-      tc::mbar_arrive(dq_empty);
       float* dst = dq_bh + (int64_t)q0 * dq_row;
+      const int nq = min(BQB, a.T - q0);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BQB; c0 += 16) {
+        uint32_t v[16];
+        tc::tmem_ld_32x32b_x16(lane_base + TB_DQ + c0, v);
+        tc::tmem_ld_wait();
+        if (c0 + 16 == BQB) {  // the whole tile has been read: TMEM may be reused
+          tc::tc_fence_before();
+          tc::mbar_arrive(dq_empty);
+        }
+        float vv[16];
 #pragma unroll
-      for (int c = 0; c < BQB; ++c)
-        if (q0 + c < a.T) atomicAdd(dst + (int64_t)c * dq_row, __uint_as_float(v[c]) * a.scale);
+        for (int j = 0; j < 16; ++j) vv[j] = __uint_as_float(v[j]) * a.scale;
+        if (c0 + 16 <= nq) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) atomicAdd(dst + (int64_t)(c0 + j) * dq_row, vv[j]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < nq) atomicAdd(dst + (int64_t)(c0 + j) * dq_row, vv[j]);
+        }
+      }
     }
   }
   tc::tc_fence_before();

@@ -398,6 +398,223 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ CTA-pair kernel
+// Same roles, but a cluster of two CTAs computes one 256 x 256 tile with
+// tcgen05.mma.cta_group::2: each CTA stages its 128 rows of A and its 128
+// rows of B (32 KB per 64-wide K slice instead of 48 KB for 128 x 256 on one
+// CTA), the even CTA's MMA thread issues M = 256 MMAs over both CTAs' shared
+// memory, and each CTA's TMEM receives its own 128 rows of the accumulator,
+// drained by its own epilogue warps.  Both CTAs' copies complete on the
+// leader's full barrier; commits arrive on both CTAs' barriers; epilogue
+// warps release an accumulator with a remote arrive on the leader.
+struct Cfg2 {
+  static constexpr int BN = 256;
+  static constexpr int A_BYTES = BM * BK * 2;         // this CTA's 128 rows of A
+  static constexpr int B_BYTES = (BN / 2) * BK * 2;   // this CTA's 128 rows of B
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = 6;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const Args p) {
+  using C = Cfg2;
+  constexpr int BN = C::BN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* tfull = empty + C::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drained = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = tc::cluster_ctarank();
+  const bool leader = (rank == 0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&tfull[i], 1);
+      tc::mbar_init(&tempty[i], 2 * (kEpiThreads / 32));  // one arrive per epilogue warp of the pair
+    }
+    tc::mbar_init(drained, 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc2(tmem_slot, C::TMEM_COLS);
+    tc::tmem_relinquish2();
+  }
+  tc::tc_fence_before();
+  tc::cluster_sync();  // both CTAs' barriers exist before any cross-CTA traffic
+  tc::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int total = p.tiles_m * p.tiles_n * p.split_k * p.batch;  // tiles_m counts 256-row tiles
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tc::tma_prefetch_desc(&tmA);
+      tc::tma_prefetch_desc(&tmB);
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int t = pair; t < total && ok; t += npairs) {
+        const TileCoord c = decode(p, t);
+        const int m0 = c.mb * 2 * BM + (int)rank * BM;
+        const int n0 = c.nb * BN + (int)rank * (BN / 2);
+        for (int kb = c.kb0; kb < c.kb1; ++kb) {
+          if (!tc::mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          if (leader) tc::mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+          uint8_t* a_dst = smem + stage * C::STAGE_BYTES;
+          uint8_t* b_dst = a_dst + C::A_BYTES;
+          const int k0 = kb * BK;
+          if (!p.a_mn) {
+            tc::tma_load_3d_pair(a_dst, &tmA, &full[stage], k0, m0, c.b);
+          } else {
+            tc::tma_load_3d_pair(a_dst, &tmA, &full[stage], m0, k0, c.b);
+            tc::tma_load_3d_pair(a_dst + 8192, &tmA, &full[stage], m0 + 64, k0, c.b);
+          }
+          if (!p.b_mn) {
+            tc::tma_load_3d_pair(b_dst, &tmB, &full[stage], k0, n0, c.b);
+          } else {
+            tc::tma_load_3d_pair(b_dst, &tmB, &full[stage], n0, k0, c.b);
+            tc::tma_load_3d_pair(b_dst + 8192, &tmB, &full[stage], n0 + 64, k0, c.b);
+          }
+          ++issued;
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // Copies land on the leader's barriers; let this CTA's stages settle.
+        for (int i = 0; i < min(issued, C::STAGES); ++i) {
+          if (--stage < 0) {
+            stage = C::STAGES - 1;
+            phase ^= 1;
+          }
+          drain_wait(&empty[stage], phase);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      const uint32_t idesc = tc::idesc_bf16_f32(2 * BM, BN, p.a_mn, p.b_mn);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = pair; t < total && ok; t += npairs) {
+        const TileCoord c = decode(p, t);
+        if (!tc::mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = c.kb0; kb < c.kb1; ++kb) {
+          if (!tc::mbar_wait(&full[stage], phase, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc::tc_fence_after();
+          const uint32_t a_base = tc::smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t b_base = a_base + C::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = p.a_mn ? tc::smem_desc_sw128(a_base + kk * 2048, 8192, 1024)
+                                       : tc::smem_desc_sw128(a_base + kk * 32, 16, 1024);
+            const uint64_t bd = p.b_mn ? tc::smem_desc_sw128(b_base + kk * 2048, 8192, 1024)
+                                       : tc::smem_desc_sw128(b_base + kk * 32, 16, 1024);
+            tc::umma_bf16_ss_pair(d_tmem, ad, bd, idesc, (kb > c.kb0 || kk > 0) ? 1u : 0u);
+          }
+          tc::umma_commit_pair(&empty[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        tc::umma_commit_pair(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+      tc::umma_commit_pair(drained);
+      drain_wait(drained, 0);
+    }
+  } else {
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    constexpr int CH = BN / 32 / 2;
+    const int row_in_tile = q * 32 + lane;
+    const uint32_t tempty_leader = tc::mapa_shared(tc::smem_u32(tempty), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = pair; t < total; t += npairs) {
+      const TileCoord c = decode(p, t);
+      bool ok = tc::mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc::tc_fence_after();
+      const int row = c.mb * 2 * BM + (int)rank * BM + row_in_tile;
+      const bool aux = epi_has_aux(p.epi);
+      float xa[32], xb[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) xa[j] = xb[j] = 0.f;
+      {
+        const int col0 = c.nb * BN + half * CH * 32;
+        if (aux && row < p.M && col0 < p.N) load_aux(p, c.b, row, col0, xa);
+      }
+#pragma unroll
+      for (int k = 0; k < CH; ++k) {
+        const int ch = half * CH + k;
+        uint32_t r[32];
+        tc::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + ch * 32, r);
+        const int col0 = c.nb * BN + ch * 32;
+        float(&cur)[32] = (k & 1) ? xb : xa;
+        float(&nxt)[32] = (k & 1) ? xa : xb;
+        if (aux && k + 1 < CH && row < p.M && col0 + 32 < p.N) load_aux(p, c.b, row, col0 + 32, nxt);
+        tc::tmem_ld_wait();
+        if (row < p.M && col0 < p.N) {
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          store_row_chunk(p, c.b, row, col0, v, cur);
+        }
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive_cluster(tempty_leader + acc * 8);
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::cluster_sync();  // no CTA leaves while its peer may still signal it
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc2(tmem_base, C::TMEM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------ host
 template <int BN>
 nc_status launch_bn(const nc_gemm_desc& d, int split, int* status, const char* tag,
@@ -445,6 +662,64 @@ nc_status launch_bn(const nc_gemm_desc& d, int split, int* status, const char* t
   Probe probe(prof, s, tag, flops, 0.0);
   gemm_tc_kernel<BN><<<grid, kThreads, C::SMEM_BYTES, s>>>(ta, tb, a);
   NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+nc_status launch_pair(const nc_gemm_desc& d, int split, int* status, const char* tag,
+                      cudaStream_t s, Profiler* prof) {
+  using C = Cfg2;
+  static bool attr_set = false;
+  if (!attr_set) {
+    NC_CUDA_TRY(cudaFuncSetAttribute(gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     C::SMEM_BYTES));
+    attr_set = true;
+  }
+  CUtensorMap ta, tb;
+  const bool ok_a = d.a_kmajor ? make_tmap_bf16_3d(&ta, d.A, d.K, d.M, d.batch, d.lda, d.stride_a, BM)
+                               : make_tmap_bf16_3d(&ta, d.A, d.M, d.K, d.batch, d.lda, d.stride_a, 64);
+  const bool ok_b = d.b_kmajor ? make_tmap_bf16_3d(&tb, d.B, d.K, d.N, d.batch, d.ldb, d.stride_b, C::BN / 2)
+                               : make_tmap_bf16_3d(&tb, d.B, d.N, d.K, d.batch, d.ldb, d.stride_b, 64);
+  if (!ok_a || !ok_b) return fail(NC_ERR_INVALID_ARG, "gemm: cuTensorMapEncodeTiled rejected an operand");
+  Args a;
+  a.M = d.M;
+  a.N = d.N;
+  a.K = d.K;
+  a.batch = d.batch;
+  a.tiles_m = (d.M + 2 * BM - 1) / (2 * BM);
+  a.tiles_n = (d.N + C::BN - 1) / C::BN;
+  a.num_kb = (d.K + BK - 1) / BK;
+  a.kb_per_split = (a.num_kb + split - 1) / split;
+  a.split_k = (a.num_kb + a.kb_per_split - 1) / a.kb_per_split;
+  a.a_mn = d.a_kmajor ? 0 : 1;
+  a.b_mn = d.b_kmajor ? 0 : 1;
+  a.epi = d.epi;
+  a.alpha = d.alpha;
+  a.beta = d.beta;
+  a.D = d.D;
+  a.ldd = d.ldd;
+  a.stride_d = d.stride_d;
+  a.aux = d.aux;
+  a.ldaux = d.ldaux;
+  a.stride_aux = d.stride_aux;
+  a.status = status;
+  const int64_t total = (int64_t)a.tiles_m * a.tiles_n * a.split_k * a.batch;
+  if (total >= (1ll << 31)) return fail(NC_ERR_INVALID_ARG, "gemm: too many tiles");
+  const int pairs = (int)std::min<int64_t>(total, num_sms() / 2);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const double flops = 2.0 * d.M * (double)d.N * d.K * d.batch;
+  Probe probe(prof, s, tag, flops, 0.0);
+  NC_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_tc2_kernel, ta, tb, a));
   return NC_OK;
 }
 
@@ -500,6 +775,15 @@ nc_status gemm_launch(const GemmLaunch& g, cudaStream_t s, Profiler* prof) {
     split = auto_split(tiles, num_kb);
   }
   if (split > num_kb) split = num_kb;
+  // 256 x 256 tiles on a CTA pair whenever M spans more than one 128-row
+  // tile and 256-wide column tiles fit N; 128 x BN on one CTA otherwise.
+  if (bn256 && d.M > BM) {
+    if (d.split_k <= 0) {
+      const int64_t tiles = (int64_t)((d.M + 2 * BM - 1) / (2 * BM)) * ((d.N + 255) / 256) * d.batch;
+      split = std::min(auto_split(tiles * 2, num_kb), num_kb);
+    }
+    return launch_pair(d, split, g.status, g.tag, s, prof);
+  }
   return bn256 ? launch_bn<256>(d, split, g.status, g.tag, s, prof)
                : launch_bn<128>(d, split, g.status, g.tag, s, prof);
 }

@@ -21,7 +21,9 @@ pytestmark = pytest.mark.gpu
 # ------------------------------------------------------------------ GEMM
 @pytest.mark.parametrize("a_k,b_k", [(1, 1), (1, 0), (0, 1), (0, 0)])
 @pytest.mark.parametrize("M,N,K", [(128, 256, 64), (200, 296, 136), (256, 128, 512),
-                                   (384, 384, 200), (64, 1280, 1280)])
+                                   (384, 384, 200), (64, 1280, 1280),
+                                   # CTA-pair tiles (256 x 256): ragged M, ragged K
+                                   (520, 512, 200), (296, 768, 136), (1024, 1280, 64)])
 def test_gemm_layouts(a_k, b_k, M, N, K):
     t = torch()
     A = inputs.bf16_normal(1, (M, K))
