@@ -157,8 +157,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (lane == 0) {
       const uint32_t id_s = tc::idesc_bf16_f32(128, FKV, 0, 0);
       const uint32_t id_pv = tc::idesc_bf16_f32(128, 128, 0, 1);
-      const uint32_t q_addr = tc::smem_u32(smem + OFF_Q);
-      const uint32_t p_addr = tc::smem_u32(smem + OFF_P);
+      // Descriptors are built once; each MMA adds a constant byte offset.
+      const uint64_t qdesc0 = tc::smem_desc_sw128(tc::smem_u32(smem + OFF_Q), 16, 1024);
+      const uint64_t kdesc0 = tc::smem_desc_sw128(tc::smem_u32(smem + OFF_K), 16, 1024);
+      const uint64_t vdesc0 = tc::smem_desc_sw128(tc::smem_u32(smem + OFF_V), KT / 2, 1024);
+      const uint64_t pdesc0 = tc::smem_desc_sw128(tc::smem_u32(smem + OFF_P), 16, 1024);
       bool ok = tc::mbar_wait(q_full, 0, abort_flag, a.status);
       for (int j = 0; j <= n && ok; ++j) {
         if (j < n) {
@@ -170,14 +173,13 @@ __global__ void __launch_bounds__(kThreads, 2)
             break;
           }
           tc::tc_fence_after();
-          const uint32_t k_addr = tc::smem_u32(smem + OFF_K + s * KT);
+          const uint64_t kd = kdesc0 + (uint64_t)((s * KT) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint32_t qo = (kk >> 2) * (TILE / 2) + (kk & 3) * 32;
-            const uint32_t ko = (kk >> 2) * (KT / 2) + (kk & 3) * 32;
-            tc::umma_bf16_ss(tmem + TM_S0 + s * FKV, tc::smem_desc_sw128(q_addr + qo, 16, 1024),
-                             tc::smem_desc_sw128(k_addr + ko, 16, 1024), id_s, kk > 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < HD / 16; ++kk)
+            tc::umma_bf16_ss(tmem + TM_S0 + s * FKV,
+                             tc::desc_add(qdesc0, (kk >> 2) * (TILE / 2) + (kk & 3) * 32),
+                             tc::desc_add(kd, (kk >> 2) * (KT / 2) + (kk & 3) * 32), id_s,
+                             kk > 0 ? 1u : 0u);
           tc::umma_commit(&s_full[s]);
           tc::umma_commit(&k_empty[s]);
         }
@@ -191,12 +193,11 @@ __global__ void __launch_bounds__(kThreads, 2)
             break;
           }
           tc::tc_fence_after();
-          const uint32_t v_addr = tc::smem_u32(smem + OFF_V + s * KT);
+          const uint64_t vd = vdesc0 + (uint64_t)((s * KT) >> 4);
 #pragma unroll
           for (int kk = 0; kk < FKV / 16; ++kk)
-            tc::umma_bf16_ss(tmem + TM_O, tc::smem_desc_sw128(p_addr + kk * 32, 16, 1024),
-                             tc::smem_desc_sw128(v_addr + kk * 2048, KT / 2, 1024), id_pv,
-                             (jj > 0 || kk > 0) ? 1u : 0u);
+            tc::umma_bf16_ss(tmem + TM_O, tc::desc_add(pdesc0, kk * 32), tc::desc_add(vd, kk * 2048),
+                             id_pv, (jj > 0 || kk > 0) ? 1u : 0u);
           tc::umma_commit(pv_done);
           tc::umma_commit(&v_empty[s]);
         }
@@ -323,33 +324,41 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 // ------------------------------------------------------------------ backward
 // One CTA per (128-key tile, head, batch row); loops over the 64-query tiles
-// at or after it.  320 threads:
-//   warp 0      TMA: K and V once, then Q_i and dO_i through a 2-stage ring;
+// at or after it.  448 threads:
+//   warp 0      TMA: K and V once, then Q_i and dO_i through a 4-stage ring
+//               (tile i's Q/dO stay operands of dV/dK(i) while tile i+1's
+//               scores are computed, so two stages would leave no prefetch);
+//               its lanes also stage lse * log2(e) and D of each tile;
 //   warp 1      MMA issue, per query tile i:
 //                 S^T  = K Q_i^T        TMEM [  0, 64)   M 128 keys, N 64
 //                 dP^T = V dO_i^T       TMEM [ 64,128)
 //                 dV  += P^T dO_i       TMEM [256,384)   N 128 (dO MN-major)
 //                 dK  += dS^T Q_i       TMEM [384,512)   N 128 (Q MN-major)
-//                 dQ^T = K^T dS^T       TMEM [128,192)   M 128 dims, N 64
-//               (K^T and dS^T are the same shared tiles read MN-major);
-//   warps 2..5  one key row each: P^T = exp(S^T/sqrt(d) - lse),
-//               dS^T = P^T (dP^T - D), both as bf16 into K-major shared
-//               tiles; at the end dK, dV rows to global memory;
-//   warps 6..9  one head-dim row each: dQ^T row -> fp32 atomic adds into dq
+//                 dQ^T = K^T dS^T       TMEM [128,256)   M 128 dims, N 64, 2 buffers
+//               (K^T and dS^T are the same shared tiles read MN-major), with
+//               S^T/dP^T of tile i+1 issued before the gradient products of i;
+//   warps 2..9  two warps per key row group, each half of the 64 columns:
+//               P^T = exp(S^T/sqrt(d) - lse), dS^T = P^T (dP^T - D) as bf16
+//               into K-major shared tiles; at the end dV (warps 2..5) and dK
+//               (warps 6..9) rows to global memory;
+//   warps 10..13 one head-dim row each: dQ^T row -> fp32 atomic adds into dq
 //               (a warp covers 32 consecutive dims of one query: coalesced).
 constexpr int BQB = 64;                  // query tile of the backward
 constexpr int QT = BQB * 128 * 2;        // 16 KB: [64 rows x 128 dims]
 constexpr int PT = 128 * BQB * 2;        // 16 KB: [128 keys x 64 queries]
+constexpr int QST = 4;                   // Q / dO stages
 constexpr int B_OFF_K = 0;
 constexpr int B_OFF_V = B_OFF_K + TILE;
-constexpr int B_OFF_Q = B_OFF_V + TILE;       // 2 stages
-constexpr int B_OFF_DO = B_OFF_Q + 2 * QT;    // 2 stages
-constexpr int B_OFF_P = B_OFF_DO + 2 * QT;
+constexpr int B_OFF_Q = B_OFF_V + TILE;         // QST stages
+constexpr int B_OFF_DO = B_OFF_Q + QST * QT;    // QST stages
+constexpr int B_OFF_P = B_OFF_DO + QST * QT;
 constexpr int B_OFF_DS = B_OFF_P + PT;
-constexpr int B_OFF_LD = B_OFF_DS + PT;  // per stage: lse * log2(e) [64], D [64] (f32)
-constexpr int B_OFF_BAR = B_OFF_LD + 2 * 2 * BQB * 4;
-constexpr int kBwdSmem = B_OFF_BAR + 256 + 1024;
-constexpr int kBwdThreads = 320;
+constexpr int B_OFF_LD = B_OFF_DS + PT;         // per stage: lse * log2(e) [64], D [64] (f32)
+constexpr int B_OFF_BAR = B_OFF_LD + QST * 2 * BQB * 4;
+constexpr int kBwdNeeded = B_OFF_BAR + 256;
+constexpr int kBwdSmem = 232448;                // the per-block maximum; slack absorbs alignment
+static_assert(kBwdNeeded + 512 <= kBwdSmem, "attention backward shared memory budget");
+constexpr int kBwdThreads = 448;
 constexpr uint32_t TB_S = 0, TB_DP = 64, TB_DQ = 128, TB_DV = 256, TB_DK = 384;
 
 struct BwdArgs {
@@ -371,19 +380,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  if ((smem - smem_raw) + kBwdNeeded > kBwdSmem) {  // never expected: base misaligned past slack
+    if (threadIdx.x == 0 && a.status) atomicExch(a.status, kDevTimeout);
+    return;
+  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + B_OFF_BAR);
   uint64_t* kv_full = bars + 0;
-  uint64_t* qd_full = bars + 1;    // [2]
-  uint64_t* qd_empty = bars + 3;   // [2]
-  uint64_t* sdp_full = bars + 5;
-  uint64_t* sdp_empty = bars + 6;
-  uint64_t* pds_full = bars + 7;
-  uint64_t* pds_empty = bars + 8;
-  uint64_t* dq_full = bars + 9;
-  uint64_t* dq_empty = bars + 10;
-  uint64_t* dkv_full = bars + 11;
-  uint64_t* drained = bars + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* qd_full = bars + 1;              // [QST]
+  uint64_t* qd_empty = bars + 1 + QST;       // [QST]
+  uint64_t* sdp_full = bars + 1 + 2 * QST;
+  uint64_t* sdp_empty = sdp_full + 1;
+  uint64_t* pds_full = sdp_full + 2;
+  uint64_t* pds_empty = sdp_full + 3;
+  uint64_t* dq_full = sdp_full + 4;          // [2]
+  uint64_t* dq_empty = sdp_full + 6;         // [2]
+  uint64_t* dkv_full = sdp_full + 8;
+  uint64_t* drained = sdp_full + 9;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sdp_full + 10);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -394,16 +407,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (threadIdx.x == 0) {
     tc::mbar_init(kv_full, 1);
-    for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&qd_full[i], 32);  // the TMA lane (with its bytes) + 32 lse/D loader lanes
+    for (int i = 0; i < QST; ++i) {
+      tc::mbar_init(&qd_full[i], 32);  // the TMA lane (with its bytes) + 31 lse/D loader lanes
       tc::mbar_init(&qd_empty[i], 1);
     }
     tc::mbar_init(sdp_full, 1);
-    tc::mbar_init(sdp_empty, 128);
-    tc::mbar_init(pds_full, 128);
+    tc::mbar_init(sdp_empty, 256);
+    tc::mbar_init(pds_full, 256);
     tc::mbar_init(pds_empty, 1);
-    tc::mbar_init(dq_full, 1);
-    tc::mbar_init(dq_empty, 128);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&dq_full[i], 1);
+      tc::mbar_init(&dq_empty[i], 128);
+    }
     tc::mbar_init(dkv_full, 1);
     tc::mbar_init(drained, 1);
     *abort_flag = 0;
@@ -437,8 +452,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     int issued = 0;
     bool ok = true;
     for (int t = 0; t < nblk; ++t) {
-      const int st = t & 1;
-      const uint32_t ph = (t >> 1) & 1;
+      const int st = t % QST;
+      const uint32_t ph = (t / QST) & 1;
       bool w = true;
       if (lane == 0) w = tc::mbar_wait(&qd_empty[st], ph ^ 1, abort_flag, a.status);
       if (!__shfl_sync(0xffffffffu, (int)w, 0)) { ok = false; break; }
@@ -464,72 +479,80 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     if (!ok && lane == 0) {
       drain_wait(kv_full, 0);
-      for (int t = max(0, issued - 2); t < issued; ++t) drain_wait(&qd_full[t & 1], (t >> 1) & 1);
+      for (int t = max(0, issued - QST); t < issued; ++t) drain_wait(&qd_full[t % QST], (t / QST) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t id_sdp = tc::idesc_bf16_f32(128, BQB, 0, 0);
       const uint32_t id_acc = tc::idesc_bf16_f32(128, 128, 0, 1);
       const uint32_t id_dq = tc::idesc_bf16_f32(128, BQB, 1, 1);
-      const uint32_t k_addr = tc::smem_u32(smem + B_OFF_K);
-      const uint32_t v_addr = tc::smem_u32(smem + B_OFF_V);
-      const uint32_t p_addr = tc::smem_u32(smem + B_OFF_P);
-      const uint32_t ds_addr = tc::smem_u32(smem + B_OFF_DS);
+      // Descriptors are built once; each MMA adds a constant byte offset.
+      const uint64_t kK = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_K), 16, 1024);
+      const uint64_t vK = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_V), 16, 1024);
+      const uint64_t kMN = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_K), TILE / 2, 1024);
+      const uint64_t qK = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_Q), 16, 1024);
+      const uint64_t doK = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_DO), 16, 1024);
+      const uint64_t qMN = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_Q), QT / 2, 1024);
+      const uint64_t doMN = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_DO), QT / 2, 1024);
+      const uint64_t pK = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_P), 16, 1024);
+      const uint64_t dsK = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_DS), 16, 1024);
+      const uint64_t dsMN = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_DS), PT, 1024);
       bool ok = tc::mbar_wait(kv_full, 0, abort_flag, a.status);
       // S^T and dP^T of query tile t into TMEM once the tile has landed and the
       // softmax warps have read the previous scores.
       auto issue_sdp = [&](int t) -> bool {
-        const int st = t & 1;
-        if (!tc::mbar_wait(&qd_full[st], (t >> 1) & 1, abort_flag, a.status)) return false;
+        const int st = t % QST;
+        if (!tc::mbar_wait(&qd_full[st], (t / QST) & 1, abort_flag, a.status)) return false;
         if (t > 0 && !tc::mbar_wait(sdp_empty, (t - 1) & 1, abort_flag, a.status)) return false;
         tc::tc_fence_after();
-        const uint32_t q_addr = tc::smem_u32(smem + B_OFF_Q + st * QT);
-        const uint32_t do_addr = tc::smem_u32(smem + B_OFF_DO + st * QT);
+        const uint64_t qd = qK + (uint64_t)((st * QT) >> 4);
+        const uint64_t dod = doK + (uint64_t)((st * QT) >> 4);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t ao = (kk >> 2) * (TILE / 2) + (kk & 3) * 32;
           const uint32_t bo = (kk >> 2) * (QT / 2) + (kk & 3) * 32;
-          tc::umma_bf16_ss(tmem + TB_S, tc::smem_desc_sw128(k_addr + ao, 16, 1024),
-                           tc::smem_desc_sw128(q_addr + bo, 16, 1024), id_sdp, kk > 0 ? 1u : 0u);
-          tc::umma_bf16_ss(tmem + TB_DP, tc::smem_desc_sw128(v_addr + ao, 16, 1024),
-                           tc::smem_desc_sw128(do_addr + bo, 16, 1024), id_sdp, kk > 0 ? 1u : 0u);
+          tc::umma_bf16_ss(tmem + TB_S, tc::desc_add(kK, ao), tc::desc_add(qd, bo), id_sdp,
+                           kk > 0 ? 1u : 0u);
+          tc::umma_bf16_ss(tmem + TB_DP, tc::desc_add(vK, ao), tc::desc_add(dod, bo), id_sdp,
+                           kk > 0 ? 1u : 0u);
         }
         tc::umma_commit(sdp_full);
         return true;
       };
       if (ok) ok = issue_sdp(0);
       for (int t = 0; t < nblk && ok; ++t) {
-        const int st = t & 1;
+        const int st = t % QST;
         if (t + 1 < nblk && !issue_sdp(t + 1)) { ok = false; break; }
+        const int db = t & 1;  // dQ accumulator of this tile
         if (!tc::mbar_wait(pds_full, t & 1, abort_flag, a.status) ||
-            !tc::mbar_wait(dq_empty, (t & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+            !tc::mbar_wait(&dq_empty[db], ((t >> 1) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
         tc::tc_fence_after();
-        const uint32_t q_addr = tc::smem_u32(smem + B_OFF_Q + st * QT);
-        const uint32_t do_addr = tc::smem_u32(smem + B_OFF_DO + st * QT);
+        const uint64_t qmn = qMN + (uint64_t)((st * QT) >> 4);
+        const uint64_t domn = doMN + (uint64_t)((st * QT) >> 4);
 #pragma unroll
         for (int kk = 0; kk < BQB / 16; ++kk) {
           const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-          tc::umma_bf16_ss(tmem + TB_DV, tc::smem_desc_sw128(p_addr + kk * 32, 16, 1024),
-                           tc::smem_desc_sw128(do_addr + kk * 2048, QT / 2, 1024), id_acc, acc);
-          tc::umma_bf16_ss(tmem + TB_DK, tc::smem_desc_sw128(ds_addr + kk * 32, 16, 1024),
-                           tc::smem_desc_sw128(q_addr + kk * 2048, QT / 2, 1024), id_acc, acc);
+          tc::umma_bf16_ss(tmem + TB_DV, tc::desc_add(pK, kk * 32), tc::desc_add(domn, kk * 2048),
+                           id_acc, acc);
+          tc::umma_bf16_ss(tmem + TB_DK, tc::desc_add(dsK, kk * 32), tc::desc_add(qmn, kk * 2048),
+                           id_acc, acc);
         }
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk)
-          tc::umma_bf16_ss(tmem + TB_DQ, tc::smem_desc_sw128(k_addr + kk * 2048, TILE / 2, 1024),
-                           tc::smem_desc_sw128(ds_addr + kk * 2048, PT, 1024), id_dq,
-                           kk > 0 ? 1u : 0u);
+          tc::umma_bf16_ss(tmem + TB_DQ + db * BQB, tc::desc_add(kMN, kk * 2048),
+                           tc::desc_add(dsMN, kk * 2048), id_dq, kk > 0 ? 1u : 0u);
         tc::umma_commit(pds_empty);
         tc::umma_commit(&qd_empty[st]);
-        tc::umma_commit(dq_full);
+        tc::umma_commit(&dq_full[db]);
       }
       if (ok) tc::umma_commit(dkv_full);
       tc::umma_commit(drained);
       drain_wait(drained, 0);
     }
-  } else if (warp < 6) {
-    // ---------------- P^T and dS^T, one key row per thread
+  } else if (warp < 10) {
+    // ---------------- P^T and dS^T: one key row per thread, half the columns per warp
     const int qw = warp & 3;
+    const int ch = (warp - 2) >> 2;  // column half: queries [32 ch, 32 ch + 32) of the tile
     const int row = qw * 32 + lane;
     const int key = kb * BKV + row;
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
@@ -537,49 +560,42 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t ds_row = tc::smem_u32(smem + B_OFF_DS) + row * 128;
     bool ok = true;
     for (int t = 0; t < nblk; ++t) {
-      const int q0 = (i0 + t) * BQB;
-      const float* ld = reinterpret_cast<const float*>(smem + B_OFF_LD) + (t & 1) * 2 * BQB;
+      const int q0 = (i0 + t) * BQB + 32 * ch;
+      const float* ld = reinterpret_cast<const float*>(smem + B_OFF_LD) + (t % QST) * 2 * BQB + 32 * ch;
       ok = tc::mbar_wait(sdp_full, t & 1, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc::tc_fence_after();
-      // The query tile's lse/D, staged by the TMA warp and published by the
-      // stage's qd_full barrier (already complete: the scores came from it).
-      ok = tc::mbar_wait(&qd_full[t & 1], (t >> 1) & 1, abort_flag, a.status);
+      uint32_t sv[32], dp[32];
+      tc::tmem_ld_32x32b_x32(lane_base + TB_S + 32 * ch, sv);
+      tc::tmem_ld_32x32b_x32(lane_base + TB_DP + 32 * ch, dp);
+      tc::tmem_ld_wait();
+      tc::tc_fence_before();
+      tc::mbar_arrive(sdp_empty);
+      // The tile's lse/D, staged by the TMA warp and published by the stage's
+      // qd_full barrier (already complete: the scores came from it).
+      ok = tc::mbar_wait(&qd_full[t % QST], (t / QST) & 1, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      // S^T and dP^T rows in four 16-column chunks, read before the buffers
-      // are handed back; P^T / dS^T packed to bf16.
-      uint32_t pp[32], pd[32];
-      {
-        uint32_t sv[64], dp[64];
+      uint32_t pp[16], pd[16];
+      const bool edge = (q0 < key + 1) || (q0 + 32 > a.T) || (key >= a.T);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          tc::tmem_ld_32x32b_x16(lane_base + TB_S + 16 * c, *reinterpret_cast<uint32_t(*)[16]>(&sv[16 * c]));
-          tc::tmem_ld_32x32b_x16(lane_base + TB_DP + 16 * c, *reinterpret_cast<uint32_t(*)[16]>(&dp[16 * c]));
+      for (int c = 0; c < 16; ++c) {
+        float p0 = ex2(__uint_as_float(sv[2 * c]) * a.sl2 - ld[2 * c]);
+        float p1 = ex2(__uint_as_float(sv[2 * c + 1]) * a.sl2 - ld[2 * c + 1]);
+        if (edge) {
+          const int qa = q0 + 2 * c, qb2 = qa + 1;
+          if (qa < key || qa >= a.T || key >= a.T) p0 = 0.f;
+          if (qb2 < key || qb2 >= a.T || key >= a.T) p1 = 0.f;
         }
-        tc::tmem_ld_wait();
-        tc::tc_fence_before();
-        tc::mbar_arrive(sdp_empty);
-        const bool edge = (q0 < key + 1) || (q0 + BQB > a.T) || (key >= a.T);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          float p0 = ex2(__uint_as_float(sv[2 * c]) * a.sl2 - ld[2 * c]);
-          float p1 = ex2(__uint_as_float(sv[2 * c + 1]) * a.sl2 - ld[2 * c + 1]);
-          if (edge) {
-            const int qa = q0 + 2 * c, qb2 = qa + 1;
-            if (qa < key || qa >= a.T || key >= a.T) p0 = 0.f;
-            if (qb2 < key || qb2 >= a.T || key >= a.T) p1 = 0.f;
-          }
-          const float d0 = p0 * (__uint_as_float(dp[2 * c]) - ld[BQB + 2 * c]);
-          const float d1 = p1 * (__uint_as_float(dp[2 * c + 1]) - ld[BQB + 2 * c + 1]);
-          pp[c] = pack_bf16x2(p0, p1);
-          pd[c] = pack_bf16x2(d0, d1);
-        }
+        const float d0 = p0 * (__uint_as_float(dp[2 * c]) - ld[BQB + 2 * c]);
+        const float d1 = p1 * (__uint_as_float(dp[2 * c + 1]) - ld[BQB + 2 * c + 1]);
+        pp[c] = pack_bf16x2(p0, p1);
+        pd[c] = pack_bf16x2(d0, d1);
       }
       ok = tc::mbar_wait(pds_empty, (t & 1) ^ 1, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const uint32_t sw = (uint32_t)((u ^ (row & 7)) << 4);
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t sw = (uint32_t)(((4 * ch + u) ^ (row & 7)) << 4);
         tc::st_shared_v4(p_row + sw, pp[4 * u], pp[4 * u + 1], pp[4 * u + 2], pp[4 * u + 3]);
         tc::st_shared_v4(ds_row + sw, pd[4 * u], pd[4 * u + 1], pd[4 * u + 2], pd[4 * u + 3]);
       }
@@ -591,28 +607,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
+      // Warps of column half 0 write dV rows, those of half 1 dK rows.
       tc::tc_fence_after();
       const int64_t grow = ((int64_t)b * a.T + key) * a.ldg + col0;
+      const uint32_t base = lane_base + (ch ? TB_DK : TB_DV);
+      const float mul = ch ? a.scale : 1.f;
+      __nv_bfloat16* dst = (ch ? a.dk : a.dv) + grow;
 #pragma unroll 1
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t base = lane_base + (which ? TB_DK : TB_DV);
-        const float mul = which ? a.scale : 1.f;
-        __nv_bfloat16* dst = (which ? a.dk : a.dv) + grow;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tc::tmem_ld_32x32b_x32(base + c * 32, o);
-          tc::tmem_ld_wait();
-          if (key < a.T) {
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tc::tmem_ld_32x32b_x32(base + c * 32, o);
+        tc::tmem_ld_wait();
+        if (key < a.T) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              uint4 v;
-              v.x = pack_bf16x2(__uint_as_float(o[8 * u + 0]) * mul, __uint_as_float(o[8 * u + 1]) * mul);
-              v.y = pack_bf16x2(__uint_as_float(o[8 * u + 2]) * mul, __uint_as_float(o[8 * u + 3]) * mul);
-              v.z = pack_bf16x2(__uint_as_float(o[8 * u + 4]) * mul, __uint_as_float(o[8 * u + 5]) * mul);
-              v.w = pack_bf16x2(__uint_as_float(o[8 * u + 6]) * mul, __uint_as_float(o[8 * u + 7]) * mul);
-              reinterpret_cast<uint4*>(dst + c * 32)[u] = v;
-            }
+          for (int u = 0; u < 4; ++u) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(o[8 * u + 0]) * mul, __uint_as_float(o[8 * u + 1]) * mul);
+            v.y = pack_bf16x2(__uint_as_float(o[8 * u + 2]) * mul, __uint_as_float(o[8 * u + 3]) * mul);
+            v.z = pack_bf16x2(__uint_as_float(o[8 * u + 4]) * mul, __uint_as_float(o[8 * u + 5]) * mul);
+            v.w = pack_bf16x2(__uint_as_float(o[8 * u + 6]) * mul, __uint_as_float(o[8 * u + 7]) * mul);
+            reinterpret_cast<uint4*>(dst + c * 32)[u] = v;
           }
         }
       }
@@ -626,7 +640,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     float* dq_bh = a.dq + (int64_t)b * a.T * dq_row + col0 + dim;
     for (int t = 0; t < nblk; ++t) {
       const int q0 = (i0 + t) * BQB;
-      bool ok = tc::mbar_wait(dq_full, t & 1, abort_flag, a.status);
+      bool ok = tc::mbar_wait(&dq_full[t & 1], (t >> 1) & 1, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc::tc_fence_after();
       float* dst = dq_bh + (int64_t)q0 * dq_row;
@@ -634,11 +648,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll 1
       for (int c0 = 0; c0 < BQB; c0 += 16) {
         uint32_t v[16];
-        tc::tmem_ld_32x32b_x16(lane_base + TB_DQ + c0, v);
+        tc::tmem_ld_32x32b_x16(lane_base + TB_DQ + (t & 1) * BQB + c0, v);
         tc::tmem_ld_wait();
         if (c0 + 16 == BQB) {  // the whole tile has been read: TMEM may be reused
           tc::tc_fence_before();
-          tc::mbar_arrive(dq_empty);
+          tc::mbar_arrive(&dq_empty[t & 1]);
         }
         float vv[16];
 #pragma unroll

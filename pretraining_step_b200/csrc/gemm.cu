@@ -299,6 +299,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_bf16_f32(BM, BN, p.a_mn, p.b_mn);
+      // Descriptors of stage 0; a stage adds STAGE_BYTES, a 16-wide K step adds
+      // 32 bytes (K-major) or 16 rows of 128 bytes (MN-major).
+      const uint32_t s0 = tc::smem_u32(smem);
+      const uint64_t adesc0 = p.a_mn ? tc::smem_desc_sw128(s0, 8192, 1024) : tc::smem_desc_sw128(s0, 16, 1024);
+      const uint64_t bdesc0 = p.b_mn ? tc::smem_desc_sw128(s0 + C::A_BYTES, 8192, 1024)
+                                     : tc::smem_desc_sw128(s0 + C::A_BYTES, 16, 1024);
+      const uint32_t a_step = p.a_mn ? 2048 : 32, b_step = p.b_mn ? 2048 : 32;
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -318,16 +325,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc::tc_fence_after();
-          const uint32_t a_base = tc::smem_u32(smem + stage * C::STAGE_BYTES);
-          const uint32_t b_base = a_base + C::A_BYTES;
+          const uint64_t ad = adesc0 + (uint64_t)((stage * C::STAGE_BYTES) >> 4);
+          const uint64_t bd = bdesc0 + (uint64_t)((stage * C::STAGE_BYTES) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = p.a_mn ? tc::smem_desc_sw128(a_base + kk * 2048, 8192, 1024)
-                                       : tc::smem_desc_sw128(a_base + kk * 32, 16, 1024);
-            const uint64_t bd = p.b_mn ? tc::smem_desc_sw128(b_base + kk * 2048, 8192, 1024)
-                                       : tc::smem_desc_sw128(b_base + kk * 32, 16, 1024);
-            tc::umma_bf16_ss(d_tmem, ad, bd, idesc, (kb > c.kb0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc::umma_bf16_ss(d_tmem, tc::desc_add(ad, kk * a_step), tc::desc_add(bd, kk * b_step),
+                             idesc, (kb > c.kb0 || kk > 0) ? 1u : 0u);
           tc::umma_commit(&empty[stage]);
           if (++stage == C::STAGES) {
             stage = 0;
@@ -517,6 +520,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       const uint32_t idesc = tc::idesc_bf16_f32(2 * BM, BN, p.a_mn, p.b_mn);
+      const uint32_t s0 = tc::smem_u32(smem);
+      const uint64_t adesc0 = p.a_mn ? tc::smem_desc_sw128(s0, 8192, 1024) : tc::smem_desc_sw128(s0, 16, 1024);
+      const uint64_t bdesc0 = p.b_mn ? tc::smem_desc_sw128(s0 + C::A_BYTES, 8192, 1024)
+                                     : tc::smem_desc_sw128(s0 + C::A_BYTES, 16, 1024);
+      const uint32_t a_step = p.a_mn ? 2048 : 32, b_step = p.b_mn ? 2048 : 32;
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -536,16 +544,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc::tc_fence_after();
-          const uint32_t a_base = tc::smem_u32(smem + stage * C::STAGE_BYTES);
-          const uint32_t b_base = a_base + C::A_BYTES;
+          const uint64_t ad = adesc0 + (uint64_t)((stage * C::STAGE_BYTES) >> 4);
+          const uint64_t bd = bdesc0 + (uint64_t)((stage * C::STAGE_BYTES) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = p.a_mn ? tc::smem_desc_sw128(a_base + kk * 2048, 8192, 1024)
-                                       : tc::smem_desc_sw128(a_base + kk * 32, 16, 1024);
-            const uint64_t bd = p.b_mn ? tc::smem_desc_sw128(b_base + kk * 2048, 8192, 1024)
-                                       : tc::smem_desc_sw128(b_base + kk * 32, 16, 1024);
-            tc::umma_bf16_ss_pair(d_tmem, ad, bd, idesc, (kb > c.kb0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc::umma_bf16_ss_pair(d_tmem, tc::desc_add(ad, kk * a_step), tc::desc_add(bd, kk * b_step),
+                                  idesc, (kb > c.kb0 || kk > 0) ? 1u : 0u);
           tc::umma_commit_pair(&empty[stage]);
           if (++stage == C::STAGES) {
             stage = 0;

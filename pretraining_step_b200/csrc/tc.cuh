@@ -265,6 +265,11 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// A descriptor advanced by `bytes` (a multiple of 16) along its start address.
+__device__ __forceinline__ uint64_t desc_add(uint64_t desc, uint32_t bytes) {
+  return desc + (uint64_t)(bytes >> 4);
+}
+
 // Instruction descriptor of kind::f16: bf16 A and B, fp32 D, M x N tile,
 // operand majorness (0 = K-major, 1 = MN-major).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {

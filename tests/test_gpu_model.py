@@ -195,3 +195,68 @@ def test_profiler_counts_launches():
     assert stats["attn_fwd"]["launches"] == depth
     assert all(v["ms"] > 0 for v in stats.values())
     m.close()
+
+
+@pytest.mark.parametrize("depth,B,T", [(12, 16, 2048), (26, 16, 2048)])
+def test_spec_init_properties_depth12_depth26(depth, B, T):
+    """The depth-12 and depth-26 workloads at full size (B = 16, T = 2048):
+    at the specified init the loss is ln 32768, every gradient except
+    lm_head's is exactly zero and lm_head's matches its closed form on
+    sampled rows."""
+    m = _gpt(depth, seed=depth)
+    tok, tgt = inputs.token_batch(depth, B, T)
+    loss = m.fwd_bwd(tok, tgt)
+    assert abs(loss - 15 * math.log(2)) / (15 * math.log(2)) < 2e-3
+    for i in [0, 1, 3, 5, 6, 6 * depth]:
+        assert not m.grad(i).any(), i
+    E = m.read(0).astype(np.float64)
+    g = m.grad(6 * depth + 1)
+    m.close()
+    N = B * T
+    x = E[tok.ravel()]
+    xf = x / np.sqrt(np.mean(x * x, axis=1, keepdims=True) + 1e-6)
+    colsum = xf.sum(axis=0) / (V * N)
+    for r in np.random.default_rng(depth).choice(V, 32, replace=False):
+        expect = colsum - xf[tgt.ravel() == r].sum(axis=0) / N
+        assert rel_fro(g[r], expect) < 2e-2
+
+
+def test_depth12_random_weights_short_rows():
+    """Depth 12 (d 768, 6 heads) on all-random weights, checked against the
+    oracle on a short batch (B = 1, T = 128) the oracle finishes quickly."""
+    depth, B, T = 12, 1, 128
+    P = inputs.random_params(depth, seed=120)
+    tok, tgt = inputs.token_batch(121, B, T)
+    m = _gpt(depth)
+    m.load(P)
+    loss = m.fwd_bwd(tok, tgt)
+    G = m.grads()
+    m.close()
+    lref, Gref, _ = oracle.gpt_fwd_bwd(depth, P, tok, tgt)
+    assert abs(loss - lref) / lref < 2e-3
+    for i, (gg, r) in enumerate(zip(G, Gref)):
+        assert rel_fro(gg, r) < 3e-2, (i, rel_fro(gg, r))
+
+
+def test_newton_schulz_sweep_sizes():
+    """The Newton-Schulz sweep at its sizes (stacks of 1664 x 1664,
+    1664 x 6656 and 6656 x 1664): one matrix of each stack against the
+    oracle, and the singular values of every wide/tall result in the band
+    the quintic maps well-conditioned inputs into."""
+    t = torch()
+    for count, rows, cols in [(64, 1664, 1664), (26, 1664, 6656), (26, 6656, 1664)]:
+        X = inputs.normal_stack(500 + rows + cols, count, rows, cols)
+        out = t.empty(count, rows, cols, dtype=t.bfloat16, device="cuda")
+        scratch = t.empty(nc.newton_schulz_scratch_bytes(count, rows, cols), dtype=t.uint8,
+                          device="cuda")
+        nc.newton_schulz(t.from_numpy(X).cuda().to(t.bfloat16), out, count, rows, cols, 5,
+                         scratch)
+        t.cuda.synchronize()
+        i = count // 2
+        got = out[i].float().cpu().numpy()
+        assert rel_fro(got, oracle.newton_schulz(X[i])) < 2e-2
+        if rows != cols:
+            for j in (0, count - 1):
+                s = np.linalg.svd(out[j].float().cpu().numpy(), compute_uv=False)
+                assert s.min() > 0.6 and s.max() < 1.22
+        del out, scratch
