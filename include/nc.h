@@ -168,7 +168,13 @@ typedef enum {
   NC_EPI_RELU2 = 3,      /* D(bf16) = max(alpha*acc, 0)^2        (ReLU^2)     */
   NC_EPI_RELU2_BWD = 4,  /* D(bf16) = 2*sqrt(aux(bf16))*alpha*acc (aux = relu(u)^2) */
   NC_EPI_AXPBY_BF16 = 5, /* D(bf16) = alpha*acc + beta*aux(bf16)              */
-  NC_EPI_ACC_F32 = 6     /* D(f32) += alpha*acc                  (atomic)     */
+  NC_EPI_ACC_F32 = 6,    /* D(f32) += alpha*acc                  (atomic)     */
+  NC_EPI_ROPE_QKNORM = 7 /* fused q|k|v projection: columns [0, 2*H*128) are q
+                            and k heads of 128, rotated by RoPE at position
+                            row % T (pairs i, i + 64) then RMS-normalised per
+                            head, rstd written to rstd_qk[which][row * H + h];
+                            columns from 2*H*128 on (v) are stored as is.
+                            D(bf16).  Needs N = 3*H*128.                    */
 } nc_epilogue;
 
 /* Batched GEMM on the tcgen05 tensor cores, D[b] = epi(op(A[b]) op(B[b])^T):
@@ -194,6 +200,13 @@ typedef struct {
   nc_epilogue epi;
   float alpha, beta;
   int split_k;
+  /* NC_EPI_ROPE_QKNORM only: sequence length T, heads H, cos/sin table
+   * (float2 [>= T][64], theta_i(pos) = pos * 10000^(-i/64)) and the two rstd
+   * outputs (f32 [M * H] each: q then k). */
+  int rope_T, rope_H;
+  const void* rope_tab;
+  float* rstd_q;
+  float* rstd_k;
 } nc_gemm_desc;
 nc_status nc_op_gemm(const nc_gemm_desc* desc, void* stream);
 

@@ -18,7 +18,7 @@ NC_OK, NC_ERR_INVALID_ARG, NC_ERR_OOM, NC_ERR_CUDA, NC_ERR_TOKEN_RANGE, NC_ERR_T
     NC_ERR_UNSUPPORTED = range(7)
 NC_INIT_SPEC, NC_INIT_ALL_RANDOM = 0, 1
 (EPI_STORE_BF16, EPI_STORE_F32, EPI_RESID_F32, EPI_RELU2, EPI_RELU2_BWD, EPI_AXPBY_BF16,
- EPI_ACC_F32) = range(7)
+ EPI_ACC_F32, EPI_ROPE_QKNORM) = range(8)
 
 
 class NcError(RuntimeError):
@@ -44,7 +44,9 @@ class GemmDesc(ctypes.Structure):
                 ("aux", ctypes.c_void_p), ("ldaux", ctypes.c_int64),
                 ("stride_aux", ctypes.c_int64),
                 ("epi", ctypes.c_int), ("alpha", ctypes.c_float), ("beta", ctypes.c_float),
-                ("split_k", ctypes.c_int)]
+                ("split_k", ctypes.c_int), ("rope_T", ctypes.c_int), ("rope_H", ctypes.c_int),
+                ("rope_tab", ctypes.c_void_p), ("rstd_q", ctypes.c_void_p),
+                ("rstd_k", ctypes.c_void_p)]
 
 
 class KernelStat(ctypes.Structure):

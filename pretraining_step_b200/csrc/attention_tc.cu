@@ -65,6 +65,21 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^x on the FMA pipe, for a share of the softmax exponentials so the MUFU
+// unit is not the only limit: 2^x = 2^floor(x) * p(x - floor(x)) with a cubic
+// p fitted here for relative error on [0, 1) with p(0) = 1 (max relative
+// error 8.6e-5, far below the bf16 rounding P receives).  Exactly 0 below
+// 2^-126, including for masked scores (x = -inf).
+__device__ __forceinline__ float ex2_fma(float x) {
+  constexpr float c1 = 0.69511570925694f, c2 = 0.22764980831700f, c3 = 0.07706263250999f;
+  const float xc = fmaxf(x, -126.f);
+  const float j = floorf(xc);
+  const float f = xc - j;
+  const float p = fmaf(fmaf(fmaf(c3, f, c2), f, c1), f, 1.f);
+  const float r = __int_as_float(__float_as_int(p) + ((int)j << 23));
+  return x < -126.f ? 0.f : r;
+}
+
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = globaltimer();
   while (!tc::mbar_try_wait(bar, parity))
@@ -225,37 +240,52 @@ __global__ void __launch_bounds__(kThreads, 2)
       tc::tmem_ld_wait();
       tc::tc_fence_before();
       tc::mbar_arrive(&s_empty[s]);
-      // Scale, mask, block maximum.
+      // Block maximum on raw scores (the scale is positive); masking only on
+      // tiles that reach the diagonal or the end of the row.
       const int k0 = j * FKV;
-      const bool diag = (k0 + FKV > qb * BQ);
-      float mx = -INFINITY;
+      float mx_raw = -INFINITY;
+      if (k0 + FKV > qb * BQ || k0 + FKV > a.T) {
 #pragma unroll
-      for (int c = 0; c < 2; ++c)
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          float x = __uint_as_float(r[c][i]) * a.sl2;
-          const int kj = k0 + c * 32 + i;
-          if ((diag && kj > qi) || kj >= a.T) x = -INFINITY;
-          r[c][i] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
-        }
+          for (int i = 0; i < 32; ++i) {
+            const int kj = k0 + c * 32 + i;
+            float x = __uint_as_float(r[c][i]);
+            if (kj > qi || kj >= a.T) x = -INFINITY;
+            r[c][i] = __float_as_uint(x);
+            mx_raw = fmaxf(mx_raw, x);
+          }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) mx_raw = fmaxf(mx_raw, __uint_as_float(r[c][i]));
+      }
+      const float mx = mx_raw * a.sl2;
       float alpha = 1.f;
       if (mx > m_used + kRescaleThreshold) {
         alpha = ex2(m_used - mx);  // 0 on the first tile
         m_used = mx;
       }
-      const float mu = (m_used == -INFINITY) ? 0.f : m_used;
+      const float neg_mu = (m_used == -INFINITY) ? 0.f : -m_used;
       l *= alpha;
+      // p = 2^(s * scale * log2 e - m): one FFMA feeding ex2 per score.
       uint32_t pk[32];
+      float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
       for (int c = 0; c < 2; ++c)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2(__uint_as_float(r[c][2 * i]) - mu);
-          const float p1 = ex2(__uint_as_float(r[c][2 * i + 1]) - mu);
-          l += p0 + p1;
+          const float x0 = fmaf(__uint_as_float(r[c][2 * i]), a.sl2, neg_mu);
+          const float x1 = fmaf(__uint_as_float(r[c][2 * i + 1]), a.sl2, neg_mu);
+          // every fourth pair on the FMA pipe, the rest on MUFU
+          const float p0 = (i & 3) == 3 ? ex2_fma(x0) : ex2(x0);
+          const float p1 = (i & 3) == 3 ? ex2_fma(x1) : ex2(x1);
+          ls0 += p0;
+          ls1 += p1;
           pk[c * 16 + i] = pack_bf16x2(p0, p1);
         }
+      l += ls0 + ls1;
       // The P tile and the O accumulator are free once the previous P V landed.
       if (j >= 1) {
         ok = tc::mbar_wait(pv_done, (j - 1) & 1, abort_flag, a.status);

@@ -17,6 +17,9 @@ enum : int {
   kDevTokenRange = 2  // a token / target id outside [0, vocab)
 };
 
+// RMSNorm epsilon of every norm in the model (pre-norms and QK-norm).
+constexpr float kNormEps = 1e-6f;
+
 // Wall-clock limit of one mbarrier wait (ns).  A correct kernel never waits
 // more than microseconds on one barrier.
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;

@@ -12,8 +12,6 @@
 namespace nc {
 namespace {
 
-constexpr float kNormEps = 1e-6f;
-
 // ------------------------------------------------------------------ embedding
 __global__ void embed_gather_kernel(const int32_t* __restrict__ tok, int64_t n, const float* __restrict__ E,
                                     int V, int d, float* __restrict__ x, int* status) {
@@ -127,55 +125,8 @@ __global__ void rope_table_kernel(float2* tab, int T, int hd) {
   tab[i] = make_float2((float)cos(th), (float)sin(th));
 }
 
-// In place on the q and k slices of qkv [n, ld] (head_dim 128): rotate pairs
-// (i, i + 64), then RMS-normalise each head; rstd [n, H] per slice.  One warp
-// per (token, head, q|k): lane l holds dims 4(l % 16) .. +3 of half l / 16, so
-// its rotation partner sits 16 lanes away (one shuffle), and every access is
-// an 8-byte vector.
-__global__ void rope_qknorm_fwd_kernel(__nv_bfloat16* __restrict__ qkv, int64_t ld, int64_t n,
-                                       int T, int H, const float2* __restrict__ tab,
-                                       float* __restrict__ rstd_q, float* __restrict__ rstd_k) {
-  const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (w >= n * H * 2) return;
-  const int which = (int)(w & 1);
-  const int64_t th = w >> 1;
-  const int h = (int)(th % H);
-  const int64_t tok = th / H;
-  const int pos = (int)(tok % T);
-  const int half = lane >> 4, j = lane & 15;
-  uint2* p = reinterpret_cast<uint2*>(qkv + tok * ld + (int64_t)which * H * 128 + (int64_t)h * 128 +
-                                      half * 64 + 4 * j);
-  const uint2 xv = *p;
-  uint2 yv;
-  yv.x = __shfl_xor_sync(0xffffffffu, xv.x, 16);
-  yv.y = __shfl_xor_sync(0xffffffffu, xv.y, 16);
-  const float4* t4 = reinterpret_cast<const float4*>(tab + (int64_t)pos * 64 + 4 * j);
-  const float4 cs01 = t4[0], cs23 = t4[1];
-  const float c[4] = {cs01.x, cs01.z, cs23.x, cs23.z};
-  const float sn[4] = {cs01.y, cs01.w, cs23.y, cs23.w};
-  const float2 x01 = unpack_bf16x2(xv.x), x23 = unpack_bf16x2(xv.y);
-  const float2 y01 = unpack_bf16x2(yv.x), y23 = unpack_bf16x2(yv.y);
-  const float x[4] = {x01.x, x01.y, x23.x, x23.y};
-  const float y[4] = {y01.x, y01.y, y23.x, y23.y};
-  float o[4];
-  float ss = 0.f;
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    // first half: x_i c - x_{i+64} s;  second half: x_i s + x_{i+64} c
-    o[e] = half == 0 ? x[e] * c[e] - y[e] * sn[e] : y[e] * sn[e] + x[e] * c[e];
-    ss += o[e] * o[e];
-  }
-  ss = warp_sum(ss);
-  const float rs = rsqrtf(ss / 128.f + kNormEps);
-  uint2 ov;
-  ov.x = pack_bf16x2(o[0] * rs, o[1] * rs);
-  ov.y = pack_bf16x2(o[2] * rs, o[3] * rs);
-  *p = ov;
-  if (lane == 0) (which ? rstd_k : rstd_q)[tok * H + h] = rs;
-}
-
-// Backward of the above for one slice: g = dL/dyhat (f32 dense [n, H*128] for
+// Backward of RoPE + QK-norm (the forward is fused into the q|k|v GEMM
+// epilogue) for one slice: g = dL/dyhat (f32 dense [n, H*128] for
 // q, or bf16 with stride ldg for k), yhat the saved normalised output.
 //   dr = r * (g - yhat * mean(g * yhat));   dx = R(-theta) dr.
 // Writes bf16 into out (stride ld_out); may run in place on the k slice.
@@ -569,17 +520,6 @@ nc_status rmsnorm_bwd(const void* dh, const float* x, const float* rstd, const f
 
 nc_status rope_table(float2* tab, int T, int hd, cudaStream_t s) {
   rope_table_kernel<<<blocks_for((int64_t)T * hd / 2, 256), 256, 0, s>>>(tab, T, hd);
-  NC_CUDA_TRY(cudaGetLastError());
-  return NC_OK;
-}
-
-nc_status rope_qknorm_fwd(void* qkv, int64_t ld, int64_t n, int T, int H, int hd,
-                          const float2* tab, float* rstd_q, float* rstd_k, cudaStream_t s,
-                          Profiler* prof) {
-  Probe probe(prof, s, "rope_qknorm_fwd", 0.0, n * H * (2.0 * hd * 2 * 2 + 8.0));
-  if (hd != 128) return fail(NC_ERR_UNSUPPORTED, "rope_qknorm: head_dim must be 128");
-  rope_qknorm_fwd_kernel<<<blocks_for(n * H * 2 * 32, 256), 256, 0, s>>>(
-      (__nv_bfloat16*)qkv, ld, n, T, H, tab, rstd_q, rstd_k);
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }

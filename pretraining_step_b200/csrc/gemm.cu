@@ -48,9 +48,28 @@ struct Args {
   int epi;
   float alpha, beta;
   void* D;
-  int64_t ldd, stride_d;
-  const void* aux;
-  int64_t ldaux, stride_aux;
+  int64_t ldd;
+  // The RoPE/QK-norm epilogue (batch 1, no aux operand) keeps its parameters
+  // in fields it does not otherwise use: the kernel argument block stays at
+  // its size (growing it by 32 bytes measurably slowed every GEMM).
+  union {
+    int64_t stride_d;
+    struct {
+      int rope_T, rope_H;
+    };
+  };
+  union {
+    const void* aux;
+    const float2* rope_tab;
+  };
+  union {
+    int64_t ldaux;
+    float* rstd_q;
+  };
+  union {
+    int64_t stride_aux;
+    float* rstd_k;
+  };
   int* status;
 };
 
@@ -200,8 +219,72 @@ __device__ __forceinline__ void store_row_chunk(const Args& p, int b, int row, i
   }
 }
 
+// Fused q|k|v epilogue: this warp's 128 accumulator columns are one head.
+// q and k heads are rotated (pairs i, i + 64, position row % T) and
+// RMS-normalised; v heads are stored as computed.  The rotation preserves
+// the norm of every pair, so a first pass over TMEM takes the head's norm
+// and a second rotates, scales and stores column chunks c and c + 2 together.
+__device__ __forceinline__ void rope_head_epilogue(const Args& p, uint32_t taddr, int b, int row,
+                                                   int col0) {
+  const bool live = row < p.M && col0 < p.N;
+  const int d = p.rope_H * 128;
+  const int region = col0 / d;  // 0: q, 1: k, 2: v (uniform across the warp)
+  float rs = 1.f;
+  if (region < 2) {
+    float ss = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t r[32];
+      tc::tmem_ld_32x32b_x32(taddr + c * 32, r);
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float x = __uint_as_float(r[j]) * p.alpha;
+        ss += x * x;
+      }
+    }
+    rs = rsqrtf(ss / 128.f + kNormEps);
+    if (live) (region ? p.rstd_k : p.rstd_q)[(int64_t)row * p.rope_H + (col0 % d) / 128] = rs;
+  }
+  (void)b;  // batch 1: stride_d holds T and H here
+  __nv_bfloat16* D = (__nv_bfloat16*)p.D + (int64_t)row * p.ldd + col0;
+  const float4* tab = reinterpret_cast<const float4*>(p.rope_tab + (int64_t)(row % p.rope_T) * 64);
+#pragma unroll 1
+  for (int cp = 0; cp < 2; ++cp) {
+    uint32_t lo[32], hi[32];
+    tc::tmem_ld_32x32b_x32(taddr + cp * 32, lo);
+    tc::tmem_ld_32x32b_x32(taddr + (cp + 2) * 32, hi);
+    tc::tmem_ld_wait();
+    float w0[32], w1[32];
+    if (region < 2) {
+#pragma unroll
+      for (int i2 = 0; i2 < 16; ++i2) {
+        const float4 cs = live ? tab[cp * 16 + i2] : make_float4(1.f, 0.f, 1.f, 0.f);
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int i = 2 * i2 + e;
+          const float c = e ? cs.z : cs.x, sn = e ? cs.w : cs.y;
+          const float x0 = __uint_as_float(lo[i]) * p.alpha, x1 = __uint_as_float(hi[i]) * p.alpha;
+          w0[i] = (x0 * c - x1 * sn) * rs;
+          w1[i] = (x0 * sn + x1 * c) * rs;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        w0[i] = __uint_as_float(lo[i]) * p.alpha;
+        w1[i] = __uint_as_float(hi[i]) * p.alpha;
+      }
+    }
+    if (live) {
+      store_bf16_chunk(D + cp * 32, 32, w0);
+      store_bf16_chunk(D + (cp + 2) * 32, 32, w1);
+    }
+  }
+}
+
 // ------------------------------------------------------------------ kernel
-template <int BN>
+template <int BN, bool ROPE>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const Args p) {
@@ -361,6 +444,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tc_fence_after();
       const int row = c.mb * BM + row_in_tile;
       const bool aux = epi_has_aux(p.epi);
+      if constexpr (ROPE) {  // separate instantiation: the other GEMMs carry no RoPE code
+        rope_head_epilogue(p, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + half * CH * 32, c.b,
+                           row, c.nb * BN + half * CH * 32);
+      } else {
       // The aux chunk is loaded one chunk ahead so its HBM latency overlaps
       // the current chunk's TMEM load, arithmetic and stores.
       float xa[32], xb[32];
@@ -386,6 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
           store_row_chunk(p, c.b, row, col0, v, cur);
         }
+      }
       }
       tc::tc_fence_before();
       tc::mbar_arrive(&tempty[acc]);
@@ -420,6 +508,7 @@ struct Cfg2 {
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
 };
 
+template <bool ROPE>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const Args p) {
@@ -579,6 +668,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::tc_fence_after();
       const int row = c.mb * 2 * BM + (int)rank * BM + row_in_tile;
       const bool aux = epi_has_aux(p.epi);
+      if constexpr (ROPE) {  // separate instantiation: the other GEMMs carry no RoPE code
+        rope_head_epilogue(p, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + half * CH * 32, c.b,
+                           row, c.nb * BN + half * CH * 32);
+      } else {
       float xa[32], xb[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j) xa[j] = xb[j] = 0.f;
@@ -603,6 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           store_row_chunk(p, c.b, row, col0, v, cur);
         }
       }
+      }
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive_cluster(tempty_leader + acc * 8);
@@ -620,13 +714,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------ host
-template <int BN>
+template <int BN, bool ROPE>
 nc_status launch_bn(const nc_gemm_desc& d, int split, int* status, const char* tag,
                     cudaStream_t s, Profiler* prof) {
   using C = Cfg<BN>;
   static bool attr_set = false;
   if (!attr_set) {
-    NC_CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN>,
+    NC_CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN, ROPE>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
     attr_set = true;
   }
@@ -658,24 +752,32 @@ nc_status launch_bn(const nc_gemm_desc& d, int split, int* status, const char* t
   a.aux = d.aux;
   a.ldaux = d.ldaux;
   a.stride_aux = d.stride_aux;
+  if (d.epi == NC_EPI_ROPE_QKNORM) {  // shares storage with stride_d and the aux fields
+    a.rope_T = d.rope_T;
+    a.rope_H = d.rope_H;
+    a.rope_tab = static_cast<const float2*>(d.rope_tab);
+    a.rstd_q = d.rstd_q;
+    a.rstd_k = d.rstd_k;
+  }
   a.status = status;
   const int64_t total = (int64_t)a.tiles_m * a.tiles_n * a.split_k * a.batch;
   if (total >= (1ll << 31)) return fail(NC_ERR_INVALID_ARG, "gemm: too many tiles");
   const int grid = (int)std::min<int64_t>(total, num_sms());
   const double flops = 2.0 * d.M * (double)d.N * d.K * d.batch;
   Probe probe(prof, s, tag, flops, 0.0);
-  gemm_tc_kernel<BN><<<grid, kThreads, C::SMEM_BYTES, s>>>(ta, tb, a);
+  gemm_tc_kernel<BN, ROPE><<<grid, kThreads, C::SMEM_BYTES, s>>>(ta, tb, a);
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }
 
+template <bool ROPE>
 nc_status launch_pair(const nc_gemm_desc& d, int split, int* status, const char* tag,
                       cudaStream_t s, Profiler* prof) {
   using C = Cfg2;
   static bool attr_set = false;
   if (!attr_set) {
-    NC_CUDA_TRY(cudaFuncSetAttribute(gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     C::SMEM_BYTES));
+    NC_CUDA_TRY(cudaFuncSetAttribute(gemm_tc2_kernel<ROPE>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
     attr_set = true;
   }
   CUtensorMap ta, tb;
@@ -705,6 +807,13 @@ nc_status launch_pair(const nc_gemm_desc& d, int split, int* status, const char*
   a.aux = d.aux;
   a.ldaux = d.ldaux;
   a.stride_aux = d.stride_aux;
+  if (d.epi == NC_EPI_ROPE_QKNORM) {  // shares storage with stride_d and the aux fields
+    a.rope_T = d.rope_T;
+    a.rope_H = d.rope_H;
+    a.rope_tab = static_cast<const float2*>(d.rope_tab);
+    a.rstd_q = d.rstd_q;
+    a.rstd_k = d.rstd_k;
+  }
   a.status = status;
   const int64_t total = (int64_t)a.tiles_m * a.tiles_n * a.split_k * a.batch;
   if (total >= (1ll << 31)) return fail(NC_ERR_INVALID_ARG, "gemm: too many tiles");
@@ -723,7 +832,7 @@ nc_status launch_pair(const nc_gemm_desc& d, int split, int* status, const char*
   cfg.numAttrs = 1;
   const double flops = 2.0 * d.M * (double)d.N * d.K * d.batch;
   Probe probe(prof, s, tag, flops, 0.0);
-  NC_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_tc2_kernel, ta, tb, a));
+  NC_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<ROPE>, ta, tb, a));
   return NC_OK;
 }
 
@@ -763,15 +872,20 @@ nc_status gemm_launch(const GemmLaunch& g, cudaStream_t s, Profiler* prof) {
   if (!aligned(d.ldd) || (reinterpret_cast<uintptr_t>(d.D) & 15) ||
       (needs_aux && (reinterpret_cast<uintptr_t>(d.aux) & 15)))
     return fail(NC_ERR_INVALID_ARG, "gemm: output / aux must be 16-byte aligned rows");
-  if (d.epi < NC_EPI_STORE_BF16 || d.epi > NC_EPI_ACC_F32)
+  if (d.epi < NC_EPI_STORE_BF16 || d.epi > NC_EPI_ROPE_QKNORM)
     return fail(NC_ERR_INVALID_ARG, "gemm: unknown epilogue");
+  const bool rope = d.epi == NC_EPI_ROPE_QKNORM;
+  if (rope && (d.rope_T < 1 || d.rope_H < 1 || d.N != 3 * 128 * d.rope_H || !d.rope_tab ||
+               !d.rstd_q || !d.rstd_k || d.alpha != 1.f || d.batch != 1))
+    return fail(NC_ERR_INVALID_ARG, "gemm: the RoPE/QK-norm epilogue needs N = 3*128*H, T, a table and rstd outputs");
   int split = d.split_k;
   if (split != 1 && d.epi != NC_EPI_ACC_F32)
     return fail(NC_ERR_INVALID_ARG, "gemm: split_k > 1 needs the accumulate epilogue");
   // N tile: 256 unless 128 wastes less of the last column tile.
   const int waste256 = ((d.N + 255) / 256) * 256 - d.N;
   const int waste128 = ((d.N + 127) / 128) * 128 - d.N;
-  const bool bn256 = d.N > 128 && waste256 <= waste128;
+  // (the RoPE/QK-norm epilogue needs 256-wide tiles: each warp-half is a head)
+  const bool bn256 = rope || (d.N > 128 && waste256 <= waste128);
   const int bn = bn256 ? 256 : 128;
   const int num_kb = (d.K + BK - 1) / BK;
   if (split <= 0) {
@@ -786,10 +900,12 @@ nc_status gemm_launch(const GemmLaunch& g, cudaStream_t s, Profiler* prof) {
       const int64_t tiles = (int64_t)((d.M + 2 * BM - 1) / (2 * BM)) * ((d.N + 255) / 256) * d.batch;
       split = std::min(auto_split(tiles * 2, num_kb), num_kb);
     }
-    return launch_pair(d, split, g.status, g.tag, s, prof);
+    return rope ? launch_pair<true>(d, split, g.status, g.tag, s, prof)
+                : launch_pair<false>(d, split, g.status, g.tag, s, prof);
   }
-  return bn256 ? launch_bn<256>(d, split, g.status, g.tag, s, prof)
-               : launch_bn<128>(d, split, g.status, g.tag, s, prof);
+  if (rope) return launch_bn<256, true>(d, split, g.status, g.tag, s, prof);
+  return bn256 ? launch_bn<256, false>(d, split, g.status, g.tag, s, prof)
+               : launch_bn<128, false>(d, split, g.status, g.tag, s, prof);
 }
 
 }  // namespace nc

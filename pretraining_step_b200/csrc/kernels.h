@@ -47,9 +47,6 @@ nc_status rmsnorm_bwd(const void* dh, const float* x, const float* rstd, const f
                       int64_t rows, int d, float* dx, void* dx_bf16, cudaStream_t s,
                       Profiler* prof);
 nc_status rope_table(float2* tab, int T, int hd, cudaStream_t s);
-nc_status rope_qknorm_fwd(void* qkv, int64_t ld, int64_t n, int T, int H, int hd,
-                          const float2* tab, float* rstd_q, float* rstd_k, cudaStream_t s,
-                          Profiler* prof);
 nc_status rope_qknorm_bwd(const float* gf, const void* gb, int64_t ldg, const void* yhat,
                           int64_t ldy, const float* rstd, int64_t n, int T, int H, int hd,
                           const float2* tab, void* out, int64_t ld_out, cudaStream_t s,

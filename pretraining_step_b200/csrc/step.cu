@@ -333,8 +333,20 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
   for (int l = 0; l < L; ++l) {
     const bf16* W = p->blocks_b + l * 12 * d2;
     NC_TRY(rmsnorm_fwd(a.x[l], N, (int)d, a.h1[l], a.r1[l], s, pr));
-    NC_TRY(proj(p, a.h1[l], N, d, W, 3 * d, a.qkv[l], 3 * d, NC_EPI_STORE_BF16, nullptr, 0));
-    NC_TRY(rope_qknorm_fwd(a.qkv[l], 3 * d, N, T, H, hd, p->rope, a.rq[l], a.rk[l], s, pr));
+    {
+      // q|k|v projection with RoPE + QK-norm fused into the epilogue.
+      GemmLaunch g{};
+      g.status = p->status;
+      g.tag = "gemm_fwd";
+      g.d.M = (int)N; g.d.N = (int)(3 * d); g.d.K = (int)d; g.d.batch = 1;
+      g.d.A = a.h1[l]; g.d.lda = d; g.d.a_kmajor = 1;
+      g.d.B = W; g.d.ldb = d; g.d.b_kmajor = 1;
+      g.d.D = a.qkv[l]; g.d.ldd = 3 * d;
+      g.d.epi = NC_EPI_ROPE_QKNORM; g.d.alpha = 1.f; g.d.split_k = 1;
+      g.d.rope_T = T; g.d.rope_H = H; g.d.rope_tab = p->rope;
+      g.d.rstd_q = a.rq[l]; g.d.rstd_k = a.rk[l];
+      NC_TRY(gemm_launch(g, s, pr));
+    }
     NC_TRY(attention_fwd(a.qkv[l], a.qkv[l] + d, a.qkv[l] + 2 * d, 3 * d, a.o[l], d, a.lse[l], B,
                          T, H, p->status, s, pr));
     NC_TRY(proj(p, a.o[l], N, d, W + 3 * d2, d, a.xmid[l], d, NC_EPI_RESID_F32, a.x[l], d));

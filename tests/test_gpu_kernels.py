@@ -241,3 +241,45 @@ def test_newton_schulz_op(count, rows, cols):
         s = np.linalg.svd(got[i], compute_uv=False)
         if rows != cols:  # wide/tall N(0,1): every normalised sigma is well above 2e-3
             assert s.min() > 0.6 and s.max() < 1.22
+
+
+@pytest.mark.parametrize("M,H,T", [(300, 2, 100), (256, 1, 256), (130, 3, 64)])
+def test_gemm_rope_qknorm_epilogue(M, H, T):
+    """q|k|v projection with RoPE + QK-norm fused into the GEMM epilogue,
+    against the oracle's matmul, rotation and RMSNorm applied per head."""
+    t = torch()
+    d = 128 * H
+    K = d
+    X = inputs.bf16_normal(80 + M, (M, K))
+    W = inputs.bf16_normal(81 + M, (3 * d, K), std=K ** -0.5)
+    pos = np.arange(M) % T
+    th = pos[:, None] * 10000.0 ** (-np.arange(64)[None, :] / 64.0)
+    tab = np.stack([np.cos(th), np.sin(th)], axis=-1).astype(np.float32)  # [M, 64, 2]
+    tab_dev = dev_f32(np.ascontiguousarray(tab[:T]))
+    D = t.empty(M, 3 * d, dtype=t.bfloat16, device="cuda")
+    rq = t.empty(M, H, dtype=t.float32, device="cuda")
+    rk = t.empty(M, H, dtype=t.float32, device="cuda")
+    desc = nc.GemmDesc()
+    desc.M, desc.N, desc.K, desc.batch = M, 3 * d, K, 1
+    tx, tw = dev_bf16(X), dev_bf16(W)
+    desc.A, desc.lda, desc.a_kmajor = tx.data_ptr(), K, 1
+    desc.B, desc.ldb, desc.b_kmajor = tw.data_ptr(), K, 1
+    desc.D, desc.ldd = D.data_ptr(), 3 * d
+    desc.epi, desc.alpha, desc.split_k = nc.EPI_ROPE_QKNORM, 1.0, 1
+    desc.rope_T, desc.rope_H, desc.rope_tab = T, H, tab_dev.data_ptr()
+    desc.rstd_q, desc.rstd_k = rq.data_ptr(), rk.data_ptr()
+    nc._check(nc.lib().nc_op_gemm(desc, None))
+    t.cuda.synchronize()
+    ref = oracle.matmul_nt(X, W)
+    expect = ref.copy()
+    rstd = np.zeros((2, M, H))
+    for which in range(2):
+        for h in range(H):
+            cols = slice(which * d + h * 128, which * d + (h + 1) * 128)
+            rot = np.stack([oracle.rope_row(ref[m, cols], int(pos[m])) for m in range(M)])
+            y, r = oracle.rmsnorm(rot)
+            expect[:, cols] = y
+            rstd[which, :, h] = r
+    assert rel_fro(host(D), expect) < 5e-3
+    np.testing.assert_allclose(host(rq), rstd[0], rtol=1e-4)
+    np.testing.assert_allclose(host(rk), rstd[1], rtol=1e-4)
