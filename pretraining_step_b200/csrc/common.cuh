@@ -42,6 +42,15 @@ __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
   return __bfloat1622float2(h);
 }
 
+// Square root by the PTX approximate instruction (relative error about
+// 2^-23, sqrt(0) = 0): one instruction where sqrtf's IEEE rounding takes a
+// branchy sequence.  Used where the result is rounded to bf16 anyway.
+__device__ __forceinline__ float sqrt_approx(float x) {
+  float y;
+  asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

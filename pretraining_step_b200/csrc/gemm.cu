@@ -18,6 +18,7 @@
 // status word and every role drains and exits.
 
 #include <algorithm>
+#include <type_traits>
 
 #include "kernels.h"
 #include "tc.cuh"
@@ -176,7 +177,7 @@ __device__ __forceinline__ void store_row_chunk(const Args& p, int b, int row, i
           const float r = fmaxf(a, 0.f);
           w[j] = r * r;
         } else if (p.epi == NC_EPI_RELU2_BWD) {
-          w[j] = 2.f * sqrtf(fmaxf(x[j], 0.f)) * a;
+          w[j] = 2.f * sqrt_approx(fmaxf(x[j], 0.f)) * a;
         } else if (p.epi == NC_EPI_AXPBY_BF16) {
           w[j] = a + p.beta * x[j];
         } else {
@@ -505,25 +506,159 @@ struct Cfg2 {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = 6;
   static constexpr int TMEM_COLS = 2 * BN;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 256 + 1024;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 512 + 1024;
 };
 
-template <bool ROPE>
-__global__ void __launch_bounds__(kThreads, 1)
-    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const Args p) {
-  using C = Cfg2;
+// The pair kernel for epilogues that read an aux operand: one operand stage
+// fewer, and each epilogue warp owns an 8 KB ring of aux chunks (its 32 rows
+// x 32 columns: two fp32 or four bf16 slots) that it fills by TMA ahead of
+// use, across tile boundaries, so the aux read overlaps the main loop.
+struct Cfg2X : Cfg2 {
+  static constexpr int STAGES = 5;
+  static constexpr int X_WARP_BYTES = 8192;
+  static constexpr int X_MAX_SLOTS = 4;
+  static constexpr int X_BYTES = (kEpiThreads / 32) * X_WARP_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + X_BYTES + 512 + 1024;
+};
+static_assert(Cfg2X::SMEM_BYTES <= 232448, "aux-ring pair GEMM exceeds shared memory");
+
+// Request aux chunk g of this warp (tile pair + (g / CH) * npairs, column
+// chunk g % CH) into its ring slot; false when that tile does not exist.
+template <int BN, int CH>
+__device__ __forceinline__ bool aux_issue(const Args& p, const CUtensorMap* tmX, uint8_t* ring,
+                                          uint64_t* xfull, int slot_bytes, int slots, int g, int pair,
+                                          int npairs, int total, int rank, int q, int half) {
+  const int t = pair + (g / CH) * npairs;
+  if (t >= total) return false;
+  const TileCoord c = decode(p, t);
+  const int slot = g & (slots - 1);
+  tc::mbar_arrive_expect_tx(&xfull[slot], slot_bytes);
+  tc::tma_load_3d(ring + slot * slot_bytes, tmX, &xfull[slot], c.nb * BN + (half * CH + g % CH) * 32,
+                  c.mb * 2 * BM + rank * BM + q * 32, c.b);
+  return true;
+}
+
+// This lane's row of one ring slot, as floats.  The slot holds 32 rows of
+// 128 bytes (fp32, 128-byte swizzle) or 64 bytes (bf16, 64-byte swizzle).
+__device__ __forceinline__ void aux_read_slot(const uint8_t* slot, int lane, bool f32, float (&x)[32]) {
+  const uint32_t base = tc::smem_u32(slot);
+  if (f32) {
+    const uint32_t row = base + lane * 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint4 u = tc::ld_shared_v4(row + ((j ^ (lane & 7)) << 4));
+      x[4 * j] = __uint_as_float(u.x); x[4 * j + 1] = __uint_as_float(u.y);
+      x[4 * j + 2] = __uint_as_float(u.z); x[4 * j + 3] = __uint_as_float(u.w);
+    }
+  } else {
+    const uint32_t row = base + lane * 64;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint4 u = tc::ld_shared_v4(row + ((j ^ ((lane >> 1) & 3)) << 4));
+      float2 f;
+      f = unpack_bf16x2(u.x); x[8 * j + 0] = f.x; x[8 * j + 1] = f.y;
+      f = unpack_bf16x2(u.y); x[8 * j + 2] = f.x; x[8 * j + 3] = f.y;
+      f = unpack_bf16x2(u.z); x[8 * j + 4] = f.x; x[8 * j + 5] = f.y;
+      f = unpack_bf16x2(u.w); x[8 * j + 6] = f.x; x[8 * j + 7] = f.y;
+    }
+  }
+}
+
+// Aux epilogues of the ring kernel: the output has the aux operand's type, so
+// each lane writes its finished row back over its aux row in the slot, and
+// the warp then stores the 32 x 32 block row by row (8 lanes per 128-byte
+// fp32 row, 4 per 64-byte bf16 row): each store instruction covers whole
+// lines instead of 16 bytes of 32 different lines.
+__device__ __forceinline__ void aux_epilogue_chunk(const Args& p, uint8_t* slot, int lane, bool f32,
+                                                   int b, int row0, int col0, const uint32_t (&r)[32]) {
+  float x[32];
+  aux_read_slot(slot, lane, f32, x);
+  const uint32_t base = tc::smem_u32(slot);
+  if (f32) {  // D = aux + alpha*acc
+    const uint32_t rowa = base + lane * 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      tc::st_shared_v4(rowa + ((j ^ (lane & 7)) << 4),
+                       __float_as_uint(x[4 * j] + p.alpha * __uint_as_float(r[4 * j])),
+                       __float_as_uint(x[4 * j + 1] + p.alpha * __uint_as_float(r[4 * j + 1])),
+                       __float_as_uint(x[4 * j + 2] + p.alpha * __uint_as_float(r[4 * j + 2])),
+                       __float_as_uint(x[4 * j + 3] + p.alpha * __uint_as_float(r[4 * j + 3])));
+  } else {
+    float w[32];
+    const bool relu2_bwd = p.epi == NC_EPI_RELU2_BWD;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float a = __uint_as_float(r[j]) * p.alpha;
+      w[j] = relu2_bwd ? 2.f * sqrt_approx(fmaxf(x[j], 0.f)) * a : a + p.beta * x[j];
+    }
+    const uint32_t rowa = base + lane * 64;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      tc::st_shared_v4(rowa + ((j ^ ((lane >> 1) & 3)) << 4), pack_bf16x2(w[8 * j], w[8 * j + 1]),
+                       pack_bf16x2(w[8 * j + 2], w[8 * j + 3]), pack_bf16x2(w[8 * j + 4], w[8 * j + 5]),
+                       pack_bf16x2(w[8 * j + 6], w[8 * j + 7]));
+  }
+  __syncwarp();
+  const int ncol = p.N - col0;  // >= 1
+  if (f32) {
+    float* D = (float*)p.D + (int64_t)b * p.stride_d + col0;
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int rr = it * 4 + (lane >> 3), cc = lane & 7;
+      const uint4 u = tc::ld_shared_v4(base + rr * 128 + ((cc ^ (rr & 7)) << 4));
+      if (row0 + rr < p.M) {
+        float* d = D + (int64_t)(row0 + rr) * p.ldd + cc * 4;
+        if (cc * 4 + 4 <= ncol) {
+          *reinterpret_cast<uint4*>(d) = u;
+        } else {
+          const uint32_t e[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if (cc * 4 + i < ncol) d[i] = __uint_as_float(e[i]);
+        }
+      }
+    }
+  } else {
+    __nv_bfloat16* D = (__nv_bfloat16*)p.D + (int64_t)b * p.stride_d + col0;
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int rr = it * 8 + (lane >> 2), cc = lane & 3;
+      const uint4 u = tc::ld_shared_v4(base + rr * 64 + ((cc ^ ((rr >> 1) & 3)) << 4));
+      if (row0 + rr < p.M) {
+        __nv_bfloat16* d = D + (int64_t)(row0 + rr) * p.ldd + cc * 8;
+        if (cc * 8 + 8 <= ncol) {
+          *reinterpret_cast<uint4*>(d) = u;
+        } else {
+          const uint32_t e[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            if (cc * 8 + i < ncol) {
+              const uint32_t h = (e[i >> 1] >> ((i & 1) * 16)) & 0xffffu;
+              d[i] = __ushort_as_bfloat16((unsigned short)h);
+            }
+        }
+      }
+    }
+  }
+}
+
+template <bool ROPE, bool XR>
+__device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUtensorMap* tmB,
+                                              const CUtensorMap* tmX, const Args& p) {
+  using C = std::conditional_t<XR, Cfg2X, Cfg2>;
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint8_t* xring_all = smem + C::STAGES * C::STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::SMEM_BYTES - 512 - 1024);
   uint64_t* empty = full + C::STAGES;
   uint64_t* tfull = empty + C::STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drained = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint64_t* xbar = drained + 2;  // XR: X_MAX_SLOTS per epilogue warp
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -540,6 +675,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(&tempty[i], 2 * (kEpiThreads / 32));  // one arrive per epilogue warp of the pair
     }
     tc::mbar_init(drained, 1);
+    if constexpr (XR) {
+      for (int i = 0; i < (kEpiThreads / 32) * Cfg2X::X_MAX_SLOTS; ++i) tc::mbar_init(&xbar[i], 1);
+    }
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -557,8 +695,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      tc::tma_prefetch_desc(&tmA);
-      tc::tma_prefetch_desc(&tmB);
+      tc::tma_prefetch_desc(tmA);
+      tc::tma_prefetch_desc(tmB);
+      if constexpr (XR) tc::tma_prefetch_desc(tmX);
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
@@ -577,16 +716,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* b_dst = a_dst + C::A_BYTES;
           const int k0 = kb * BK;
           if (!p.a_mn) {
-            tc::tma_load_3d_pair(a_dst, &tmA, &full[stage], k0, m0, c.b);
+            tc::tma_load_3d_pair(a_dst, tmA, &full[stage], k0, m0, c.b);
           } else {
-            tc::tma_load_3d_pair(a_dst, &tmA, &full[stage], m0, k0, c.b);
-            tc::tma_load_3d_pair(a_dst + 8192, &tmA, &full[stage], m0 + 64, k0, c.b);
+            tc::tma_load_3d_pair(a_dst, tmA, &full[stage], m0, k0, c.b);
+            tc::tma_load_3d_pair(a_dst + 8192, tmA, &full[stage], m0 + 64, k0, c.b);
           }
           if (!p.b_mn) {
-            tc::tma_load_3d_pair(b_dst, &tmB, &full[stage], k0, n0, c.b);
+            tc::tma_load_3d_pair(b_dst, tmB, &full[stage], k0, n0, c.b);
           } else {
-            tc::tma_load_3d_pair(b_dst, &tmB, &full[stage], n0, k0, c.b);
-            tc::tma_load_3d_pair(b_dst + 8192, &tmB, &full[stage], n0 + 64, k0, c.b);
+            tc::tma_load_3d_pair(b_dst, tmB, &full[stage], n0, k0, c.b);
+            tc::tma_load_3d_pair(b_dst + 8192, tmB, &full[stage], n0 + 64, k0, c.b);
           }
           ++issued;
           if (++stage == C::STAGES) {
@@ -661,6 +800,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tempty_leader = tc::mapa_shared(tc::smem_u32(tempty), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
+    // XR: this warp's aux ring; chunk g (counted over this warp's tiles)
+    // lives in slot g % slots.  Chunks [g_use, g_use + slots) are in flight.
+    const bool xf32 = p.epi == NC_EPI_RESID_F32;
+    const int slot_bytes = xf32 ? 4096 : 2048;
+    const int slots = XR ? Cfg2X::X_WARP_BYTES / slot_bytes : 1;
+    const int slot_shift = slots == 4 ? 2 : 1;
+    uint8_t* ring = xring_all + (warp - 2) * (XR ? Cfg2X::X_WARP_BYTES : 0);
+    uint64_t* xfull = xbar + (warp - 2) * Cfg2X::X_MAX_SLOTS;
+    int g_use = 0;
+    if constexpr (XR) {
+      if (lane == 0)
+        for (int g = 0; g < slots; ++g)
+          aux_issue<BN, CH>(p, tmX, ring, xfull, slot_bytes, slots, g, pair, npairs, total, (int)rank, q,
+                            half);
+    }
+    bool xabort = false;
     for (int t = pair; t < total; t += npairs) {
       const TileCoord c = decode(p, t);
       bool ok = tc::mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status);
@@ -671,6 +826,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (ROPE) {  // separate instantiation: the other GEMMs carry no RoPE code
         rope_head_epilogue(p, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + half * CH * 32, c.b,
                            row, c.nb * BN + half * CH * 32);
+      } else if constexpr (XR) {
+#pragma unroll
+        for (int k = 0; k < CH; ++k) {
+          const int ch = half * CH + k;
+          uint32_t r[32];
+          tc::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + ch * 32, r);
+          const int col0 = c.nb * BN + ch * 32;
+          const int slot = g_use & (slots - 1);
+          const bool got = tc::mbar_wait(&xfull[slot], (g_use >> slot_shift) & 1, abort_flag, p.status);
+          tc::tmem_ld_wait();
+          if (!__all_sync(0xffffffffu, got)) {
+            xabort = true;
+            break;
+          }
+          if (col0 < p.N)
+            aux_epilogue_chunk(p, ring + slot * slot_bytes, lane, xf32, c.b, row - lane, col0, r);
+          // Every lane is done with the slot: order its accesses before the
+          // TMA refill of the same slot with the chunk `slots` ahead.
+          tc::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            aux_issue<BN, CH>(p, tmX, ring, xfull, slot_bytes, slots, g_use + slots, pair, npairs, total,
+                              (int)rank, q, half);
+          }
+          ++g_use;
+        }
+        if (xabort) break;
       } else {
       float xa[32], xb[32];
 #pragma unroll
@@ -703,6 +885,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
+    if constexpr (XR) {
+      // After an abort, let the aux copies still in flight land before the
+      // CTA exits (chunks past the last tile were never requested).
+      for (int g = g_use; g < g_use + slots; ++g)
+        if (pair + (g / CH) * npairs < total) drain_wait(&xfull[g & (slots - 1)], (g >> slot_shift) & 1);
+    }
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -711,6 +899,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::tc_fence_after();
     tc::tmem_dealloc2(tmem_base, C::TMEM_COLS);
   }
+}
+
+
+template <bool ROPE>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const Args p) {
+  gemm_tc2_body<ROPE, false>(&tmA, &tmB, nullptr, p);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc2_aux_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmX, const Args p) {
+  gemm_tc2_body<false, true>(&tmA, &tmB, &tmX, p);
 }
 
 // ------------------------------------------------------------------ host
@@ -770,17 +972,27 @@ nc_status launch_bn(const nc_gemm_desc& d, int split, int* status, const char* t
   return NC_OK;
 }
 
-template <bool ROPE>
+template <bool ROPE, bool XR>
 nc_status launch_pair(const nc_gemm_desc& d, int split, int* status, const char* tag,
                       cudaStream_t s, Profiler* prof) {
-  using C = Cfg2;
+  using C = std::conditional_t<XR, Cfg2X, Cfg2>;
   static bool attr_set = false;
   if (!attr_set) {
-    NC_CUDA_TRY(cudaFuncSetAttribute(gemm_tc2_kernel<ROPE>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+    if constexpr (XR)
+      NC_CUDA_TRY(cudaFuncSetAttribute(gemm_tc2_aux_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::SMEM_BYTES));
+    else
+      NC_CUDA_TRY(cudaFuncSetAttribute(gemm_tc2_kernel<ROPE>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
     attr_set = true;
   }
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tx;
+  if constexpr (XR) {
+    // aux chunks of 32 columns x 32 rows: 128-byte rows (fp32) or 64-byte rows (bf16)
+    const bool f32 = d.epi == NC_EPI_RESID_F32;
+    if (!make_tmap_3d(&tx, d.aux, f32, d.N, d.M, d.batch, d.ldaux, d.stride_aux, 32, 32, f32 ? 128 : 64))
+      return fail(NC_ERR_INVALID_ARG, "gemm: cuTensorMapEncodeTiled rejected the aux operand");
+  }
   const bool ok_a = d.a_kmajor ? make_tmap_bf16_3d(&ta, d.A, d.K, d.M, d.batch, d.lda, d.stride_a, BM)
                                : make_tmap_bf16_3d(&ta, d.A, d.M, d.K, d.batch, d.lda, d.stride_a, 64);
   const bool ok_b = d.b_kmajor ? make_tmap_bf16_3d(&tb, d.B, d.K, d.N, d.batch, d.ldb, d.stride_b, C::BN / 2)
@@ -832,7 +1044,10 @@ nc_status launch_pair(const nc_gemm_desc& d, int split, int* status, const char*
   cfg.numAttrs = 1;
   const double flops = 2.0 * d.M * (double)d.N * d.K * d.batch;
   Probe probe(prof, s, tag, flops, 0.0);
-  NC_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<ROPE>, ta, tb, a));
+  if constexpr (XR)
+    NC_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_tc2_aux_kernel, ta, tb, tx, a));
+  else
+    NC_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<ROPE>, ta, tb, a));
   return NC_OK;
 }
 
@@ -900,8 +1115,12 @@ nc_status gemm_launch(const GemmLaunch& g, cudaStream_t s, Profiler* prof) {
       const int64_t tiles = (int64_t)((d.M + 2 * BM - 1) / (2 * BM)) * ((d.N + 255) / 256) * d.batch;
       split = std::min(auto_split(tiles * 2, num_kb), num_kb);
     }
-    return rope ? launch_pair<true>(d, split, g.status, g.tag, s, prof)
-                : launch_pair<false>(d, split, g.status, g.tag, s, prof);
+    if (rope) return launch_pair<true, false>(d, split, g.status, g.tag, s, prof);
+    // Aux epilogues read the aux operand by TMA (rows and batch strides of
+    // 16-byte multiples, which the checks above already imply).
+    if (needs_aux && (d.batch == 1 || aligned(d.stride_aux)))
+      return launch_pair<false, true>(d, split, g.status, g.tag, s, prof);
+    return launch_pair<false, false>(d, split, g.status, g.tag, s, prof);
   }
   if (rope) return launch_bn<256, true>(d, split, g.status, g.tag, s, prof);
   return bn256 ? launch_bn<256, false>(d, split, g.status, g.tag, s, prof)

@@ -16,6 +16,12 @@ namespace nc {
 bool make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                        uint64_t batch, int64_t ld, int64_t bstride, uint32_t box_outer);
 
+// 3-D TMA tensor map of fp32 (f32) or bf16 elements with an explicit box
+// {box_inner, box_outer, 1} and swizzle span (0, 32, 64 or 128 bytes).
+bool make_tmap_3d(CUtensorMap* m, const void* base, bool f32, uint64_t inner, uint64_t outer,
+                  uint64_t batch, int64_t ld, int64_t bstride, uint32_t box_inner, uint32_t box_outer,
+                  int swizzle_bytes);
+
 struct GemmLaunch {
   nc_gemm_desc d;
   int* status;             // device status word (may be null)

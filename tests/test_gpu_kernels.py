@@ -50,9 +50,13 @@ def test_gemm_f32_store_and_alpha(a_k, b_k):
     assert rel_fro(host(D), 0.5 * oracle.matmul_nt(A, B)) < 2e-5
 
 
-def test_gemm_residual_relu2_and_backward_epilogues():
+@pytest.mark.parametrize("M,N,K", [(300, 384, 256),   # 128-wide tiles on one CTA
+                                   (600, 512, 256),   # CTA pairs, ragged M
+                                   # more 256 x 256 tiles than CTA pairs: the aux ring
+                                   # runs ahead across tile boundaries; ragged M and N
+                                   (8200, 1000, 128)])
+def test_gemm_residual_relu2_and_backward_epilogues(M, N, K):
     t = torch()
-    M, N, K = 300, 384, 256
     A = inputs.bf16_normal(5, (M, K))
     B = inputs.bf16_normal(6, (N, K), std=0.1)
     acc = oracle.matmul_nt(A, B)
@@ -79,6 +83,29 @@ def test_gemm_residual_relu2_and_backward_epilogues():
             alpha=2.0315, beta=-4.775)
     t.cuda.synchronize()
     assert rel_fro(host(D4), 2.0315 * acc - 4.775 * Aux) < 5e-3
+
+
+def test_gemm_batched_aux_epilogues():
+    """Batched (strided) GEMMs with an aux operand, on CTA-pair tiles: the
+    alpha*acc + beta*aux form of the Newton-Schulz steps and the fp32 residual."""
+    t = torch()
+    bt, M, N, K = 3, 520, 512, 192
+    A = inputs.bf16_normal(40, (bt, M, K))
+    B = inputs.bf16_normal(41, (bt, N, K), std=0.1)
+    Aux = inputs.bf16_normal(42, (bt, M, N))
+    R = np.random.default_rng(43).standard_normal((bt, M, N)).astype(np.float32)
+    D = t.empty(bt, M, N, dtype=t.bfloat16, device="cuda")
+    nc.gemm(M, N, K, dev_bf16(A), dev_bf16(B), D, batch=bt, stride_a=M * K, stride_b=N * K,
+            stride_d=M * N, epi=nc.EPI_AXPBY_BF16, aux=dev_bf16(Aux), stride_aux=M * N,
+            alpha=-0.5, beta=1.5)
+    D2 = t.empty(bt, M, N, dtype=t.float32, device="cuda")
+    nc.gemm(M, N, K, dev_bf16(A), dev_bf16(B), D2, batch=bt, stride_a=M * K, stride_b=N * K,
+            stride_d=M * N, epi=nc.EPI_RESID_F32, aux=dev_f32(R), stride_aux=M * N)
+    t.cuda.synchronize()
+    for i in range(bt):
+        acc = oracle.matmul_nt(A[i], B[i])
+        assert rel_fro(host(D[i]), -0.5 * acc + 1.5 * Aux[i]) < 5e-3
+        assert rel_fro(host(D2[i]), R[i] + acc) < 2e-5
 
 
 @pytest.mark.parametrize("split", [1, 3, 7])
