@@ -42,7 +42,10 @@ constexpr int OFF_K = OFF_Q + TILE;    // 2 stages
 constexpr int OFF_V = OFF_K + 2 * KT;  // 2 stages
 constexpr int OFF_P = OFF_V + 2 * KT;
 constexpr int OFF_BAR = OFF_P + PTF;
-constexpr int kSmem = OFF_BAR + 256 + 1024;  // 112 KB + barriers: two CTAs per SM
+// 112 KB + barriers, with no alignment slack: two CTAs and their 1 KB
+// system reservations fit the SM's 228 KB only this way.  The dynamic window
+// starts 1024-byte aligned; the kernel checks that before using it.
+constexpr int kSmem = OFF_BAR + 256;
 constexpr uint32_t TM_S0 = 0, TM_O = 128, kFwdTmemCols = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.f;  // log2 units
@@ -89,9 +92,12 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 __global__ void __launch_bounds__(kThreads, 2)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const FwdArgs a) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if ((tc::smem_u32(smem_raw) & 1023u) != 0) {  // never expected; no room to realign
+    if (threadIdx.x == 0 && a.status) atomicExch(a.status, kDevTimeout);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;   // [2]
@@ -283,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           const float p1 = (i & 3) == 3 ? ex2_fma(x1) : ex2(x1);
           ls0 += p0;
           ls1 += p1;
-          pk[c * 16 + i] = pack_bf16x2(p0, p1);
+          pk[c * 16 + i] = pack_bf16x2_alu(p0, p1);
         }
       l += ls0 + ls1;
       // The P tile and the O accumulator are free once the previous P V landed.
@@ -618,8 +624,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         const float d0 = p0 * (__uint_as_float(dp[2 * c]) - ld[BQB + 2 * c]);
         const float d1 = p1 * (__uint_as_float(dp[2 * c + 1]) - ld[BQB + 2 * c + 1]);
-        pp[c] = pack_bf16x2(p0, p1);
-        pd[c] = pack_bf16x2(d0, d1);
+        pp[c] = pack_bf16x2_alu(p0, p1);
+        pd[c] = pack_bf16x2_alu(d0, d1);
       }
       ok = tc::mbar_wait(pds_empty, (t & 1) ^ 1, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
