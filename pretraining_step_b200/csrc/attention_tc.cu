@@ -1,22 +1,30 @@
-// attention_tc.cu -- causal attention forward on the tcgen05 tensor cores.
+// attention_tc.cu -- causal attention forward and backward on the tcgen05
+// tensor cores.
 //
-// One CTA per (128-query tile, head, batch row), heaviest tiles first.
-// 192 threads in three roles:
-//   warp 0      TMA: the Q tile once, then K and V tiles of 128 keys through
-//               two-stage rings (128-byte swizzle, zero fill past T);
-//   warp 1      TMEM owner and single-thread MMA issue:
-//                 S_j = Q K_j^T  -> TMEM S[j % 2]   (M 128, N 128, K 128)
-//                 O  += P_j V_j  -> TMEM O          (P from shared memory,
-//                                                    V read MN-major)
-//               S_{j+1} is issued before O += P_j V_j, so the tensor pipe
-//               computes the next scores while the softmax warps work;
-//   warps 2..5  softmax: each thread owns one query row.  It reads its row of
-//               S from TMEM, applies scale and causal mask, and writes
-//               P = exp2(S - m) as bf16 into a K-major shared tile.  The row
-//               maximum m is raised only when the block maximum exceeds it by
-//               more than 2^8 (the factor then rescales the O row in TMEM);
-//               otherwise the stale maximum is kept and P stays below 2^8.
+// Forward: one CTA per (128-query tile, head, batch row), heaviest tiles
+// first, two CTAs per SM.  192 threads in three roles:
+//   warp 0      TMA: the Q tile once, then K and V tiles of 128 keys
+//               (128-byte swizzle, zero fill past T), one buffer each;
+//   warp 1      TMEM owner and single-thread MMA issue, per key tile j:
+//                 S  = Q K_j^T  -> TMEM [0, 128)     (M 128, N 128, K 128)
+//                 O += P_j V_j  -> TMEM [128, 256)   (A = P_j from TMEM,
+//                                                     V read MN-major)
+//               All operands keep N = 128: with A and B both in shared
+//               memory a 64-wide N is bound by shared-memory bandwidth;
+//               P never touches shared memory at all;
+//   warps 2..5  softmax: each thread owns one query row.  A first pass over
+//               its row of S in TMEM takes the block maximum; a second
+//               applies scale and causal mask and writes P = exp2(S - m) as
+//               bf16 over the scores it has consumed (P chunk c lands in the
+//               columns of score chunk c / 2).  The row maximum m is raised
+//               only when the block maximum exceeds it by more than 2^8 (the
+//               factor then rescales the O row in TMEM); otherwise the stale
+//               maximum is kept and P stays below 2^8.
 //               At the end: O / l to global memory, lse = (m + log2 l) ln 2.
+// The MMAs of a CTA run in issue order, so S_{j+1} (issued after P_j V_j)
+// never overwrites P_j early, and the commit that publishes S_j also
+// guarantees P_{j-1} V_{j-1} has finished with P_{j-1} and with O.  The other
+// CTA on the SM keeps the tensor pipe busy while this one's softmax runs.
 // All mbarrier waits are bounded; a timeout sets the status word and every
 // role drains (in-flight copies and MMAs) before TMEM is released.
 
@@ -31,22 +39,20 @@ namespace {
 
 constexpr int HD = 128;
 constexpr int BQ = 128;
-constexpr int BKV = 128;  // key tile of the backward
-constexpr int FKV = 64;   // key tile of the forward
-constexpr int kThreads = 192;
+constexpr int BKV = 128;  // key tile (forward and backward)
+constexpr int kThreads = 320;  // forward: TMA warp, MMA warp, 8 softmax warps
 constexpr int TILE = 128 * 128 * 2;  // one 128 x 128 bf16 tile: two 64-column swizzled boxes
-constexpr int KT = FKV * 128 * 2;    // forward K / V tile: [64 keys x 128 dims]
-constexpr int PTF = 128 * FKV * 2;   // forward P tile: [128 queries x 64 keys]
 constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + TILE;    // 2 stages
-constexpr int OFF_V = OFF_K + 2 * KT;  // 2 stages
-constexpr int OFF_P = OFF_V + 2 * KT;
-constexpr int OFF_BAR = OFF_P + PTF;
-// 112 KB + barriers, with no alignment slack: two CTAs and their 1 KB
-// system reservations fit the SM's 228 KB only this way.  The dynamic window
-// starts 1024-byte aligned; the kernel checks that before using it.
-constexpr int kSmem = OFF_BAR + 256;
-constexpr uint32_t TM_S0 = 0, TM_O = 128, kFwdTmemCols = 256;
+constexpr int OFF_K = OFF_Q + TILE;
+constexpr int OFF_V = OFF_K + TILE;
+constexpr int OFF_BAR = OFF_V + TILE;
+// 96 KB + barriers: two CTAs and their 1 KB system reservations fit the SM's
+// 228 KB.  The dynamic window starts 1024-byte aligned; the kernel checks
+// that before using it (no slack is reserved to realign).
+constexpr int OFF_X = OFF_BAR + 256;   // [2 tiles][2 halves][128 rows] partial row maxima
+constexpr int OFF_L = OFF_X + 2048;    // [2 halves][128 rows] partial row sums
+constexpr int kSmem = OFF_L + 1024;
+constexpr uint32_t TM_S = 0, TM_O = 128, kFwdTmemCols = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.f;  // log2 units
 
@@ -100,36 +106,36 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint8_t* smem = smem_raw;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;   // [2]
-  uint64_t* k_empty = bars + 3;  // [2]
-  uint64_t* v_full = bars + 5;   // [2]
-  uint64_t* v_empty = bars + 7;  // [2]
-  uint64_t* s_full = bars + 9;   // [2]
-  uint64_t* s_empty = bars + 11; // [2]
-  uint64_t* p_full = bars + 13;
-  uint64_t* pv_done = bars + 14;
-  uint64_t* drained = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = bars + 2;
+  uint64_t* v_full = bars + 3;
+  uint64_t* v_empty = bars + 4;
+  uint64_t* s_full = bars + 5;
+  uint64_t* p_full = bars + 6;
+  uint64_t* o_full = bars + 7;
+  uint64_t* drained = bars + 8;
+  uint64_t* mx_ready = bars + 9;
+  uint64_t* l_ready = bars + 10;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qb = a.nqb - 1 - (int)blockIdx.x;
   const int h = blockIdx.y, b = blockIdx.z;
-  const int n = min((qb + 1) * BQ, a.T + FKV - 1) / FKV;  // causal: key tiles up to the diagonal
+  const int n = qb + 1;  // causal: key tiles up to the diagonal (BKV == BQ)
 
   if (threadIdx.x == 0) {
     tc::mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&k_full[i], 1);
-      tc::mbar_init(&k_empty[i], 1);
-      tc::mbar_init(&v_full[i], 1);
-      tc::mbar_init(&v_empty[i], 1);
-      tc::mbar_init(&s_full[i], 1);
-      tc::mbar_init(&s_empty[i], 128);
-    }
-    tc::mbar_init(p_full, 128);
-    tc::mbar_init(pv_done, 1);
+    tc::mbar_init(k_full, 1);
+    tc::mbar_init(k_empty, 1);
+    tc::mbar_init(v_full, 1);
+    tc::mbar_init(v_empty, 1);
+    tc::mbar_init(s_full, 1);
+    tc::mbar_init(p_full, 256);
+    tc::mbar_init(o_full, 1);
     tc::mbar_init(drained, 1);
+    tc::mbar_init(mx_ready, 256);
+    tc::mbar_init(l_ready, 256);
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
@@ -154,120 +160,117 @@ __global__ void __launch_bounds__(kThreads, 2)
       int issued_k = 0, issued_v = 0;
       bool ok = true;
       for (int j = 0; j < n && ok; ++j) {
-        const int s = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!tc::mbar_wait(&k_empty[s], ph ^ 1, abort_flag, a.status)) { ok = false; break; }
-        tc::mbar_arrive_expect_tx(&k_full[s], KT);
-        tc::tma_load_3d(smem + OFF_K + s * KT, &tk, &k_full[s], col0, j * FKV, b);
-        tc::tma_load_3d(smem + OFF_K + s * KT + KT / 2, &tk, &k_full[s], col0 + 64, j * FKV, b);
+        const uint32_t ph = j & 1;
+        if (!tc::mbar_wait(k_empty, ph ^ 1, abort_flag, a.status)) { ok = false; break; }
+        tc::mbar_arrive_expect_tx(k_full, TILE);
+        tc::tma_load_3d(smem + OFF_K, &tk, k_full, col0, j * BKV, b);
+        tc::tma_load_3d(smem + OFF_K + TILE / 2, &tk, k_full, col0 + 64, j * BKV, b);
         ++issued_k;
-        if (!tc::mbar_wait(&v_empty[s], ph ^ 1, abort_flag, a.status)) { ok = false; break; }
-        tc::mbar_arrive_expect_tx(&v_full[s], KT);
-        tc::tma_load_3d(smem + OFF_V + s * KT, &tv, &v_full[s], col0, j * FKV, b);
-        tc::tma_load_3d(smem + OFF_V + s * KT + KT / 2, &tv, &v_full[s], col0 + 64, j * FKV, b);
+        if (!tc::mbar_wait(v_empty, ph ^ 1, abort_flag, a.status)) { ok = false; break; }
+        tc::mbar_arrive_expect_tx(v_full, TILE);
+        tc::tma_load_3d(smem + OFF_V, &tv, v_full, col0, j * BKV, b);
+        tc::tma_load_3d(smem + OFF_V + TILE / 2, &tv, v_full, col0 + 64, j * BKV, b);
         ++issued_v;
       }
       if (!ok) {
         // Let in-flight copies land before the CTA can exit.
         drain_wait(q_full, 0);
-        for (int j = max(0, issued_k - 2); j < issued_k; ++j) drain_wait(&k_full[j & 1], (j >> 1) & 1);
-        for (int j = max(0, issued_v - 2); j < issued_v; ++j) drain_wait(&v_full[j & 1], (j >> 1) & 1);
+        if (issued_k > 0) drain_wait(k_full, (issued_k - 1) & 1);
+        if (issued_v > 0) drain_wait(v_full, (issued_v - 1) & 1);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t id_s = tc::idesc_bf16_f32(128, FKV, 0, 0);
-      const uint32_t id_pv = tc::idesc_bf16_f32(128, 128, 0, 1);
+      const uint32_t id_s = tc::idesc_bf16_f32(128, BKV, 0, 0);
+      const uint32_t id_pv = tc::idesc_bf16_f32(128, HD, 0, 1);
       // Descriptors are built once; each MMA adds a constant byte offset.
-      const uint64_t qdesc0 = tc::smem_desc_sw128(tc::smem_u32(smem + OFF_Q), 16, 1024);
-      const uint64_t kdesc0 = tc::smem_desc_sw128(tc::smem_u32(smem + OFF_K), 16, 1024);
-      const uint64_t vdesc0 = tc::smem_desc_sw128(tc::smem_u32(smem + OFF_V), KT / 2, 1024);
-      const uint64_t pdesc0 = tc::smem_desc_sw128(tc::smem_u32(smem + OFF_P), 16, 1024);
+      const uint64_t qdesc = tc::smem_desc_sw128(tc::smem_u32(smem + OFF_Q), 16, 1024);
+      const uint64_t kdesc = tc::smem_desc_sw128(tc::smem_u32(smem + OFF_K), 16, 1024);
+      const uint64_t vdesc = tc::smem_desc_sw128(tc::smem_u32(smem + OFF_V), TILE / 2, 1024);
       bool ok = tc::mbar_wait(q_full, 0, abort_flag, a.status);
-      for (int j = 0; j <= n && ok; ++j) {
-        if (j < n) {
-          const int s = j & 1;
-          const uint32_t ph = (j >> 1) & 1;
-          if (!tc::mbar_wait(&k_full[s], ph, abort_flag, a.status) ||
-              !tc::mbar_wait(&s_empty[s], ph ^ 1, abort_flag, a.status)) {
-            ok = false;
-            break;
-          }
-          tc::tc_fence_after();
-          const uint64_t kd = kdesc0 + (uint64_t)((s * KT) >> 4);
+      for (int j = 0; j < n && ok; ++j) {
+        const uint32_t ph = j & 1;
+        if (!tc::mbar_wait(k_full, ph, abort_flag, a.status)) { ok = false; break; }
+        tc::tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk)
-            tc::umma_bf16_ss(tmem + TM_S0 + s * FKV,
-                             tc::desc_add(qdesc0, (kk >> 2) * (TILE / 2) + (kk & 3) * 32),
-                             tc::desc_add(kd, (kk >> 2) * (KT / 2) + (kk & 3) * 32), id_s,
-                             kk > 0 ? 1u : 0u);
-          tc::umma_commit(&s_full[s]);
-          tc::umma_commit(&k_empty[s]);
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (TILE / 2) + (kk & 3) * 32;
+          tc::umma_bf16_ss(tmem + TM_S, tc::desc_add(qdesc, off), tc::desc_add(kdesc, off), id_s,
+                           kk > 0 ? 1u : 0u);
         }
-        if (j >= 1) {
-          const int jj = j - 1;
-          const int s = jj & 1;
-          const uint32_t ph = (jj >> 1) & 1;
-          if (!tc::mbar_wait(&v_full[s], ph, abort_flag, a.status) ||
-              !tc::mbar_wait(p_full, jj & 1, abort_flag, a.status)) {
-            ok = false;
-            break;
-          }
-          tc::tc_fence_after();
-          const uint64_t vd = vdesc0 + (uint64_t)((s * KT) >> 4);
+        tc::umma_commit(s_full);
+        tc::umma_commit(k_empty);
+        if (!tc::mbar_wait(p_full, ph, abort_flag, a.status) ||
+            !tc::mbar_wait(v_full, ph, abort_flag, a.status)) {
+          ok = false;
+          break;
+        }
+        tc::tc_fence_after();
+        // P_j is bf16 in TMEM: keys [64 h, 64 h + 64) in columns [64 h, 64 h + 32)
+        // (over the scores of the softmax half that owns them); key step kk
+        // (16 keys) is 8 columns.
 #pragma unroll
-          for (int kk = 0; kk < FKV / 16; ++kk)
-            tc::umma_bf16_ss(tmem + TM_O, tc::desc_add(pdesc0, kk * 32), tc::desc_add(vd, kk * 2048),
-                             id_pv, (jj > 0 || kk > 0) ? 1u : 0u);
-          tc::umma_commit(pv_done);
-          tc::umma_commit(&v_empty[s]);
-        }
+        for (int kk = 0; kk < BKV / 16; ++kk)
+          tc::umma_bf16_ts(tmem + TM_O, tmem + TM_S + (kk >> 2) * 64 + (kk & 3) * 8,
+                           tc::desc_add(vdesc, kk * 2048), id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        tc::umma_commit(v_empty);
       }
+      if (ok) tc::umma_commit(o_full);
       tc::umma_commit(drained);
       drain_wait(drained, 0);
     }
   } else {
+    // Two threads per query row: warps 2..5 take keys [0, 64) of every tile,
+    // warps 6..9 keys [64, 128) (a warp may only reach the TMEM lanes of
+    // quarter warp % 4, which both warps of a pair share).
     const int qw = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row = qw * 32 + lane;
     const int qi = qb * BQ + row;
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
-    const uint32_t p_row = tc::smem_u32(smem + OFF_P) + row * 128;
+    const uint32_t s_base = lane_base + TM_S + half * 64;
+    const uint32_t o_base = lane_base + TM_O + half * 64;
+    float* xm = reinterpret_cast<float*>(smem + OFF_X);
+    float* lsum = reinterpret_cast<float*>(smem + OFF_L);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
-      const int s = j & 1;
-      const uint32_t ph = (j >> 1) & 1;
-      ok = tc::mbar_wait(&s_full[s], ph, abort_flag, a.status);
+      ok = tc::mbar_wait(s_full, j & 1, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc::tc_fence_after();
+      const int k0 = j * BKV + half * 64;
+      const bool edge = j * BKV + BKV > qb * BQ || j * BKV + BKV > a.T;  // reaches the diagonal or T
+      // This half's 64 scores, read once; masked ones become -inf.
       uint32_t r[2][32];
-#pragma unroll
-      for (int c = 0; c < 2; ++c) tc::tmem_ld_32x32b_x32(lane_base + TM_S0 + s * FKV + c * 32, r[c]);
+      tc::tmem_ld_32x32b_x32(s_base, r[0]);
+      tc::tmem_ld_32x32b_x32(s_base + 32, r[1]);
       tc::tmem_ld_wait();
-      tc::tc_fence_before();
-      tc::mbar_arrive(&s_empty[s]);
-      // Block maximum on raw scores (the scale is positive); masking only on
-      // tiles that reach the diagonal or the end of the row.
-      const int k0 = j * FKV;
-      float mx_raw = -INFINITY;
-      if (k0 + FKV > qb * BQ || k0 + FKV > a.T) {
+      if (edge) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
+        for (int c2 = 0; c2 < 2; ++c2)
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const int kj = k0 + c * 32 + i;
-            float x = __uint_as_float(r[c][i]);
-            if (kj > qi || kj >= a.T) x = -INFINITY;
-            r[c][i] = __float_as_uint(x);
-            mx_raw = fmaxf(mx_raw, x);
+            const int kj = k0 + c2 * 32 + i;
+            if (kj > qi || kj >= a.T) r[c2][i] = __float_as_uint(-INFINITY);
           }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; ++i) mx_raw = fmaxf(mx_raw, __uint_as_float(r[c][i]));
       }
-      const float mx = mx_raw * a.sl2;
+      // Block maximum of the raw scores (the scale is positive): eight
+      // independent chains here, then the two halves of the row combined
+      // through shared memory.
+      float pm[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) pm[u] = -INFINITY;
+#pragma unroll
+      for (int c2 = 0; c2 < 2; ++c2)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) pm[i & 7] = fmaxf(pm[i & 7], __uint_as_float(r[c2][i]));
+      float* xmj = xm + (j & 1) * 256;
+      xmj[half * 128 + row] = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                    fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+      tc::mbar_arrive(mx_ready);
+      ok = tc::mbar_wait(mx_ready, j & 1, abort_flag, a.status);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      const float mx = fmaxf(xmj[row], xmj[128 + row]) * a.sl2;
       float alpha = 1.f;
       if (mx > m_used + kRescaleThreshold) {
         alpha = ex2(m_used - mx);  // 0 on the first tile
@@ -275,63 +278,58 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       const float neg_mu = (m_used == -INFINITY) ? 0.f : -m_used;
       l *= alpha;
-      // p = 2^(s * scale * log2 e - m): one FFMA feeding ex2 per score.
-      uint32_t pk[32];
-      float ls0 = 0.f, ls1 = 0.f;
+      // p = 2^(s * scale * log2 e - m), one FFMA feeding ex2 per score; P
+      // chunk c2 (32 keys, 16 packed columns) over this half's first scores.
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 2; ++c)
+      for (int c2 = 0; c2 < 2; ++c2) {
+        uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float x0 = fmaf(__uint_as_float(r[c][2 * i]), a.sl2, neg_mu);
-          const float x1 = fmaf(__uint_as_float(r[c][2 * i + 1]), a.sl2, neg_mu);
-          // every fourth pair on the FMA pipe, the rest on MUFU
-          const float p0 = (i & 3) == 3 ? ex2_fma(x0) : ex2(x0);
-          const float p1 = (i & 3) == 3 ? ex2_fma(x1) : ex2(x1);
-          ls0 += p0;
-          ls1 += p1;
-          pk[c * 16 + i] = pack_bf16x2_alu(p0, p1);
+          const float p0 = ex2(fmaf(__uint_as_float(r[c2][2 * i]), a.sl2, neg_mu));
+          const float p1 = ex2(fmaf(__uint_as_float(r[c2][2 * i + 1]), a.sl2, neg_mu));
+          ls[(2 * i) & 3] += p0;
+          ls[(2 * i + 1) & 3] += p1;
+          pk[i] = pack_bf16x2(p0, p1);
         }
-      l += ls0 + ls1;
-      // The P tile and the O accumulator are free once the previous P V landed.
-      if (j >= 1) {
-        ok = tc::mbar_wait(pv_done, (j - 1) & 1, abort_flag, a.status);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        tc::tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        tc::tmem_st_32x32b_x16(s_base + c2 * 16, pk);
+      }
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      // O is idle here: the commit that published S_j also covers P_{j-1} V_{j-1}.
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tc::tmem_ld_32x32b_x32(lane_base + TM_O + c * 32, o);
-            tc::tmem_ld_wait();
+        for (int c = 0; c < 2; ++c) {
+          uint32_t o[32];
+          tc::tmem_ld_32x32b_x32(o_base + c * 32, o);
+          tc::tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tc::tmem_st_32x32b_x32(lane_base + TM_O + c * 32, o);
-          }
-          tc::tmem_st_wait();
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tc::tmem_st_32x32b_x32(o_base + c * 32, o);
         }
       }
-      // P row -> K-major swizzled tile: 16-byte unit u of key chunk ch sits at
-      // row*128 + ((u ^ (row & 7)) * 16) inside the chunk.
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        tc::st_shared_v4(p_row + ((u ^ (row & 7)) << 4), pk[4 * u], pk[4 * u + 1], pk[4 * u + 2],
-                         pk[4 * u + 3]);
-      tc::fence_proxy_async_smem();
+      tc::tmem_st_wait();
       tc::tc_fence_before();
       tc::mbar_arrive(p_full);
     }
     if (ok) {
-      ok = tc::mbar_wait(pv_done, (n - 1) & 1, abort_flag, a.status);
+      ok = tc::mbar_wait(o_full, 0, abort_flag, a.status);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {  // the row sum is split over the two halves
+      lsum[half * 128 + row] = l;
+      tc::mbar_arrive(l_ready);
+      ok = tc::mbar_wait(l_ready, 0, abort_flag, a.status);
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
       tc::tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* orow = a.o + ((int64_t)b * a.T + qi) * a.ldo + col0;
+      const float lt = lsum[row] + lsum[128 + row];
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      __nv_bfloat16* orow = a.o + ((int64_t)b * a.T + qi) * a.ldo + col0 + half * 64;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t o[32];
-        tc::tmem_ld_32x32b_x32(lane_base + TM_O + c * 32, o);
+        tc::tmem_ld_32x32b_x32(o_base + c * 32, o);
         tc::tmem_ld_wait();
         if (qi < a.T) {
 #pragma unroll
@@ -345,8 +343,8 @@ __global__ void __launch_bounds__(kThreads, 2)
           }
         }
       }
-      if (qi < a.T)
-        a.lse[((int64_t)b * a.H + h) * a.T + qi] = (m_used + log2f(l)) * 0.69314718055994531f;
+      if (half == 0 && qi < a.T)
+        a.lse[((int64_t)b * a.H + h) * a.T + qi] = (m_used + log2f(lt)) * 0.69314718055994531f;
     }
   }
   tc::tc_fence_before();
@@ -733,8 +731,8 @@ nc_status attention_fwd(const void* q, const void* k, const void* v, int64_t ld,
   const uint64_t cols = (uint64_t)H * HD;
   // Box heights must match the tile sizes the kernel's byte counts assume.
   if (!make_tmap_bf16_3d(&mq, q, cols, T, B, ld, (int64_t)T * ld, BQ) ||
-      !make_tmap_bf16_3d(&mk, k, cols, T, B, ld, (int64_t)T * ld, FKV) ||
-      !make_tmap_bf16_3d(&mv, v, cols, T, B, ld, (int64_t)T * ld, FKV))
+      !make_tmap_bf16_3d(&mk, k, cols, T, B, ld, (int64_t)T * ld, BKV) ||
+      !make_tmap_bf16_3d(&mv, v, cols, T, B, ld, (int64_t)T * ld, BKV))
     return fail(NC_ERR_INVALID_ARG, "attention_fwd: cuTensorMapEncodeTiled rejected q/k/v");
   FwdArgs a;
   a.T = T;
