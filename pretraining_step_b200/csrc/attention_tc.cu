@@ -2,7 +2,7 @@
 // tensor cores.
 //
 // Forward: one CTA per (128-query tile, head, batch row), heaviest tiles
-// first, two CTAs per SM.  192 threads in three roles:
+// first, two CTAs per SM.  320 threads in three roles:
 //   warp 0      TMA: the Q tile once, then K and V tiles of 128 keys
 //               (128-byte swizzle, zero fill past T), one buffer each;
 //   warp 1      TMEM owner and single-thread MMA issue, per key tile j:
@@ -12,15 +12,16 @@
 //               All operands keep N = 128: with A and B both in shared
 //               memory a 64-wide N is bound by shared-memory bandwidth;
 //               P never touches shared memory at all;
-//   warps 2..5  softmax: each thread owns one query row.  A first pass over
-//               its row of S in TMEM takes the block maximum; a second
-//               applies scale and causal mask and writes P = exp2(S - m) as
-//               bf16 over the scores it has consumed (P chunk c lands in the
-//               columns of score chunk c / 2).  The row maximum m is raised
-//               only when the block maximum exceeds it by more than 2^8 (the
-//               factor then rescales the O row in TMEM); otherwise the stale
-//               maximum is kept and P stays below 2^8.
-//               At the end: O / l to global memory, lse = (m + log2 l) ln 2.
+//   warps 2..9  softmax, two threads per query row (warps 2..5 keys
+//               [0, 64) of each tile, warps 6..9 keys [64, 128)).  Each
+//               reads its 64 scores once, the pair agrees on the block
+//               maximum through shared memory, and each writes its
+//               P = exp2(S - m) as bf16 over its own first scores.  The row
+//               maximum m is raised only when the block maximum exceeds it
+//               by more than 2^8 (the factor then rescales the O row in
+//               TMEM); otherwise the stale maximum is kept and P stays below
+//               2^8.  At the end: O / l to global memory,
+//               lse = (m + log2 l) ln 2.
 // The MMAs of a CTA run in issue order, so S_{j+1} (issued after P_j V_j)
 // never overwrites P_j early, and the commit that publishes S_j also
 // guarantees P_{j-1} V_{j-1} has finished with P_{j-1} and with O.  The other
@@ -72,21 +73,6 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// 2^x on the FMA pipe, for a share of the softmax exponentials so the MUFU
-// unit is not the only limit: 2^x = 2^floor(x) * p(x - floor(x)) with a cubic
-// p fitted here for relative error on [0, 1) with p(0) = 1 (max relative
-// error 8.6e-5, far below the bf16 rounding P receives).  Exactly 0 below
-// 2^-126, including for masked scores (x = -inf).
-__device__ __forceinline__ float ex2_fma(float x) {
-  constexpr float c1 = 0.69511570925694f, c2 = 0.22764980831700f, c3 = 0.07706263250999f;
-  const float xc = fmaxf(x, -126.f);
-  const float j = floorf(xc);
-  const float f = xc - j;
-  const float p = fmaf(fmaf(fmaf(c3, f, c2), f, c1), f, 1.f);
-  const float r = __int_as_float(__float_as_int(p) + ((int)j << 23));
-  return x < -126.f ? 0.f : r;
 }
 
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
@@ -622,8 +608,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         const float d0 = p0 * (__uint_as_float(dp[2 * c]) - ld[BQB + 2 * c]);
         const float d1 = p1 * (__uint_as_float(dp[2 * c + 1]) - ld[BQB + 2 * c + 1]);
-        pp[c] = pack_bf16x2_alu(p0, p1);
-        pd[c] = pack_bf16x2_alu(d0, d1);
+        pp[c] = pack_bf16x2(p0, p1);
+        pd[c] = pack_bf16x2(d0, d1);
       }
       ok = tc::mbar_wait(pds_empty, (t & 1) ^ 1, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }

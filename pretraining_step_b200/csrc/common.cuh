@@ -42,14 +42,6 @@ __device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
   return __bfloat1622float2(h);
 }
 
-// Two finite floats -> bf16x2 on the integer pipe: add half an ulp of bf16 to
-// the bit pattern (ties round away from zero, the only difference from
-// round-to-nearest-even), then keep the two high halves.  Keeps the
-// conversion unit free where it also serves the exponentials.
-__device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi) {
-  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
-}
-
 // Square root by the PTX approximate instruction (relative error about
 // 2^-23, sqrt(0) = 0): one instruction where sqrtf's IEEE rounding takes a
 // branchy sequence.  Used where the result is rounded to bf16 anyway.

@@ -210,9 +210,18 @@ __device__ __forceinline__ void store_row_chunk(const Args& p, int b, int row, i
     }
     case NC_EPI_ACC_F32: {
       float* D = (float*)p.D + off;
+      if (nvalid == 32) {  // 16-byte vector reductions (rows are 32-byte aligned)
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (j < nvalid) atomicAdd(D + j, v[j] * p.alpha);
+        for (int j = 0; j < 8; ++j)
+          asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(D + 4 * j),
+                       "f"(v[4 * j] * p.alpha), "f"(v[4 * j + 1] * p.alpha), "f"(v[4 * j + 2] * p.alpha),
+                       "f"(v[4 * j + 3] * p.alpha)
+                       : "memory");
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < nvalid) atomicAdd(D + j, v[j] * p.alpha);
+      }
       break;
     }
     default:
