@@ -223,7 +223,9 @@ nc_status nc_op_attention_fwd(const void* q, const void* k, const void* v, int64
 
 /* Causal attention backward: from dO (bf16, stride ldo) and the forward's
  * O, lse: dq (f32, [B,T,H,128] dense, OVERWRITTEN), dk, dv (bf16, stride
- * ldg).  delta_scratch: f32 [B, H, T] workspace. */
+ * ldg).  delta_scratch: f32 [B, H, T] workspace.  Every operand row must be
+ * 16-byte aligned (strides multiples of 8 elements) and H <= 16; otherwise
+ * NC_ERR_INVALID_ARG / NC_ERR_UNSUPPORTED before anything is launched. */
 nc_status nc_op_attention_bwd(const void* q, const void* k, const void* v, int64_t ld,
                               const void* o, const void* dout, int64_t ldo, const float* lse,
                               float* dq, void* dk, void* dv, int64_t ldg, float* delta_scratch,

@@ -15,24 +15,66 @@ namespace {
 constexpr int HD = 128;
 
 // D[b, h, t] = sum_i dO[b, t, h, i] * O[b, t, h, i]; one warp per (token, head).
-__global__ void attn_bwd_delta_kernel(const __nv_bfloat16* __restrict__ o,
-                                      const __nv_bfloat16* __restrict__ dout, int64_t ldo,
-                                      float* __restrict__ delta, int B, int T, int H) {
-  const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (w >= (int64_t)B * T * H) return;
-  const int h = (int)(w % H);
-  const int64_t tok = w / H;
-  const int64_t off = tok * ldo + (int64_t)h * HD + lane * 4;
-  const uint2 x = *reinterpret_cast<const uint2*>(o + off);
-  const uint2 y = *reinterpret_cast<const uint2*>(dout + off);
-  const float2 x0 = unpack_bf16x2(x.x), x1 = unpack_bf16x2(x.y);
-  const float2 y0 = unpack_bf16x2(y.x), y1 = unpack_bf16x2(y.y);
-  float s = x0.x * y0.x + x0.y * y0.y + x1.x * y1.x + x1.y * y1.y;
-  s = warp_sum(s);
-  if (lane == 0) {
-    const int64_t bb = tok / T, t = tok % T;
-    delta[(bb * H + h) * T + t] = s;
+// D[b, h, t] = sum_d dO[t, h, d] O[t, h, d].  A warp takes one token (all
+// heads): every lane's 16-byte loads of both rows are issued before any
+// arithmetic, so a warp keeps 2 * H * 256 bytes in flight; half-warps hold
+// one head per step.  The block's 32 tokens go through shared memory so the
+// [B, H, T] writes are 128-byte runs along t.
+constexpr int kDeltaTok = 32;     // tokens per block (8 warps x 4)
+constexpr int kDeltaMaxH = 16;    // heads per token handled here
+__global__ void __launch_bounds__(256) attn_bwd_delta_kernel(const __nv_bfloat16* __restrict__ o,
+                                                           const __nv_bfloat16* __restrict__ dout,
+                                                           int64_t ldo, float* __restrict__ delta,
+                                                           int B, int T, int H) {
+  __shared__ float red[kDeltaMaxH][kDeltaTok];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t ntok = (int64_t)B * T;
+  const int64_t tok0 = (int64_t)blockIdx.x * kDeltaTok;
+  const int units = H * (HD / 8);  // 16-byte units per row
+  for (int k = 0; k < kDeltaTok / 8; ++k) {
+    const int lt = warp * (kDeltaTok / 8) + k;
+    const int64_t tok = tok0 + lt;
+    if (tok >= ntok) break;
+    const __nv_bfloat16* orow = o + tok * ldo;
+    const __nv_bfloat16* drow = dout + tok * ldo;
+    uint4 xs[kDeltaMaxH / 2], ys[kDeltaMaxH / 2];
+#pragma unroll
+    for (int i = 0; i < kDeltaMaxH / 2; ++i) {
+      const int u = lane + 32 * i;
+      if (u < units) {
+        xs[i] = reinterpret_cast<const uint4*>(orow)[u];
+        ys[i] = reinterpret_cast<const uint4*>(drow)[u];
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kDeltaMaxH / 2; ++i) {
+      const int u = lane + 32 * i;
+      float sum = 0.f;
+      if (u < units) {
+        const uint32_t* xa = reinterpret_cast<const uint32_t*>(&xs[i]);
+        const uint32_t* ya = reinterpret_cast<const uint32_t*>(&ys[i]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 xv = unpack_bf16x2(xa[e]), yv = unpack_bf16x2(ya[e]);
+          sum = fmaf(xv.x, yv.x, fmaf(xv.y, yv.y, sum));
+        }
+      }
+      // lanes [0, 16) hold head 2 i, lanes [16, 32) head 2 i + 1
+#pragma unroll
+      for (int sh = 8; sh > 0; sh >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, sh);
+      const int hh = 2 * i + (lane >> 4);
+      if ((lane & 15) == 0 && hh < H) red[hh][lt] = sum;
+    }
+  }
+  __syncthreads();
+  // Write [B, H, T]: thread (h, t) for the block's tokens.
+  for (int idx = threadIdx.x; idx < H * kDeltaTok; idx += blockDim.x) {
+    const int hh = idx / kDeltaTok, lt = idx % kDeltaTok;
+    const int64_t tok = tok0 + lt;
+    if (tok < ntok) {
+      const int64_t bb = tok / T, t = tok % T;
+      delta[(bb * H + hh) * T + t] = red[hh][lt];
+    }
   }
 }
 
@@ -47,10 +89,13 @@ nc_status attention_bwd(const void* q, const void* k, const void* v, int64_t ld,
     return fail(NC_ERR_INVALID_ARG, "attention_bwd: bad arguments");
   if (ld % 8 || ldo % 8 || ldg % 8)
     return fail(NC_ERR_INVALID_ARG, "attention_bwd: strides must be multiples of 8");
+  if (H > kDeltaMaxH) return fail(NC_ERR_UNSUPPORTED, "attention_bwd: at most 16 heads");
+  if ((reinterpret_cast<uintptr_t>(o) | reinterpret_cast<uintptr_t>(dout)) & 15)
+    return fail(NC_ERR_INVALID_ARG, "attention_bwd: O and dO rows must be 16-byte aligned");
   const int64_t rows = (int64_t)B * T * H;
   {
     Probe probe(prof, s, "attn_bwd_delta", 0.0, rows * HD * 2.0 * 2 + rows * 4.0);
-    attn_bwd_delta_kernel<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, s>>>(
+    attn_bwd_delta_kernel<<<(unsigned)(((int64_t)B * T + kDeltaTok - 1) / kDeltaTok), 256, 0, s>>>(
         (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, ldo, delta, B, T, H);
     NC_CUDA_TRY(cudaGetLastError());
   }
