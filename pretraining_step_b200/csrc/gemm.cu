@@ -39,7 +39,9 @@ struct Cfg {
   static constexpr int STAGES = (BN == 256) ? 4 : 6;
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+  static constexpr int X_WARP_BYTES = 4096;  // per epilogue warp: one staging slot (RoPE epilogue)
+  static constexpr int X_BYTES = (kEpiThreads / 32) * X_WARP_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + X_BYTES + BAR_BYTES + 1024;
 };
 
 struct Args {
@@ -229,13 +231,81 @@ __device__ __forceinline__ void store_row_chunk(const Args& p, int b, int row, i
   }
 }
 
+// Store one finished 32 x 32 block of a warp (row `lane` in w) through its
+// shared-memory slot: each lane writes its row (fp32: 128-byte rows with the
+// 128-byte swizzle; bf16: 64-byte rows with the 64-byte swizzle), then the
+// warp stores the block row by row (8 lanes per fp32 row, 4 per bf16 row), so
+// each store instruction covers whole lines instead of 16 bytes of 32
+// different lines.  Rows past M and columns past N are skipped.
+__device__ __forceinline__ void stage_store_chunk(const Args& p, uint8_t* slot, int lane, bool f32, int b,
+                                                  int row0, int col0, const float (&w)[32]) {
+  const uint32_t base = tc::smem_u32(slot);
+  if (f32) {
+    const uint32_t rowa = base + lane * 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      tc::st_shared_v4(rowa + ((j ^ (lane & 7)) << 4), __float_as_uint(w[4 * j]), __float_as_uint(w[4 * j + 1]),
+                       __float_as_uint(w[4 * j + 2]), __float_as_uint(w[4 * j + 3]));
+  } else {
+    const uint32_t rowa = base + lane * 64;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      tc::st_shared_v4(rowa + ((j ^ ((lane >> 1) & 3)) << 4), pack_bf16x2(w[8 * j], w[8 * j + 1]),
+                       pack_bf16x2(w[8 * j + 2], w[8 * j + 3]), pack_bf16x2(w[8 * j + 4], w[8 * j + 5]),
+                       pack_bf16x2(w[8 * j + 6], w[8 * j + 7]));
+  }
+  __syncwarp();
+  const int ncol = p.N - col0;  // >= 1
+  if (f32) {
+    float* D = (float*)p.D + (int64_t)b * p.stride_d + col0;
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int rr = it * 4 + (lane >> 3), cc = lane & 7;
+      const uint4 u = tc::ld_shared_v4(base + rr * 128 + ((cc ^ (rr & 7)) << 4));
+      if (row0 + rr < p.M) {
+        float* d = D + (int64_t)(row0 + rr) * p.ldd + cc * 4;
+        if (cc * 4 + 4 <= ncol) {
+          *reinterpret_cast<uint4*>(d) = u;
+        } else {
+          const uint32_t e[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if (cc * 4 + i < ncol) d[i] = __uint_as_float(e[i]);
+        }
+      }
+    }
+  } else {
+    __nv_bfloat16* D = (__nv_bfloat16*)p.D + (int64_t)b * p.stride_d + col0;
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int rr = it * 8 + (lane >> 2), cc = lane & 3;
+      const uint4 u = tc::ld_shared_v4(base + rr * 64 + ((cc ^ ((rr >> 1) & 3)) << 4));
+      if (row0 + rr < p.M) {
+        __nv_bfloat16* d = D + (int64_t)(row0 + rr) * p.ldd + cc * 8;
+        if (cc * 8 + 8 <= ncol) {
+          *reinterpret_cast<uint4*>(d) = u;
+        } else {
+          const uint32_t e[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            if (cc * 8 + i < ncol) {
+              const uint32_t h = (e[i >> 1] >> ((i & 1) * 16)) & 0xffffu;
+              d[i] = __ushort_as_bfloat16((unsigned short)h);
+            }
+        }
+      }
+    }
+  }
+  __syncwarp();  // the slot may be rewritten by the warp's next chunk
+}
+
 // Fused q|k|v epilogue: this warp's 128 accumulator columns are one head.
 // q and k heads are rotated (pairs i, i + 64, position row % T) and
 // RMS-normalised; v heads are stored as computed.  The rotation preserves
 // the norm of every pair, so a first pass over TMEM takes the head's norm
 // and a second rotates, scales and stores column chunks c and c + 2 together.
 __device__ __forceinline__ void rope_head_epilogue(const Args& p, uint32_t taddr, int b, int row,
-                                                   int col0) {
+                                                   int col0, uint8_t* slot, int lane) {
   const bool live = row < p.M && col0 < p.N;
   const int d = p.rope_H * 128;
   const int region = col0 / d;  // 0: q, 1: k, 2: v (uniform across the warp)
@@ -257,7 +327,6 @@ __device__ __forceinline__ void rope_head_epilogue(const Args& p, uint32_t taddr
     if (live) (region ? p.rstd_k : p.rstd_q)[(int64_t)row * p.rope_H + (col0 % d) / 128] = rs;
   }
   (void)b;  // batch 1: stride_d holds T and H here
-  __nv_bfloat16* D = (__nv_bfloat16*)p.D + (int64_t)row * p.ldd + col0;
   const float4* tab = reinterpret_cast<const float4*>(p.rope_tab + (int64_t)(row % p.rope_T) * 64);
 #pragma unroll 1
   for (int cp = 0; cp < 2; ++cp) {
@@ -286,10 +355,8 @@ __device__ __forceinline__ void rope_head_epilogue(const Args& p, uint32_t taddr
         w1[i] = __uint_as_float(hi[i]) * p.alpha;
       }
     }
-    if (live) {
-      store_bf16_chunk(D + cp * 32, 32, w0);
-      store_bf16_chunk(D + (cp + 2) * 32, 32, w1);
-    }
+    stage_store_chunk(p, slot, lane, false, 0, row - lane, col0 + cp * 32, w0);
+    stage_store_chunk(p, slot, lane, false, 0, row - lane, col0 + (cp + 2) * 32, w1);
   }
 }
 
@@ -302,7 +369,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint8_t* stage_slots = smem + C::STAGES * C::STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES + C::X_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* tfull = empty + C::STAGES;
   uint64_t* tempty = tfull + 2;
@@ -456,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool aux = epi_has_aux(p.epi);
       if constexpr (ROPE) {  // separate instantiation: the other GEMMs carry no RoPE code
         rope_head_epilogue(p, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + half * CH * 32, c.b,
-                           row, c.nb * BN + half * CH * 32);
+                           row, c.nb * BN + half * CH * 32, stage_slots + (warp - 2) * C::X_WARP_BYTES, lane);
       } else {
       // The aux chunk is loaded one chunk ahead so its HBM latency overlaps
       // the current chunk's TMEM load, arithmetic and stores.
@@ -515,8 +583,11 @@ struct Cfg2 {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = 6;
   static constexpr int TMEM_COLS = 2 * BN;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 512 + 1024;
+  static constexpr int X_WARP_BYTES = 4096;  // per epilogue warp: one staging slot
+  static constexpr int X_BYTES = (kEpiThreads / 32) * X_WARP_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + X_BYTES + 512 + 1024;
 };
+static_assert(Cfg2::SMEM_BYTES <= 232448, "pair GEMM exceeds shared memory");
 
 // The pair kernel for epilogues that read an aux operand: one operand stage
 // fewer, and each epilogue warp owns an 8 KB ring of aux chunks (its 32 rows
@@ -574,81 +645,26 @@ __device__ __forceinline__ void aux_read_slot(const uint8_t* slot, int lane, boo
 }
 
 // Aux epilogues of the ring kernel: the output has the aux operand's type, so
-// each lane writes its finished row back over its aux row in the slot, and
-// the warp then stores the 32 x 32 block row by row (8 lanes per 128-byte
-// fp32 row, 4 per 64-byte bf16 row): each store instruction covers whole
-// lines instead of 16 bytes of 32 different lines.
+// the finished rows go out through the slot that held the aux rows.
 __device__ __forceinline__ void aux_epilogue_chunk(const Args& p, uint8_t* slot, int lane, bool f32,
                                                    int b, int row0, int col0, const uint32_t (&r)[32]) {
   float x[32];
   aux_read_slot(slot, lane, f32, x);
-  const uint32_t base = tc::smem_u32(slot);
-  if (f32) {  // D = aux + alpha*acc
-    const uint32_t rowa = base + lane * 128;
+  __syncwarp();  // every lane has read its aux row before any is overwritten
+  float w[32];
+  const bool relu2_bwd = p.epi == NC_EPI_RELU2_BWD;
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      tc::st_shared_v4(rowa + ((j ^ (lane & 7)) << 4),
-                       __float_as_uint(x[4 * j] + p.alpha * __uint_as_float(r[4 * j])),
-                       __float_as_uint(x[4 * j + 1] + p.alpha * __uint_as_float(r[4 * j + 1])),
-                       __float_as_uint(x[4 * j + 2] + p.alpha * __uint_as_float(r[4 * j + 2])),
-                       __float_as_uint(x[4 * j + 3] + p.alpha * __uint_as_float(r[4 * j + 3])));
-  } else {
-    float w[32];
-    const bool relu2_bwd = p.epi == NC_EPI_RELU2_BWD;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const float a = __uint_as_float(r[j]) * p.alpha;
-      w[j] = relu2_bwd ? 2.f * sqrt_approx(fmaxf(x[j], 0.f)) * a : a + p.beta * x[j];
-    }
-    const uint32_t rowa = base + lane * 64;
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      tc::st_shared_v4(rowa + ((j ^ ((lane >> 1) & 3)) << 4), pack_bf16x2(w[8 * j], w[8 * j + 1]),
-                       pack_bf16x2(w[8 * j + 2], w[8 * j + 3]), pack_bf16x2(w[8 * j + 4], w[8 * j + 5]),
-                       pack_bf16x2(w[8 * j + 6], w[8 * j + 7]));
+  for (int j = 0; j < 32; ++j) {
+    const float a = __uint_as_float(r[j]) * p.alpha;
+    w[j] = f32 ? x[j] + a : (relu2_bwd ? 2.f * sqrt_approx(fmaxf(x[j], 0.f)) * a : a + p.beta * x[j]);
   }
-  __syncwarp();
-  const int ncol = p.N - col0;  // >= 1
-  if (f32) {
-    float* D = (float*)p.D + (int64_t)b * p.stride_d + col0;
-#pragma unroll
-    for (int it = 0; it < 8; ++it) {
-      const int rr = it * 4 + (lane >> 3), cc = lane & 7;
-      const uint4 u = tc::ld_shared_v4(base + rr * 128 + ((cc ^ (rr & 7)) << 4));
-      if (row0 + rr < p.M) {
-        float* d = D + (int64_t)(row0 + rr) * p.ldd + cc * 4;
-        if (cc * 4 + 4 <= ncol) {
-          *reinterpret_cast<uint4*>(d) = u;
-        } else {
-          const uint32_t e[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            if (cc * 4 + i < ncol) d[i] = __uint_as_float(e[i]);
-        }
-      }
-    }
-  } else {
-    __nv_bfloat16* D = (__nv_bfloat16*)p.D + (int64_t)b * p.stride_d + col0;
-#pragma unroll
-    for (int it = 0; it < 4; ++it) {
-      const int rr = it * 8 + (lane >> 2), cc = lane & 3;
-      const uint4 u = tc::ld_shared_v4(base + rr * 64 + ((cc ^ ((rr >> 1) & 3)) << 4));
-      if (row0 + rr < p.M) {
-        __nv_bfloat16* d = D + (int64_t)(row0 + rr) * p.ldd + cc * 8;
-        if (cc * 8 + 8 <= ncol) {
-          *reinterpret_cast<uint4*>(d) = u;
-        } else {
-          const uint32_t e[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            if (cc * 8 + i < ncol) {
-              const uint32_t h = (e[i >> 1] >> ((i & 1) * 16)) & 0xffffu;
-              d[i] = __ushort_as_bfloat16((unsigned short)h);
-            }
-        }
-      }
-    }
-  }
+  stage_store_chunk(p, slot, lane, f32, b, row0, col0, w);
+}
+
+// Plain epilogues (bf16 / fp32 store, ReLU^2) of the pair kernel through the
+// warp's staging slot; the accumulate and aux forms keep their own path.
+__device__ __forceinline__ bool epi_staged(int epi) {
+  return epi == NC_EPI_STORE_BF16 || epi == NC_EPI_RELU2 || epi == NC_EPI_STORE_F32;
 }
 
 template <bool ROPE, bool XR>
@@ -815,7 +831,7 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
     const int slot_bytes = xf32 ? 4096 : 2048;
     const int slots = XR ? Cfg2X::X_WARP_BYTES / slot_bytes : 1;
     const int slot_shift = slots == 4 ? 2 : 1;
-    uint8_t* ring = xring_all + (warp - 2) * (XR ? Cfg2X::X_WARP_BYTES : 0);
+    uint8_t* ring = xring_all + (warp - 2) * C::X_WARP_BYTES;  // XR: aux ring; else: staging slot
     uint64_t* xfull = xbar + (warp - 2) * Cfg2X::X_MAX_SLOTS;
     int g_use = 0;
     if constexpr (XR) {
@@ -834,7 +850,7 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
       const bool aux = epi_has_aux(p.epi);
       if constexpr (ROPE) {  // separate instantiation: the other GEMMs carry no RoPE code
         rope_head_epilogue(p, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + half * CH * 32, c.b,
-                           row, c.nb * BN + half * CH * 32);
+                           row, c.nb * BN + half * CH * 32, ring, lane);
       } else if constexpr (XR) {
 #pragma unroll
         for (int k = 0; k < CH; ++k) {
@@ -862,6 +878,25 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
           ++g_use;
         }
         if (xabort) break;
+      } else if (epi_staged(p.epi)) {
+        const bool f32 = p.epi == NC_EPI_STORE_F32;
+#pragma unroll
+        for (int k = 0; k < CH; ++k) {
+          const int ch = half * CH + k;
+          uint32_t r[32];
+          tc::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + ch * 32, r);
+          const int col0 = c.nb * BN + ch * 32;
+          tc::tmem_ld_wait();
+          if (col0 < p.N) {
+            float w[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float a = __uint_as_float(r[j]) * p.alpha;
+              w[j] = p.epi == NC_EPI_RELU2 ? fmaxf(a, 0.f) * fmaxf(a, 0.f) : a;
+            }
+            stage_store_chunk(p, ring, lane, f32, c.b, row - lane, col0, w);
+          }
+        }
       } else {
       float xa[32], xb[32];
 #pragma unroll
