@@ -80,12 +80,31 @@ struct TileCoord {
   int b, mb, nb, kb0, kb1;
 };
 
+// Tile order inside one (split, batch) plane.  Column tiles run fastest, so
+// the CTAs running at the same time share A rows.  On planes much wider than
+// the grid (the 32768-wide lm_head) that order sweeps all of B once per row
+// of tiles while the output stream evicts it from L2 (2.7x the algorithmic
+// DRAM bytes); there tiles go in groups of kGroupM row tiles, column tiles
+// outer and row tiles inner, so concurrent CTAs share a few B column tiles
+// and a group's A rows, which stay in L2.
+constexpr int kGroupM = 16;
+constexpr int kGroupMinTilesN = 32;
 __device__ __forceinline__ TileCoord decode(const Args& p, int t) {
   TileCoord c;
-  c.nb = t % p.tiles_n;
-  t /= p.tiles_n;
-  c.mb = t % p.tiles_m;
-  t /= p.tiles_m;
+  const int plane = p.tiles_m * p.tiles_n;
+  const int r = t % plane;
+  t /= plane;
+  if (p.tiles_n > kGroupMinTilesN) {
+    const int gsize = kGroupM * p.tiles_n;
+    const int g = r / gsize;
+    const int gm = min(kGroupM, p.tiles_m - g * kGroupM);  // rows in this (possibly last) group
+    const int in = r - g * gsize;
+    c.mb = g * kGroupM + in % gm;
+    c.nb = in / gm;
+  } else {
+    c.nb = r % p.tiles_n;
+    c.mb = r / p.tiles_n;
+  }
   const int ks = t % p.split_k;
   c.b = t / p.split_k;
   c.kb0 = ks * p.kb_per_split;
