@@ -208,9 +208,10 @@ __global__ void __launch_bounds__(kCeThreads, 2) ce_fwd_bwd_kernel(__nv_bfloat16
 #pragma unroll
   for (int c = 0; c < kCeChunks; ++c) {
     const int idx = threadIdx.x + c * kCeThreads;
+    buf[c] = make_uint4(0u, 0u, 0u, 0u);
     if (idx < nchunk) {
       buf[c] = zr[idx];
-      const uint32_t* u = reinterpret_cast<const uint32_t*>(&buf[c]);
+      const uint32_t u[4] = {buf[c].x, buf[c].y, buf[c].z, buf[c].w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const float2 f = unpack_bf16x2(u[j]);
@@ -229,17 +230,23 @@ __global__ void __launch_bounds__(kCeThreads, 2) ce_fwd_bwd_kernel(__nv_bfloat16
   }
   __syncthreads();
   mx = s_bcast;
+  // e = exp(z - max), summed in fp32 and kept (as bf16) in place of z, so the
+  // gradient pass scales by 1 / sum instead of exponentiating again.
   float se = 0.f;
 #pragma unroll
   for (int c = 0; c < kCeChunks; ++c) {
     const int idx = threadIdx.x + c * kCeThreads;
     if (idx < nchunk) {
-      const uint32_t* u = reinterpret_cast<const uint32_t*>(&buf[c]);
+      const uint32_t u[4] = {buf[c].x, buf[c].y, buf[c].z, buf[c].w};
+      uint32_t e[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const float2 f = unpack_bf16x2(u[j]);
-        se += __expf(f.x - mx) + __expf(f.y - mx);
+        const float e0 = __expf(f.x - mx), e1 = __expf(f.y - mx);
+        se += e0 + e1;
+        e[j] = pack_bf16x2(e0, e1);
       }
+      buf[c] = make_uint4(e[0], e[1], e[2], e[3]);
     }
   }
   se = warp_sum(se);
@@ -249,28 +256,26 @@ __global__ void __launch_bounds__(kCeThreads, 2) ce_fwd_bwd_kernel(__nv_bfloat16
   if (threadIdx.x == 0) {
     float s = 0.f;
     for (int i = 0; i < kCeThreads / 32; ++i) s += red[i];
-    const float lse = mx + logf(s);
-    s_bcast = lse;
-    loss_rows[row] = lse - s_zt;
+    loss_rows[row] = mx + logf(s) - s_zt;
+    s_bcast = 1.f / s;
   }
   __syncthreads();
-  const float lse = s_bcast;
+  const float scale = s_bcast * inv_n;  // softmax = e / sum, then times 1/n
 #pragma unroll
   for (int c = 0; c < kCeChunks; ++c) {
     const int idx = threadIdx.x + c * kCeThreads;
     if (idx < nchunk) {
-      const uint32_t* u = reinterpret_cast<const uint32_t*>(&buf[c]);
-      uint4 o;
-      uint32_t* ou = reinterpret_cast<uint32_t*>(&o);
+      const uint32_t u[4] = {buf[c].x, buf[c].y, buf[c].z, buf[c].w};
+      uint32_t ou[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const float2 f = unpack_bf16x2(u[j]);
         const int col = idx * 8 + 2 * j;
-        float p0 = __expf(f.x - lse) - (col == t ? 1.f : 0.f);
-        float p1 = __expf(f.y - lse) - (col + 1 == t ? 1.f : 0.f);
-        ou[j] = pack_bf16x2(p0 * inv_n, p1 * inv_n);
+        const float p0 = f.x * scale - (col == t ? inv_n : 0.f);
+        const float p1 = f.y * scale - (col + 1 == t ? inv_n : 0.f);
+        ou[j] = pack_bf16x2(p0, p1);
       }
-      zr[idx] = o;
+      zr[idx] = make_uint4(ou[0], ou[1], ou[2], ou[3]);
     }
   }
 }
