@@ -32,6 +32,11 @@ METRIC = "train tokens/s and MFU (bf16 peak) at depth-20 GPT, 1×B200"
 DEPTH, B, T, V = 20, 32, 2048, 32768
 LR, MOMENTUM = 0.02, 0.95
 NOMINAL_BF16_TFLOPS = 2250.0
+# DRAM bytes (read + write) per GEMM launch, averaged over the 273 GEMM
+# launches of one step of this workload: ncu dram__bytes_read.sum +
+# dram__bytes_write.sum, profiles/step_d20_b32_t2048_launches.md.  Valid
+# for the GEMM kernels as captured there; set to None when they change.
+GEMM_DRAM_BYTES_PER_LAUNCH = 1017.3e6
 
 
 def model_flops_per_token(depth=DEPTH, seq=T, vocab=V):
@@ -40,6 +45,38 @@ def model_flops_per_token(depth=DEPTH, seq=T, vocab=V):
     d = 64 * depth
     n_mm = 12 * depth * d * d + vocab * d
     return 6.0 * n_mm + 6.0 * depth * d * seq
+
+
+def gemm_algorithmic_bytes_per_step(depth=DEPTH, batch=B, seq=T, vocab=V):
+    """Operand and result bytes of every GEMM launch of one step, each operand
+    read once and each result written once (bf16 2 B, fp32 4 B; a split-K
+    weight gradient counts as one fp32 write).  Returns (bytes, launches)."""
+    d, f, n = 64 * depth, 4 * 64 * depth, batch * seq
+    bf, f4 = 2, 4
+    per_layer = [
+        n * d * bf + 3 * d * d * bf + n * 3 * d * bf,          # q|k|v (+ RoPE / QK-norm)
+        n * d * bf + d * d * bf + 2 * n * d * f4,              # o-projection + fp32 residual
+        n * d * bf + f * d * bf + n * f * bf,                  # MLP up + ReLU^2
+        n * f * bf + d * f * bf + 2 * n * d * f4,              # MLP down + fp32 residual
+        n * d * bf + d * f * bf + 2 * n * f * bf,              # du = dy W_down, 2 sqrt(a)
+        n * f * bf + f * d * bf + n * d * bf,                  # dh = du W_up
+        n * d * bf + d * d * bf + n * d * bf,                  # dh = dy W_o
+        n * 3 * d * bf + 3 * d * d * bf + n * d * bf,          # dh = dqkv W_qkv
+        n * d * bf + n * f * bf + d * f * f4,                  # dW_down
+        n * f * bf + n * d * bf + f * d * f4,                  # dW_up
+        2 * n * d * bf + d * d * f4,                           # dW_o
+        n * 3 * d * bf + n * d * bf + 3 * d * d * f4,          # dW_qkv
+    ]
+    lm = [n * d * bf + vocab * d * bf + n * vocab * bf,       # logits
+          n * vocab * bf + vocab * d * bf + n * d * bf,       # dh = dz W
+          n * vocab * bf + n * d * bf + vocab * d * f4]       # dW = dz^T h
+    sq, wide = 4 * depth, 2 * depth                           # Newton-Schulz stacks
+    ns = 0
+    for cnt, m, k in ((sq, d, d), (wide, d, f)):
+        x, a = cnt * m * k * bf, cnt * m * m * bf
+        ns += 5 * ((x + a) + (a + a) + (a + x + x))         # A = X X^T; B = cA^2 + bA; Y = BX + aX
+    total = depth * sum(per_layer) + sum(lm) + ns
+    return float(total), depth * len(per_layer) + len(lm) + 30
 
 
 def ns_flops(depth=DEPTH):
@@ -321,6 +358,7 @@ def run_native(args, rank, world, local_rank):
     g_ms = sum(v["ms"] for k, v in prof.items() if k.startswith("gemm_")) or 1.0
     g_n = sum(v["launches"] for k, v in prof.items() if k.startswith("gemm_"))
     gemm_ach = g_fl / (g_ms / 1e3) / 1e12
+    gemm_alg_bytes, gemm_alg_launches = gemm_algorithmic_bytes_per_step()
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
@@ -338,7 +376,10 @@ def run_native(args, rank, world, local_rank):
         "final_loss": final_loss,
         "roofline": {"kernel": "gemm_tc (all classes)", "bound": "tensor", "achieved": gemm_ach,
                      "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                     "frac": gemm_ach / peaks["bf16_tflops_sustained"], "traffic": None,
+                     "frac": gemm_ach / peaks["bf16_tflops_sustained"],
+                     "traffic": GEMM_DRAM_BYTES_PER_LAUNCH,
+                     "traffic_unit": "bytes per launch (ncu DRAM read + write, mean over the step's GEMM launches)",
+                     "traffic_algorithmic": gemm_alg_bytes / gemm_alg_launches,
                      "peak_source": peak_kind + " bf16_tflops_sustained",
                      "launches": g_n, "ms": g_ms, "share": g_ms / total_ms},
         "kernels": kernels,
