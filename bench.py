@@ -79,6 +79,24 @@ def gemm_algorithmic_bytes_per_step(depth=DEPTH, batch=B, seq=T, vocab=V):
     return float(total), depth * len(per_layer) + len(lm) + 30
 
 
+def max_over_ranks(x, world, device="cpu"):
+    """The largest x over the ranks of the default process group (x itself on
+    one rank).  Multi-GPU device times are reported as this maximum."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_tokens_per_s(steps, world, ms_max, batch=B, seq=T):
+    """Whole-job throughput of `world` replicas that each ran `steps` steps of
+    batch x seq tokens, timed by the slowest rank (ms_max)."""
+    return steps * batch * seq * world / (ms_max / 1e3)
+
+
 def ns_flops(depth=DEPTH):
     """Newton-Schulz FLOPs of one Muon step (5 iterations, m <= n Gram form)."""
     d = 64 * depth
@@ -294,11 +312,7 @@ def run_native(args, rank, world, local_rank):
     prof = m.profile_read()
     m.profile(False)
     clk = clocks.stop()
-    ms_max = ms
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, world, dev)
     final_loss = float(loss_dev.item())
 
     # ---- end-to-end through the C ABI with host buffers
@@ -322,11 +336,7 @@ def run_native(args, rank, world, local_rank):
         f1.record(stream)
     m.sync()
     torch.cuda.synchronize()
-    e2e_ms = f0.elapsed_time(f1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), world, dev)
     m.close()
 
     cpu = None
@@ -335,8 +345,7 @@ def run_native(args, rank, world, local_rank):
 
     if rank != 0:
         return 0
-    tokens = args.steps * B * T * world
-    value = tokens / (ms_max / 1e3)
+    value = replica_tokens_per_s(args.steps, world, ms_max)
     tflops = value * model_flops_per_token() / 1e12
     # Dominant kernel: the tcgen05 GEMM (largest share of device time).
     total_ms = sum(v["ms"] for v in prof.values()) or 1.0
@@ -384,7 +393,7 @@ def run_native(args, rank, world, local_rank):
                      "launches": g_n, "ms": g_ms, "share": g_ms / total_ms},
         "kernels": kernels,
         "gpu_launches": int(launches),
-        "e2e": {"value": e2e_steps * B * T * world / (e2e_ms / 1e3), "unit": "tokens/s",
+        "e2e": {"value": replica_tokens_per_s(e2e_steps, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": 2 * B * T * 4, "d2h_bytes_per_step": 8,
                 "steps": e2e_steps},
         "clocks": clk,
