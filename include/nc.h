@@ -79,8 +79,8 @@ typedef struct {
  * from a counter-based SplitMix64 stream and Box-Muller: element i of
  * tensor t uses splitmix64(key_t + 2i) and splitmix64(key_t + 2i + 1),
  * key_t = splitmix64(seed ^ splitmix64(t + 1)).
- * depth: an even number in [2, 64] (head_dim 128; depth 1, whose single
- * head is 64 wide, returns NC_ERR_UNSUPPORTED in this build);
+ * depth: an even number in [2, 32] (head_dim 128, at most 16 heads; depth 1,
+ * whose single head is 64 wide, returns NC_ERR_UNSUPPORTED in this build);
  * vocab: [8, 32768], multiple of 8.
  * Parameters, Muon momentum (zero) and bf16 copies are allocated here;
  * activations are allocated by the first nc_gpt_fwd_bwd of a given B*T.

@@ -486,9 +486,9 @@ const char* nc_status_string(nc_status s) {
 nc_status nc_gpt_init_ex(int depth, int vocab, uint64_t seed, int flags, nc_params** out) {
   if (!out) return fail(NC_ERR_INVALID_ARG, "init: null output");
   *out = nullptr;
-  if (depth < 1 || depth > 64 || vocab < 8 || vocab > 32768 || vocab % 8 ||
+  if (depth < 1 || depth > 32 || vocab < 8 || vocab > 32768 || vocab % 8 ||
       (flags != NC_INIT_SPEC && flags != NC_INIT_ALL_RANDOM))
-    return fail(NC_ERR_INVALID_ARG, "init: depth in [1, 64], vocab in [8, 32768] (multiple of 8)");
+    return fail(NC_ERR_INVALID_ARG, "init: depth in [1, 32], vocab in [8, 32768] (multiple of 8)");
   if (depth % 2)
     return fail(NC_ERR_UNSUPPORTED, "init: odd depth gives a head width other than 128");
   nc_params* p = new nc_params();

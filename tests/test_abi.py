@@ -71,3 +71,13 @@ def test_bf16_rounding_is_exact_and_nearest_even():
     r = inputs.round_to_bf16(x)
     assert r[0] == 1.0 and r[1] == 1.0 and r[2] == 1.0 + 2 ** -7 and r[3] == -2.5
     assert np.all((r.view(np.uint32) & 0xFFFF) == 0)
+
+
+@pytest.mark.parametrize("depth,vocab,status", [(34, 512, "NC_ERR_INVALID_ARG"),   # 17 heads
+                                                (3, 512, "NC_ERR_UNSUPPORTED"),    # odd depth
+                                                (2, 12, "NC_ERR_INVALID_ARG")])    # vocab % 8
+def test_init_rejects_unsupported_shapes(depth, vocab, status):
+    """Shape validation runs before any CUDA call, so it is checked here."""
+    with pytest.raises(binding.NcError) as e:
+        binding.GPT(depth, vocab=vocab, seed=1)
+    assert e.value.status == getattr(binding, status)

@@ -134,6 +134,7 @@ def test_token_out_of_range_is_an_error_not_a_fault():
     m.close()
 
 
+
 def test_accumulation_invariant_on_gpu():
     depth, B, T = 2, 4, 64
     P = inputs.random_params(depth, seed=26)
