@@ -166,7 +166,8 @@ typedef enum {
   NC_EPI_STORE_F32 = 1,  /* D(f32)  = alpha*acc                               */
   NC_EPI_RESID_F32 = 2,  /* D(f32)  = aux(f32) + alpha*acc       (residual)   */
   NC_EPI_RELU2 = 3,      /* D(bf16) = max(alpha*acc, 0)^2        (ReLU^2)     */
-  NC_EPI_RELU2_BWD = 4,  /* D(bf16) = 2*sqrt(aux(bf16))*alpha*acc (aux = relu(u)^2) */
+  NC_EPI_RELU2_BWD = 4,  /* D(bf16) = 2*sqrt(aux(bf16))*alpha*acc (aux = relu(u)^2;
+                            sqrt by sqrt.approx, relative error ~2^-23)     */
   NC_EPI_AXPBY_BF16 = 5, /* D(bf16) = alpha*acc + beta*aux(bf16)              */
   NC_EPI_ACC_F32 = 6,    /* D(f32) += alpha*acc                  (atomic)     */
   NC_EPI_ROPE_QKNORM = 7 /* fused q|k|v projection: columns [0, 2*H*128) are q
