@@ -47,6 +47,9 @@ def lib():
                                        ctypes.c_double, dp]
         L.oc_muon_update.argtypes = [dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                      ctypes.c_double]
+        L.oc_adamw_update.argtypes = [dp, dp, dp, dp, ctypes.c_int64, ctypes.c_double,
+                                      ctypes.c_double, ctypes.c_double, ctypes.c_double,
+                                      ctypes.c_double, ctypes.c_int]
         _lib = L
     return _lib
 
@@ -173,6 +176,14 @@ def muon_update(W, M, G, lr, mu):
     rows, cols = W.shape
     assert lib().oc_muon_update(_dp(W), _dp(M), _dp(G), rows, cols, lr, mu) == 0
     return W, M
+
+
+def adamw_update(W, m, v, g, lr, b1, b2, eps, wd, t):
+    """AdamW step t on copies of W, m, v (any shape); returns (W, m, v)."""
+    W, m, v, g = _f64(W).copy(), _f64(m).copy(), _f64(v).copy(), _f64(g)
+    assert lib().oc_adamw_update(_dp(W), _dp(m), _dp(v), _dp(g), W.size, lr, b1, b2, eps, wd,
+                                 t) == 0
+    return W, m, v
 
 
 def param_numel(depth, idx, vocab=32768):

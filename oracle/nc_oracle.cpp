@@ -532,4 +532,17 @@ int oc_muon_update(double* W, double* M, const double* G, int rows, int cols, do
   return 0;
 }
 
+int oc_adamw_update(double* W, double* m, double* v, const double* g, int64_t n, double lr,
+                    double b1, double b2, double eps, double wd, int t) {
+  if (!W || !m || !v || !g || n < 1 || t < 1) return -1;
+  const double c1 = 1.0 - std::pow(b1, t), c2 = 1.0 - std::pow(b2, t);
+  for (int64_t i = 0; i < n; ++i) {
+    m[i] = b1 * m[i] + (1.0 - b1) * g[i];
+    v[i] = b2 * v[i] + (1.0 - b2) * g[i] * g[i];
+    const double mhat = m[i] / c1, vhat = v[i] / c2;
+    W[i] -= lr * (mhat / (std::sqrt(vhat) + eps) + wd * W[i]);
+  }
+  return 0;
+}
+
 }  // extern "C"

@@ -122,6 +122,16 @@ int oc_newton_schulz(const double* G, int rows, int cols, int steps, double a, d
  * W, M: [rows, cols] double; G: [rows, cols] double. */
 int oc_muon_update(double* W, double* M, const double* G, int rows, int cols, double lr, double mu);
 
+/* AdamW step t (t >= 1) on one tensor of n elements, in place (guide,
+ * section "2. Otimizador Muon": the embeddings and lm_head take AdamW; the
+ * pages give no hyperparameters, so they are arguments).  Decoupled weight
+ * decay and bias correction:
+ *   m <- b1 m + (1 - b1) g;   v <- b2 v + (1 - b2) g^2
+ *   W <- W - lr * ( (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps) + wd * W )
+ * where the decay term uses W before this step. */
+int oc_adamw_update(double* W, double* m, double* v, const double* g, int64_t n, double lr,
+                    double b1, double b2, double eps, double wd, int t);
+
 #ifdef __cplusplus
 }
 #endif

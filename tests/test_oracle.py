@@ -305,6 +305,80 @@ def test_muon_update_momentum_and_apply():
     np.testing.assert_allclose((W - W1) / lr, oracle.newton_schulz(mu * M + G), atol=1e-10)
 
 
+# ------------------------------------------------------------------ AdamW (embeddings, lm_head)
+ADAM = dict(lr=0.01, b1=0.9, b2=0.95, eps=1e-8)
+
+
+def test_adamw_first_step_is_a_normalised_sign_step():
+    """Step 1 with no decay: bias correction makes m-hat = g and v-hat = g^2
+    exactly, so each weight moves by lr * g / (|g| + eps); g = 0 stays put."""
+    rng = np.random.default_rng(30)
+    W, g = rng.standard_normal(500), rng.standard_normal(500)
+    g[::7] = 0.0
+    z = np.zeros(500)
+    W1, m1, v1 = oracle.adamw_update(W, z, z, g, wd=0.0, t=1, **ADAM)
+    np.testing.assert_allclose(W - W1, ADAM["lr"] * g / (np.abs(g) + ADAM["eps"]), rtol=1e-12, atol=1e-18)
+    assert np.all(W1[::7] == W[::7])
+
+
+def test_adamw_constant_gradient_moves_linearly():
+    """With the same g every step the bias-corrected moments stay g and g^2,
+    so after t steps W = W0 - t * lr * g / (|g| + eps) (no decay)."""
+    rng = np.random.default_rng(31)
+    W0, g = rng.standard_normal(300), rng.standard_normal(300)
+    W, m, v = W0, np.zeros(300), np.zeros(300)
+    for t in range(1, 8):
+        W, m, v = oracle.adamw_update(W, m, v, g, wd=0.0, t=t, **ADAM)
+        np.testing.assert_allclose(W0 - W, t * ADAM["lr"] * g / (np.abs(g) + ADAM["eps"]), rtol=1e-10)
+
+
+def test_adamw_decay_is_decoupled():
+    """Zero gradient: the moments stay zero and only the decoupled decay acts,
+    W_t = W0 (1 - lr wd)^t (a decay folded into g would move m and v)."""
+    rng = np.random.default_rng(32)
+    W0 = rng.standard_normal(200)
+    W, m, v = W0, np.zeros(200), np.zeros(200)
+    wd = 0.1
+    for t in range(1, 5):
+        W, m, v = oracle.adamw_update(W, m, v, np.zeros(200), wd=wd, t=t, **ADAM)
+        assert np.all(m == 0) and np.all(v == 0)
+        np.testing.assert_allclose(W, W0 * (1 - ADAM["lr"] * wd) ** t, rtol=1e-13)
+
+
+def test_adamw_moments_after_two_steps():
+    rng = np.random.default_rng(33)
+    g1, g2 = rng.standard_normal(100), rng.standard_normal(100)
+    z = np.zeros(100)
+    b1, b2 = ADAM["b1"], ADAM["b2"]
+    W1, m1, v1 = oracle.adamw_update(z, z, z, g1, wd=0.0, t=1, **ADAM)
+    W2, m2, v2 = oracle.adamw_update(W1, m1, v1, g2, wd=0.0, t=2, **ADAM)
+    np.testing.assert_allclose(m2, (1 - b1) * (b1 * g1 + g2), rtol=1e-13)
+    np.testing.assert_allclose(v2, (1 - b2) * (b2 * g1 ** 2 + g2 ** 2), rtol=1e-13)
+    mhat, vhat = m2 / (1 - b1 ** 2), v2 / (1 - b2 ** 2)
+    np.testing.assert_allclose(W1 - W2, ADAM["lr"] * mhat / (np.sqrt(vhat) + ADAM["eps"]), rtol=1e-10)
+
+
+def test_adamw_is_invariant_to_gradient_scale_and_odd_in_its_sign():
+    """With eps = 0 the update depends on g only through its direction per
+    element: scaling every gradient by c > 0 changes nothing, and flipping the
+    sign of g flips the step (both fail if the square root or a moment is
+    misplaced)."""
+    rng = np.random.default_rng(34)
+    W0 = rng.standard_normal(120)
+    gs = [rng.standard_normal(120) for _ in range(3)]
+    hp = dict(ADAM, eps=0.0)
+
+    def run(scale):
+        W, m, v = W0, np.zeros(120), np.zeros(120)
+        for t, g in enumerate(gs, 1):
+            W, m, v = oracle.adamw_update(W, m, v, scale * g, wd=0.0, t=t, **hp)
+        return W
+
+    base = run(1.0)
+    np.testing.assert_allclose(run(37.5), base, rtol=1e-12)
+    np.testing.assert_allclose(W0 - run(-2.0), -(W0 - base), rtol=1e-10)
+
+
 # ------------------------------------------------------------------ forward composition
 def _rms(x):
     return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + 1e-6)
