@@ -413,6 +413,27 @@ def run_op(args):
     torch.manual_seed(0)
     dims = [int(x) for x in args.shape.split(",")]
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    if args.op == "adamw":
+        # AdamW on the depth-20 embedding and lm_head ([V, d] each): HBM-bound.
+        m = nc.GPT(DEPTH, vocab=V, seed=7, all_random=True)
+        step = lambda: m.adamw_step(0.2, 0.004, 0.8, 0.95, 1e-10, 0.0)
+        for _ in range(args.warmup):
+            step()
+        m.sync()
+        ev[0].record()
+        for _ in range(args.steps):
+            step()
+        ev[1].record()
+        torch.cuda.synchronize()
+        ms = ev[0].elapsed_time(ev[1]) / args.steps
+        n = V * 64 * DEPTH
+        nbytes = 2 * n * (16.0 + 12.0) + n * 2.0  # g, m, v, W in; m, v, W out; lm_head bf16
+        m.close()
+        print(json.dumps({"op": "adamw", "shape": [V, 64 * DEPTH], "ms_per_launch": ms,
+                          "gbs": nbytes / (ms / 1e3) / 1e9,
+                          "frac_of_hbm": nbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                          "peak_source": peak_kind, "algorithmic_bytes": nbytes}), flush=True)
+        return 0
     if args.op == "gemm":
         M, N, K = dims[:3]
         ak = dims[3] if len(dims) > 3 else 1
@@ -476,7 +497,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["gemm", "attn", "attn_bwd"], default=None,
+    ap.add_argument("--op", choices=["gemm", "attn", "attn_bwd", "adamw"], default=None,
                     help="time one kernel class alone instead of the step")
     ap.add_argument("--shape", default="16384,5120,1280")
     args = ap.parse_args()

@@ -152,6 +152,23 @@ nc_status nc_gpt_fwd_bwd_async(nc_params* p, const int32_t* tokens, const int32_
  * lm_head are not touched (the guide gives them to AdamW).  Asynchronous. */
 nc_status nc_muon_step(nc_params* p, const nc_grads* g, float lr, float momentum);
 
+/* AdamW step on the embedding (wte, lr_embed) and lm_head (lr_head) from
+ * their gradients in g (guide, section "2. Otimizador Muon": embeddings and
+ * lm_head take AdamW; the pages give no hyperparameters, so all are
+ * arguments).  With t the number of calls on this handle so far (1 for the
+ * first), per element:
+ *   m <- beta1 m + (1 - beta1) g;   v <- beta2 v + (1 - beta2) g^2
+ *   W <- W - lr ((m / (1 - beta1^t)) / (sqrt(v / (1 - beta2^t)) + eps)
+ *                + weight_decay W)        (decoupled decay, W before the step)
+ * in fp32; lm_head's bf16 working copy is refreshed.  The moments (fp32,
+ * 4 * vocab * d floats) are allocated and zeroed by the first call; the
+ * block matrices are not touched (nc_muon_step).  Asynchronous.
+ * Errors: NC_ERR_INVALID_ARG (null, gradients of another handle,
+ * lr / eps / weight_decay < 0, betas outside [0, 1)), NC_ERR_TIMEOUT
+ * (poisoned handle), NC_ERR_CUDA. */
+nc_status nc_adamw_step(nc_params* p, const nc_grads* g, float lr_embed, float lr_head, float beta1,
+                        float beta2, float eps, float weight_decay);
+
 /* Wait for the handle's stream; returns the first device-side error. */
 nc_status nc_sync(nc_params* p);
 

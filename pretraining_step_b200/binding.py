@@ -90,6 +90,7 @@ def lib():
         "nc_gpt_fwd_bwd": (ci, [vp, vp, vp, ci, ci, ctypes.POINTER(cf), vp]),
         "nc_gpt_fwd_bwd_async": (ci, [vp, vp, vp, ci, ci, vp, vp]),
         "nc_muon_step": (ci, [vp, vp, cf, cf]),
+        "nc_adamw_step": (ci, [vp, vp, cf, cf, cf, cf, cf, cf]),
         "nc_sync": (ci, [vp]),
         "nc_op_gemm": (ci, [ctypes.POINTER(GemmDesc), vp]),
         "nc_op_rmsnorm": (ci, [vp, i64, ci, vp, vp, vp]),
@@ -242,6 +243,11 @@ class GPT:
 
     def muon_step(self, lr, momentum):
         _check(lib().nc_muon_step(self.h, self.g, lr, momentum))
+
+    def adamw_step(self, lr_embed, lr_head, beta1, beta2, eps, weight_decay):
+        """AdamW on the embedding and lm_head from the current gradients."""
+        _check(lib().nc_adamw_step(self.h, self.g, lr_embed, lr_head, beta1, beta2, eps,
+                                   weight_decay))
 
     def sync(self):
         _check(lib().nc_sync(self.h))

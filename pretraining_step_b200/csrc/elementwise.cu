@@ -1,8 +1,8 @@
 // elementwise.cu -- the memory-bound kernels of the step: embedding gather
 // and scatter-add, RMSNorm forward/backward, RoPE + QK-norm forward/backward,
 // fused softmax cross-entropy (loss and logits gradient in one pass),
-// parameter init, bf16 refresh, and the Muon momentum / normalise / apply
-// passes.  One warp per row where a row reduction is needed (warp-shuffle
+// parameter init, bf16 refresh, the Muon momentum / normalise / apply
+// passes and the AdamW step of the embedding and lm_head.  One warp per row where a row reduction is needed (warp-shuffle
 // sums, fp32 statistics), 16-byte vector accesses where rows allow.
 
 #include "common.cuh"
@@ -618,6 +618,66 @@ nc_status scale_bf16(const void* x, int rows, int cols, int transpose, const flo
   dim3 grid((cols + 31) / 32, (rows + 31) / 32, count);
   scale_bf16_kernel<<<grid, dim3(32, 8), 0, s>>>((const __nv_bfloat16*)x, rows, cols, transpose,
                                                  sumsq, eps, (__nv_bfloat16*)y);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+// ------------------------------------------------------------------ AdamW
+namespace {
+
+// One AdamW step on n contiguous fp32 elements (guide, section "2. Otimizador
+// Muon": the embeddings and lm_head take AdamW), decoupled weight decay and
+// bias correction ic1 = 1/(1 - b1^t), ic2 = 1/(1 - b2^t):
+//   m <- b1 m + (1 - b1) g;  v <- b2 v + (1 - b2) g^2;
+//   W <- W - lr ((m ic1) / (sqrt(v ic2) + eps) + wd W);  Wb <- bf16(W) if given.
+// Four elements per thread (16-byte accesses), grid-stride.
+__device__ __forceinline__ float adamw_elem(float& w, float& m, float& v, float g, float lr, float b1,
+                                            float b2, float eps, float wd, float ic1, float ic2) {
+  m = b1 * m + (1.f - b1) * g;
+  v = b2 * v + (1.f - b2) * g * g;
+  w -= lr * ((m * ic1) / (sqrtf(v * ic2) + eps) + wd * w);
+  return w;
+}
+
+__global__ void adamw_kernel(float* __restrict__ W, __nv_bfloat16* __restrict__ Wb,
+                             float* __restrict__ M, float* __restrict__ Vs,
+                             const float* __restrict__ G, int64_t n, float lr, float b1, float b2,
+                             float eps, float wd, float ic1, float ic2) {
+  const int64_t n4 = n / 4;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
+    float4 w = reinterpret_cast<float4*>(W)[i];
+    float4 m = reinterpret_cast<float4*>(M)[i];
+    float4 v = reinterpret_cast<float4*>(Vs)[i];
+    const float4 g = reinterpret_cast<const float4*>(G)[i];
+    adamw_elem(w.x, m.x, v.x, g.x, lr, b1, b2, eps, wd, ic1, ic2);
+    adamw_elem(w.y, m.y, v.y, g.y, lr, b1, b2, eps, wd, ic1, ic2);
+    adamw_elem(w.z, m.z, v.z, g.z, lr, b1, b2, eps, wd, ic1, ic2);
+    adamw_elem(w.w, m.w, v.w, g.w, lr, b1, b2, eps, wd, ic1, ic2);
+    reinterpret_cast<float4*>(W)[i] = w;
+    reinterpret_cast<float4*>(M)[i] = m;
+    reinterpret_cast<float4*>(Vs)[i] = v;
+    if (Wb) reinterpret_cast<uint2*>(Wb)[i] = make_uint2(pack_bf16x2(w.x, w.y), pack_bf16x2(w.z, w.w));
+  }
+  for (int64_t i = n4 * 4 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+    const float w = adamw_elem(W[i], M[i], Vs[i], G[i], lr, b1, b2, eps, wd, ic1, ic2);
+    if (Wb) Wb[i] = f2bf(w);
+  }
+}
+
+}  // namespace
+
+nc_status adamw(float* W, void* Wb, float* m, float* v, const float* g, int64_t n, float lr,
+                float b1, float b2, float eps, float wd, int t, cudaStream_t s, Profiler* prof) {
+  if (n < 1 || t < 1 || !W || !m || !v || !g) return fail(NC_ERR_INVALID_ARG, "adamw: bad arguments");
+  if ((reinterpret_cast<uintptr_t>(W) | reinterpret_cast<uintptr_t>(m) | reinterpret_cast<uintptr_t>(v) |
+       reinterpret_cast<uintptr_t>(g) | reinterpret_cast<uintptr_t>(Wb)) & 15)
+    return fail(NC_ERR_INVALID_ARG, "adamw: buffers must be 16-byte aligned");
+  const double ic1 = 1.0 / (1.0 - std::pow((double)b1, t)), ic2 = 1.0 / (1.0 - std::pow((double)b2, t));
+  Probe probe(prof, s, "adamw", 0.0, (double)n * (16.0 + 12.0 + (Wb ? 2.0 : 0.0)));
+  const unsigned grid = (unsigned)std::min<int64_t>(blocks_for((n + 3) / 4, 256), 148 * 8);
+  adamw_kernel<<<grid, 256, 0, s>>>(W, static_cast<__nv_bfloat16*>(Wb), m, v, g, n, lr, b1, b2, eps, wd,
+                                    (float)ic1, (float)ic2);
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }

@@ -69,6 +69,10 @@ nc_status muon_prep(const float* src, int64_t src_stride, int rows, int cols, in
 nc_status muon_apply(float* W, void* Wb, int64_t w_stride, int rows, int cols, int transpose,
                      const void* X, int64_t x_stride, float lr, int L, cudaStream_t s,
                      Profiler* prof);
+// AdamW step t on n fp32 elements in place; Wb (bf16 copy) refreshed when
+// not null.
+nc_status adamw(float* W, void* Wb, float* m, float* v, const float* g, int64_t n, float lr,
+                float b1, float b2, float eps, float wd, int t, cudaStream_t s, Profiler* prof);
 nc_status sumsq_bf16(const void* x, int64_t n, int count, float* out, cudaStream_t s,
                      Profiler* prof);
 nc_status scale_bf16(const void* x, int rows, int cols, int transpose, const float* sumsq,

@@ -102,6 +102,10 @@ struct nc_params {
   // Muon
   float* sumsq = nullptr;
   nc::bf16 *xsq = nullptr, *xw = nullptr, *nsws = nullptr;
+  // AdamW state of wte and lm_head (first and second moments, allocated
+  // and zeroed by the first nc_adamw_step) and the step count
+  float* adam = nullptr;
+  int adam_t = 0;
   // RoPE table
   float2* rope = nullptr;
   int rope_T = 0;
@@ -552,6 +556,7 @@ void nc_params_free(nc_params* p) {
   else cudaDeviceSynchronize();
   if (p->act.mem) cudaFree(p->act.mem);
   if (p->rope) cudaFree(p->rope);
+  if (p->adam) cudaFree(p->adam);
   if (p->pmem) cudaFree(p->pmem);
   if (p->h_loss) cudaFreeHost(p->h_loss);
   if (p->h_status) cudaFreeHost(p->h_status);
@@ -711,6 +716,27 @@ nc_status nc_gpt_fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* tar
 nc_status nc_muon_step(nc_params* p, const nc_grads* g, float lr, float momentum) {
   if (!p) return fail(NC_ERR_INVALID_ARG, "muon: null handle");
   return muon(p, g, lr, momentum);
+}
+
+nc_status nc_adamw_step(nc_params* p, const nc_grads* g, float lr_embed, float lr_head, float beta1,
+                        float beta2, float eps, float weight_decay) {
+  if (!p) return fail(NC_ERR_INVALID_ARG, "adamw: null handle");
+  if (p->poisoned) return fail(NC_ERR_TIMEOUT, "handle poisoned by an earlier device timeout");
+  if (!g || g->p != p) return fail(NC_ERR_INVALID_ARG, "adamw: gradients of another model");
+  if (!(lr_embed >= 0.f) || !(lr_head >= 0.f) || !(beta1 >= 0.f && beta1 < 1.f) ||
+      !(beta2 >= 0.f && beta2 < 1.f) || !(eps >= 0.f) || !(weight_decay >= 0.f))
+    return fail(NC_ERR_INVALID_ARG, "adamw: lr, eps, weight_decay >= 0 and betas in [0, 1)");
+  const int64_t n = (int64_t)p->vocab * p->d;  // wte and lm_head are both [V, d]
+  if (!p->adam) {
+    NC_CUDA_TRY(cudaMalloc(&p->adam, sizeof(float) * 4 * n));
+    NC_CUDA_TRY(cudaMemsetAsync(p->adam, 0, sizeof(float) * 4 * n, p->stream));
+  }
+  const int t = ++p->adam_t;
+  NC_TRY(adamw(p->wte, nullptr, p->adam, p->adam + n, g->wte, n, lr_embed, beta1, beta2, eps,
+               weight_decay, t, p->stream, p->prof));
+  NC_TRY(adamw(p->lm, p->lm_b, p->adam + 2 * n, p->adam + 3 * n, g->lm, n, lr_head, beta1, beta2,
+               eps, weight_decay, t, p->stream, p->prof));
+  return NC_OK;
 }
 
 nc_status nc_sync(nc_params* p) {

@@ -81,3 +81,8 @@ def test_init_rejects_unsupported_shapes(depth, vocab, status):
     with pytest.raises(binding.NcError) as e:
         binding.GPT(depth, vocab=vocab, seed=1)
     assert e.value.status == getattr(binding, status)
+
+
+def test_adamw_step_refuses_a_null_handle():
+    st = binding.lib().nc_adamw_step(None, None, 0.1, 0.1, 0.9, 0.95, 1e-8, 0.0)
+    assert st == binding.NC_ERR_INVALID_ARG

@@ -183,6 +183,56 @@ def test_muon_step_parity():
     m.close()
 
 
+def _device_u16(ptr, n):
+    """n uint16 at a raw device pointer, copied to the host."""
+    t = torch()
+
+    class _View:
+        __cuda_array_interface__ = {"shape": (n,), "typestr": "<u2", "data": (ptr, False),
+                                    "version": 3}
+
+    return t.as_tensor(_View(), device="cuda").cpu().numpy()
+
+
+def test_adamw_step_parity():
+    """AdamW on given gradients (embedding and lm_head) against the oracle
+    over three steps (the step count and bias correction kept by the handle),
+    with zero gradient entries and weight decay; the block matrices stay put
+    and lm_head's bf16 working copy is the rounded master."""
+    depth, vocab = 2, 512
+    hp = dict(beta1=0.8, beta2=0.95, eps=1e-10, weight_decay=0.01)
+    lr_e, lr_h = 0.05, 0.004
+    m = _gpt(depth, vocab=vocab, seed=40, all_random=True)
+    W0 = m.params()
+    n = m.num_tensors()
+    rng = np.random.default_rng(41)
+    ref = {0: [W0[0].astype(np.float64), 0.0, 0.0], n - 1: [W0[-1].astype(np.float64), 0.0, 0.0]}
+    for t in range(1, 4):
+        G = [rng.standard_normal(sh).astype(np.float32) * 0.1 for sh in m.shapes()]
+        G[0][::5] = 0.0
+        for i in range(n):
+            m.write_grad(i, G[i])
+        m.adamw_step(lr_e, lr_h, **hp)
+        for i, lr in ((0, lr_e), (n - 1, lr_h)):
+            w, mm, vv = ref[i]
+            mm = np.zeros_like(w) if t == 1 else mm
+            vv = np.zeros_like(w) if t == 1 else vv
+            ref[i] = list(oracle.adamw_update(w, mm, vv, G[i], lr, hp["beta1"], hp["beta2"],
+                                              hp["eps"], hp["weight_decay"], t))
+    m.sync()
+    W = m.params()
+    for i in (0, n - 1):
+        np.testing.assert_allclose(W[i], ref[i][0], rtol=2e-6, atol=2e-7)
+        assert rel_fro(W0[i] - W[i], W0[i] - ref[i][0]) < 1e-5
+    for i in range(1, n - 1):
+        assert np.array_equal(W[i], W0[i])
+    info = m.tensor_info(n - 1)
+    bits = _device_u16(info.data_bf16, W[-1].size)
+    want = (inputs.round_to_bf16(W[-1]).reshape(-1).view(np.uint32) >> 16).astype(np.uint16)
+    assert np.array_equal(bits, want)
+    m.close()
+
+
 def test_profiler_counts_launches():
     depth, B, T = 2, 1, 64
     m = _gpt(depth)
