@@ -47,6 +47,11 @@ def lib():
                                        ctypes.c_double, dp]
         L.oc_muon_update.argtypes = [dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_double,
                                      ctypes.c_double]
+        L.oc_attention_ex.argtypes = [dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                      ctypes.c_int, ctypes.c_int, ctypes.c_int, dp, dp]
+        L.oc_attention_bwd_ex.argtypes = [dp, dp, dp, dp, dp, ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          dp, dp, dp]
         L.oc_adamw_update.argtypes = [dp, dp, dp, dp, ctypes.c_int64, ctypes.c_double,
                                       ctypes.c_double, ctypes.c_double, ctypes.c_double,
                                       ctypes.c_double, ctypes.c_int]
@@ -129,6 +134,30 @@ def attention_bwd(q, k, v, lse, dout):
     dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
     assert lib().oc_attention_bwd(_dp(q), _dp(k), _dp(v), _dp(lse), _dp(dout), B, T, H, hd,
                                   _dp(dq), _dp(dk), _dp(dv)) == 0
+    return dq, dk, dv
+
+
+def attention_ex(q, k, v, window=-1):
+    """Causal attention with KV heads k, v: [B, T, Hkv, hd] shared by groups of
+    H / Hkv query heads and a left window (-1: none) -> (o, lse)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, T, H, hd = q.shape
+    Hkv = k.shape[2]
+    o = np.empty_like(q)
+    lse = np.empty((B, H, T), dtype=np.float64)
+    assert lib().oc_attention_ex(_dp(q), _dp(k), _dp(v), B, T, H, Hkv, hd, window, _dp(o),
+                                 _dp(lse)) == 0
+    return o, lse
+
+
+def attention_bwd_ex(q, k, v, lse, dout, window=-1):
+    """Gradients (dq [B, T, H, hd], dk, dv [B, T, Hkv, hd]) of attention_ex."""
+    q, k, v, lse, dout = _f64(q), _f64(k), _f64(v), _f64(lse), _f64(dout)
+    B, T, H, hd = q.shape
+    Hkv = k.shape[2]
+    dq, dk, dv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    assert lib().oc_attention_bwd_ex(_dp(q), _dp(k), _dp(v), _dp(lse), _dp(dout), B, T, H, Hkv,
+                                     hd, window, _dp(dq), _dp(dk), _dp(dv)) == 0
     return dq, dk, dv
 
 

@@ -16,6 +16,7 @@
 
 #include "nc_oracle.h"
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -228,6 +229,94 @@ void attention_bwd(const double* q, const double* k, const double* v, const doub
     }
 }
 
+// Causal attention with grouped KV heads and a left window (guide, section
+// "1. Modelo GPT": "GQA: atencao com menos heads KV", "atencao de janela ...
+// 'SSSL'", and the flash-attention call with causal=True, window_size):
+// query head hh reads KV head hh / (H / Hkv); query t sees keys
+// j in [t - window, t] (window < 0: no lower bound).  q, o: [B, T, H, hd];
+// k, v: [B, T, Hkv, hd]; lse [B, H, T].
+void attention_fwd_gw(const double* q, const double* k, const double* v, int B, int T, int H,
+                      int Hkv, int hd, int window, double* o, double* lse) {
+  const double scale = 1.0 / std::sqrt((double)hd);
+  const int64_t rq = (int64_t)H * hd, rk = (int64_t)Hkv * hd;
+  const int group = H / Hkv;
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int b = 0; b < B; ++b)
+    for (int hh = 0; hh < H; ++hh) {
+      const int hk = hh / group;
+      std::vector<double> s(T);
+      for (int t = 0; t < T; ++t) {
+        const int j0 = window < 0 ? 0 : std::max(0, t - window);
+        const double* qt = q + ((int64_t)b * T + t) * rq + (int64_t)hh * hd;
+        double m = -INFINITY;
+        for (int j = j0; j <= t; ++j) {
+          const double* kj = k + ((int64_t)b * T + j) * rk + (int64_t)hk * hd;
+          double acc = 0;
+          for (int i = 0; i < hd; ++i) acc += qt[i] * kj[i];
+          s[j] = acc * scale;
+          if (s[j] > m) m = s[j];
+        }
+        double l = 0;
+        for (int j = j0; j <= t; ++j) l += std::exp(s[j] - m);
+        const double ls = m + std::log(l);
+        lse[((int64_t)b * H + hh) * T + t] = ls;
+        double* ot = o + ((int64_t)b * T + t) * rq + (int64_t)hh * hd;
+        for (int i = 0; i < hd; ++i) ot[i] = 0;
+        for (int j = j0; j <= t; ++j) {
+          const double p = std::exp(s[j] - ls);
+          const double* vj = v + ((int64_t)b * T + j) * rk + (int64_t)hk * hd;
+          for (int i = 0; i < hd; ++i) ot[i] += p * vj[i];
+        }
+      }
+    }
+}
+
+// Reverse mode of attention_fwd_gw (same formulas as attention_bwd).  The
+// query heads of one KV head run in one thread, in head order, because they
+// all add into that KV head's dk and dv.
+void attention_bwd_gw(const double* q, const double* k, const double* v, const double* lse,
+                      const double* dout, int B, int T, int H, int Hkv, int hd, int window,
+                      double* dq, double* dk, double* dv) {
+  const double scale = 1.0 / std::sqrt((double)hd);
+  const int64_t rq = (int64_t)H * hd, rk = (int64_t)Hkv * hd;
+  const int group = H / Hkv;
+  std::memset(dq, 0, sizeof(double) * B * T * rq);
+  std::memset(dk, 0, sizeof(double) * B * T * rk);
+  std::memset(dv, 0, sizeof(double) * B * T * rk);
+#pragma omp parallel for collapse(2) schedule(static)
+  for (int b = 0; b < B; ++b)
+    for (int hk = 0; hk < Hkv; ++hk) {
+      std::vector<double> p(T), dp(T);
+      for (int hh = hk * group; hh < (hk + 1) * group; ++hh)
+        for (int t = 0; t < T; ++t) {
+          const int j0 = window < 0 ? 0 : std::max(0, t - window);
+          const int64_t rt = ((int64_t)b * T + t) * rq + (int64_t)hh * hd;
+          const double ls = lse[((int64_t)b * H + hh) * T + t];
+          double D = 0;
+          for (int j = j0; j <= t; ++j) {
+            const int64_t rj = ((int64_t)b * T + j) * rk + (int64_t)hk * hd;
+            double sc = 0, g = 0;
+            for (int i = 0; i < hd; ++i) {
+              sc += q[rt + i] * k[rj + i];
+              g += dout[rt + i] * v[rj + i];
+            }
+            p[j] = std::exp(sc * scale - ls);
+            dp[j] = g;
+            D += p[j] * g;
+          }
+          for (int j = j0; j <= t; ++j) {
+            const int64_t rj = ((int64_t)b * T + j) * rk + (int64_t)hk * hd;
+            const double ds = p[j] * (dp[j] - D);
+            for (int i = 0; i < hd; ++i) {
+              dq[rt + i] += scale * ds * k[rj + i];
+              dk[rj + i] += scale * ds * q[rt + i];
+              dv[rj + i] += p[j] * dout[rt + i];
+            }
+          }
+        }
+    }
+}
+
 // ---------------------------------------------------------------- Newton-Schulz
 // Plain product c[m, n] = a[m, k] * b[k, n].
 void mm_plain(const double* a, const double* b, int m, int k, int n, double* c) {
@@ -367,6 +456,24 @@ int oc_attention_bwd(const double* q, const double* k, const double* v, const do
   if (!q || !k || !v || !lse || !dout || !dq || !dk || !dv || B < 0 || T < 0 || H < 1 || hd < 1)
     return -1;
   attention_bwd(q, k, v, lse, dout, B, T, H, hd, dq, dk, dv);
+  return 0;
+}
+
+int oc_attention_ex(const double* q, const double* k, const double* v, int B, int T, int H, int Hkv,
+                    int hd, int window, double* o, double* lse) {
+  if (!q || !k || !v || !o || !lse || B < 0 || T < 0 || H < 1 || hd < 1 || Hkv < 1 || H % Hkv)
+    return -1;
+  attention_fwd_gw(q, k, v, B, T, H, Hkv, hd, window, o, lse);
+  return 0;
+}
+
+int oc_attention_bwd_ex(const double* q, const double* k, const double* v, const double* lse,
+                        const double* dout, int B, int T, int H, int Hkv, int hd, int window,
+                        double* dq, double* dk, double* dv) {
+  if (!q || !k || !v || !lse || !dout || !dq || !dk || !dv || B < 0 || T < 0 || H < 1 || hd < 1 ||
+      Hkv < 1 || H % Hkv)
+    return -1;
+  attention_bwd_gw(q, k, v, lse, dout, B, T, H, Hkv, hd, window, dq, dk, dv);
   return 0;
 }
 

@@ -89,6 +89,18 @@ int oc_rope_row(double* v, int hd, int64_t pos, double base);
 int oc_attention(const double* q, const double* k, const double* v, int B, int T, int H, int hd,
                  double* o, double* lse, double* probs);
 
+/* Causal attention with grouped KV heads and a left window: query head h
+ * reads KV head h / (H / Hkv) (H a multiple of Hkv); query t sees keys
+ * j in [t - window, t], every key up to t when window < 0.  q, o:
+ * [B, T, H, hd]; k, v: [B, T, Hkv, hd]; lse [B, H, T].  With Hkv = H and
+ * window < 0 it is oc_attention. */
+int oc_attention_ex(const double* q, const double* k, const double* v, int B, int T, int H, int Hkv,
+                    int hd, int window, double* o, double* lse);
+/* Its reverse mode: dq [B, T, H, hd], dk, dv [B, T, Hkv, hd], OVERWRITTEN. */
+int oc_attention_bwd_ex(const double* q, const double* k, const double* v, const double* lse,
+                        const double* dout, int B, int T, int H, int Hkv, int hd, int window,
+                        double* dq, double* dk, double* dv);
+
 /* Reverse mode of oc_attention: from dout [B, T, H, hd] and the forward's
  * lse, the gradients dq, dk, dv (same layout), OVERWRITTEN. */
 int oc_attention_bwd(const double* q, const double* k, const double* v, const double* lse,

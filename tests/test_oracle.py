@@ -305,6 +305,96 @@ def test_muon_update_momentum_and_apply():
     np.testing.assert_allclose((W - W1) / lr, oracle.newton_schulz(mu * M + G), atol=1e-10)
 
 
+# ------------------------------------------------------------------ windowed / grouped-KV attention
+def _qkv(seed, B, T, H, Hkv, hd):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((B, T, H, hd)), rng.standard_normal((B, T, Hkv, hd)),
+            rng.standard_normal((B, T, Hkv, hd)))
+
+
+@pytest.mark.parametrize("window", [-1, 9, 40])
+def test_attention_ex_without_groups_or_window_is_the_causal_oracle(window):
+    """Hkv = H and a window reaching back past the row start reduce it to the
+    pinned full-causal oracle, forward and backward."""
+    B, T, H, hd = 2, 9, 3, 8
+    q, k, v = _qkv(60, B, T, H, H, hd)
+    o, lse = oracle.attention_ex(q, k, v, window=window)
+    o_ref, lse_ref, _ = oracle.attention(q, k, v)
+    np.testing.assert_allclose(o, o_ref, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(lse, lse_ref, rtol=1e-13)
+    dout = np.random.default_rng(61).standard_normal(q.shape)
+    for a, b in zip(oracle.attention_bwd_ex(q, k, v, lse, dout, window=window),
+                    oracle.attention_bwd(q, k, v, lse_ref, dout)):
+        np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-13)
+
+
+def test_attention_ex_window_zero_sees_only_itself():
+    B, T, H, Hkv, hd = 1, 7, 4, 2, 8
+    q, k, v = _qkv(62, B, T, H, Hkv, hd)
+    o, lse = oracle.attention_ex(q, k, v, window=0)
+    kv = np.repeat(np.arange(Hkv), H // Hkv)
+    np.testing.assert_allclose(o, v[:, :, kv, :], rtol=1e-14)
+    s = np.einsum("bthd,bthd->bht", q, k[:, :, kv, :]) / math.sqrt(hd)
+    np.testing.assert_allclose(lse, s, rtol=1e-13)
+
+
+def test_attention_ex_groups_equal_repeated_heads():
+    """GQA is MHA on K/V heads repeated over each group; the K/V gradients
+    are the sums of the repeated heads' gradients (the pinned MHA oracle)."""
+    B, T, H, Hkv, hd = 2, 11, 6, 2, 8
+    q, k, v = _qkv(63, B, T, H, Hkv, hd)
+    rep = np.repeat(np.arange(Hkv), H // Hkv)
+    o, lse = oracle.attention_ex(q, k, v)
+    o_ref, lse_ref, _ = oracle.attention(q, k[:, :, rep, :], v[:, :, rep, :])
+    np.testing.assert_allclose(o, o_ref, rtol=1e-13, atol=1e-14)
+    dout = np.random.default_rng(64).standard_normal(q.shape)
+    dq, dk, dv = oracle.attention_bwd_ex(q, k, v, lse, dout)
+    dq_r, dk_r, dv_r = oracle.attention_bwd(q, k[:, :, rep, :], v[:, :, rep, :], lse_ref, dout)
+    np.testing.assert_allclose(dq, dq_r, rtol=1e-12, atol=1e-13)
+    g = H // Hkv
+    np.testing.assert_allclose(dk, dk_r.reshape(B, T, Hkv, g, hd).sum(3), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(dv, dv_r.reshape(B, T, Hkv, g, hd).sum(3), rtol=1e-12, atol=1e-13)
+
+
+def test_attention_ex_window_brute_force():
+    """Tiny case against an explicit masked softmax written here."""
+    B, T, H, Hkv, hd, W = 1, 10, 4, 2, 5, 3
+    q, k, v = _qkv(65, B, T, H, Hkv, hd)
+    o, lse = oracle.attention_ex(q, k, v, window=W)
+    for h in range(H):
+        hk = h // (H // Hkv)
+        for t in range(T):
+            js = [j for j in range(T) if t - W <= j <= t]
+            s = np.array([q[0, t, h] @ k[0, j, hk] for j in js]) / math.sqrt(hd)
+            p = np.exp(s - s.max())
+            p /= p.sum()
+            np.testing.assert_allclose(o[0, t, h], p @ v[0, js, hk], rtol=1e-12)
+            np.testing.assert_allclose(lse[0, h, t], s.max() + math.log(np.exp(s - s.max()).sum()),
+                                       rtol=1e-13)
+
+
+def test_attention_ex_backward_finite_differences():
+    B, T, H, Hkv, hd, W = 1, 6, 4, 2, 3, 2
+    q, k, v = _qkv(66, B, T, H, Hkv, hd)
+    R = np.random.default_rng(67).standard_normal(q.shape)
+    loss = lambda q_, k_, v_: float((oracle.attention_ex(q_, k_, v_, window=W)[0] * R).sum())
+    o, lse = oracle.attention_ex(q, k, v, window=W)
+    grads = oracle.attention_bwd_ex(q, k, v, lse, R, window=W)
+    rng = np.random.default_rng(68)
+    eps = 1e-6
+    for which, x in enumerate((q, k, v)):
+        for _ in range(6):
+            idx = tuple(rng.integers(0, n) for n in x.shape)
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p = [q, k, v]
+            args_m = [q, k, v]
+            args_p[which], args_m[which] = xp, xm
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+            assert abs(fd - grads[which][idx]) < 1e-6 * max(1.0, abs(fd)), (which, idx)
+
+
 # ------------------------------------------------------------------ AdamW (embeddings, lm_head)
 ADAM = dict(lr=0.01, b1=0.9, b2=0.95, eps=1e-8)
 
