@@ -249,6 +249,26 @@ nc_status nc_op_attention_bwd(const void* q, const void* k, const void* v, int64
                               float* dq, void* dk, void* dv, int64_t ldg, float* delta_scratch,
                               int B, int T, int H, void* stream);
 
+/* Causal attention with grouped KV heads and a left window (guide, section
+ * "1. Modelo GPT": "GQA: atencao com menos heads KV" and "atencao de janela:
+ * contexto curto/longo alternado (ex: 'SSSL')", passed to flash attention as
+ * causal=True with a window_size; the pages give no window length).
+ * q, o, dO, dq hold H heads of 128 per row (row strides ldq, ldo; dq dense
+ * [B, T, H, 128]); k, v, dk, dv hold Hkv heads (strides ldkv, ldg), H a
+ * multiple of Hkv; query head h reads KV head h / (H / Hkv).  Query t sees
+ * keys [t - window, t]; window < 0 means every key up to t.  With Hkv = H,
+ * ldkv = ldq and window < 0 these are nc_op_attention_fwd / _bwd.  Layouts,
+ * alignment (16-byte rows) and errors otherwise as those; H <= 16 for the
+ * backward. */
+nc_status nc_op_attention_fwd_ex(const void* q, int64_t ldq, const void* k, const void* v,
+                                 int64_t ldkv, void* o, int64_t ldo, float* lse, int B, int T, int H,
+                                 int Hkv, int window, void* stream);
+nc_status nc_op_attention_bwd_ex(const void* q, int64_t ldq, const void* k, const void* v,
+                                 int64_t ldkv, const void* o, const void* dout, int64_t ldo,
+                                 const float* lse, float* dq, void* dk, void* dv, int64_t ldg,
+                                 float* delta_scratch, int B, int T, int H, int Hkv, int window,
+                                 void* stream);
+
 /* Causal attention backward like nc_op_attention_bwd, for callers that
  * cannot allocate device memory (no cudaMalloc / cudaFree of their own, no
  * workspace they can lend): a caller running while another component owns

@@ -99,6 +99,10 @@ def lib():
                                      ci, ci, ci, vp]),
         "nc_op_attention_bwd_noalloc": (ci, [vp, vp, vp, i64, vp, vp, i64, vp, vp, vp, vp,
                                              i64, ci, ci, ci, vp]),
+        "nc_op_attention_fwd_ex": (ci, [vp, i64, vp, vp, i64, vp, i64, vp, ci, ci, ci, ci, ci,
+                                        vp]),
+        "nc_op_attention_bwd_ex": (ci, [vp, i64, vp, vp, i64, vp, vp, i64, vp, vp, vp, vp, i64,
+                                        vp, ci, ci, ci, ci, ci, vp]),
         "nc_newton_schulz_scratch_bytes": (ctypes.c_size_t, [ci, ci, ci]),
         "nc_op_newton_schulz": (ci, [vp, vp, ci, ci, ci, ci, vp, vp]),
         "nc_profile_enable": (ci, [vp, ci]),
@@ -299,6 +303,20 @@ def attention_bwd(q, k, v, ld, o, dout, ldo, lse, dq, dk, dv, ldg, delta, B, T, 
     _check(lib().nc_op_attention_bwd(_ptr(q), _ptr(k), _ptr(v), ld, _ptr(o), _ptr(dout), ldo,
                                      _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), ldg, _ptr(delta),
                                      B, T, H, _stream(stream)))
+
+
+def attention_fwd_ex(q, ldq, k, v, ldkv, o, ldo, lse, B, T, H, Hkv, window, stream=None):
+    """Causal attention with Hkv KV heads shared by groups of query heads and a
+    left window (window < 0: none)."""
+    _check(lib().nc_op_attention_fwd_ex(_ptr(q), ldq, _ptr(k), _ptr(v), ldkv, _ptr(o), ldo,
+                                        _ptr(lse), B, T, H, Hkv, window, _stream(stream)))
+
+
+def attention_bwd_ex(q, ldq, k, v, ldkv, o, dout, ldo, lse, dq, dk, dv, ldg, delta, B, T, H,
+                     Hkv, window, stream=None):
+    _check(lib().nc_op_attention_bwd_ex(_ptr(q), ldq, _ptr(k), _ptr(v), ldkv, _ptr(o),
+                                        _ptr(dout), ldo, _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                                        ldg, _ptr(delta), B, T, H, Hkv, window, _stream(stream)))
 
 
 def attention_bwd_noalloc(q, k, v, ld, o, dout, ldo, lse, dq, dk, dv, ldg, B, T, H,

@@ -80,14 +80,14 @@ __global__ void __launch_bounds__(256) attn_bwd_delta_kernel(const __nv_bfloat16
 
 }  // namespace
 
-nc_status attention_bwd(const void* q, const void* k, const void* v, int64_t ld, const void* o,
-                        const void* dout, int64_t ldo, const float* lse, float* dq, void* dk,
-                        void* dv, int64_t ldg, float* delta, int B, int T, int H, int* status,
-                        cudaStream_t s, Profiler* prof) {
-  if (B < 1 || T < 1 || H < 1 || !q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv ||
-      !delta)
-    return fail(NC_ERR_INVALID_ARG, "attention_bwd: bad arguments");
-  if (ld % 8 || ldo % 8 || ldg % 8)
+nc_status attention_bwd_ex(const void* q, int64_t ldq, const void* k, const void* v, int64_t ldkv,
+                           const void* o, const void* dout, int64_t ldo, const float* lse,
+                           float* dq, void* dk, void* dv, int64_t ldg, float* delta, int B, int T,
+                           int H, int Hkv, int window, int* status, cudaStream_t s, Profiler* prof) {
+  if (B < 1 || T < 1 || H < 1 || Hkv < 1 || H % Hkv || !q || !k || !v || !o || !dout || !lse ||
+      !dq || !dk || !dv || !delta)
+    return fail(NC_ERR_INVALID_ARG, "attention_bwd: bad arguments (H must be a multiple of Hkv)");
+  if (ldq % 8 || ldkv % 8 || ldo % 8 || ldg % 8)
     return fail(NC_ERR_INVALID_ARG, "attention_bwd: strides must be multiples of 8");
   if (H > kDeltaMaxH) return fail(NC_ERR_UNSUPPORTED, "attention_bwd: at most 16 heads");
   if ((reinterpret_cast<uintptr_t>(o) | reinterpret_cast<uintptr_t>(dout)) & 15)
@@ -100,8 +100,16 @@ nc_status attention_bwd(const void* q, const void* k, const void* v, int64_t ld,
     NC_CUDA_TRY(cudaGetLastError());
   }
   NC_CUDA_TRY(cudaMemsetAsync(dq, 0, sizeof(float) * rows * HD, s));
-  return attention_bwd_tc(q, k, v, ld, dout, ldo, lse, delta, dq, dk, dv, ldg, B, T, H, status, s,
-                          prof);
+  return attention_bwd_tc_ex(q, ldq, k, v, ldkv, dout, ldo, lse, delta, dq, dk, dv, ldg, B, T, H,
+                             Hkv, window, status, s, prof);
+}
+
+nc_status attention_bwd(const void* q, const void* k, const void* v, int64_t ld, const void* o,
+                        const void* dout, int64_t ldo, const float* lse, float* dq, void* dk,
+                        void* dv, int64_t ldg, float* delta, int B, int T, int H, int* status,
+                        cudaStream_t s, Profiler* prof) {
+  return attention_bwd_ex(q, ld, k, v, ld, o, dout, ldo, lse, dq, dk, dv, ldg, delta, B, T, H, H, -1,
+                          status, s, prof);
 }
 
 // ------------------------------------------------------------------ allocation-free backward

@@ -64,6 +64,8 @@ struct FwdArgs {
   int64_t ldo;
   float* lse;
   int H;
+  int group;   // query heads per KV head (1: one KV head per query head)
+  int window;  // query t sees keys [t - window, t]; < 0: every key up to t
   int* status;
 };
 
@@ -81,6 +83,9 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     if (globaltimer() - t0 > kWaitTimeoutNs) return;
 }
 
+// GW: grouped KV heads or a window in play; the plain instance (every query
+// head its own KV head, no window) compiles with those as constants.
+template <bool GW>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const FwdArgs a) {
@@ -108,7 +113,12 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qb = a.nqb - 1 - (int)blockIdx.x;
   const int h = blockIdx.y, b = blockIdx.z;
-  const int n = qb + 1;  // causal: key tiles up to the diagonal (BKV == BQ)
+  const int group = GW ? a.group : 1;
+  const int window = GW ? a.window : -1;
+  // Key tiles from the first one the window reaches to the diagonal (BKV == BQ).
+  const int lo_key = window < 0 ? 0 : qb * BQ - window;
+  const int j_lo = lo_key <= 0 ? 0 : lo_key / BKV;
+  const int n = qb - j_lo + 1;
 
   if (threadIdx.x == 0) {
     tc::mbar_init(q_full, 1);
@@ -134,6 +144,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int col0 = h * HD;
+  const int kcol0 = (h / group) * HD;  // this query head's KV head
 
   if (warp == 0) {
     if (lane == 0) {
@@ -149,13 +160,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t ph = j & 1;
         if (!tc::mbar_wait(k_empty, ph ^ 1, abort_flag, a.status)) { ok = false; break; }
         tc::mbar_arrive_expect_tx(k_full, TILE);
-        tc::tma_load_3d(smem + OFF_K, &tk, k_full, col0, j * BKV, b);
-        tc::tma_load_3d(smem + OFF_K + TILE / 2, &tk, k_full, col0 + 64, j * BKV, b);
+        tc::tma_load_3d(smem + OFF_K, &tk, k_full, kcol0, (j_lo + j) * BKV, b);
+        tc::tma_load_3d(smem + OFF_K + TILE / 2, &tk, k_full, kcol0 + 64, (j_lo + j) * BKV, b);
         ++issued_k;
         if (!tc::mbar_wait(v_empty, ph ^ 1, abort_flag, a.status)) { ok = false; break; }
         tc::mbar_arrive_expect_tx(v_full, TILE);
-        tc::tma_load_3d(smem + OFF_V, &tv, v_full, col0, j * BKV, b);
-        tc::tma_load_3d(smem + OFF_V + TILE / 2, &tv, v_full, col0 + 64, j * BKV, b);
+        tc::tma_load_3d(smem + OFF_V, &tv, v_full, kcol0, (j_lo + j) * BKV, b);
+        tc::tma_load_3d(smem + OFF_V + TILE / 2, &tv, v_full, kcol0 + 64, (j_lo + j) * BKV, b);
         ++issued_v;
       }
       if (!ok) {
@@ -213,6 +224,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int half = (warp - 2) >> 2;
     const int row = qw * 32 + lane;
     const int qi = qb * BQ + row;
+    // Keys this row sees: [key_lo, key_hi].
+    const int key_hi = min(qi, a.T - 1);
+    const int key_lo = window < 0 ? 0 : qi - window;
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
     const uint32_t s_base = lane_base + TM_S + half * 64;
     const uint32_t o_base = lane_base + TM_O + half * 64;
@@ -224,8 +238,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       ok = tc::mbar_wait(s_full, j & 1, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc::tc_fence_after();
-      const int k0 = j * BKV + half * 64;
-      const bool edge = j * BKV + BKV > qb * BQ || j * BKV + BKV > a.T;  // reaches the diagonal or T
+      const int kt0 = (j_lo + j) * BKV;  // first key of the tile
+      const int k0 = kt0 + half * 64;
+      // The tile reaches the diagonal, T, or below the window of some row.
+      const bool edge = kt0 + BKV > min(qb * BQ, a.T) ||
+                        (window >= 0 && kt0 + window < qb * BQ + BQ - 1);
       // This half's 64 scores, read once; masked ones become -inf.
       uint32_t r[2][32];
       tc::tmem_ld_32x32b_x32(s_base, r[0]);
@@ -237,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const int kj = k0 + c2 * 32 + i;
-            if (kj > qi || kj >= a.T) r[c2][i] = __float_as_uint(-INFINITY);
+            if (kj > key_hi || kj < key_lo) r[c2][i] = __float_as_uint(-INFINITY);
           }
       }
       // Block maximum of the raw scores (the scale is positive): eight
@@ -383,6 +400,8 @@ constexpr uint32_t TB_S = 0, TB_DP = 64, TB_DQ = 128, TB_DV = 256, TB_DK = 384;
 
 struct BwdArgs {
   int T, H, nkb, nqb;
+  int group;   // query heads per KV head
+  int window;  // query t sees keys [t - window, t]; < 0: every key up to t
   float sl2, scale;
   const float* lse;
   const float* delta;
@@ -420,10 +439,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int kb = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;  // hk: the KV head
   const int i0 = (kb * BKV) / BQB;
-  const int nblk = a.nqb - i0;  // query tiles at or after this key tile
-  const int col0 = h * HD;
+  // Query tiles at or after this key tile, up to the last one a window reaches;
+  // every query head of the KV head's group in turn (tile t: head
+  // hk * group + t / nqt, query tile i0 + t % nqt), so dK and dV accumulate
+  // over the whole group in TMEM.
+  const int i_hi = a.window < 0 ? a.nqb - 1 : min(a.nqb - 1, (kb * BKV + BKV - 1 + a.window) / BQB);
+  const int nqt = i_hi - i0 + 1;
+  const int nblk = a.group * nqt;
+  const int kcol0 = hk * HD;
 
   if (threadIdx.x == 0) {
     tc::mbar_init(kv_full, 1);
@@ -456,8 +481,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (warp == 0) {
     // Lane 0 issues the TMA copies; all 32 lanes stage lse * log2(e) and D of
     // the query tile into shared memory and arrive on the same barrier.
-    const float* lse_bh = a.lse + ((int64_t)b * a.H + h) * a.T;
-    const float* d_bh = a.delta + ((int64_t)b * a.H + h) * a.T;
     if (lane == 0) {
       tc::tma_prefetch_desc(&tq);
       tc::tma_prefetch_desc(&tk);
@@ -465,8 +488,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc::tma_prefetch_desc(&tdo);
       tc::mbar_arrive_expect_tx(kv_full, 2 * TILE);
       for (int c = 0; c < 2; ++c) {
-        tc::tma_load_3d(smem + B_OFF_K + c * (TILE / 2), &tk, kv_full, col0 + 64 * c, kb * BKV, b);
-        tc::tma_load_3d(smem + B_OFF_V + c * (TILE / 2), &tv, kv_full, col0 + 64 * c, kb * BKV, b);
+        tc::tma_load_3d(smem + B_OFF_K + c * (TILE / 2), &tk, kv_full, kcol0 + 64 * c, kb * BKV, b);
+        tc::tma_load_3d(smem + B_OFF_V + c * (TILE / 2), &tv, kv_full, kcol0 + 64 * c, kb * BKV, b);
       }
     }
     int issued = 0;
@@ -477,7 +500,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       bool w = true;
       if (lane == 0) w = tc::mbar_wait(&qd_empty[st], ph ^ 1, abort_flag, a.status);
       if (!__shfl_sync(0xffffffffu, (int)w, 0)) { ok = false; break; }
-      const int q0 = (i0 + t) * BQB;
+      const int hq = hk * a.group + t / nqt;
+      const int q0 = (i0 + t % nqt) * BQB;
+      const int qcol0 = hq * HD;
+      const float* lse_bh = a.lse + ((int64_t)b * a.H + hq) * a.T;
+      const float* d_bh = a.delta + ((int64_t)b * a.H + hq) * a.T;
       float* ld = reinterpret_cast<float*>(smem + B_OFF_LD) + st * 2 * BQB;
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
@@ -489,8 +516,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (lane == 0) {
         tc::mbar_arrive_expect_tx(&qd_full[st], 2 * QT);
         for (int c = 0; c < 2; ++c) {
-          tc::tma_load_3d(smem + B_OFF_Q + st * QT + c * (QT / 2), &tq, &qd_full[st], col0 + 64 * c, q0, b);
-          tc::tma_load_3d(smem + B_OFF_DO + st * QT + c * (QT / 2), &tdo, &qd_full[st], col0 + 64 * c, q0, b);
+          tc::tma_load_3d(smem + B_OFF_Q + st * QT + c * (QT / 2), &tq, &qd_full[st], qcol0 + 64 * c, q0, b);
+          tc::tma_load_3d(smem + B_OFF_DO + st * QT + c * (QT / 2), &tdo, &qd_full[st], qcol0 + 64 * c, q0, b);
         }
       } else {
         tc::mbar_arrive(&qd_full[st]);
@@ -580,7 +607,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t ds_row = tc::smem_u32(smem + B_OFF_DS) + row * 128;
     bool ok = true;
     for (int t = 0; t < nblk; ++t) {
-      const int q0 = (i0 + t) * BQB + 32 * ch;
+      const int q0 = (i0 + t % nqt) * BQB + 32 * ch;
       const float* ld = reinterpret_cast<const float*>(smem + B_OFF_LD) + (t % QST) * 2 * BQB + 32 * ch;
       ok = tc::mbar_wait(sdp_full, t & 1, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
@@ -596,15 +623,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = tc::mbar_wait(&qd_full[t % QST], (t / QST) & 1, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       uint32_t pp[16], pd[16];
-      const bool edge = (q0 < key + 1) || (q0 + 32 > a.T) || (key >= a.T);
+      const bool edge = (q0 < key + 1) || (q0 + 32 > a.T) || (key >= a.T) ||
+                        (a.window >= 0 && q0 + 31 > key + a.window);  // diagonal, T or window
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
         float p0 = ex2(__uint_as_float(sv[2 * c]) * a.sl2 - ld[2 * c]);
         float p1 = ex2(__uint_as_float(sv[2 * c + 1]) * a.sl2 - ld[2 * c + 1]);
         if (edge) {
           const int qa = q0 + 2 * c, qb2 = qa + 1;
-          if (qa < key || qa >= a.T || key >= a.T) p0 = 0.f;
-          if (qb2 < key || qb2 >= a.T || key >= a.T) p1 = 0.f;
+          if (qa < key || qa >= a.T || key >= a.T || (a.window >= 0 && qa > key + a.window)) p0 = 0.f;
+          if (qb2 < key || qb2 >= a.T || key >= a.T || (a.window >= 0 && qb2 > key + a.window)) p1 = 0.f;
         }
         const float d0 = p0 * (__uint_as_float(dp[2 * c]) - ld[BQB + 2 * c]);
         const float d1 = p1 * (__uint_as_float(dp[2 * c + 1]) - ld[BQB + 2 * c + 1]);
@@ -629,7 +657,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (ok) {
       // Warps of column half 0 write dV rows, those of half 1 dK rows.
       tc::tc_fence_after();
-      const int64_t grow = ((int64_t)b * a.T + key) * a.ldg + col0;
+      const int64_t grow = ((int64_t)b * a.T + key) * a.ldg + kcol0;
       const uint32_t base = lane_base + (ch ? TB_DK : TB_DV);
       const float mul = ch ? a.scale : 1.f;
       __nv_bfloat16* dst = (ch ? a.dk : a.dv) + grow;
@@ -657,9 +685,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int dim = qw * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
     const int64_t dq_row = (int64_t)a.H * HD;
-    float* dq_bh = a.dq + (int64_t)b * a.T * dq_row + col0 + dim;
     for (int t = 0; t < nblk; ++t) {
-      const int q0 = (i0 + t) * BQB;
+      const int q0 = (i0 + t % nqt) * BQB;
+      float* dq_bh = a.dq + (int64_t)b * a.T * dq_row + (hk * a.group + t / nqt) * HD + dim;
       bool ok = tc::mbar_wait(&dq_full[t & 1], (t >> 1) & 1, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc::tc_fence_after();
@@ -698,27 +726,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 }  // namespace
 
-nc_status attention_fwd(const void* q, const void* k, const void* v, int64_t ld, void* o,
-                        int64_t ldo, float* lse, int B, int T, int H, int* status, cudaStream_t s,
-                        Profiler* prof) {
-  if (B < 1 || T < 1 || H < 1 || !q || !k || !v || !o || !lse)
-    return fail(NC_ERR_INVALID_ARG, "attention_fwd: bad arguments");
-  if (ld % 8 || ldo % 8 ||
+// Query-key pairs a causal window keeps: sum over t of min(t, window) + 1
+// (every key up to t when window < 0).
+double causal_pairs(int T, int window) {
+  if (window < 0 || window >= T - 1) return (double)T * (T + 1) / 2.0;
+  const double w = window;
+  return (w + 1) * (w + 2) / 2.0 + (T - w - 1) * (w + 1);  // rows t <= w, then rows t > w
+}
+
+nc_status attention_fwd_ex(const void* q, int64_t ldq, const void* k, const void* v, int64_t ldkv,
+                           void* o, int64_t ldo, float* lse, int B, int T, int H, int Hkv,
+                           int window, int* status, cudaStream_t s, Profiler* prof) {
+  if (B < 1 || T < 1 || H < 1 || Hkv < 1 || H % Hkv || !q || !k || !v || !o || !lse)
+    return fail(NC_ERR_INVALID_ARG, "attention_fwd: bad arguments (H must be a multiple of Hkv)");
+  if (ldq % 8 || ldkv % 8 || ldo % 8 ||
       ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
         reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o)) & 15))
     return fail(NC_ERR_INVALID_ARG, "attention_fwd: rows must be 16-byte aligned");
   static bool attr = false;
   if (!attr) {
-    NC_CUDA_TRY(cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     kSmem));
+    NC_CUDA_TRY(cudaFuncSetAttribute(attn_fwd_tc_kernel<false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem));
+    NC_CUDA_TRY(cudaFuncSetAttribute(attn_fwd_tc_kernel<true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem));
     attr = true;
   }
   CUtensorMap mq, mk, mv;
-  const uint64_t cols = (uint64_t)H * HD;
   // Box heights must match the tile sizes the kernel's byte counts assume.
-  if (!make_tmap_bf16_3d(&mq, q, cols, T, B, ld, (int64_t)T * ld, BQ) ||
-      !make_tmap_bf16_3d(&mk, k, cols, T, B, ld, (int64_t)T * ld, BKV) ||
-      !make_tmap_bf16_3d(&mv, v, cols, T, B, ld, (int64_t)T * ld, BKV))
+  if (!make_tmap_bf16_3d(&mq, q, (uint64_t)H * HD, T, B, ldq, (int64_t)T * ldq, BQ) ||
+      !make_tmap_bf16_3d(&mk, k, (uint64_t)Hkv * HD, T, B, ldkv, (int64_t)T * ldkv, BKV) ||
+      !make_tmap_bf16_3d(&mv, v, (uint64_t)Hkv * HD, T, B, ldkv, (int64_t)T * ldkv, BKV))
     return fail(NC_ERR_INVALID_ARG, "attention_fwd: cuTensorMapEncodeTiled rejected q/k/v");
   FwdArgs a;
   a.T = T;
@@ -728,43 +765,57 @@ nc_status attention_fwd(const void* q, const void* k, const void* v, int64_t ld,
   a.ldo = ldo;
   a.lse = lse;
   a.H = H;
+  a.group = H / Hkv;
+  a.window = window < 0 ? -1 : window;
   a.status = status;
-  const double flops = 4.0 * B * H * HD * ((double)T * (T + 1) / 2.0);
+  const double flops = 4.0 * B * H * HD * causal_pairs(T, a.window);
   Probe probe(prof, s, "attn_fwd", flops, 0.0);
   dim3 grid(a.nqb, H, B);
-  attn_fwd_tc_kernel<<<grid, kThreads, kSmem, s>>>(mq, mk, mv, a);
+  if (a.group > 1 || a.window >= 0)
+    attn_fwd_tc_kernel<true><<<grid, kThreads, kSmem, s>>>(mq, mk, mv, a);
+  else
+    attn_fwd_tc_kernel<false><<<grid, kThreads, kSmem, s>>>(mq, mk, mv, a);
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }
 
+nc_status attention_fwd(const void* q, const void* k, const void* v, int64_t ld, void* o,
+                        int64_t ldo, float* lse, int B, int T, int H, int* status, cudaStream_t s,
+                        Profiler* prof) {
+  return attention_fwd_ex(q, ld, k, v, ld, o, ldo, lse, B, T, H, H, -1, status, s, prof);
+}
 
-nc_status attention_bwd_tc(const void* q, const void* k, const void* v, int64_t ld,
-                           const void* dout, int64_t ldo, const float* lse, const float* delta,
-                           float* dq, void* dk, void* dv, int64_t ldg, int B, int T, int H,
-                           int* status, cudaStream_t s, Profiler* prof) {
+
+nc_status attention_bwd_tc_ex(const void* q, int64_t ldq, const void* k, const void* v, int64_t ldkv,
+                              const void* dout, int64_t ldo, const float* lse, const float* delta,
+                              float* dq, void* dk, void* dv, int64_t ldg, int B, int T, int H,
+                              int Hkv, int window, int* status, cudaStream_t s, Profiler* prof) {
   static bool attr = false;
   if (!attr) {
     NC_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc_kernel,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdSmem));
     attr = true;
   }
-  if (ld % 8 || ldo % 8 || ldg % 8 ||
+  if (Hkv < 1 || H % Hkv) return fail(NC_ERR_INVALID_ARG, "attention_bwd: H must be a multiple of Hkv");
+  if (ldq % 8 || ldkv % 8 || ldo % 8 || ldg % 8 ||
       ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
         reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(dout) |
         reinterpret_cast<uintptr_t>(dk) | reinterpret_cast<uintptr_t>(dv)) & 15))
     return fail(NC_ERR_INVALID_ARG, "attention_bwd: rows must be 16-byte aligned");
   CUtensorMap mq, mk, mv, mdo;
-  const uint64_t cols = (uint64_t)H * HD;
-  if (!make_tmap_bf16_3d(&mq, q, cols, T, B, ld, (int64_t)T * ld, BQB) ||
-      !make_tmap_bf16_3d(&mk, k, cols, T, B, ld, (int64_t)T * ld, BKV) ||
-      !make_tmap_bf16_3d(&mv, v, cols, T, B, ld, (int64_t)T * ld, BKV) ||
-      !make_tmap_bf16_3d(&mdo, dout, cols, T, B, ldo, (int64_t)T * ldo, BQB))
+  const uint64_t qcols = (uint64_t)H * HD, kvcols = (uint64_t)Hkv * HD;
+  if (!make_tmap_bf16_3d(&mq, q, qcols, T, B, ldq, (int64_t)T * ldq, BQB) ||
+      !make_tmap_bf16_3d(&mk, k, kvcols, T, B, ldkv, (int64_t)T * ldkv, BKV) ||
+      !make_tmap_bf16_3d(&mv, v, kvcols, T, B, ldkv, (int64_t)T * ldkv, BKV) ||
+      !make_tmap_bf16_3d(&mdo, dout, qcols, T, B, ldo, (int64_t)T * ldo, BQB))
     return fail(NC_ERR_INVALID_ARG, "attention_bwd: cuTensorMapEncodeTiled rejected an operand");
   BwdArgs a;
   a.T = T;
   a.H = H;
   a.nkb = (T + BKV - 1) / BKV;
   a.nqb = (T + BQB - 1) / BQB;
+  a.group = H / Hkv;
+  a.window = window < 0 ? -1 : window;
   a.scale = (float)(1.0 / std::sqrt((double)HD));
   a.sl2 = (float)(1.4426950408889634 / std::sqrt((double)HD));
   a.lse = lse;
@@ -774,12 +825,20 @@ nc_status attention_bwd_tc(const void* q, const void* k, const void* v, int64_t 
   a.dv = static_cast<__nv_bfloat16*>(dv);
   a.ldg = ldg;
   a.status = status;
-  const double flops = 10.0 * B * H * HD * ((double)T * (T + 1) / 2.0);
+  const double flops = 10.0 * B * H * HD * causal_pairs(T, a.window);
   Probe probe(prof, s, "attn_bwd", flops, 0.0);
-  dim3 grid(a.nkb, H, B);
+  dim3 grid(a.nkb, Hkv, B);  // one CTA per key tile and KV head; it loops over the group
   attn_bwd_tc_kernel<<<grid, kBwdThreads, kBwdSmem, s>>>(mq, mk, mv, mdo, a);
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
+}
+
+nc_status attention_bwd_tc(const void* q, const void* k, const void* v, int64_t ld,
+                           const void* dout, int64_t ldo, const float* lse, const float* delta,
+                           float* dq, void* dk, void* dv, int64_t ldg, int B, int T, int H,
+                           int* status, cudaStream_t s, Profiler* prof) {
+  return attention_bwd_tc_ex(q, ld, k, v, ld, dout, ldo, lse, delta, dq, dk, dv, ldg, B, T, H, H, -1,
+                             status, s, prof);
 }
 
 }  // namespace nc

@@ -42,6 +42,21 @@ nc_status attention_bwd_tc(const void* q, const void* k, const void* v, int64_t 
                            const void* dout, int64_t ldo, const float* lse, const float* delta,
                            float* dq, void* dk, void* dv, int64_t ldg, int B, int T, int H,
                            int* status, cudaStream_t s, Profiler* prof);
+// Grouped KV heads (Hkv divides H; q / o / dO / dq rows hold H heads, k / v /
+// dk / dv rows Hkv heads) and a left window (query t sees keys
+// [t - window, t]; < 0: every key up to t).  The calls above are these with
+// Hkv = H, one row stride for q, k and v, and no window.
+nc_status attention_fwd_ex(const void* q, int64_t ldq, const void* k, const void* v, int64_t ldkv,
+                           void* o, int64_t ldo, float* lse, int B, int T, int H, int Hkv,
+                           int window, int* status, cudaStream_t s, Profiler* prof);
+nc_status attention_bwd_ex(const void* q, int64_t ldq, const void* k, const void* v, int64_t ldkv,
+                           const void* o, const void* dout, int64_t ldo, const float* lse,
+                           float* dq, void* dk, void* dv, int64_t ldg, float* delta, int B, int T,
+                           int H, int Hkv, int window, int* status, cudaStream_t s, Profiler* prof);
+nc_status attention_bwd_tc_ex(const void* q, int64_t ldq, const void* k, const void* v, int64_t ldkv,
+                              const void* dout, int64_t ldo, const float* lse, const float* delta,
+                              float* dq, void* dk, void* dv, int64_t ldg, int B, int T, int H,
+                              int Hkv, int window, int* status, cudaStream_t s, Profiler* prof);
 
 nc_status embed_gather(const int32_t* tok, int64_t n, const float* E, int V, int d, float* x,
                        int* status, cudaStream_t s, Profiler* prof);

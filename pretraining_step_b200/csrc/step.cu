@@ -789,6 +789,22 @@ nc_status nc_op_attention_bwd(const void* q, const void* k, const void* v, int64
                        nullptr, static_cast<cudaStream_t>(stream), nullptr);
 }
 
+nc_status nc_op_attention_fwd_ex(const void* q, int64_t ldq, const void* k, const void* v,
+                                 int64_t ldkv, void* o, int64_t ldo, float* lse, int B, int T, int H,
+                                 int Hkv, int window, void* stream) {
+  return attention_fwd_ex(q, ldq, k, v, ldkv, o, ldo, lse, B, T, H, Hkv, window, nullptr,
+                          static_cast<cudaStream_t>(stream), nullptr);
+}
+
+nc_status nc_op_attention_bwd_ex(const void* q, int64_t ldq, const void* k, const void* v,
+                                 int64_t ldkv, const void* o, const void* dout, int64_t ldo,
+                                 const float* lse, float* dq, void* dk, void* dv, int64_t ldg,
+                                 float* delta_scratch, int B, int T, int H, int Hkv, int window,
+                                 void* stream) {
+  return attention_bwd_ex(q, ldq, k, v, ldkv, o, dout, ldo, lse, dq, dk, dv, ldg, delta_scratch, B,
+                          T, H, Hkv, window, nullptr, static_cast<cudaStream_t>(stream), nullptr);
+}
+
 size_t nc_newton_schulz_scratch_bytes(int count, int rows, int cols) {
   if (count < 1 || rows < 1 || cols < 1) return 0;
   const int64_t m = std::min(rows, cols), n = std::max(rows, cols);

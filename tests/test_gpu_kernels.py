@@ -232,6 +232,46 @@ def test_attention_backward(B, T, H):
     assert rel_fro(host(dqkv[:, 2 * d:]), rv.reshape(B * T, d)) < 1e-2
 
 
+@pytest.mark.parametrize("B,T,H,Hkv,window", [(1, 300, 4, 2, 100),   # window inside one tile
+                                               (2, 333, 2, 1, 129),   # just past a tile
+                                               (1, 520, 4, 1, 0),     # self only, one KV head
+                                               (1, 256, 3, 3, -1),    # no window, no groups
+                                               (1, 700, 2, 2, 255)])
+def test_attention_grouped_kv_and_window(B, T, H, Hkv, window):
+    """Causal attention with Hkv KV heads and a left window, forward and
+    backward, against the oracle's grouped / windowed attention."""
+    t = torch()
+    dq_, dkv_ = H * 128, Hkv * 128
+    width = dq_ + 2 * dkv_
+    qkv = inputs.bf16_normal(70 + T + window, (B * T, width))
+    q = qkv[:, :dq_].reshape(B, T, H, 128)
+    k = qkv[:, dq_:dq_ + dkv_].reshape(B, T, Hkv, 128)
+    v = qkv[:, dq_ + dkv_:].reshape(B, T, Hkv, 128)
+    dev = dev_bf16(qkv)
+    o = t.empty(B * T, dq_, dtype=t.bfloat16, device="cuda")
+    lse = t.empty(B, H, T, dtype=t.float32, device="cuda")
+    nc.attention_fwd_ex(dev, width, dev[:, dq_:], dev[:, dq_ + dkv_:], width, o, dq_, lse, B, T, H,
+                        Hkv, window)
+    t.cuda.synchronize()
+    oref, lref = oracle.attention_ex(q, k, v, window=window)
+    assert rel_fro(host(o), oref.reshape(B * T, dq_)) < 5e-3
+    np.testing.assert_allclose(host(lse), lref, rtol=2e-4, atol=2e-4)
+    # Backward from the oracle's O and lse (O rounded to bf16 like the saved activation).
+    o_b = inputs.round_to_bf16(oref.reshape(B * T, dq_).astype(np.float32))
+    dout = inputs.bf16_normal(71 + T, (B * T, dq_))
+    dqf = t.empty(B * T, dq_, dtype=t.float32, device="cuda")
+    dkv = t.zeros(B * T, 2 * dkv_, dtype=t.bfloat16, device="cuda")
+    delta = t.empty(B, H, T, dtype=t.float32, device="cuda")
+    nc.attention_bwd_ex(dev, width, dev[:, dq_:], dev[:, dq_ + dkv_:], width, dev_bf16(o_b),
+                        dev_bf16(dout), dq_, dev_f32(lref.astype(np.float32)), dqf, dkv[:, :dkv_],
+                        dkv[:, dkv_:], 2 * dkv_, delta, B, T, H, Hkv, window)
+    t.cuda.synchronize()
+    rq, rk, rv = oracle.attention_bwd_ex(q, k, v, lref, dout.reshape(B, T, H, 128), window=window)
+    assert rel_fro(host(dqf), rq.reshape(B * T, dq_)) < 1e-2
+    assert rel_fro(host(dkv[:, :dkv_]), rk.reshape(B * T, dkv_)) < 1e-2
+    assert rel_fro(host(dkv[:, dkv_:]), rv.reshape(B * T, dkv_)) < 1e-2
+
+
 def test_attention_full_length_sampled_heads():
     """T = 2048 (the step's sequence length), one batch row, two heads."""
     t = torch()
