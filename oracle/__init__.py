@@ -52,6 +52,14 @@ def lib():
         L.oc_attention_bwd_ex.argtypes = [dp, dp, dp, dp, dp, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                           dp, dp, dp]
+        L.oc_dims_ex.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, i64p]
+        L.oc_param_numel_ex.argtypes = [ctypes.c_int] * 4
+        L.oc_param_numel_ex.restype = ctypes.c_int64
+        L.oc_init_params_ex.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_uint64,
+                                        ctypes.c_int, ctypes.c_void_p]
+        L.oc_gpt_fwd_bwd_ex.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                        ctypes.c_int, ctypes.c_int, dp, ctypes.c_void_p, dp]
         L.oc_adamw_update.argtypes = [dp, dp, dp, dp, ctypes.c_int64, ctypes.c_double,
                                       ctypes.c_double, ctypes.c_double, ctypes.c_double,
                                       ctypes.c_double, ctypes.c_int]
@@ -67,34 +75,45 @@ def _f64(a):
     return np.ascontiguousarray(a, dtype=np.float64)
 
 
-def dims(depth, vocab=32768):
-    out = (ctypes.c_int64 * 6)()
-    if lib().oc_dims(depth, vocab, out) != 0:
-        raise ValueError("invalid depth/vocab")
-    d, H, hd, F, n_t, n_b = list(out)
+def dims(depth, vocab=32768, n_kv_head=0):
+    """Model shape; n_kv_head <= 0 means one KV head per query head."""
+    out = (ctypes.c_int64 * 7)()
+    if lib().oc_dims_ex(depth, vocab, n_kv_head, out) != 0:
+        raise ValueError("invalid depth/vocab/n_kv_head")
+    d, H, hd, F, n_t, n_b, Hkv = list(out)
     return dict(d=d, n_head=H, head_dim=hd, mlp=F, n_tensors=n_t, n_block=n_b, vocab=vocab,
-                depth=depth)
+                depth=depth, n_kv_head=Hkv)
 
 
-def param_shapes(depth, vocab=32768):
-    s = dims(depth, vocab)
+def param_shapes(depth, vocab=32768, n_kv_head=0):
+    s = dims(depth, vocab, n_kv_head)
     d, F, V = s["d"], s["mlp"], vocab
+    dkv = s["n_kv_head"] * s["head_dim"]
     shapes = [(V, d)]
     for _ in range(depth):
-        shapes += [(d, d), (d, d), (d, d), (d, d), (F, d), (d, F)]
+        shapes += [(d, d), (dkv, d), (dkv, d), (d, d), (F, d), (d, F)]
     shapes.append((V, d))
     return shapes
+
+
+def window_pattern(pattern, depth, short):
+    """Per-layer windows from a short/long pattern string such as "SSSL"
+    (guide, section "1. Modelo GPT"): layer l takes pattern[l % len];
+    'S' is a left window of `short` keys, 'L' full causal (-1)."""
+    if not pattern or any(c not in "SL" for c in pattern):
+        raise ValueError("pattern of 'S' and 'L'")
+    return [short if pattern[l % len(pattern)] == "S" else -1 for l in range(depth)]
 
 
 def splitmix64(x):
     return int(lib().oc_splitmix64(ctypes.c_uint64(x & 0xFFFFFFFFFFFFFFFF)))
 
 
-def init_params(depth, vocab=32768, seed=0, spec_zero=True):
-    shapes = param_shapes(depth, vocab)
+def init_params(depth, vocab=32768, seed=0, spec_zero=True, n_kv_head=0):
+    shapes = param_shapes(depth, vocab, n_kv_head)
     arrs = [np.empty(s, dtype=np.float32) for s in shapes]
     ptrs = (ctypes.c_void_p * len(arrs))(*[a.ctypes.data for a in arrs])
-    if lib().oc_init_params(depth, vocab, seed, 1 if spec_zero else 0, ptrs) != 0:
+    if lib().oc_init_params_ex(depth, vocab, n_kv_head, seed, 1 if spec_zero else 0, ptrs) != 0:
         raise ValueError("oc_init_params failed")
     return arrs
 
@@ -170,8 +189,11 @@ def matmul_nt(x, w):
     return y
 
 
-def gpt_fwd_bwd(depth, params, tokens, targets, vocab=32768, grads=True, want_logits=False):
-    """Returns (loss, grads list of float64 arrays or None, logits or None)."""
+def gpt_fwd_bwd(depth, params, tokens, targets, vocab=32768, grads=True, want_logits=False,
+                n_kv_head=0, window=None):
+    """Returns (loss, grads list of float64 arrays or None, logits or None).
+    n_kv_head: grouped KV heads (<= 0: one per query head); window: None
+    (full causal) or one window per layer (negative: full causal)."""
     params = [np.ascontiguousarray(p, dtype=np.float32) for p in params]
     tokens = np.ascontiguousarray(tokens, dtype=np.int32)
     targets = np.ascontiguousarray(targets, dtype=np.int32)
@@ -182,8 +204,14 @@ def gpt_fwd_bwd(depth, params, tokens, targets, vocab=32768, grads=True, want_lo
     gptr = (ctypes.c_void_p * len(params))(*[a.ctypes.data for a in g]) if grads else None
     logits = np.empty((B * T, vocab), dtype=np.float64) if want_logits else None
     lp = _dp(logits) if want_logits else ctypes.cast(None, ctypes.POINTER(ctypes.c_double))
-    rc = lib().oc_gpt_fwd_bwd(depth, vocab, pptr, tokens.ctypes.data, targets.ctypes.data, B, T,
-                              ctypes.byref(loss), gptr, lp)
+    win = None
+    if window is not None:
+        win = np.ascontiguousarray(window, dtype=np.int32)
+        if win.shape != (depth,):
+            raise ValueError("one window per layer")
+    rc = lib().oc_gpt_fwd_bwd_ex(depth, vocab, n_kv_head, win.ctypes.data if win is not None else None,
+                                 pptr, tokens.ctypes.data, targets.ctypes.data, B, T,
+                                 ctypes.byref(loss), gptr, lp)
     if rc == -2:
         raise ValueError("token id out of range")
     if rc != 0:
@@ -215,5 +243,5 @@ def adamw_update(W, m, v, g, lr, b1, b2, eps, wd, t):
     return W, m, v
 
 
-def param_numel(depth, idx, vocab=32768):
-    return int(lib().oc_param_numel(depth, vocab, idx))
+def param_numel(depth, idx, vocab=32768, n_kv_head=0):
+    return int(lib().oc_param_numel_ex(depth, vocab, n_kv_head, idx))

@@ -31,7 +31,7 @@ constexpr int kNsSteps = 5;
 constexpr double kNsEps = 1e-7;      // Frobenius-normalisation eps (reading)
 
 struct Dims {
-  int L, d, H, hd, F, V;
+  int L, d, H, hd, F, V, Hkv;
 };
 
 bool make_dims(int depth, int vocab, Dims* s) {
@@ -43,6 +43,19 @@ bool make_dims(int depth, int vocab, Dims* s) {
   s->H = s->d / s->hd;
   s->F = 4 * s->d;
   s->V = vocab;
+  s->Hkv = s->H;
+  return true;
+}
+
+// Grouped KV heads (guide, section "1. Modelo GPT": "GQA: atencao com menos
+// heads KV"): n_kv_head <= 0 keeps one KV head per query head; otherwise it
+// must divide n_head.  wk and wv then have n_kv_head * head_dim rows.
+bool make_dims_kv(int depth, int vocab, int n_kv_head, Dims* s) {
+  if (!make_dims(depth, vocab, s)) return false;
+  if (n_kv_head > 0) {
+    if (n_kv_head > s->H || s->H % n_kv_head) return false;
+    s->Hkv = n_kv_head;
+  }
   return true;
 }
 
@@ -52,6 +65,7 @@ int64_t numel_of(const Dims& s, int idx) {
   if (idx == 0 || idx == n - 1) return (int64_t)s.V * s.d;
   const int j = (idx - 1) % 6;
   if (j == 4 || j == 5) return (int64_t)s.F * s.d;
+  if (j == 1 || j == 2) return (int64_t)s.Hkv * s.hd * s.d;
   return (int64_t)s.d * s.d;
 }
 
@@ -387,17 +401,34 @@ int oc_dims(int depth, int vocab, int64_t* out) {
   return 0;
 }
 
-int64_t oc_param_numel(int depth, int vocab, int idx) {
+int oc_dims_ex(int depth, int vocab, int n_kv_head, int64_t* out) {
   Dims s;
-  if (!make_dims(depth, vocab, &s)) return -1;
+  if (!out || !make_dims_kv(depth, vocab, n_kv_head, &s)) return -1;
+  oc_dims(depth, vocab, out);
+  out[6] = s.Hkv;
+  return 0;
+}
+
+int64_t oc_param_numel(int depth, int vocab, int idx) {
+  return oc_param_numel_ex(depth, vocab, 0, idx);
+}
+
+int64_t oc_param_numel_ex(int depth, int vocab, int n_kv_head, int idx) {
+  Dims s;
+  if (!make_dims_kv(depth, vocab, n_kv_head, &s)) return -1;
   return numel_of(s, idx);
 }
 
 uint64_t oc_splitmix64(uint64_t x) { return splitmix64(x); }
 
 int oc_init_params(int depth, int vocab, uint64_t seed, int spec_zero, float* const* params) {
+  return oc_init_params_ex(depth, vocab, 0, seed, spec_zero, params);
+}
+
+int oc_init_params_ex(int depth, int vocab, int n_kv_head, uint64_t seed, int spec_zero,
+                      float* const* params) {
   Dims s;
-  if (!params || !make_dims(depth, vocab, &s)) return -1;
+  if (!params || !make_dims_kv(depth, vocab, n_kv_head, &s)) return -1;
   const int n_t = 6 * s.L + 2;
   const double two_pi = 6.283185307179586476925286766559;
   for (int t = 0; t < n_t; ++t) {
@@ -486,11 +517,22 @@ int oc_matmul_nt(const double* x, const double* w, int64_t rows, int64_t n, int6
 int oc_gpt_fwd_bwd(int depth, int vocab, const float* const* params, const int32_t* tokens,
                    const int32_t* targets, int B, int T, double* loss, double* const* grads,
                    double* logits) {
+  return oc_gpt_fwd_bwd_ex(depth, vocab, 0, nullptr, params, tokens, targets, B, T, loss, grads,
+                           logits);
+}
+
+int oc_gpt_fwd_bwd_ex(int depth, int vocab, int n_kv_head, const int32_t* window,
+                      const float* const* params, const int32_t* tokens, const int32_t* targets,
+                      int B, int T, double* loss, double* const* grads, double* logits) {
   Dims s;
-  if (!params || !tokens || !targets || !loss || B < 1 || T < 1 || !make_dims(depth, vocab, &s))
+  if (!params || !tokens || !targets || !loss || B < 1 || T < 1 ||
+      !make_dims_kv(depth, vocab, n_kv_head, &s))
     return -1;
-  const int L = s.L, d = s.d, H = s.H, hd = s.hd, F = s.F, V = s.V;
+  const int L = s.L, d = s.d, H = s.H, hd = s.hd, F = s.F, V = s.V, Hkv = s.Hkv;
+  const int dkv = Hkv * hd;  // width of k and v
   const int64_t N = (int64_t)B * T;
+  // Window of layer l: keys t - win(l) .. t (negative: every key up to t).
+  auto win = [&](int l) { return window ? window[l] : -1; };
   for (int64_t n = 0; n < N; ++n)
     if (tokens[n] < 0 || tokens[n] >= V || targets[n] < 0 || targets[n] >= V) return -2;
   const float* wte = params[0];
@@ -498,11 +540,11 @@ int oc_gpt_fwd_bwd(int depth, int vocab, const float* const* params, const int32
   auto W = [&](int l, int j) { return params[1 + 6 * l + j]; };
 
   typedef std::vector<double> vec;
-  const int64_t Nd = N * d, NF = N * F, NH = N * H;
+  const int64_t Nd = N * d, NF = N * F, NH = N * H, Nkv = N * dkv, NHkv = N * Hkv;
   // Saved forward state per layer.
   std::vector<vec> xin(L, vec(Nd)), h1(L, vec(Nd)), r1(L, vec(N)), qr(L, vec(Nd)),
-      kr(L, vec(Nd)), rq(L, vec(NH)), rk(L, vec(NH)), qn(L, vec(Nd)), kn(L, vec(Nd)),
-      vv(L, vec(Nd)), ao(L, vec(Nd)), lse(L, vec(NH)), xmid(L, vec(Nd)), h2(L, vec(Nd)),
+      kr(L, vec(Nkv)), rq(L, vec(NH)), rk(L, vec(NHkv)), qn(L, vec(Nd)), kn(L, vec(Nkv)),
+      vv(L, vec(Nkv)), ao(L, vec(Nd)), lse(L, vec(NH)), xmid(L, vec(Nd)), h2(L, vec(Nd)),
       r2(L, vec(N)), uu(L, vec(NF)), aa(L, vec(NF));
   vec x(Nd), tmp(Nd);
 
@@ -514,21 +556,24 @@ int oc_gpt_fwd_bwd(int depth, int vocab, const float* const* params, const int32
     xin[l] = x;
     for (int64_t n = 0; n < N; ++n) rms_row(&x[n * d], d, &h1[l][n * d], &r1[l][n]);
     mm_nt(h1[l].data(), W(l, 0), N, d, d, qr[l].data());
-    mm_nt(h1[l].data(), W(l, 1), N, d, d, kr[l].data());
-    mm_nt(h1[l].data(), W(l, 2), N, d, d, vv[l].data());
+    mm_nt(h1[l].data(), W(l, 1), N, dkv, d, kr[l].data());
+    mm_nt(h1[l].data(), W(l, 2), N, dkv, d, vv[l].data());
     // RoPE, then RMSNorm over each head (QK normalisation).
     for (int64_t n = 0; n < N; ++n) {
       const int64_t pos = n % T;
       for (int hh = 0; hh < H; ++hh) {
         const int64_t off = n * d + (int64_t)hh * hd;
         rope_row(&qr[l][off], hd, pos, kRopeBase, +1);
-        rope_row(&kr[l][off], hd, pos, kRopeBase, +1);
         rms_row(&qr[l][off], hd, &qn[l][off], &rq[l][n * H + hh]);
-        rms_row(&kr[l][off], hd, &kn[l][off], &rk[l][n * H + hh]);
+      }
+      for (int hh = 0; hh < Hkv; ++hh) {
+        const int64_t off = n * dkv + (int64_t)hh * hd;
+        rope_row(&kr[l][off], hd, pos, kRopeBase, +1);
+        rms_row(&kr[l][off], hd, &kn[l][off], &rk[l][n * Hkv + hh]);
       }
     }
-    attention_fwd(qn[l].data(), kn[l].data(), vv[l].data(), B, T, H, hd, ao[l].data(),
-                  lse[l].data(), nullptr);
+    attention_fwd_gw(qn[l].data(), kn[l].data(), vv[l].data(), B, T, H, Hkv, hd, win(l),
+                     ao[l].data(), lse[l].data());
     mm_nt(ao[l].data(), W(l, 3), N, d, d, tmp.data());
     for (int64_t i = 0; i < Nd; ++i) x[i] += tmp[i];
     xmid[l] = x;
@@ -574,7 +619,7 @@ int oc_gpt_fwd_bwd(int depth, int vocab, const float* const* params, const int32
   mm_nn_acc(dz.data(), wlm, N, V, d, dhf.data(), false);
   for (int64_t n = 0; n < N; ++n) rms_row_bwd_acc(&dhf[n * d], &x[n * d], rf[n], d, &dx[n * d]);
 
-  vec da(NF), du(NF), dh(Nd), dxm(Nd), dao(Nd), dqn(Nd), dkn(Nd), dvv(Nd), dq(Nd), dk(Nd);
+  vec da(NF), du(NF), dh(Nd), dxm(Nd), dao(Nd), dqn(Nd), dkn(Nkv), dvv(Nkv), dq(Nd), dk(Nkv);
   for (int l = L - 1; l >= 0; --l) {
     // x_out = xmid + a W_down^T
     mm_tn(dx.data(), aa[l].data(), N, d, F, grads[1 + 6 * l + 5]);
@@ -588,8 +633,8 @@ int oc_gpt_fwd_bwd(int depth, int vocab, const float* const* params, const int32
     // xmid = xin + o W_o^T
     mm_tn(dxm.data(), ao[l].data(), N, d, d, grads[1 + 6 * l + 3]);
     mm_nn_acc(dxm.data(), W(l, 3), N, d, d, dao.data(), false);
-    attention_bwd(qn[l].data(), kn[l].data(), vv[l].data(), lse[l].data(), dao.data(), B, T, H,
-                  hd, dqn.data(), dkn.data(), dvv.data());
+    attention_bwd_gw(qn[l].data(), kn[l].data(), vv[l].data(), lse[l].data(), dao.data(), B, T,
+                     H, Hkv, hd, win(l), dqn.data(), dkn.data(), dvv.data());
     // Through QK-norm, then RoPE (its transpose is the rotation by -theta).
     std::fill(dq.begin(), dq.end(), 0.0);
     std::fill(dk.begin(), dk.end(), 0.0);
@@ -598,17 +643,20 @@ int oc_gpt_fwd_bwd(int depth, int vocab, const float* const* params, const int32
       for (int hh = 0; hh < H; ++hh) {
         const int64_t off = n * d + (int64_t)hh * hd;
         rms_row_bwd_acc(&dqn[off], &qr[l][off], rq[l][n * H + hh], hd, &dq[off]);
-        rms_row_bwd_acc(&dkn[off], &kr[l][off], rk[l][n * H + hh], hd, &dk[off]);
         rope_row(&dq[off], hd, pos, kRopeBase, -1);
+      }
+      for (int hh = 0; hh < Hkv; ++hh) {
+        const int64_t off = n * dkv + (int64_t)hh * hd;
+        rms_row_bwd_acc(&dkn[off], &kr[l][off], rk[l][n * Hkv + hh], hd, &dk[off]);
         rope_row(&dk[off], hd, pos, kRopeBase, -1);
       }
     }
     mm_tn(dq.data(), h1[l].data(), N, d, d, grads[1 + 6 * l + 0]);
-    mm_tn(dk.data(), h1[l].data(), N, d, d, grads[1 + 6 * l + 1]);
-    mm_tn(dvv.data(), h1[l].data(), N, d, d, grads[1 + 6 * l + 2]);
+    mm_tn(dk.data(), h1[l].data(), N, dkv, d, grads[1 + 6 * l + 1]);
+    mm_tn(dvv.data(), h1[l].data(), N, dkv, d, grads[1 + 6 * l + 2]);
     mm_nn_acc(dq.data(), W(l, 0), N, d, d, dh.data(), false);
-    mm_nn_acc(dk.data(), W(l, 1), N, d, d, dh.data(), true);
-    mm_nn_acc(dvv.data(), W(l, 2), N, d, d, dh.data(), true);
+    mm_nn_acc(dk.data(), W(l, 1), N, dkv, d, dh.data(), true);
+    mm_nn_acc(dvv.data(), W(l, 2), N, dkv, d, dh.data(), true);
     dx = dxm;
     for (int64_t n = 0; n < N; ++n)
       rms_row_bwd_acc(&dh[n * d], &xin[l][n * d], r1[l][n], d, &dx[n * d]);

@@ -33,8 +33,8 @@
  * Parameter layout (the interface both sides follow, in this order):
  *   0            wte     [V, d]        token embedding
  *   1 + 6l + 0   wq_l    [d, d]
- *   1 + 6l + 1   wk_l    [d, d]
- *   1 + 6l + 2   wv_l    [d, d]
+ *   1 + 6l + 1   wk_l    [d, d]        ([n_kv_head * head_dim, d] in the
+ *   1 + 6l + 2   wv_l    [d, d]         grouped-KV variant, the *_ex calls)
  *   1 + 6l + 3   wo_l    [d, d]
  *   1 + 6l + 4   wup_l   [4d, d]
  *   1 + 6l + 5   wdown_l [d, 4d]
@@ -61,6 +61,14 @@ int oc_dims(int depth, int vocab, int64_t* out);
 /* Number of elements of parameter tensor `idx` (layout above), -1 if out of range. */
 int64_t oc_param_numel(int depth, int vocab, int idx);
 
+/* Variant with grouped KV heads (guide, section "1. Modelo GPT": "GQA:
+ * atencao com menos heads KV").  n_kv_head <= 0 means one KV head per
+ * query head (the calls above); otherwise it must divide n_head, and wk,
+ * wv have n_kv_head * head_dim rows.  oc_dims_ex also writes
+ * out[6] = n_kv_head.  Same return values as above. */
+int oc_dims_ex(int depth, int vocab, int n_kv_head, int64_t* out);
+int64_t oc_param_numel_ex(int depth, int vocab, int n_kv_head, int idx);
+
 /* SplitMix64 mixing function (Steele, Lea & Flood, OOPSLA 2014), exposed
  * so its published test values can be checked. */
 uint64_t oc_splitmix64(uint64_t x);
@@ -75,6 +83,10 @@ uint64_t oc_splitmix64(uint64_t x);
  * spec_zero == 0: every tensor is random, lm_head with std 1/sqrt(d).
  * params[i] points to caller-owned float storage of oc_param_numel(i). */
 int oc_init_params(int depth, int vocab, uint64_t seed, int spec_zero, float* const* params);
+/* Same draw for the grouped-KV layout: tensor t takes the first
+ * oc_param_numel_ex(t) numbers of its stream. */
+int oc_init_params_ex(int depth, int vocab, int n_kv_head, uint64_t seed, int spec_zero,
+                      float* const* params);
 
 /* Parameter-free RMSNorm over rows: y = x / sqrt(mean(x^2) + eps). rstd may be NULL. */
 int oc_rmsnorm(const double* x, int64_t rows, int cols, double eps, double* y, double* rstd);
@@ -120,6 +132,17 @@ int oc_matmul_nt(const double* x, const double* w, int64_t rows, int64_t n, int6
 int oc_gpt_fwd_bwd(int depth, int vocab, const float* const* params, const int32_t* tokens,
                    const int32_t* targets, int B, int T, double* loss, double* const* grads,
                    double* logits);
+
+/* Same model with grouped KV heads and a window per layer (guide, section
+ * "1. Modelo GPT": fewer KV heads; short and long context alternating
+ * across layers, e.g. "SSSL", through the window_size of the attention
+ * call).  Layer l attends with oc_attention_ex's window window[l] (negative:
+ * full causal); window == NULL is full causal everywhere.  Query head h
+ * reads KV head h / (n_head / n_kv_head).  With n_kv_head <= 0 and
+ * window == NULL this is oc_gpt_fwd_bwd. */
+int oc_gpt_fwd_bwd_ex(int depth, int vocab, int n_kv_head, const int32_t* window,
+                      const float* const* params, const int32_t* tokens, const int32_t* targets,
+                      int B, int T, double* loss, double* const* grads, double* logits);
 
 /* Newton-Schulz orthogonalisation of one matrix G [rows, cols]:
  * X = G / (||G||_F + eps_norm), then `steps` iterations of the quintic in

@@ -74,26 +74,28 @@ def round_to_bf16(a):
     return r.astype(np.uint32).view(np.float32).reshape(a.shape)
 
 
-def param_shapes(depth, vocab=32768):
+def param_shapes(depth, vocab=32768, n_kv_head=0):
     """Shapes of the 6*depth + 2 parameter tensors, in interface order:
     wte [V, d]; per layer wq, wk, wv, wo [d, d], wup [4d, d], wdown [d, 4d];
-    lm_head [V, d].  d = 64 * depth."""
+    lm_head [V, d].  d = 64 * depth.  With n_kv_head > 0, wk and wv have
+    n_kv_head * head_dim rows (head_dim = min(128, d))."""
     d = 64 * depth
     F = 4 * d
+    dkv = n_kv_head * min(128, d) if n_kv_head > 0 else d
     shapes = [(vocab, d)]
     for _ in range(depth):
-        shapes += [(d, d), (d, d), (d, d), (d, d), (F, d), (d, F)]
+        shapes += [(d, d), (dkv, d), (dkv, d), (d, d), (F, d), (d, F)]
     shapes.append((vocab, d))
     return shapes
 
 
-def random_params(depth, seed, vocab=32768, head_std=None, bf16_exact=True):
+def random_params(depth, seed, vocab=32768, head_std=None, bf16_exact=True, n_kv_head=0):
     """Every tensor drawn N(0, 1/fan_in) (embedding std 1; lm_head std
     head_std, default 1/sqrt(d)), from numpy's PCG64 with the given seed.
     With bf16_exact the values are rounded to bf16 so both sides see the
     same numbers."""
     rng = np.random.default_rng(seed)
-    shapes = param_shapes(depth, vocab)
+    shapes = param_shapes(depth, vocab, n_kv_head)
     d = 64 * depth
     out = []
     for i, (r, c) in enumerate(shapes):

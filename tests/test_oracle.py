@@ -580,3 +580,149 @@ def test_head_and_hidden_permutations_leave_loss_unchanged():
     R[1], R[2] = R[1][swap], R[2][swap]
     l2, _, _ = oracle.gpt_fwd_bwd(depth, R, tok, tgt, vocab=V_SMALL, grads=False)
     assert abs(l0 - l2) > 1e-6
+
+
+# ------------------------------------------------ model with grouped KV heads and windows
+# Guide, section "1. Modelo GPT": fewer KV heads (GQA) and a short/long window
+# alternating across layers ("SSSL"); the window is the attention call's
+# window_size.  Reading: query head h reads KV head h // (H / Hkv); a window w
+# lets query t see keys t - w .. t.
+
+def _repeat_kv(P, depth, H, Hkv):
+    """MHA parameters equivalent to grouped ones: KV head g's rows repeated
+    for each query head h with h // (H / Hkv) == g."""
+    Q = [p.copy() for p in P]
+    group = H // Hkv
+    for l in range(depth):
+        for j in (1, 2):
+            w = P[1 + 6 * l + j]
+            Q[1 + 6 * l + j] = np.repeat(w.reshape(Hkv, 128, -1), group, axis=0).reshape(H * 128, -1)
+    return Q
+
+
+def test_model_grouped_kv_equals_repeated_kv_heads():
+    """depth 8: four query heads on two KV heads.  The grouped model equals the
+    multi-head model whose wk / wv repeat each KV head for its group, in loss,
+    logits and every gradient; the KV gradient is the sum over the group.  A
+    mapping h % Hkv instead of h // group fails here."""
+    depth, T, H, Hkv = 8, 6, 4, 2
+    P = inputs.random_params(depth, seed=40, vocab=V_SMALL, head_std=0.5, n_kv_head=Hkv)
+    tok, tgt = inputs.token_batch(41, 2, T, vocab=V_SMALL)
+    lg, Gg, zg = oracle.gpt_fwd_bwd(depth, P, tok, tgt, vocab=V_SMALL, want_logits=True,
+                                    n_kv_head=Hkv)
+    Q = _repeat_kv(P, depth, H, Hkv)
+    lm, Gm, zm = oracle.gpt_fwd_bwd(depth, Q, tok, tgt, vocab=V_SMALL, want_logits=True)
+    assert abs(lg - lm) < 1e-12
+    np.testing.assert_allclose(zg, zm, rtol=0, atol=1e-11)
+    for i, (gg, gm) in enumerate(zip(Gg, Gm)):
+        l, j = (i - 1) // 6, (i - 1) % 6
+        if 1 <= i <= 6 * depth and j in (1, 2):
+            gm = gm.reshape(Hkv, H // Hkv, 128, -1).sum(axis=1).reshape(gg.shape)
+        np.testing.assert_allclose(gg, gm, rtol=1e-9, atol=1e-12 * np.abs(gm).max())
+    # The other mapping (h % Hkv) is a different model.
+    R = [p.copy() for p in Q]
+    for l in range(depth):
+        for j in (1, 2):
+            w = P[1 + 6 * l + j].reshape(Hkv, 128, -1)
+            R[1 + 6 * l + j] = np.concatenate([w] * (H // Hkv), axis=0).reshape(H * 128, -1)
+    lr, _, _ = oracle.gpt_fwd_bwd(depth, R, tok, tgt, vocab=V_SMALL, grads=False)
+    assert abs(lg - lr) > 1e-6
+
+
+def test_model_window_covering_the_row_is_full_causal():
+    depth, T = 4, 9
+    P = inputs.random_params(depth, seed=42, vocab=V_SMALL, head_std=0.5, n_kv_head=1)
+    tok, tgt = inputs.token_batch(43, 1, T, vocab=V_SMALL)
+    l0, G0, _ = oracle.gpt_fwd_bwd(depth, P, tok, tgt, vocab=V_SMALL, n_kv_head=1)
+    l1, G1, _ = oracle.gpt_fwd_bwd(depth, P, tok, tgt, vocab=V_SMALL, n_kv_head=1,
+                                   window=[T - 1, -1, T + 5, T - 1])
+    assert abs(l0 - l1) < 1e-12  # the loss is an OpenMP reduction: order not fixed
+    assert all(np.array_equal(a, b) for a, b in zip(G0, G1))
+    l2, _, _ = oracle.gpt_fwd_bwd(depth, P, tok, tgt, vocab=V_SMALL, n_kv_head=1,
+                                  window=[T - 2, -1, -1, -1], grads=False)
+    assert abs(l2 - l0) > 1e-6  # the last query loses its first key
+
+
+def test_model_window_zero_makes_positions_independent():
+    """With w = 0 every query sees only its own key, so attention returns v and
+    position t's logits depend on token t alone: they equal those of a row of
+    length 1 holding that token (RoPE and the scores drop out)."""
+    depth, T = 4, 7
+    P = inputs.random_params(depth, seed=44, vocab=V_SMALL, head_std=0.5, n_kv_head=1)
+    tok, tgt = inputs.token_batch(45, 1, T, vocab=V_SMALL)
+    _, _, z = oracle.gpt_fwd_bwd(depth, P, tok, tgt, vocab=V_SMALL, grads=False, want_logits=True,
+                                 n_kv_head=1, window=[0] * depth)
+    _, _, z1 = oracle.gpt_fwd_bwd(depth, P, tok.reshape(T, 1), tgt.reshape(T, 1), vocab=V_SMALL,
+                                  grads=False, want_logits=True, n_kv_head=1)
+    np.testing.assert_allclose(z, z1, rtol=0, atol=1e-12)
+
+
+def test_model_window_receptive_field_is_depth_times_window():
+    """Windows w in all L layers: position t reads tokens t - L*w .. t.  A token
+    change at p leaves logits beyond p + L*w bit-identical and changes the
+    logits at p + L*w (an off-by-one in the window's edge fails one side).  A
+    full-causal layer among them reaches every later position."""
+    depth, T, w, p = 4, 16, 2, 1
+    P = inputs.random_params(depth, seed=46, vocab=V_SMALL, head_std=0.5, n_kv_head=2)
+    tok, tgt = inputs.token_batch(47, 1, T, vocab=V_SMALL)
+    tok2 = tok.copy()
+    tok2[0, p] = (tok2[0, p] + 1) % V_SMALL
+
+    def z(t, window):
+        return oracle.gpt_fwd_bwd(depth, P, t, tgt, vocab=V_SMALL, grads=False, want_logits=True,
+                                  n_kv_head=2, window=window)[2]
+
+    za, zb = z(tok, [w] * depth), z(tok2, [w] * depth)
+    edge = p + depth * w
+    assert np.array_equal(za[:p], zb[:p])
+    assert np.array_equal(za[edge + 1:], zb[edge + 1:])
+    assert not np.allclose(za[edge], zb[edge], rtol=0, atol=1e-9)
+    pattern = oracle.window_pattern("SSSL", depth, w)
+    assert pattern == [w, w, w, -1]
+    zc, zd = z(tok, pattern), z(tok2, pattern)
+    assert all(not np.allclose(zc[t], zd[t], rtol=0, atol=1e-9) for t in range(p, T))
+
+
+def test_model_grouped_windowed_gradients_central_finite_differences():
+    """Central differences through a depth-4 model with one KV head for two
+    query heads and windows (2, full, 0, 5) at T = 8, every tensor."""
+    depth, T, window = 4, 8, [2, -1, 0, 5]
+    P = inputs.random_params(depth, seed=48, vocab=V_SMALL, head_std=0.5, bf16_exact=False,
+                             n_kv_head=1)
+    tok, tgt = inputs.token_batch(49, 1, T, vocab=V_SMALL)
+    _, G, _ = oracle.gpt_fwd_bwd(depth, P, tok, tgt, vocab=V_SMALL, n_kv_head=1, window=window)
+    rng = np.random.default_rng(50)
+    h = 2.0 ** -12
+    for ti, (p, g) in enumerate(zip(P, G)):
+        scale = np.abs(g).max()
+        # At w = 0 a query sees only its own key: q and k drop out, so wq and
+        # wk of that layer get exactly zero gradient; every other tensor not.
+        dead = 1 <= ti <= 6 * depth and window[(ti - 1) // 6] == 0 and (ti - 1) % 6 in (0, 1)
+        assert (scale == 0) == dead, ti
+        scale = scale if scale > 0 else 1e-6
+        picks = [np.unravel_index(np.argmax(np.abs(g)), g.shape)]
+        picks += [tuple(rng.integers(0, s) for s in g.shape) for _ in range(2)]
+        if ti == 0:
+            picks = [(int(tok[0, j]), int(rng.integers(0, p.shape[1]))) for j in range(2)]
+        for idx in picks:
+            Pp = [q.copy() for q in P]
+            Pm = [q.copy() for q in P]
+            Pp[ti][idx] += np.float32(h)
+            Pm[ti][idx] -= np.float32(h)
+            lp = oracle.gpt_fwd_bwd(depth, Pp, tok, tgt, vocab=V_SMALL, grads=False, n_kv_head=1,
+                                    window=window)[0]
+            lm = oracle.gpt_fwd_bwd(depth, Pm, tok, tgt, vocab=V_SMALL, grads=False, n_kv_head=1,
+                                    window=window)[0]
+            fd = (lp - lm) / (float(Pp[ti][idx]) - float(Pm[ti][idx]))
+            assert abs(fd - g[idx]) <= 2e-5 * scale + 1e-9, (ti, idx, fd, g[idx], scale)
+
+
+def test_model_grouped_kv_shapes_and_bad_counts():
+    s = oracle.dims(8, V_SMALL, n_kv_head=2)
+    assert (s["n_head"], s["n_kv_head"]) == (4, 2)
+    assert oracle.param_shapes(8, V_SMALL, 2)[2] == (256, 512)
+    assert oracle.param_numel(8, 2, V_SMALL, n_kv_head=2) == 256 * 512
+    assert oracle.param_shapes(8, V_SMALL, 2) == inputs.param_shapes(8, V_SMALL, 2)
+    for bad in (3, 5, 8):
+        with pytest.raises(ValueError):
+            oracle.dims(8, V_SMALL, n_kv_head=bad)
