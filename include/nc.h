@@ -88,6 +88,30 @@ typedef struct {
  * Errors: NC_ERR_INVALID_ARG (depth/vocab), NC_ERR_OOM, NC_ERR_CUDA. */
 nc_status nc_gpt_init(int depth, int vocab, uint64_t seed, nc_params** out);
 nc_status nc_gpt_init_ex(int depth, int vocab, uint64_t seed, int flags, nc_params** out);
+
+/* Model variants of the guide's section "1. Modelo GPT": fewer KV heads
+ * ("GQA") and attention windows that alternate short and long context
+ * across layers (the "SSSL" pattern, passed to the attention call as its
+ * window_size).
+ *   n_kv_head: 0 = one KV head per query head (the default model); else it
+ *     must divide n_head = d / 128.  wk and wv then have n_kv_head * 128
+ *     rows, and query head h reads KV head h / (n_head / n_kv_head).
+ *   window: NULL = full causal attention in every layer; else `depth`
+ *     entries (borrowed, read during this call only): layer l lets query t
+ *     see keys t - window[l] .. t; a negative entry is full causal.  A
+ *     pattern string maps to it as layer l taking the pattern's letter
+ *     l % length, 'S' a short window, 'L' full causal.
+ * depth, vocab, seed and flags as for nc_gpt_init_ex.  Errors: as
+ * nc_gpt_init_ex, and NC_ERR_INVALID_ARG for an n_kv_head that does not
+ * divide n_head. */
+typedef struct {
+  int depth, vocab;
+  uint64_t seed;
+  int flags;
+  int n_kv_head;
+  const int32_t* window;
+} nc_model_config;
+nc_status nc_gpt_init_config(const nc_model_config* cfg, nc_params** out);
 void nc_params_free(nc_params* p);
 
 /* Stream all later work of this handle is enqueued on (a cudaStream_t). */
@@ -96,7 +120,9 @@ nc_status nc_set_stream(nc_params* p, void* cuda_stream);
 /* Number of parameter tensors (6*depth + 2) and their descriptors, in the
  * order: wte [V,d]; per layer wq, wk, wv, wo [d,d], wup [4d,d],
  * wdown [d,4d]; lm_head [V,d].  wq, wk, wv of a layer are adjacent in
- * memory (one [3d, d] matrix). */
+ * memory (one [3d, d] matrix).  With n_kv_head set (nc_gpt_init_config),
+ * wk and wv are [128 n_kv_head, d] and the three form one
+ * [d + 256 n_kv_head, d] matrix. */
 int nc_num_tensors(const nc_params* p);
 nc_status nc_tensor_info(const nc_params* p, int idx, nc_tensor_desc* out);
 
@@ -187,12 +213,14 @@ typedef enum {
                             sqrt by sqrt.approx, relative error ~2^-23)     */
   NC_EPI_AXPBY_BF16 = 5, /* D(bf16) = alpha*acc + beta*aux(bf16)              */
   NC_EPI_ACC_F32 = 6,    /* D(f32) += alpha*acc                  (atomic)     */
-  NC_EPI_ROPE_QKNORM = 7 /* fused q|k|v projection: columns [0, 2*H*128) are q
-                            and k heads of 128, rotated by RoPE at position
-                            row % T (pairs i, i + 64) then RMS-normalised per
-                            head, rstd written to rstd_qk[which][row * H + h];
-                            columns from 2*H*128 on (v) are stored as is.
-                            D(bf16).  Needs N = 3*H*128.                    */
+  NC_EPI_ROPE_QKNORM = 7 /* fused q|k|v projection: columns [0, H*128) are H q
+                            heads and [H*128, (H+Hkv)*128) Hkv k heads of
+                            128, rotated by RoPE at position row % T (pairs
+                            i, i + 64) then RMS-normalised per head, rstd
+                            written to rstd_q[row * H + h] and
+                            rstd_k[row * Hkv + h]; the Hkv v heads after them
+                            are stored as is.  D(bf16).  Needs
+                            N = (H + 2*Hkv)*128 (Hkv = H when rope_Hkv is 0). */
 } nc_epilogue;
 
 /* Batched GEMM on the tcgen05 tensor cores, D[b] = epi(op(A[b]) op(B[b])^T):
@@ -218,13 +246,16 @@ typedef struct {
   nc_epilogue epi;
   float alpha, beta;
   int split_k;
-  /* NC_EPI_ROPE_QKNORM only: sequence length T, heads H, cos/sin table
-   * (float2 [>= T][64], theta_i(pos) = pos * 10000^(-i/64)) and the two rstd
-   * outputs (f32 [M * H] each: q then k). */
+  /* NC_EPI_ROPE_QKNORM only: sequence length T, query heads H, cos/sin
+   * table (float2 [>= T][64], theta_i(pos) = pos * 10000^(-i/64)) and the
+   * two rstd outputs (f32 [M * H] for q, [M * Hkv] for k). */
   int rope_T, rope_H;
   const void* rope_tab;
   float* rstd_q;
   float* rstd_k;
+  /* KV heads of the fused projection, 1 <= rope_Hkv <= rope_H; 0 means
+   * rope_H (one KV head per query head). */
+  int rope_Hkv;
 } nc_gemm_desc;
 nc_status nc_op_gemm(const nc_gemm_desc* desc, void* stream);
 

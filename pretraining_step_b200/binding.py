@@ -46,7 +46,13 @@ class GemmDesc(ctypes.Structure):
                 ("epi", ctypes.c_int), ("alpha", ctypes.c_float), ("beta", ctypes.c_float),
                 ("split_k", ctypes.c_int), ("rope_T", ctypes.c_int), ("rope_H", ctypes.c_int),
                 ("rope_tab", ctypes.c_void_p), ("rstd_q", ctypes.c_void_p),
-                ("rstd_k", ctypes.c_void_p)]
+                ("rstd_k", ctypes.c_void_p), ("rope_Hkv", ctypes.c_int)]
+
+
+class ModelConfig(ctypes.Structure):
+    _fields_ = [("depth", ctypes.c_int), ("vocab", ctypes.c_int), ("seed", ctypes.c_uint64),
+                ("flags", ctypes.c_int), ("n_kv_head", ctypes.c_int),
+                ("window", ctypes.c_void_p)]
 
 
 class KernelStat(ctypes.Structure):
@@ -74,6 +80,7 @@ def lib():
     sig = {
         "nc_gpt_init": (ci, [ci, ci, ctypes.c_uint64, ctypes.POINTER(vp)]),
         "nc_gpt_init_ex": (ci, [ci, ci, ctypes.c_uint64, ci, ctypes.POINTER(vp)]),
+        "nc_gpt_init_config": (ci, [ctypes.POINTER(ModelConfig), ctypes.POINTER(vp)]),
         "nc_params_free": (None, [vp]),
         "nc_set_stream": (ci, [vp, vp]),
         "nc_num_tensors": (ci, [vp]),
@@ -144,14 +151,33 @@ def _stream(stream):
 
 
 # ------------------------------------------------------------------ model
-class GPT:
-    """One model (nc_params) and its gradients (nc_grads)."""
+def window_pattern(pattern, depth, short):
+    """Per-layer windows from a short/long pattern such as "SSSL": layer l
+    takes the letter l % len(pattern); 'S' is a left window of `short` keys,
+    'L' full causal (-1)."""
+    if not pattern or any(c not in "SL" for c in pattern):
+        raise ValueError("pattern of 'S' and 'L'")
+    return [short if pattern[l % len(pattern)] == "S" else -1 for l in range(depth)]
 
-    def __init__(self, depth, vocab=32768, seed=0, all_random=False, stream=None):
+
+class GPT:
+    """One model (nc_params) and its gradients (nc_grads).  n_kv_head: KV
+    heads (0: one per query head); window: None or one causal left window
+    per layer (negative: full causal)."""
+
+    def __init__(self, depth, vocab=32768, seed=0, all_random=False, stream=None, n_kv_head=0,
+                 window=None):
         h = vp()
-        _check(lib().nc_gpt_init_ex(depth, vocab, seed,
-                                    NC_INIT_ALL_RANDOM if all_random else NC_INIT_SPEC,
-                                    ctypes.byref(h)))
+        cfg = ModelConfig(depth=depth, vocab=vocab, seed=seed,
+                          flags=NC_INIT_ALL_RANDOM if all_random else NC_INIT_SPEC,
+                          n_kv_head=n_kv_head, window=None)
+        win = None
+        if window is not None:
+            if len(window) != depth:
+                raise ValueError("one window per layer")
+            win = (ctypes.c_int32 * depth)(*[int(w) for w in window])
+            cfg.window = ctypes.cast(win, ctypes.c_void_p)
+        _check(lib().nc_gpt_init_config(ctypes.byref(cfg), ctypes.byref(h)))
         self.h = h
         g = vp()
         st = lib().nc_grads_create(self.h, ctypes.byref(g))
@@ -160,6 +186,7 @@ class GPT:
             _check(st)
         self.g = g
         self.depth, self.vocab = depth, vocab
+        self.n_kv_head, self.window = n_kv_head, None if window is None else list(window)
         if stream is not None:
             self.set_stream(stream)
 

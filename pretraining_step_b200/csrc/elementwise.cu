@@ -331,22 +331,25 @@ __global__ void f32_to_bf16_kernel(const float* __restrict__ in, __nv_bfloat16* 
 }
 
 // ------------------------------------------------------------------ Muon
-// Block matrices of layer l live at l * 12 d^2: wq, wk, wv, wo (d x d) at
-// j * d^2, wup (4d x d) at 4 d^2, wdown (d x 4d) at 8 d^2.
-__device__ __forceinline__ void mat_of(int64_t d, int j, int64_t* off, int64_t* size) {
-  const int64_t d2 = d * d;
-  *off = j < 4 ? j * d2 : (j == 4 ? 4 * d2 : 8 * d2);
-  *size = j < 4 ? d2 : 4 * d2;
+// Block matrices of layer l live at l * (10 d^2 + 2 dkv d), in the order
+// wq (d x d), wk and wv (dkv x d each; dkv = d with one KV head per query
+// head), wo (d x d), wup (4d x d), wdown (d x 4d).
+__device__ __forceinline__ void mat_of(int64_t d, int64_t dkv, int j, int64_t* off,
+                                       int64_t* size) {
+  const int64_t d2 = d * d, kv = dkv * d;
+  *off = j == 0 ? 0 : j == 1 ? d2 : j == 2 ? d2 + kv : j == 3 ? d2 + 2 * kv
+       : j == 4 ? 2 * d2 + 2 * kv : 6 * d2 + 2 * kv;
+  *size = (j == 1 || j == 2) ? kv : (j >= 4 ? 4 * d2 : d2);
 }
 
 // M <- mu*M + G over matrix (blockIdx.y = l*6 + j); sumsq[l*6 + j] += ||M||^2.
 __global__ void muon_momentum_kernel(float* __restrict__ M, const float* __restrict__ G, int d,
-                                     float mu, float* __restrict__ sumsq) {
+                                     int dkv, float mu, float* __restrict__ sumsq) {
   const int mat = blockIdx.y;
   const int l = mat / 6, j = mat % 6;
   int64_t off, size;
-  mat_of(d, j, &off, &size);
-  off += (int64_t)l * 12 * d * d;
+  mat_of(d, dkv, j, &off, &size);
+  off += (int64_t)l * (10ll * d * d + 2ll * dkv * d);
   float4* m4 = reinterpret_cast<float4*>(M + off);
   const float4* g4 = reinterpret_cast<const float4*>(G + off);
   float ss = 0.f;
@@ -572,11 +575,12 @@ nc_status f32_to_bf16(const float* in, void* out, int64_t n, cudaStream_t s, Pro
   return NC_OK;
 }
 
-nc_status muon_momentum(float* M, const float* G, int L, int d, float mu, float* sumsq,
+nc_status muon_momentum(float* M, const float* G, int L, int d, int dkv, float mu, float* sumsq,
                         cudaStream_t s, Profiler* prof) {
-  Probe probe(prof, s, "muon_momentum", 0.0, 12.0 * L * (double)d * d * 12.0);
+  Probe probe(prof, s, "muon_momentum", 0.0,
+              12.0 * L * (10.0 * d * d + 2.0 * dkv * (double)d));
   dim3 grid(64, 6 * L);
-  muon_momentum_kernel<<<grid, 256, 0, s>>>(M, G, d, mu, sumsq);
+  muon_momentum_kernel<<<grid, 256, 0, s>>>(M, G, d, dkv, mu, sumsq);
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }

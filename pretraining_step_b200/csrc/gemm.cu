@@ -58,7 +58,8 @@ struct Args {
   union {
     int64_t stride_d;
     struct {
-      int rope_T, rope_H;
+      int rope_T;
+      int16_t rope_H, rope_Hkv;  // query heads, KV heads
     };
   };
   union {
@@ -318,16 +319,18 @@ __device__ __forceinline__ void stage_store_chunk(const Args& p, uint8_t* slot, 
   __syncwarp();  // the slot may be rewritten by the warp's next chunk
 }
 
-// Fused q|k|v epilogue: this warp's 128 accumulator columns are one head.
-// q and k heads are rotated (pairs i, i + 64, position row % T) and
-// RMS-normalised; v heads are stored as computed.  The rotation preserves
-// the norm of every pair, so a first pass over TMEM takes the head's norm
-// and a second rotates, scales and stores column chunks c and c + 2 together.
+// Fused q|k|v epilogue: this warp's 128 accumulator columns are one head
+// (col0 is a multiple of 128): rope_H q heads, then rope_Hkv k heads, then
+// rope_Hkv v heads.  q and k heads are rotated (pairs i, i + 64, position
+// row % T) and RMS-normalised; v heads are stored as computed.  The rotation
+// preserves the norm of every pair, so a first pass over TMEM takes the
+// head's norm and a second rotates, scales and stores column chunks c and
+// c + 2 together.
 __device__ __forceinline__ void rope_head_epilogue(const Args& p, uint32_t taddr, int b, int row,
                                                    int col0, uint8_t* slot, int lane) {
   const bool live = row < p.M && col0 < p.N;
-  const int d = p.rope_H * 128;
-  const int region = col0 / d;  // 0: q, 1: k, 2: v (uniform across the warp)
+  const int hq = col0 >> 7;  // head index over q|k|v (uniform across the warp)
+  const int region = hq < p.rope_H ? 0 : (hq < p.rope_H + p.rope_Hkv ? 1 : 2);  // q, k, v
   float rs = 1.f;
   if (region < 2) {
     float ss = 0.f;
@@ -343,7 +346,10 @@ __device__ __forceinline__ void rope_head_epilogue(const Args& p, uint32_t taddr
       }
     }
     rs = rsqrtf(ss / 128.f + kNormEps);
-    if (live) (region ? p.rstd_k : p.rstd_q)[(int64_t)row * p.rope_H + (col0 % d) / 128] = rs;
+    if (live) {
+      if (region) p.rstd_k[(int64_t)row * p.rope_Hkv + (hq - p.rope_H)] = rs;
+      else p.rstd_q[(int64_t)row * p.rope_H + hq] = rs;
+    }
   }
   (void)b;  // batch 1: stride_d holds T and H here
   const float4* tab = reinterpret_cast<const float4*>(p.rope_tab + (int64_t)(row % p.rope_T) * 64);
@@ -1019,7 +1025,8 @@ nc_status launch_bn(const nc_gemm_desc& d, int split, int* status, const char* t
   a.stride_aux = d.stride_aux;
   if (d.epi == NC_EPI_ROPE_QKNORM) {  // shares storage with stride_d and the aux fields
     a.rope_T = d.rope_T;
-    a.rope_H = d.rope_H;
+    a.rope_H = (int16_t)d.rope_H;
+    a.rope_Hkv = (int16_t)(d.rope_Hkv > 0 ? d.rope_Hkv : d.rope_H);
     a.rope_tab = static_cast<const float2*>(d.rope_tab);
     a.rstd_q = d.rstd_q;
     a.rstd_k = d.rstd_k;
@@ -1084,7 +1091,8 @@ nc_status launch_pair(const nc_gemm_desc& d, int split, int* status, const char*
   a.stride_aux = d.stride_aux;
   if (d.epi == NC_EPI_ROPE_QKNORM) {  // shares storage with stride_d and the aux fields
     a.rope_T = d.rope_T;
-    a.rope_H = d.rope_H;
+    a.rope_H = (int16_t)d.rope_H;
+    a.rope_Hkv = (int16_t)(d.rope_Hkv > 0 ? d.rope_Hkv : d.rope_H);
     a.rope_tab = static_cast<const float2*>(d.rope_tab);
     a.rstd_q = d.rstd_q;
     a.rstd_k = d.rstd_k;
@@ -1153,9 +1161,11 @@ nc_status gemm_launch(const GemmLaunch& g, cudaStream_t s, Profiler* prof) {
   if (d.epi < NC_EPI_STORE_BF16 || d.epi > NC_EPI_ROPE_QKNORM)
     return fail(NC_ERR_INVALID_ARG, "gemm: unknown epilogue");
   const bool rope = d.epi == NC_EPI_ROPE_QKNORM;
-  if (rope && (d.rope_T < 1 || d.rope_H < 1 || d.N != 3 * 128 * d.rope_H || !d.rope_tab ||
-               !d.rstd_q || !d.rstd_k || d.alpha != 1.f || d.batch != 1))
-    return fail(NC_ERR_INVALID_ARG, "gemm: the RoPE/QK-norm epilogue needs N = 3*128*H, T, a table and rstd outputs");
+  const int rope_kv = d.rope_Hkv > 0 ? d.rope_Hkv : d.rope_H;
+  if (rope && (d.rope_T < 1 || d.rope_H < 1 || d.rope_H > 4096 || rope_kv > d.rope_H ||
+               d.N != 128 * (d.rope_H + 2 * rope_kv) || !d.rope_tab || !d.rstd_q || !d.rstd_k ||
+               d.alpha != 1.f || d.batch != 1))
+    return fail(NC_ERR_INVALID_ARG, "gemm: the RoPE/QK-norm epilogue needs N = 128*(H + 2*Hkv), Hkv <= H, T, a table and rstd outputs");
   int split = d.split_k;
   if (split != 1 && d.epi != NC_EPI_ACC_F32)
     return fail(NC_ERR_INVALID_ARG, "gemm: split_k > 1 needs the accumulate epilogue");

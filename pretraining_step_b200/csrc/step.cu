@@ -6,14 +6,19 @@
 // section "1. Modelo GPT"):  x0 = wte[tok];  per layer
 //   h1 = rms(x);  [q k v] = h1 [wq wk wv]^T;  q, k <- rms_head(rope(.));
 //   o = causal_attention(q, k, v);  x <- x + o wo^T;
+// (k and v have Hkv heads, query head h reading KV head h / (H / Hkv); a
+// layer may attend through a causal left window: the guide's fewer KV heads
+// and short/long window pattern.  The default is Hkv = H, no windows.)
 //   h2 = rms(x);  a = relu(h2 wup^T)^2;  x <- x + a wdown^T;
 // then z = rms(x) lm_head^T and loss = mean(lse(z) - z[target]).
 // Residual stream and every row statistic are fp32; GEMM operands are bf16
 // with fp32 accumulation in TMEM.
 //
 // Memory layout in HBM (one allocation per role):
-//   wte [V,d] f32;  blocks [L][12 d^2] f32 masters + bf16 copies, layer l at
-//   l*12d^2: wq | wk | wv (one [3d,d] matrix) | wo | wup [4d,d] | wdown [d,4d];
+//   wte [V,d] f32;  blocks [L][10 d^2 + 2 dkv d] f32 masters + bf16 copies
+//   (dkv = 128 Hkv; = d by default, 12 d^2 per layer): wq [d,d] | wk [dkv,d]
+//   | wv [dkv,d] (one [d + 2 dkv, d] matrix) | wo [d,d] | wup [4d,d] |
+//   wdown [d,4d];
 //   lm_head [V,d] f32 + bf16;  Muon momentum like blocks (f32).
 //   Activations per B*T tokens: x_0..x_L and the mid-layer residuals (f32),
 //   h1, h2, qkv, o, a (bf16), row statistics (f32), logits [N,V] bf16
@@ -92,6 +97,8 @@ struct Acts {
 
 struct nc_params {
   int depth = 0, vocab = 0, d = 0, H = 0, hd = 0, F = 0;
+  int Hkv = 0, dkv = 0;     // KV heads and the width of k, v (dkv = 128 Hkv)
+  std::vector<int> window;  // per layer: causal left window, -1 = full causal
   cudaStream_t stream = nullptr;
   nc::Profiler* prof = nullptr;
   int* status = nullptr;  // device status word
@@ -102,6 +109,7 @@ struct nc_params {
   // Muon
   float* sumsq = nullptr;
   nc::bf16 *xsq = nullptr, *xw = nullptr, *nsws = nullptr;
+  nc::bf16* xkv = nullptr;  // wk, wv stack when dkv < d (their own Newton-Schulz shape)
   // AdamW state of wte and lm_head (first and second moments, allocated
   // and zeroed by the first nc_adamw_step) and the step count
   float* adam = nullptr;
@@ -124,12 +132,29 @@ struct nc_grads {
 namespace nc {
 namespace {
 
-int64_t block_elems(const nc_params* p) { return 12ll * p->depth * p->d * p->d; }
+// Elements of one layer's block matrices and the offset of matrix j
+// (0..5: wq, wk, wv, wo, wup, wdown) inside it.
+int64_t layer_elems(const nc_params* p) {
+  return 10ll * p->d * p->d + 2ll * p->dkv * p->d;
+}
+int64_t mat_offset(const nc_params* p, int j) {
+  const int64_t d2 = (int64_t)p->d * p->d, kv = (int64_t)p->dkv * p->d;
+  switch (j) {
+    case 0: return 0;
+    case 1: return d2;
+    case 2: return d2 + kv;
+    case 3: return d2 + 2 * kv;
+    case 4: return 2 * d2 + 2 * kv;
+    default: return 6 * d2 + 2 * kv;
+  }
+}
+int64_t block_elems(const nc_params* p) { return p->depth * layer_elems(p); }
+int64_t qkv_width(const nc_params* p) { return (int64_t)p->d + 2ll * p->dkv; }
 
 // Offset and shape of parameter tensor idx (interface order).
 void tensor_layout(const nc_params* p, int idx, int64_t* off, int64_t* rows, int64_t* cols,
                    const char** name, int* layer) {
-  const int64_t d = p->d, d2 = d * d;
+  const int64_t d = p->d;
   const int n = 6 * p->depth + 2;
   *layer = -1;
   if (idx == 0) {
@@ -141,8 +166,8 @@ void tensor_layout(const nc_params* p, int idx, int64_t* off, int64_t* rows, int
     static const char* names[6] = {"wq", "wk", "wv", "wo", "wup", "wdown"};
     *layer = l;
     *name = names[j];
-    *off = l * 12 * d2 + (j < 4 ? j * d2 : (j == 4 ? 4 * d2 : 8 * d2));
-    *rows = (j == 4) ? 4 * d : d;
+    *off = l * layer_elems(p) + mat_offset(p, j);
+    *rows = (j == 4) ? 4 * d : (j == 1 || j == 2) ? p->dkv : d;
     *cols = (j == 5) ? 4 * d : d;
   }
 }
@@ -195,17 +220,17 @@ nc_status ensure_acts(nc_params* p, int B, int T) {
     a = Acts();
   }
   const int L = p->depth;
-  const int64_t d = p->d, F = p->F, V = p->vocab, H = p->H;
+  const int64_t d = p->d, F = p->F, V = p->vocab, H = p->H, Hkv = p->Hkv, Q = qkv_width(p);
   // Sizes in bytes, each rounded to 256.
   auto r = [](int64_t bytes) { return (bytes + 255) & ~int64_t(255); };
   int64_t total = 0;
   total += 2 * r(4 * N);                                     // tok, tgt
   total += (L + 1) * r(4 * N * d) + L * r(4 * N * d);        // x, xmid
-  total += 2 * L * r(4 * N) + 2 * L * r(4 * N * H);          // r1 r2 rq rk
+  total += 2 * L * r(4 * N) + L * r(4 * N * H) + L * r(4 * N * Hkv);  // r1 r2 rq rk
   total += L * r(4 * N * H);                                 // lse [B,H,T]
-  total += 2 * L * r(2 * N * d) + L * r(2 * N * 3 * d) + L * r(2 * N * d) + L * r(2 * N * F);
+  total += 2 * L * r(2 * N * d) + L * r(2 * N * Q) + L * r(2 * N * d) + L * r(2 * N * F);
   total += r(2 * N * d) + r(4 * N) + r(2 * N * V) + r(4 * N) + r(4);  // hf rf logits loss
-  total += 2 * r(4 * N * d) + 2 * r(2 * N * d) + r(2 * N * F) + r(2 * N * 3 * d) +
+  total += 2 * r(4 * N * d) + 2 * r(2 * N * d) + r(2 * N * F) + r(2 * N * Q) +
            r(4 * N * d) + r(4 * N * H);                      // backward scratch
   void* mem = nullptr;
   cudaError_t e = cudaMalloc(&mem, (size_t)total);
@@ -226,11 +251,11 @@ nc_status ensure_acts(nc_params* p, int B, int T) {
     a.r1.push_back(ar.take<float>(N));
     a.r2.push_back(ar.take<float>(N));
     a.rq.push_back(ar.take<float>(N * H));
-    a.rk.push_back(ar.take<float>(N * H));
+    a.rk.push_back(ar.take<float>(N * Hkv));
     a.lse.push_back(ar.take<float>(N * H));
     a.h1.push_back(ar.take<bf16>(N * d));
     a.h2.push_back(ar.take<bf16>(N * d));
-    a.qkv.push_back(ar.take<bf16>(N * 3 * d));
+    a.qkv.push_back(ar.take<bf16>(N * Q));
     a.o.push_back(ar.take<bf16>(N * d));
     a.a.push_back(ar.take<bf16>(N * F));
   }
@@ -244,7 +269,7 @@ nc_status ensure_acts(nc_params* p, int B, int T) {
   a.dxb = ar.take<bf16>(N * d);
   a.dh = ar.take<bf16>(N * d);
   a.du = ar.take<bf16>(N * F);
-  a.dqkv = ar.take<bf16>(N * 3 * d);
+  a.dqkv = ar.take<bf16>(N * Q);
   a.dq = ar.take<float>(N * d);
   a.delta = ar.take<float>(N * H);
   if (ar.used > ar.size) return fail(NC_ERR_CUDA, "activation arena overflow");
@@ -317,8 +342,10 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
   Acts& a = p->act;
   cudaStream_t s = p->stream;
   Profiler* pr = p->prof;
-  const int L = p->depth, H = p->H, hd = p->hd, V = p->vocab;
-  const int64_t N = (int64_t)B * T, d = p->d, F = p->F, d2 = d * d;
+  const int L = p->depth, H = p->H, Hkv = p->Hkv, hd = p->hd, V = p->vocab;
+  const int64_t N = (int64_t)B * T, d = p->d, F = p->F, dkv = p->dkv, Q = qkv_width(p);
+  const int64_t LS = layer_elems(p);
+  const int64_t o_wo = mat_offset(p, 3), o_up = mat_offset(p, 4), o_down = mat_offset(p, 5);
 
   const int32_t* tok = tokens;
   const int32_t* tgt = targets;
@@ -335,28 +362,28 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
   // ---------------- forward
   NC_TRY(embed_gather(tok, N, p->wte, V, (int)d, a.x[0], p->status, s, pr));
   for (int l = 0; l < L; ++l) {
-    const bf16* W = p->blocks_b + l * 12 * d2;
+    const bf16* W = p->blocks_b + l * LS;
     NC_TRY(rmsnorm_fwd(a.x[l], N, (int)d, a.h1[l], a.r1[l], s, pr));
     {
       // q|k|v projection with RoPE + QK-norm fused into the epilogue.
       GemmLaunch g{};
       g.status = p->status;
       g.tag = "gemm_fwd";
-      g.d.M = (int)N; g.d.N = (int)(3 * d); g.d.K = (int)d; g.d.batch = 1;
+      g.d.M = (int)N; g.d.N = (int)Q; g.d.K = (int)d; g.d.batch = 1;
       g.d.A = a.h1[l]; g.d.lda = d; g.d.a_kmajor = 1;
       g.d.B = W; g.d.ldb = d; g.d.b_kmajor = 1;
-      g.d.D = a.qkv[l]; g.d.ldd = 3 * d;
+      g.d.D = a.qkv[l]; g.d.ldd = Q;
       g.d.epi = NC_EPI_ROPE_QKNORM; g.d.alpha = 1.f; g.d.split_k = 1;
-      g.d.rope_T = T; g.d.rope_H = H; g.d.rope_tab = p->rope;
+      g.d.rope_T = T; g.d.rope_H = H; g.d.rope_Hkv = Hkv; g.d.rope_tab = p->rope;
       g.d.rstd_q = a.rq[l]; g.d.rstd_k = a.rk[l];
       NC_TRY(gemm_launch(g, s, pr));
     }
-    NC_TRY(attention_fwd(a.qkv[l], a.qkv[l] + d, a.qkv[l] + 2 * d, 3 * d, a.o[l], d, a.lse[l], B,
-                         T, H, p->status, s, pr));
-    NC_TRY(proj(p, a.o[l], N, d, W + 3 * d2, d, a.xmid[l], d, NC_EPI_RESID_F32, a.x[l], d));
+    NC_TRY(attention_fwd_ex(a.qkv[l], Q, a.qkv[l] + d, a.qkv[l] + d + dkv, Q, a.o[l], d,
+                            a.lse[l], B, T, H, Hkv, p->window[l], p->status, s, pr));
+    NC_TRY(proj(p, a.o[l], N, d, W + o_wo, d, a.xmid[l], d, NC_EPI_RESID_F32, a.x[l], d));
     NC_TRY(rmsnorm_fwd(a.xmid[l], N, (int)d, a.h2[l], a.r2[l], s, pr));
-    NC_TRY(proj(p, a.h2[l], N, d, W + 4 * d2, F, a.a[l], F, NC_EPI_RELU2, nullptr, 0));
-    NC_TRY(proj(p, a.a[l], N, F, W + 8 * d2, d, a.x[l + 1], d, NC_EPI_RESID_F32, a.xmid[l], d));
+    NC_TRY(proj(p, a.h2[l], N, d, W + o_up, F, a.a[l], F, NC_EPI_RELU2, nullptr, 0));
+    NC_TRY(proj(p, a.a[l], N, F, W + o_down, d, a.x[l + 1], d, NC_EPI_RESID_F32, a.xmid[l], d));
   }
   NC_TRY(rmsnorm_fwd(a.x[L], N, (int)d, a.hf, a.rf, s, pr));
   NC_TRY(proj(p, a.hf, N, d, p->lm_b, V, a.logits, V, NC_EPI_STORE_BF16, nullptr, 0,
@@ -372,27 +399,27 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
   float* dxn = a.dx1;
   NC_TRY(rmsnorm_bwd(a.dh, a.x[L], a.rf, nullptr, N, (int)d, dx, a.dxb, s, pr));
   for (int l = L - 1; l >= 0; --l) {
-    const bf16* W = p->blocks_b + l * 12 * d2;
-    float* G = g->blocks + l * 12 * d2;
+    const bf16* W = p->blocks_b + l * LS;
+    float* G = g->blocks + l * LS;
     // MLP: x_out = xmid + a wdown^T, a = relu(h2 wup^T)^2
-    NC_TRY(proj_dw(p, a.dxb, d, d, a.a[l], F, F, N, G + 8 * d2));
-    NC_TRY(proj_dx(p, a.dxb, N, d, W + 8 * d2, F, a.du, F, NC_EPI_RELU2_BWD, a.a[l], F));
-    NC_TRY(proj_dw(p, a.du, F, F, a.h2[l], d, d, N, G + 4 * d2));
-    NC_TRY(proj_dx(p, a.du, N, F, W + 4 * d2, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0));
+    NC_TRY(proj_dw(p, a.dxb, d, d, a.a[l], F, F, N, G + o_down));
+    NC_TRY(proj_dx(p, a.dxb, N, d, W + o_down, F, a.du, F, NC_EPI_RELU2_BWD, a.a[l], F));
+    NC_TRY(proj_dw(p, a.du, F, F, a.h2[l], d, d, N, G + o_up));
+    NC_TRY(proj_dx(p, a.du, N, F, W + o_up, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0));
     NC_TRY(rmsnorm_bwd(a.dh, a.xmid[l], a.r2[l], dx, N, (int)d, dxn, a.dxb, s, pr));
     std::swap(dx, dxn);
     // Attention: xmid = x + o wo^T
-    NC_TRY(proj_dw(p, a.dxb, d, d, a.o[l], d, d, N, G + 3 * d2));
-    NC_TRY(proj_dx(p, a.dxb, N, d, W + 3 * d2, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0));
-    NC_TRY(attention_bwd(a.qkv[l], a.qkv[l] + d, a.qkv[l] + 2 * d, 3 * d, a.o[l], a.dh, d,
-                         a.lse[l], a.dq, a.dqkv + d, a.dqkv + 2 * d, 3 * d, a.delta, B, T, H,
-                         p->status, s, pr));
-    NC_TRY(rope_qknorm_bwd(a.dq, nullptr, 0, a.qkv[l], 3 * d, a.rq[l], N, T, H, hd, p->rope,
-                           a.dqkv, 3 * d, s, pr));
-    NC_TRY(rope_qknorm_bwd(nullptr, a.dqkv + d, 3 * d, a.qkv[l] + d, 3 * d, a.rk[l], N, T, H, hd,
-                           p->rope, a.dqkv + d, 3 * d, s, pr));
-    NC_TRY(proj_dw(p, a.dqkv, 3 * d, 3 * d, a.h1[l], d, d, N, G));
-    NC_TRY(proj_dx(p, a.dqkv, N, 3 * d, W, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0));
+    NC_TRY(proj_dw(p, a.dxb, d, d, a.o[l], d, d, N, G + o_wo));
+    NC_TRY(proj_dx(p, a.dxb, N, d, W + o_wo, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0));
+    NC_TRY(attention_bwd_ex(a.qkv[l], Q, a.qkv[l] + d, a.qkv[l] + d + dkv, Q, a.o[l], a.dh, d,
+                            a.lse[l], a.dq, a.dqkv + d, a.dqkv + d + dkv, Q, a.delta, B, T, H, Hkv,
+                            p->window[l], p->status, s, pr));
+    NC_TRY(rope_qknorm_bwd(a.dq, nullptr, 0, a.qkv[l], Q, a.rq[l], N, T, H, hd, p->rope, a.dqkv,
+                           Q, s, pr));
+    NC_TRY(rope_qknorm_bwd(nullptr, a.dqkv + d, Q, a.qkv[l] + d, Q, a.rk[l], N, T, Hkv, hd,
+                           p->rope, a.dqkv + d, Q, s, pr));
+    NC_TRY(proj_dw(p, a.dqkv, Q, Q, a.h1[l], d, d, N, G));
+    NC_TRY(proj_dx(p, a.dqkv, N, Q, W, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0));
     NC_TRY(rmsnorm_bwd(a.dh, a.x[l], a.r1[l], dx, N, (int)d, dxn, a.dxb, s, pr));
     std::swap(dx, dxn);
   }
@@ -406,24 +433,45 @@ nc_status muon(nc_params* p, const nc_grads* g, float lr, float mu) {
   cudaStream_t s = p->stream;
   Profiler* pr = p->prof;
   const int L = p->depth;
-  const int64_t d = p->d, d2 = d * d;
+  const int64_t d = p->d, d2 = d * d, dkv = p->dkv, kv = dkv * d, LS = layer_elems(p);
   NC_CUDA_TRY(cudaMemsetAsync(p->sumsq, 0, sizeof(float) * 6 * L, s));
-  NC_TRY(muon_momentum(p->mom, g->blocks, L, (int)d, mu, p->sumsq, s, pr));
-  for (int j = 0; j < 4; ++j)
-    NC_TRY(muon_prep(p->mom + j * d2, 12 * d2, (int)d, (int)d, 0, p->xsq + j * d2, 4 * d2,
-                     p->sumsq, j, L, s, pr));
-  NC_TRY(muon_prep(p->mom + 4 * d2, 12 * d2, (int)(4 * d), (int)d, 1, p->xw, 8 * d2, p->sumsq, 4,
-                   L, s, pr));
-  NC_TRY(muon_prep(p->mom + 8 * d2, 12 * d2, (int)d, (int)(4 * d), 0, p->xw + 4 * d2, 8 * d2,
+  NC_TRY(muon_momentum(p->mom, g->blocks, L, (int)d, (int)dkv, mu, p->sumsq, s, pr));
+  // Orthogonalisation stacks by shape: the d x d matrices (wq, wo, and wk, wv
+  // when dkv = d) in xsq; wk, wv as dkv x d in xkv when dkv < d; wup
+  // (transposed) and wdown as d x 4d in xw.  Stacks are [layer][matrix].
+  const bool kv_square = dkv == d;
+  const int n_sq = kv_square ? 4 : 2;
+  const int sq_of[4] = {0, kv_square ? 1 : 3, 2, 3};
+  for (int i = 0; i < n_sq; ++i)
+    NC_TRY(muon_prep(p->mom + mat_offset(p, sq_of[i]), LS, (int)d, (int)d, 0, p->xsq + i * d2,
+                     n_sq * d2, p->sumsq, sq_of[i], L, s, pr));
+  if (!kv_square)
+    for (int i = 0; i < 2; ++i)
+      NC_TRY(muon_prep(p->mom + mat_offset(p, 1 + i), LS, (int)dkv, (int)d, 0, p->xkv + i * kv,
+                       2 * kv, p->sumsq, 1 + i, L, s, pr));
+  NC_TRY(muon_prep(p->mom + mat_offset(p, 4), LS, (int)(4 * d), (int)d, 1, p->xw, 8 * d2,
+                   p->sumsq, 4, L, s, pr));
+  NC_TRY(muon_prep(p->mom + mat_offset(p, 5), LS, (int)d, (int)(4 * d), 0, p->xw + 4 * d2, 8 * d2,
                    p->sumsq, 5, L, s, pr));
-  NC_TRY(newton_schulz_wide(p->xsq, 4 * L, (int)d, (int)d, 5, p->nsws, p->status, s, pr));
+  NC_TRY(newton_schulz_wide(p->xsq, n_sq * L, (int)d, (int)d, 5, p->nsws, p->status, s, pr));
+  if (!kv_square)
+    NC_TRY(newton_schulz_wide(p->xkv, 2 * L, (int)dkv, (int)d, 5, p->nsws, p->status, s, pr));
   NC_TRY(newton_schulz_wide(p->xw, 2 * L, (int)d, (int)(4 * d), 5, p->nsws, p->status, s, pr));
-  for (int j = 0; j < 4; ++j)
-    NC_TRY(muon_apply(p->blocks + j * d2, p->blocks_b + j * d2, 12 * d2, (int)d, (int)d, 0,
-                      p->xsq + j * d2, 4 * d2, lr, L, s, pr));
-  NC_TRY(muon_apply(p->blocks + 4 * d2, p->blocks_b + 4 * d2, 12 * d2, (int)(4 * d), (int)d, 1,
-                    p->xw, 8 * d2, lr, L, s, pr));
-  NC_TRY(muon_apply(p->blocks + 8 * d2, p->blocks_b + 8 * d2, 12 * d2, (int)d, (int)(4 * d), 0,
+  for (int i = 0; i < n_sq; ++i) {
+    const int64_t o = mat_offset(p, sq_of[i]);
+    NC_TRY(muon_apply(p->blocks + o, p->blocks_b + o, LS, (int)d, (int)d, 0, p->xsq + i * d2,
+                      n_sq * d2, lr, L, s, pr));
+  }
+  if (!kv_square)
+    for (int i = 0; i < 2; ++i) {
+      const int64_t o = mat_offset(p, 1 + i);
+      NC_TRY(muon_apply(p->blocks + o, p->blocks_b + o, LS, (int)dkv, (int)d, 0, p->xkv + i * kv,
+                        2 * kv, lr, L, s, pr));
+    }
+  const int64_t o_up = mat_offset(p, 4), o_down = mat_offset(p, 5);
+  NC_TRY(muon_apply(p->blocks + o_up, p->blocks_b + o_up, LS, (int)(4 * d), (int)d, 1, p->xw,
+                    8 * d2, lr, L, s, pr));
+  NC_TRY(muon_apply(p->blocks + o_down, p->blocks_b + o_down, LS, (int)d, (int)(4 * d), 0,
                     p->xw + 4 * d2, 8 * d2, lr, L, s, pr));
   return NC_OK;
 }
@@ -487,27 +535,42 @@ const char* nc_status_string(nc_status s) {
   return "unknown";
 }
 
-nc_status nc_gpt_init_ex(int depth, int vocab, uint64_t seed, int flags, nc_params** out) {
-  if (!out) return fail(NC_ERR_INVALID_ARG, "init: null output");
+nc_status nc_gpt_init_config(const nc_model_config* cfg, nc_params** out) {
+  if (!out || !cfg) return fail(NC_ERR_INVALID_ARG, "init: null argument");
   *out = nullptr;
+  const int depth = cfg->depth, vocab = cfg->vocab, flags = cfg->flags;
   if (depth < 1 || depth > 32 || vocab < 8 || vocab > 32768 || vocab % 8 ||
       (flags != NC_INIT_SPEC && flags != NC_INIT_ALL_RANDOM))
     return fail(NC_ERR_INVALID_ARG, "init: depth in [1, 32], vocab in [8, 32768] (multiple of 8)");
   if (depth % 2)
     return fail(NC_ERR_UNSUPPORTED, "init: odd depth gives a head width other than 128");
+  const int H = 64 * depth / 128;
+  const int Hkv = cfg->n_kv_head > 0 ? cfg->n_kv_head : H;
+  if (cfg->n_kv_head < 0 || Hkv > H || H % Hkv)
+    return fail(NC_ERR_INVALID_ARG, "init: n_kv_head must divide the number of heads");
   nc_params* p = new nc_params();
   p->depth = depth;
   p->vocab = vocab;
   p->d = 64 * depth;
   p->hd = 128;
-  p->H = p->d / 128;
+  p->H = H;
+  p->Hkv = Hkv;
+  p->dkv = 128 * Hkv;
   p->F = 4 * p->d;
+  p->window.assign(depth, -1);
+  if (cfg->window)
+    for (int l = 0; l < depth; ++l) p->window[l] = cfg->window[l] < 0 ? -1 : cfg->window[l];
   p->prof = profiler_create();
-  const int64_t d = p->d, V = vocab, be = block_elems(p);
-  const int64_t sq = 4ll * depth * d * d, wide = 8ll * depth * d * d, ws = 12ll * depth * d * d;
+  const int64_t d = p->d, V = vocab, be = block_elems(p), dkv = p->dkv;
+  // Newton-Schulz stacks (see muon): squares, the dkv x d stack, the d x 4d
+  // stack, and the workspace of the largest call (12 L d^2 covers each).
+  const int64_t sq = (dkv == d ? 4ll : 2ll) * depth * d * d;
+  const int64_t kvs = dkv == d ? 0 : 2ll * depth * dkv * d;
+  const int64_t wide = 8ll * depth * d * d, ws = 12ll * depth * d * d;
   auto r = [](int64_t bytes) { return (bytes + 255) & ~int64_t(255); };
   const int64_t total = r(4 * V * d) * 2 + r(4 * be) * 2 + r(2 * be) + r(2 * V * d) +
-                        r(4 * 6 * depth) + r(2 * sq) + r(2 * wide) + r(2 * ws) + r(4);
+                        r(4 * 6 * depth) + r(2 * sq) + r(2 * kvs) + r(2 * wide) + r(2 * ws) +
+                        r(4);
   cudaError_t e = cudaMalloc(&p->pmem, (size_t)total);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -524,6 +587,7 @@ nc_status nc_gpt_init_ex(int depth, int vocab, uint64_t seed, int flags, nc_para
   p->lm_b = ar.take<bf16>(V * d);
   p->sumsq = ar.take<float>(6 * depth);
   p->xsq = ar.take<bf16>(sq);
+  p->xkv = kvs ? ar.take<bf16>(kvs) : nullptr;
   p->xw = ar.take<bf16>(wide);
   p->nsws = ar.take<bf16>(ws);
   p->status = ar.take<int>(1);
@@ -535,7 +599,7 @@ nc_status nc_gpt_init_ex(int depth, int vocab, uint64_t seed, int flags, nc_para
     st = fail(NC_ERR_CUDA, "momentum clear failed");
   if (st == NC_OK && cudaMemsetAsync(p->status, 0, sizeof(int), p->stream) != cudaSuccess)
     st = fail(NC_ERR_CUDA, "status clear failed");
-  if (st == NC_OK) st = init_model(p, seed, flags);
+  if (st == NC_OK) st = init_model(p, cfg->seed, flags);
   if (st == NC_OK && cudaStreamSynchronize(p->stream) != cudaSuccess)
     st = fail(NC_ERR_CUDA, "init synchronisation failed");
   if (st != NC_OK) {
@@ -544,6 +608,15 @@ nc_status nc_gpt_init_ex(int depth, int vocab, uint64_t seed, int flags, nc_para
   }
   *out = p;
   return NC_OK;
+}
+
+nc_status nc_gpt_init_ex(int depth, int vocab, uint64_t seed, int flags, nc_params** out) {
+  nc_model_config cfg{};
+  cfg.depth = depth;
+  cfg.vocab = vocab;
+  cfg.seed = seed;
+  cfg.flags = flags;
+  return nc_gpt_init_config(&cfg, out);
 }
 
 nc_status nc_gpt_init(int depth, int vocab, uint64_t seed, nc_params** out) {

@@ -86,3 +86,20 @@ def test_init_rejects_unsupported_shapes(depth, vocab, status):
 def test_adamw_step_refuses_a_null_handle():
     st = binding.lib().nc_adamw_step(None, None, 0.1, 0.1, 0.9, 0.95, 1e-8, 0.0)
     assert st == binding.NC_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("depth,n_kv_head", [(8, 3), (8, 5), (4, 4), (8, -1)])
+def test_init_rejects_kv_heads_that_do_not_divide_the_heads(depth, n_kv_head):
+    """depth 8 has 4 heads, depth 4 has 2: the KV-head count must divide them."""
+    with pytest.raises(binding.NcError) as e:
+        binding.GPT(depth, vocab=512, seed=1, n_kv_head=n_kv_head)
+    assert e.value.status == binding.NC_ERR_INVALID_ARG
+
+
+def test_window_pattern_repeats_over_layers():
+    assert binding.window_pattern("SSSL", 6, 128) == [128, 128, 128, -1, 128, 128]
+    assert binding.window_pattern("L", 2, 5) == [-1, -1]
+    with pytest.raises(ValueError):
+        binding.window_pattern("SXL", 4, 8)
+    with pytest.raises(ValueError):
+        binding.GPT(4, vocab=512, window=[1, 2, 3])

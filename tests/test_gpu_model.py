@@ -42,6 +42,42 @@ def test_fwd_bwd_parity(depth, B, T, vocab):
         assert rel_fro(g, r) < 3e-2, (i, names[i], rel_fro(g, r))
 
 
+@pytest.mark.parametrize("depth,B,T,vocab,n_kv,window", [
+    (4, 2, 200, 512, 1, [64, -1, 0, 129]),          # two query heads on one KV head
+    (8, 1, 300, 32768, 2, "SSSL:100"),              # four on two, the SSSL pattern
+    (6, 1, 256, 512, 1, [255, 5, -1, 128, 0, 300]),  # three on one
+    (4, 1, 130, 512, 0, [1, 127, 128, -1]),          # windows alone
+])
+def test_fwd_bwd_parity_grouped_kv_and_windows(depth, B, T, vocab, n_kv, window):
+    """The model variant with fewer KV heads and per-layer windows against the
+    oracle's, at the same bars as the default model."""
+    if isinstance(window, str):
+        pat, short = window.split(":")
+        window = nc.window_pattern(pat, depth, int(short))
+        assert window == oracle.window_pattern(pat, depth, int(short))
+    P = inputs.random_params(depth, seed=120 + depth, vocab=vocab, n_kv_head=n_kv)
+    tok, tgt = inputs.token_batch(121 + T, B, T, vocab=vocab)
+    m = _gpt(depth, vocab=vocab, n_kv_head=n_kv, window=window)
+    assert m.shapes() == [p.shape for p in P]
+    m.load(P)
+    loss = m.fwd_bwd(tok, tgt)
+    G = m.grads()
+    m.close()
+    lref, Gref, _ = oracle.gpt_fwd_bwd(depth, P, tok, tgt, vocab=vocab, n_kv_head=n_kv,
+                                       window=window)
+    assert abs(loss - lref) / lref < 2e-3, (loss, lref)
+    names = ["wte"] + ["wq", "wk", "wv", "wo", "wup", "wdown"] * depth + ["lm_head"]
+    for i, (g, r) in enumerate(zip(G, Gref)):
+        if not np.any(r):
+            # wq / wk of a window-0 layer: zero in exact arithmetic (a query
+            # sees only its own key); here rounding noise of dP - D, far below
+            # the layer's wv gradient.
+            l = (i - 1) // 6
+            assert np.abs(g).max() <= 1e-3 * np.abs(Gref[1 + 6 * l + 2]).max(), (i, names[i])
+            continue
+        assert rel_fro(g, r) < 3e-2, (i, names[i], rel_fro(g, r))
+
+
 def test_spec_init_loss_and_gradients_at_full_size():
     """Depth 20, B = 32, T = 2048 (the headline workload) at the specified
     init: loss = ln 32768, every gradient but lm_head's exactly zero, and
@@ -67,12 +103,14 @@ def test_spec_init_loss_and_gradients_at_full_size():
         assert rel_fro(g[r], expect) < 2e-2
 
 
-def test_init_matches_the_oracle_generator():
+@pytest.mark.parametrize("n_kv", [0, 1])
+def test_init_matches_the_oracle_generator(n_kv):
     depth = 4
-    m = _gpt(depth, seed=7)
+    m = _gpt(depth, seed=7, n_kv_head=n_kv)
     P = m.params()
     m.close()
-    R = oracle.init_params(depth, V, seed=7, spec_zero=True)
+    R = oracle.init_params(depth, V, seed=7, spec_zero=True, n_kv_head=n_kv)
+    assert [p.shape for p in P] == [r.shape for r in R]
     for i, (a, b) in enumerate(zip(P, R)):
         if not b.any():
             assert not a.any(), i
@@ -153,11 +191,13 @@ def test_accumulation_invariant_on_gpu():
         assert rel_fro(g, a) < 2e-2, i
 
 
-def test_muon_step_parity():
+@pytest.mark.parametrize("depth,n_kv", [(2, 0), (4, 1), (8, 2)])
+def test_muon_step_parity(depth, n_kv):
     """Muon on given gradients: momentum M = mu*M + G exactly in fp32, and
-    W_new = W - lr * NS5(M) against the oracle over two steps."""
-    depth, lr, mu = 2, 0.02, 0.95
-    m = _gpt(depth, seed=28, all_random=True)
+    W_new = W - lr * NS5(M) against the oracle over two steps.  With grouped
+    KV heads wk and wv are [128 n_kv, d] and orthogonalised as such."""
+    lr, mu = 0.02, 0.95
+    m = _gpt(depth, seed=28, all_random=True, n_kv_head=n_kv)
     W0 = m.params()
     n = m.num_tensors()
     rng = np.random.default_rng(29)
