@@ -60,6 +60,16 @@ def lib():
         L.oc_gpt_fwd_bwd_ex.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                         ctypes.c_int, ctypes.c_int, dp, ctypes.c_void_p, dp]
+        L.oc_gpt_fwd_bwd_fp8.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
+                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                         ctypes.c_int, dp, ctypes.c_void_p, dp]
+        L.oc_e4m3_round.argtypes = [ctypes.c_double]
+        L.oc_e4m3_round.restype = ctypes.c_double
+        L.oc_fp8_scale.argtypes = [dp, ctypes.c_int64]
+        L.oc_fp8_scale.restype = ctypes.c_float
+        L.oc_fp8_matmul_nt.argtypes = [dp, dp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                       ctypes.c_int, dp]
         L.oc_adamw_update.argtypes = [dp, dp, dp, dp, ctypes.c_int64, ctypes.c_double,
                                       ctypes.c_double, ctypes.c_double, ctypes.c_double,
                                       ctypes.c_double, ctypes.c_int]
@@ -190,10 +200,12 @@ def matmul_nt(x, w):
 
 
 def gpt_fwd_bwd(depth, params, tokens, targets, vocab=32768, grads=True, want_logits=False,
-                n_kv_head=0, window=None):
+                n_kv_head=0, window=None, fp8=None):
     """Returns (loss, grads list of float64 arrays or None, logits or None).
     n_kv_head: grouped KV heads (<= 0: one per query head); window: None
-    (full causal) or one window per layer (negative: full causal)."""
+    (full causal) or one window per layer (negative: full causal); fp8:
+    None (exact GEMMs), "e4m3" or "scale" (the block projections' GEMMs on
+    scaled operands, rounded to E4M3 or not)."""
     params = [np.ascontiguousarray(p, dtype=np.float32) for p in params]
     tokens = np.ascontiguousarray(tokens, dtype=np.int32)
     targets = np.ascontiguousarray(targets, dtype=np.int32)
@@ -209,14 +221,38 @@ def gpt_fwd_bwd(depth, params, tokens, targets, vocab=32768, grads=True, want_lo
         win = np.ascontiguousarray(window, dtype=np.int32)
         if win.shape != (depth,):
             raise ValueError("one window per layer")
-    rc = lib().oc_gpt_fwd_bwd_ex(depth, vocab, n_kv_head, win.ctypes.data if win is not None else None,
-                                 pptr, tokens.ctypes.data, targets.ctypes.data, B, T,
-                                 ctypes.byref(loss), gptr, lp)
+    wp = win.ctypes.data if win is not None else None
+    if fp8 is None:
+        rc = lib().oc_gpt_fwd_bwd_ex(depth, vocab, n_kv_head, wp, pptr, tokens.ctypes.data,
+                                     targets.ctypes.data, B, T, ctypes.byref(loss), gptr, lp)
+    else:
+        fmt = {"e4m3": 1, "scale": 0}[fp8]
+        rc = lib().oc_gpt_fwd_bwd_fp8(depth, vocab, n_kv_head, wp, fmt, pptr, tokens.ctypes.data,
+                                      targets.ctypes.data, B, T, ctypes.byref(loss), gptr, lp)
     if rc == -2:
         raise ValueError("token id out of range")
     if rc != 0:
         raise ValueError("oc_gpt_fwd_bwd failed (%d)" % rc)
     return loss.value, g, logits
+
+
+def e4m3_round(x):
+    """Nearest E4M3 value(s) (ties to even, saturating to 448), elementwise."""
+    f = np.vectorize(lambda v: lib().oc_e4m3_round(float(v)), otypes=[np.float64])
+    return f(np.asarray(x, dtype=np.float64))
+
+
+def fp8_scale(x):
+    x = _f64(x)
+    return float(lib().oc_fp8_scale(_dp(x), x.size))
+
+
+def fp8_matmul_nt(x, w, fmt="e4m3"):
+    x, w = _f64(x), _f64(w)
+    y = np.empty((x.shape[0], w.shape[0]))
+    assert lib().oc_fp8_matmul_nt(_dp(x), _dp(w), x.shape[0], w.shape[0], x.shape[1],
+                                  {"e4m3": 1, "scale": 0}[fmt], _dp(y)) == 0
+    return y
 
 
 def newton_schulz(G, steps=NS_STEPS, coeffs=NS_COEFFS, eps=NS_EPS):

@@ -384,6 +384,91 @@ void newton_schulz(const double* G, int rows, int cols, int steps, double a, dou
   }
 }
 
+// ---------------------------------------------------------------- FP8
+// "Treinamento FP8 disponivel via --fp8" (guide, section "1. Modelo GPT",
+// and the d26 run of its results table) with no recipe given.  Reading: the
+// GEMMs of the block projections take operands in the OCP 8-bit format
+// E4M3 (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits, no
+// infinities, largest finite 448 = 1.75 * 2^8, smallest normal 2^-6,
+// subnormals k * 2^-9), each operand tensor with one dynamic scale.
+
+// Nearest E4M3 value of a (ties to the even mantissa), saturating to +-448
+// ("satfinite": magnitudes above 448, infinities included, become 448).
+double e4m3_round(double a) {
+  if (std::isnan(a)) return a;
+  const double mag = std::fabs(a);
+  double q;
+  if (mag >= 448.0) {
+    q = 448.0;
+  } else {
+    int e2;
+    std::frexp(mag, &e2);  // mag = f * 2^e2, f in [0.5, 1): leading bit 2^(e2 - 1)
+    // Spacing of the grid around mag: 2^(e - 3) in the binade [2^e, 2^(e+1)),
+    // and the subnormal spacing 2^-9 below 2^-6.
+    const int e = mag < 0x1.0p-6 ? -6 : e2 - 1;
+    const double step = std::ldexp(1.0, e - 3);
+    q = std::nearbyint(mag / step) * step;  // default rounding: to nearest, ties to even
+  }
+  return std::signbit(a) ? -q : q;
+}
+
+// Scale of one operand tensor: s = 448 / amax, in fp32 arithmetic as a
+// kernel computes it (amax over the fp32 values; 1 when all are zero).
+float fp8_scale(const double* x, int64_t n) {
+  float amax = 0.f;
+  for (int64_t i = 0; i < n; ++i) amax = std::max(amax, std::fabs((float)x[i]));
+  return amax > 0.f ? 448.0f / amax : 1.0f;
+}
+
+// q_i = e4m3(fp32(x_i) * s) with the fp32 product; fmt 0 keeps the scaled
+// fp32 value (scaling without rounding, a check of the surrounding steps).
+float fp8_quantize(const double* x, int64_t n, int fmt, double* q) {
+  const float sc = fp8_scale(x, n);
+  for (int64_t i = 0; i < n; ++i) {
+    const float y = (float)x[i] * sc;
+    q[i] = fmt ? e4m3_round((double)y) : (double)y;
+  }
+  return sc;
+}
+
+template <class TW>
+std::vector<double> as_f64(const TW* w, int64_t n) {
+  return std::vector<double>(w, w + n);
+}
+
+// y = x W^T on quantised operands: (Q(x) Q(W)^T) / (s_x s_W).
+void fp8_mm_nt(const double* x, const double* w, int64_t rows, int64_t n, int64_t k, int fmt,
+               double* y) {
+  std::vector<double> qx(rows * k), qw(n * k);
+  const double sx = fp8_quantize(x, rows * k, fmt, qx.data());
+  const double sw = fp8_quantize(w, n * k, fmt, qw.data());
+  mm_nt(qx.data(), qw.data(), rows, n, k, y);
+  const double inv = 1.0 / (sx * sw);
+  for (int64_t i = 0; i < rows * n; ++i) y[i] *= inv;
+}
+
+// dx (+)= dy W on quantised operands.
+void fp8_mm_nn(const double* dy, const double* w, int64_t rows, int64_t n, int64_t k, int fmt,
+               double* dx, bool accumulate) {
+  std::vector<double> qd(rows * n), qw(n * k), t(rows * k);
+  const double sd = fp8_quantize(dy, rows * n, fmt, qd.data());
+  const double sw = fp8_quantize(w, n * k, fmt, qw.data());
+  mm_nn_acc(qd.data(), qw.data(), rows, n, k, t.data(), false);
+  const double inv = 1.0 / (sd * sw);
+  for (int64_t i = 0; i < rows * k; ++i) dx[i] = (accumulate ? dx[i] : 0.0) + t[i] * inv;
+}
+
+// dW = dy^T x on quantised operands.
+void fp8_mm_tn(const double* dy, const double* x, int64_t rows, int64_t n, int64_t k, int fmt,
+               double* dw) {
+  std::vector<double> qd(rows * n), qx(rows * k);
+  const double sd = fp8_quantize(dy, rows * n, fmt, qd.data());
+  const double sx = fp8_quantize(x, rows * k, fmt, qx.data());
+  mm_tn(qd.data(), qx.data(), rows, n, k, dw);
+  const double inv = 1.0 / (sd * sx);
+  for (int64_t i = 0; i < n * k; ++i) dw[i] *= inv;
+}
+
 }  // namespace
 
 // ==================================================================== C ABI
@@ -514,6 +599,10 @@ int oc_matmul_nt(const double* x, const double* w, int64_t rows, int64_t n, int6
   return 0;
 }
 
+static int gpt_impl(int depth, int vocab, int n_kv_head, const int32_t* window, int fp8,
+                    const float* const* params, const int32_t* tokens, const int32_t* targets,
+                    int B, int T, double* loss, double* const* grads, double* logits);
+
 int oc_gpt_fwd_bwd(int depth, int vocab, const float* const* params, const int32_t* tokens,
                    const int32_t* targets, int B, int T, double* loss, double* const* grads,
                    double* logits) {
@@ -524,6 +613,38 @@ int oc_gpt_fwd_bwd(int depth, int vocab, const float* const* params, const int32
 int oc_gpt_fwd_bwd_ex(int depth, int vocab, int n_kv_head, const int32_t* window,
                       const float* const* params, const int32_t* tokens, const int32_t* targets,
                       int B, int T, double* loss, double* const* grads, double* logits) {
+  return gpt_impl(depth, vocab, n_kv_head, window, -1, params, tokens, targets, B, T, loss, grads,
+                  logits);
+}
+
+int oc_gpt_fwd_bwd_fp8(int depth, int vocab, int n_kv_head, const int32_t* window, int fmt,
+                       const float* const* params, const int32_t* tokens, const int32_t* targets,
+                       int B, int T, double* loss, double* const* grads, double* logits) {
+  if (fmt != 0 && fmt != 1) return -1;
+  return gpt_impl(depth, vocab, n_kv_head, window, fmt, params, tokens, targets, B, T, loss, grads,
+                  logits);
+}
+
+double oc_e4m3_round(double x) { return e4m3_round(x); }
+
+float oc_fp8_scale(const double* x, int64_t n) {
+  return (x && n > 0) ? fp8_scale(x, n) : -1.0f;
+}
+
+int oc_fp8_matmul_nt(const double* x, const double* w, int64_t rows, int64_t n, int64_t k,
+                     int fmt, double* y) {
+  if (!x || !w || !y || rows < 1 || n < 1 || k < 1 || (fmt != 0 && fmt != 1)) return -1;
+  fp8_mm_nt(x, w, rows, n, k, fmt, y);
+  return 0;
+}
+
+// The model of oc_gpt_fwd_bwd_ex; fp8 < 0: exact GEMMs, fp8 >= 0: the block
+// projections' GEMMs on quantised operands (fp8_mm_*, format fp8), the q|k|v
+// projection as one [d + 2 dkv, d] tensor with one scale (its weights and its
+// output gradient each quantised as a whole).
+static int gpt_impl(int depth, int vocab, int n_kv_head, const int32_t* window, int fp8,
+                    const float* const* params, const int32_t* tokens, const int32_t* targets,
+                    int B, int T, double* loss, double* const* grads, double* logits) {
   Dims s;
   if (!params || !tokens || !targets || !loss || B < 1 || T < 1 ||
       !make_dims_kv(depth, vocab, n_kv_head, &s))
@@ -540,6 +661,31 @@ int oc_gpt_fwd_bwd_ex(int depth, int vocab, int n_kv_head, const int32_t* window
   auto W = [&](int l, int j) { return params[1 + 6 * l + j]; };
 
   typedef std::vector<double> vec;
+  // Projections y = x W^T, dx (+)= dy W, dW = dy^T x: exact, or on fp8 operands.
+  auto lin_nt = [&](const double* xx, const float* w, int64_t rows, int64_t n, int64_t k,
+                    double* y) {
+    if (fp8 < 0) mm_nt(xx, w, rows, n, k, y);
+    else fp8_mm_nt(xx, as_f64(w, n * k).data(), rows, n, k, fp8, y);
+  };
+  auto lin_nn = [&](const double* dy, const float* w, int64_t rows, int64_t n, int64_t k,
+                    double* dx, bool accumulate) {
+    if (fp8 < 0) mm_nn_acc(dy, w, rows, n, k, dx, accumulate);
+    else fp8_mm_nn(dy, as_f64(w, n * k).data(), rows, n, k, fp8, dx, accumulate);
+  };
+  auto lin_tn = [&](const double* dy, const double* xx, int64_t rows, int64_t n, int64_t k,
+                    double* dw) {
+    if (fp8 < 0) mm_tn(dy, xx, rows, n, k, dw);
+    else fp8_mm_tn(dy, xx, rows, n, k, fp8, dw);
+  };
+  const int Qw = d + 2 * dkv;  // width of the fused q|k|v projection
+  // [wq; wk; wv] of layer l as one row-major [Qw, d] matrix (fp8 only).
+  auto wqkv = [&](int l) {
+    vec w((int64_t)Qw * d);
+    std::copy(W(l, 0), W(l, 0) + (int64_t)d * d, w.begin());
+    std::copy(W(l, 1), W(l, 1) + (int64_t)dkv * d, w.begin() + (int64_t)d * d);
+    std::copy(W(l, 2), W(l, 2) + (int64_t)dkv * d, w.begin() + (int64_t)(d + dkv) * d);
+    return w;
+  };
   const int64_t Nd = N * d, NF = N * F, NH = N * H, Nkv = N * dkv, NHkv = N * Hkv;
   // Saved forward state per layer.
   std::vector<vec> xin(L, vec(Nd)), h1(L, vec(Nd)), r1(L, vec(N)), qr(L, vec(Nd)),
@@ -555,9 +701,19 @@ int oc_gpt_fwd_bwd_ex(int depth, int vocab, int n_kv_head, const int32_t* window
   for (int l = 0; l < L; ++l) {
     xin[l] = x;
     for (int64_t n = 0; n < N; ++n) rms_row(&x[n * d], d, &h1[l][n * d], &r1[l][n]);
-    mm_nt(h1[l].data(), W(l, 0), N, d, d, qr[l].data());
-    mm_nt(h1[l].data(), W(l, 1), N, dkv, d, kr[l].data());
-    mm_nt(h1[l].data(), W(l, 2), N, dkv, d, vv[l].data());
+    if (fp8 < 0) {
+      mm_nt(h1[l].data(), W(l, 0), N, d, d, qr[l].data());
+      mm_nt(h1[l].data(), W(l, 1), N, dkv, d, kr[l].data());
+      mm_nt(h1[l].data(), W(l, 2), N, dkv, d, vv[l].data());
+    } else {
+      vec y(N * Qw);
+      fp8_mm_nt(h1[l].data(), wqkv(l).data(), N, Qw, d, fp8, y.data());
+      for (int64_t n = 0; n < N; ++n) {
+        std::copy(&y[n * Qw], &y[n * Qw] + d, &qr[l][n * d]);
+        std::copy(&y[n * Qw] + d, &y[n * Qw] + d + dkv, &kr[l][n * dkv]);
+        std::copy(&y[n * Qw] + d + dkv, &y[n * Qw] + Qw, &vv[l][n * dkv]);
+      }
+    }
     // RoPE, then RMSNorm over each head (QK normalisation).
     for (int64_t n = 0; n < N; ++n) {
       const int64_t pos = n % T;
@@ -574,16 +730,16 @@ int oc_gpt_fwd_bwd_ex(int depth, int vocab, int n_kv_head, const int32_t* window
     }
     attention_fwd_gw(qn[l].data(), kn[l].data(), vv[l].data(), B, T, H, Hkv, hd, win(l),
                      ao[l].data(), lse[l].data());
-    mm_nt(ao[l].data(), W(l, 3), N, d, d, tmp.data());
+    lin_nt(ao[l].data(), W(l, 3), N, d, d, tmp.data());
     for (int64_t i = 0; i < Nd; ++i) x[i] += tmp[i];
     xmid[l] = x;
     for (int64_t n = 0; n < N; ++n) rms_row(&x[n * d], d, &h2[l][n * d], &r2[l][n]);
-    mm_nt(h2[l].data(), W(l, 4), N, F, d, uu[l].data());
+    lin_nt(h2[l].data(), W(l, 4), N, F, d, uu[l].data());
     for (int64_t i = 0; i < NF; ++i) {
       const double r = uu[l][i] > 0 ? uu[l][i] : 0.0;
       aa[l][i] = r * r;
     }
-    mm_nt(aa[l].data(), W(l, 5), N, d, F, tmp.data());
+    lin_nt(aa[l].data(), W(l, 5), N, d, F, tmp.data());
     for (int64_t i = 0; i < Nd; ++i) x[i] += tmp[i];
   }
 
@@ -622,17 +778,17 @@ int oc_gpt_fwd_bwd_ex(int depth, int vocab, int n_kv_head, const int32_t* window
   vec da(NF), du(NF), dh(Nd), dxm(Nd), dao(Nd), dqn(Nd), dkn(Nkv), dvv(Nkv), dq(Nd), dk(Nkv);
   for (int l = L - 1; l >= 0; --l) {
     // x_out = xmid + a W_down^T
-    mm_tn(dx.data(), aa[l].data(), N, d, F, grads[1 + 6 * l + 5]);
-    mm_nn_acc(dx.data(), W(l, 5), N, d, F, da.data(), false);
+    lin_tn(dx.data(), aa[l].data(), N, d, F, grads[1 + 6 * l + 5]);
+    lin_nn(dx.data(), W(l, 5), N, d, F, da.data(), false);
     for (int64_t i = 0; i < NF; ++i) du[i] = uu[l][i] > 0 ? 2.0 * uu[l][i] * da[i] : 0.0;
-    mm_tn(du.data(), h2[l].data(), N, F, d, grads[1 + 6 * l + 4]);
-    mm_nn_acc(du.data(), W(l, 4), N, F, d, dh.data(), false);
+    lin_tn(du.data(), h2[l].data(), N, F, d, grads[1 + 6 * l + 4]);
+    lin_nn(du.data(), W(l, 4), N, F, d, dh.data(), false);
     dxm = dx;
     for (int64_t n = 0; n < N; ++n)
       rms_row_bwd_acc(&dh[n * d], &xmid[l][n * d], r2[l][n], d, &dxm[n * d]);
     // xmid = xin + o W_o^T
-    mm_tn(dxm.data(), ao[l].data(), N, d, d, grads[1 + 6 * l + 3]);
-    mm_nn_acc(dxm.data(), W(l, 3), N, d, d, dao.data(), false);
+    lin_tn(dxm.data(), ao[l].data(), N, d, d, grads[1 + 6 * l + 3]);
+    lin_nn(dxm.data(), W(l, 3), N, d, d, dao.data(), false);
     attention_bwd_gw(qn[l].data(), kn[l].data(), vv[l].data(), lse[l].data(), dao.data(), B, T,
                      H, Hkv, hd, win(l), dqn.data(), dkn.data(), dvv.data());
     // Through QK-norm, then RoPE (its transpose is the rotation by -theta).
@@ -651,12 +807,27 @@ int oc_gpt_fwd_bwd_ex(int depth, int vocab, int n_kv_head, const int32_t* window
         rope_row(&dk[off], hd, pos, kRopeBase, -1);
       }
     }
-    mm_tn(dq.data(), h1[l].data(), N, d, d, grads[1 + 6 * l + 0]);
-    mm_tn(dk.data(), h1[l].data(), N, dkv, d, grads[1 + 6 * l + 1]);
-    mm_tn(dvv.data(), h1[l].data(), N, dkv, d, grads[1 + 6 * l + 2]);
-    mm_nn_acc(dq.data(), W(l, 0), N, d, d, dh.data(), false);
-    mm_nn_acc(dk.data(), W(l, 1), N, dkv, d, dh.data(), true);
-    mm_nn_acc(dvv.data(), W(l, 2), N, dkv, d, dh.data(), true);
+    if (fp8 < 0) {
+      mm_tn(dq.data(), h1[l].data(), N, d, d, grads[1 + 6 * l + 0]);
+      mm_tn(dk.data(), h1[l].data(), N, dkv, d, grads[1 + 6 * l + 1]);
+      mm_tn(dvv.data(), h1[l].data(), N, dkv, d, grads[1 + 6 * l + 2]);
+      mm_nn_acc(dq.data(), W(l, 0), N, d, d, dh.data(), false);
+      mm_nn_acc(dk.data(), W(l, 1), N, dkv, d, dh.data(), true);
+      mm_nn_acc(dvv.data(), W(l, 2), N, dkv, d, dh.data(), true);
+    } else {
+      vec g(N * Qw), gw((int64_t)Qw * d);
+      for (int64_t n = 0; n < N; ++n) {
+        std::copy(&dq[n * d], &dq[n * d] + d, &g[n * Qw]);
+        std::copy(&dk[n * dkv], &dk[n * dkv] + dkv, &g[n * Qw] + d);
+        std::copy(&dvv[n * dkv], &dvv[n * dkv] + dkv, &g[n * Qw] + d + dkv);
+      }
+      fp8_mm_tn(g.data(), h1[l].data(), N, Qw, d, fp8, gw.data());
+      std::copy(gw.begin(), gw.begin() + (int64_t)d * d, grads[1 + 6 * l + 0]);
+      std::copy(gw.begin() + (int64_t)d * d, gw.begin() + (int64_t)(d + dkv) * d,
+                grads[1 + 6 * l + 1]);
+      std::copy(gw.begin() + (int64_t)(d + dkv) * d, gw.end(), grads[1 + 6 * l + 2]);
+      fp8_mm_nn(g.data(), wqkv(l).data(), N, Qw, d, fp8, dh.data(), false);
+    }
     dx = dxm;
     for (int64_t n = 0; n < N; ++n)
       rms_row_bwd_acc(&dh[n * d], &xin[l][n * d], r1[l][n], d, &dx[n * d]);

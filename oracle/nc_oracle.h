@@ -144,6 +144,30 @@ int oc_gpt_fwd_bwd_ex(int depth, int vocab, int n_kv_head, const int32_t* window
                       const float* const* params, const int32_t* tokens, const int32_t* targets,
                       int B, int T, double* loss, double* const* grads, double* logits);
 
+/* FP8 ("Treinamento FP8 disponivel via --fp8", guide section "1. Modelo GPT";
+ * the pages give no recipe, so this is the reading): the OCP E4M3 format
+ * (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no infinities,
+ * largest finite 448, subnormals k * 2^-9).
+ * oc_e4m3_round: nearest E4M3 value, ties to the even mantissa, magnitudes
+ *   above 448 (infinities too) saturate to 448; NaN stays NaN.
+ * oc_fp8_scale: per-tensor scale s = 448 / max|fp32(x_i)| in fp32
+ *   arithmetic (1 if all are zero; -1 on a bad argument).
+ * oc_fp8_matmul_nt: y = (Q(x) Q(w)^T) / (s_x s_w) with Q(t)_i =
+ *   e4m3(fp32(t_i) * s_t) (fmt 1) or fp32(t_i) * s_t (fmt 0, scaling
+ *   alone); x [rows, k], w [n, k].
+ * oc_gpt_fwd_bwd_fp8: oc_gpt_fwd_bwd_ex with every GEMM of the block
+ *   projections (forward, input gradient, weight gradient of wq|wk|wv, wo,
+ *   wup, wdown) computed that way; the fused q|k|v weight [d + 2 dkv, d]
+ *   and its output gradient are one tensor each; attention, the embedding
+ *   and lm_head stay exact.  fmt as above. */
+double oc_e4m3_round(double x);
+float oc_fp8_scale(const double* x, int64_t n);
+int oc_fp8_matmul_nt(const double* x, const double* w, int64_t rows, int64_t n, int64_t k,
+                     int fmt, double* y);
+int oc_gpt_fwd_bwd_fp8(int depth, int vocab, int n_kv_head, const int32_t* window, int fmt,
+                       const float* const* params, const int32_t* tokens, const int32_t* targets,
+                       int B, int T, double* loss, double* const* grads, double* logits);
+
 /* Newton-Schulz orthogonalisation of one matrix G [rows, cols]:
  * X = G / (||G||_F + eps_norm), then `steps` iterations of the quintic in
  * the page's right-hand form on the orientation whose Gram X^T X is the

@@ -726,3 +726,219 @@ def test_model_grouped_kv_shapes_and_bad_counts():
     for bad in (3, 5, 8):
         with pytest.raises(ValueError):
             oracle.dims(8, V_SMALL, n_kv_head=bad)
+
+
+# ------------------------------------------------------------------ FP8 (E4M3)
+# The OCP 8-bit format E4M3, built here from its definition: 1 sign, 4
+# exponent bits (bias 7), 3 mantissa bits; exponent field 0 is subnormal
+# (m/8 * 2^-6); the code S.1111.111 is NaN, so the largest finite is
+# 1.75 * 2^8 = 448; no infinities.
+
+def _e4m3_table():
+    vals = []
+    for e in range(16):
+        for m in range(8):
+            if e == 15 and m == 7:
+                continue  # NaN
+            vals.append(m / 8 * 2.0 ** -6 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7))
+    return np.array(sorted(vals))  # 127 non-negative finite values
+
+
+def _e4m3_nearest(x, table):
+    """Brute force: the table entry nearest |x|, ties to the even code, then
+    the sign; saturating at 448."""
+    out = np.empty_like(x)
+    codes = np.arange(len(table))  # sorted order == code order for non-negatives
+    for i, v in enumerate(x):
+        a = min(abs(v), 448.0)
+        dist = np.abs(table - a)
+        best = np.flatnonzero(dist == dist.min())
+        if len(best) > 1:  # a tie: the even code, i.e. the even mantissa
+            best = best[codes[best] % 2 == 0]
+        out[i] = math.copysign(table[best[0]], v)
+    return out
+
+
+def test_e4m3_table_has_the_format_landmarks():
+    t = _e4m3_table()
+    assert len(t) == 127 and t[0] == 0 and t[-1] == 448.0
+    assert t[1] == 2.0 ** -9 and 2.0 ** -6 in t and 240.0 in t and 480.0 not in t
+
+
+def test_e4m3_round_is_the_nearest_value_ties_to_even():
+    t = _e4m3_table()
+    rng = np.random.default_rng(60)
+    x = np.concatenate([
+        rng.standard_normal(3000) * 10.0 ** rng.uniform(-4, 3, 3000),  # every binade
+        (t[1:] + t[:-1]) / 2,                                           # every midpoint
+        -(t[1:] + t[:-1]) / 2,
+        t, -t, [449.0, 463.9, 464.0, 1e6, -1e30],                       # saturation
+    ])
+    np.testing.assert_array_equal(oracle.e4m3_round(x), _e4m3_nearest(x, t))
+
+
+def test_e4m3_round_special_values():
+    r = oracle.e4m3_round([np.inf, -np.inf, np.nan, 0.0, -0.0])
+    assert r[0] == 448 and r[1] == -448 and np.isnan(r[2]) and r[3] == 0
+    assert math.copysign(1, r[4]) == -1
+
+
+def test_fp8_scale_is_448_over_amax_in_fp32():
+    x = np.array([0.3, -1.7, 0.01])
+    assert oracle.fp8_scale(x) == np.float32(448.0) / np.float32(1.7)
+    assert oracle.fp8_scale(np.zeros(5)) == 1.0
+
+
+def test_fp8_matmul_brute_force():
+    """Per-tensor scaling and E4M3 rounding written here with the table:
+    y = (Q(x) Q(w)^T) / (s_x s_w), Q(t) = e4m3(fp32(t) * s_t)."""
+    t = _e4m3_table()
+    rng = np.random.default_rng(61)
+    x = rng.standard_normal((5, 24)) * 3.0
+    w = rng.standard_normal((7, 24)) * 0.02
+
+    def q(a):
+        s = np.float32(448.0) / np.float32(np.abs(a.astype(np.float32)).max())
+        y = (a.astype(np.float32) * s).astype(np.float64)
+        return _e4m3_nearest(y.ravel(), t).reshape(a.shape), float(s)
+
+    qx, sx = q(x)
+    qw, sw = q(w)
+    ref = qx @ qw.T / (sx * sw)
+    np.testing.assert_allclose(oracle.fp8_matmul_nt(x, w), ref, rtol=1e-12, atol=1e-15)
+    # Scaling alone is exact up to fp32 rounding of the operands.
+    np.testing.assert_allclose(oracle.fp8_matmul_nt(x, w, "scale"), x @ w.T, rtol=1e-5,
+                               atol=1e-6 * np.abs(x @ w.T).max())
+    # The error is the format's resolution: rounding to 3 mantissa bits leaves
+    # an RMS relative error near 2^-3 / sqrt(12) / 1.44 = 2.5% per operand,
+    # about 3.5% for the product of two (Gaussian operands, K = 256).
+    g = np.random.default_rng(67)
+    xg, wg = g.standard_normal((64, 256)), g.standard_normal((128, 256))
+    exact = xg @ wg.T
+    rel = np.linalg.norm(oracle.fp8_matmul_nt(xg, wg) - exact) / np.linalg.norm(exact)
+    assert 0.025 < rel < 0.05, rel
+
+
+def test_fp8_matmul_is_invariant_to_power_of_two_scaling():
+    """s absorbs a factor 2^j exactly, so the quantised codes do not move."""
+    rng = np.random.default_rng(62)
+    x = rng.standard_normal((6, 32))
+    w = rng.standard_normal((5, 32))
+    y = oracle.fp8_matmul_nt(x, w)
+    np.testing.assert_array_equal(oracle.fp8_matmul_nt(x * 8.0, w / 32.0), y / 4.0)
+
+
+def test_fp8_model_scaling_alone_is_the_exact_model():
+    """With scaling but no rounding, the FP8 plumbing (which operand is scaled
+    by which factor, the fused q|k|v tensor) must give back the exact model
+    up to fp32 rounding of the GEMM operands."""
+    depth, T = 4, 8
+    P = inputs.random_params(depth, seed=63, vocab=V_SMALL, head_std=0.5, n_kv_head=1)
+    tok, tgt = inputs.token_batch(64, 2, T, vocab=V_SMALL)
+    win = [3, -1, 0, 5]
+    l0, G0, _ = oracle.gpt_fwd_bwd(depth, P, tok, tgt, vocab=V_SMALL, n_kv_head=1, window=win)
+    l1, G1, _ = oracle.gpt_fwd_bwd(depth, P, tok, tgt, vocab=V_SMALL, n_kv_head=1, window=win,
+                                   fp8="scale")
+    assert abs(l1 - l0) < 1e-6 * abs(l0)
+    for i, (a, b) in enumerate(zip(G0, G1)):
+        tol = 1e-5 * max(np.abs(a).max(), 1e-12)
+        np.testing.assert_allclose(b, a, rtol=0, atol=tol, err_msg=str(i))
+
+
+def test_fp8_model_e4m3_is_close_to_the_exact_model():
+    """E4M3 operands: the loss moves by well under 1% and each gradient by the
+    few-percent-per-GEMM error compounded along its path (under 30% here,
+    depth 2), yet visibly; lm_head's own product stays exact, so its
+    gradient is among the closest."""
+    depth, T = 2, 16
+    P = inputs.random_params(depth, seed=65, vocab=V_SMALL, head_std=0.05)
+    tok, tgt = inputs.token_batch(66, 2, T, vocab=V_SMALL)
+    l0, G0, _ = oracle.gpt_fwd_bwd(depth, P, tok, tgt, vocab=V_SMALL)
+    l1, G1, _ = oracle.gpt_fwd_bwd(depth, P, tok, tgt, vocab=V_SMALL, fp8="e4m3")
+    assert 1e-5 < abs(l1 - l0) < 1e-2 * abs(l0)
+    rel = [np.linalg.norm(b - a) / np.linalg.norm(a) for a, b in zip(G0, G1)]
+    assert all(1e-3 < r < 0.3 for r in rel), rel
+    assert rel[-1] < 0.15 and rel[-1] <= np.median(rel)
+
+
+def _quant_table(a, t):
+    """Q(a) and s written here: s = 448 / amax in fp32, codes from the table."""
+    a32 = np.asarray(a, dtype=np.float32)
+    amax = np.abs(a32).max()
+    s = np.float32(448.0) / amax if amax > 0 else np.float32(1.0)
+    y = (a32 * s).astype(np.float64)  # the fp32 product
+    return _e4m3_nearest(y.ravel(), t).reshape(a32.shape), float(s)
+
+
+def test_fp8_rounding_decision_is_taken_on_the_fp32_product():
+    """Values whose fp32 product x * s lands exactly on an E4M3 tie although
+    the exact product does not: the code follows the fp32 product (ties to
+    even), as a kernel's would."""
+    t = _e4m3_table()
+    s = np.float32(448.0) / np.float32(3.3)  # amax 3.3 sets s
+    picked = []
+    for tie in ((t[1:] + t[:-1]) / 2)[20:120]:
+        c = np.float32(tie / float(s))
+        for x in (np.nextafter(c, np.float32(0)), c, np.nextafter(c, np.float32(10))):
+            exact = float(x) * float(s)
+            if float(np.float32(x) * s) == tie and exact != tie:
+                picked.append(float(x))
+    assert len(picked) >= 10
+    x = np.array([3.3] + picked)
+    w = np.eye(len(x))[:1]  # a single output: y_0 = Q(x)_0 * Q(w)_0 / (s_x s_w)
+    qx, sx = _quant_table(x, t)
+    # Q(w) = e4m3(1 * 448) = 448, s_w = 448, so y_j = Q(x)_j / s_x for a w
+    # that selects element j; check every picked element this way.
+    for j in range(len(x)):
+        wj = np.zeros((1, len(x)))
+        wj[0, j] = 1.0
+        y = oracle.fp8_matmul_nt(x[None, :], wj)[0, 0]
+        assert abs(y - qx[j] / sx) <= 1e-12 * abs(qx[j] / sx), (j, x[j])  # codes 1/8 apart
+
+
+def test_fp8_model_mlp_gradients_brute_force():
+    """depth 1 with wo = 0: attention adds nothing, so the MLP sees the
+    embedding and everything its weight gradients need is computed here on
+    quantised operands (Q(t) = e4m3(fp32(t) s_t), s_t = 448 / amax):
+      u = Q(h) Q(wup)^T / ss, a = relu(u)^2, m = Q(a) Q(wdown)^T / ss,
+      x_f = x + m, loss through the final RMSNorm and the exact lm_head;
+      dW_down = Q(dx_f)^T Q(a) / ss,  da = Q(dx_f) Q(wdown) / ss,
+      du = 2 relu(u) da,  dW_up = Q(du)^T Q(h) / ss.
+    This covers a forward, an input-gradient and two weight-gradient GEMMs."""
+    V, T = V_SMALL, 6
+    t = _e4m3_table()
+    P = inputs.random_params(1, seed=68, vocab=V, head_std=0.5)
+    P[4] = np.zeros_like(P[4])  # wo
+    tok, tgt = inputs.token_batch(70, 2, T, vocab=V)
+    _, G, _ = oracle.gpt_fwd_bwd(1, P, tok, tgt, vocab=V, fp8="e4m3")
+    N = tok.size
+
+    def qmm(a, b):  # a b^T on quantised operands
+        qa, sa = _quant_table(a, t)
+        qb, sb = _quant_table(b, t)
+        return qa @ qb.T / (sa * sb)
+
+    def rms_fwd_bwd(x, dy=None):
+        r = 1.0 / np.sqrt(np.mean(x * x, axis=1, keepdims=True) + 1e-6)
+        if dy is None:
+            return x * r
+        return r * dy - (r ** 3 / x.shape[1]) * x * np.sum(dy * x, axis=1, keepdims=True)
+
+    x = P[0][tok.ravel()].astype(np.float64)
+    h = rms_fwd_bwd(x)
+    u = qmm(h, P[5])
+    a = np.maximum(u, 0.0) ** 2
+    xf = x + qmm(a, P[6])
+    lm = P[-1].astype(np.float64)
+    z = rms_fwd_bwd(xf) @ lm.T
+    p = np.exp(z - z.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    p[np.arange(N), tgt.ravel()] -= 1.0
+    dxf = rms_fwd_bwd(xf, (p / N) @ lm)
+    dwdown = qmm(dxf.T, a.T)          # Q(dx_f)^T Q(a)
+    da = qmm(dxf, P[6].T.copy())      # Q(dx_f) Q(wdown)
+    du = 2.0 * np.maximum(u, 0.0) * da
+    dwup = qmm(du.T, h.T)
+    for got, ref in ((G[6], dwdown), (G[5], dwup)):
+        np.testing.assert_allclose(got, ref, rtol=1e-9, atol=1e-12 * np.abs(ref).max())
+    assert not np.any(G[1]) and not np.any(G[2]) and not np.any(G[3])  # wq wk wv: wo = 0
