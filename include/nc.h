@@ -178,6 +178,25 @@ nc_status nc_gpt_fwd_bwd_async(nc_params* p, const int32_t* tokens, const int32_
  * lm_head are not touched (the guide gives them to AdamW).  Asynchronous. */
 nc_status nc_muon_step(nc_params* p, const nc_grads* g, float lr, float momentum);
 
+/* The step as one CUDA graph.  nc_step_capture records, without running
+ * it, one nc_gpt_fwd_bwd_async(p, tokens, targets, B, T, loss_dev, g)
+ * followed by nc_muon_step(p, g, lr, momentum) on the handle's stream into
+ * a graph the handle owns (replacing an earlier one); nc_step_replay
+ * launches that graph on the handle's stream.  A replay reads the token and
+ * target buffers given at capture (refill them in place between replays),
+ * writes the loss to loss_dev and updates the weights, exactly like the two
+ * calls it recorded.  tokens, targets, loss_dev: device memory that must
+ * outlive the graph; the handle needs a non-default stream (nc_set_stream).
+ * Activations for B*T tokens are allocated before the capture; a later call
+ * that reallocates them (another B*T) or the RoPE table (a longer T), or
+ * freeing g, releases the graph.  Profiling is paused during the capture;
+ * replays add the graph's kernel count to nc_launch_count.
+ * Errors: NC_ERR_INVALID_ARG (host pointers, default stream, no captured
+ * step), NC_ERR_TIMEOUT (poisoned handle), NC_ERR_OOM, NC_ERR_CUDA. */
+nc_status nc_step_capture(nc_params* p, const int32_t* tokens, const int32_t* targets, int B, int T,
+                          float* loss_dev, nc_grads* g, float lr, float momentum);
+nc_status nc_step_replay(nc_params* p);
+
 /* AdamW step on the embedding (wte, lr_embed) and lm_head (lr_head) from
  * their gradients in g (guide, section "2. Otimizador Muon": embeddings and
  * lm_head take AdamW; the pages give no hyperparameters, so all are

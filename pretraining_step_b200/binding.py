@@ -98,6 +98,8 @@ def lib():
         "nc_gpt_fwd_bwd_async": (ci, [vp, vp, vp, ci, ci, vp, vp]),
         "nc_muon_step": (ci, [vp, vp, cf, cf]),
         "nc_adamw_step": (ci, [vp, vp, cf, cf, cf, cf, cf, cf]),
+        "nc_step_capture": (ci, [vp, vp, vp, ci, ci, vp, vp, cf, cf]),
+        "nc_step_replay": (ci, [vp]),
         "nc_sync": (ci, [vp]),
         "nc_op_gemm": (ci, [ctypes.POINTER(GemmDesc), vp]),
         "nc_op_rmsnorm": (ci, [vp, i64, ci, vp, vp, vp]),
@@ -274,6 +276,18 @@ class GPT:
 
     def muon_step(self, lr, momentum):
         _check(lib().nc_muon_step(self.h, self.g, lr, momentum))
+
+    def capture_step(self, tokens, targets, loss_dev, lr, momentum):
+        """Record fwd_bwd_async + muon_step as one CUDA graph (nothing runs).
+        tokens, targets, loss_dev: device tensors kept alive by this object
+        for as long as the graph may replay."""
+        B, T = tokens.shape
+        _check(lib().nc_step_capture(self.h, _ptr(tokens), _ptr(targets), B, T, _ptr(loss_dev),
+                                     self.g, lr, momentum))
+        self._graph_io = (tokens, targets, loss_dev)
+
+    def replay_step(self):
+        _check(lib().nc_step_replay(self.h))
 
     def adamw_step(self, lr_embed, lr_head, beta1, beta2, eps, weight_decay):
         """AdamW on the embedding and lm_head from the current gradients."""

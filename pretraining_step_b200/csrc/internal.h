@@ -45,5 +45,9 @@ void profiler_destroy(Profiler*);
 void profiler_enable(Profiler*, bool on);
 nc_status profiler_read(Profiler*, nc_kernel_stat* out, int max, int* n);
 int64_t profiler_launches(const Profiler*);
+bool profiler_enabled(const Profiler*);
+// Adds n to the launch count (graph replays; a capture takes back the
+// launches it recorded but did not run).
+void profiler_add_launches(Profiler*, int64_t n);
 
 }  // namespace nc

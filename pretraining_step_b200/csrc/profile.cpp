@@ -63,6 +63,12 @@ void profiler_enable(Profiler* p, bool on) {
 
 int64_t profiler_launches(const Profiler* p) { return p ? p->launches : 0; }
 
+bool profiler_enabled(const Profiler* p) { return p && p->on; }
+
+void profiler_add_launches(Profiler* p, int64_t n) {
+  if (p) p->launches += n;
+}
+
 Probe::Probe(Profiler* prof_, cudaStream_t s, const char* name, double flops, double bytes)
     : prof(prof_), stream(s), slot(-1) {
   if (!prof) return;

@@ -121,6 +121,11 @@ struct nc_params {
   // pinned host staging for loss + status
   float* h_loss = nullptr;
   int* h_status = nullptr;
+  // One captured step (nc_step_capture) and its kernel launches per replay.
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t graph_exec = nullptr;
+  int64_t graph_launches = 0;
+  const nc_grads* graph_g = nullptr;  // the gradients the captured step writes
 };
 
 struct nc_grads {
@@ -199,8 +204,20 @@ nc_status sync_and_check(nc_params* p, const float* loss_dev) {
   return s;
 }
 
+// A captured step holds the addresses of the activations and the RoPE
+// table: it is released before either is reallocated.
+void drop_graph(nc_params* p) {
+  if (p->graph_exec) cudaGraphExecDestroy(p->graph_exec);
+  if (p->graph) cudaGraphDestroy(p->graph);
+  p->graph_exec = nullptr;
+  p->graph = nullptr;
+  p->graph_launches = 0;
+  p->graph_g = nullptr;
+}
+
 nc_status ensure_rope(nc_params* p, int T) {
   if (p->rope_T >= T) return NC_OK;
+  drop_graph(p);
   int newT = std::max(T, 2048);
   if (p->rope) cudaFree(p->rope);
   p->rope = nullptr;
@@ -216,6 +233,7 @@ nc_status ensure_acts(nc_params* p, int B, int T) {
   if (a.mem && a.N == N && a.B == B && a.T == T) return NC_OK;
   if (a.mem) {
     NC_CUDA_TRY(cudaStreamSynchronize(p->stream));
+    drop_graph(p);
     cudaFree(a.mem);
     a = Acts();
   }
@@ -627,6 +645,7 @@ void nc_params_free(nc_params* p) {
   if (!p) return;
   if (p->stream) cudaStreamSynchronize(p->stream);
   else cudaDeviceSynchronize();
+  drop_graph(p);
   if (p->act.mem) cudaFree(p->act.mem);
   if (p->rope) cudaFree(p->rope);
   if (p->adam) cudaFree(p->adam);
@@ -734,6 +753,7 @@ nc_status nc_grads_create(const nc_params* p, nc_grads** out) {
 void nc_grads_free(nc_grads* g) {
   if (!g) return;
   cudaDeviceSynchronize();
+  if (g->p && g->p->graph_g == g) drop_graph(const_cast<nc_params*>(g->p));
   if (g->mem) cudaFree(g->mem);
   delete g;
 }
@@ -789,6 +809,63 @@ nc_status nc_gpt_fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* tar
 nc_status nc_muon_step(nc_params* p, const nc_grads* g, float lr, float momentum) {
   if (!p) return fail(NC_ERR_INVALID_ARG, "muon: null handle");
   return muon(p, g, lr, momentum);
+}
+
+nc_status nc_step_capture(nc_params* p, const int32_t* tokens, const int32_t* targets, int B, int T,
+                          float* loss_dev, nc_grads* g, float lr, float momentum) {
+  if (!p) return fail(NC_ERR_INVALID_ARG, "step_capture: null handle");
+  if (p->poisoned) return fail(NC_ERR_TIMEOUT, "handle poisoned by an earlier device timeout");
+  if (!p->stream)
+    return fail(NC_ERR_INVALID_ARG, "step_capture: set a non-default stream first (nc_set_stream)");
+  if (!tokens || !targets || !loss_dev || !g || g->p != p || B < 1 || T < 1 ||
+      (int64_t)B * T > (1 << 24))
+    return fail(NC_ERR_INVALID_ARG, "step_capture: bad arguments");
+  if (!is_device_ptr(tokens) || !is_device_ptr(targets) || !is_device_ptr(loss_dev))
+    return fail(NC_ERR_INVALID_ARG, "step_capture: tokens, targets and loss must be device memory");
+  // Everything that allocates happens before the capture.
+  NC_TRY(ensure_acts(p, B, T));
+  NC_TRY(ensure_rope(p, T));
+  drop_graph(p);
+  const bool prof_on = profiler_enabled(p->prof);
+  profiler_enable(p->prof, false);
+  const int64_t launches0 = profiler_launches(p->prof);
+  cudaError_t e = cudaStreamBeginCapture(p->stream, cudaStreamCaptureModeRelaxed);
+  if (e != cudaSuccess) {
+    profiler_enable(p->prof, prof_on);
+    return cuda_fail(e, "step_capture: begin capture");
+  }
+  nc_status st = fwd_bwd(p, tokens, targets, B, T, loss_dev, g);
+  if (st == NC_OK) st = muon(p, g, lr, momentum);
+  cudaGraph_t graph = nullptr;
+  e = cudaStreamEndCapture(p->stream, &graph);  // always ends the capture
+  profiler_enable(p->prof, prof_on);
+  const int64_t n = profiler_launches(p->prof) - launches0;
+  profiler_add_launches(p->prof, -n);  // recorded, not run
+  if (st != NC_OK || e != cudaSuccess) {
+    if (graph) cudaGraphDestroy(graph);
+    cudaGetLastError();
+    return st != NC_OK ? st : cuda_fail(e, "step_capture: end capture");
+  }
+  cudaGraphExec_t exec = nullptr;
+  e = cudaGraphInstantiate(&exec, graph, 0);
+  if (e != cudaSuccess) {
+    cudaGraphDestroy(graph);
+    return cuda_fail(e, "step_capture: instantiate");
+  }
+  p->graph = graph;
+  p->graph_exec = exec;
+  p->graph_launches = n;
+  p->graph_g = g;
+  return NC_OK;
+}
+
+nc_status nc_step_replay(nc_params* p) {
+  if (!p || !p->graph_exec) return fail(NC_ERR_INVALID_ARG, "step_replay: no captured step");
+  if (p->poisoned) return fail(NC_ERR_TIMEOUT, "handle poisoned by an earlier device timeout");
+  if (!p->stream) return fail(NC_ERR_INVALID_ARG, "step_replay: the handle's stream was reset");
+  NC_CUDA_TRY(cudaGraphLaunch(p->graph_exec, p->stream));
+  profiler_add_launches(p->prof, p->graph_launches);
+  return NC_OK;
 }
 
 nc_status nc_adamw_step(nc_params* p, const nc_grads* g, float lr_embed, float lr_head, float beta1,

@@ -103,3 +103,9 @@ def test_window_pattern_repeats_over_layers():
         binding.window_pattern("SXL", 4, 8)
     with pytest.raises(ValueError):
         binding.GPT(4, vocab=512, window=[1, 2, 3])
+
+
+def test_step_graph_calls_refuse_a_null_handle():
+    L = binding.lib()
+    assert L.nc_step_replay(None) == binding.NC_ERR_INVALID_ARG
+    assert L.nc_step_capture(None, None, None, 1, 1, None, None, 0.1, 0.9) == binding.NC_ERR_INVALID_ARG

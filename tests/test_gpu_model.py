@@ -351,3 +351,4 @@ def test_newton_schulz_sweep_sizes():
                 s = np.linalg.svd(out[j].float().cpu().numpy(), compute_uv=False)
                 assert s.min() > 0.6 and s.max() < 1.22
         del out, scratch
+
