@@ -175,17 +175,20 @@ class ClockSampler:
 def cpu_oracle_sample(budget_s=20.0, per_step=False):
     """Time the oracle on a bounded sample of the workload and convert to the
     workload's tokens/s: forward+backward on a short row (cost per token) and
-    the Newton-Schulz of one matrix of each Muon shape (cost per matrix)."""
+    the Newton-Schulz of one matrix of each Muon shape (cost per matrix), on
+    all host cores; then the same at one thread on a smaller sample (2
+    tokens, one (d/2) x (d/2) Newton-Schulz scaled by its FLOPs)."""
+    import numpy as np
     import oracle
     from pretraining_step_b200 import inputs
     oracle.lib()
+    threads_all = oracle.threads()
     P = inputs.random_params(DEPTH, seed=1)
     t_tok = 16
     tok, tgt = inputs.token_batch(2, 1, t_tok)
     t0 = time.perf_counter()
     oracle.gpt_fwd_bwd(DEPTH, P, tok, tgt)
     fb = time.perf_counter() - t0
-    d = 64 * DEPTH
     t0 = time.perf_counter()
     oracle.newton_schulz(P[1])                  # one d x d matrix (of 80)
     ns_sq = time.perf_counter() - t0
@@ -193,16 +196,41 @@ def cpu_oracle_sample(budget_s=20.0, per_step=False):
     oracle.newton_schulz(P[5])                  # one 4d x d matrix (of 40)
     ns_w = time.perf_counter() - t0
     step_s = fb / t_tok * (B * T) + 4 * DEPTH * ns_sq + 2 * DEPTH * ns_w
+    # One thread.  Newton-Schulz costs 6 n^3 per iteration for an n x n matrix
+    # and 18 n^3 for the 4n x n one (4 m n^2 + 2 n^3 with m = 4n), so the
+    # (d/2)^2 sample scales by 8 to d x d and by 24 to 4d x d.
+    oracle.threads(1)
+    try:
+        t1_tok = 2
+        tok1, tgt1 = inputs.token_batch(3, 1, t1_tok)
+        t0 = time.perf_counter()
+        oracle.gpt_fwd_bwd(DEPTH, P, tok1, tgt1)
+        fb1 = time.perf_counter() - t0
+        d = 64 * DEPTH
+        G = np.asarray(P[1][: d // 2, : d // 2], dtype=np.float64)
+        t0 = time.perf_counter()
+        oracle.newton_schulz(G)
+        ns1 = time.perf_counter() - t0
+    finally:
+        oracle.threads(threads_all)
+    step1_s = fb1 / t1_tok * (B * T) + 4 * DEPTH * 8 * ns1 + 2 * DEPTH * 24 * ns1
     return {
         "value": (B * T) / step_s,
         "unit": "tokens/s",
-        "cores": int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1)),
+        "cores": threads_all,
         "kind": "oracle",
-        "sample": ("double-precision CPU oracle: forward+backward of depth 20 on 1 x %d tokens "
-                   "(%.1f s) scaled to 65536 tokens, plus Newton-Schulz of one 1280x1280 "
-                   "(%.1f s) and one 5120x1280 matrix (%.1f s) scaled to 80 + 40 matrices"
-                   % (t_tok, fb, ns_sq, ns_w)),
+        "sample": ("double-precision CPU oracle on %d threads: forward+backward of depth 20 on "
+                   "1 x %d tokens (%.1f s) scaled to 65536 tokens, plus Newton-Schulz of one "
+                   "1280x1280 (%.1f s) and one 5120x1280 matrix (%.1f s) scaled to 80 + 40 "
+                   "matrices" % (threads_all, t_tok, fb, ns_sq, ns_w)),
         "sample_seconds": fb + ns_sq + ns_w,
+        "one_thread": {
+            "value": (B * T) / step1_s, "unit": "tokens/s", "cores": 1,
+            "sample": ("forward+backward on 1 x %d tokens (%.1f s) scaled to 65536 tokens, "
+                       "plus Newton-Schulz of one 640x640 matrix (%.1f s) scaled by FLOPs to "
+                       "80 x 1280^2 and 40 x 5120x1280" % (t1_tok, fb1, ns1)),
+            "sample_seconds": fb1 + ns1,
+        },
     }
 
 

@@ -64,6 +64,8 @@ def lib():
                                          ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
                                          ctypes.c_int, dp, ctypes.c_void_p, dp]
+        L.oc_threads.argtypes = [ctypes.c_int]
+        L.oc_threads.restype = ctypes.c_int
         L.oc_e4m3_round.argtypes = [ctypes.c_double]
         L.oc_e4m3_round.restype = ctypes.c_double
         L.oc_fp8_scale.argtypes = [dp, ctypes.c_int64]
@@ -234,6 +236,12 @@ def gpt_fwd_bwd(depth, params, tokens, targets, vocab=32768, grads=True, want_lo
     if rc != 0:
         raise ValueError("oc_gpt_fwd_bwd failed (%d)" % rc)
     return loss.value, g, logits
+
+
+def threads(n=0):
+    """OpenMP threads of later oracle calls (n > 0 sets them); returns the
+    count in effect."""
+    return int(lib().oc_threads(n))
 
 
 def e4m3_round(x):

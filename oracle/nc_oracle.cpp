@@ -16,6 +16,8 @@
 
 #include "nc_oracle.h"
 
+#include <omp.h>
+
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
@@ -626,6 +628,11 @@ int oc_gpt_fwd_bwd_fp8(int depth, int vocab, int n_kv_head, const int32_t* windo
 }
 
 double oc_e4m3_round(double x) { return e4m3_round(x); }
+
+int oc_threads(int n) {
+  if (n > 0) omp_set_num_threads(n);
+  return omp_get_max_threads();
+}
 
 float oc_fp8_scale(const double* x, int64_t n) {
   return (x && n > 0) ? fp8_scale(x, n) : -1.0f;

@@ -161,6 +161,10 @@ int oc_gpt_fwd_bwd_ex(int depth, int vocab, int n_kv_head, const int32_t* window
  *   and its output gradient are one tensor each; attention, the embedding
  *   and lm_head stay exact.  fmt as above. */
 double oc_e4m3_round(double x);
+
+/* OpenMP threads of later calls: n > 0 sets them; returns the count in
+ * effect (for timing the oracle at one thread and at all cores). */
+int oc_threads(int n);
 float oc_fp8_scale(const double* x, int64_t n);
 int oc_fp8_matmul_nt(const double* x, const double* w, int64_t rows, int64_t n, int64_t k,
                      int fmt, double* y);
