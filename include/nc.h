@@ -217,6 +217,12 @@ nc_status nc_adamw_step(nc_params* p, const nc_grads* g, float lr_embed, float l
 /* Wait for the handle's stream; returns the first device-side error. */
 nc_status nc_sync(nc_params* p);
 
+/* Testing hook: device address of the handle's status word (one int, 0 =
+ * no error; 1 = an expired bounded wait, 2 = a token id out of range), so a
+ * test can plant a device-side error code and check how the host reports
+ * it without making any kernel fail.  NULL for a null handle. */
+int* nc_debug_status_word(nc_params* p);
+
 /* ------------------------------------------------------------------ ops
  * Single kernels of the step, for kernel-level checks and the
  * Newton-Schulz sweep.  All pointers are device pointers; all calls are

@@ -101,6 +101,7 @@ def lib():
         "nc_step_capture": (ci, [vp, vp, vp, ci, ci, vp, vp, cf, cf]),
         "nc_step_replay": (ci, [vp]),
         "nc_sync": (ci, [vp]),
+        "nc_debug_status_word": (vp, [vp]),
         "nc_op_gemm": (ci, [ctypes.POINTER(GemmDesc), vp]),
         "nc_op_rmsnorm": (ci, [vp, i64, ci, vp, vp, vp]),
         "nc_op_attention_fwd": (ci, [vp, vp, vp, i64, vp, i64, vp, ci, ci, ci, vp]),

@@ -894,6 +894,8 @@ nc_status nc_sync(nc_params* p) {
   return sync_and_check(p, nullptr);
 }
 
+int* nc_debug_status_word(nc_params* p) { return p ? p->status : nullptr; }
+
 nc_status nc_profile_enable(nc_params* p, int on) {
   if (!p) return fail(NC_ERR_INVALID_ARG, "profile: null handle");
   profiler_enable(p->prof, on != 0);

@@ -31,3 +31,36 @@ def test_expired_wait_reports_status_and_leaves_the_context_usable(tmp_path):
     assert int(waited_ok) == 0          # the wait gave up
     assert 0.95 * LIMIT_MS <= float(ms) < 3 * LIMIT_MS  # (the device timer's own granularity)
     assert int(after) == 1              # the next kernel ran
+
+
+def test_planted_timeout_status_poisons_the_handle():
+    """Host side of the same path: a timeout code in the status word (planted
+    here instead of produced by a stuck kernel) surfaces as NC_ERR_TIMEOUT
+    at the next synchronising call, and the handle then refuses work."""
+    import numpy as np
+    from pretraining_step_b200 import binding as nc
+    from pretraining_step_b200 import inputs
+
+    from gpu_util import torch
+    t = torch()
+    m = nc.GPT(2, vocab=512, seed=3)
+    ptr = nc.lib().nc_debug_status_word(m.h)
+    assert ptr
+
+    class _Word:
+        __cuda_array_interface__ = {"shape": (1,), "typestr": "<i4", "data": (ptr, False),
+                                    "version": 3}
+
+    word = t.as_tensor(_Word(), device="cuda")  # aliases the status word
+    m.sync()                                      # no error yet
+    word.fill_(DEV_TIMEOUT)
+    t.cuda.synchronize()
+    with pytest.raises(nc.NcError) as e:
+        m.sync()
+    assert e.value.status == nc.NC_ERR_TIMEOUT
+    tok, tgt = inputs.token_batch(4, 1, 16, vocab=512)
+    with pytest.raises(nc.NcError) as e:
+        m.fwd_bwd(tok, tgt)
+    assert e.value.status == nc.NC_ERR_TIMEOUT
+    assert np.isfinite(m.read(0)).all()  # the parameters are still readable
+    m.close()
