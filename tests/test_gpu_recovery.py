@@ -1,11 +1,14 @@
-"""Failure detection without a fault: a bounded device wait that runs out.
+"""Failure detection and recovery without a GPU fault.
 
-A kernel waits, through the library's tc::mbar_wait, on an mbarrier that
-nothing arrives on.  After the wall-clock limit (2 s) the wait records the
-timeout in the device status word and the kernel returns; the launch
-completes without a CUDA error, the host reads the status, and the next
-kernel runs normally.  The probe is compiled from
-tests/gpu_probes/wait_timeout.cu."""
+- A kernel waits, through the library's tc::mbar_wait, on an mbarrier that
+  nothing arrives on.  After the wall-clock limit (2 s) the wait records the
+  timeout in the device status word and the kernel returns; the launch
+  completes without a CUDA error, the host reads the status, and the next
+  kernel runs normally (probe: tests/gpu_probes/wait_timeout.cu).
+- A timeout code planted in a handle's status word surfaces as
+  NC_ERR_TIMEOUT and poisons the handle.
+- An activation request far beyond the device's memory returns NC_ERR_OOM
+  and the handle keeps working."""
 import os
 import subprocess
 
@@ -63,4 +66,24 @@ def test_planted_timeout_status_poisons_the_handle():
         m.fwd_bwd(tok, tgt)
     assert e.value.status == nc.NC_ERR_TIMEOUT
     assert np.isfinite(m.read(0)).all()  # the parameters are still readable
+    m.close()
+
+
+def test_activation_request_beyond_memory_is_oom_and_the_handle_recovers():
+    """B*T = 2^24 tokens at vocabulary 32768 asks for over a terabyte of
+    activations (the bf16 logits alone are 1 TiB): the allocation fails, the
+    call returns NC_ERR_OOM before touching the device, and a normal step on
+    the same handle then succeeds."""
+    import numpy as np
+    from pretraining_step_b200 import binding as nc
+    from pretraining_step_b200 import inputs
+
+    m = nc.GPT(2, seed=5)
+    big = np.zeros((4096, 4096), dtype=np.int32)
+    with pytest.raises(nc.NcError) as e:
+        m.fwd_bwd(big, big)
+    assert e.value.status == nc.NC_ERR_OOM
+    tok, tgt = inputs.token_batch(6, 1, 64)
+    loss = m.fwd_bwd(tok, tgt)
+    assert abs(loss - np.log(32768)) < 1e-3  # specified init: zero lm_head
     m.close()
