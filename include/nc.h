@@ -45,7 +45,7 @@ typedef enum {
   NC_ERR_CUDA = 3,        /* a CUDA runtime call failed                     */
   NC_ERR_TOKEN_RANGE = 4, /* a token or target id outside [0, vocab)        */
   NC_ERR_TIMEOUT = 5,     /* a bounded device wait expired; handle poisoned */
-  NC_ERR_UNSUPPORTED = 6  /* valid request this build does not implement    */
+  NC_ERR_UNSUPPORTED = 6  /* valid request this library does not implement  */
 } nc_status;
 
 typedef enum { NC_F32 = 0, NC_BF16 = 1, NC_I32 = 2 } nc_dtype;
@@ -80,7 +80,7 @@ typedef struct {
  * tensor t uses splitmix64(key_t + 2i) and splitmix64(key_t + 2i + 1),
  * key_t = splitmix64(seed ^ splitmix64(t + 1)).
  * depth: an even number in [2, 32] (head_dim 128, at most 16 heads; depth 1,
- * whose single head is 64 wide, returns NC_ERR_UNSUPPORTED in this build);
+ * whose single head is 64 wide, returns NC_ERR_UNSUPPORTED);
  * vocab: [8, 32768], multiple of 8.
  * Parameters, Muon momentum (zero) and bf16 copies are allocated here;
  * activations are allocated by the first nc_gpt_fwd_bwd of a given B*T.
