@@ -312,7 +312,8 @@ nc_status nc_op_attention_bwd(const void* q, const void* k, const void* v, int64
  * q, o, dO, dq hold H heads of 128 per row (row strides ldq, ldo; dq dense
  * [B, T, H, 128]); k, v, dk, dv hold Hkv heads (strides ldkv, ldg), H a
  * multiple of Hkv; query head h reads KV head h / (H / Hkv).  Query t sees
- * keys [t - window, t]; window < 0 means every key up to t.  With Hkv = H,
+ * keys [t - window, t]; window < 0 means every key up to t, and so does
+ * any window of T - 1 or more (it runs as unbounded).  With Hkv = H,
  * ldkv = ldq and window < 0 these are nc_op_attention_fwd / _bwd.  Layouts,
  * alignment (16-byte rows) and errors otherwise as those; H <= 16 for the
  * backward. */

@@ -766,7 +766,9 @@ nc_status attention_fwd_ex(const void* q, int64_t ldq, const void* k, const void
   a.lse = lse;
   a.H = H;
   a.group = H / Hkv;
-  a.window = window < 0 ? -1 : window;
+  // A window of T - 1 or more keys is full causal: such a window runs as
+  // unbounded, which also keeps the kernels' window sums (up to ~2T) in range.
+  a.window = (window < 0 || window >= T - 1) ? -1 : window;
   a.status = status;
   const double flops = 4.0 * B * H * HD * causal_pairs(T, a.window);
   Probe probe(prof, s, "attn_fwd", flops, 0.0);
@@ -815,7 +817,7 @@ nc_status attention_bwd_tc_ex(const void* q, int64_t ldq, const void* k, const v
   a.nkb = (T + BKV - 1) / BKV;
   a.nqb = (T + BQB - 1) / BQB;
   a.group = H / Hkv;
-  a.window = window < 0 ? -1 : window;
+  a.window = (window < 0 || window >= T - 1) ? -1 : window;  // as in the forward
   a.scale = (float)(1.0 / std::sqrt((double)HD));
   a.sl2 = (float)(1.4426950408889634 / std::sqrt((double)HD));
   a.lse = lse;
