@@ -47,6 +47,23 @@ def model_flops_per_token(depth=DEPTH, seq=T, vocab=V):
     return 6.0 * n_mm + 6.0 * depth * d * seq
 
 
+def step_flops_per_token(depth, seq, vocab, n_kv_head=0, windows=None):
+    """model_flops_per_token for the model with grouped KV heads and per-layer
+    windows: N_mm = L (10 d^2 + 2 dkv d) + V d, and each layer's attention
+    counts the (query, key) band a window of w keys leaves in the causal
+    triangle, T w - w^2 / 2 (T^2 / 2 for full causal, the convention of
+    6 L d T)."""
+    d = 64 * depth
+    H = d // 128
+    dkv = 128 * (n_kv_head if n_kv_head > 0 else H)
+    n_mm = depth * (10 * d * d + 2 * dkv * d) + vocab * d
+    attn = 0.0
+    for l in range(depth):
+        w = seq if windows is None or windows[l] < 0 else min(windows[l], seq)
+        attn += 12.0 * d * (seq * w - w * w / 2.0) / seq
+    return 6.0 * n_mm + attn
+
+
 def gemm_algorithmic_bytes_per_step(depth=DEPTH, batch=B, seq=T, vocab=V):
     """Operand and result bytes of every GEMM launch of one step, each operand
     read once and each result written once (bf16 2 B, fp32 4 B; a split-K
@@ -441,6 +458,8 @@ def run_op(args):
     torch.manual_seed(0)
     dims = [int(x) for x in args.shape.split(",")]
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    if args.op == "step":
+        return run_step_variant(args, dims, peaks, peak_kind)
     if args.op == "adamw":
         # AdamW on the depth-20 embedding and lm_head ([V, d] each): HBM-bound.
         m = nc.GPT(DEPTH, vocab=V, seed=7, all_random=True)
@@ -518,6 +537,53 @@ def run_op(args):
     return 0
 
 
+def run_step_variant(args, dims, peaks, peak_kind):
+    """The forward + backward + Muon step of any model configuration
+    (--shape depth,B,T, grouped KV heads, per-layer windows), inputs
+    resident, device-timed on the model's stream."""
+    import torch
+    from pretraining_step_b200 import binding as nc
+    from pretraining_step_b200 import inputs
+    depth, Bb, T_ = dims
+    windows = None
+    if args.window_pattern:
+        windows = nc.window_pattern(args.window_pattern, depth, args.short_window)
+    stream = torch.cuda.Stream()
+    m = nc.GPT(depth, vocab=V, seed=1234, all_random=True, stream=stream,
+               n_kv_head=args.kv_heads, window=windows)
+    tk, tg = inputs.token_batch(20, Bb, T_)
+    tok, tgt = torch.from_numpy(tk).cuda(), torch.from_numpy(tg).cuda()
+    loss = torch.zeros(1, dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+
+    def step():
+        m.fwd_bwd_async(tok, tgt, loss)
+        m.muon_step(LR, MOMENTUM)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+        m.sync()
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+    m.sync()
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    m.close()
+    tok_s = Bb * T_ / (ms / 1e3)
+    fpt = step_flops_per_token(depth, T_, V, args.kv_heads, windows)
+    print(json.dumps({"op": "step", "depth": depth, "B": Bb, "T": T_, "kv_heads": args.kv_heads,
+                      "windows": windows, "ms_per_step": ms, "tokens_per_s": tok_s,
+                      "flops_per_token": fpt, "tflops": tok_s * fpt / 1e12,
+                      "mfu": tok_s * fpt / 1e12 / NOMINAL_BF16_TFLOPS,
+                      "peak_source": peak_kind}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -525,8 +591,13 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["gemm", "attn", "attn_bwd", "adamw"], default=None,
-                    help="time one kernel class alone instead of the step")
+    ap.add_argument("--op", choices=["gemm", "attn", "attn_bwd", "adamw", "step"], default=None,
+                    help="time one kernel class alone instead of the step ('step': the whole "
+                         "step of the model --shape depth,B,T with the options below)")
+    ap.add_argument("--kv-heads", type=int, default=0, help="--op step: KV heads (0: one per head)")
+    ap.add_argument("--window-pattern", default=None,
+                    help="--op step: per-layer pattern of S (short window) and L (full causal)")
+    ap.add_argument("--short-window", type=int, default=1024, help="--op step: the S window")
     ap.add_argument("--shape", default="16384,5120,1280")
     args = ap.parse_args()
     if args.warmup < 3:
