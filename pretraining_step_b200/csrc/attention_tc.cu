@@ -412,6 +412,10 @@ struct BwdArgs {
   int* status;
 };
 
+// GW: grouped KV heads or a window in play; the plain instance compiles
+// with group 1 and no window as constants (its tile t is query tile i0 + t
+// of head hk).
+template <bool GW>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
@@ -440,14 +444,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kb = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;  // hk: the KV head
+  const int group = GW ? a.group : 1;
+  const int window = GW ? a.window : -1;
   const int i0 = (kb * BKV) / BQB;
   // Query tiles at or after this key tile, up to the last one a window reaches;
   // every query head of the KV head's group in turn (tile t: head
   // hk * group + t / nqt, query tile i0 + t % nqt), so dK and dV accumulate
   // over the whole group in TMEM.
-  const int i_hi = a.window < 0 ? a.nqb - 1 : min(a.nqb - 1, (kb * BKV + BKV - 1 + a.window) / BQB);
+  const int i_hi = window < 0 ? a.nqb - 1 : min(a.nqb - 1, (kb * BKV + BKV - 1 + window) / BQB);
   const int nqt = i_hi - i0 + 1;
-  const int nblk = a.group * nqt;
+  const int nblk = group * nqt;
   const int kcol0 = hk * HD;
 
   if (threadIdx.x == 0) {
@@ -500,8 +506,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       bool w = true;
       if (lane == 0) w = tc::mbar_wait(&qd_empty[st], ph ^ 1, abort_flag, a.status);
       if (!__shfl_sync(0xffffffffu, (int)w, 0)) { ok = false; break; }
-      const int hq = hk * a.group + t / nqt;
-      const int q0 = (i0 + t % nqt) * BQB;
+      const int hq = GW ? hk * group + t / nqt : hk;
+      const int q0 = (i0 + (GW ? t % nqt : t)) * BQB;
       const int qcol0 = hq * HD;
       const float* lse_bh = a.lse + ((int64_t)b * a.H + hq) * a.T;
       const float* d_bh = a.delta + ((int64_t)b * a.H + hq) * a.T;
@@ -607,7 +613,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t ds_row = tc::smem_u32(smem + B_OFF_DS) + row * 128;
     bool ok = true;
     for (int t = 0; t < nblk; ++t) {
-      const int q0 = (i0 + t % nqt) * BQB + 32 * ch;
+      const int q0 = (i0 + (GW ? t % nqt : t)) * BQB + 32 * ch;
       const float* ld = reinterpret_cast<const float*>(smem + B_OFF_LD) + (t % QST) * 2 * BQB + 32 * ch;
       ok = tc::mbar_wait(sdp_full, t & 1, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
@@ -624,15 +630,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       uint32_t pp[16], pd[16];
       const bool edge = (q0 < key + 1) || (q0 + 32 > a.T) || (key >= a.T) ||
-                        (a.window >= 0 && q0 + 31 > key + a.window);  // diagonal, T or window
+                        (window >= 0 && q0 + 31 > key + window);  // diagonal, T or window
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
         float p0 = ex2(__uint_as_float(sv[2 * c]) * a.sl2 - ld[2 * c]);
         float p1 = ex2(__uint_as_float(sv[2 * c + 1]) * a.sl2 - ld[2 * c + 1]);
         if (edge) {
           const int qa = q0 + 2 * c, qb2 = qa + 1;
-          if (qa < key || qa >= a.T || key >= a.T || (a.window >= 0 && qa > key + a.window)) p0 = 0.f;
-          if (qb2 < key || qb2 >= a.T || key >= a.T || (a.window >= 0 && qb2 > key + a.window)) p1 = 0.f;
+          if (qa < key || qa >= a.T || key >= a.T || (window >= 0 && qa > key + window)) p0 = 0.f;
+          if (qb2 < key || qb2 >= a.T || key >= a.T || (window >= 0 && qb2 > key + window)) p1 = 0.f;
         }
         const float d0 = p0 * (__uint_as_float(dp[2 * c]) - ld[BQB + 2 * c]);
         const float d1 = p1 * (__uint_as_float(dp[2 * c + 1]) - ld[BQB + 2 * c + 1]);
@@ -686,8 +692,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
     const int64_t dq_row = (int64_t)a.H * HD;
     for (int t = 0; t < nblk; ++t) {
-      const int q0 = (i0 + t % nqt) * BQB;
-      float* dq_bh = a.dq + (int64_t)b * a.T * dq_row + (hk * a.group + t / nqt) * HD + dim;
+      const int q0 = (i0 + (GW ? t % nqt : t)) * BQB;
+      float* dq_bh = a.dq + (int64_t)b * a.T * dq_row + (GW ? hk * group + t / nqt : hk) * HD + dim;
       bool ok = tc::mbar_wait(&dq_full[t & 1], (t >> 1) & 1, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc::tc_fence_after();
@@ -743,14 +749,14 @@ nc_status attention_fwd_ex(const void* q, int64_t ldq, const void* k, const void
       ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
         reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(o)) & 15))
     return fail(NC_ERR_INVALID_ARG, "attention_fwd: rows must be 16-byte aligned");
-  static bool attr = false;
-  if (!attr) {
+  static DeviceOnce attr;
+  NC_TRY(once_per_device(attr, []() -> nc_status {
     NC_CUDA_TRY(cudaFuncSetAttribute(attn_fwd_tc_kernel<false>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem));
     NC_CUDA_TRY(cudaFuncSetAttribute(attn_fwd_tc_kernel<true>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem));
-    attr = true;
-  }
+    return NC_OK;
+  }));
   CUtensorMap mq, mk, mv;
   // Box heights must match the tile sizes the kernel's byte counts assume.
   if (!make_tmap_bf16_3d(&mq, q, (uint64_t)H * HD, T, B, ldq, (int64_t)T * ldq, BQ) ||
@@ -792,12 +798,14 @@ nc_status attention_bwd_tc_ex(const void* q, int64_t ldq, const void* k, const v
                               const void* dout, int64_t ldo, const float* lse, const float* delta,
                               float* dq, void* dk, void* dv, int64_t ldg, int B, int T, int H,
                               int Hkv, int window, int* status, cudaStream_t s, Profiler* prof) {
-  static bool attr = false;
-  if (!attr) {
-    NC_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc_kernel,
+  static DeviceOnce attr;
+  NC_TRY(once_per_device(attr, []() -> nc_status {
+    NC_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc_kernel<false>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdSmem));
-    attr = true;
-  }
+    NC_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc_kernel<true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdSmem));
+    return NC_OK;
+  }));
   if (Hkv < 1 || H % Hkv) return fail(NC_ERR_INVALID_ARG, "attention_bwd: H must be a multiple of Hkv");
   if (ldq % 8 || ldkv % 8 || ldo % 8 || ldg % 8 ||
       ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
@@ -830,7 +838,10 @@ nc_status attention_bwd_tc_ex(const void* q, int64_t ldq, const void* k, const v
   const double flops = 10.0 * B * H * HD * causal_pairs(T, a.window);
   Probe probe(prof, s, "attn_bwd", flops, 0.0);
   dim3 grid(a.nkb, Hkv, B);  // one CTA per key tile and KV head; it loops over the group
-  attn_bwd_tc_kernel<<<grid, kBwdThreads, kBwdSmem, s>>>(mq, mk, mv, mdo, a);
+  if (a.group > 1 || a.window >= 0)
+    attn_bwd_tc_kernel<true><<<grid, kBwdThreads, kBwdSmem, s>>>(mq, mk, mv, mdo, a);
+  else
+    attn_bwd_tc_kernel<false><<<grid, kBwdThreads, kBwdSmem, s>>>(mq, mk, mv, mdo, a);
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }

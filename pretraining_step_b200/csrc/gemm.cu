@@ -989,12 +989,12 @@ template <int BN, bool ROPE>
 nc_status launch_bn(const nc_gemm_desc& d, int split, int* status, const char* tag,
                     cudaStream_t s, Profiler* prof) {
   using C = Cfg<BN>;
-  static bool attr_set = false;
-  if (!attr_set) {
+  static DeviceOnce smem_attr;
+  NC_TRY(once_per_device(smem_attr, []() -> nc_status {
     NC_CUDA_TRY(cudaFuncSetAttribute(gemm_tc_kernel<BN, ROPE>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
-    attr_set = true;
-  }
+    return NC_OK;
+  }));
   CUtensorMap ta, tb;
   const bool ok_a = d.a_kmajor ? make_tmap_bf16_3d(&ta, d.A, d.K, d.M, d.batch, d.lda, d.stride_a, BM)
                                : make_tmap_bf16_3d(&ta, d.A, d.M, d.K, d.batch, d.lda, d.stride_a, 64);
@@ -1046,16 +1046,16 @@ template <bool ROPE, bool XR>
 nc_status launch_pair(const nc_gemm_desc& d, int split, int* status, const char* tag,
                       cudaStream_t s, Profiler* prof) {
   using C = std::conditional_t<XR, Cfg2X, Cfg2>;
-  static bool attr_set = false;
-  if (!attr_set) {
+  static DeviceOnce smem_attr;
+  NC_TRY(once_per_device(smem_attr, []() -> nc_status {
     if constexpr (XR)
       NC_CUDA_TRY(cudaFuncSetAttribute(gemm_tc2_aux_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM_BYTES));
     else
       NC_CUDA_TRY(cudaFuncSetAttribute(gemm_tc2_kernel<ROPE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
-    attr_set = true;
-  }
+    return NC_OK;
+  }));
   CUtensorMap ta, tb, tx;
   if constexpr (XR) {
     // aux chunks of 32 columns x 32 rows: 128-byte rows (fp32) or 64-byte rows (bf16)

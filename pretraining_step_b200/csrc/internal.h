@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
 #include <string>
 
 #include "../../include/nc.h"
@@ -29,6 +30,27 @@ nc_status cuda_fail(cudaError_t e, const char* what);
   } while (0)
 
 int num_sms();
+
+// Setup that holds per device, such as a kernel's shared-memory limit
+// (cudaFuncSetAttribute): once_per_device(o, f) runs f the first time each
+// device (0..63; beyond that, every time) reaches it, and again after a
+// failure.  Thread-safe.
+struct DeviceOnce {
+  std::mutex m;
+  uint64_t done = 0;
+};
+template <class F>
+nc_status once_per_device(DeviceOnce& o, F&& f) {
+  int dev = 0;
+  NC_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return f();
+  const uint64_t bit = 1ull << dev;
+  std::lock_guard<std::mutex> lock(o.m);
+  if (o.done & bit) return NC_OK;
+  const nc_status st = f();
+  if (st == NC_OK) o.done |= bit;
+  return st;
+}
 
 // Per-kernel-class timing (profile.cpp).  Every launch site wraps its launch
 // in a Probe; with profiling off it only counts the launch.
