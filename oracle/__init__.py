@@ -68,7 +68,7 @@ def lib():
         L.oc_threads.restype = ctypes.c_int
         L.oc_e4m3_round.argtypes = [ctypes.c_double]
         L.oc_e4m3_round.restype = ctypes.c_double
-        L.oc_fp8_scale.argtypes = [dp, ctypes.c_int64]
+        L.oc_fp8_scale.argtypes = [dp, ctypes.c_int64, ctypes.c_int]
         L.oc_fp8_scale.restype = ctypes.c_float
         L.oc_fp8_matmul_nt.argtypes = [dp, dp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                        ctypes.c_int, dp]
@@ -250,9 +250,10 @@ def e4m3_round(x):
     return f(np.asarray(x, dtype=np.float64))
 
 
-def fp8_scale(x):
+def fp8_scale(x, activation=False):
+    """448 / amax of the values x is quantised from (bf16 for an activation)."""
     x = _f64(x)
-    return float(lib().oc_fp8_scale(_dp(x), x.size))
+    return float(lib().oc_fp8_scale(_dp(x), x.size, 1 if activation else 0))
 
 
 def fp8_matmul_nt(x, w, fmt="e4m3"):

@@ -414,20 +414,40 @@ double e4m3_round(double a) {
   return std::signbit(a) ? -q : q;
 }
 
+// Nearest bfloat16 value of the fp32 value v, ties to even: the storage
+// format of activations and their gradients, from which a kernel quantises.
+float bf16_round(float v) {
+  if (std::isnan(v)) return v;
+  uint32_t u;
+  std::memcpy(&u, &v, 4);
+  u = (u + 0x7FFFu + ((u >> 16) & 1u)) & 0xFFFF0000u;
+  float r;
+  std::memcpy(&r, &u, 4);
+  return r;
+}
+
+// The value a tensor is quantised from: fp32(x), rounded on to bf16 for an
+// activation or gradient (bf16 in memory) in E4M3 mode; weights quantise
+// from their fp32 masters.  Scaling alone (fmt 0) keeps fp32 everywhere.
+inline float fp8_source(double x, int fmt, bool act) {
+  return (fmt && act) ? bf16_round((float)x) : (float)x;
+}
+
 // Scale of one operand tensor: s = 448 / amax, in fp32 arithmetic as a
-// kernel computes it (amax over the fp32 values; 1 when all are zero).
-float fp8_scale(const double* x, int64_t n) {
+// kernel computes it (amax over the source values; 1 when all are zero).
+float fp8_scale(const double* x, int64_t n, int fmt = 1, bool act = false) {
   float amax = 0.f;
-  for (int64_t i = 0; i < n; ++i) amax = std::max(amax, std::fabs((float)x[i]));
+  for (int64_t i = 0; i < n; ++i) amax = std::max(amax, std::fabs(fp8_source(x[i], fmt, act)));
   return amax > 0.f ? 448.0f / amax : 1.0f;
 }
 
-// q_i = e4m3(fp32(x_i) * s) with the fp32 product; fmt 0 keeps the scaled
-// fp32 value (scaling without rounding, a check of the surrounding steps).
-float fp8_quantize(const double* x, int64_t n, int fmt, double* q) {
-  const float sc = fp8_scale(x, n);
+// q_i = e4m3(v_i * s) with the fp32 product of the source value v_i; fmt 0
+// keeps the scaled fp32 value (scaling without rounding, a check of the
+// surrounding steps).
+float fp8_quantize(const double* x, int64_t n, int fmt, bool act, double* q) {
+  const float sc = fp8_scale(x, n, fmt, act);
   for (int64_t i = 0; i < n; ++i) {
-    const float y = (float)x[i] * sc;
+    const float y = fp8_source(x[i], fmt, act) * sc;
     q[i] = fmt ? e4m3_round((double)y) : (double)y;
   }
   return sc;
@@ -438,34 +458,35 @@ std::vector<double> as_f64(const TW* w, int64_t n) {
   return std::vector<double>(w, w + n);
 }
 
-// y = x W^T on quantised operands: (Q(x) Q(W)^T) / (s_x s_W).
+// y = x W^T on quantised operands: (Q(x) Q(W)^T) / (s_x s_W); x is an
+// activation, W a weight.
 void fp8_mm_nt(const double* x, const double* w, int64_t rows, int64_t n, int64_t k, int fmt,
                double* y) {
   std::vector<double> qx(rows * k), qw(n * k);
-  const double sx = fp8_quantize(x, rows * k, fmt, qx.data());
-  const double sw = fp8_quantize(w, n * k, fmt, qw.data());
+  const double sx = fp8_quantize(x, rows * k, fmt, true, qx.data());
+  const double sw = fp8_quantize(w, n * k, fmt, false, qw.data());
   mm_nt(qx.data(), qw.data(), rows, n, k, y);
   const double inv = 1.0 / (sx * sw);
   for (int64_t i = 0; i < rows * n; ++i) y[i] *= inv;
 }
 
-// dx (+)= dy W on quantised operands.
+// dx (+)= dy W on quantised operands (dy a gradient, W a weight).
 void fp8_mm_nn(const double* dy, const double* w, int64_t rows, int64_t n, int64_t k, int fmt,
                double* dx, bool accumulate) {
   std::vector<double> qd(rows * n), qw(n * k), t(rows * k);
-  const double sd = fp8_quantize(dy, rows * n, fmt, qd.data());
-  const double sw = fp8_quantize(w, n * k, fmt, qw.data());
+  const double sd = fp8_quantize(dy, rows * n, fmt, true, qd.data());
+  const double sw = fp8_quantize(w, n * k, fmt, false, qw.data());
   mm_nn_acc(qd.data(), qw.data(), rows, n, k, t.data(), false);
   const double inv = 1.0 / (sd * sw);
   for (int64_t i = 0; i < rows * k; ++i) dx[i] = (accumulate ? dx[i] : 0.0) + t[i] * inv;
 }
 
-// dW = dy^T x on quantised operands.
+// dW = dy^T x on quantised operands (both activations or gradients).
 void fp8_mm_tn(const double* dy, const double* x, int64_t rows, int64_t n, int64_t k, int fmt,
                double* dw) {
   std::vector<double> qd(rows * n), qx(rows * k);
-  const double sd = fp8_quantize(dy, rows * n, fmt, qd.data());
-  const double sx = fp8_quantize(x, rows * k, fmt, qx.data());
+  const double sd = fp8_quantize(dy, rows * n, fmt, true, qd.data());
+  const double sx = fp8_quantize(x, rows * k, fmt, true, qx.data());
   mm_tn(qd.data(), qx.data(), rows, n, k, dw);
   const double inv = 1.0 / (sd * sx);
   for (int64_t i = 0; i < n * k; ++i) dw[i] *= inv;
@@ -634,8 +655,8 @@ int oc_threads(int n) {
   return omp_get_max_threads();
 }
 
-float oc_fp8_scale(const double* x, int64_t n) {
-  return (x && n > 0) ? fp8_scale(x, n) : -1.0f;
+float oc_fp8_scale(const double* x, int64_t n, int act) {
+  return (x && n > 0) ? fp8_scale(x, n, 1, act != 0) : -1.0f;
 }
 
 int oc_fp8_matmul_nt(const double* x, const double* w, int64_t rows, int64_t n, int64_t k,

@@ -150,11 +150,15 @@ int oc_gpt_fwd_bwd_ex(int depth, int vocab, int n_kv_head, const int32_t* window
  * largest finite 448, subnormals k * 2^-9).
  * oc_e4m3_round: nearest E4M3 value, ties to the even mantissa, magnitudes
  *   above 448 (infinities too) saturate to 448; NaN stays NaN.
- * oc_fp8_scale: per-tensor scale s = 448 / max|fp32(x_i)| in fp32
- *   arithmetic (1 if all are zero; -1 on a bad argument).
+ * Operands are quantised from the values a kernel holds: weights from
+ * fp32(t_i), activations and their gradients (bf16 in memory) from
+ * bf16(fp32(t_i)) -- the decision taken in the kernel's precision.
+ * oc_fp8_scale: per-tensor scale s = 448 / max|v_i| in fp32 arithmetic,
+ *   v the source values (act != 0: an activation); 1 if all are zero; -1
+ *   on a bad argument.
  * oc_fp8_matmul_nt: y = (Q(x) Q(w)^T) / (s_x s_w) with Q(t)_i =
- *   e4m3(fp32(t_i) * s_t) (fmt 1) or fp32(t_i) * s_t (fmt 0, scaling
- *   alone); x [rows, k], w [n, k].
+ *   e4m3(v_i * s_t) (fmt 1) or fp32(t_i) * s_t (fmt 0, scaling alone, no
+ *   bf16 step); x [rows, k] an activation, w [n, k] a weight.
  * oc_gpt_fwd_bwd_fp8: oc_gpt_fwd_bwd_ex with every GEMM of the block
  *   projections (forward, input gradient, weight gradient of wq|wk|wv, wo,
  *   wup, wdown) computed that way; the fused q|k|v weight [d + 2 dkv, d]
@@ -165,7 +169,7 @@ double oc_e4m3_round(double x);
 /* OpenMP threads of later calls: n > 0 sets them; returns the count in
  * effect (for timing the oracle at one thread and at all cores). */
 int oc_threads(int n);
-float oc_fp8_scale(const double* x, int64_t n);
+float oc_fp8_scale(const double* x, int64_t n, int act);
 int oc_fp8_matmul_nt(const double* x, const double* w, int64_t rows, int64_t n, int64_t k,
                      int fmt, double* y);
 int oc_gpt_fwd_bwd_fp8(int depth, int vocab, int n_kv_head, const int32_t* window, int fmt,

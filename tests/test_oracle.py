@@ -786,24 +786,21 @@ def test_e4m3_round_special_values():
 def test_fp8_scale_is_448_over_amax_in_fp32():
     x = np.array([0.3, -1.7, 0.01])
     assert oracle.fp8_scale(x) == np.float32(448.0) / np.float32(1.7)
+    # an activation's amax is that of its bf16 value (1.7 -> 1.703125)
+    assert oracle.fp8_scale(x, activation=True) == np.float32(448.0) / np.float32(1.703125)
     assert oracle.fp8_scale(np.zeros(5)) == 1.0
 
 
 def test_fp8_matmul_brute_force():
     """Per-tensor scaling and E4M3 rounding written here with the table:
-    y = (Q(x) Q(w)^T) / (s_x s_w), Q(t) = e4m3(fp32(t) * s_t)."""
+    y = (Q(x) Q(w)^T) / (s_x s_w), Q(t) = e4m3(v * s_t) with v the value a
+    kernel holds: bf16 for the activation x, fp32 for the weight w."""
     t = _e4m3_table()
     rng = np.random.default_rng(61)
     x = rng.standard_normal((5, 24)) * 3.0
     w = rng.standard_normal((7, 24)) * 0.02
-
-    def q(a):
-        s = np.float32(448.0) / np.float32(np.abs(a.astype(np.float32)).max())
-        y = (a.astype(np.float32) * s).astype(np.float64)
-        return _e4m3_nearest(y.ravel(), t).reshape(a.shape), float(s)
-
-    qx, sx = q(x)
-    qw, sw = q(w)
+    qx, sx = _quant_table(x, t, act=True)
+    qw, sw = _quant_table(w, t)
     ref = qx @ qw.T / (sx * sw)
     np.testing.assert_allclose(oracle.fp8_matmul_nt(x, w), ref, rtol=1e-12, atol=1e-15)
     # Scaling alone is exact up to fp32 rounding of the operands.
@@ -861,9 +858,12 @@ def test_fp8_model_e4m3_is_close_to_the_exact_model():
     assert rel[-1] < 0.15 and rel[-1] <= np.median(rel)
 
 
-def _quant_table(a, t):
-    """Q(a) and s written here: s = 448 / amax in fp32, codes from the table."""
+def _quant_table(a, t, act=False):
+    """Q(a) and s written here: s = 448 / amax in fp32, codes from the table;
+    an activation is first rounded to bf16 (the value a kernel holds)."""
     a32 = np.asarray(a, dtype=np.float32)
+    if act:
+        a32 = inputs.round_to_bf16(a32)
     amax = np.abs(a32).max()
     s = np.float32(448.0) / amax if amax > 0 else np.float32(1.0)
     y = (a32 * s).astype(np.float64)  # the fp32 product
@@ -884,22 +884,19 @@ def test_fp8_rounding_decision_is_taken_on_the_fp32_product():
             if float(np.float32(x) * s) == tie and exact != tie:
                 picked.append(float(x))
     assert len(picked) >= 10
-    x = np.array([3.3] + picked)
-    w = np.eye(len(x))[:1]  # a single output: y_0 = Q(x)_0 * Q(w)_0 / (s_x s_w)
-    qx, sx = _quant_table(x, t)
-    # Q(w) = e4m3(1 * 448) = 448, s_w = 448, so y_j = Q(x)_j / s_x for a w
-    # that selects element j; check every picked element this way.
-    for j in range(len(x)):
-        wj = np.zeros((1, len(x)))
-        wj[0, j] = 1.0
-        y = oracle.fp8_matmul_nt(x[None, :], wj)[0, 0]
-        assert abs(y - qx[j] / sx) <= 1e-12 * abs(qx[j] / sx), (j, x[j])  # codes 1/8 apart
+    # The values go in as a weight (quantised from fp32); the activation is the
+    # identity, whose codes are exact (448 at s = 448), so y[j] = Q(w)_j / s_w.
+    w = np.array([[3.3] + picked])
+    qw, sw = _quant_table(w, t)
+    y = oracle.fp8_matmul_nt(np.eye(w.shape[1]), w)[:, 0]
+    np.testing.assert_allclose(y, qw[0] / sw, rtol=1e-12, atol=0)  # codes 1/8 apart
 
 
 def test_fp8_model_mlp_gradients_brute_force():
     """depth 1 with wo = 0: attention adds nothing, so the MLP sees the
     embedding and everything its weight gradients need is computed here on
-    quantised operands (Q(t) = e4m3(fp32(t) s_t), s_t = 448 / amax):
+    quantised operands (Q(t) = e4m3(v s_t), s_t = 448 / amax, v = bf16(t)
+    for activations and gradients, fp32(t) for the weights):
       u = Q(h) Q(wup)^T / ss, a = relu(u)^2, m = Q(a) Q(wdown)^T / ss,
       x_f = x + m, loss through the final RMSNorm and the exact lm_head;
       dW_down = Q(dx_f)^T Q(a) / ss,  da = Q(dx_f) Q(wdown) / ss,
@@ -913,9 +910,9 @@ def test_fp8_model_mlp_gradients_brute_force():
     _, G, _ = oracle.gpt_fwd_bwd(1, P, tok, tgt, vocab=V, fp8="e4m3")
     N = tok.size
 
-    def qmm(a, b):  # a b^T on quantised operands
-        qa, sa = _quant_table(a, t)
-        qb, sb = _quant_table(b, t)
+    def qmm(a, b, a_act=True, b_act=True):  # a b^T on quantised operands
+        qa, sa = _quant_table(a, t, a_act)
+        qb, sb = _quant_table(b, t, b_act)
         return qa @ qb.T / (sa * sb)
 
     def rms_fwd_bwd(x, dy=None):
@@ -926,9 +923,9 @@ def test_fp8_model_mlp_gradients_brute_force():
 
     x = P[0][tok.ravel()].astype(np.float64)
     h = rms_fwd_bwd(x)
-    u = qmm(h, P[5])
+    u = qmm(h, P[5], b_act=False)
     a = np.maximum(u, 0.0) ** 2
-    xf = x + qmm(a, P[6])
+    xf = x + qmm(a, P[6], b_act=False)
     lm = P[-1].astype(np.float64)
     z = rms_fwd_bwd(xf) @ lm.T
     p = np.exp(z - z.max(axis=1, keepdims=True))
@@ -936,7 +933,7 @@ def test_fp8_model_mlp_gradients_brute_force():
     p[np.arange(N), tgt.ravel()] -= 1.0
     dxf = rms_fwd_bwd(xf, (p / N) @ lm)
     dwdown = qmm(dxf.T, a.T)          # Q(dx_f)^T Q(a)
-    da = qmm(dxf, P[6].T.copy())      # Q(dx_f) Q(wdown)
+    da = qmm(dxf, P[6].T.copy(), b_act=False)  # Q(dx_f) Q(wdown)
     du = 2.0 * np.maximum(u, 0.0) * da
     dwup = qmm(du.T, h.T)
     for got, ref in ((G[6], dwdown), (G[5], dwup)):
