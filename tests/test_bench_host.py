@@ -27,3 +27,35 @@ def test_window_term_tracks_the_pairs_a_window_leaves():
                 bench.step_flops_per_token(depth, T, 8, 0, [0, 0]))
         band = term / (2 * 12.0 * d) * T                   # the convention's pair count, minus w = 0
         assert abs(band - (pairs - T)) <= max(1.0, 0.01 * pairs), (w, band, pairs - T)
+
+
+def test_newton_schulz_flops_closed_form():
+    """Per iteration, a d x d matrix costs three d^3 products (6 d^3) and a
+    d x 4d one X X^T, A A, B X (8 + 2 + 8 = 18 d^3); 4L squares, 2L wide, five
+    iterations: 300 L d^3."""
+    for depth in (2, 12, 20, 26):
+        d = 64 * depth
+        assert bench.ns_flops(depth) == 300.0 * depth * d ** 3
+
+
+def test_training_flops_per_token_at_three_depths():
+    """6 N_mm + 6 L d T with N_mm = 12 L d^2 + V d: 0.774, 2.926 and 6.042
+    GFLOP per token at depths 12, 20 and 26 (T 2048, V 32768)."""
+    for depth, gflop in ((12, 0.774), (20, 2.926), (26, 6.042)):
+        assert abs(bench.model_flops_per_token(depth) / 1e9 - gflop) < 5e-4
+
+
+def test_gemm_byte_model_counts_every_launch_of_the_step():
+    """Twelve GEMMs per layer, three for lm_head and thirty for Newton-Schulz
+    (five iterations of three products on two stacks): 273 at depth 20, with
+    231.1 GB of operands and results."""
+    total, launches = bench.gemm_algorithmic_bytes_per_step()
+    assert launches == 20 * 12 + 3 + 30 == 273
+    assert abs(total / 1e9 - 231.1) < 0.1
+    # Doubling the batch doubles every activation term and leaves weights.
+    t2, _ = bench.gemm_algorithmic_bytes_per_step(batch=2 * bench.B)
+    assert total < t2 < 2 * total
+
+
+def test_replica_throughput_counts_all_ranks():
+    assert bench.replica_tokens_per_s(10, 4, 1000.0) == 10 * bench.B * bench.T * 4
