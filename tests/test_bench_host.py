@@ -59,3 +59,15 @@ def test_gemm_byte_model_counts_every_launch_of_the_step():
 
 def test_replica_throughput_counts_all_ranks():
     assert bench.replica_tokens_per_s(10, 4, 1000.0) == 10 * bench.B * bench.T * 4
+
+
+def test_step_times_are_the_gaps_between_marks():
+    class Mark:
+        def __init__(self, t):
+            self.t = t
+
+        def elapsed_time(self, other):
+            return other.t - self.t
+
+    marks = [Mark(t) for t in (0.0, 2.0, 5.0, 6.5)]
+    assert bench.step_times_ms(marks) == [2.0, 3.0, 1.5]
