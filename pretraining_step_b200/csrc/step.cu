@@ -350,8 +350,10 @@ nc_status proj_dw(nc_params* p, const bf16* dy, int64_t ldy, int64_t Mo, const b
   return gemm_launch(g, p->stream, p->prof);
 }
 
+// ids_on_device: the caller has established that tokens and targets are
+// device memory (a graph capture, which records no pointer queries).
 nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, int B, int T,
-                  float* loss_dev, nc_grads* g) {
+                  float* loss_dev, nc_grads* g, bool ids_on_device = false) {
   if (p->poisoned) return fail(NC_ERR_TIMEOUT, "handle poisoned by an earlier device timeout");
   if (!tokens || !targets || !g || g->p != p || B < 1 || T < 1 || (int64_t)B * T > (1 << 24))
     return fail(NC_ERR_INVALID_ARG, "fwd_bwd: bad arguments");
@@ -367,11 +369,11 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
 
   const int32_t* tok = tokens;
   const int32_t* tgt = targets;
-  if (!is_device_ptr(tokens)) {
+  if (!ids_on_device && !is_device_ptr(tokens)) {
     NC_CUDA_TRY(cudaMemcpyAsync(a.tok, tokens, 4 * N, cudaMemcpyHostToDevice, s));
     tok = a.tok;
   }
-  if (!is_device_ptr(targets)) {
+  if (!ids_on_device && !is_device_ptr(targets)) {
     NC_CUDA_TRY(cudaMemcpyAsync(a.tgt, targets, 4 * N, cudaMemcpyHostToDevice, s));
     tgt = a.tgt;
   }
@@ -834,7 +836,7 @@ nc_status nc_step_capture(nc_params* p, const int32_t* tokens, const int32_t* ta
     profiler_enable(p->prof, prof_on);
     return cuda_fail(e, "step_capture: begin capture");
   }
-  nc_status st = fwd_bwd(p, tokens, targets, B, T, loss_dev, g);
+  nc_status st = fwd_bwd(p, tokens, targets, B, T, loss_dev, g, true);
   if (st == NC_OK) st = muon(p, g, lr, momentum);
   cudaGraph_t graph = nullptr;
   e = cudaStreamEndCapture(p->stream, &graph);  // always ends the capture
