@@ -33,6 +33,14 @@ def test_library_exports_every_declared_symbol():
     assert not missing, missing
 
 
+def test_binding_declares_a_signature_for_every_entry_point():
+    """Every function of the C ABI is marshalled with declared argument and
+    result types (ctypes would otherwise pass Python ints as C int)."""
+    L = binding.lib()
+    undeclared = [n for n in sorted(_declared()) if getattr(L, n).argtypes is None]
+    assert not undeclared, undeclared
+
+
 def test_status_strings():
     assert binding.status_string(binding.NC_OK) == "ok"
     assert binding.status_string(binding.NC_ERR_TIMEOUT) == "device wait timed out"
