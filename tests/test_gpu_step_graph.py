@@ -18,8 +18,12 @@ def _gpt(depth, **kw):
 def test_step_graph_matches_eager_steps():
     """A captured step (fwd + bwd + Muon as one CUDA graph) replayed over
     three batches written in place matches the same calls made eagerly on a
-    twin model: losses and weights agree up to the order of the weight
-    gradient's atomic sums."""
+    twin model.  The step is not bitwise deterministic: the weight-gradient
+    split-K sums, the attention dQ sums, the embedding scatter and Muon's
+    squared norms are fp32 atomics whose order varies, and Newton-Schulz
+    magnifies that noise along small singular directions.  So a third model,
+    an eager twin of the first, measures the spread two eager runs show, and
+    the graph must stay within a small multiple of it."""
     t = torch()
     depth, B, T, lr, mu = 2, 2, 128, 0.02, 0.95
     s = t.cuda.Stream()
@@ -34,10 +38,12 @@ def test_step_graph_matches_eager_steps():
     w.close()
     a = _gpt(depth, seed=31, all_random=True, stream=s)
     b = _gpt(depth, seed=31, all_random=True, stream=s)
+    c = _gpt(depth, seed=31, all_random=True, stream=s)  # eager control
     tok_d = t.zeros((B, T), dtype=t.int32, device=dev)
     tgt_d = t.zeros((B, T), dtype=t.int32, device=dev)
     loss_a = t.zeros(1, dtype=t.float32, device=dev)
     loss_b = t.zeros(1, dtype=t.float32, device=dev)
+    loss_c = t.zeros(1, dtype=t.float32, device=dev)
     t.cuda.synchronize()
     launches0 = b.launch_count()
     b.capture_step(tok_d, tgt_d, loss_b, lr, mu)
@@ -52,17 +58,26 @@ def test_step_graph_matches_eager_steps():
             tgt_d.copy_(t.from_numpy(tg))
             a.fwd_bwd_async(tok_d, tgt_d, loss_a)
             a.muon_step(lr, mu)
+            c.fwd_bwd_async(tok_d, tgt_d, loss_c)
+            c.muon_step(lr, mu)
             b.replay_step()
         a.sync()
         b.sync()
-        la, lb = float(loss_a.item()), float(loss_b.item())
-        assert abs(la - lb) <= 1e-4 * abs(la), (i, la, lb)
+        c.sync()
+        la, lb, lc = float(loss_a.item()), float(loss_b.item()), float(loss_c.item())
+        assert abs(la - lb) <= max(3 * abs(la - lc), 1e-4 * abs(la)), (i, la, lb, lc)
     assert b.launch_count() - launches0 == a.launch_count() - la0 > 0  # same kernels per step
-    for i, (x, y, w0) in enumerate(zip(a.params(), b.params(), W0)):
-        moved = np.linalg.norm(x.astype(np.float64) - w0)
+    diff, spread = 0.0, 0.0
+    for i, (x, y, z, w0) in enumerate(zip(a.params(), b.params(), c.params(), W0)):
+        x = x.astype(np.float64)
+        moved = np.linalg.norm(x - w0)
         if moved == 0:  # wte and lm_head: not Muon's
-            assert np.array_equal(x, y), i
-        else:
-            assert np.linalg.norm(x.astype(np.float64) - y) <= 1e-3 * moved, i
+            assert np.array_equal(x, y) and np.array_equal(x, z), i
+            continue
+        diff = max(diff, np.linalg.norm(x - y) / moved)
+        spread = max(spread, np.linalg.norm(x - z) / moved)
+    assert spread < 0.1, spread  # the eager noise itself stays small
+    assert diff <= max(3 * spread, 1e-3), (diff, spread)
     a.close()
     b.close()
+    c.close()
