@@ -32,11 +32,13 @@ METRIC = "train tokens/s and MFU (bf16 peak) at depth-20 GPT, 1×B200"
 DEPTH, B, T, V = 20, 32, 2048, 32768
 LR, MOMENTUM = 0.02, 0.95
 NOMINAL_BF16_TFLOPS = 2250.0
-# DRAM bytes (read + write) per GEMM launch, averaged over the 273 GEMM
-# launches of one step of this workload: ncu dram__bytes_read.sum +
-# dram__bytes_write.sum, profiles/step_d20_b32_t2048_launches.md.  Valid
-# for the GEMM kernels as captured there; set to None when they change.
-GEMM_DRAM_BYTES_PER_LAUNCH = 1017.3e6
+# DRAM traffic of the GEMM engine: ncu dram__bytes_read.sum +
+# dram__bytes_write.sum of one launch of each GEMM class on a small case
+# (profiles/gemm_traffic_by_class.md), as a ratio to that launch's
+# algorithmic operand + result bytes.  The step's traffic per GEMM launch is
+# each class's algorithmic bytes times its ratio, averaged over the launches.
+# None until captured for the kernels as they stand.
+GEMM_TRAFFIC_RATIO = None
 
 
 def model_flops_per_token(depth=DEPTH, seq=T, vocab=V):
@@ -64,21 +66,27 @@ def step_flops_per_token(depth, seq, vocab, n_kv_head=0, windows=None):
     return 6.0 * n_mm + attn
 
 
-def gemm_algorithmic_bytes_per_step(depth=DEPTH, batch=B, seq=T, vocab=V):
+def gemm_algorithmic_bytes_by_class(depth=DEPTH, batch=B, seq=T, vocab=V):
     """Operand and result bytes of every GEMM launch of one step, each operand
     read once and each result written once (bf16 2 B, fp32 4 B; a split-K
-    weight gradient counts as one fp32 write).  Returns (bytes, launches)."""
+    weight gradient counts as one fp32 write), summed per launch class:
+    fwd, dgrad, wgrad (the block projections), lmhead, ns (Newton-Schulz).
+    Returns ({class: bytes}, {class: launches})."""
     d, f, n = 64 * depth, 4 * 64 * depth, batch * seq
     bf, f4 = 2, 4
-    per_layer = [
+    fwd = [
         n * d * bf + 3 * d * d * bf + n * 3 * d * bf,          # q|k|v (+ RoPE / QK-norm)
         n * d * bf + d * d * bf + 2 * n * d * f4,              # o-projection + fp32 residual
         n * d * bf + f * d * bf + n * f * bf,                  # MLP up + ReLU^2
         n * f * bf + d * f * bf + 2 * n * d * f4,              # MLP down + fp32 residual
+    ]
+    dgrad = [
         n * d * bf + d * f * bf + 2 * n * f * bf,              # du = dy W_down, 2 sqrt(a)
         n * f * bf + f * d * bf + n * d * bf,                  # dh = du W_up
         n * d * bf + d * d * bf + n * d * bf,                  # dh = dy W_o
         n * 3 * d * bf + 3 * d * d * bf + n * d * bf,          # dh = dqkv W_qkv
+    ]
+    wgrad = [
         n * d * bf + n * f * bf + d * f * f4,                  # dW_down
         n * f * bf + n * d * bf + f * d * f4,                  # dW_up
         2 * n * d * bf + d * d * f4,                           # dW_o
@@ -92,8 +100,17 @@ def gemm_algorithmic_bytes_per_step(depth=DEPTH, batch=B, seq=T, vocab=V):
     for cnt, m, k in ((sq, d, d), (wide, d, f)):
         x, a = cnt * m * k * bf, cnt * m * m * bf
         ns += 5 * ((x + a) + (a + a) + (a + x + x))         # A = X X^T; B = cA^2 + bA; Y = BX + aX
-    total = depth * sum(per_layer) + sum(lm) + ns
-    return float(total), depth * len(per_layer) + len(lm) + 30
+    nbytes = {"fwd": float(depth * sum(fwd)), "dgrad": float(depth * sum(dgrad)),
+              "wgrad": float(depth * sum(wgrad)), "lmhead": float(sum(lm)), "ns": float(ns)}
+    launches = {"fwd": 4 * depth, "dgrad": 4 * depth, "wgrad": 4 * depth, "lmhead": 3, "ns": 30}
+    return nbytes, launches
+
+
+def gemm_algorithmic_bytes_per_step(depth=DEPTH, batch=B, seq=T, vocab=V):
+    """All GEMM classes of gemm_algorithmic_bytes_by_class together.
+    Returns (bytes, launches)."""
+    nbytes, launches = gemm_algorithmic_bytes_by_class(depth, batch, seq, vocab)
+    return float(sum(nbytes.values())), sum(launches.values())
 
 
 def max_over_ranks(x, world, device="cpu"):
@@ -126,6 +143,25 @@ def ns_flops(depth=DEPTH):
     sq = 2 * d ** 3 * 3                      # X X^T, A A, B X for d x d
     wide = 2 * (d * d * 4 * d) * 2 + 2 * d ** 3  # X X^T and B X at n = 4d, A A at d
     return 5.0 * (4 * depth * sq + 2 * depth * wide)
+
+
+def tensor_peak_at(sm_mhz, sms=148):
+    """Dense bf16 tcgen05 rate at a given SM clock: 8192 FLOP per clock per
+    SM (M128 x N256 x K16 in 128 clocks), in TFLOP/s."""
+    return 8192.0 * sms * sm_mhz * 1e6 / 1e12
+
+
+def gemm_traffic_per_launch(depth=DEPTH, batch=B, seq=T, vocab=V):
+    """Modelled DRAM bytes per GEMM launch of one step from the per-class
+    ratios of GEMM_TRAFFIC_RATIO (None when no capture covers the kernels)."""
+    if not GEMM_TRAFFIC_RATIO:
+        return None, "no small-case capture of the current GEMM kernels"
+    by_class, _ = gemm_algorithmic_bytes_by_class(depth, batch, seq, vocab)
+    total = sum(GEMM_TRAFFIC_RATIO[c] * b for c, b in by_class.items())
+    _, launches = gemm_algorithmic_bytes_per_step(depth, batch, seq, vocab)
+    return total / launches, ("per-class DRAM/algorithmic ratios from one-launch ncu captures "
+                              "(profiles/gemm_traffic_by_class.md) times each class's "
+                              "algorithmic bytes in the step")
 
 
 def workload_name():
@@ -195,30 +231,68 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU oracle sample
-def cpu_oracle_sample(budget_s=20.0, per_step=False):
+def host_cpu():
+    """CPU model name and logical core count of this host."""
+    name = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    name = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return name, os.cpu_count() or 1
+
+
+def oracle_attention_seconds(heads, seed=5):
+    """Oracle causal attention forward + backward of one row of T = 2048
+    tokens with `heads` heads of 128 (the oracle parallelises over heads)."""
+    import oracle
+    from pretraining_step_b200 import inputs
+    d = heads * 128
+    qkv = inputs.bf16_normal(seed, (T, 3 * d))
+    q = qkv[:, :d].reshape(1, T, heads, 128)
+    k = qkv[:, d:2 * d].reshape(1, T, heads, 128)
+    v = qkv[:, 2 * d:].reshape(1, T, heads, 128)
+    t0 = time.perf_counter()
+    o, lse, _ = oracle.attention(q, k, v)
+    oracle.attention_bwd(q, k, v, lse, o)
+    return time.perf_counter() - t0
+
+
+def cpu_oracle_sample():
     """Time the oracle on a bounded sample of the workload and convert to the
-    workload's tokens/s: forward+backward on a short row (cost per token) and
-    the Newton-Schulz of one matrix of each Muon shape (cost per matrix), on
-    all host cores; then the same at one thread on a smaller sample (2
-    tokens, one (d/2) x (d/2) Newton-Schulz scaled by its FLOPs)."""
+    workload's tokens/s.  A B = 1, T = 2048 row of depth 20 is far beyond a
+    few seconds of fp64 work, so its two parts are timed separately: the
+    per-token part (every projection, norm and the loss) from forward +
+    backward on a 16-token row, and the part quadratic in T (causal attention
+    forward + backward) on one T = 2048 row with as many heads as threads,
+    scaled to the step's 32 rows x 20 layers x 10 heads; plus the
+    Newton-Schulz of one matrix of each Muon shape, scaled to 80 + 40.  Then
+    the same at one thread on a smaller sample."""
     import numpy as np
     import oracle
     from pretraining_step_b200 import inputs
     oracle.lib()
     threads_all = oracle.threads()
+    cpu_name, nproc = host_cpu()
     P = inputs.random_params(DEPTH, seed=1)
     t_tok = 16
     tok, tgt = inputs.token_batch(2, 1, t_tok)
     t0 = time.perf_counter()
     oracle.gpt_fwd_bwd(DEPTH, P, tok, tgt)
     fb = time.perf_counter() - t0
+    heads = max(1, min(threads_all, 16))
+    att = oracle_attention_seconds(heads)
+    head_rows = B * DEPTH * (64 * DEPTH // 128)      # (row, layer, head) attention units
     t0 = time.perf_counter()
     oracle.newton_schulz(P[1])                  # one d x d matrix (of 80)
     ns_sq = time.perf_counter() - t0
     t0 = time.perf_counter()
     oracle.newton_schulz(P[5])                  # one 4d x d matrix (of 40)
     ns_w = time.perf_counter() - t0
-    step_s = fb / t_tok * (B * T) + 4 * DEPTH * ns_sq + 2 * DEPTH * ns_w
+    step_s = fb / t_tok * (B * T) + att / heads * head_rows + 4 * DEPTH * ns_sq + 2 * DEPTH * ns_w
     # One thread.  Newton-Schulz costs 6 n^3 per iteration for an n x n matrix
     # and 18 n^3 for the 4n x n one (4 m n^2 + 2 n^3 with m = 4n), so the
     # (d/2)^2 sample scales by 8 to d x d and by 24 to 4d x d.
@@ -229,6 +303,7 @@ def cpu_oracle_sample(budget_s=20.0, per_step=False):
         t0 = time.perf_counter()
         oracle.gpt_fwd_bwd(DEPTH, P, tok1, tgt1)
         fb1 = time.perf_counter() - t0
+        att1 = oracle_attention_seconds(1)
         d = 64 * DEPTH
         G = np.asarray(P[1][: d // 2, : d // 2], dtype=np.float64)
         t0 = time.perf_counter()
@@ -236,55 +311,70 @@ def cpu_oracle_sample(budget_s=20.0, per_step=False):
         ns1 = time.perf_counter() - t0
     finally:
         oracle.threads(threads_all)
-    step1_s = fb1 / t1_tok * (B * T) + 4 * DEPTH * 8 * ns1 + 2 * DEPTH * 24 * ns1
+    step1_s = fb1 / t1_tok * (B * T) + att1 * head_rows + 4 * DEPTH * 8 * ns1 + \
+        2 * DEPTH * 24 * ns1
     return {
         "value": (B * T) / step_s,
         "unit": "tokens/s",
         "cores": threads_all,
         "kind": "oracle",
-        "sample": ("double-precision CPU oracle on %d threads: forward+backward of depth 20 on "
-                   "1 x %d tokens (%.1f s) scaled to 65536 tokens, plus Newton-Schulz of one "
-                   "1280x1280 (%.1f s) and one 5120x1280 matrix (%.1f s) scaled to 80 + 40 "
-                   "matrices" % (threads_all, t_tok, fb, ns_sq, ns_w)),
-        "sample_seconds": fb + ns_sq + ns_w,
+        "host": {"cpu": cpu_name, "nproc": nproc, "omp_threads": threads_all},
+        "sample": ("double-precision CPU oracle on %d threads: per-token part from forward + "
+                   "backward of depth 20 on 1 x %d tokens (%.1f s) scaled to 65536 tokens; "
+                   "attention forward + backward of one T=2048 row with %d heads (%.1f s) "
+                   "scaled to 32 rows x 20 layers x 10 heads; Newton-Schulz of one 1280x1280 "
+                   "(%.1f s) and one 5120x1280 matrix (%.1f s) scaled to 80 + 40 matrices"
+                   % (threads_all, t_tok, fb, heads, att, ns_sq, ns_w)),
+        "sample_seconds": fb + att + ns_sq + ns_w,
         "one_thread": {
             "value": (B * T) / step1_s, "unit": "tokens/s", "cores": 1,
             "sample": ("forward+backward on 1 x %d tokens (%.1f s) scaled to 65536 tokens, "
-                       "plus Newton-Schulz of one 640x640 matrix (%.1f s) scaled by FLOPs to "
-                       "80 x 1280^2 and 40 x 5120x1280" % (t1_tok, fb1, ns1)),
-            "sample_seconds": fb1 + ns1,
+                       "attention of one T=2048 head (%.1f s) scaled to 6400 head-rows, "
+                       "Newton-Schulz of one 640x640 matrix (%.1f s) scaled by FLOPs to "
+                       "80 x 1280^2 and 40 x 5120x1280" % (t1_tok, fb1, att1, ns1)),
+            "sample_seconds": fb1 + att1 + ns1,
         },
     }
 
 
 # ------------------------------------------------------------------ reference arm
 def run_reference(args, rank):
+    """The oracle, as it stands, on the host cores: each step is a bounded
+    sample of the workload (forward + backward on an 8-token row, the
+    attention forward + backward of one T = 2048 row, and the Newton-Schulz
+    of one block matrix), converted to the 65536-token step's time."""
     if rank != 0:
         return 0
     from pretraining_step_b200 import inputs
     import oracle
     oracle.lib()
+    threads = oracle.threads()
+    heads = max(1, min(threads, 16))
+    head_rows = B * DEPTH * (64 * DEPTH // 128)
     P = inputs.random_params(DEPTH, seed=1)
     t_tok = 8
-    times_fb, times_ns = [], {"sq": [], "w": []}
+    times_fb, times_att, times_ns = [], [], {"sq": [], "w": []}
     for step in range(args.warmup + args.steps):
         tok, tgt = inputs.token_batch(100 + step, 1, t_tok)
         t0 = time.perf_counter()
         oracle.gpt_fwd_bwd(DEPTH, P, tok, tgt)
         fb = time.perf_counter() - t0
+        att = oracle_attention_seconds(heads, seed=200 + step)
         which = "sq" if step % 2 == 0 else "w"
         t0 = time.perf_counter()
         oracle.newton_schulz(P[1] if which == "sq" else P[5])
         ns = time.perf_counter() - t0
         if step >= args.warmup:
             times_fb.append(fb)
+            times_att.append(att)
             times_ns[which].append(ns)
     fb_tok = float(np.mean(times_fb)) / t_tok
+    att_row = float(np.mean(times_att)) / heads
     ns_sq = float(np.mean(times_ns["sq"])) if times_ns["sq"] else 0.0
     ns_w = float(np.mean(times_ns["w"])) if times_ns["w"] else ns_sq * 4.5
-    step_s = fb_tok * B * T + 4 * DEPTH * ns_sq + 2 * DEPTH * ns_w
+    step_s = fb_tok * B * T + att_row * head_rows + 4 * DEPTH * ns_sq + 2 * DEPTH * ns_w
     value = B * T / step_s
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    cpu_name, nproc = host_cpu()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
@@ -292,11 +382,13 @@ def run_reference(args, rank):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": workload_name(), "global_batch": B, "seq_len": T,
                    "parallelism": "none (host cores)"},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": "each step: oracle forward+backward on 1 x %d tokens and "
-                                   "Newton-Schulz of one block matrix (alternating 1280x1280 / "
-                                   "5120x1280), scaled to the 65536-token step and 120 "
-                                   "matrices" % t_tok},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "host": {"cpu": cpu_name, "nproc": nproc, "omp_threads": threads},
+                         "sample": "each step: oracle forward+backward on 1 x %d tokens, "
+                                   "attention forward+backward of one T=2048 row with %d "
+                                   "heads, and Newton-Schulz of one block matrix (alternating "
+                                   "1280x1280 / 5120x1280), scaled to the 65536-token step, "
+                                   "6400 attention head-rows and 120 matrices" % (t_tok, heads)},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -340,11 +432,24 @@ def run_native(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
-    # ---- device-timed region (inputs resident)
+    # The step as one CUDA graph: it reads its token ids from tok_g / tgt_g,
+    # refilled on the stream from the resident batches before every replay.
+    tok_g = torch.empty_like(toks[0])
+    tgt_g = torch.empty_like(tgts[0])
+    m.capture_step(tok_g, tgt_g, loss_dev, LR, MOMENTUM)
+
+    def replay(i):
+        tok_g.copy_(toks[i % nbat])
+        tgt_g.copy_(tgts[i % nbat])
+        m.replay_step()
+
+    with torch.cuda.stream(stream):
+        replay(0)  # first launch of the instantiated graph, untimed
+        m.sync()
+
+    # ---- device-timed region (inputs resident, no per-launch profiling events)
     clocks = ClockSampler(local_rank)
     clocks.start()
-    m.profile(True)
-    m.profile_read()  # reset
     launches0 = m.launch_count()
     barrier()
     torch.cuda.synchronize()
@@ -355,7 +460,7 @@ def run_native(args, rank, world, local_rank):
         e0.record(stream)
         marks[0].record(stream)
         for i in range(args.steps):
-            step(i)
+            replay(i)
             marks[i + 1].record(stream)
         e1.record(stream)
     m.sync()
@@ -363,12 +468,28 @@ def run_native(args, rank, world, local_rank):
     barrier()
     launches = m.launch_count() - launches0
     ms = e0.elapsed_time(e1)
-    prof = m.profile_read()
-    m.profile(False)
     clk = clocks.stop()
     ms_max = max_over_ranks(ms, world, dev)
     median_max = max_over_ranks(float(np.median(step_times_ms(marks))), world, dev)
     final_loss = float(loss_dev.item())
+
+    # ---- profiled pass: the same step run eagerly with CUDA events around
+    # every launch (on the launch stream), for the per-kernel table only.
+    prof_steps = 3
+    m.profile(True)
+    m.profile_read()  # reset
+    pe0 = torch.cuda.Event(enable_timing=True)
+    pe1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        pe0.record(stream)
+        for i in range(prof_steps):
+            step(i)
+        pe1.record(stream)
+    m.sync()
+    torch.cuda.synchronize()
+    prof = m.profile_read()
+    m.profile(False)
+    prof_ms_per_step = pe0.elapsed_time(pe1) / prof_steps
 
     # ---- end-to-end through the C ABI with host buffers
     pin_tok = [torch.from_numpy(inputs.token_batch(20 + 97 * rank + i, B, T)[0]).pin_memory()
@@ -423,6 +544,7 @@ def run_native(args, rank, world, local_rank):
     g_n = sum(v["launches"] for k, v in prof.items() if k.startswith("gemm_"))
     gemm_ach = g_fl / (g_ms / 1e3) / 1e12
     gemm_alg_bytes, gemm_alg_launches = gemm_algorithmic_bytes_per_step()
+    gemm_traffic, traffic_source = gemm_traffic_per_launch()
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
@@ -442,11 +564,18 @@ def run_native(args, rank, world, local_rank):
         "roofline": {"kernel": "gemm_tc (all classes)", "bound": "tensor", "achieved": gemm_ach,
                      "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
                      "frac": gemm_ach / peaks["bf16_tflops_sustained"],
-                     "traffic": GEMM_DRAM_BYTES_PER_LAUNCH,
-                     "traffic_unit": "bytes per launch (ncu DRAM read + write, mean over the step's GEMM launches)",
+                     "frac_at_step_clock": (gemm_ach / tensor_peak_at(clk["sm_mhz"])
+                                            if clk else None),
+                     "traffic": gemm_traffic,
+                     "traffic_unit": "bytes per launch",
+                     "traffic_source": traffic_source,
                      "traffic_algorithmic": gemm_alg_bytes / gemm_alg_launches,
                      "peak_source": peak_kind + " bf16_tflops_sustained",
-                     "launches": g_n, "ms": g_ms, "share": g_ms / total_ms},
+                     "launches_per_step": g_n / prof_steps, "ms_per_step": g_ms / prof_steps,
+                     "share": g_ms / total_ms},
+        "kernels_pass": {"steps": prof_steps, "ms_per_step": prof_ms_per_step,
+                         "how": "eager steps after the timed region, CUDA events around "
+                                "every launch on the launch stream"},
         "kernels": kernels,
         "gpu_launches": int(launches),
         "e2e": {"value": replica_tokens_per_s(e2e_steps, world, e2e_ms), "unit": "tokens/s",
@@ -471,6 +600,10 @@ def run_op(args):
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     if args.op == "step":
         return run_step_variant(args, dims, peaks, peak_kind)
+    if args.op == "ns_sweep":
+        return run_ns_sweep(args, peaks, peak_kind)
+    if args.op == "gemm_traffic":
+        return run_gemm_traffic(args)
     if args.op == "adamw":
         # AdamW on the depth-20 embedding and lm_head ([V, d] each): HBM-bound.
         m = nc.GPT(DEPTH, vocab=V, seed=7, all_random=True)
@@ -548,6 +681,136 @@ def run_op(args):
     return 0
 
 
+NS_SWEEP = ((64, 1664, 1664), (26, 1664, 6656), (26, 6656, 1664))
+
+
+def ns_sweep_flops(stacks=NS_SWEEP, steps=5):
+    """Newton-Schulz FLOPs of the sweep: per step and matrix, with m <= n the
+    short side, X X^T (2 m^2 n), A A (2 m^3) and B X (2 m^2 n)."""
+    tot = 0.0
+    for count, rows, cols in stacks:
+        m, n = min(rows, cols), max(rows, cols)
+        tot += count * steps * (4.0 * m * m * n + 2.0 * m ** 3)
+    return tot
+
+
+def run_ns_sweep(args, peaks, peak_kind):
+    """The Muon Newton-Schulz sweep alone: 5 quintic steps on seeded N(0, 1)
+    bf16 stacks of 64 x 1664^2, 26 x 1664x6656 and 26 x 6656x1664, each
+    Frobenius-normalised first (nc_op_newton_schulz), device-timed."""
+    import torch
+    from pretraining_step_b200 import binding as nc
+    g = torch.Generator(device="cuda")
+    stacks = []
+    for i, (count, rows, cols) in enumerate(NS_SWEEP):
+        g.manual_seed(500 + i)
+        x = torch.randn(count, rows, cols, generator=g, device="cuda").to(torch.bfloat16)
+        out = torch.empty_like(x)
+        scratch = torch.empty(nc.newton_schulz_scratch_bytes(count, rows, cols),
+                              dtype=torch.uint8, device="cuda")
+        stacks.append((count, rows, cols, x, out, scratch))
+
+    def sweep():
+        for count, rows, cols, x, out, scratch in stacks:
+            nc.newton_schulz(x, out, count, rows, cols, 5, scratch)
+
+    for _ in range(args.warmup):
+        sweep()
+    nc.op_sync()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record()
+    for _ in range(args.steps):
+        sweep()
+    ev[1].record()
+    nc.op_sync()
+    torch.cuda.synchronize()
+    ms = ev[0].elapsed_time(ev[1]) / args.steps
+    fl = ns_sweep_flops()
+    tf = fl / (ms / 1e3) / 1e12
+    print(json.dumps({"op": "ns_sweep", "stacks": [list(t[:3]) for t in stacks],
+                      "ms_per_sweep": ms, "tflop_per_sweep": fl / 1e12, "tflops": tf,
+                      "frac_of_sustained_peak": tf / peaks["bf16_tflops_sustained"],
+                      "peak_source": peak_kind}), flush=True)
+    return 0
+
+
+def gemm_traffic_cases(ntok, depth=DEPTH, vocab=V):
+    """The GEMMs of one layer, the lm_head and one Newton-Schulz stack as the
+    step launches them, at ntok tokens: (class, name, M, N, K, a_kmajor,
+    b_kmajor, epilogue, algorithmic bytes).  The q|k|v projection runs with
+    the plain bf16 store in place of its RoPE + QK-norm epilogue (the same
+    operand and result bytes)."""
+    from pretraining_step_b200 import binding as nc
+    d, f, n = 64 * depth, 4 * 64 * depth, ntok
+    bf, f4 = 2, 4
+    return [
+        ("fwd", "qkv", n, 3 * d, d, 1, 1, nc.EPI_STORE_BF16, n * d * bf + 3 * d * d * bf + n * 3 * d * bf),
+        ("fwd", "o_resid", n, d, d, 1, 1, nc.EPI_RESID_F32, n * d * bf + d * d * bf + 2 * n * d * f4),
+        ("fwd", "up_relu2", n, f, d, 1, 1, nc.EPI_RELU2, n * d * bf + f * d * bf + n * f * bf),
+        ("fwd", "down_resid", n, d, f, 1, 1, nc.EPI_RESID_F32, n * f * bf + d * f * bf + 2 * n * d * f4),
+        ("dgrad", "du_relu2bwd", n, f, d, 1, 0, nc.EPI_RELU2_BWD, n * d * bf + d * f * bf + 2 * n * f * bf),
+        ("dgrad", "dh_up", n, d, f, 1, 0, nc.EPI_STORE_BF16, n * f * bf + f * d * bf + n * d * bf),
+        ("dgrad", "dh_o", n, d, d, 1, 0, nc.EPI_STORE_BF16, n * d * bf + d * d * bf + n * d * bf),
+        ("dgrad", "dh_qkv", n, d, 3 * d, 1, 0, nc.EPI_STORE_BF16, n * 3 * d * bf + 3 * d * d * bf + n * d * bf),
+        ("wgrad", "dW_down", d, f, n, 0, 0, nc.EPI_ACC_F32, n * d * bf + n * f * bf + d * f * f4),
+        ("wgrad", "dW_up", f, d, n, 0, 0, nc.EPI_ACC_F32, n * f * bf + n * d * bf + f * d * f4),
+        ("wgrad", "dW_o", d, d, n, 0, 0, nc.EPI_ACC_F32, 2 * n * d * bf + d * d * f4),
+        ("wgrad", "dW_qkv", 3 * d, d, n, 0, 0, nc.EPI_ACC_F32, n * 3 * d * bf + n * d * bf + 3 * d * d * f4),
+        ("lmhead", "logits", n, vocab, d, 1, 1, nc.EPI_STORE_BF16, n * d * bf + vocab * d * bf + n * vocab * bf),
+        ("lmhead", "dh_lm", n, d, vocab, 1, 0, nc.EPI_STORE_BF16, n * vocab * bf + vocab * d * bf + n * d * bf),
+        ("lmhead", "dW_lm", vocab, d, n, 0, 0, nc.EPI_ACC_F32, n * vocab * bf + n * d * bf + vocab * d * f4),
+    ]
+
+
+def run_gemm_traffic(args):
+    """One launch of each GEMM of the step (gemm_traffic_cases at --shape
+    ntok tokens, default 16384) after one untimed launch of each, plus one
+    Newton-Schulz call on the square stack, for a one-launch-per-kernel ncu
+    capture of DRAM bytes (-k regex:gemm_tc -s <untimed launches>).  Prints
+    the launch order with each launch's algorithmic bytes."""
+    import torch
+    from pretraining_step_b200 import binding as nc
+    ntok = int(args.shape.split(",")[0]) if args.shape != "16384,5120,1280" else 16384
+    cases = gemm_traffic_cases(ntok)
+    bufs = []
+    for cls, name, M, N, K, ak, bk, epi, nbytes in cases:
+        A = (torch.randn(M * K, device="cuda") * 0.5).to(torch.bfloat16)
+        Bm = (torch.randn(N * K, device="cuda") * K ** -0.5).to(torch.bfloat16)
+        f32 = epi in (nc.EPI_RESID_F32, nc.EPI_ACC_F32)
+        D = torch.zeros(M * N, device="cuda", dtype=torch.float32 if f32 else torch.bfloat16)
+        aux = None
+        if epi == nc.EPI_RESID_F32:
+            aux = torch.randn(M * N, device="cuda")
+        elif epi == nc.EPI_RELU2_BWD:
+            aux = torch.rand(M * N, device="cuda").to(torch.bfloat16)
+        bufs.append((M, N, K, ak, bk, epi, A, Bm, D, aux))
+    d = 64 * DEPTH
+    cnt = 4 * DEPTH
+    X = torch.randn(cnt, d, d, device="cuda").to(torch.bfloat16)
+    out = torch.empty_like(X)
+    scratch = torch.empty(nc.newton_schulz_scratch_bytes(cnt, d, d), dtype=torch.uint8, device="cuda")
+
+    def run_all():
+        for M, N, K, ak, bk, epi, A, Bm, D, aux in bufs:
+            nc.gemm(M, N, K, A, Bm, D, a_kmajor=ak, b_kmajor=bk, epi=epi, aux=aux,
+                    split_k=0 if epi == nc.EPI_ACC_F32 else 1)
+        nc.newton_schulz(X, out, cnt, d, d, 5, scratch)
+
+    run_all()      # untimed: 15 GEMMs + 15 Newton-Schulz GEMMs
+    nc.op_sync()
+    run_all()      # the captured pass
+    nc.op_sync()
+    ns_x = cnt * d * d * 2
+    ns_a = cnt * d * d * 2
+    ns_bytes = [(ns_x + ns_a), (ns_a + ns_a), (ns_a + ns_x + ns_x)] * 5
+    order = [(c[0], c[1], c[8]) for c in cases] + \
+        [("ns", "ns_%s_%d" % (("XXt", "AA", "BX")[i % 3], i // 3), b) for i, b in enumerate(ns_bytes)]
+    print(json.dumps({"op": "gemm_traffic", "tokens": ntok, "untimed_gemm_launches": len(order),
+                      "launches": [{"class": c, "name": n, "algorithmic_bytes": b}
+                                   for c, n, b in order]}), flush=True)
+    return 0
+
+
 def run_step_variant(args, dims, peaks, peak_kind):
     """The forward + backward + Muon step of any model configuration
     (--shape depth,B,T, grouped KV heads, per-layer windows), inputs
@@ -602,7 +865,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["gemm", "attn", "attn_bwd", "adamw", "step"], default=None,
+    ap.add_argument("--op", choices=["gemm", "attn", "attn_bwd", "adamw", "step", "ns_sweep",
+                                     "gemm_traffic"],
+                    default=None,
                     help="time one kernel class alone instead of the step ('step': the whole "
                          "step of the model --shape depth,B,T with the options below)")
     ap.add_argument("--kv-heads", type=int, default=0, help="--op step: KV heads (0: one per head)")

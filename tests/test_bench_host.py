@@ -71,3 +71,30 @@ def test_step_times_are_the_gaps_between_marks():
 
     marks = [Mark(t) for t in (0.0, 2.0, 5.0, 6.5)]
     assert bench.step_times_ms(marks) == [2.0, 3.0, 1.5]
+
+
+def test_ns_sweep_flops_match_the_square_and_wide_counts():
+    """The Newton-Schulz sweep (64 x 1664^2, 26 x 1664x6656, 26 x 6656x1664, five
+    steps): a square n x n matrix costs 6 n^3 per step and a 1 : 4 one 18 m^3
+    (m the short side), whichever way it stands: 30.41 TFLOP in all."""
+    n = 1664
+    assert bench.ns_sweep_flops(((1, n, n),), steps=1) == 6.0 * n ** 3
+    assert bench.ns_sweep_flops(((1, n, 4 * n),), steps=1) == 18.0 * n ** 3
+    assert bench.ns_sweep_flops(((1, 4 * n, n),), steps=1) == 18.0 * n ** 3
+    total = 5 * (64 * 6.0 + 2 * 26 * 18.0) * n ** 3
+    assert bench.ns_sweep_flops() == total
+    assert abs(total / 1e12 - 30.41) < 0.01
+
+
+def test_gemm_byte_classes_sum_to_the_step():
+    by_class, launches = bench.gemm_algorithmic_bytes_by_class()
+    total, n = bench.gemm_algorithmic_bytes_per_step()
+    assert sum(by_class.values()) == total and sum(launches.values()) == n
+    assert set(by_class) == {"fwd", "dgrad", "wgrad", "lmhead", "ns"}
+
+
+def test_tensor_peak_at_a_clock():
+    """148 SMs x 8192 FLOP per clock: 2.38 PFLOP/s at the 1965 MHz maximum,
+    1.82 at 1500 MHz."""
+    assert abs(bench.tensor_peak_at(1965.0) - 2382.3) < 0.1
+    assert abs(bench.tensor_peak_at(1500.0) - 1818.6) < 0.1
