@@ -226,7 +226,38 @@ int* nc_debug_status_word(nc_params* p);
 /* ------------------------------------------------------------------ ops
  * Single kernels of the step, for kernel-level checks and the
  * Newton-Schulz sweep.  All pointers are device pointers; all calls are
- * asynchronous on `stream` (a cudaStream_t, NULL = legacy default). */
+ * asynchronous on `stream` (a cudaStream_t, NULL = legacy default).
+ * Argument errors return at once, before anything is launched.  Errors a
+ * kernel finds on the device (a bounded wait that expired, which leaves the
+ * outputs incomplete; a token id out of range) are recorded in one op
+ * status word per device, shared by every nc_op_* call on that device from
+ * any stream or thread, and returned by the next nc_op_sync. */
+
+/* Wait for `stream`, then return and clear the device's op status word:
+ * NC_OK, NC_ERR_TIMEOUT (an op's bounded wait expired; its outputs are
+ * incomplete) or NC_ERR_TOKEN_RANGE.  NC_ERR_CUDA if the wait itself fails. */
+nc_status nc_op_sync(void* stream);
+
+/* Testing hook: device address of the current device's op status word (one
+ * int, 0 = no error, 1 = an expired wait, 2 = a token id out of range), so a
+ * test can plant a code and check how nc_op_sync reports it.  NULL if the
+ * address cannot be looked up. */
+int* nc_debug_op_status_word(void);
+
+/* Testing hook: y[i] = 2^x[i] by the polynomial the attention forward uses
+ * for a share of its softmax exponentials (device pointers, n floats):
+ * nearest-integer range reduction and a cubic on [-0.5, 0.5], relative
+ * error below 7.5e-5 for x in [-125, 126]; x below -125 gives 2^-125. */
+nc_status nc_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream);
+
+/* Embedding gather, the first step of the forward (guide, section "1. Modelo
+ * GPT": token embedding, untied from lm_head): x[i, :] = E[tokens[i], :]
+ * for i < n, copied bit for bit (fp32 rows of d floats; E [vocab, d] and x
+ * [n, d] dense, 16-byte aligned, d a multiple of 4).  An id outside
+ * [0, vocab) is clamped to the nearest valid row for the read (row 0 below,
+ * row vocab - 1 above) and recorded as NC_ERR_TOKEN_RANGE for nc_op_sync. */
+nc_status nc_op_embed_gather(const int32_t* tokens, int64_t n, const float* E, int vocab, int d,
+                             float* x, void* stream);
 
 /* Epilogues of the GEMM engine. */
 typedef enum {
@@ -339,7 +370,10 @@ nc_status nc_op_attention_bwd_ex(const void* q, int64_t ldq, const void* k, cons
  * return NC_ERR_INVALID_ARG before anything is launched.  Nothing is
  * allocated: no cudaMalloc, cudaFree or allocating library routine.
  * The first call on each device looks up the array's device address (with
- * that device current) and should come before any stream capture.
+ * that device current) and should come before any stream capture.  The
+ * address is kept for the life of the process, so it stays valid only while
+ * that device's primary context does: calls after a cudaDeviceReset are not
+ * supported.
  * Every call shares the array and it keeps the last call's contents (each
  * call rewrites the entries it uses before reading them); calls that overlap
  * on the GPU (different streams, or graphs running concurrently) race on it.

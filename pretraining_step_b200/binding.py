@@ -104,6 +104,10 @@ def lib():
         "nc_debug_status_word": (vp, [vp]),
         "nc_op_gemm": (ci, [ctypes.POINTER(GemmDesc), vp]),
         "nc_op_rmsnorm": (ci, [vp, i64, ci, vp, vp, vp]),
+        "nc_op_embed_gather": (ci, [vp, i64, vp, ci, ci, vp, vp]),
+        "nc_op_sync": (ci, [vp]),
+        "nc_debug_op_status_word": (vp, []),
+        "nc_debug_exp2_poly": (ci, [vp, vp, i64, vp]),
         "nc_op_attention_fwd": (ci, [vp, vp, vp, i64, vp, i64, vp, ci, ci, ci, vp]),
         "nc_op_attention_bwd": (ci, [vp, vp, vp, i64, vp, vp, i64, vp, vp, vp, vp, i64, vp,
                                      ci, ci, ci, vp]),
@@ -329,6 +333,23 @@ def gemm(M, N, K, A, B, D, *, lda=None, ldb=None, ldd=None, a_kmajor=True, b_kma
     d.stride_aux = stride_aux
     d.epi, d.alpha, d.beta, d.split_k = epi, alpha, beta, split_k
     _check(lib().nc_op_gemm(ctypes.byref(d), _stream(stream)))
+
+
+def embed_gather(tokens, n, E, vocab, d, x, stream=None):
+    """x[i] = E[tokens[i]] (fp32 rows, bit for bit); ids out of range are
+    clamped and reported by op_sync."""
+    _check(lib().nc_op_embed_gather(_ptr(tokens), n, _ptr(E), vocab, d, _ptr(x), _stream(stream)))
+
+
+def exp2_poly(x, y, n, stream=None):
+    """Testing hook: the attention forward's polynomial 2^x, elementwise."""
+    _check(lib().nc_debug_exp2_poly(_ptr(x), _ptr(y), n, _stream(stream)))
+
+
+def op_sync(stream=None):
+    """Wait for the stream and raise NcError if an op recorded a device-side
+    error (the device's op status word is cleared)."""
+    _check(lib().nc_op_sync(_stream(stream)))
 
 
 def rmsnorm(x, y, rstd, rows, cols, stream=None):

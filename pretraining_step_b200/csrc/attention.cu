@@ -83,7 +83,8 @@ __global__ void __launch_bounds__(256) attn_bwd_delta_kernel(const __nv_bfloat16
 nc_status attention_bwd_ex(const void* q, int64_t ldq, const void* k, const void* v, int64_t ldkv,
                            const void* o, const void* dout, int64_t ldo, const float* lse,
                            float* dq, void* dk, void* dv, int64_t ldg, float* delta, int B, int T,
-                           int H, int Hkv, int window, int* status, cudaStream_t s, Profiler* prof) {
+                           int H, int Hkv, int window, const float2* rope_tab, const float* rstd_k,
+                           int* status, cudaStream_t s, Profiler* prof) {
   if (B < 1 || T < 1 || H < 1 || Hkv < 1 || H % Hkv || !q || !k || !v || !o || !dout || !lse ||
       !dq || !dk || !dv || !delta)
     return fail(NC_ERR_INVALID_ARG, "attention_bwd: bad arguments (H must be a multiple of Hkv)");
@@ -101,7 +102,31 @@ nc_status attention_bwd_ex(const void* q, int64_t ldq, const void* k, const void
   }
   NC_CUDA_TRY(cudaMemsetAsync(dq, 0, sizeof(float) * rows * HD, s));
   return attention_bwd_tc_ex(q, ldq, k, v, ldkv, dout, ldo, lse, delta, dq, dk, dv, ldg, B, T, H,
-                             Hkv, window, status, s, prof);
+                             Hkv, window, rope_tab, rstd_k, nullptr, 0, status, s, prof);
+}
+
+nc_status attention_bwd_model(const void* q, int64_t ldq, const void* k, const void* v,
+                              int64_t ldkv, const void* o, const void* dout, int64_t ldo,
+                              const float* lse, float* delta, void* ds, int64_t ld_ds,
+                              void* dq_out, void* dk, void* dv, int64_t ldg, int B, int T, int H,
+                              int Hkv, int window, const float2* rope_tab, const float* rstd_q,
+                              const float* rstd_k, int* status, cudaStream_t s, Profiler* prof) {
+  if (B < 1 || T < 1 || H < 1 || Hkv < 1 || H % Hkv || H > kDeltaMaxH || !o || !dout || !delta ||
+      !ds || !rope_tab || !rstd_q || !rstd_k)
+    return fail(NC_ERR_INVALID_ARG, "attention_bwd_model: bad arguments");
+  if (ldo % 8 || ((reinterpret_cast<uintptr_t>(o) | reinterpret_cast<uintptr_t>(dout)) & 15))
+    return fail(NC_ERR_INVALID_ARG, "attention_bwd_model: O and dO rows must be 16-byte aligned");
+  const int64_t rows = (int64_t)B * T * H;
+  {
+    Probe probe(prof, s, "attn_bwd_delta", 0.0, rows * HD * 2.0 * 2 + rows * 4.0);
+    attn_bwd_delta_kernel<<<(unsigned)(((int64_t)B * T + kDeltaTok - 1) / kDeltaTok), 256, 0, s>>>(
+        (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, ldo, delta, B, T, H);
+    NC_CUDA_TRY(cudaGetLastError());
+  }
+  NC_TRY(attention_bwd_tc_ex(q, ldq, k, v, ldkv, dout, ldo, lse, delta, nullptr, dk, dv, ldg, B, T,
+                             H, Hkv, window, rope_tab, rstd_k, ds, ld_ds, status, s, prof));
+  return attention_dq_ex(ds, ld_ds, k, ldkv, B, T, H, Hkv, window, q, ldq, rstd_q, rope_tab, dq_out,
+                         ldg, status, s, prof);
 }
 
 nc_status attention_bwd(const void* q, const void* k, const void* v, int64_t ld, const void* o,
@@ -109,7 +134,7 @@ nc_status attention_bwd(const void* q, const void* k, const void* v, int64_t ld,
                         void* dv, int64_t ldg, float* delta, int B, int T, int H, int* status,
                         cudaStream_t s, Profiler* prof) {
   return attention_bwd_ex(q, ld, k, v, ld, o, dout, ldo, lse, dq, dk, dv, ldg, delta, B, T, H, H, -1,
-                          status, s, prof);
+                          nullptr, nullptr, status, s, prof);
 }
 
 // ------------------------------------------------------------------ allocation-free backward
@@ -163,6 +188,8 @@ extern "C" nc_status nc_op_attention_bwd_noalloc(const void* q, const void* k, c
   NC_TRY(noalloc_scratch(&delta));
   // The row-sum pass rewrites every entry it reads, so nothing from an
   // earlier call leaks into this one and no clearing is needed.
-  return attention_bwd(q, k, v, ld, o, dout, ldo, lse, dq, dk, dv, ldg, delta, B, T, H, nullptr,
+  int* st = nullptr;
+  NC_TRY(op_status_word(&st));
+  return attention_bwd(q, k, v, ld, o, dout, ldo, lse, dq, dk, dv, ldg, delta, B, T, H, st,
                        static_cast<cudaStream_t>(stream), nullptr);
 }

@@ -359,44 +359,385 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 
+// ------------------------------------------------------------------ forward, two query tiles
+// The plain forward (one KV head per query head, no window) at one CTA per
+// SM: the CTA takes query tiles 2p and 2p + 1 of one (head, batch row) and
+// streams their shared key/value tiles once.  Its two score chains
+// interleave on the tensor pipe, so one tile's softmax runs while the
+// other tile's products execute:
+//   tensor:  ... PV_a(j)  S_a(j+1)  PV_b(j)  S_b(j+1)  PV_a(j+1) ...
+// 320 threads:
+//   warp 0       TMA: both Q tiles once, then K_j and V_j through two stages
+//                each (a stage is released when both tiles' products that
+//                read it are done);
+//   warp 1       TMEM owner and single-thread MMA issue in the order above;
+//   warps 2..5   softmax of tile a, warps 6..9 softmax of tile b: one thread
+//                per query row holding its 128 scores, so the row maximum
+//                needs no exchange between threads; the maximum is raised
+//                only past 2^8 (O rescaled in TMEM then), and P is written as
+//                bf16 over the scores it replaces (key k in column k / 2).
+//                A share of the exponentials (POLY of every 32) runs on the
+//                FMA pipe as a polynomial, the rest on the exponential unit,
+//                whose 16 results per clock per SM would otherwise bound
+//                the softmax at the pace of the tile's two products.
+// TMEM columns: S_a [0,128), S_b [128,256), O_a [256,384), O_b [384,512).
+// The MMAs run in issue order, so S_x(j+1) never overwrites P_x(j) before
+// PV_x(j) has read it, and the commit that publishes S_x(j+1) also covers
+// PV_x(j): O_x is idle while tile x's softmax runs.
+constexpr int kPPThreads = 320;
+constexpr int PP_OFF_QA = 0;       // Q_a, then Q_b at + TILE
+constexpr int PP_OFF_K = 2 * TILE;   // 2 stages
+constexpr int PP_OFF_V = 4 * TILE;   // 2 stages
+constexpr int PP_OFF_BAR = 6 * TILE;
+constexpr int kPPSmem = PP_OFF_BAR + 512;
+constexpr int kPolyExp = 8;  // exponentials per 32 scores evaluated by polynomial
+
+// 2^x on the FMA pipe (x <= 126): x = n + f with n the nearest integer
+// (rounded by adding 1.5 * 2^23, whose low mantissa bits then hold n) and
+// f in [-0.5, 0.5]; 2^f by the cubic that minimises the largest relative
+// error on that interval (Remez exchange, relative error below 7.5e-5,
+// under a thirtieth of a bf16 step); 2^n is added into the exponent field.
+// Arguments below -125 return 2^-125 (a tiny normal number, not 0).
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = x + 12582912.f;
+  const float f = x - (t - 12582912.f);
+  float p = fmaf(0.05517167f, f, 0.24261113f);
+  p = fmaf(p, f, 0.69326097f);
+  p = fmaf(p, f, 0.99992806f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+static_assert(kPPSmem <= 232448, "two-tile forward shared memory budget");
+
+__global__ void __launch_bounds__(kPPThreads, 1)
+    attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                       const __grid_constant__ CUtensorMap tv, const FwdArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if ((tc::smem_u32(smem_raw) & 1023u) != 0) {  // never expected; no room to realign
+    if (threadIdx.x == 0 && a.status) atomicExch(a.status, kDevTimeout);
+    return;
+  }
+  uint8_t* smem = smem_raw;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PP_OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* k_empty = bars + 3;   // [2]
+  uint64_t* v_full = bars + 5;    // [2]
+  uint64_t* v_empty = bars + 7;   // [2]
+  uint64_t* s_full = bars + 9;    // [2 tiles]
+  uint64_t* p_full = bars + 11;   // [2 tiles]
+  uint64_t* o_full = bars + 13;   // [2 tiles]
+  uint64_t* drained = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int npairs = (a.nqb + 1) / 2;
+  const int pr = npairs - 1 - (int)blockIdx.x;  // heaviest pairs first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int qt0 = 2 * pr;                        // tile a; tile b = qt0 + 1 when it exists
+  const bool has_b = qt0 + 1 < a.nqb;
+  const int nkv = has_b ? qt0 + 2 : qt0 + 1;     // key tiles 0 .. the last tile's diagonal
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&k_full[i], 1);
+      tc::mbar_init(&k_empty[i], 1);
+      tc::mbar_init(&v_full[i], 1);
+      tc::mbar_init(&v_empty[i], 1);
+      tc::mbar_init(&s_full[i], 1);
+      tc::mbar_init(&p_full[i], 128);
+      tc::mbar_init(&o_full[i], 1);
+    }
+    tc::mbar_init(drained, 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int col0 = h * HD;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tc::tma_prefetch_desc(&tq);
+      tc::tma_prefetch_desc(&tk);
+      tc::tma_prefetch_desc(&tv);
+      tc::mbar_arrive_expect_tx(q_full, has_b ? 2 * TILE : TILE);
+      for (int x = 0; x < (has_b ? 2 : 1); ++x)
+        for (int c = 0; c < 2; ++c)
+          tc::tma_load_3d(smem + PP_OFF_QA + x * TILE + c * (TILE / 2), &tq, q_full, col0 + 64 * c,
+                          (qt0 + x) * BQ, b);
+      int issued_k = 0, issued_v = 0;
+      bool ok = true;
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int st = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!tc::mbar_wait(&k_empty[st], ph ^ 1, abort_flag, a.status)) { ok = false; break; }
+        tc::mbar_arrive_expect_tx(&k_full[st], TILE);
+        for (int c = 0; c < 2; ++c)
+          tc::tma_load_3d(smem + PP_OFF_K + st * TILE + c * (TILE / 2), &tk, &k_full[st],
+                          col0 + 64 * c, j * BKV, b);
+        ++issued_k;
+        if (!tc::mbar_wait(&v_empty[st], ph ^ 1, abort_flag, a.status)) { ok = false; break; }
+        tc::mbar_arrive_expect_tx(&v_full[st], TILE);
+        for (int c = 0; c < 2; ++c)
+          tc::tma_load_3d(smem + PP_OFF_V + st * TILE + c * (TILE / 2), &tv, &v_full[st],
+                          col0 + 64 * c, j * BKV, b);
+        ++issued_v;
+      }
+      if (!ok) {
+        drain_wait(q_full, 0);
+        for (int j = max(0, issued_k - 2); j < issued_k; ++j) drain_wait(&k_full[j & 1], (j >> 1) & 1);
+        for (int j = max(0, issued_v - 2); j < issued_v; ++j) drain_wait(&v_full[j & 1], (j >> 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id_s = tc::idesc_bf16_f32(128, BKV, 0, 0);
+      const uint32_t id_pv = tc::idesc_bf16_f32(128, HD, 0, 1);
+      const uint64_t qdesc = tc::smem_desc_sw128(tc::smem_u32(smem + PP_OFF_QA), 16, 1024);
+      const uint64_t kdesc = tc::smem_desc_sw128(tc::smem_u32(smem + PP_OFF_K), 16, 1024);
+      const uint64_t vdesc = tc::smem_desc_sw128(tc::smem_u32(smem + PP_OFF_V), TILE / 2, 1024);
+      // S_x(j) = Q_x K_j^T into tile x's score columns.
+      auto issue_s = [&](int x, int j) {
+        const uint64_t qd = tc::desc_add(qdesc, x * TILE);
+        const uint64_t kd = tc::desc_add(kdesc, (j & 1) * TILE);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (TILE / 2) + (kk & 3) * 32;
+          tc::umma_bf16_ss(tmem + 128 * x, tc::desc_add(qd, off), tc::desc_add(kd, off), id_s,
+                           kk > 0 ? 1u : 0u);
+        }
+        tc::umma_commit(&s_full[x]);
+      };
+      // O_x += P_x(j) V_j, P from TMEM (key k in column k / 2 of the tile's
+      // score block; 16 keys per MMA).
+      auto issue_pv = [&](int x, int j) {
+        const uint64_t vd = tc::desc_add(vdesc, (j & 1) * TILE);
+#pragma unroll
+        for (int kk = 0; kk < BKV / 16; ++kk)
+          tc::umma_bf16_ts(tmem + 256 + 128 * x, tmem + 128 * x + kk * 8,
+                           tc::desc_add(vd, kk * 2048), id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      const int last[2] = {qt0, qt0 + 1};  // each tile's last key tile (its diagonal)
+      bool ok = tc::mbar_wait(q_full, 0, abort_flag, a.status) &&
+                tc::mbar_wait(&k_full[0], 0, abort_flag, a.status);
+      if (ok) {
+        tc::tc_fence_after();
+        issue_s(0, 0);
+        if (has_b) issue_s(1, 0);
+        tc::umma_commit(&k_empty[0]);
+      }
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int st = j & 1;
+        if (!tc::mbar_wait(&v_full[st], (j >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+        bool k_next = false;  // K_{j+1} has landed
+        for (int x = 0; x < (has_b ? 2 : 1); ++x) {
+          if (j > last[x]) continue;
+          if (!tc::mbar_wait(&p_full[x], j & 1, abort_flag, a.status)) { ok = false; break; }
+          tc::tc_fence_after();
+          issue_pv(x, j);
+          if (j == last[x]) {
+            tc::umma_commit(&o_full[x]);
+            continue;
+          }
+          if (!k_next) {
+            if (!tc::mbar_wait(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag, a.status)) {
+              ok = false;
+              break;
+            }
+            tc::tc_fence_after();
+            k_next = true;
+          }
+          issue_s(x, j + 1);
+        }
+        if (!ok) break;
+        tc::umma_commit(&v_empty[st]);
+        if (k_next) tc::umma_commit(&k_empty[(j + 1) & 1]);
+      }
+      tc::umma_commit(drained);
+      drain_wait(drained, 0);
+    }
+  } else if (warp < 10) {
+    // Softmax of tile x: warps 2..5 (x = 0) and 6..9 (x = 1), one thread per
+    // query row (a warp may only reach the TMEM lanes of quarter warp % 4).
+    const int x = (warp - 2) >> 2;
+    const int qw = warp & 3;
+    const int row = qw * 32 + lane;
+    if (x == 0 || has_b) {
+      const int qb = qt0 + x;
+      const int qi = qb * BQ + row;
+      const int key_hi = min(qi, a.T - 1);
+      const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
+      const uint32_t s_base = lane_base + 128 * x;
+      const uint32_t o_base = lane_base + 256 + 128 * x;
+      float m_used = -INFINITY, l = 0.f;
+      bool ok = true;
+      for (int j = 0; j <= qb; ++j) {
+        ok = tc::mbar_wait(&s_full[x], j & 1, abort_flag, a.status);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc::tc_fence_after();
+        uint32_t r[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tc::tmem_ld_32x32b_x32(s_base + 32 * c, r[c]);
+        tc::tmem_ld_wait();
+        // The diagonal tile or the tile that reaches T: keys past this row's
+        // last visible key become -inf.
+        const bool edge = j * BKV + BKV > min(qb * BQ, a.T);
+        if (edge) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (j * BKV + 32 * c + i > key_hi) r[c][i] = __float_as_uint(-INFINITY);
+        }
+        float pm[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) pm[u] = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) pm[i & 7] = fmaxf(pm[i & 7], __uint_as_float(r[c][i]));
+        const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7]))) * a.sl2;
+        float alpha = 1.f;
+        if (mx > m_used + kRescaleThreshold) {
+          alpha = ex2(m_used - mx);  // 0 on the first tile
+          m_used = mx;
+        }
+        const float neg_mu = (m_used == -INFINITY) ? 0.f : -m_used;
+        l *= alpha;
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float x0 = fmaf(__uint_as_float(r[c][2 * i]), a.sl2, neg_mu);
+            const float x1 = fmaf(__uint_as_float(r[c][2 * i + 1]), a.sl2, neg_mu);
+            // Edge tiles take every exponential from the exponential unit, so
+            // masked keys give exactly 0.
+            const float p0 = (!edge && 2 * i < kPolyExp) ? exp2_poly(x0) : ex2(x0);
+            const float p1 = (!edge && 2 * i + 1 < kPolyExp) ? exp2_poly(x1) : ex2(x1);
+            ls[(2 * i) & 3] += p0;
+            ls[(2 * i + 1) & 3] += p1;
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+          // Keys [32 c, 32 c + 32) to columns [16 c, 16 c + 16): over scores
+          // already held in registers.
+          tc::tmem_st_32x32b_x16(s_base + 16 * c, pk);
+        }
+        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        // O is idle here: the commit that published S_j also covers P_{j-1} V_{j-1}.
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tc::tmem_ld_32x32b_x32(o_base + c * 32, o);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tc::tmem_st_32x32b_x32(o_base + c * 32, o);
+          }
+        }
+        tc::tmem_st_wait();
+        tc::tc_fence_before();
+        tc::mbar_arrive(&p_full[x]);
+      }
+      if (ok) {
+        ok = tc::mbar_wait(&o_full[x], 0, abort_flag, a.status);
+        ok = __all_sync(0xffffffffu, ok);
+      }
+      if (ok) {
+        tc::tc_fence_after();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        __nv_bfloat16* orow = a.o + ((int64_t)b * a.T + qi) * a.ldo + col0;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tc::tmem_ld_32x32b_x32(o_base + c * 32, o);
+          tc::tmem_ld_wait();
+          if (qi < a.T) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              uint4 v;
+              v.x = pack_bf16x2(__uint_as_float(o[8 * u + 0]) * inv, __uint_as_float(o[8 * u + 1]) * inv);
+              v.y = pack_bf16x2(__uint_as_float(o[8 * u + 2]) * inv, __uint_as_float(o[8 * u + 3]) * inv);
+              v.z = pack_bf16x2(__uint_as_float(o[8 * u + 4]) * inv, __uint_as_float(o[8 * u + 5]) * inv);
+              v.w = pack_bf16x2(__uint_as_float(o[8 * u + 6]) * inv, __uint_as_float(o[8 * u + 7]) * inv);
+              reinterpret_cast<uint4*>(orow + c * 32)[u] = v;
+            }
+          }
+        }
+        if (qi < a.T)
+          a.lse[((int64_t)b * a.H + h) * a.T + qi] = (m_used + log2f(l)) * 0.69314718055994531f;
+      }
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 // ------------------------------------------------------------------ backward
-// One CTA per (128-key tile, head, batch row); loops over the 64-query tiles
-// at or after it.  448 threads:
-//   warp 0      TMA: K and V once, then Q_i and dO_i through a 4-stage ring
-//               (tile i's Q/dO stay operands of dV/dK(i) while tile i+1's
-//               scores are computed, so two stages would leave no prefetch);
-//               its lanes also stage lse * log2(e) and D of each tile;
-//   warp 1      MMA issue, per query tile i:
-//                 S^T  = K Q_i^T        TMEM [  0, 64)   M 128 keys, N 64
-//                 dP^T = V dO_i^T       TMEM [ 64,128)
-//                 dV  += P^T dO_i       TMEM [256,384)   N 128 (dO MN-major)
-//                 dK  += dS^T Q_i       TMEM [384,512)   N 128 (Q MN-major)
-//                 dQ^T = K^T dS^T       TMEM [128,256)   M 128 dims, N 64, 2 buffers
-//               (K^T and dS^T are the same shared tiles read MN-major), with
-//               S^T/dP^T of tile i+1 issued before the gradient products of i;
-//   warps 2..9  two warps per key row group, each half of the 64 columns:
-//               P^T = exp(S^T/sqrt(d) - lse), dS^T = P^T (dP^T - D) as bf16
-//               into K-major shared tiles; at the end dV (warps 2..5) and dK
-//               (warps 6..9) rows to global memory;
-//   warps 10..13 one head-dim row each: dQ^T row -> fp32 atomic adds into dq
-//               (a warp covers 32 consecutive dims of one query: coalesced).
-constexpr int BQB = 64;                  // query tile of the backward
-constexpr int QT = BQB * 128 * 2;        // 16 KB: [64 rows x 128 dims]
-constexpr int PT = 128 * BQB * 2;        // 16 KB: [128 keys x 64 queries]
-constexpr int QST = 4;                   // Q / dO stages
+// One CTA per (128-key tile, KV head, batch row); it loops over the 128-query
+// tiles at or after its keys (every query head of the KV head's group in
+// turn).  Every product is a 128 x 128 x 128 tcgen05 MMA, and the two score
+// gradients that feed the key-side products (P^T and dS^T) reach the tensor
+// core from TMEM, so their shared-memory operand traffic is one tile per
+// product instead of two.  448 threads:
+//   warp 0      TMA: K and V once, then Q_i and dO_i (two stages each, their
+//               own barriers, so dO of tile i + 2 can land while Q_i is still
+//               an operand); its lanes also stage lse * log2(e) (with Q) and
+//               D (with dO) of the tile;
+//   warp 1      TMEM owner and single-thread MMA issue, per query tile i:
+//                 dV  += P_i^T dO_i     (A = P^T from TMEM, dO MN-major)
+//                 S^T_{i+1} = K Q_{i+1}^T            -> TMEM S
+//                 dK  += dS_i^T Q_i     (A = dS^T from TMEM, Q MN-major)
+//                 dQ_i = dS_i K         -> TMEM DP   (dS and K read MN-major)
+//                 dP^T_{i+1} = V dO_{i+1}^T          -> TMEM DP, once the dQ
+//                                                       warps have read dQ_i
+//               The MMAs of a CTA run in issue order, so S^T_{i+1} never
+//               overwrites P_i^T before dV has read it, and dQ_i never
+//               overwrites dS_i^T before dK has read it;
+//   warps 2..9  two per key row group (TMEM lane quarter), each half of the
+//               tile's 128 queries: P^T = exp2(S^T sl2 - lse2) written back
+//               as bf16 over its own first scores; then dS^T = P^T (dP^T - D)
+//               as bf16 over its own first dP^T columns and into the shared
+//               dS tile the dQ product reads; at the end dV (warps 2..5) and
+//               dK (warps 6..9) rows to global memory;
+//   warps 10..13 one query row each: the tile's dQ rows leave TMEM through
+//               the shared dS tile (free once the dQ product has read it),
+//               staged as fp32 boxes of 32 queries x 32 dims with the 128-byte
+//               swizzle, and are added into dq by TMA bulk reductions
+//               (cp.reduce.async.bulk.tensor ... .add): the sums happen in L2
+//               on whole lines, with no per-thread atomics.
+// TMEM columns: dV [0,128), dK [128,256), S^T/P^T [256,384), dP^T/dS^T and
+// dQ [384,512).  All mbarrier waits are bounded; on a timeout every role
+// drains its in-flight copies and MMAs before TMEM is released.
+constexpr int BQB = 128;                 // query tile of the backward
 constexpr int B_OFF_K = 0;
 constexpr int B_OFF_V = B_OFF_K + TILE;
-constexpr int B_OFF_Q = B_OFF_V + TILE;         // QST stages
-constexpr int B_OFF_DO = B_OFF_Q + QST * QT;    // QST stages
-constexpr int B_OFF_P = B_OFF_DO + QST * QT;
-constexpr int B_OFF_DS = B_OFF_P + PT;
-constexpr int B_OFF_LD = B_OFF_DS + PT;         // per stage: lse * log2(e) [64], D [64] (f32)
-constexpr int B_OFF_BAR = B_OFF_LD + QST * 2 * BQB * 4;
-constexpr int kBwdNeeded = B_OFF_BAR + 256;
-constexpr int kBwdSmem = 232448;                // the per-block maximum; slack absorbs alignment
-static_assert(kBwdNeeded + 512 <= kBwdSmem, "attention backward shared memory budget");
+constexpr int B_OFF_Q = B_OFF_V + TILE;       // 2 stages
+constexpr int B_OFF_DO = B_OFF_Q + 2 * TILE;  // 2 stages
+constexpr int B_OFF_DS = B_OFF_DO + 2 * TILE; // [2 query halves][128 keys][64 queries] bf16
+constexpr int B_OFF_LQ = B_OFF_DS + TILE;     // [2 stages][128] lse * log2(e)
+constexpr int B_OFF_LD = B_OFF_LQ + 2 * BQB * 4;  // [2 stages][128] D
+constexpr int B_OFF_BAR = B_OFF_LD + 2 * BQB * 4;
+constexpr int kBwdSmem = B_OFF_BAR + 256;
+static_assert(kBwdSmem <= 232448, "attention backward shared memory budget");
 constexpr int kBwdThreads = 448;
-constexpr uint32_t TB_S = 0, TB_DP = 64, TB_DQ = 128, TB_DV = 256, TB_DK = 384;
+constexpr uint32_t TB_DV = 0, TB_DK = 128, TB_S = 256, TB_DP = 384;
 
 struct BwdArgs {
   int T, H, nkb, nqb;
@@ -410,43 +751,55 @@ struct BwdArgs {
   __nv_bfloat16* dv;
   int64_t ldg;
   int* status;
+  // Non-null: dK leaves through the backward of the k-side RoPE + QK-norm
+  // (the forward applies them in the q|k|v projection's epilogue), using
+  // the saved normalised k (the K operand itself), rstd_k [B*T, Hkv] and
+  // the cos/sin table [T][64].
+  const float2* rope_tab;
+  const float* rstd_k;
+  int Hkv;
 };
 
 // GW: grouped KV heads or a window in play; the plain instance compiles
 // with group 1 and no window as constants (its tile t is query tile i0 + t
-// of head hk).
-template <bool GW>
+// of head hk).  SDS: instead of the dQ product, every dS^T tile goes to
+// global memory (tdq is then the map of the bf16 dS^T buffer [B*H][T keys][T
+// queries]) for the query-side kernel (attn_dq_kernel) to contract with K;
+// warp 10 issues those stores and the other dQ warps have nothing to do.
+template <bool GW, bool SDS>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
-                       const BwdArgs a) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  if ((smem - smem_raw) + kBwdNeeded > kBwdSmem) {  // never expected: base misaligned past slack
+                       const __grid_constant__ CUtensorMap tdq, const BwdArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if ((tc::smem_u32(smem_raw) & 1023u) != 0) {  // never expected; no room to realign
     if (threadIdx.x == 0 && a.status) atomicExch(a.status, kDevTimeout);
     return;
   }
+  uint8_t* smem = smem_raw;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + B_OFF_BAR);
   uint64_t* kv_full = bars + 0;
-  uint64_t* qd_full = bars + 1;              // [QST]
-  uint64_t* qd_empty = bars + 1 + QST;       // [QST]
-  uint64_t* sdp_full = bars + 1 + 2 * QST;
-  uint64_t* sdp_empty = sdp_full + 1;
-  uint64_t* pds_full = sdp_full + 2;
-  uint64_t* pds_empty = sdp_full + 3;
-  uint64_t* dq_full = sdp_full + 4;          // [2]
-  uint64_t* dq_empty = sdp_full + 6;         // [2]
-  uint64_t* dkv_full = sdp_full + 8;
-  uint64_t* drained = sdp_full + 9;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sdp_full + 10);
+  uint64_t* q_full = bars + 1;    // [2]
+  uint64_t* q_empty = bars + 3;   // [2]
+  uint64_t* do_full = bars + 5;   // [2]
+  uint64_t* do_empty = bars + 7;  // [2]
+  uint64_t* s_full = bars + 9;
+  uint64_t* p_full = bars + 10;
+  uint64_t* dp_full = bars + 11;
+  uint64_t* ds_full = bars + 12;
+  uint64_t* ds_empty = bars + 13;
+  uint64_t* dq_full = bars + 14;
+  uint64_t* dq_empty = bars + 15;
+  uint64_t* dkv_full = bars + 16;
+  uint64_t* drained = bars + 17;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kb = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;  // hk: the KV head
   const int group = GW ? a.group : 1;
   const int window = GW ? a.window : -1;
-  const int i0 = (kb * BKV) / BQB;
+  const int i0 = kb;  // BQB == BKV: the first query tile that reaches these keys
   // Query tiles at or after this key tile, up to the last one a window reaches;
   // every query head of the KV head's group in turn (tile t: head
   // hk * group + t / nqt, query tile i0 + t % nqt), so dK and dV accumulate
@@ -458,18 +811,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (threadIdx.x == 0) {
     tc::mbar_init(kv_full, 1);
-    for (int i = 0; i < QST; ++i) {
-      tc::mbar_init(&qd_full[i], 32);  // the TMA lane (with its bytes) + 31 lse/D loader lanes
-      tc::mbar_init(&qd_empty[i], 1);
-    }
-    tc::mbar_init(sdp_full, 1);
-    tc::mbar_init(sdp_empty, 256);
-    tc::mbar_init(pds_full, 256);
-    tc::mbar_init(pds_empty, 1);
     for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&dq_full[i], 1);
-      tc::mbar_init(&dq_empty[i], 128);
+      tc::mbar_init(&q_full[i], 32);  // the TMA lane (with its bytes) + 31 staging lanes
+      tc::mbar_init(&q_empty[i], 1);
+      tc::mbar_init(&do_full[i], 32);
+      tc::mbar_init(&do_empty[i], 1);
     }
+    tc::mbar_init(s_full, 1);
+    tc::mbar_init(p_full, 256);
+    tc::mbar_init(dp_full, 1);
+    tc::mbar_init(ds_full, 256);
+    // One lane of each dQ warp once its staging is read; with SDS the lane
+    // that stored the tile.
+    tc::mbar_init(ds_empty, SDS ? 1 : 4);
+    tc::mbar_init(dq_full, 1);
+    tc::mbar_init(dq_empty, 128);
     tc::mbar_init(dkv_full, 1);
     tc::mbar_init(drained, 1);
     *abort_flag = 0;
@@ -485,188 +841,333 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // Lane 0 issues the TMA copies; all 32 lanes stage lse * log2(e) and D of
-    // the query tile into shared memory and arrive on the same barrier.
+    // Lane 0 issues the TMA copies; all 32 lanes stage lse * log2(e) (with Q)
+    // and D (with dO) of the query tile and arrive on the same barriers.
     if (lane == 0) {
       tc::tma_prefetch_desc(&tq);
       tc::tma_prefetch_desc(&tk);
       tc::tma_prefetch_desc(&tv);
       tc::tma_prefetch_desc(&tdo);
+      tc::tma_prefetch_desc(&tdq);
       tc::mbar_arrive_expect_tx(kv_full, 2 * TILE);
       for (int c = 0; c < 2; ++c) {
         tc::tma_load_3d(smem + B_OFF_K + c * (TILE / 2), &tk, kv_full, kcol0 + 64 * c, kb * BKV, b);
         tc::tma_load_3d(smem + B_OFF_V + c * (TILE / 2), &tv, kv_full, kcol0 + 64 * c, kb * BKV, b);
       }
     }
-    int issued = 0;
+    int issued_q = 0, issued_do = 0;
     bool ok = true;
     for (int t = 0; t < nblk; ++t) {
-      const int st = t % QST;
-      const uint32_t ph = (t / QST) & 1;
-      bool w = true;
-      if (lane == 0) w = tc::mbar_wait(&qd_empty[st], ph ^ 1, abort_flag, a.status);
-      if (!__shfl_sync(0xffffffffu, (int)w, 0)) { ok = false; break; }
+      const int st = t & 1;
+      const uint32_t ph = (t >> 1) & 1;
       const int hq = GW ? hk * group + t / nqt : hk;
       const int q0 = (i0 + (GW ? t % nqt : t)) * BQB;
       const int qcol0 = hq * HD;
+      bool w = true;
+      if (lane == 0) w = tc::mbar_wait(&q_empty[st], ph ^ 1, abort_flag, a.status);
+      if (!__shfl_sync(0xffffffffu, (int)w, 0)) { ok = false; break; }
       const float* lse_bh = a.lse + ((int64_t)b * a.H + hq) * a.T;
-      const float* d_bh = a.delta + ((int64_t)b * a.H + hq) * a.T;
-      float* ld = reinterpret_cast<float*>(smem + B_OFF_LD) + st * 2 * BQB;
+      float* lq = reinterpret_cast<float*>(smem + B_OFF_LQ) + st * BQB;
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int c = lane + 32 * u;
-        const int q = q0 + c;
-        ld[c] = q < a.T ? lse_bh[q] * 1.4426950408889634f : INFINITY;
-        ld[BQB + c] = q < a.T ? d_bh[q] : 0.f;
+      for (int u = 0; u < 4; ++u) {
+        const int q = q0 + lane + 32 * u;
+        lq[lane + 32 * u] = q < a.T ? lse_bh[q] * 1.4426950408889634f : INFINITY;
       }
       if (lane == 0) {
-        tc::mbar_arrive_expect_tx(&qd_full[st], 2 * QT);
-        for (int c = 0; c < 2; ++c) {
-          tc::tma_load_3d(smem + B_OFF_Q + st * QT + c * (QT / 2), &tq, &qd_full[st], qcol0 + 64 * c, q0, b);
-          tc::tma_load_3d(smem + B_OFF_DO + st * QT + c * (QT / 2), &tdo, &qd_full[st], qcol0 + 64 * c, q0, b);
-        }
+        tc::mbar_arrive_expect_tx(&q_full[st], TILE);
+        for (int c = 0; c < 2; ++c)
+          tc::tma_load_3d(smem + B_OFF_Q + st * TILE + c * (TILE / 2), &tq, &q_full[st], qcol0 + 64 * c, q0, b);
       } else {
-        tc::mbar_arrive(&qd_full[st]);
+        tc::mbar_arrive(&q_full[st]);
       }
-      ++issued;
+      ++issued_q;
+      if (lane == 0) w = tc::mbar_wait(&do_empty[st], ph ^ 1, abort_flag, a.status);
+      if (!__shfl_sync(0xffffffffu, (int)w, 0)) { ok = false; break; }
+      const float* d_bh = a.delta + ((int64_t)b * a.H + hq) * a.T;
+      float* ldd = reinterpret_cast<float*>(smem + B_OFF_LD) + st * BQB;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int q = q0 + lane + 32 * u;
+        ldd[lane + 32 * u] = q < a.T ? d_bh[q] : 0.f;
+      }
+      if (lane == 0) {
+        tc::mbar_arrive_expect_tx(&do_full[st], TILE);
+        for (int c = 0; c < 2; ++c)
+          tc::tma_load_3d(smem + B_OFF_DO + st * TILE + c * (TILE / 2), &tdo, &do_full[st], qcol0 + 64 * c, q0, b);
+      } else {
+        tc::mbar_arrive(&do_full[st]);
+      }
+      ++issued_do;
     }
     if (!ok && lane == 0) {
       drain_wait(kv_full, 0);
-      for (int t = max(0, issued - QST); t < issued; ++t) drain_wait(&qd_full[t % QST], (t / QST) & 1);
+      for (int t = max(0, issued_q - 2); t < issued_q; ++t) drain_wait(&q_full[t & 1], (t >> 1) & 1);
+      for (int t = max(0, issued_do - 2); t < issued_do; ++t) drain_wait(&do_full[t & 1], (t >> 1) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t id_sdp = tc::idesc_bf16_f32(128, BQB, 0, 0);
-      const uint32_t id_acc = tc::idesc_bf16_f32(128, 128, 0, 1);
-      const uint32_t id_dq = tc::idesc_bf16_f32(128, BQB, 1, 1);
+      const uint32_t id_ss = tc::idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
+      const uint32_t id_ts = tc::idesc_bf16_f32(128, 128, 0, 1);  // dV, dK: A from TMEM
+      const uint32_t id_dq = tc::idesc_bf16_f32(128, 128, 1, 1);  // dQ: both MN-major
       // Descriptors are built once; each MMA adds a constant byte offset.
       const uint64_t kK = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_K), 16, 1024);
       const uint64_t vK = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_V), 16, 1024);
       const uint64_t kMN = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_K), TILE / 2, 1024);
       const uint64_t qK = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_Q), 16, 1024);
       const uint64_t doK = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_DO), 16, 1024);
-      const uint64_t qMN = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_Q), QT / 2, 1024);
-      const uint64_t doMN = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_DO), QT / 2, 1024);
-      const uint64_t pK = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_P), 16, 1024);
-      const uint64_t dsK = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_DS), 16, 1024);
-      const uint64_t dsMN = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_DS), PT, 1024);
+      const uint64_t qMN = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_Q), TILE / 2, 1024);
+      const uint64_t doMN = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_DO), TILE / 2, 1024);
+      const uint64_t dsMN = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_DS), TILE / 2, 1024);
       bool ok = tc::mbar_wait(kv_full, 0, abort_flag, a.status);
-      // S^T and dP^T of query tile t into TMEM once the tile has landed and the
-      // softmax warps have read the previous scores.
-      auto issue_sdp = [&](int t) -> bool {
-        const int st = t % QST;
-        if (!tc::mbar_wait(&qd_full[st], (t / QST) & 1, abort_flag, a.status)) return false;
-        if (t > 0 && !tc::mbar_wait(sdp_empty, (t - 1) & 1, abort_flag, a.status)) return false;
+      // S^T of tile t once its Q has landed; the S columns are free because
+      // every earlier MMA that reads them (dV of tile t - 1) was issued first.
+      auto issue_s = [&](int t) -> bool {
+        const int st = t & 1;
+        if (!tc::mbar_wait(&q_full[st], (t >> 1) & 1, abort_flag, a.status)) return false;
         tc::tc_fence_after();
-        const uint64_t qd = qK + (uint64_t)((st * QT) >> 4);
-        const uint64_t dod = doK + (uint64_t)((st * QT) >> 4);
+        const uint64_t qd = tc::desc_add(qK, st * TILE);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t ao = (kk >> 2) * (TILE / 2) + (kk & 3) * 32;
-          const uint32_t bo = (kk >> 2) * (QT / 2) + (kk & 3) * 32;
-          tc::umma_bf16_ss(tmem + TB_S, tc::desc_add(kK, ao), tc::desc_add(qd, bo), id_sdp,
-                           kk > 0 ? 1u : 0u);
-          tc::umma_bf16_ss(tmem + TB_DP, tc::desc_add(vK, ao), tc::desc_add(dod, bo), id_sdp,
+          const uint32_t off = (kk >> 2) * (TILE / 2) + (kk & 3) * 32;
+          tc::umma_bf16_ss(tmem + TB_S, tc::desc_add(kK, off), tc::desc_add(qd, off), id_ss,
                            kk > 0 ? 1u : 0u);
         }
-        tc::umma_commit(sdp_full);
+        tc::umma_commit(s_full);
         return true;
       };
-      if (ok) ok = issue_sdp(0);
-      for (int t = 0; t < nblk && ok; ++t) {
-        const int st = t % QST;
-        if (t + 1 < nblk && !issue_sdp(t + 1)) { ok = false; break; }
-        const int db = t & 1;  // dQ accumulator of this tile
-        if (!tc::mbar_wait(pds_full, t & 1, abort_flag, a.status) ||
-            !tc::mbar_wait(&dq_empty[db], ((t >> 1) & 1) ^ 1, abort_flag, a.status)) { ok = false; break; }
+      // dP^T of tile t once its dO has landed (the DP columns are free: the
+      // dQ warps have read the previous tile's dQ).
+      auto issue_dp = [&](int t) -> bool {
+        const int st = t & 1;
+        if (!tc::mbar_wait(&do_full[st], (t >> 1) & 1, abort_flag, a.status)) return false;
         tc::tc_fence_after();
-        const uint64_t qmn = qMN + (uint64_t)((st * QT) >> 4);
-        const uint64_t domn = doMN + (uint64_t)((st * QT) >> 4);
+        const uint64_t dod = tc::desc_add(doK, st * TILE);
 #pragma unroll
-        for (int kk = 0; kk < BQB / 16; ++kk) {
-          const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-          tc::umma_bf16_ss(tmem + TB_DV, tc::desc_add(pK, kk * 32), tc::desc_add(domn, kk * 2048),
-                           id_acc, acc);
-          tc::umma_bf16_ss(tmem + TB_DK, tc::desc_add(dsK, kk * 32), tc::desc_add(qmn, kk * 2048),
-                           id_acc, acc);
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (TILE / 2) + (kk & 3) * 32;
+          tc::umma_bf16_ss(tmem + TB_DP, tc::desc_add(vK, off), tc::desc_add(dod, off), id_ss,
+                           kk > 0 ? 1u : 0u);
         }
+        tc::umma_commit(dp_full);
+        return true;
+      };
+      if (ok) ok = issue_s(0) && issue_dp(0);
+      for (int t = 0; t < nblk && ok; ++t) {
+        const int st = t & 1;
+        if (!tc::mbar_wait(p_full, t & 1, abort_flag, a.status)) { ok = false; break; }
+        tc::tc_fence_after();
+        // dV += P^T dO: query step kk (16 queries) is 8 packed columns of the
+        // softmax half that owns it (half h at column 64 h).
+        const uint64_t domn = tc::desc_add(doMN, st * TILE);
 #pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk)
-          tc::umma_bf16_ss(tmem + TB_DQ + db * BQB, tc::desc_add(kMN, kk * 2048),
-                           tc::desc_add(dsMN, kk * 2048), id_dq, kk > 0 ? 1u : 0u);
-        tc::umma_commit(pds_empty);
-        tc::umma_commit(&qd_empty[st]);
-        tc::umma_commit(&dq_full[db]);
+        for (int kk = 0; kk < BQB / 16; ++kk)
+          tc::umma_bf16_ts(tmem + TB_DV, tmem + TB_S + (kk >> 2) * 64 + (kk & 3) * 8,
+                           tc::desc_add(domn, kk * 2048), id_ts, (t > 0 || kk > 0) ? 1u : 0u);
+        tc::umma_commit(&do_empty[st]);
+        if (t + 1 < nblk && !issue_s(t + 1)) { ok = false; break; }
+        if (!tc::mbar_wait(ds_full, t & 1, abort_flag, a.status)) { ok = false; break; }
+        tc::tc_fence_after();
+        const uint64_t qmn = tc::desc_add(qMN, st * TILE);
+#pragma unroll
+        for (int kk = 0; kk < BQB / 16; ++kk)
+          tc::umma_bf16_ts(tmem + TB_DK, tmem + TB_DP + (kk >> 2) * 64 + (kk & 3) * 8,
+                           tc::desc_add(qmn, kk * 2048), id_ts, (t > 0 || kk > 0) ? 1u : 0u);
+        tc::umma_commit(&q_empty[st]);
+        if (!SDS) {
+          // dQ = dS K (one query per TMEM lane): key step kk (16 keys) is 2 KB
+          // into both MN-major tiles.
+#pragma unroll
+          for (int kk = 0; kk < BKV / 16; ++kk)
+            tc::umma_bf16_ss(tmem + TB_DP, tc::desc_add(dsMN, kk * 2048),
+                             tc::desc_add(kMN, kk * 2048), id_dq, kk > 0 ? 1u : 0u);
+          tc::umma_commit(dq_full);
+        }
+        if (t + 1 < nblk) {
+          if (!SDS) {
+            if (!tc::mbar_wait(dq_empty, t & 1, abort_flag, a.status)) { ok = false; break; }
+            tc::tc_fence_after();
+          }
+          // With SDS the DP columns are free once dK (issued just before) has
+          // read dS^T from them: the MMAs run in issue order.
+          if (!issue_dp(t + 1)) { ok = false; break; }
+        }
       }
       if (ok) tc::umma_commit(dkv_full);
       tc::umma_commit(drained);
       drain_wait(drained, 0);
     }
   } else if (warp < 10) {
-    // ---------------- P^T and dS^T: one key row per thread, half the columns per warp
+    // ---------------- P^T and dS^T: one key row per thread, half the queries per warp
     const int qw = warp & 3;
-    const int ch = (warp - 2) >> 2;  // column half: queries [32 ch, 32 ch + 32) of the tile
+    const int hf = (warp - 2) >> 2;  // query half: [64 hf, 64 hf + 64) of the tile
     const int row = qw * 32 + lane;
     const int key = kb * BKV + row;
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
-    const uint32_t p_row = tc::smem_u32(smem + B_OFF_P) + row * 128;
-    const uint32_t ds_row = tc::smem_u32(smem + B_OFF_DS) + row * 128;
+    const uint32_t s_col = lane_base + TB_S + 64 * hf;
+    const uint32_t dp_col = lane_base + TB_DP + 64 * hf;
+    const uint32_t ds_row = tc::smem_u32(smem + B_OFF_DS) + hf * (TILE / 2) + row * 128;
     bool ok = true;
     for (int t = 0; t < nblk; ++t) {
-      const int q0 = (i0 + (GW ? t % nqt : t)) * BQB + 32 * ch;
-      const float* ld = reinterpret_cast<const float*>(smem + B_OFF_LD) + (t % QST) * 2 * BQB + 32 * ch;
-      ok = tc::mbar_wait(sdp_full, t & 1, abort_flag, a.status);
+      const int st = t & 1;
+      const uint32_t ph = (t >> 1) & 1;
+      const int qh = (i0 + (GW ? t % nqt : t)) * BQB + 64 * hf;  // first query of this half
+      ok = tc::mbar_wait(s_full, t & 1, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc::tc_fence_after();
-      uint32_t sv[32], dp[32];
-      tc::tmem_ld_32x32b_x32(lane_base + TB_S + 32 * ch, sv);
-      tc::tmem_ld_32x32b_x32(lane_base + TB_DP + 32 * ch, dp);
-      tc::tmem_ld_wait();
-      tc::tc_fence_before();
-      tc::mbar_arrive(sdp_empty);
-      // The tile's lse/D, staged by the TMA warp and published by the stage's
-      // qd_full barrier (already complete: the scores came from it).
-      ok = tc::mbar_wait(&qd_full[t % QST], (t / QST) & 1, abort_flag, a.status);
+      // The tile's lse, staged by the TMA warp and published by the stage's
+      // q_full barrier (already complete: the scores came from it).
+      ok = tc::mbar_wait(&q_full[st], ph, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      uint32_t pp[16], pd[16];
-      const bool edge = (q0 < key + 1) || (q0 + 32 > a.T) || (key >= a.T) ||
-                        (window >= 0 && q0 + 31 > key + window);  // diagonal, T or window
+      const float* lq = reinterpret_cast<const float*>(smem + B_OFF_LQ) + st * BQB + 64 * hf;
+      // The half reaches the diagonal, T, or past the window of this key.
+      const bool edge = (qh < key) || (qh + 63 >= a.T) || (key >= a.T) ||
+                        (window >= 0 && qh + 63 > key + window);
+      uint32_t pk[2][16];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        float p0 = ex2(__uint_as_float(sv[2 * c]) * a.sl2 - ld[2 * c]);
-        float p1 = ex2(__uint_as_float(sv[2 * c + 1]) * a.sl2 - ld[2 * c + 1]);
-        if (edge) {
-          const int qa = q0 + 2 * c, qb2 = qa + 1;
-          if (qa < key || qa >= a.T || key >= a.T || (window >= 0 && qa > key + window)) p0 = 0.f;
-          if (qb2 < key || qb2 >= a.T || key >= a.T || (window >= 0 && qb2 > key + window)) p1 = 0.f;
+      for (int c = 0; c < 2; ++c) {
+        uint32_t sv[32];
+        tc::tmem_ld_32x32b_x32(s_col + 32 * c, sv);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int j = 32 * c + 2 * i;
+          float p0 = ex2(fmaf(__uint_as_float(sv[2 * i]), a.sl2, -lq[j]));
+          float p1 = ex2(fmaf(__uint_as_float(sv[2 * i + 1]), a.sl2, -lq[j + 1]));
+          if (edge) {
+            const int qa = qh + j, qb2 = qa + 1;
+            if (qa < key || qa >= a.T || key >= a.T || (window >= 0 && qa > key + window)) p0 = 0.f;
+            if (qb2 < key || qb2 >= a.T || key >= a.T || (window >= 0 && qb2 > key + window)) p1 = 0.f;
+          }
+          pk[c][i] = pack_bf16x2(p0, p1);
         }
-        const float d0 = p0 * (__uint_as_float(dp[2 * c]) - ld[BQB + 2 * c]);
-        const float d1 = p1 * (__uint_as_float(dp[2 * c + 1]) - ld[BQB + 2 * c + 1]);
-        pp[c] = pack_bf16x2(p0, p1);
-        pd[c] = pack_bf16x2(d0, d1);
       }
-      ok = tc::mbar_wait(pds_empty, (t & 1) ^ 1, abort_flag, a.status);
+      tc::tmem_st_32x32b_x16(s_col, pk[0]);
+      tc::tmem_st_32x32b_x16(s_col + 16, pk[1]);
+      tc::tmem_st_wait();
+      tc::tc_fence_before();
+      tc::mbar_arrive(p_full);
+      // dS^T = P^T (dP^T - D), from the bf16 P the dV product reads.
+      ok = tc::mbar_wait(dp_full, t & 1, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc::tc_fence_after();
+      ok = tc::mbar_wait(&do_full[st], ph, abort_flag, a.status);  // D, staged with dO
+      // The shared dS tile is free once the previous tile's dQ product is done.
+      ok = ok && tc::mbar_wait(ds_empty, (t & 1) ^ 1, abort_flag, a.status);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      const float* ld = reinterpret_cast<const float*>(smem + B_OFF_LD) + st * BQB + 64 * hf;
+      // 32 queries at a time: chunk c's dS^T goes over the dP^T columns of
+      // queries [16 c, 16 c + 16), which chunk 0 has already read.
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const uint32_t sw = (uint32_t)(((4 * ch + u) ^ (row & 7)) << 4);
-        tc::st_shared_v4(p_row + sw, pp[4 * u], pp[4 * u + 1], pp[4 * u + 2], pp[4 * u + 3]);
-        tc::st_shared_v4(ds_row + sw, pd[4 * u], pd[4 * u + 1], pd[4 * u + 2], pd[4 * u + 3]);
+      for (int c = 0; c < 2; ++c) {
+        uint32_t dpv[32];
+        tc::tmem_ld_32x32b_x32(dp_col + 32 * c, dpv);
+        tc::tmem_ld_wait();
+        uint32_t pd[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int j = 32 * c + 2 * i;
+          const float2 p = unpack_bf16x2(pk[c][i]);
+          const float d0 = p.x * (__uint_as_float(dpv[2 * i]) - ld[j]);
+          const float d1 = p.y * (__uint_as_float(dpv[2 * i + 1]) - ld[j + 1]);
+          pd[i] = pack_bf16x2(d0, d1);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t sw = (uint32_t)(((4 * c + u) ^ (row & 7)) << 4);
+          tc::st_shared_v4(ds_row + sw, pd[4 * u], pd[4 * u + 1], pd[4 * u + 2], pd[4 * u + 3]);
+        }
+        tc::tmem_st_32x32b_x16(dp_col + 16 * c, pd);
       }
+      tc::tmem_st_wait();
       tc::fence_proxy_async_smem();
-      tc::mbar_arrive(pds_full);
+      tc::tc_fence_before();
+      tc::mbar_arrive(ds_full);
     }
     if (ok) {
       ok = tc::mbar_wait(dkv_full, 0, abort_flag, a.status);
       ok = __all_sync(0xffffffffu, ok);
     }
-    if (ok) {
-      // Warps of column half 0 write dV rows, those of half 1 dK rows.
+    if (ok && hf == 1 && a.rope_tab) {
+      // dK through the RoPE + QK-norm backward: with g = dK, yhat the saved
+      // normalised k (this CTA's K tile) and r its 1/rms,
+      //   dr = r (g - yhat mean(g yhat)),  dk = R(-theta) dr  (pairs i, i + 64).
+      tc::tc_fence_after();
+      const uint32_t krow = tc::smem_u32(smem + B_OFF_K) + row * 128;
+      // 32 dims of yhat: chunk c is box c / 2, 16-byte units 4 (c % 2) .. + 3.
+      auto load_y = [&](int c, float (&y)[32]) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint4 w = tc::ld_shared_v4(krow + (c >> 1) * (TILE / 2) +
+                                           ((((c & 1) * 4 + u) ^ (row & 7)) << 4));
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = unpack_bf16x2(ws[e]);
+            y[8 * u + 2 * e] = f.x;
+            y[8 * u + 2 * e + 1] = f.y;
+          }
+        }
+      };
+      float dot = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t g[32];
+        float y[32];
+        tc::tmem_ld_32x32b_x32(lane_base + TB_DK + 32 * c, g);
+        load_y(c, y);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) dot = fmaf(__uint_as_float(g[i]), y[i], dot);
+      }
+      // Keys at or past T (a ragged last tile) take part in the warp-wide
+      // TMEM loads but read and write nothing in global memory.
+      const bool live = key < a.T;
+      const int64_t tok = (int64_t)b * a.T + (live ? key : 0);
+      const float r = live ? a.rstd_k[tok * a.Hkv + hk] : 0.f;
+      const float m = dot * a.scale / 128.f;
+      __nv_bfloat16* dst = a.dk + tok * a.ldg + kcol0;
+      const float2* cs = a.rope_tab + (int64_t)(live ? key : 0) * 64;
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        uint32_t g0[32], g1[32];
+        float y0[32], y1[32];
+        tc::tmem_ld_32x32b_x32(lane_base + TB_DK + 32 * c, g0);
+        tc::tmem_ld_32x32b_x32(lane_base + TB_DK + 64 + 32 * c, g1);
+        load_y(c, y0);
+        load_y(c + 2, y1);
+        tc::tmem_ld_wait();
+        if (live) {
+          uint32_t lo[16], hi[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float o_lo[2], o_hi[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const float d0 = r * (__uint_as_float(g0[i + e]) * a.scale - y0[i + e] * m);
+              const float d1 = r * (__uint_as_float(g1[i + e]) * a.scale - y1[i + e] * m);
+              const float2 t = cs[32 * c + i + e];  // (cos, sin) of pair 32 c + i + e
+              o_lo[e] = d0 * t.x + d1 * t.y;
+              o_hi[e] = d1 * t.x - d0 * t.y;
+            }
+            lo[i / 2] = pack_bf16x2(o_lo[0], o_lo[1]);
+            hi[i / 2] = pack_bf16x2(o_hi[0], o_hi[1]);
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            reinterpret_cast<uint4*>(dst + 32 * c)[u] =
+                make_uint4(lo[4 * u], lo[4 * u + 1], lo[4 * u + 2], lo[4 * u + 3]);
+            reinterpret_cast<uint4*>(dst + 64 + 32 * c)[u] =
+                make_uint4(hi[4 * u], hi[4 * u + 1], hi[4 * u + 2], hi[4 * u + 3]);
+          }
+        }
+      }
+    } else if (ok) {
+      // Warps of query half 0 write dV rows, those of half 1 dK rows.
       tc::tc_fence_after();
       const int64_t grow = ((int64_t)b * a.T + key) * a.ldg + kcol0;
-      const uint32_t base = lane_base + (ch ? TB_DK : TB_DV);
-      const float mul = ch ? a.scale : 1.f;
-      __nv_bfloat16* dst = (ch ? a.dk : a.dv) + grow;
+      const uint32_t base = lane_base + (hf ? TB_DK : TB_DV);
+      const float mul = hf ? a.scale : 1.f;
+      __nv_bfloat16* dst = (hf ? a.dk : a.dv) + grow;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t o[32];
@@ -686,40 +1187,74 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
   } else {
-    // ---------------- dQ^T rows: one head-dim per thread, atomics into dq
+    if (SDS) {
+      // ---------------- dS^T tiles to global memory (one lane of warp 10)
+      if (warp == 10 && lane == 0) {
+        for (int t = 0; t < nblk; ++t) {
+          const int q0 = (i0 + (GW ? t % nqt : t)) * BQB;
+          const int hq = GW ? hk * group + t / nqt : hk;
+          if (!tc::mbar_wait(ds_full, t & 1, abort_flag, a.status)) break;
+          for (int c = 0; c < 2; ++c)
+            tc::tma_store_3d(&tdq, tc::smem_u32(smem + B_OFF_DS) + c * (TILE / 2), q0 + 64 * c,
+                             kb * BKV, b * a.H + hq);
+          tc::bulk_commit_group();
+          tc::bulk_wait_group_read0();  // the tile may be rewritten once read
+          tc::mbar_arrive(ds_empty);
+        }
+        tc::bulk_wait_group0();
+      }
+    } else {
+    // ---------------- dQ rows: one query per thread, TMA bulk reductions into dq
     const int qw = warp & 3;
-    const int dim = qw * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
-    const int64_t dq_row = (int64_t)a.H * HD;
+    // This warp's 8 KB of the dS tile: its 32 queries x 64 dims as two
+    // swizzled 32 x 32 fp32 boxes.
+    const uint32_t slot = tc::smem_u32(smem + B_OFF_DS) + qw * 8192;
+    bool pending = false;  // this warp has bulk reductions in flight
     for (int t = 0; t < nblk; ++t) {
-      const int q0 = (i0 + (GW ? t % nqt : t)) * BQB;
-      float* dq_bh = a.dq + (int64_t)b * a.T * dq_row + (GW ? hk * group + t / nqt : hk) * HD + dim;
-      bool ok = tc::mbar_wait(&dq_full[t & 1], (t >> 1) & 1, abort_flag, a.status);
+      const int q0 = (i0 + (GW ? t % nqt : t)) * BQB + 32 * qw;
+      const int dcol = (GW ? hk * group + t / nqt : hk) * HD;
+      bool ok = tc::mbar_wait(dq_full, t & 1, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc::tc_fence_after();
-      float* dst = dq_bh + (int64_t)q0 * dq_row;
-      const int nq = min(BQB, a.T - q0);
-#pragma unroll 1
-      for (int c0 = 0; c0 < BQB; c0 += 16) {
-        uint32_t v[16];
-        tc::tmem_ld_32x32b_x16(lane_base + TB_DQ + (t & 1) * BQB + c0, v);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {  // dims [64 hh, 64 hh + 64)
+        uint32_t v[2][32];
+        tc::tmem_ld_32x32b_x32(lane_base + TB_DP + 64 * hh, v[0]);
+        tc::tmem_ld_32x32b_x32(lane_base + TB_DP + 64 * hh + 32, v[1]);
         tc::tmem_ld_wait();
-        if (c0 + 16 == BQB) {  // the whole tile has been read: TMEM may be reused
+        if (hh == 1) {  // every dQ column read: the MMA warp may reuse them
           tc::tc_fence_before();
-          tc::mbar_arrive(&dq_empty[t & 1]);
+          tc::mbar_arrive(dq_empty);
         }
-        float vv[16];
+        if (hh == 1 && lane == 0) tc::bulk_wait_group_read0();  // the first half's boxes are read
+        __syncwarp();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) vv[j] = __uint_as_float(v[j]) * a.scale;
-        if (c0 + 16 <= nq) {
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
-          for (int j = 0; j < 16; ++j) atomicAdd(dst + (int64_t)(c0 + j) * dq_row, vv[j]);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (c0 + j < nq) atomicAdd(dst + (int64_t)(c0 + j) * dq_row, vv[j]);
+          for (int u = 0; u < 8; ++u)
+            tc::st_shared_v4(slot + c * 4096 + lane * 128 + ((u ^ (lane & 7)) << 4),
+                             __float_as_uint(__uint_as_float(v[c][4 * u]) * a.scale),
+                             __float_as_uint(__uint_as_float(v[c][4 * u + 1]) * a.scale),
+                             __float_as_uint(__uint_as_float(v[c][4 * u + 2]) * a.scale),
+                             __float_as_uint(__uint_as_float(v[c][4 * u + 3]) * a.scale));
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          for (int c = 0; c < 2; ++c)
+            tc::tma_reduce_add_3d(&tdq, slot + c * 4096, dcol + 64 * hh + 32 * c, q0, b);
+          tc::bulk_commit_group();
         }
       }
+      pending = true;
+      // The dS tile is the next tile's again once these boxes are read.
+      if (lane == 0) {
+        tc::bulk_wait_group_read0();
+        tc::mbar_arrive(ds_empty);
+      }
+      __syncwarp();
+    }
+    if (pending && lane == 0) tc::bulk_wait_group0();
     }
   }
   tc::tc_fence_before();
@@ -730,6 +1265,226 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 }
 
+
+// ------------------------------------------------------------------ dQ from stored dS
+// Query side of the backward when the key-side kernel stored dS^T: one CTA per
+// (128-query tile, query head, batch row), heaviest tiles first, accumulating
+//   dQ = sum over key tiles kb of dS(i, kb) K_kb        (M 128 queries, N 128 dims)
+// in TMEM through a three-stage TMA ring of the dS^T tile ([128 keys][128
+// queries], read MN-major) and the K tile ([128 keys][128 dims], MN-major).
+// The epilogue takes dQ through the backward of the q-side RoPE + QK-norm:
+// with g = dQ / sqrt(128), yhat the saved normalised q and r its 1/rms,
+//   dr = r (g - yhat mean(g yhat)),  dq = R(-theta) dr  (pairs i, i + 64),
+// written as bf16 into the q slice of the q|k|v gradient.  192 threads:
+// warp 0 TMA, warp 1 TMEM owner and MMA issue, warps 2..5 one query row each.
+constexpr int kDqThreads = 192;
+constexpr int kDqStages = 3;
+constexpr int DQ_STAGE = 2 * TILE;  // dS^T tile + K tile
+constexpr int DQ_OFF_BAR = kDqStages * DQ_STAGE;
+constexpr int kDqSmem = DQ_OFF_BAR + 256;
+static_assert(kDqSmem <= 232448, "dQ kernel shared memory budget");
+
+struct DqArgs {
+  int T, H, nqb;
+  int group;   // query heads per KV head
+  int window;  // query t sees keys [t - window, t]; < 0: every key up to t
+  float scale;
+  const __nv_bfloat16* yhat;  // saved normalised q: row tok at yhat + tok * ldy, head h at + h * 128
+  int64_t ldy;
+  const float* rstd_q;        // [B * T, H]
+  const float2* rope_tab;     // [T][64] (cos, sin)
+  __nv_bfloat16* out;         // dq rows: out + tok * ldo + h * 128
+  int64_t ldo;
+  int* status;
+};
+
+template <bool GW>
+__global__ void __launch_bounds__(kDqThreads, 1)
+    attn_dq_kernel(const __grid_constant__ CUtensorMap tds, const __grid_constant__ CUtensorMap tk,
+                   const DqArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if ((tc::smem_u32(smem_raw) & 1023u) != 0) {  // never expected; no room to realign
+    if (threadIdx.x == 0 && a.status) atomicExch(a.status, kDevTimeout);
+    return;
+  }
+  uint8_t* smem = smem_raw;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DQ_OFF_BAR);
+  uint64_t* full = bars;                    // [kDqStages]
+  uint64_t* empty = bars + kDqStages;       // [kDqStages]
+  uint64_t* acc_full = bars + 2 * kDqStages;
+  uint64_t* drained = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qi = a.nqb - 1 - (int)blockIdx.x;  // heaviest tiles first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int hk = GW ? h / a.group : h;
+  const int window = GW ? a.window : -1;
+  // Key tiles whose dS^T tiles the key-side kernel stored for this query
+  // tile: from the first one a window reaches to the diagonal.
+  const int lo = window < 0 ? 0 : qi * BQB - BKV + 1 - window;
+  const int kb_lo = lo <= 0 ? 0 : (lo + BKV - 1) / BKV;
+  const int n = qi - kb_lo + 1;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kDqStages; ++i) {
+      tc::mbar_init(&full[i], 1);
+      tc::mbar_init(&empty[i], 1);
+    }
+    tc::mbar_init(acc_full, 1);
+    tc::mbar_init(drained, 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, 128);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tc::tma_prefetch_desc(&tds);
+      tc::tma_prefetch_desc(&tk);
+      int issued = 0;
+      bool ok = true;
+      for (int t = 0; t < n; ++t) {
+        const int st = t % kDqStages;
+        const uint32_t ph = (t / kDqStages) & 1;
+        if (!tc::mbar_wait(&empty[st], ph ^ 1, abort_flag, a.status)) { ok = false; break; }
+        const int kb = kb_lo + t;
+        uint8_t* base = smem + st * DQ_STAGE;
+        tc::mbar_arrive_expect_tx(&full[st], 2 * TILE);
+        for (int c = 0; c < 2; ++c) {
+          tc::tma_load_3d(base + c * (TILE / 2), &tds, &full[st], qi * BQB + 64 * c, kb * BKV,
+                          b * a.H + h);
+          tc::tma_load_3d(base + TILE + c * (TILE / 2), &tk, &full[st], hk * HD + 64 * c, kb * BKV, b);
+        }
+        ++issued;
+      }
+      if (!ok)
+        for (int t = max(0, issued - kDqStages); t < issued; ++t)
+          drain_wait(&full[t % kDqStages], (t / kDqStages) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id = tc::idesc_bf16_f32(128, 128, 1, 1);
+      const uint64_t ad = tc::smem_desc_sw128(tc::smem_u32(smem), TILE / 2, 1024);
+      const uint64_t bd = tc::smem_desc_sw128(tc::smem_u32(smem + TILE), TILE / 2, 1024);
+      bool ok = true;
+      for (int t = 0; t < n && ok; ++t) {
+        const int st = t % kDqStages;
+        if (!tc::mbar_wait(&full[st], (t / kDqStages) & 1, abort_flag, a.status)) { ok = false; break; }
+        tc::tc_fence_after();
+        const uint64_t a0 = tc::desc_add(ad, st * DQ_STAGE), b0 = tc::desc_add(bd, st * DQ_STAGE);
+#pragma unroll
+        for (int kk = 0; kk < BKV / 16; ++kk)
+          tc::umma_bf16_ss(tmem, tc::desc_add(a0, kk * 2048), tc::desc_add(b0, kk * 2048), id,
+                           (t > 0 || kk > 0) ? 1u : 0u);
+        tc::umma_commit(&empty[st]);
+      }
+      if (ok) tc::umma_commit(acc_full);
+      tc::umma_commit(drained);
+      drain_wait(drained, 0);
+    }
+  } else {
+    // Epilogue: one query row per thread (warp w reaches TMEM lanes of quarter w % 4).
+    const int qw = warp & 3;
+    const int row = qw * 32 + lane;
+    const int q = qi * BQB + row;
+    const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
+    bool ok = tc::mbar_wait(acc_full, 0, abort_flag, a.status);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc::tc_fence_after();
+      const bool live = q < a.T;
+      const int64_t tok = (int64_t)b * a.T + (live ? q : 0);
+      const __nv_bfloat16* yrow = a.yhat + tok * a.ldy + h * HD;
+      // 32 dims of yhat starting at dim 32 c.
+      auto load_y = [&](int c, float (&y)[32]) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint4 w = live ? reinterpret_cast<const uint4*>(yrow + 32 * c)[u]
+                               : make_uint4(0u, 0u, 0u, 0u);
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = unpack_bf16x2(ws[e]);
+            y[8 * u + 2 * e] = f.x;
+            y[8 * u + 2 * e + 1] = f.y;
+          }
+        }
+      };
+      float dot = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t g[32];
+        float y[32];
+        tc::tmem_ld_32x32b_x32(lane_base + 32 * c, g);
+        load_y(c, y);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) dot = fmaf(__uint_as_float(g[i]), y[i], dot);
+      }
+      const float r = live ? a.rstd_q[tok * a.H + h] : 0.f;
+      const float m = dot * a.scale / 128.f;
+      __nv_bfloat16* dst = a.out + tok * a.ldo + h * HD;
+      const float2* cs = a.rope_tab + (int64_t)(live ? q : 0) * 64;
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        uint32_t g0[32], g1[32];
+        float y0[32], y1[32];
+        tc::tmem_ld_32x32b_x32(lane_base + 32 * c, g0);
+        tc::tmem_ld_32x32b_x32(lane_base + 64 + 32 * c, g1);
+        load_y(c, y0);
+        load_y(c + 2, y1);
+        tc::tmem_ld_wait();
+        if (live) {
+          uint32_t lo_[16], hi_[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float o_lo[2], o_hi[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const float d0 = r * (__uint_as_float(g0[i + e]) * a.scale - y0[i + e] * m);
+              const float d1 = r * (__uint_as_float(g1[i + e]) * a.scale - y1[i + e] * m);
+              const float2 tt = cs[32 * c + i + e];  // (cos, sin) of pair 32 c + i + e
+              o_lo[e] = d0 * tt.x + d1 * tt.y;
+              o_hi[e] = d1 * tt.x - d0 * tt.y;
+            }
+            lo_[i / 2] = pack_bf16x2(o_lo[0], o_lo[1]);
+            hi_[i / 2] = pack_bf16x2(o_hi[0], o_hi[1]);
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            reinterpret_cast<uint4*>(dst + 32 * c)[u] =
+                make_uint4(lo_[4 * u], lo_[4 * u + 1], lo_[4 * u + 2], lo_[4 * u + 3]);
+            reinterpret_cast<uint4*>(dst + 64 + 32 * c)[u] =
+                make_uint4(hi_[4 * u], hi_[4 * u + 1], hi_[4 * u + 2], hi_[4 * u + 3]);
+          }
+        }
+      }
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 128);
+  }
+}
+
+}  // namespace
+
+namespace {
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = exp2_poly(x[i]);
+}
 }  // namespace
 
 // Query-key pairs a causal window keeps: sum over t of min(t, window) + 1
@@ -755,6 +1510,8 @@ nc_status attention_fwd_ex(const void* q, int64_t ldq, const void* k, const void
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem));
     NC_CUDA_TRY(cudaFuncSetAttribute(attn_fwd_tc_kernel<true>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem));
+    NC_CUDA_TRY(cudaFuncSetAttribute(attn_fwd_pp_kernel,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kPPSmem));
     return NC_OK;
   }));
   CUtensorMap mq, mk, mv;
@@ -778,11 +1535,13 @@ nc_status attention_fwd_ex(const void* q, int64_t ldq, const void* k, const void
   a.status = status;
   const double flops = 4.0 * B * H * HD * causal_pairs(T, a.window);
   Probe probe(prof, s, "attn_fwd", flops, 0.0);
-  dim3 grid(a.nqb, H, B);
-  if (a.group > 1 || a.window >= 0)
+  if (a.group > 1 || a.window >= 0) {
+    dim3 grid(a.nqb, H, B);
     attn_fwd_tc_kernel<true><<<grid, kThreads, kSmem, s>>>(mq, mk, mv, a);
-  else
-    attn_fwd_tc_kernel<false><<<grid, kThreads, kSmem, s>>>(mq, mk, mv, a);
+  } else {
+    dim3 grid((a.nqb + 1) / 2, H, B);  // two query tiles per CTA
+    attn_fwd_pp_kernel<<<grid, kPPThreads, kPPSmem, s>>>(mq, mk, mv, a);
+  }
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }
@@ -797,28 +1556,46 @@ nc_status attention_fwd(const void* q, const void* k, const void* v, int64_t ld,
 nc_status attention_bwd_tc_ex(const void* q, int64_t ldq, const void* k, const void* v, int64_t ldkv,
                               const void* dout, int64_t ldo, const float* lse, const float* delta,
                               float* dq, void* dk, void* dv, int64_t ldg, int B, int T, int H,
-                              int Hkv, int window, int* status, cudaStream_t s, Profiler* prof) {
+                              int Hkv, int window, const float2* rope_tab, const float* rstd_k,
+                              void* ds, int64_t ld_ds, int* status, cudaStream_t s,
+                              Profiler* prof) {
   static DeviceOnce attr;
   NC_TRY(once_per_device(attr, []() -> nc_status {
-    NC_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc_kernel<false>,
+    NC_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc_kernel<false, false>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdSmem));
-    NC_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc_kernel<true>,
+    NC_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc_kernel<true, false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdSmem));
+    NC_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc_kernel<false, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdSmem));
+    NC_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc_kernel<true, true>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdSmem));
     return NC_OK;
   }));
+  const bool sds = ds != nullptr;
   if (Hkv < 1 || H % Hkv) return fail(NC_ERR_INVALID_ARG, "attention_bwd: H must be a multiple of Hkv");
   if (ldq % 8 || ldkv % 8 || ldo % 8 || ldg % 8 ||
       ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
         reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(dout) |
         reinterpret_cast<uintptr_t>(dk) | reinterpret_cast<uintptr_t>(dv)) & 15))
     return fail(NC_ERR_INVALID_ARG, "attention_bwd: rows must be 16-byte aligned");
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdq;
   const uint64_t qcols = (uint64_t)H * HD, kvcols = (uint64_t)Hkv * HD;
   if (!make_tmap_bf16_3d(&mq, q, qcols, T, B, ldq, (int64_t)T * ldq, BQB) ||
       !make_tmap_bf16_3d(&mk, k, kvcols, T, B, ldkv, (int64_t)T * ldkv, BKV) ||
       !make_tmap_bf16_3d(&mv, v, kvcols, T, B, ldkv, (int64_t)T * ldkv, BKV) ||
       !make_tmap_bf16_3d(&mdo, dout, qcols, T, B, ldo, (int64_t)T * ldo, BQB))
     return fail(NC_ERR_INVALID_ARG, "attention_bwd: cuTensorMapEncodeTiled rejected an operand");
+  if (sds) {
+    // dS^T (bf16 [B * H][T keys][T queries], row stride ld_ds): 64 x 128 boxes.
+    if (ld_ds < T || ld_ds % 8 || (reinterpret_cast<uintptr_t>(ds) & 15) ||
+        !make_tmap_bf16_3d(&mdq, ds, T, T, (uint64_t)B * H, ld_ds, (int64_t)T * ld_ds, BKV))
+      return fail(NC_ERR_INVALID_ARG, "attention_bwd: dS buffer rejected");
+  } else {
+    // dq (fp32, dense [B, T, H * 128]): 32 x 32 boxes, 128-byte swizzle.
+    if ((reinterpret_cast<uintptr_t>(dq) & 15) ||
+        !make_tmap_3d(&mdq, dq, true, qcols, T, B, (int64_t)qcols, (int64_t)T * qcols, 32, 32, 128))
+      return fail(NC_ERR_INVALID_ARG, "attention_bwd: dq rejected (16-byte aligned fp32)");
+  }
   BwdArgs a;
   a.T = T;
   a.H = H;
@@ -835,13 +1612,23 @@ nc_status attention_bwd_tc_ex(const void* q, int64_t ldq, const void* k, const v
   a.dv = static_cast<__nv_bfloat16*>(dv);
   a.ldg = ldg;
   a.status = status;
-  const double flops = 10.0 * B * H * HD * causal_pairs(T, a.window);
+  a.rope_tab = rope_tab;
+  a.rstd_k = rstd_k;
+  a.Hkv = Hkv;
+  // Five products per (query, key) pair, or four when dQ is left to the
+  // query-side kernel.
+  const double flops = (sds ? 8.0 : 10.0) * B * H * HD * causal_pairs(T, a.window);
   Probe probe(prof, s, "attn_bwd", flops, 0.0);
   dim3 grid(a.nkb, Hkv, B);  // one CTA per key tile and KV head; it loops over the group
-  if (a.group > 1 || a.window >= 0)
-    attn_bwd_tc_kernel<true><<<grid, kBwdThreads, kBwdSmem, s>>>(mq, mk, mv, mdo, a);
+  const bool gw = a.group > 1 || a.window >= 0;
+  if (gw && sds)
+    attn_bwd_tc_kernel<true, true><<<grid, kBwdThreads, kBwdSmem, s>>>(mq, mk, mv, mdo, mdq, a);
+  else if (gw)
+    attn_bwd_tc_kernel<true, false><<<grid, kBwdThreads, kBwdSmem, s>>>(mq, mk, mv, mdo, mdq, a);
+  else if (sds)
+    attn_bwd_tc_kernel<false, true><<<grid, kBwdThreads, kBwdSmem, s>>>(mq, mk, mv, mdo, mdq, a);
   else
-    attn_bwd_tc_kernel<false><<<grid, kBwdThreads, kBwdSmem, s>>>(mq, mk, mv, mdo, a);
+    attn_bwd_tc_kernel<false, false><<<grid, kBwdThreads, kBwdSmem, s>>>(mq, mk, mv, mdo, mdq, a);
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }
@@ -851,7 +1638,64 @@ nc_status attention_bwd_tc(const void* q, const void* k, const void* v, int64_t 
                            float* dq, void* dk, void* dv, int64_t ldg, int B, int T, int H,
                            int* status, cudaStream_t s, Profiler* prof) {
   return attention_bwd_tc_ex(q, ld, k, v, ld, dout, ldo, lse, delta, dq, dk, dv, ldg, B, T, H, H, -1,
-                             status, s, prof);
+                             nullptr, nullptr, nullptr, 0, status, s, prof);
+}
+
+nc_status attention_dq_ex(const void* ds, int64_t ld_ds, const void* k, int64_t ldkv, int B, int T,
+                          int H, int Hkv, int window, const void* yhat, int64_t ldy,
+                          const float* rstd_q, const float2* rope_tab, void* out, int64_t ldo,
+                          int* status, cudaStream_t s, Profiler* prof) {
+  static DeviceOnce attr;
+  NC_TRY(once_per_device(attr, []() -> nc_status {
+    NC_CUDA_TRY(cudaFuncSetAttribute(attn_dq_kernel<false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmem));
+    NC_CUDA_TRY(cudaFuncSetAttribute(attn_dq_kernel<true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmem));
+    return NC_OK;
+  }));
+  if (B < 1 || T < 1 || H < 1 || Hkv < 1 || H % Hkv || !ds || !k || !yhat || !rstd_q ||
+      !rope_tab || !out)
+    return fail(NC_ERR_INVALID_ARG, "attention_dq: bad arguments");
+  if (ldkv % 8 || ldy % 8 || ldo % 8 || ld_ds < T || ld_ds % 8 ||
+      ((reinterpret_cast<uintptr_t>(ds) | reinterpret_cast<uintptr_t>(k) |
+        reinterpret_cast<uintptr_t>(yhat) | reinterpret_cast<uintptr_t>(out)) & 15))
+    return fail(NC_ERR_INVALID_ARG, "attention_dq: rows must be 16-byte aligned");
+  CUtensorMap mds, mk;
+  if (!make_tmap_bf16_3d(&mds, ds, T, T, (uint64_t)B * H, ld_ds, (int64_t)T * ld_ds, BKV) ||
+      !make_tmap_bf16_3d(&mk, k, (uint64_t)Hkv * HD, T, B, ldkv, (int64_t)T * ldkv, BKV))
+    return fail(NC_ERR_INVALID_ARG, "attention_dq: cuTensorMapEncodeTiled rejected an operand");
+  DqArgs a;
+  a.T = T;
+  a.H = H;
+  a.nqb = (T + BQB - 1) / BQB;
+  a.group = H / Hkv;
+  a.window = (window < 0 || window >= T - 1) ? -1 : window;
+  a.scale = (float)(1.0 / std::sqrt((double)HD));
+  a.yhat = static_cast<const __nv_bfloat16*>(yhat);
+  a.ldy = ldy;
+  a.rstd_q = rstd_q;
+  a.rope_tab = rope_tab;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.ldo = ldo;
+  a.status = status;
+  const double flops = 2.0 * B * H * HD * causal_pairs(T, a.window);
+  Probe probe(prof, s, "attn_bwd_dq", flops, 0.0);
+  dim3 grid(a.nqb, H, B);
+  if (a.group > 1 || a.window >= 0)
+    attn_dq_kernel<true><<<grid, kDqThreads, kDqSmem, s>>>(mds, mk, a);
+  else
+    attn_dq_kernel<false><<<grid, kDqThreads, kDqSmem, s>>>(mds, mk, a);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
 }
 
 }  // namespace nc
+
+extern "C" nc_status nc_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
+  using namespace nc;
+  if (n < 0 || (n > 0 && (!x || !y))) return fail(NC_ERR_INVALID_ARG, "exp2_poly: bad arguments");
+  if (n == 0) return NC_OK;
+  exp2_poly_kernel<<<(unsigned)((n + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}

@@ -1,5 +1,5 @@
 // elementwise.cu -- the memory-bound kernels of the step: embedding gather
-// and scatter-add, RMSNorm forward/backward, RoPE + QK-norm forward/backward,
+// and scatter-add, RMSNorm forward/backward, the RoPE table,
 // fused softmax cross-entropy (loss and logits gradient in one pass),
 // parameter init, bf16 refresh, the Muon momentum / normalise / apply
 // passes and the AdamW step of the embedding and lm_head.  One warp per row where a row reduction is needed (warp-shuffle
@@ -39,10 +39,10 @@ __global__ void embed_scatter_kernel(const int32_t* __restrict__ tok, int64_t n,
   float* dst = dE + (int64_t)id * d;
   for (int i = lane; i < d / 4; i += 32) {
     const float4 g = src[i];
-    atomicAdd(dst + 4 * i + 0, g.x);
-    atomicAdd(dst + 4 * i + 1, g.y);
-    atomicAdd(dst + 4 * i + 2, g.z);
-    atomicAdd(dst + 4 * i + 3, g.w);
+    // One 16-byte vector reduction per float4 (rows are 16-byte aligned).
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 4 * i), "f"(g.x),
+                 "f"(g.y), "f"(g.z), "f"(g.w)
+                 : "memory");
   }
 }
 
@@ -72,45 +72,43 @@ __global__ void rmsnorm_fwd_kernel(const float* __restrict__ x, int64_t rows, in
   if (lane == 0 && rstd) rstd[r] = rs;
 }
 
-// dx = dres + r * (dh - y * mean(dh * y)), y = x * r; fp32 out and a bf16 copy.
-__global__ void rmsnorm_bwd_kernel(const __nv_bfloat16* __restrict__ dh, const float* __restrict__ x,
-                                   const float* __restrict__ rstd, const float* __restrict__ dres,
-                                   int64_t rows, int d, float* __restrict__ dx,
-                                   __nv_bfloat16* __restrict__ dx_bf16) {
+// dx = dres + r * (dh - y * mean(dh * y)) with y = x * r the norm's output,
+// read as the bf16 activation the forward saved (the operand the next GEMM
+// consumed); fp32 out and a bf16 copy.  One warp per row, two passes over
+// dh and y (the second from L1/L2), 16-byte fp32 and 8-byte bf16 accesses.
+__global__ void __launch_bounds__(256) rmsnorm_bwd_kernel(
+    const __nv_bfloat16* __restrict__ dh, const __nv_bfloat16* __restrict__ y,
+    const float* __restrict__ rstd, const float* __restrict__ dres, int64_t rows, int d,
+    float* __restrict__ dx, __nv_bfloat16* __restrict__ dx_bf16) {
   const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (r >= rows) return;
-  const float rs = rstd[r];
-  const float4* xr = reinterpret_cast<const float4*>(x + r * d);
+  const int n4 = d / 4;
   const uint2* gr = reinterpret_cast<const uint2*>(dh + r * d);
+  const uint2* yr = reinterpret_cast<const uint2*>(y + r * d);
   float dot = 0.f;
-  for (int i = lane; i < d / 4; i += 32) {
-    const float4 v = xr[i];
-    const uint2 u = gr[i];
-    const float2 g0 = unpack_bf16x2(u.x), g1 = unpack_bf16x2(u.y);
-    dot += g0.x * v.x + g0.y * v.y + g1.x * v.z + g1.y * v.w;
+  for (int i = lane; i < n4; i += 32) {
+    const uint2 g = gr[i], v = yr[i];
+    const float2 g0 = unpack_bf16x2(g.x), g1 = unpack_bf16x2(g.y);
+    const float2 y0 = unpack_bf16x2(v.x), y1 = unpack_bf16x2(v.y);
+    dot += g0.x * y0.x + g0.y * y0.y + g1.x * y1.x + g1.y * y1.y;
   }
-  dot = warp_sum(dot) * rs;
-  const float m = dot / d;
+  const float m = warp_sum(dot) / d;
+  const float rs = rstd[r];
   const float4* rr = dres ? reinterpret_cast<const float4*>(dres + r * d) : nullptr;
   float4* o = reinterpret_cast<float4*>(dx + r * d);
   uint2* ob = dx_bf16 ? reinterpret_cast<uint2*>(dx_bf16 + r * d) : nullptr;
-  for (int i = lane; i < d / 4; i += 32) {
-    const float4 v = xr[i];
-    const uint2 u = gr[i];
-    const float2 g0 = unpack_bf16x2(u.x), g1 = unpack_bf16x2(u.y);
+  for (int i = lane; i < n4; i += 32) {
+    const uint2 g = gr[i], v = yr[i];
+    const float2 g0 = unpack_bf16x2(g.x), g1 = unpack_bf16x2(g.y);
+    const float2 y0 = unpack_bf16x2(v.x), y1 = unpack_bf16x2(v.y);
     float4 res = rr ? rr[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-    res.x += rs * (g0.x - v.x * rs * m);
-    res.y += rs * (g0.y - v.y * rs * m);
-    res.z += rs * (g1.x - v.z * rs * m);
-    res.w += rs * (g1.y - v.w * rs * m);
+    res.x += rs * (g0.x - y0.x * m);
+    res.y += rs * (g0.y - y0.y * m);
+    res.z += rs * (g1.x - y1.x * m);
+    res.w += rs * (g1.y - y1.y * m);
     o[i] = res;
-    if (ob) {
-      uint2 w;
-      w.x = pack_bf16x2(res.x, res.y);
-      w.y = pack_bf16x2(res.z, res.w);
-      ob[i] = w;
-    }
+    if (ob) ob[i] = make_uint2(pack_bf16x2(res.x, res.y), pack_bf16x2(res.z, res.w));
   }
 }
 
@@ -123,60 +121,6 @@ __global__ void rope_table_kernel(float2* tab, int T, int hd) {
   const int pos = (int)(i / half), j = (int)(i % half);
   const double th = (double)pos * pow(10000.0, -2.0 * j / hd);
   tab[i] = make_float2((float)cos(th), (float)sin(th));
-}
-
-// Backward of RoPE + QK-norm (the forward is fused into the q|k|v GEMM
-// epilogue) for one slice: g = dL/dyhat (f32 dense [n, H*128] for
-// q, or bf16 with stride ldg for k), yhat the saved normalised output.
-//   dr = r * (g - yhat * mean(g * yhat));   dx = R(-theta) dr.
-// Writes bf16 into out (stride ld_out); may run in place on the k slice.
-__global__ void rope_qknorm_bwd_kernel(const float* __restrict__ gf, const __nv_bfloat16* gb,
-                                       int64_t ldg, const __nv_bfloat16* __restrict__ yhat,
-                                       int64_t ldy, const float* __restrict__ rstd, int64_t n,
-                                       int T, int H, const float2* __restrict__ tab,
-                                       __nv_bfloat16* out, int64_t ld_out) {
-  const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (w >= n * H) return;
-  const int h = (int)(w % H);
-  const int64_t tok = w / H;
-  const int pos = (int)(tok % T);
-  const int half = lane >> 4, j = lane & 15;
-  const int col = h * 128 + half * 64 + 4 * j;
-  float g[4];
-  if (gf) {
-    const float4 v = *reinterpret_cast<const float4*>(gf + tok * ((int64_t)H * 128) + col);
-    g[0] = v.x; g[1] = v.y; g[2] = v.z; g[3] = v.w;
-  } else {
-    const uint2 v = *reinterpret_cast<const uint2*>(gb + tok * ldg + col);
-    const float2 a0 = unpack_bf16x2(v.x), a1 = unpack_bf16x2(v.y);
-    g[0] = a0.x; g[1] = a0.y; g[2] = a1.x; g[3] = a1.y;
-  }
-  const uint2 yv = *reinterpret_cast<const uint2*>(yhat + tok * ldy + col);
-  const float2 y01 = unpack_bf16x2(yv.x), y23 = unpack_bf16x2(yv.y);
-  const float y[4] = {y01.x, y01.y, y23.x, y23.y};
-  float dot = g[0] * y[0] + g[1] * y[1] + g[2] * y[2] + g[3] * y[3];
-  dot = warp_sum(dot);
-  const float rs = rstd[tok * H + h];
-  const float m = dot / 128.f;
-  float dr[4], pr[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) dr[e] = rs * (g[e] - y[e] * m);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) pr[e] = __shfl_xor_sync(0xffffffffu, dr[e], 16);
-  const float4* t4 = reinterpret_cast<const float4*>(tab + (int64_t)pos * 64 + 4 * j);
-  const float4 cs01 = t4[0], cs23 = t4[1];
-  const float c[4] = {cs01.x, cs01.z, cs23.x, cs23.z};
-  const float sn[4] = {cs01.y, cs01.w, cs23.y, cs23.w};
-  float o[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e)
-    // first half: dr_i c + dr_{i+64} s;  second half: -dr_i s + dr_{i+64} c
-    o[e] = half == 0 ? dr[e] * c[e] + pr[e] * sn[e] : dr[e] * c[e] - pr[e] * sn[e];
-  uint2 ov;
-  ov.x = pack_bf16x2(o[0], o[1]);
-  ov.y = pack_bf16x2(o[2], o[3]);
-  *reinterpret_cast<uint2*>(out + tok * ld_out + col) = ov;
 }
 
 // ------------------------------------------------------------------ cross-entropy
@@ -375,61 +319,119 @@ __global__ void muon_momentum_kernel(float* __restrict__ M, const float* __restr
   }
 }
 
-// X = bf16(M / (||M|| + eps)), optionally transposed, 32 x 32 tiles.
-// src matrix (rows x cols, fp32) of layer blockIdx.z at src + z*src_stride;
-// dst (bf16) at dst + z*dst_stride; norm index = z*6 + j.
-__global__ void muon_prep_kernel(const float* __restrict__ src, int64_t src_stride, int rows,
-                                 int cols, int transpose, __nv_bfloat16* __restrict__ dst,
-                                 int64_t dst_stride, const float* __restrict__ sumsq, int j,
-                                 float eps) {
-  __shared__ float tile[32][33];
+// X = bf16(M / (||M|| + eps)) for matrix j of layer blockIdx.y (src at
+// src + y*src_stride, dst at dst + y*dst_stride, norm index y*6 + j), same
+// orientation: 16-byte fp32 loads, 8-byte bf16 stores, grid-stride.
+__global__ void muon_prep_kernel(const float* __restrict__ src, int64_t src_stride, int64_t n4,
+                                 __nv_bfloat16* __restrict__ dst, int64_t dst_stride,
+                                 const float* __restrict__ sumsq, int j, float eps) {
+  const int z = blockIdx.y;
+  const float inv = 1.f / (sqrtf(sumsq[z * 6 + j]) + eps);
+  const float4* s4 = reinterpret_cast<const float4*>(src + z * src_stride);
+  uint2* d2 = reinterpret_cast<uint2*>(dst + z * dst_stride);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 v = s4[i];
+    d2[i] = make_uint2(pack_bf16x2(v.x * inv, v.y * inv), pack_bf16x2(v.z * inv, v.w * inv));
+  }
+}
+
+// The same, transposed (dst is cols x rows), through 64 x 64 shared tiles:
+// each thread reads 16-byte rows of the fp32 source and writes 8-byte runs
+// of the bf16 destination (256 threads, 4 passes of 16 rows each way).
+__global__ void __launch_bounds__(256) muon_prep_t_kernel(
+    const float* __restrict__ src, int64_t src_stride, int rows, int cols,
+    __nv_bfloat16* __restrict__ dst, int64_t dst_stride, const float* __restrict__ sumsq, int j,
+    float eps) {
+  __shared__ float tile[64][65];
   const int z = blockIdx.z;
   const float inv = 1.f / (sqrtf(sumsq[z * 6 + j]) + eps);
   const float* s = src + z * src_stride;
   __nv_bfloat16* dd = dst + z * dst_stride;
-  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int r = r0 + i, c = c0 + threadIdx.x;
-    tile[i][threadIdx.x] = (r < rows && c < cols) ? s[(int64_t)r * cols + c] * inv : 0.f;
+  const int r0 = blockIdx.y * 64, c0 = blockIdx.x * 64;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;  // 16 x 16
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const int i = ty + 16 * p, r = r0 + i, c = c0 + 4 * tx;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < rows && c < cols) v = *reinterpret_cast<const float4*>(s + (int64_t)r * cols + c);
+    tile[i][4 * tx] = v.x;
+    tile[i][4 * tx + 1] = v.y;
+    tile[i][4 * tx + 2] = v.z;
+    tile[i][4 * tx + 3] = v.w;
   }
   __syncthreads();
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    if (!transpose) {
-      const int r = r0 + i, c = c0 + threadIdx.x;
-      if (r < rows && c < cols) dd[(int64_t)r * cols + c] = f2bf(tile[i][threadIdx.x]);
-    } else {
-      const int r = c0 + i, c = r0 + threadIdx.x;  // dst is cols x rows
-      if (r < cols && c < rows) dd[(int64_t)r * rows + c] = f2bf(tile[threadIdx.x][i]);
-    }
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const int i = ty + 16 * p;  // destination row c0 + i, columns r0 + 4 tx ..
+    const int r = c0 + i, c = r0 + 4 * tx;
+    if (r < cols && c < rows)
+      *reinterpret_cast<uint2*>(dd + (int64_t)r * rows + c) =
+          make_uint2(pack_bf16x2(tile[4 * tx][i] * inv, tile[4 * tx + 1][i] * inv),
+                     pack_bf16x2(tile[4 * tx + 2][i] * inv, tile[4 * tx + 3][i] * inv));
   }
 }
 
-// W <- W - lr * X^(T), bf16 copy refreshed.  W (rows x cols) per layer z.
+// W <- W - lr * X and its bf16 copy refreshed, same orientation, per layer
+// blockIdx.y: 16-byte fp32, 8-byte bf16 accesses, grid-stride.
 __global__ void muon_apply_kernel(float* __restrict__ W, __nv_bfloat16* __restrict__ Wb,
-                                  int64_t w_stride, int rows, int cols, int transpose,
-                                  const __nv_bfloat16* __restrict__ X, int64_t x_stride,
-                                  float lr) {
-  __shared__ float tile[32][33];
+                                  int64_t w_stride, int64_t n4, const __nv_bfloat16* __restrict__ X,
+                                  int64_t x_stride, float lr) {
+  const int z = blockIdx.y;
+  float4* w4 = reinterpret_cast<float4*>(W + z * w_stride);
+  uint2* wb2 = reinterpret_cast<uint2*>(Wb + z * w_stride);
+  const uint2* x2 = reinterpret_cast<const uint2*>(X + z * x_stride);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float4 w = w4[i];
+    const uint2 x = x2[i];
+    const float2 x01 = unpack_bf16x2(x.x), x23 = unpack_bf16x2(x.y);
+    w.x -= lr * x01.x;
+    w.y -= lr * x01.y;
+    w.z -= lr * x23.x;
+    w.w -= lr * x23.y;
+    w4[i] = w;
+    wb2[i] = make_uint2(pack_bf16x2(w.x, w.y), pack_bf16x2(w.z, w.w));
+  }
+}
+
+// The same with X stored transposed (cols x rows): X staged through a 64 x 64
+// shared tile, W (rows x cols) updated in 16-byte runs.
+__global__ void __launch_bounds__(256) muon_apply_t_kernel(
+    float* __restrict__ W, __nv_bfloat16* __restrict__ Wb, int64_t w_stride, int rows, int cols,
+    const __nv_bfloat16* __restrict__ X, int64_t x_stride, float lr) {
+  __shared__ float tile[64][65];
   const int z = blockIdx.z;
   float* w = W + z * w_stride;
   __nv_bfloat16* wb = Wb + z * w_stride;
   const __nv_bfloat16* x = X + z * x_stride;
-  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
-  if (transpose) {
-    // X is cols x rows: stage X[c0.., r0..] then read it transposed.
-    for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-      const int xr = c0 + i, xc = r0 + threadIdx.x;
-      tile[i][threadIdx.x] = (xr < cols && xc < rows) ? bf2f(x[(int64_t)xr * rows + xc]) : 0.f;
-    }
-    __syncthreads();
+  const int r0 = blockIdx.y * 64, c0 = blockIdx.x * 64;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  // X rows c0 .. c0 + 63 (W's columns), X columns r0 .. r0 + 63 (W's rows).
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const int i = ty + 16 * p, xr = c0 + i, xc = r0 + 4 * tx;
+    uint2 u = make_uint2(0u, 0u);
+    if (xr < cols && xc < rows) u = *reinterpret_cast<const uint2*>(x + (int64_t)xr * rows + xc);
+    const float2 a0 = unpack_bf16x2(u.x), a1 = unpack_bf16x2(u.y);
+    tile[i][4 * tx] = a0.x;
+    tile[i][4 * tx + 1] = a0.y;
+    tile[i][4 * tx + 2] = a1.x;
+    tile[i][4 * tx + 3] = a1.y;
   }
-  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
-    const int r = r0 + i, c = c0 + threadIdx.x;
+  __syncthreads();
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const int i = ty + 16 * p, r = r0 + i, c = c0 + 4 * tx;
     if (r < rows && c < cols) {
-      const float u = transpose ? tile[threadIdx.x][i] : bf2f(x[(int64_t)r * cols + c]);
-      const float nw = w[(int64_t)r * cols + c] - lr * u;
-      w[(int64_t)r * cols + c] = nw;
-      wb[(int64_t)r * cols + c] = f2bf(nw);
+      float4 v = *reinterpret_cast<float4*>(w + (int64_t)r * cols + c);
+      v.x -= lr * tile[4 * tx][i];
+      v.y -= lr * tile[4 * tx + 1][i];
+      v.z -= lr * tile[4 * tx + 2][i];
+      v.w -= lr * tile[4 * tx + 3][i];
+      *reinterpret_cast<float4*>(w + (int64_t)r * cols + c) = v;
+      *reinterpret_cast<uint2*>(wb + (int64_t)r * cols + c) =
+          make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
     }
   }
 }
@@ -515,32 +517,21 @@ nc_status rmsnorm_fwd(const float* x, int64_t rows, int d, void* y, float* rstd,
   return NC_OK;
 }
 
-nc_status rmsnorm_bwd(const void* dh, const float* x, const float* rstd, const float* dres,
+nc_status rmsnorm_bwd(const void* dh, const void* y, const float* rstd, const float* dres,
                       int64_t rows, int d, float* dx, void* dx_bf16, cudaStream_t s,
                       Profiler* prof) {
+  if (d % 4) return fail(NC_ERR_UNSUPPORTED, "rmsnorm_bwd: width must be a multiple of 4");
   Probe probe(prof, s, "rmsnorm_bwd", 0.0,
-              rows * ((2.0 + 4.0 + (dres ? 4.0 : 0.0) + 4.0 + (dx_bf16 ? 2.0 : 0.0)) * d + 4.0));
+              rows * ((2.0 + 2.0 + (dres ? 4.0 : 0.0) + 4.0 + (dx_bf16 ? 2.0 : 0.0)) * d + 4.0));
   rmsnorm_bwd_kernel<<<blocks_for(rows * 32, 256), 256, 0, s>>>(
-      (const __nv_bfloat16*)dh, x, rstd, dres, rows, d, dx, (__nv_bfloat16*)dx_bf16);
+      (const __nv_bfloat16*)dh, (const __nv_bfloat16*)y, rstd, dres, rows, d, dx,
+      (__nv_bfloat16*)dx_bf16);
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }
 
 nc_status rope_table(float2* tab, int T, int hd, cudaStream_t s) {
   rope_table_kernel<<<blocks_for((int64_t)T * hd / 2, 256), 256, 0, s>>>(tab, T, hd);
-  NC_CUDA_TRY(cudaGetLastError());
-  return NC_OK;
-}
-
-nc_status rope_qknorm_bwd(const float* gf, const void* gb, int64_t ldg, const void* yhat,
-                          int64_t ldy, const float* rstd, int64_t n, int T, int H, int hd,
-                          const float2* tab, void* out, int64_t ld_out, cudaStream_t s,
-                          Profiler* prof) {
-  Probe probe(prof, s, "rope_qknorm_bwd", 0.0, n * H * (hd * ((gf ? 4.0 : 2.0) + 2.0 + 2.0) + 4.0));
-  if (hd != 128) return fail(NC_ERR_UNSUPPORTED, "rope_qknorm: head_dim must be 128");
-  rope_qknorm_bwd_kernel<<<blocks_for(n * H * 32, 256), 256, 0, s>>>(
-      gf, (const __nv_bfloat16*)gb, ldg, (const __nv_bfloat16*)yhat, ldy, rstd, n, T, H, tab,
-      (__nv_bfloat16*)out, ld_out);
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }
@@ -588,10 +579,19 @@ nc_status muon_momentum(float* M, const float* G, int L, int d, int dkv, float m
 nc_status muon_prep(const float* src, int64_t src_stride, int rows, int cols, int transpose,
                     void* dst, int64_t dst_stride, const float* sumsq, int j, int L,
                     cudaStream_t s, Profiler* prof) {
+  if (rows % 4 || cols % 4 || src_stride % 4 || dst_stride % 4)
+    return fail(NC_ERR_INVALID_ARG, "muon_prep: dims and strides must be multiples of 4");
   Probe probe(prof, s, "muon_prep", 0.0, (double)L * rows * cols * 6.0);
-  dim3 grid((cols + 31) / 32, (rows + 31) / 32, L);
-  muon_prep_kernel<<<grid, dim3(32, 8), 0, s>>>(src, src_stride, rows, cols, transpose,
-                                                (__nv_bfloat16*)dst, dst_stride, sumsq, j, 1e-7f);
+  if (transpose) {
+    dim3 grid((cols + 63) / 64, (rows + 63) / 64, L);
+    muon_prep_t_kernel<<<grid, 256, 0, s>>>(src, src_stride, rows, cols, (__nv_bfloat16*)dst,
+                                            dst_stride, sumsq, j, 1e-7f);
+  } else {
+    const int64_t n4 = (int64_t)rows * cols / 4;
+    dim3 grid((unsigned)std::min<int64_t>(blocks_for(n4, 256), 4 * num_sms() / std::max(L, 1) + 1), L);
+    muon_prep_kernel<<<grid, 256, 0, s>>>(src, src_stride, n4, (__nv_bfloat16*)dst, dst_stride,
+                                          sumsq, j, 1e-7f);
+  }
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }
@@ -599,10 +599,19 @@ nc_status muon_prep(const float* src, int64_t src_stride, int rows, int cols, in
 nc_status muon_apply(float* W, void* Wb, int64_t w_stride, int rows, int cols, int transpose,
                      const void* X, int64_t x_stride, float lr, int L, cudaStream_t s,
                      Profiler* prof) {
+  if (rows % 4 || cols % 4 || w_stride % 4 || x_stride % 4)
+    return fail(NC_ERR_INVALID_ARG, "muon_apply: dims and strides must be multiples of 4");
   Probe probe(prof, s, "muon_apply", 0.0, (double)L * rows * cols * 12.0);
-  dim3 grid((cols + 31) / 32, (rows + 31) / 32, L);
-  muon_apply_kernel<<<grid, dim3(32, 8), 0, s>>>(W, (__nv_bfloat16*)Wb, w_stride, rows, cols,
-                                                 transpose, (const __nv_bfloat16*)X, x_stride, lr);
+  if (transpose) {
+    dim3 grid((cols + 63) / 64, (rows + 63) / 64, L);
+    muon_apply_t_kernel<<<grid, 256, 0, s>>>(W, (__nv_bfloat16*)Wb, w_stride, rows, cols,
+                                             (const __nv_bfloat16*)X, x_stride, lr);
+  } else {
+    const int64_t n4 = (int64_t)rows * cols / 4;
+    dim3 grid((unsigned)std::min<int64_t>(blocks_for(n4, 256), 4 * num_sms() / std::max(L, 1) + 1), L);
+    muon_apply_kernel<<<grid, 256, 0, s>>>(W, (__nv_bfloat16*)Wb, w_stride, n4,
+                                           (const __nv_bfloat16*)X, x_stride, lr);
+  }
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }

@@ -52,6 +52,12 @@ nc_status once_per_device(DeviceOnce& o, F&& f) {
   return st;
 }
 
+// Device address of the library's op status word on the current device (a
+// file-scope __device__ int, looked up once per device): the single-kernel
+// entry points (nc_op_*) hand it to their kernels as the status word, and
+// nc_op_sync reads and clears it.
+nc_status op_status_word(int** out);
+
 // Per-kernel-class timing (profile.cpp).  Every launch site wraps its launch
 // in a Probe; with profiling off it only counts the launch.
 struct Profiler;

@@ -49,14 +49,42 @@ nc_status attention_bwd_tc(const void* q, const void* k, const void* v, int64_t 
 nc_status attention_fwd_ex(const void* q, int64_t ldq, const void* k, const void* v, int64_t ldkv,
                            void* o, int64_t ldo, float* lse, int B, int T, int H, int Hkv,
                            int window, int* status, cudaStream_t s, Profiler* prof);
+// rope_tab / rstd_k non-null: dk receives the gradient of the k slice before
+// its RoPE + QK-norm (the saved k being their output), i.e. the k-side
+// backward of the q|k|v projection's epilogue is applied in the attention
+// backward's dK epilogue; null: dk is the gradient of the k operand.
 nc_status attention_bwd_ex(const void* q, int64_t ldq, const void* k, const void* v, int64_t ldkv,
                            const void* o, const void* dout, int64_t ldo, const float* lse,
                            float* dq, void* dk, void* dv, int64_t ldg, float* delta, int B, int T,
-                           int H, int Hkv, int window, int* status, cudaStream_t s, Profiler* prof);
+                           int H, int Hkv, int window, const float2* rope_tab, const float* rstd_k,
+                           int* status, cudaStream_t s, Profiler* prof);
+// ds non-null: the kernel stores every dS^T tile (bf16 [B*H][T keys][T
+// queries], row stride ld_ds, a multiple of 8 >= T) instead of computing dQ,
+// and dq is not touched; attention_dq_ex then contracts it with K.
 nc_status attention_bwd_tc_ex(const void* q, int64_t ldq, const void* k, const void* v, int64_t ldkv,
                               const void* dout, int64_t ldo, const float* lse, const float* delta,
                               float* dq, void* dk, void* dv, int64_t ldg, int B, int T, int H,
-                              int Hkv, int window, int* status, cudaStream_t s, Profiler* prof);
+                              int Hkv, int window, const float2* rope_tab, const float* rstd_k,
+                              void* ds, int64_t ld_ds, int* status, cudaStream_t s,
+                              Profiler* prof);
+// dQ = dS K / sqrt(128) from the stored dS^T tiles, through the backward of
+// the q-side RoPE + QK-norm (yhat: the saved normalised q, row stride ldy;
+// rstd_q [B*T, H]), written as bf16 rows of stride ldo (the q slice of the
+// q|k|v gradient).
+nc_status attention_dq_ex(const void* ds, int64_t ld_ds, const void* k, int64_t ldkv, int B, int T,
+                          int H, int Hkv, int window, const void* yhat, int64_t ldy,
+                          const float* rstd_q, const float2* rope_tab, void* out, int64_t ldo,
+                          int* status, cudaStream_t s, Profiler* prof);
+// The model's attention backward: the row sums D, the key-side kernel with
+// the k-side RoPE + QK-norm backward in its dK epilogue and dS^T stored to
+// ds, then the query-side kernel with the q-side backward in its epilogue.
+// dq_out, dk, dv: the q, k, v slices of the bf16 q|k|v gradient.
+nc_status attention_bwd_model(const void* q, int64_t ldq, const void* k, const void* v,
+                              int64_t ldkv, const void* o, const void* dout, int64_t ldo,
+                              const float* lse, float* delta, void* ds, int64_t ld_ds,
+                              void* dq_out, void* dk, void* dv, int64_t ldg, int B, int T, int H,
+                              int Hkv, int window, const float2* rope_tab, const float* rstd_q,
+                              const float* rstd_k, int* status, cudaStream_t s, Profiler* prof);
 
 nc_status embed_gather(const int32_t* tok, int64_t n, const float* E, int V, int d, float* x,
                        int* status, cudaStream_t s, Profiler* prof);
@@ -64,14 +92,11 @@ nc_status embed_scatter(const int32_t* tok, int64_t n, const float* dx, int V, i
                         cudaStream_t s, Profiler* prof);
 nc_status rmsnorm_fwd(const float* x, int64_t rows, int d, void* y, float* rstd, cudaStream_t s,
                       Profiler* prof);
-nc_status rmsnorm_bwd(const void* dh, const float* x, const float* rstd, const float* dres,
+// y: the norm's saved bf16 output (x * rstd as the forward stored it).
+nc_status rmsnorm_bwd(const void* dh, const void* y, const float* rstd, const float* dres,
                       int64_t rows, int d, float* dx, void* dx_bf16, cudaStream_t s,
                       Profiler* prof);
 nc_status rope_table(float2* tab, int T, int hd, cudaStream_t s);
-nc_status rope_qknorm_bwd(const float* gf, const void* gb, int64_t ldg, const void* yhat,
-                          int64_t ldy, const float* rstd, int64_t n, int T, int H, int hd,
-                          const float2* tab, void* out, int64_t ld_out, cudaStream_t s,
-                          Profiler* prof);
 nc_status ce_fwd_bwd(void* z, const int32_t* tgt, int64_t n, int V, float* loss_rows,
                      float* loss_out, int* status, cudaStream_t s, Profiler* prof);
 nc_status init_normal(float* out, int64_t n, uint64_t key, float stdv, cudaStream_t s);

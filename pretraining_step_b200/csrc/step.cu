@@ -87,9 +87,10 @@ struct Acts {
   std::vector<float*> x, xmid, r1, r2, rq, rk, lse;
   std::vector<bf16*> h1, h2, qkv, o, a;
   bf16 *hf = nullptr, *logits = nullptr, *dxb = nullptr, *dh = nullptr, *du = nullptr,
-       *dqkv = nullptr;
+       *dqkv = nullptr, *ds = nullptr;
+  int64_t ld_ds = 0;  // row stride of ds: T rounded up to a multiple of 8
   float *rf = nullptr, *loss_rows = nullptr, *loss = nullptr, *dx0 = nullptr, *dx1 = nullptr,
-        *dq = nullptr, *delta = nullptr;
+        *delta = nullptr;
 };
 
 }  // namespace
@@ -248,8 +249,10 @@ nc_status ensure_acts(nc_params* p, int B, int T) {
   total += L * r(4 * N * H);                                 // lse [B,H,T]
   total += 2 * L * r(2 * N * d) + L * r(2 * N * Q) + L * r(2 * N * d) + L * r(2 * N * F);
   total += r(2 * N * d) + r(4 * N) + r(2 * N * V) + r(4 * N) + r(4);  // hf rf logits loss
+  const int64_t ld_ds = (T + 7) & ~int64_t(7);
   total += 2 * r(4 * N * d) + 2 * r(2 * N * d) + r(2 * N * F) + r(2 * N * Q) +
-           r(4 * N * d) + r(4 * N * H);                      // backward scratch
+           r(4 * N * H);                                     // backward scratch
+  total += r(2 * (int64_t)B * H * T * ld_ds);                // attention dS^T tiles
   void* mem = nullptr;
   cudaError_t e = cudaMalloc(&mem, (size_t)total);
   if (e != cudaSuccess) {
@@ -288,8 +291,9 @@ nc_status ensure_acts(nc_params* p, int B, int T) {
   a.dh = ar.take<bf16>(N * d);
   a.du = ar.take<bf16>(N * F);
   a.dqkv = ar.take<bf16>(N * Q);
-  a.dq = ar.take<float>(N * d);
   a.delta = ar.take<float>(N * H);
+  a.ld_ds = ld_ds;
+  a.ds = ar.take<bf16>((int64_t)B * H * T * ld_ds);
   if (ar.used > ar.size) return fail(NC_ERR_CUDA, "activation arena overflow");
   return NC_OK;
 }
@@ -417,7 +421,7 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
                  "gemm_lmhead"));
   float* dx = a.dx0;
   float* dxn = a.dx1;
-  NC_TRY(rmsnorm_bwd(a.dh, a.x[L], a.rf, nullptr, N, (int)d, dx, a.dxb, s, pr));
+  NC_TRY(rmsnorm_bwd(a.dh, a.hf, a.rf, nullptr, N, (int)d, dx, a.dxb, s, pr));
   for (int l = L - 1; l >= 0; --l) {
     const bf16* W = p->blocks_b + l * LS;
     float* G = g->blocks + l * LS;
@@ -426,21 +430,20 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
     NC_TRY(proj_dx(p, a.dxb, N, d, W + o_down, F, a.du, F, NC_EPI_RELU2_BWD, a.a[l], F));
     NC_TRY(proj_dw(p, a.du, F, F, a.h2[l], d, d, N, G + o_up));
     NC_TRY(proj_dx(p, a.du, N, F, W + o_up, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0));
-    NC_TRY(rmsnorm_bwd(a.dh, a.xmid[l], a.r2[l], dx, N, (int)d, dxn, a.dxb, s, pr));
+    NC_TRY(rmsnorm_bwd(a.dh, a.h2[l], a.r2[l], dx, N, (int)d, dxn, a.dxb, s, pr));
     std::swap(dx, dxn);
     // Attention: xmid = x + o wo^T
     NC_TRY(proj_dw(p, a.dxb, d, d, a.o[l], d, d, N, G + o_wo));
     NC_TRY(proj_dx(p, a.dxb, N, d, W + o_wo, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0));
-    NC_TRY(attention_bwd_ex(a.qkv[l], Q, a.qkv[l] + d, a.qkv[l] + d + dkv, Q, a.o[l], a.dh, d,
-                            a.lse[l], a.dq, a.dqkv + d, a.dqkv + d + dkv, Q, a.delta, B, T, H, Hkv,
-                            p->window[l], p->status, s, pr));
-    NC_TRY(rope_qknorm_bwd(a.dq, nullptr, 0, a.qkv[l], Q, a.rq[l], N, T, H, hd, p->rope, a.dqkv,
-                           Q, s, pr));
-    NC_TRY(rope_qknorm_bwd(nullptr, a.dqkv + d, Q, a.qkv[l] + d, Q, a.rk[l], N, T, Hkv, hd,
-                           p->rope, a.dqkv + d, Q, s, pr));
+    // Key side (dK through the k-side RoPE + QK-norm backward, dV, dS^T to
+    // a.ds), then the query side (dQ = dS K through the q-side backward).
+    NC_TRY(attention_bwd_model(a.qkv[l], Q, a.qkv[l] + d, a.qkv[l] + d + dkv, Q, a.o[l], a.dh, d,
+                               a.lse[l], a.delta, a.ds, a.ld_ds, a.dqkv, a.dqkv + d,
+                               a.dqkv + d + dkv, Q, B, T, H, Hkv, p->window[l], p->rope, a.rq[l],
+                               a.rk[l], p->status, s, pr));
     NC_TRY(proj_dw(p, a.dqkv, Q, Q, a.h1[l], d, d, N, G));
     NC_TRY(proj_dx(p, a.dqkv, N, Q, W, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0));
-    NC_TRY(rmsnorm_bwd(a.dh, a.x[l], a.r1[l], dx, N, (int)d, dxn, a.dxb, s, pr));
+    NC_TRY(rmsnorm_bwd(a.dh, a.h1[l], a.r1[l], dx, N, (int)d, dxn, a.dxb, s, pr));
     std::swap(dx, dxn);
   }
   NC_TRY(embed_scatter(tok, N, dx, V, (int)d, g->wte, s, pr));
@@ -533,6 +536,37 @@ nc_status init_model(nc_params* p, uint64_t seed, int flags) {
 }
 
 }  // namespace
+}  // namespace nc
+
+// ------------------------------------------------------------------ op status word
+// One status word per device for the single-kernel entry points, which have
+// no handle to carry one: a bounded wait that expires, a kernel that finds
+// its shared memory misaligned or a token id out of range records its code
+// here, and nc_op_sync returns it.  A file-scope __device__ variable, so no
+// allocation is involved; its device address comes from
+// cudaGetSymbolAddress (in host code the name only stands for the symbol).
+namespace nc {
+namespace {
+__device__ int g_op_status;
+constexpr int kMaxStatusDevices = 64;
+std::mutex g_op_status_mu;
+int* g_op_status_ptr[kMaxStatusDevices] = {};
+}  // namespace
+
+nc_status op_status_word(int** out) {
+  int dev = 0;
+  NC_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxStatusDevices) return fail(NC_ERR_UNSUPPORTED, "device index too large");
+  std::lock_guard<std::mutex> lock(g_op_status_mu);
+  if (!g_op_status_ptr[dev]) {
+    void* ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_op_status);
+    if (e != cudaSuccess || !ptr) return cuda_fail(e, "cudaGetSymbolAddress(op status word)");
+    g_op_status_ptr[dev] = static_cast<int*>(ptr);
+  }
+  *out = g_op_status_ptr[dev];
+  return NC_OK;
+}
 }  // namespace nc
 
 // ==================================================================== C ABI
@@ -916,7 +950,7 @@ nc_status nc_op_gemm(const nc_gemm_desc* desc, void* stream) {
   if (!desc) return fail(NC_ERR_INVALID_ARG, "gemm: null descriptor");
   GemmLaunch g{};
   g.d = *desc;
-  g.status = nullptr;
+  NC_TRY(op_status_word(&g.status));
   if (g.d.split_k < 0) return fail(NC_ERR_INVALID_ARG, "gemm: split_k < 0");
   if (g.d.split_k == 0) g.d.split_k = 1;
   return gemm_launch(g, static_cast<cudaStream_t>(stream), nullptr);
@@ -929,24 +963,64 @@ nc_status nc_op_rmsnorm(const float* x, int64_t rows, int cols, void* y_bf16, fl
   return rmsnorm_fwd(x, rows, cols, y_bf16, rstd, static_cast<cudaStream_t>(stream), nullptr);
 }
 
+nc_status nc_op_embed_gather(const int32_t* tokens, int64_t n, const float* E, int vocab, int d,
+                             float* x, void* stream) {
+  if (n < 0 || vocab < 1 || d < 4 || d % 4 || (n > 0 && (!tokens || !E || !x)))
+    return fail(NC_ERR_INVALID_ARG, "embed_gather: bad arguments (d a positive multiple of 4)");
+  if ((reinterpret_cast<uintptr_t>(E) | reinterpret_cast<uintptr_t>(x)) & 15)
+    return fail(NC_ERR_INVALID_ARG, "embed_gather: E and x must be 16-byte aligned");
+  if (n == 0) return NC_OK;
+  int* st = nullptr;
+  NC_TRY(op_status_word(&st));
+  return embed_gather(tokens, n, E, vocab, d, x, st, static_cast<cudaStream_t>(stream), nullptr);
+}
+
+nc_status nc_op_sync(void* stream) {
+  int* word = nullptr;
+  NC_TRY(op_status_word(&word));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int h = 0;
+  NC_CUDA_TRY(cudaMemcpyAsync(&h, word, sizeof(int), cudaMemcpyDeviceToHost, s));
+  NC_CUDA_TRY(cudaStreamSynchronize(s));
+  if (h == kDevOk) return NC_OK;
+  NC_CUDA_TRY(cudaMemsetAsync(word, 0, sizeof(int), s));
+  NC_CUDA_TRY(cudaStreamSynchronize(s));
+  if (h == kDevTimeout)
+    return fail(NC_ERR_TIMEOUT, "an op's bounded device wait expired (or its shared memory was "
+                                "misaligned); its outputs are incomplete");
+  if (h == kDevTokenRange) return fail(NC_ERR_TOKEN_RANGE, "an op read a token id out of [0, vocab)");
+  return fail(NC_ERR_CUDA, "unknown op status");
+}
+
+int* nc_debug_op_status_word(void) {
+  int* word = nullptr;
+  return op_status_word(&word) == NC_OK ? word : nullptr;
+}
+
 nc_status nc_op_attention_fwd(const void* q, const void* k, const void* v, int64_t ld, void* o,
                               int64_t ldo, float* lse, int B, int T, int H, void* stream) {
-  return attention_fwd(q, k, v, ld, o, ldo, lse, B, T, H, nullptr,
-                       static_cast<cudaStream_t>(stream), nullptr);
+  int* st = nullptr;
+  NC_TRY(op_status_word(&st));
+  return attention_fwd(q, k, v, ld, o, ldo, lse, B, T, H, st, static_cast<cudaStream_t>(stream),
+                       nullptr);
 }
 
 nc_status nc_op_attention_bwd(const void* q, const void* k, const void* v, int64_t ld,
                               const void* o, const void* dout, int64_t ldo, const float* lse,
                               float* dq, void* dk, void* dv, int64_t ldg, float* delta_scratch,
                               int B, int T, int H, void* stream) {
+  int* st = nullptr;
+  NC_TRY(op_status_word(&st));
   return attention_bwd(q, k, v, ld, o, dout, ldo, lse, dq, dk, dv, ldg, delta_scratch, B, T, H,
-                       nullptr, static_cast<cudaStream_t>(stream), nullptr);
+                       st, static_cast<cudaStream_t>(stream), nullptr);
 }
 
 nc_status nc_op_attention_fwd_ex(const void* q, int64_t ldq, const void* k, const void* v,
                                  int64_t ldkv, void* o, int64_t ldo, float* lse, int B, int T, int H,
                                  int Hkv, int window, void* stream) {
-  return attention_fwd_ex(q, ldq, k, v, ldkv, o, ldo, lse, B, T, H, Hkv, window, nullptr,
+  int* st = nullptr;
+  NC_TRY(op_status_word(&st));
+  return attention_fwd_ex(q, ldq, k, v, ldkv, o, ldo, lse, B, T, H, Hkv, window, st,
                           static_cast<cudaStream_t>(stream), nullptr);
 }
 
@@ -955,8 +1029,11 @@ nc_status nc_op_attention_bwd_ex(const void* q, int64_t ldq, const void* k, cons
                                  const float* lse, float* dq, void* dk, void* dv, int64_t ldg,
                                  float* delta_scratch, int B, int T, int H, int Hkv, int window,
                                  void* stream) {
+  int* st = nullptr;
+  NC_TRY(op_status_word(&st));
   return attention_bwd_ex(q, ldq, k, v, ldkv, o, dout, ldo, lse, dq, dk, dv, ldg, delta_scratch, B,
-                          T, H, Hkv, window, nullptr, static_cast<cudaStream_t>(stream), nullptr);
+                          T, H, Hkv, window, nullptr, nullptr, st, static_cast<cudaStream_t>(stream),
+                          nullptr);
 }
 
 size_t nc_newton_schulz_scratch_bytes(int count, int rows, int cols) {
@@ -982,7 +1059,9 @@ nc_status nc_op_newton_schulz(const void* x_bf16, void* out_bf16, int count, int
   NC_CUDA_TRY(cudaMemsetAsync(norms, 0, sizeof(float) * count, s));
   NC_TRY(sumsq_bf16(x_bf16, mn, count, norms, s, nullptr));
   NC_TRY(scale_bf16(x_bf16, rows, cols, tall ? 1 : 0, norms, 1e-7f, X, count, s, nullptr));
-  NC_TRY(newton_schulz_wide(X, count, m, n, steps, ws, nullptr, s, nullptr));
+  int* st = nullptr;
+  NC_TRY(op_status_word(&st));
+  NC_TRY(newton_schulz_wide(X, count, m, n, steps, ws, st, s, nullptr));
   // Back to the caller's orientation (no scaling).
   NC_TRY(scale_bf16(X, m, n, tall ? 1 : 0, nullptr, 0.f, out_bf16, count, s, nullptr));
   return NC_OK;

@@ -179,12 +179,104 @@ def test_rmsnorm(rows, cols):
     np.testing.assert_allclose(host(r), rr, rtol=1e-5)
 
 
+# ------------------------------------------------------------------ embedding gather
+@pytest.mark.parametrize("ids", ["uniform", "zipf"])
+def test_embed_gather_is_bit_exact(ids):
+    """x = E[tok] bit for bit at the step's size (65536 ids, d = 1280, V =
+    32768) through the gather kernel the model's forward launches; E holds
+    full fp32 mantissas, so any conversion or partial copy would show."""
+    t = torch()
+    N, d, V = 65536, 1280, 32768
+    if ids == "uniform":
+        tok, _ = inputs.token_batch(80, 32, 2048)
+    else:
+        tok, _ = inputs.zipf_token_batch(81, 32, 2048)
+    tok = tok.reshape(-1)
+    assert tok.min() >= 0 and tok.max() < V
+    E = np.random.default_rng(82).standard_normal((V, d)).astype(np.float32)
+    Ed = t.from_numpy(E).cuda()
+    x = t.full((N, d), float("nan"), dtype=t.float32, device="cuda")
+    nc.embed_gather(t.from_numpy(tok).cuda(), N, Ed, V, d, x)
+    nc.op_sync()
+    assert np.array_equal(x.cpu().numpy().view(np.uint32), E[tok].view(np.uint32))
+
+
+def test_embed_gather_out_of_range_ids_are_clamped_and_reported():
+    """Ids below 0 read row 0 and ids at or above V read row V - 1 (nothing
+    out of bounds); the op status word turns them into NC_ERR_TOKEN_RANGE at
+    the next op_sync, which also clears it."""
+    t = torch()
+    V, d = 1000, 256
+    tok = np.array([3, -1, 999, 1000, 5, -7, 123456, 0], dtype=np.int32)
+    E = np.random.default_rng(83).standard_normal((V, d)).astype(np.float32)
+    x = t.empty((len(tok), d), dtype=t.float32, device="cuda")
+    nc.op_sync()  # nothing pending
+    nc.embed_gather(t.from_numpy(tok).cuda(), len(tok), t.from_numpy(E).cuda(), V, d, x)
+    with pytest.raises(nc.NcError) as e:
+        nc.op_sync()
+    assert e.value.status == nc.NC_ERR_TOKEN_RANGE
+    nc.op_sync()  # cleared
+    expect = E[np.clip(tok, 0, V - 1)]
+    assert np.array_equal(x.cpu().numpy(), expect)
+
+
+def test_planted_op_status_is_reported_once():
+    """An expired bounded wait inside an op (planted here as its status code,
+    not produced by a stuck kernel) surfaces as NC_ERR_TIMEOUT at the next
+    op_sync and is cleared by it."""
+    t = torch()
+    ptr = nc.lib().nc_debug_op_status_word()
+    assert ptr
+
+    class _Word:
+        __cuda_array_interface__ = {"shape": (1,), "typestr": "<i4", "data": (ptr, False),
+                                    "version": 3}
+
+    word = t.as_tensor(_Word(), device="cuda")
+    nc.op_sync()
+    word.fill_(1)
+    t.cuda.synchronize()
+    with pytest.raises(nc.NcError) as e:
+        nc.op_sync()
+    assert e.value.status == nc.NC_ERR_TIMEOUT
+    nc.op_sync()
+
+
 # ------------------------------------------------------------------ attention
 def _attn_inputs(B, T, H, seed):
     # q, k with unit RMS per head (as after QK-norm), v normal; fused [B*T, 3d] rows.
     d = H * 128
     qkv = inputs.bf16_normal(seed, (B * T, 3 * d))
     return qkv
+
+
+def test_exp2_polynomial_against_the_exact_power():
+    """The polynomial 2^x of the attention forward (a share of its softmax
+    exponentials) against 2^x in fp64 over the range the softmax feeds it
+    ([-125, 8]; scores minus a running maximum kept within 2^8): relative
+    error below 1e-4 (the cubic's own bound is 7.5e-5, plus fp32 rounding),
+    integer arguments included, and arguments below -125 (-inf too) giving
+    2^-125 to the same accuracy."""
+    t = torch()
+    rng = np.random.default_rng(90)
+    x = np.concatenate([np.linspace(-125.0, 8.0, 200001), rng.uniform(-30.0, 8.0, 100000),
+                        np.arange(-125.0, 9.0)]).astype(np.float32)
+    xd = t.from_numpy(x).cuda()
+    y = t.empty_like(xd)
+    nc.exp2_poly(xd, y, x.size)
+    t.cuda.synchronize()
+    yh = y.cpu().numpy().astype(np.float64)
+    exact = np.exp2(x.astype(np.float64))
+    rel = np.abs(yh / exact - 1.0)
+    assert rel.max() < 1e-4, (rel.max(), x[rel.argmax()])
+    ints = np.arange(-125.0, 9.0)
+    yi = yh[-ints.size:]
+    assert np.max(np.abs(yi / np.exp2(ints) - 1.0)) < 1e-4
+    low = t.tensor([-126.0, -200.0, float("-inf")], device="cuda")
+    yl = t.empty_like(low)
+    nc.exp2_poly(low, yl, 3)
+    t.cuda.synchronize()
+    assert np.max(np.abs(yl.cpu().numpy().astype(np.float64) / 2.0 ** -125 - 1.0)) < 1e-4
 
 
 @pytest.mark.parametrize("B,T,H", [(1, 64, 1), (2, 200, 2), (1, 1, 1), (1, 577, 3)])
@@ -289,6 +381,34 @@ def test_attention_full_length_sampled_heads():
     oref, lref, _ = oracle.attention(q, k, v)
     assert rel_fro(host(o), oref.reshape(B * T, d)) < 5e-3
     np.testing.assert_allclose(host(lse), lref, rtol=2e-4, atol=2e-4)
+
+
+def test_attention_backward_full_length():
+    """The backward at the step's sequence length, T = 2048 (16 key tiles,
+    each looping over up to 16 query tiles), one batch row, two heads,
+    against the oracle's backward from the oracle's O and lse."""
+    t = torch()
+    B, T, H = 1, 2048, 2
+    d = H * 128
+    qkv = _attn_inputs(B, T, H, 61)
+    q = qkv[:, :d].reshape(B, T, H, 128)
+    k = qkv[:, d:2 * d].reshape(B, T, H, 128)
+    v = qkv[:, 2 * d:].reshape(B, T, H, 128)
+    oref, lref, _ = oracle.attention(q, k, v)
+    o_b = inputs.round_to_bf16(oref.reshape(B * T, d).astype(np.float32))
+    dout = inputs.bf16_normal(62, (B * T, d))
+    dqkv = t.zeros(B * T, 3 * d, dtype=t.bfloat16, device="cuda")
+    dqf = t.empty(B * T, d, dtype=t.float32, device="cuda")
+    delta = t.empty(B, H, T, dtype=t.float32, device="cuda")
+    tq = dev_bf16(qkv)
+    nc.attention_bwd(tq, tq[:, d:], tq[:, 2 * d:], 3 * d, dev_bf16(o_b), dev_bf16(dout), d,
+                     dev_f32(lref.astype(np.float32)), dqf, dqkv[:, d:], dqkv[:, 2 * d:], 3 * d,
+                     delta, B, T, H)
+    t.cuda.synchronize()
+    rq, rk, rv = oracle.attention_bwd(q, k, v, lref, dout.reshape(B, T, H, 128))
+    assert rel_fro(host(dqf), rq.reshape(B * T, d)) < 1e-2
+    assert rel_fro(host(dqkv[:, d:2 * d]), rk.reshape(B * T, d)) < 1e-2
+    assert rel_fro(host(dqkv[:, 2 * d:]), rv.reshape(B * T, d)) < 1e-2
 
 
 # ------------------------------------------------------------------ Newton-Schulz

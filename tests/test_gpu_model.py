@@ -78,6 +78,42 @@ def test_fwd_bwd_parity_grouped_kv_and_windows(depth, B, T, vocab, n_kv, window)
         assert rel_fro(g, r) < 3e-2, (i, names[i], rel_fro(g, r))
 
 
+def test_depth20_random_weights_short_row():
+    """The headline depth (20: d 1280, 10 heads, MLP 5120, V 32768) with every
+    matrix random, on one 128-token row: loss and every gradient tensor
+    against the oracle at the step's bars."""
+    depth, B, T = 20, 1, 128
+    P = inputs.random_params(depth, seed=200)
+    tok, tgt = inputs.token_batch(201, B, T)
+    m = _gpt(depth)
+    m.load(P)
+    loss = m.fwd_bwd(tok, tgt)
+    G = m.grads()
+    m.close()
+    lref, Gref, _ = oracle.gpt_fwd_bwd(depth, P, tok, tgt)
+    assert abs(loss - lref) / lref < 2e-3, (loss, lref)
+    names = ["wte"] + ["wq", "wk", "wv", "wo", "wup", "wdown"] * depth + ["lm_head"]
+    worst = max((rel_fro(g, r), i) for i, (g, r) in enumerate(zip(G, Gref)))
+    assert worst[0] < 3e-2, (worst, names[worst[1]])
+
+
+def test_depth20_full_length_row_loss():
+    """Depth 20 with random weights on one row of the step's length (T =
+    2048, 16 query and key tiles per head in every attention kernel): the
+    loss against the oracle's forward."""
+    depth, B, T = 20, 1, 2048
+    P = inputs.random_params(depth, seed=210)
+    tok, tgt = inputs.token_batch(211, B, T)
+    m = _gpt(depth)
+    m.load(P)
+    loss = m.fwd_bwd(tok, tgt)
+    G = m.grads()
+    m.close()
+    assert all(np.isfinite(g).all() for g in G)
+    lref, _, _ = oracle.gpt_fwd_bwd(depth, P, tok, tgt, grads=False)
+    assert abs(loss - lref) / lref < 2e-3, (loss, lref)
+
+
 def test_spec_init_loss_and_gradients_at_full_size():
     """Depth 20, B = 32, T = 2048 (the headline workload) at the specified
     init: loss = ln 32768, every gradient but lm_head's exactly zero, and
@@ -116,25 +152,6 @@ def test_init_matches_the_oracle_generator(n_kv):
             assert not a.any(), i
         else:
             assert np.max(np.abs(a - b)) <= 1e-6 * np.max(np.abs(b)), i
-
-
-def test_embedding_gather_is_bit_exact():
-    """With every block matrix and lm_head zero, the final hidden state is
-    rms(E[tok]); the lm_head gradient then carries E[tok] exactly through
-    the gather: checked via d(loss)/d(lm_head) against the closed form with
-    tolerance only for the later arithmetic, and the gather itself via a
-    one-hot embedding whose rows are distinct powers of two."""
-    depth, B, T, vocab = 2, 1, 16, 64
-    m = _gpt(depth, vocab=vocab)
-    P = [np.zeros(s, np.float32) for s in m.shapes()]
-    E = (2.0 ** -np.arange(vocab)[:, None] * np.ones((1, 128))).astype(np.float32)
-    P[0] = E
-    m.load(P)
-    tok, tgt = inputs.token_batch(22, B, T, vocab=vocab)
-    m.fwd_bwd(tok, tgt)
-    # dE[tok] gets all of dx0; with zero blocks and head, dx0 = 0 and dE = 0.
-    assert not m.grad(0).any()
-    m.close()
 
 
 def test_host_and_device_token_pointers_agree():
