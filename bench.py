@@ -823,9 +823,10 @@ def run_step_variant(args, dims, peaks, peak_kind):
     if args.window_pattern:
         windows = nc.window_pattern(args.window_pattern, depth, args.short_window)
     stream = torch.cuda.Stream()
-    m = nc.GPT(depth, vocab=V, seed=1234, all_random=True, stream=stream,
+    vocab = args.vocab
+    m = nc.GPT(depth, vocab=vocab, seed=1234, all_random=True, stream=stream,
                n_kv_head=args.kv_heads, window=windows)
-    tk, tg = inputs.token_batch(20, Bb, T_)
+    tk, tg = inputs.token_batch(20, Bb, T_, vocab=vocab)
     tok, tgt = torch.from_numpy(tk).cuda(), torch.from_numpy(tg).cuda()
     loss = torch.zeros(1, dtype=torch.float32, device="cuda")
     torch.cuda.synchronize()
@@ -847,10 +848,13 @@ def run_step_variant(args, dims, peaks, peak_kind):
     m.sync()
     torch.cuda.synchronize()
     ms = ev0.elapsed_time(ev1) / args.steps
+    free, total = torch.cuda.mem_get_info()  # the model's buffers are all still held here
     m.close()
     tok_s = Bb * T_ / (ms / 1e3)
-    fpt = step_flops_per_token(depth, T_, V, args.kv_heads, windows)
-    print(json.dumps({"op": "step", "depth": depth, "B": Bb, "T": T_, "kv_heads": args.kv_heads,
+    fpt = step_flops_per_token(depth, T_, vocab, args.kv_heads, windows)
+    print(json.dumps({"op": "step", "depth": depth, "B": Bb, "T": T_, "vocab": vocab,
+                      "kv_heads": args.kv_heads, "device_gb_in_use": (total - free) / 1e9,
+                      "device_gb_total": total / 1e9,
                       "windows": windows, "ms_per_step": ms, "tokens_per_s": tok_s,
                       "flops_per_token": fpt, "tflops": tok_s * fpt / 1e12,
                       "mfu": tok_s * fpt / 1e12 / NOMINAL_BF16_TFLOPS,
@@ -874,6 +878,8 @@ def main():
     ap.add_argument("--window-pattern", default=None,
                     help="--op step: per-layer pattern of S (short window) and L (full causal)")
     ap.add_argument("--short-window", type=int, default=1024, help="--op step: the S window")
+    ap.add_argument("--vocab", type=int, default=V,
+                    help="--op step: vocabulary (smaller only for kernel captures on a small case)")
     ap.add_argument("--shape", default="16384,5120,1280")
     args = ap.parse_args()
     if args.warmup < 3:
