@@ -376,10 +376,6 @@ __global__ void __launch_bounds__(kThreads, 2)
 //                needs no exchange between threads; the maximum is raised
 //                only past 2^8 (O rescaled in TMEM then), and P is written as
 //                bf16 over the scores it replaces (key k in column k / 2).
-//                A share of the exponentials (POLY of every 32) runs on the
-//                FMA pipe as a polynomial, the rest on the exponential unit,
-//                whose 16 results per clock per SM would otherwise bound
-//                the softmax at the pace of the tile's two products.
 // TMEM columns: S_a [0,128), S_b [128,256), O_a [256,384), O_b [384,512).
 // The MMAs run in issue order, so S_x(j+1) never overwrites P_x(j) before
 // PV_x(j) has read it, and the commit that publishes S_x(j+1) also covers
@@ -390,25 +386,6 @@ constexpr int PP_OFF_K = 2 * TILE;   // 2 stages
 constexpr int PP_OFF_V = 4 * TILE;   // 2 stages
 constexpr int PP_OFF_BAR = 6 * TILE;
 constexpr int kPPSmem = PP_OFF_BAR + 512;
-constexpr int kPolyExp = 8;  // exponentials per 32 scores evaluated by polynomial
-
-// 2^x on the FMA pipe (x <= 126): x = n + f with n the nearest integer
-// (rounded by adding 1.5 * 2^23, whose low mantissa bits then hold n) and
-// f in [-0.5, 0.5]; 2^f by the cubic that minimises the largest relative
-// error on that interval (Remez exchange, relative error below 7.5e-5,
-// under a thirtieth of a bf16 step); 2^n is added into the exponent field.
-// Arguments below -125 return 2^-125 (a tiny normal number, not 0).
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = x + 12582912.f;
-  const float f = x - (t - 12582912.f);
-  float p = fmaf(0.05517167f, f, 0.24261113f);
-  p = fmaf(p, f, 0.69326097f);
-  p = fmaf(p, f, 0.99992806f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-static_assert(kPPSmem <= 232448, "two-tile forward shared memory budget");
-
 __global__ void __launch_bounds__(kPPThreads, 1)
     attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const FwdArgs a) {
@@ -620,12 +597,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float x0 = fmaf(__uint_as_float(r[c][2 * i]), a.sl2, neg_mu);
-            const float x1 = fmaf(__uint_as_float(r[c][2 * i + 1]), a.sl2, neg_mu);
-            // Edge tiles take every exponential from the exponential unit, so
-            // masked keys give exactly 0.
-            const float p0 = (!edge && 2 * i < kPolyExp) ? exp2_poly(x0) : ex2(x0);
-            const float p1 = (!edge && 2 * i + 1 < kPolyExp) ? exp2_poly(x1) : ex2(x1);
+            const float p0 = ex2(fmaf(__uint_as_float(r[c][2 * i]), a.sl2, neg_mu));
+            const float p1 = ex2(fmaf(__uint_as_float(r[c][2 * i + 1]), a.sl2, neg_mu));
             ls[(2 * i) & 3] += p0;
             ls[(2 * i + 1) & 3] += p1;
             pk[i] = pack_bf16x2(p0, p1);
@@ -1027,19 +1000,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int c = 0; c < 2; ++c) {
         uint32_t sv[32];
         tc::tmem_ld_32x32b_x32(s_col + 32 * c, sv);
-        tc::tmem_ld_wait();
+        // The chunk's 32 lse values as eight 16-byte shared loads, issued
+        // while the scores are in flight.
+        float l[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int j = 32 * c + 2 * i;
-          float p0 = ex2(fmaf(__uint_as_float(sv[2 * i]), a.sl2, -lq[j]));
-          float p1 = ex2(fmaf(__uint_as_float(sv[2 * i + 1]), a.sl2, -lq[j + 1]));
-          if (edge) {
-            const int qa = qh + j, qb2 = qa + 1;
-            if (qa < key || qa >= a.T || key >= a.T || (window >= 0 && qa > key + window)) p0 = 0.f;
-            if (qb2 < key || qb2 >= a.T || key >= a.T || (window >= 0 && qb2 > key + window)) p1 = 0.f;
-          }
-          pk[c][i] = pack_bf16x2(p0, p1);
+        for (int u = 0; u < 8; ++u) {
+          const float4 v = reinterpret_cast<const float4*>(lq + 32 * c)[u];
+          l[4 * u] = v.x;
+          l[4 * u + 1] = v.y;
+          l[4 * u + 2] = v.z;
+          l[4 * u + 3] = v.w;
         }
+        tc::tmem_ld_wait();
+        // Every argument first, then the 32 independent exponentials.
+        float p[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) p[i] = fmaf(__uint_as_float(sv[i]), a.sl2, -l[i]);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) p[i] = ex2(p[i]);
+        if (edge) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int qa = qh + 32 * c + i;
+            if (qa < key || qa >= a.T || key >= a.T || (window >= 0 && qa > key + window)) p[i] = 0.f;
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[c][i] = pack_bf16x2(p[2 * i], p[2 * i + 1]);
       }
       tc::tmem_st_32x32b_x16(s_col, pk[0]);
       tc::tmem_st_32x32b_x16(s_col + 16, pk[1]);
@@ -1061,14 +1048,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int c = 0; c < 2; ++c) {
         uint32_t dpv[32];
         tc::tmem_ld_32x32b_x32(dp_col + 32 * c, dpv);
+        float dl[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float4 v = reinterpret_cast<const float4*>(ld + 32 * c)[u];
+          dl[4 * u] = v.x;
+          dl[4 * u + 1] = v.y;
+          dl[4 * u + 2] = v.z;
+          dl[4 * u + 3] = v.w;
+        }
         tc::tmem_ld_wait();
         uint32_t pd[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const int j = 32 * c + 2 * i;
           const float2 p = unpack_bf16x2(pk[c][i]);
-          const float d0 = p.x * (__uint_as_float(dpv[2 * i]) - ld[j]);
-          const float d1 = p.y * (__uint_as_float(dpv[2 * i + 1]) - ld[j + 1]);
+          const float d0 = p.x * (__uint_as_float(dpv[2 * i]) - dl[2 * i]);
+          const float d1 = p.y * (__uint_as_float(dpv[2 * i + 1]) - dl[2 * i + 1]);
           pd[i] = pack_bf16x2(d0, d1);
         }
 #pragma unroll
@@ -1267,25 +1262,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 
 // ------------------------------------------------------------------ dQ from stored dS
-// Query side of the backward when the key-side kernel stored dS^T: one CTA per
-// (128-query tile, query head, batch row), heaviest tiles first, accumulating
+// Query side of the backward when the key-side kernel stored dS^T: a
+// persistent kernel (one CTA per SM) walks the work items (128-query tile,
+// query head, batch row), heaviest tiles first, and for each accumulates
 //   dQ = sum over key tiles kb of dS(i, kb) K_kb        (M 128 queries, N 128 dims)
-// in TMEM through a three-stage TMA ring of the dS^T tile ([128 keys][128
-// queries], read MN-major) and the K tile ([128 keys][128 dims], MN-major).
-// The epilogue takes dQ through the backward of the q-side RoPE + QK-norm:
-// with g = dQ / sqrt(128), yhat the saved normalised q and r its 1/rms,
+// in TMEM from the dS^T tile ([128 keys][128 queries], read MN-major) and the
+// K tile ([128 keys][128 dims], MN-major), each through its own TMA ring.
+// Two TMEM accumulators alternate between items, so one item's epilogue
+// runs while the next item's tiles stream in and multiply.  The epilogue
+// takes dQ through the backward of the q-side RoPE + QK-norm: with
+// g = dQ / sqrt(128), yhat the saved normalised q and r its 1/rms,
 //   dr = r (g - yhat mean(g yhat)),  dq = R(-theta) dr  (pairs i, i + 64),
 // written as bf16 into the q slice of the q|k|v gradient.  192 threads:
 // warp 0 TMA, warp 1 TMEM owner and MMA issue, warps 2..5 one query row each.
 constexpr int kDqThreads = 192;
-constexpr int kDqStages = 3;
-constexpr int DQ_STAGE = 2 * TILE;  // dS^T tile + K tile
-constexpr int DQ_OFF_BAR = kDqStages * DQ_STAGE;
+// The dS^T tiles come from HBM (written by the key-side kernel, far larger
+// than L2) and get a four-deep ring; a K tile is shared by the 16 query
+// tiles of its (head, row), so it mostly hits L2 and two stages suffice.
+constexpr int kDqDsStages = 4;
+constexpr int kDqKStages = 2;
+constexpr int DQ_OFF_K = kDqDsStages * TILE;
+constexpr int DQ_OFF_BAR = DQ_OFF_K + kDqKStages * TILE;
 constexpr int kDqSmem = DQ_OFF_BAR + 256;
 static_assert(kDqSmem <= 232448, "dQ kernel shared memory budget");
 
 struct DqArgs {
-  int T, H, nqb;
+  int T, H, B, nqb;
   int group;   // query heads per KV head
   int window;  // query t sees keys [t - window, t]; < 0: every key up to t
   float scale;
@@ -1296,6 +1298,43 @@ struct DqArgs {
   __nv_bfloat16* out;         // dq rows: out + tok * ldo + h * 128
   int64_t ldo;
   int* status;
+};
+
+// Work item w (heaviest first): query tile, head, batch row, and the key
+// tiles [kb_lo, qi] whose dS^T tiles the key-side kernel stored for it.
+struct DqItem {
+  int qi, h, b, kb_lo, n;
+};
+__device__ __forceinline__ DqItem dq_item(const DqArgs& a, int w, int window) {
+  DqItem it;
+  const int hb = a.H * a.B;
+  it.qi = a.nqb - 1 - w / hb;
+  const int rest = w % hb;
+  it.h = rest % a.H;
+  it.b = rest / a.H;
+  const int lo = window < 0 ? 0 : it.qi * BQB - BKV + 1 - window;
+  it.kb_lo = lo <= 0 ? 0 : (lo + BKV - 1) / BKV;
+  it.n = it.qi - it.kb_lo + 1;
+  return it;
+}
+
+// Walks this CTA's key tiles in order: item w (stride gridDim.x), tile t of it.
+struct DqCursor {
+  int w, t;
+  DqItem m;
+  __device__ __forceinline__ bool valid(int nitems) const { return w < nitems; }
+  __device__ __forceinline__ void start(const DqArgs& a, int window) {
+    w = blockIdx.x;
+    t = 0;
+    m = dq_item(a, w, window);
+  }
+  __device__ __forceinline__ void next(const DqArgs& a, int window, int nitems) {
+    if (++t == m.n) {
+      t = 0;
+      w += gridDim.x;
+      if (w < nitems) m = dq_item(a, w, window);
+    }
+  }
 };
 
 template <bool GW>
@@ -1309,36 +1348,39 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   }
   uint8_t* smem = smem_raw;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DQ_OFF_BAR);
-  uint64_t* full = bars;                    // [kDqStages]
-  uint64_t* empty = bars + kDqStages;       // [kDqStages]
-  uint64_t* acc_full = bars + 2 * kDqStages;
-  uint64_t* drained = acc_full + 1;
+  uint64_t* ds_full = bars;                        // [kDqDsStages]
+  uint64_t* ds_empty = bars + kDqDsStages;         // [kDqDsStages]
+  uint64_t* k_full = bars + 2 * kDqDsStages;       // [kDqKStages]
+  uint64_t* k_empty = k_full + kDqKStages;         // [kDqKStages]
+  uint64_t* acc_full = k_empty + kDqKStages;       // [2]
+  uint64_t* acc_empty = acc_full + 2;              // [2]
+  uint64_t* drained = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qi = a.nqb - 1 - (int)blockIdx.x;  // heaviest tiles first
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int hk = GW ? h / a.group : h;
   const int window = GW ? a.window : -1;
-  // Key tiles whose dS^T tiles the key-side kernel stored for this query
-  // tile: from the first one a window reaches to the diagonal.
-  const int lo = window < 0 ? 0 : qi * BQB - BKV + 1 - window;
-  const int kb_lo = lo <= 0 ? 0 : (lo + BKV - 1) / BKV;
-  const int n = qi - kb_lo + 1;
+  const int nitems = a.nqb * a.H * a.B;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kDqStages; ++i) {
-      tc::mbar_init(&full[i], 1);
-      tc::mbar_init(&empty[i], 1);
+    for (int i = 0; i < kDqDsStages; ++i) {
+      tc::mbar_init(&ds_full[i], 1);
+      tc::mbar_init(&ds_empty[i], 1);
     }
-    tc::mbar_init(acc_full, 1);
+    for (int i = 0; i < kDqKStages; ++i) {
+      tc::mbar_init(&k_full[i], 1);
+      tc::mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&acc_full[i], 1);
+      tc::mbar_init(&acc_empty[i], 128);
+    }
     tc::mbar_init(drained, 1);
     *abort_flag = 0;
     tc::fence_mbar_init();
   }
   if (warp == 1) {
-    tc::tmem_alloc(tmem_slot, 128);
+    tc::tmem_alloc(tmem_slot, 256);
     tc::tmem_relinquish();
   }
   tc::tc_fence_before();
@@ -1350,44 +1392,86 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     if (lane == 0) {
       tc::tma_prefetch_desc(&tds);
       tc::tma_prefetch_desc(&tk);
-      int issued = 0;
+      // dS^T tile u and K tile u - (ring depth difference): the dS^T ring
+      // runs kDqDsStages tiles ahead of the tensor core, the K ring kDqKStages.
+      constexpr int lag = kDqDsStages - kDqKStages;
+      DqCursor cd, ck;
+      cd.start(a, window);
+      ck.start(a, window);
+      int issued_d = 0, issued_k = 0;
       bool ok = true;
-      for (int t = 0; t < n; ++t) {
-        const int st = t % kDqStages;
-        const uint32_t ph = (t / kDqStages) & 1;
-        if (!tc::mbar_wait(&empty[st], ph ^ 1, abort_flag, a.status)) { ok = false; break; }
-        const int kb = kb_lo + t;
-        uint8_t* base = smem + st * DQ_STAGE;
-        tc::mbar_arrive_expect_tx(&full[st], 2 * TILE);
-        for (int c = 0; c < 2; ++c) {
-          tc::tma_load_3d(base + c * (TILE / 2), &tds, &full[st], qi * BQB + 64 * c, kb * BKV,
-                          b * a.H + h);
-          tc::tma_load_3d(base + TILE + c * (TILE / 2), &tk, &full[st], hk * HD + 64 * c, kb * BKV, b);
+      for (int u = 0; ok && (cd.valid(nitems) || ck.valid(nitems)); ++u) {
+        if (cd.valid(nitems)) {
+          const int st = issued_d % kDqDsStages;
+          if (!tc::mbar_wait(&ds_empty[st], ((issued_d / kDqDsStages) & 1) ^ 1, abort_flag,
+                             a.status)) {
+            ok = false;
+            break;
+          }
+          tc::mbar_arrive_expect_tx(&ds_full[st], TILE);
+          for (int c = 0; c < 2; ++c)
+            tc::tma_load_3d(smem + st * TILE + c * (TILE / 2), &tds, &ds_full[st],
+                            cd.m.qi * BQB + 64 * c, (cd.m.kb_lo + cd.t) * BKV, cd.m.b * a.H + cd.m.h);
+          ++issued_d;
+          cd.next(a, window, nitems);
         }
-        ++issued;
+        if (u >= lag && ck.valid(nitems)) {
+          const int st = issued_k % kDqKStages;
+          if (!tc::mbar_wait(&k_empty[st], ((issued_k / kDqKStages) & 1) ^ 1, abort_flag,
+                             a.status)) {
+            ok = false;
+            break;
+          }
+          const int hk = GW ? ck.m.h / a.group : ck.m.h;
+          tc::mbar_arrive_expect_tx(&k_full[st], TILE);
+          for (int c = 0; c < 2; ++c)
+            tc::tma_load_3d(smem + DQ_OFF_K + st * TILE + c * (TILE / 2), &tk, &k_full[st],
+                            hk * HD + 64 * c, (ck.m.kb_lo + ck.t) * BKV, ck.m.b);
+          ++issued_k;
+          ck.next(a, window, nitems);
+        }
       }
-      if (!ok)
-        for (int t = max(0, issued - kDqStages); t < issued; ++t)
-          drain_wait(&full[t % kDqStages], (t / kDqStages) & 1);
+      if (!ok) {
+        for (int i = max(0, issued_d - kDqDsStages); i < issued_d; ++i)
+          drain_wait(&ds_full[i % kDqDsStages], (i / kDqDsStages) & 1);
+        for (int i = max(0, issued_k - kDqKStages); i < issued_k; ++i)
+          drain_wait(&k_full[i % kDqKStages], (i / kDqKStages) & 1);
+      }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t id = tc::idesc_bf16_f32(128, 128, 1, 1);
       const uint64_t ad = tc::smem_desc_sw128(tc::smem_u32(smem), TILE / 2, 1024);
-      const uint64_t bd = tc::smem_desc_sw128(tc::smem_u32(smem + TILE), TILE / 2, 1024);
+      const uint64_t bd = tc::smem_desc_sw128(tc::smem_u32(smem + DQ_OFF_K), TILE / 2, 1024);
+      int it = 0, item = 0;
       bool ok = true;
-      for (int t = 0; t < n && ok; ++t) {
-        const int st = t % kDqStages;
-        if (!tc::mbar_wait(&full[st], (t / kDqStages) & 1, abort_flag, a.status)) { ok = false; break; }
+      for (int w = blockIdx.x; w < nitems && ok; w += gridDim.x, ++item) {
+        const DqItem m = dq_item(a, w, window);
+        const int buf = item & 1;
+        // The epilogue of the item two back has read this accumulator.
+        if (!tc::mbar_wait(&acc_empty[buf], ((item >> 1) & 1) ^ 1, abort_flag, a.status)) {
+          ok = false;
+          break;
+        }
         tc::tc_fence_after();
-        const uint64_t a0 = tc::desc_add(ad, st * DQ_STAGE), b0 = tc::desc_add(bd, st * DQ_STAGE);
+        for (int t = 0; t < m.n; ++t, ++it) {
+          const int sd = it % kDqDsStages, sk = it % kDqKStages;
+          if (!tc::mbar_wait(&ds_full[sd], (it / kDqDsStages) & 1, abort_flag, a.status) ||
+              !tc::mbar_wait(&k_full[sk], (it / kDqKStages) & 1, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
+          tc::tc_fence_after();
+          const uint64_t a0 = tc::desc_add(ad, sd * TILE), b0 = tc::desc_add(bd, sk * TILE);
 #pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk)
-          tc::umma_bf16_ss(tmem, tc::desc_add(a0, kk * 2048), tc::desc_add(b0, kk * 2048), id,
-                           (t > 0 || kk > 0) ? 1u : 0u);
-        tc::umma_commit(&empty[st]);
+          for (int kk = 0; kk < BKV / 16; ++kk)
+            tc::umma_bf16_ss(tmem + 128 * buf, tc::desc_add(a0, kk * 2048), tc::desc_add(b0, kk * 2048),
+                             id, (t > 0 || kk > 0) ? 1u : 0u);
+          tc::umma_commit(&ds_empty[sd]);
+          tc::umma_commit(&k_empty[sk]);
+        }
+        if (ok) tc::umma_commit(&acc_full[buf]);
       }
-      if (ok) tc::umma_commit(acc_full);
       tc::umma_commit(drained);
       drain_wait(drained, 0);
     }
@@ -1395,25 +1479,29 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     // Epilogue: one query row per thread (warp w reaches TMEM lanes of quarter w % 4).
     const int qw = warp & 3;
     const int row = qw * 32 + lane;
-    const int q = qi * BQB + row;
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
-    bool ok = tc::mbar_wait(acc_full, 0, abort_flag, a.status);
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
+    int item = 0;
+    for (int w = blockIdx.x; w < nitems; w += gridDim.x, ++item) {
+      const DqItem m = dq_item(a, w, window);
+      const int buf = item & 1;
+      const uint32_t acc = lane_base + 128 * buf;
+      bool ok = tc::mbar_wait(&acc_full[buf], (item >> 1) & 1, abort_flag, a.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
       tc::tc_fence_after();
+      const int q = m.qi * BQB + row;
       const bool live = q < a.T;
-      const int64_t tok = (int64_t)b * a.T + (live ? q : 0);
-      const __nv_bfloat16* yrow = a.yhat + tok * a.ldy + h * HD;
+      const int64_t tok = (int64_t)m.b * a.T + (live ? q : 0);
+      const __nv_bfloat16* yrow = a.yhat + tok * a.ldy + m.h * HD;
       // 32 dims of yhat starting at dim 32 c.
       auto load_y = [&](int c, float (&y)[32]) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const uint4 w = live ? reinterpret_cast<const uint4*>(yrow + 32 * c)[u]
+          const uint4 v = live ? reinterpret_cast<const uint4*>(yrow + 32 * c)[u]
                                : make_uint4(0u, 0u, 0u, 0u);
-          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+          const uint32_t vs[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float2 f = unpack_bf16x2(ws[e]);
+            const float2 f = unpack_bf16x2(vs[e]);
             y[8 * u + 2 * e] = f.x;
             y[8 * u + 2 * e + 1] = f.y;
           }
@@ -1424,25 +1512,29 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       for (int c = 0; c < 4; ++c) {
         uint32_t g[32];
         float y[32];
-        tc::tmem_ld_32x32b_x32(lane_base + 32 * c, g);
+        tc::tmem_ld_32x32b_x32(acc + 32 * c, g);
         load_y(c, y);
         tc::tmem_ld_wait();
 #pragma unroll
         for (int i = 0; i < 32; ++i) dot = fmaf(__uint_as_float(g[i]), y[i], dot);
       }
-      const float r = live ? a.rstd_q[tok * a.H + h] : 0.f;
-      const float m = dot * a.scale / 128.f;
-      __nv_bfloat16* dst = a.out + tok * a.ldo + h * HD;
+      const float r = live ? a.rstd_q[tok * a.H + m.h] : 0.f;
+      const float mean = dot * a.scale / 128.f;
+      __nv_bfloat16* dst = a.out + tok * a.ldo + m.h * HD;
       const float2* cs = a.rope_tab + (int64_t)(live ? q : 0) * 64;
 #pragma unroll 1
       for (int c = 0; c < 2; ++c) {
         uint32_t g0[32], g1[32];
         float y0[32], y1[32];
-        tc::tmem_ld_32x32b_x32(lane_base + 32 * c, g0);
-        tc::tmem_ld_32x32b_x32(lane_base + 64 + 32 * c, g1);
+        tc::tmem_ld_32x32b_x32(acc + 32 * c, g0);
+        tc::tmem_ld_32x32b_x32(acc + 64 + 32 * c, g1);
         load_y(c, y0);
         load_y(c + 2, y1);
         tc::tmem_ld_wait();
+        if (c == 1) {  // the accumulator is read: the MMA warp may reuse it
+          tc::tc_fence_before();
+          tc::mbar_arrive(&acc_empty[buf]);
+        }
         if (live) {
           uint32_t lo_[16], hi_[16];
 #pragma unroll
@@ -1450,8 +1542,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             float o_lo[2], o_hi[2];
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-              const float d0 = r * (__uint_as_float(g0[i + e]) * a.scale - y0[i + e] * m);
-              const float d1 = r * (__uint_as_float(g1[i + e]) * a.scale - y1[i + e] * m);
+              const float d0 = r * (__uint_as_float(g0[i + e]) * a.scale - y0[i + e] * mean);
+              const float d1 = r * (__uint_as_float(g1[i + e]) * a.scale - y1[i + e] * mean);
               const float2 tt = cs[32 * c + i + e];  // (cos, sin) of pair 32 c + i + e
               o_lo[e] = d0 * tt.x + d1 * tt.y;
               o_hi[e] = d1 * tt.x - d0 * tt.y;
@@ -1474,17 +1566,10 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc::tc_fence_after();
-    tc::tmem_dealloc(tmem, 128);
+    tc::tmem_dealloc(tmem, 256);
   }
 }
 
-}  // namespace
-
-namespace {
-__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) y[i] = exp2_poly(x[i]);
-}
 }  // namespace
 
 // Query-key pairs a causal window keeps: sum over t of min(t, window) + 1
@@ -1667,6 +1752,7 @@ nc_status attention_dq_ex(const void* ds, int64_t ld_ds, const void* k, int64_t 
   DqArgs a;
   a.T = T;
   a.H = H;
+  a.B = B;
   a.nqb = (T + BQB - 1) / BQB;
   a.group = H / Hkv;
   a.window = (window < 0 || window >= T - 1) ? -1 : window;
@@ -1680,7 +1766,9 @@ nc_status attention_dq_ex(const void* ds, int64_t ld_ds, const void* k, int64_t 
   a.status = status;
   const double flops = 2.0 * B * H * HD * causal_pairs(T, a.window);
   Probe probe(prof, s, "attn_bwd_dq", flops, 0.0);
-  dim3 grid(a.nqb, H, B);
+  // Persistent: one CTA per SM (or per work item when there are fewer).
+  const int nitems = a.nqb * H * B;
+  const unsigned grid = (unsigned)std::min(nitems, num_sms());
   if (a.group > 1 || a.window >= 0)
     attn_dq_kernel<true><<<grid, kDqThreads, kDqSmem, s>>>(mds, mk, a);
   else
@@ -1690,12 +1778,3 @@ nc_status attention_dq_ex(const void* ds, int64_t ld_ds, const void* k, int64_t 
 }
 
 }  // namespace nc
-
-extern "C" nc_status nc_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
-  using namespace nc;
-  if (n < 0 || (n > 0 && (!x || !y))) return fail(NC_ERR_INVALID_ARG, "exp2_poly: bad arguments");
-  if (n == 0) return NC_OK;
-  exp2_poly_kernel<<<(unsigned)((n + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
-  NC_CUDA_TRY(cudaGetLastError());
-  return NC_OK;
-}
