@@ -37,8 +37,8 @@ NOMINAL_BF16_TFLOPS = 2250.0
 # (profiles/gemm_traffic_by_class.md), as a ratio to that launch's
 # algorithmic operand + result bytes.  The step's traffic per GEMM launch is
 # each class's algorithmic bytes times its ratio, averaged over the launches.
-# None until captured for the kernels as they stand.
-GEMM_TRAFFIC_RATIO = None
+# None when no capture covers the kernels as they stand.
+GEMM_TRAFFIC_RATIO = {"fwd": 0.88, "dgrad": 0.898, "wgrad": 1.369, "lmhead": 1.368, "ns": 0.942}
 
 
 def model_flops_per_token(depth=DEPTH, seq=T, vocab=V):
