@@ -244,12 +244,6 @@ nc_status nc_op_sync(void* stream);
  * address cannot be looked up. */
 int* nc_debug_op_status_word(void);
 
-/* Testing hook: y[i] = 2^x[i] by the polynomial the attention forward uses
- * for a share of its softmax exponentials (device pointers, n floats):
- * nearest-integer range reduction and a cubic on [-0.5, 0.5], relative
- * error below 7.5e-5 for x in [-125, 126]; x below -125 gives 2^-125. */
-nc_status nc_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream);
-
 /* Embedding gather, the first step of the forward (guide, section "1. Modelo
  * GPT": token embedding, untied from lm_head): x[i, :] = E[tokens[i], :]
  * for i < n, copied bit for bit (fp32 rows of d floats; E [vocab, d] and x

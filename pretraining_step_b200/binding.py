@@ -107,7 +107,6 @@ def lib():
         "nc_op_embed_gather": (ci, [vp, i64, vp, ci, ci, vp, vp]),
         "nc_op_sync": (ci, [vp]),
         "nc_debug_op_status_word": (vp, []),
-        "nc_debug_exp2_poly": (ci, [vp, vp, i64, vp]),
         "nc_op_attention_fwd": (ci, [vp, vp, vp, i64, vp, i64, vp, ci, ci, ci, vp]),
         "nc_op_attention_bwd": (ci, [vp, vp, vp, i64, vp, vp, i64, vp, vp, vp, vp, i64, vp,
                                      ci, ci, ci, vp]),
@@ -339,11 +338,6 @@ def embed_gather(tokens, n, E, vocab, d, x, stream=None):
     """x[i] = E[tokens[i]] (fp32 rows, bit for bit); ids out of range are
     clamped and reported by op_sync."""
     _check(lib().nc_op_embed_gather(_ptr(tokens), n, _ptr(E), vocab, d, _ptr(x), _stream(stream)))
-
-
-def exp2_poly(x, y, n, stream=None):
-    """Testing hook: the attention forward's polynomial 2^x, elementwise."""
-    _check(lib().nc_debug_exp2_poly(_ptr(x), _ptr(y), n, _stream(stream)))
 
 
 def op_sync(stream=None):

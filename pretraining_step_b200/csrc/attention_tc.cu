@@ -1273,16 +1273,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // takes dQ through the backward of the q-side RoPE + QK-norm: with
 // g = dQ / sqrt(128), yhat the saved normalised q and r its 1/rms,
 //   dr = r (g - yhat mean(g yhat)),  dq = R(-theta) dr  (pairs i, i + 64),
-// written as bf16 into the q slice of the q|k|v gradient.  192 threads:
-// warp 0 TMA, warp 1 TMEM owner and MMA issue, warps 2..5 one query row each.
-constexpr int kDqThreads = 192;
+// written as bf16 into the q slice of the q|k|v gradient.  320 threads:
+// warp 0 TMA, warp 1 TMEM owner and MMA issue, warps 2..9 the epilogue, two
+// threads per query row, each holding 32 whole RoPE pairs (dims
+// [32 s, 32 s + 32) and [64 + 32 s, 96 + 32 s) for side s): the saved q row
+// and its cos/sin are loaded before the accumulator is waited for, and the
+// pair of threads combines its two halves of mean(g yhat) through shared
+// memory.
+constexpr int kDqThreads = 320;
 // The dS^T tiles come from HBM (written by the key-side kernel, far larger
 // than L2) and get a four-deep ring; a K tile is shared by the 16 query
 // tiles of its (head, row), so it mostly hits L2 and two stages suffice.
 constexpr int kDqDsStages = 4;
 constexpr int kDqKStages = 2;
 constexpr int DQ_OFF_K = kDqDsStages * TILE;
-constexpr int DQ_OFF_BAR = DQ_OFF_K + kDqKStages * TILE;
+constexpr int DQ_OFF_DOT = DQ_OFF_K + kDqKStages * TILE;  // [2 accumulators][2 sides][128 rows] f32
+constexpr int DQ_OFF_BAR = DQ_OFF_DOT + 2 * 2 * 128 * 4;
 constexpr int kDqSmem = DQ_OFF_BAR + 256;
 static_assert(kDqSmem <= 232448, "dQ kernel shared memory budget");
 
@@ -1354,7 +1360,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
   uint64_t* k_empty = k_full + kDqKStages;         // [kDqKStages]
   uint64_t* acc_full = k_empty + kDqKStages;       // [2]
   uint64_t* acc_empty = acc_full + 2;              // [2]
-  uint64_t* drained = acc_empty + 2;
+  uint64_t* dot_ready = acc_empty + 2;             // [2]
+  uint64_t* drained = dot_ready + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drained + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -1373,7 +1380,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       tc::mbar_init(&acc_full[i], 1);
-      tc::mbar_init(&acc_empty[i], 128);
+      tc::mbar_init(&acc_empty[i], 256);
+      tc::mbar_init(&dot_ready[i], 256);
     }
     tc::mbar_init(drained, 1);
     *abort_flag = 0;
@@ -1476,86 +1484,97 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       drain_wait(drained, 0);
     }
   } else {
-    // Epilogue: one query row per thread (warp w reaches TMEM lanes of quarter w % 4).
+    // Epilogue: warps 2..9, a TMEM lane quarter each (warp % 4) and one side
+    // of the row's RoPE pairs ((warp - 2) / 4).
     const int qw = warp & 3;
+    const int side = (warp - 2) >> 2;
     const int row = qw * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
+    float* dots = reinterpret_cast<float*>(smem + DQ_OFF_DOT);
     int item = 0;
     for (int w = blockIdx.x; w < nitems; w += gridDim.x, ++item) {
       const DqItem m = dq_item(a, w, window);
       const int buf = item & 1;
       const uint32_t acc = lane_base + 128 * buf;
-      bool ok = tc::mbar_wait(&acc_full[buf], (item >> 1) & 1, abort_flag, a.status);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc::tc_fence_after();
       const int q = m.qi * BQB + row;
       const bool live = q < a.T;
       const int64_t tok = (int64_t)m.b * a.T + (live ? q : 0);
-      const __nv_bfloat16* yrow = a.yhat + tok * a.ldy + m.h * HD;
-      // 32 dims of yhat starting at dim 32 c.
-      auto load_y = [&](int c, float (&y)[32]) {
+      // Everything the row needs besides the accumulator, loaded before it
+      // is waited for: the saved normalised q (dims 32 side + [0, 32) and
+      // 64 + 32 side + [0, 32)), 1/rms and the 32 pairs' (cos, sin).
+      const __nv_bfloat16* yrow = a.yhat + tok * a.ldy + m.h * HD + 32 * side;
+      uint4 yv[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const uint4 v = live ? reinterpret_cast<const uint4*>(yrow + 32 * c)[u]
-                               : make_uint4(0u, 0u, 0u, 0u);
-          const uint32_t vs[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = unpack_bf16x2(vs[e]);
-            y[8 * u + 2 * e] = f.x;
-            y[8 * u + 2 * e + 1] = f.y;
-          }
-        }
-      };
-      float dot = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t g[32];
-        float y[32];
-        tc::tmem_ld_32x32b_x32(acc + 32 * c, g);
-        load_y(c, y);
-        tc::tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) dot = fmaf(__uint_as_float(g[i]), y[i], dot);
+      for (int u = 0; u < 4; ++u) {
+        yv[u] = live ? reinterpret_cast<const uint4*>(yrow)[u] : make_uint4(0u, 0u, 0u, 0u);
+        yv[4 + u] = live ? reinterpret_cast<const uint4*>(yrow + 64)[u] : make_uint4(0u, 0u, 0u, 0u);
       }
       const float r = live ? a.rstd_q[tok * a.H + m.h] : 0.f;
-      const float mean = dot * a.scale / 128.f;
-      __nv_bfloat16* dst = a.out + tok * a.ldo + m.h * HD;
-      const float2* cs = a.rope_tab + (int64_t)(live ? q : 0) * 64;
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        uint32_t g0[32], g1[32];
-        float y0[32], y1[32];
-        tc::tmem_ld_32x32b_x32(acc + 32 * c, g0);
-        tc::tmem_ld_32x32b_x32(acc + 64 + 32 * c, g1);
-        load_y(c, y0);
-        load_y(c + 2, y1);
+      const float4* cs4 = reinterpret_cast<const float4*>(a.rope_tab + (int64_t)(live ? q : 0) * 64 + 32 * side);
+      float4 cs[16];  // pairs 32 side + 2 i, + 2 i + 1: (cos, sin, cos, sin)
+#pragma unroll
+      for (int i = 0; i < 16; ++i) cs[i] = cs4[i];
+      bool ok = tc::mbar_wait(&acc_full[buf], (item >> 1) & 1, abort_flag, a.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc::tc_fence_after();
+      // yhat element j of half hh (j < 32) from the packed row.
+      auto yel = [&](int hh, int j) -> float {
+        const uint4 v = yv[4 * hh + (j >> 3)];
+        const uint32_t wv = (j & 7) < 2 ? v.x : (j & 7) < 4 ? v.y : (j & 7) < 6 ? v.z : v.w;
+        const float2 f = unpack_bf16x2(wv);
+        return (j & 1) ? f.y : f.x;
+      };
+      float dot = 0.f;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t g[16];
+          tc::tmem_ld_32x32b_x16(acc + 64 * hh + 32 * side + 16 * c, g);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) dot = fmaf(__uint_as_float(g[i]), yel(hh, 16 * c + i), dot);
+        }
+      // The row's two halves of sum(g yhat) meet in shared memory.
+      float* dslot = dots + buf * 256;
+      dslot[side * 128 + row] = dot;
+      tc::mbar_arrive(&dot_ready[buf]);
+      ok = tc::mbar_wait(&dot_ready[buf], (item >> 1) & 1, abort_flag, a.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const float mean = (dslot[row] + dslot[128 + row]) * a.scale / 128.f;
+      __nv_bfloat16* dst = a.out + tok * a.ldo + m.h * HD + 32 * side;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {  // pairs 32 side + 16 c + [0, 16)
+        uint32_t g0[16], g1[16];
+        tc::tmem_ld_32x32b_x16(acc + 32 * side + 16 * c, g0);
+        tc::tmem_ld_32x32b_x16(acc + 64 + 32 * side + 16 * c, g1);
         tc::tmem_ld_wait();
         if (c == 1) {  // the accumulator is read: the MMA warp may reuse it
           tc::tc_fence_before();
           tc::mbar_arrive(&acc_empty[buf]);
         }
-        if (live) {
-          uint32_t lo_[16], hi_[16];
+        uint32_t lo_[8], hi_[8];
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float o_lo[2], o_hi[2];
+        for (int i = 0; i < 16; i += 2) {
+          const float4 t4 = cs[(16 * c + i) / 2];
+          const float cc[2] = {t4.x, t4.z}, sn[2] = {t4.y, t4.w};
+          float o_lo[2], o_hi[2];
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const float d0 = r * (__uint_as_float(g0[i + e]) * a.scale - y0[i + e] * mean);
-              const float d1 = r * (__uint_as_float(g1[i + e]) * a.scale - y1[i + e] * mean);
-              const float2 tt = cs[32 * c + i + e];  // (cos, sin) of pair 32 c + i + e
-              o_lo[e] = d0 * tt.x + d1 * tt.y;
-              o_hi[e] = d1 * tt.x - d0 * tt.y;
-            }
-            lo_[i / 2] = pack_bf16x2(o_lo[0], o_lo[1]);
-            hi_[i / 2] = pack_bf16x2(o_hi[0], o_hi[1]);
+          for (int e = 0; e < 2; ++e) {
+            const float d0 = r * (__uint_as_float(g0[i + e]) * a.scale - yel(0, 16 * c + i + e) * mean);
+            const float d1 = r * (__uint_as_float(g1[i + e]) * a.scale - yel(1, 16 * c + i + e) * mean);
+            o_lo[e] = d0 * cc[e] + d1 * sn[e];
+            o_hi[e] = d1 * cc[e] - d0 * sn[e];
           }
+          lo_[i / 2] = pack_bf16x2(o_lo[0], o_lo[1]);
+          hi_[i / 2] = pack_bf16x2(o_hi[0], o_hi[1]);
+        }
+        if (live) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            reinterpret_cast<uint4*>(dst + 32 * c)[u] =
+          for (int u = 0; u < 2; ++u) {
+            reinterpret_cast<uint4*>(dst + 16 * c)[u] =
                 make_uint4(lo_[4 * u], lo_[4 * u + 1], lo_[4 * u + 2], lo_[4 * u + 3]);
-            reinterpret_cast<uint4*>(dst + 64 + 32 * c)[u] =
+            reinterpret_cast<uint4*>(dst + 64 + 16 * c)[u] =
                 make_uint4(hi_[4 * u], hi_[4 * u + 1], hi_[4 * u + 2], hi_[4 * u + 3]);
           }
         }
