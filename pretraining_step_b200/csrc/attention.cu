@@ -83,8 +83,7 @@ __global__ void __launch_bounds__(256) attn_bwd_delta_kernel(const __nv_bfloat16
 nc_status attention_bwd_ex(const void* q, int64_t ldq, const void* k, const void* v, int64_t ldkv,
                            const void* o, const void* dout, int64_t ldo, const float* lse,
                            float* dq, void* dk, void* dv, int64_t ldg, float* delta, int B, int T,
-                           int H, int Hkv, int window, const float2* rope_tab, const float* rstd_k,
-                           int* status, cudaStream_t s, Profiler* prof) {
+                           int H, int Hkv, int window, int* status, cudaStream_t s, Profiler* prof) {
   if (B < 1 || T < 1 || H < 1 || Hkv < 1 || H % Hkv || !q || !k || !v || !o || !dout || !lse ||
       !dq || !dk || !dv || !delta)
     return fail(NC_ERR_INVALID_ARG, "attention_bwd: bad arguments (H must be a multiple of Hkv)");
@@ -102,17 +101,18 @@ nc_status attention_bwd_ex(const void* q, int64_t ldq, const void* k, const void
   }
   NC_CUDA_TRY(cudaMemsetAsync(dq, 0, sizeof(float) * rows * HD, s));
   return attention_bwd_tc_ex(q, ldq, k, v, ldkv, dout, ldo, lse, delta, dq, dk, dv, ldg, B, T, H,
-                             Hkv, window, rope_tab, rstd_k, nullptr, 0, status, s, prof);
+                             Hkv, window, nullptr, 0, nullptr, nullptr, 0, status, s, prof);
 }
 
 nc_status attention_bwd_model(const void* q, int64_t ldq, const void* k, const void* v,
                               int64_t ldkv, const void* o, const void* dout, int64_t ldo,
                               const float* lse, float* delta, void* ds, int64_t ld_ds,
                               void* dq_out, void* dk, void* dv, int64_t ldg, int B, int T, int H,
-                              int Hkv, int window, const float2* rope_tab, const float* rstd_q,
-                              const float* rstd_k, int* status, cudaStream_t s, Profiler* prof) {
+                              int Hkv, int window, const float2* rope_tab, int rope_T,
+                              const float* rstd_q, const float* rstd_k, int* status, cudaStream_t s,
+                              Profiler* prof) {
   if (B < 1 || T < 1 || H < 1 || Hkv < 1 || H % Hkv || H > kDeltaMaxH || !o || !dout || !delta ||
-      !ds || !rope_tab || !rstd_q || !rstd_k)
+      !ds || !rope_tab || rope_T < T || !rstd_q || !rstd_k)
     return fail(NC_ERR_INVALID_ARG, "attention_bwd_model: bad arguments");
   if (ldo % 8 || ((reinterpret_cast<uintptr_t>(o) | reinterpret_cast<uintptr_t>(dout)) & 15))
     return fail(NC_ERR_INVALID_ARG, "attention_bwd_model: O and dO rows must be 16-byte aligned");
@@ -124,9 +124,9 @@ nc_status attention_bwd_model(const void* q, int64_t ldq, const void* k, const v
     NC_CUDA_TRY(cudaGetLastError());
   }
   NC_TRY(attention_bwd_tc_ex(q, ldq, k, v, ldkv, dout, ldo, lse, delta, nullptr, dk, dv, ldg, B, T,
-                             H, Hkv, window, rope_tab, rstd_k, ds, ld_ds, status, s, prof));
-  return attention_dq_ex(ds, ld_ds, k, ldkv, B, T, H, Hkv, window, q, ldq, rstd_q, rope_tab, dq_out,
-                         ldg, status, s, prof);
+                             H, Hkv, window, rope_tab, rope_T, rstd_k, ds, ld_ds, status, s, prof));
+  return attention_dq_ex(ds, ld_ds, k, ldkv, B, T, H, Hkv, window, q, ldq, rstd_q, rope_tab, rope_T,
+                         dq_out, ldg, status, s, prof);
 }
 
 nc_status attention_bwd(const void* q, const void* k, const void* v, int64_t ld, const void* o,
@@ -134,7 +134,7 @@ nc_status attention_bwd(const void* q, const void* k, const void* v, int64_t ld,
                         void* dv, int64_t ldg, float* delta, int B, int T, int H, int* status,
                         cudaStream_t s, Profiler* prof) {
   return attention_bwd_ex(q, ld, k, v, ld, o, dout, ldo, lse, dq, dk, dv, ldg, delta, B, T, H, H, -1,
-                          nullptr, nullptr, status, s, prof);
+                          status, s, prof);
 }
 
 // ------------------------------------------------------------------ allocation-free backward

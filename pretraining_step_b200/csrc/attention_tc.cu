@@ -724,22 +724,23 @@ struct BwdArgs {
   __nv_bfloat16* dv;
   int64_t ldg;
   int* status;
-  // Non-null: dK leaves through the backward of the k-side RoPE + QK-norm
-  // (the forward applies them in the q|k|v projection's epilogue), using
-  // the saved normalised k (the K operand itself), rstd_k [B*T, Hkv] and
-  // the cos/sin table [T][64].
+  int B;
+  // Persistent key-side kernel: dK leaves through the backward of the k-side
+  // RoPE + QK-norm (the forward applies them in the q|k|v projection's
+  // epilogue), using the saved normalised k (the K operand itself), rstd_k
+  // [B*T, Hkv] and the cos/sin table (rope_table()'s buffer).
   const float2* rope_tab;
+  int rope_T;  // positions of the table (its grouped copy starts at rope_tab + rope_T * 64)
   const float* rstd_k;
   int Hkv;
 };
 
 // GW: grouped KV heads or a window in play; the plain instance compiles
 // with group 1 and no window as constants (its tile t is query tile i0 + t
-// of head hk).  SDS: instead of the dQ product, every dS^T tile goes to
-// global memory (tdq is then the map of the bf16 dS^T buffer [B*H][T keys][T
-// queries]) for the query-side kernel (attn_dq_kernel) to contract with K;
-// warp 10 issues those stores and the other dQ warps have nothing to do.
-template <bool GW, bool SDS>
+// of head hk).  This form computes dQ itself (fp32, TMA bulk reductions);
+// the model's backward uses the persistent key-side kernel and the dQ
+// kernel instead.
+template <bool GW>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
@@ -794,9 +795,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tc::mbar_init(p_full, 256);
     tc::mbar_init(dp_full, 1);
     tc::mbar_init(ds_full, 256);
-    // One lane of each dQ warp once its staging is read; with SDS the lane
-    // that stored the tile.
-    tc::mbar_init(ds_empty, SDS ? 1 : 4);
+    // One lane of each dQ warp once its staging is read.
+    tc::mbar_init(ds_empty, 4);
     tc::mbar_init(dq_full, 1);
     tc::mbar_init(dq_empty, 128);
     tc::mbar_init(dkv_full, 1);
@@ -946,22 +946,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc::umma_bf16_ts(tmem + TB_DK, tmem + TB_DP + (kk >> 2) * 64 + (kk & 3) * 8,
                            tc::desc_add(qmn, kk * 2048), id_ts, (t > 0 || kk > 0) ? 1u : 0u);
         tc::umma_commit(&q_empty[st]);
-        if (!SDS) {
-          // dQ = dS K (one query per TMEM lane): key step kk (16 keys) is 2 KB
-          // into both MN-major tiles.
+        // dQ = dS K (one query per TMEM lane): key step kk (16 keys) is 2 KB
+        // into both MN-major tiles.
 #pragma unroll
-          for (int kk = 0; kk < BKV / 16; ++kk)
-            tc::umma_bf16_ss(tmem + TB_DP, tc::desc_add(dsMN, kk * 2048),
-                             tc::desc_add(kMN, kk * 2048), id_dq, kk > 0 ? 1u : 0u);
-          tc::umma_commit(dq_full);
-        }
+        for (int kk = 0; kk < BKV / 16; ++kk)
+          tc::umma_bf16_ss(tmem + TB_DP, tc::desc_add(dsMN, kk * 2048),
+                           tc::desc_add(kMN, kk * 2048), id_dq, kk > 0 ? 1u : 0u);
+        tc::umma_commit(dq_full);
         if (t + 1 < nblk) {
-          if (!SDS) {
-            if (!tc::mbar_wait(dq_empty, t & 1, abort_flag, a.status)) { ok = false; break; }
-            tc::tc_fence_after();
-          }
-          // With SDS the DP columns are free once dK (issued just before) has
-          // read dS^T from them: the MMAs run in issue order.
+          if (!tc::mbar_wait(dq_empty, t & 1, abort_flag, a.status)) { ok = false; break; }
+          tc::tc_fence_after();
           if (!issue_dp(t + 1)) { ok = false; break; }
         }
       }
@@ -1082,81 +1076,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = tc::mbar_wait(dkv_full, 0, abort_flag, a.status);
       ok = __all_sync(0xffffffffu, ok);
     }
-    if (ok && hf == 1 && a.rope_tab) {
-      // dK through the RoPE + QK-norm backward: with g = dK, yhat the saved
-      // normalised k (this CTA's K tile) and r its 1/rms,
-      //   dr = r (g - yhat mean(g yhat)),  dk = R(-theta) dr  (pairs i, i + 64).
-      tc::tc_fence_after();
-      const uint32_t krow = tc::smem_u32(smem + B_OFF_K) + row * 128;
-      // 32 dims of yhat: chunk c is box c / 2, 16-byte units 4 (c % 2) .. + 3.
-      auto load_y = [&](int c, float (&y)[32]) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const uint4 w = tc::ld_shared_v4(krow + (c >> 1) * (TILE / 2) +
-                                           ((((c & 1) * 4 + u) ^ (row & 7)) << 4));
-          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = unpack_bf16x2(ws[e]);
-            y[8 * u + 2 * e] = f.x;
-            y[8 * u + 2 * e + 1] = f.y;
-          }
-        }
-      };
-      float dot = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t g[32];
-        float y[32];
-        tc::tmem_ld_32x32b_x32(lane_base + TB_DK + 32 * c, g);
-        load_y(c, y);
-        tc::tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) dot = fmaf(__uint_as_float(g[i]), y[i], dot);
-      }
-      // Keys at or past T (a ragged last tile) take part in the warp-wide
-      // TMEM loads but read and write nothing in global memory.
-      const bool live = key < a.T;
-      const int64_t tok = (int64_t)b * a.T + (live ? key : 0);
-      const float r = live ? a.rstd_k[tok * a.Hkv + hk] : 0.f;
-      const float m = dot * a.scale / 128.f;
-      __nv_bfloat16* dst = a.dk + tok * a.ldg + kcol0;
-      const float2* cs = a.rope_tab + (int64_t)(live ? key : 0) * 64;
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        uint32_t g0[32], g1[32];
-        float y0[32], y1[32];
-        tc::tmem_ld_32x32b_x32(lane_base + TB_DK + 32 * c, g0);
-        tc::tmem_ld_32x32b_x32(lane_base + TB_DK + 64 + 32 * c, g1);
-        load_y(c, y0);
-        load_y(c + 2, y1);
-        tc::tmem_ld_wait();
-        if (live) {
-          uint32_t lo[16], hi[16];
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float o_lo[2], o_hi[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const float d0 = r * (__uint_as_float(g0[i + e]) * a.scale - y0[i + e] * m);
-              const float d1 = r * (__uint_as_float(g1[i + e]) * a.scale - y1[i + e] * m);
-              const float2 t = cs[32 * c + i + e];  // (cos, sin) of pair 32 c + i + e
-              o_lo[e] = d0 * t.x + d1 * t.y;
-              o_hi[e] = d1 * t.x - d0 * t.y;
-            }
-            lo[i / 2] = pack_bf16x2(o_lo[0], o_lo[1]);
-            hi[i / 2] = pack_bf16x2(o_hi[0], o_hi[1]);
-          }
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            reinterpret_cast<uint4*>(dst + 32 * c)[u] =
-                make_uint4(lo[4 * u], lo[4 * u + 1], lo[4 * u + 2], lo[4 * u + 3]);
-            reinterpret_cast<uint4*>(dst + 64 + 32 * c)[u] =
-                make_uint4(hi[4 * u], hi[4 * u + 1], hi[4 * u + 2], hi[4 * u + 3]);
-          }
-        }
-      }
-    } else if (ok) {
+    if (ok) {
       // Warps of query half 0 write dV rows, those of half 1 dK rows.
       tc::tc_fence_after();
       const int64_t grow = ((int64_t)b * a.T + key) * a.ldg + kcol0;
@@ -1182,23 +1102,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
   } else {
-    if (SDS) {
-      // ---------------- dS^T tiles to global memory (one lane of warp 10)
-      if (warp == 10 && lane == 0) {
-        for (int t = 0; t < nblk; ++t) {
-          const int q0 = (i0 + (GW ? t % nqt : t)) * BQB;
-          const int hq = GW ? hk * group + t / nqt : hk;
-          if (!tc::mbar_wait(ds_full, t & 1, abort_flag, a.status)) break;
-          for (int c = 0; c < 2; ++c)
-            tc::tma_store_3d(&tdq, tc::smem_u32(smem + B_OFF_DS) + c * (TILE / 2), q0 + 64 * c,
-                             kb * BKV, b * a.H + hq);
-          tc::bulk_commit_group();
-          tc::bulk_wait_group_read0();  // the tile may be rewritten once read
-          tc::mbar_arrive(ds_empty);
-        }
-        tc::bulk_wait_group0();
-      }
-    } else {
     // ---------------- dQ rows: one query per thread, TMA bulk reductions into dq
     const int qw = warp & 3;
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
@@ -1250,7 +1153,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       __syncwarp();
     }
     if (pending && lane == 0) tc::bulk_wait_group0();
-    }
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -1261,10 +1163,622 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 
+// ------------------------------------------------------------------ key side, persistent
+// The key-side backward of the split form as a persistent kernel: one CTA
+// per SM walks work items (128-key tile, KV head, batch row) in balanced
+// pairs (KvCursor).  Per item it accumulates dV and dK in TMEM
+// over the query tiles (and query heads of the KV head's group) that reach
+// its keys, exactly as the one-item-per-CTA form does, and stores every dS^T
+// tile for the query-side kernel; in addition the tile pipeline runs on
+// across item boundaries:
+//   * K and V of the next item are loaded as soon as the MMAs that read the
+//     current ones (the item's last S^T and dP^T) are done, so the next
+//     item's first scores follow the current item's last ones directly;
+//   * the dV / dK epilogue (k-side RoPE + QK-norm backward included) runs on
+//     warps of its own while the next item's tiles are processed; the MMA
+//     warp only waits for it before the next item's first dV and dK
+//     products, which overwrite the accumulators.
+// 512 threads (128 registers each), four warps per role group so that each
+// group's warps cover the four TMEM lane quarters:
+//   warp 0      TMA: K and V per item, Q_i and dO_i of every tile (two stages
+//               each), lse * log2(e) and D staged by all its lanes;
+//   warp 1      TMEM owner and single-thread MMA issue (products as in the
+//               one-item-per-CTA form);
+//   warp 2      one lane stores each dS^T tile (TMA) once the softmax warps
+//               have written it to shared memory; warp 3 idles;
+//   warps 4..11 P^T and dS^T, two threads per key row;
+//   warps 12..15 epilogue, one key row per thread: the row of yhat (the
+//               normalised k, the K operand itself) is copied from shared
+//               memory while the item runs, so K's buffer can take the next
+//               item; at the item's end dV goes out, then dK through
+//               dr = r (g - yhat mean(g yhat)), dk = R(-theta) dr.
+constexpr int kKvThreads = 512;
+constexpr int KV_OFF_TI = B_OFF_BAR;        // [2 stages] (first query, key tile) of the tile
+constexpr int KV_OFF_BAR = KV_OFF_TI + 64;
+constexpr int kKvSmem = KV_OFF_BAR + 256;
+static_assert(kKvSmem <= 232448, "persistent key-side shared memory budget");
+
+// Work item: key tile, KV head, batch row, and its tile count.
+struct KvItem {
+  int kb, hk, b, nqt, nblk;
+};
+
+// This CTA's work items in order.  Items come in pairs of one (KV head,
+// row): key tile j, then key tile nkb - 1 - j.  Under the causal mask the
+// pair's tile counts add up to nqb + 1 whatever j is, so dealing pair p to
+// CTA p mod gridDim.x balances the work; the pairs of one (KV head, row) are
+// consecutive, so the CTAs working at the same time read the same Q and dO
+// tiles, which then come from L2.  t is the tile of the current item and n
+// counts the items walked.
+struct KvCursor {
+  int p, sub, n, t;
+  bool valid;
+  KvItem m;
+  __device__ __forceinline__ void load(const BwdArgs& a, int npairs, int group, int window) {
+    valid = p < npairs;
+    if (!valid) return;
+    const int ppg = (a.nkb + 1) / 2;
+    const int grp = p / ppg;
+    const int j = p - grp * ppg;
+    m.kb = sub ? a.nkb - 1 - j : j;
+    m.hk = grp % a.Hkv;
+    m.b = grp / a.Hkv;
+    const int i_hi = window < 0 ? a.nqb - 1 : min(a.nqb - 1, (m.kb * BKV + BKV - 1 + window) / BQB);
+    m.nqt = i_hi - m.kb + 1;
+    m.nblk = group * m.nqt;
+  }
+  __device__ __forceinline__ void start(const BwdArgs& a, int npairs, int group, int window) {
+    p = blockIdx.x;
+    sub = 0;
+    n = 0;
+    t = 0;
+    load(a, npairs, group, window);
+  }
+  __device__ __forceinline__ void next_item(const BwdArgs& a, int npairs, int group, int window) {
+    const int j = p % ((a.nkb + 1) / 2);
+    if (sub == 0 && a.nkb - 1 - j != j) {
+      sub = 1;
+    } else {
+      sub = 0;
+      p += gridDim.x;
+    }
+    ++n;
+    t = 0;
+    load(a, npairs, group, window);
+  }
+  __device__ __forceinline__ void next(const BwdArgs& a, int npairs, int group, int window) {
+    if (++t == m.nblk) next_item(a, npairs, group, window);
+  }
+  // Query head and first query of the current tile.
+  __device__ __forceinline__ int hq(int group) const { return m.hk * group + t / m.nqt; }
+  __device__ __forceinline__ int q0() const { return (m.kb + t % m.nqt) * BQB; }
+};
+
+// Tiles of all this CTA's items.
+__device__ __forceinline__ int kv_tiles_total(const BwdArgs& a, int npairs, int group, int window) {
+  KvCursor c;
+  int total = 0;
+  for (c.start(a, npairs, group, window); c.valid; c.next_item(a, npairs, group, window)) total += c.m.nblk;
+  return total;
+}
+
+template <bool GW>
+__global__ void __launch_bounds__(kKvThreads)
+    attn_bwd_kv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                       const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
+                       const __grid_constant__ CUtensorMap tds, const BwdArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if ((tc::smem_u32(smem_raw) & 1023u) != 0) {  // never expected; no room to realign
+    if (threadIdx.x == 0 && a.status) atomicExch(a.status, kDevTimeout);
+    return;
+  }
+  uint8_t* smem = smem_raw;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + KV_OFF_BAR);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* kv_empty = bars + 1;   // the item's MMAs have read K and V
+  uint64_t* k_copied = bars + 2;   // the epilogue has copied its yhat rows
+  uint64_t* q_full = bars + 3;     // [2]
+  uint64_t* q_empty = bars + 5;    // [2]
+  uint64_t* do_full = bars + 7;    // [2]
+  uint64_t* do_empty = bars + 9;   // [2]
+  uint64_t* s_full = bars + 11;
+  uint64_t* p_full = bars + 12;
+  uint64_t* dp_full = bars + 13;
+  uint64_t* ds_full = bars + 14;
+  uint64_t* ds_empty = bars + 15;
+  uint64_t* dkv_full = bars + 16;  // the item's dV and dK are final
+  uint64_t* dv_empty = bars + 17;  // the epilogue has read dV
+  uint64_t* dk_empty = bars + 18;  // ... and dK
+  uint64_t* drained = bars + 19;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 20);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int group = GW ? a.group : 1;
+  const int window = GW ? a.window : -1;
+  const int npairs = (a.nkb + 1) / 2 * a.Hkv * a.B;
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(kv_full, 1);
+    tc::mbar_init(kv_empty, 1);
+    tc::mbar_init(k_copied, 128);
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&q_full[i], 32);  // the TMA lane (with its bytes) + 31 staging lanes
+      tc::mbar_init(&q_empty[i], 1);
+      tc::mbar_init(&do_full[i], 32);
+      tc::mbar_init(&do_empty[i], 1);
+    }
+    tc::mbar_init(s_full, 1);
+    tc::mbar_init(p_full, 256);
+    tc::mbar_init(dp_full, 1);
+    tc::mbar_init(ds_full, 256);
+    tc::mbar_init(ds_empty, 1);
+    tc::mbar_init(dkv_full, 1);
+    tc::mbar_init(dv_empty, 128);
+    tc::mbar_init(dk_empty, 128);
+    tc::mbar_init(drained, 1);
+    *abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // Lane 0 issues the TMA copies; all 32 lanes stage lse * log2(e) (with Q)
+    // and D (with dO) of the query tile and arrive on the same barriers.
+    if (lane == 0) {
+      tc::tma_prefetch_desc(&tq);
+      tc::tma_prefetch_desc(&tk);
+      tc::tma_prefetch_desc(&tv);
+      tc::tma_prefetch_desc(&tdo);
+      tc::tma_prefetch_desc(&tds);
+    }
+    KvCursor c;
+    c.start(a, npairs, group, window);
+    int issued_q = 0, issued_do = 0, issued_kv = 0;
+    bool ok = true;
+    for (int g = 0; c.valid; ++g) {
+      const int st = g & 1;
+      const uint32_t ph = (g >> 1) & 1;
+      bool w = true;
+      if (c.t == 0) {
+        // K and V of the item, once the previous item's MMAs have read them
+        // and the epilogue has copied its yhat rows.
+        if (lane == 0 && c.n > 0)
+          w = tc::mbar_wait(kv_empty, (c.n - 1) & 1, abort_flag, a.status) &&
+              tc::mbar_wait(k_copied, (c.n - 1) & 1, abort_flag, a.status);
+        if (!__shfl_sync(0xffffffffu, (int)w, 0)) { ok = false; break; }
+        if (lane == 0) {
+          tc::mbar_arrive_expect_tx(kv_full, 2 * TILE);
+          for (int h = 0; h < 2; ++h) {
+            tc::tma_load_3d(smem + B_OFF_K + h * (TILE / 2), &tk, kv_full, c.m.hk * HD + 64 * h,
+                            c.m.kb * BKV, c.m.b);
+            tc::tma_load_3d(smem + B_OFF_V + h * (TILE / 2), &tv, kv_full, c.m.hk * HD + 64 * h,
+                            c.m.kb * BKV, c.m.b);
+          }
+        }
+        ++issued_kv;
+      }
+      const int hq = GW ? c.hq(group) : c.m.hk;
+      const int q0 = GW ? c.q0() : (c.m.kb + c.t) * BQB;
+      const int qcol0 = hq * HD;
+      if (lane == 0) w = tc::mbar_wait(&q_empty[st], ph ^ 1, abort_flag, a.status);
+      if (!__shfl_sync(0xffffffffu, (int)w, 0)) { ok = false; break; }
+      const float* lse_bh = a.lse + ((int64_t)c.m.b * a.H + hq) * a.T;
+      float* lq = reinterpret_cast<float*>(smem + B_OFF_LQ) + st * BQB;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int q = q0 + lane + 32 * u;
+        lq[lane + 32 * u] = q < a.T ? lse_bh[q] * 1.4426950408889634f : INFINITY;
+      }
+      if (lane == 0) {
+        reinterpret_cast<int2*>(smem + KV_OFF_TI)[st] = make_int2(q0, c.m.kb);
+        tc::mbar_arrive_expect_tx(&q_full[st], TILE);
+        for (int h = 0; h < 2; ++h)
+          tc::tma_load_3d(smem + B_OFF_Q + st * TILE + h * (TILE / 2), &tq, &q_full[st], qcol0 + 64 * h,
+                          q0, c.m.b);
+      } else {
+        tc::mbar_arrive(&q_full[st]);
+      }
+      ++issued_q;
+      if (lane == 0) w = tc::mbar_wait(&do_empty[st], ph ^ 1, abort_flag, a.status);
+      if (!__shfl_sync(0xffffffffu, (int)w, 0)) { ok = false; break; }
+      const float* d_bh = a.delta + ((int64_t)c.m.b * a.H + hq) * a.T;
+      float* ldd = reinterpret_cast<float*>(smem + B_OFF_LD) + st * BQB;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int q = q0 + lane + 32 * u;
+        ldd[lane + 32 * u] = q < a.T ? d_bh[q] : 0.f;
+      }
+      if (lane == 0) {
+        tc::mbar_arrive_expect_tx(&do_full[st], TILE);
+        for (int h = 0; h < 2; ++h)
+          tc::tma_load_3d(smem + B_OFF_DO + st * TILE + h * (TILE / 2), &tdo, &do_full[st],
+                          qcol0 + 64 * h, q0, c.m.b);
+      } else {
+        tc::mbar_arrive(&do_full[st]);
+      }
+      ++issued_do;
+      c.next(a, npairs, group, window);
+    }
+    if (!ok && lane == 0) {
+      if (issued_kv > 0) drain_wait(kv_full, (issued_kv - 1) & 1);
+      for (int t = max(0, issued_q - 2); t < issued_q; ++t) drain_wait(&q_full[t & 1], (t >> 1) & 1);
+      for (int t = max(0, issued_do - 2); t < issued_do; ++t) drain_wait(&do_full[t & 1], (t >> 1) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id_ss = tc::idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
+      const uint32_t id_ts = tc::idesc_bf16_f32(128, 128, 0, 1);  // dV, dK: A from TMEM
+      const uint64_t kK = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_K), 16, 1024);
+      const uint64_t vK = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_V), 16, 1024);
+      const uint64_t qK = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_Q), 16, 1024);
+      const uint64_t doK = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_DO), 16, 1024);
+      const uint64_t qMN = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_Q), TILE / 2, 1024);
+      const uint64_t doMN = tc::smem_desc_sw128(tc::smem_u32(smem + B_OFF_DO), TILE / 2, 1024);
+      // S^T of tile g once its Q has landed; the S columns are free because
+      // every earlier MMA that reads them (dV of tile g - 1) was issued first.
+      auto issue_s = [&](int g) -> bool {
+        const int st = g & 1;
+        if (!tc::mbar_wait(&q_full[st], (g >> 1) & 1, abort_flag, a.status)) return false;
+        tc::tc_fence_after();
+        const uint64_t qd = tc::desc_add(qK, st * TILE);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (TILE / 2) + (kk & 3) * 32;
+          tc::umma_bf16_ss(tmem + TB_S, tc::desc_add(kK, off), tc::desc_add(qd, off), id_ss,
+                           kk > 0 ? 1u : 0u);
+        }
+        tc::umma_commit(s_full);
+        return true;
+      };
+      // dP^T of tile g once its dO has landed (the DP columns are free: dK of
+      // tile g - 1, which reads dS^T from them, was issued first).
+      auto issue_dp = [&](int g) -> bool {
+        const int st = g & 1;
+        if (!tc::mbar_wait(&do_full[st], (g >> 1) & 1, abort_flag, a.status)) return false;
+        tc::tc_fence_after();
+        const uint64_t dod = tc::desc_add(doK, st * TILE);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (TILE / 2) + (kk & 3) * 32;
+          tc::umma_bf16_ss(tmem + TB_DP, tc::desc_add(vK, off), tc::desc_add(dod, off), id_ss,
+                           kk > 0 ? 1u : 0u);
+        }
+        tc::umma_commit(dp_full);
+        return true;
+      };
+      KvCursor c, nx;
+      c.start(a, npairs, group, window);
+      bool ok = c.valid && tc::mbar_wait(kv_full, 0, abort_flag, a.status);
+      if (ok) ok = issue_s(0) && issue_dp(0);
+      // The item's last S^T and dP^T have been issued: K and V are free once
+      // they complete.
+      if (ok && c.m.nblk == 1) tc::umma_commit(kv_empty);
+      for (int g = 0; c.valid && ok; ++g) {
+        const int st = g & 1;
+        nx = c;
+        nx.next(a, npairs, group, window);
+        if (!tc::mbar_wait(p_full, g & 1, abort_flag, a.status)) { ok = false; break; }
+        // The first product of an item overwrites dV: the epilogue must have
+        // read the previous item's.
+        if (c.t == 0 && c.n > 0 && !tc::mbar_wait(dv_empty, (c.n - 1) & 1, abort_flag, a.status)) {
+          ok = false;
+          break;
+        }
+        tc::tc_fence_after();
+        // dV += P^T dO: query step kk (16 queries) is 8 packed columns of the
+        // softmax half that owns it (half h at column 64 h).
+        const uint64_t domn = tc::desc_add(doMN, st * TILE);
+#pragma unroll
+        for (int kk = 0; kk < BQB / 16; ++kk)
+          tc::umma_bf16_ts(tmem + TB_DV, tmem + TB_S + (kk >> 2) * 64 + (kk & 3) * 8,
+                           tc::desc_add(domn, kk * 2048), id_ts, (c.t > 0 || kk > 0) ? 1u : 0u);
+        tc::umma_commit(&do_empty[st]);
+        if (nx.valid) {
+          if (nx.t == 0 && !tc::mbar_wait(kv_full, nx.n & 1, abort_flag, a.status)) { ok = false; break; }
+          if (!issue_s(g + 1)) { ok = false; break; }
+        }
+        if (!tc::mbar_wait(ds_full, g & 1, abort_flag, a.status)) { ok = false; break; }
+        if (c.t == 0 && c.n > 0 && !tc::mbar_wait(dk_empty, (c.n - 1) & 1, abort_flag, a.status)) {
+          ok = false;
+          break;
+        }
+        tc::tc_fence_after();
+        const uint64_t qmn = tc::desc_add(qMN, st * TILE);
+#pragma unroll
+        for (int kk = 0; kk < BQB / 16; ++kk)
+          tc::umma_bf16_ts(tmem + TB_DK, tmem + TB_DP + (kk >> 2) * 64 + (kk & 3) * 8,
+                           tc::desc_add(qmn, kk * 2048), id_ts, (c.t > 0 || kk > 0) ? 1u : 0u);
+        tc::umma_commit(&q_empty[st]);
+        if (c.t == c.m.nblk - 1) tc::umma_commit(dkv_full);
+        if (nx.valid) {
+          if (!issue_dp(g + 1)) { ok = false; break; }
+          if (nx.t == nx.m.nblk - 1) tc::umma_commit(kv_empty);
+        }
+        c = nx;
+      }
+      tc::umma_commit(drained);
+      drain_wait(drained, 0);
+    }
+  } else if (warp == 2) {
+    // ---------------- dS^T tiles to global memory (one lane of warp 2)
+    if (lane == 0) {
+      KvCursor c;
+      c.start(a, npairs, group, window);
+      bool pending = false;
+      for (int g = 0; c.valid; ++g, c.next(a, npairs, group, window)) {
+        const int q0 = GW ? c.q0() : (c.m.kb + c.t) * BQB;
+        const int hq = GW ? c.hq(group) : c.m.hk;
+        if (!tc::mbar_wait(ds_full, g & 1, abort_flag, a.status)) break;
+        for (int h = 0; h < 2; ++h)
+          tc::tma_store_3d(&tds, tc::smem_u32(smem + B_OFF_DS) + h * (TILE / 2), q0 + 64 * h,
+                           c.m.kb * BKV, c.m.b * a.H + hq);
+        tc::bulk_commit_group();
+        pending = true;
+        tc::bulk_wait_group_read0();  // the tile may be rewritten once read
+        tc::mbar_arrive(ds_empty);
+      }
+      if (pending) tc::bulk_wait_group0();
+    }
+  } else if (warp < 4) {
+    // warp 3: no role
+  } else if (warp < 12) {
+    // ---------------- P^T and dS^T: one key row per thread, half the queries per warp
+    const int qw = warp & 3;
+    const int hf = (warp - 4) >> 2;  // query half: [64 hf, 64 hf + 64) of the tile
+    const int row = qw * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
+    const uint32_t s_col = lane_base + TB_S + 64 * hf;
+    const uint32_t dp_col = lane_base + TB_DP + 64 * hf;
+    const uint32_t ds_row = tc::smem_u32(smem + B_OFF_DS) + hf * (TILE / 2) + row * 128;
+    const int total = kv_tiles_total(a, npairs, group, window);
+    for (int g = 0; g < total; ++g) {
+      const int st = g & 1;
+      const uint32_t ph = (g >> 1) & 1;
+      bool ok = tc::mbar_wait(s_full, g & 1, abort_flag, a.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc::tc_fence_after();
+      // The tile's lse and coordinates, staged by the TMA warp and published
+      // by the stage's q_full barrier (already complete: the scores came
+      // from it).
+      ok = tc::mbar_wait(&q_full[st], ph, abort_flag, a.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const int2 ti = reinterpret_cast<const int2*>(smem + KV_OFF_TI)[st];
+      const int key = ti.y * BKV + row;
+      const int qh = ti.x + 64 * hf;  // first query of this half
+      const float* lq = reinterpret_cast<const float*>(smem + B_OFF_LQ) + st * BQB + 64 * hf;
+      // The half reaches the diagonal, T, or past the window of this key.
+      const bool edge = (qh < key) || (qh + 63 >= a.T) || (key >= a.T) ||
+                        (window >= 0 && qh + 63 > key + window);
+      uint32_t pk[2][16];
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t sv[32];
+        tc::tmem_ld_32x32b_x32(s_col + 32 * cc, sv);
+        // The chunk's 32 lse values as eight 16-byte shared loads, issued
+        // while the scores are in flight.
+        float l[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float4 v = reinterpret_cast<const float4*>(lq + 32 * cc)[u];
+          l[4 * u] = v.x;
+          l[4 * u + 1] = v.y;
+          l[4 * u + 2] = v.z;
+          l[4 * u + 3] = v.w;
+        }
+        tc::tmem_ld_wait();
+        // Every argument first, then the 32 independent exponentials.
+        float p[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) p[i] = fmaf(__uint_as_float(sv[i]), a.sl2, -l[i]);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) p[i] = ex2(p[i]);
+        if (edge) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int qa = qh + 32 * cc + i;
+            if (qa < key || qa >= a.T || key >= a.T || (window >= 0 && qa > key + window)) p[i] = 0.f;
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[cc][i] = pack_bf16x2(p[2 * i], p[2 * i + 1]);
+      }
+      tc::tmem_st_32x32b_x16(s_col, pk[0]);
+      tc::tmem_st_32x32b_x16(s_col + 16, pk[1]);
+      tc::tmem_st_wait();
+      tc::tc_fence_before();
+      tc::mbar_arrive(p_full);
+      // dS^T = P^T (dP^T - D), from the bf16 P the dV product reads.
+      ok = tc::mbar_wait(dp_full, g & 1, abort_flag, a.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc::tc_fence_after();
+      ok = tc::mbar_wait(&do_full[st], ph, abort_flag, a.status);  // D, staged with dO
+      // The shared dS tile is free once the previous tile's store has read it.
+      ok = ok && tc::mbar_wait(ds_empty, (g & 1) ^ 1, abort_flag, a.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const float* ld = reinterpret_cast<const float*>(smem + B_OFF_LD) + st * BQB + 64 * hf;
+      // 32 queries at a time: chunk cc's dS^T goes over the dP^T columns of
+      // queries [16 cc, 16 cc + 16), which chunk 0 has already read.
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t dpv[32];
+        tc::tmem_ld_32x32b_x32(dp_col + 32 * cc, dpv);
+        float dl[32];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float4 v = reinterpret_cast<const float4*>(ld + 32 * cc)[u];
+          dl[4 * u] = v.x;
+          dl[4 * u + 1] = v.y;
+          dl[4 * u + 2] = v.z;
+          dl[4 * u + 3] = v.w;
+        }
+        tc::tmem_ld_wait();
+        uint32_t pd[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float2 p = unpack_bf16x2(pk[cc][i]);
+          const float d0 = p.x * (__uint_as_float(dpv[2 * i]) - dl[2 * i]);
+          const float d1 = p.y * (__uint_as_float(dpv[2 * i + 1]) - dl[2 * i + 1]);
+          pd[i] = pack_bf16x2(d0, d1);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t sw = (uint32_t)(((4 * cc + u) ^ (row & 7)) << 4);
+          tc::st_shared_v4(ds_row + sw, pd[4 * u], pd[4 * u + 1], pd[4 * u + 2], pd[4 * u + 3]);
+        }
+        tc::tmem_st_32x32b_x16(dp_col + 16 * cc, pd);
+      }
+      tc::tmem_st_wait();
+      tc::fence_proxy_async_smem();
+      tc::tc_fence_before();
+      tc::mbar_arrive(ds_full);
+    }
+  } else {
+    // ---------------- epilogue: one key row per thread
+    const int qw = warp & 3;
+    const int row = qw * 32 + lane;
+    const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
+    const uint32_t krow = tc::smem_u32(smem + B_OFF_K) + row * 128;
+    KvCursor c;
+    c.start(a, npairs, group, window);
+    for (; c.valid; c.next_item(a, npairs, group, window)) {
+      const int n = c.n;
+      // yhat of this key row (dims [8 u, 8 u + 8) in yv[u]) while the item runs.
+      bool ok = tc::mbar_wait(kv_full, n & 1, abort_flag, a.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      uint4 yv[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        yv[u] = tc::ld_shared_v4(krow + (u >> 3) * (TILE / 2) + (((u & 7) ^ (row & 7)) << 4));
+      tc::mbar_arrive(k_copied);
+      const int key = c.m.kb * BKV + row;
+      // Keys at or past T (a ragged last tile) take part in the warp-wide
+      // TMEM loads but read and write nothing in global memory.
+      const bool live = key < a.T;
+      const int64_t tok = (int64_t)c.m.b * a.T + (live ? key : 0);
+      const int kcol0 = c.m.hk * HD;
+      const float r = live ? a.rstd_k[tok * a.Hkv + c.m.hk] : 0.f;
+      // (cos, sin) of four consecutive pairs of this key are 32 contiguous
+      // bytes of the grouped table, so a warp's 32 keys read 1 KB at once.
+      const float* csg = reinterpret_cast<const float*>(a.rope_tab + (int64_t)a.rope_T * 64) +
+                         (int64_t)(live ? key : 0) * 8;
+      const int64_t cs_step = (int64_t)a.rope_T * 8;  // floats from one group of 4 pairs to the next
+      float csn0[8], csn1[8];  // pairs [8 j, 8 j + 4) and [8 j + 4, 8 j + 8) of the next chunk j
+      tc::ld_global_v8f(csg, csn0);
+      tc::ld_global_v8f(csg + cs_step, csn1);
+      ok = tc::mbar_wait(dkv_full, n & 1, abort_flag, a.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc::tc_fence_after();
+      {
+        __nv_bfloat16* dst = a.dv + tok * a.ldg + kcol0;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[32];
+          tc::tmem_ld_32x32b_x32(lane_base + TB_DV + 32 * cc, o);
+          tc::tmem_ld_wait();
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1]));
+          if (live) {
+            tc::st_global_v8(dst + 32 * cc, w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]);
+            tc::st_global_v8(dst + 32 * cc + 16, w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]);
+          }
+        }
+      }
+      tc::tc_fence_before();
+      tc::mbar_arrive(dv_empty);
+      // yhat element j from the packed row.
+      auto yel = [&](int j) -> float {
+        const uint4 v = yv[j >> 3];
+        const uint32_t wv = (j & 7) < 2 ? v.x : (j & 7) < 4 ? v.y : (j & 7) < 6 ? v.z : v.w;
+        const float2 f = unpack_bf16x2(wv);
+        return (j & 1) ? f.y : f.x;
+      };
+      // The same element, unpacked by an instruction the compiler may not
+      // merge with the first pass's: yhat then stays packed (64 registers)
+      // between the two passes instead of as 128 floats.
+      auto yel2 = [&](int j) -> float {
+        const uint4 v = yv[j >> 3];
+        const uint32_t wv = (j & 7) < 2 ? v.x : (j & 7) < 4 ? v.y : (j & 7) < 6 ? v.z : v.w;
+        uint32_t u;
+        if (j & 1)
+          asm volatile("and.b32 %0, %1, 0xffff0000;" : "=r"(u) : "r"(wv));
+        else
+          asm volatile("shl.b32 %0, %1, 16;" : "=r"(u) : "r"(wv));
+        return __uint_as_float(u);
+      };
+      float dot = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t gv[32];
+        tc::tmem_ld_32x32b_x32(lane_base + TB_DK + 32 * cc, gv);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) dot = fmaf(__uint_as_float(gv[i]), yel(32 * cc + i), dot);
+      }
+      const float mean = dot * a.scale / 128.f;
+      __nv_bfloat16* dst = a.dk + tok * a.ldg + kcol0;
+      uint32_t lo[8], hi[8];  // two chunks' outputs, stored as 32 bytes each
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {  // pairs [8 j, 8 j + 8): dims 8 j + i and 64 + 8 j + i
+        float cs[16];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          cs[u] = csn0[u];
+          cs[8 + u] = csn1[u];
+        }
+        if (j + 1 < 8) {
+          tc::ld_global_v8f(csg + (2 * j + 2) * cs_step, csn0);
+          tc::ld_global_v8f(csg + (2 * j + 3) * cs_step, csn1);
+        }
+        uint32_t g0[8], g1[8];
+        tc::tmem_ld_32x32b_x8(lane_base + TB_DK + 8 * j, g0);
+        tc::tmem_ld_32x32b_x8(lane_base + TB_DK + 64 + 8 * j, g1);
+        tc::tmem_ld_wait();
+        if (j == 7) {  // dK is read: the MMA warp may overwrite it
+          tc::tc_fence_before();
+          tc::mbar_arrive(dk_empty);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) {
+          float o_lo[2], o_hi[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float cv = cs[2 * (i + e)], sv = cs[2 * (i + e) + 1];
+            const float d0 = r * (__uint_as_float(g0[i + e]) * a.scale - yel2(8 * j + i + e) * mean);
+            const float d1 = r * (__uint_as_float(g1[i + e]) * a.scale - yel2(64 + 8 * j + i + e) * mean);
+            o_lo[e] = d0 * cv + d1 * sv;
+            o_hi[e] = d1 * cv - d0 * sv;
+          }
+          lo[(j & 1) * 4 + i / 2] = pack_bf16x2(o_lo[0], o_lo[1]);
+          hi[(j & 1) * 4 + i / 2] = pack_bf16x2(o_hi[0], o_hi[1]);
+        }
+        if ((j & 1) && live) {
+          tc::st_global_v8(dst + 8 * (j - 1), lo[0], lo[1], lo[2], lo[3], lo[4], lo[5], lo[6], lo[7]);
+          tc::st_global_v8(dst + 64 + 8 * (j - 1), hi[0], hi[1], hi[2], hi[3], hi[4], hi[5], hi[6], hi[7]);
+        }
+      }
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 // ------------------------------------------------------------------ dQ from stored dS
 // Query side of the backward when the key-side kernel stored dS^T: a
 // persistent kernel (one CTA per SM) walks the work items (128-query tile,
-// query head, batch row), heaviest tiles first, and for each accumulates
+// query head, batch row) in balanced pairs (see DqWalk), and for each accumulates
 //   dQ = sum over key tiles kb of dS(i, kb) K_kb        (M 128 queries, N 128 dims)
 // in TMEM from the dS^T tile ([128 keys][128 queries], read MN-major) and the
 // K tile ([128 keys][128 dims], MN-major), each through its own TMA ring.
@@ -1282,10 +1796,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // memory.
 constexpr int kDqThreads = 320;
 // The dS^T tiles come from HBM (written by the key-side kernel, far larger
-// than L2) and get a four-deep ring; a K tile is shared by the 16 query
-// tiles of its (head, row), so it mostly hits L2 and two stages suffice.
+// than L2) and get a four-deep ring; a K tile is shared by the query tiles
+// of its (head, row), which the item order keeps close together in time, so
+// it mostly hits L2 and three stages cover that latency.
 constexpr int kDqDsStages = 4;
-constexpr int kDqKStages = 2;
+constexpr int kDqKStages = 3;
 constexpr int DQ_OFF_K = kDqDsStages * TILE;
 constexpr int DQ_OFF_DOT = DQ_OFF_K + kDqKStages * TILE;  // [2 accumulators][2 sides][128 rows] f32
 constexpr int DQ_OFF_BAR = DQ_OFF_DOT + 2 * 2 * 128 * 4;
@@ -1300,45 +1815,72 @@ struct DqArgs {
   const __nv_bfloat16* yhat;  // saved normalised q: row tok at yhat + tok * ldy, head h at + h * 128
   int64_t ldy;
   const float* rstd_q;        // [B * T, H]
-  const float2* rope_tab;     // [T][64] (cos, sin)
+  const float2* rope_tab;     // [rope_T][64] (cos, sin), then the grouped copy
+  int rope_T;
   __nv_bfloat16* out;         // dq rows: out + tok * ldo + h * 128
   int64_t ldo;
   int* status;
 };
 
-// Work item w (heaviest first): query tile, head, batch row, and the key
-// tiles [kb_lo, qi] whose dS^T tiles the key-side kernel stored for it.
+// Work item: query tile, head, batch row, and the key tiles [kb_lo, qi]
+// whose dS^T tiles the key-side kernel stored for it.
 struct DqItem {
   int qi, h, b, kb_lo, n;
 };
-__device__ __forceinline__ DqItem dq_item(const DqArgs& a, int w, int window) {
-  DqItem it;
-  const int hb = a.H * a.B;
-  it.qi = a.nqb - 1 - w / hb;
-  const int rest = w % hb;
-  it.h = rest % a.H;
-  it.b = rest / a.H;
-  const int lo = window < 0 ? 0 : it.qi * BQB - BKV + 1 - window;
-  it.kb_lo = lo <= 0 ? 0 : (lo + BKV - 1) / BKV;
-  it.n = it.qi - it.kb_lo + 1;
-  return it;
-}
 
-// Walks this CTA's key tiles in order: item w (stride gridDim.x), tile t of it.
-struct DqCursor {
-  int w, t;
-  DqItem m;
-  __device__ __forceinline__ bool valid(int nitems) const { return w < nitems; }
-  __device__ __forceinline__ void start(const DqArgs& a, int window) {
-    w = blockIdx.x;
-    t = 0;
-    m = dq_item(a, w, window);
+// This CTA's work items in order.  Items come in pairs of one (head, row):
+// query tile nqb - 1 - j, then tile j.  Under the causal mask the pair's tile
+// counts add up to nqb + 1 whatever j is, so dealing pair p to CTA
+// p mod gridDim.x balances the work; the pairs of one (head, row) are
+// consecutive, so the CTAs working at the same time share its K tiles in L2.
+struct DqWalk {
+  int p, sub;
+  __device__ __forceinline__ void start() {
+    p = blockIdx.x;
+    sub = 0;
   }
-  __device__ __forceinline__ void next(const DqArgs& a, int window, int nitems) {
+  __device__ __forceinline__ bool valid(int npairs) const { return p < npairs; }
+  __device__ __forceinline__ DqItem item(const DqArgs& a, int window) const {
+    const int ppg = (a.nqb + 1) / 2;
+    const int grp = p / ppg;
+    const int j = p - grp * ppg;
+    DqItem it;
+    it.qi = sub ? j : a.nqb - 1 - j;
+    it.h = grp % a.H;
+    it.b = grp / a.H;
+    const int lo = window < 0 ? 0 : it.qi * BQB - BKV + 1 - window;
+    it.kb_lo = lo <= 0 ? 0 : (lo + BKV - 1) / BKV;
+    it.n = it.qi - it.kb_lo + 1;
+    return it;
+  }
+  __device__ __forceinline__ void next(const DqArgs& a) {
+    const int ppg = (a.nqb + 1) / 2;
+    const int j = p % ppg;
+    if (sub == 0 && a.nqb - 1 - j != j) {
+      sub = 1;
+    } else {
+      sub = 0;
+      p += gridDim.x;
+    }
+  }
+};
+
+// Walks this CTA's key tiles in order: tile t of the walk's current item.
+struct DqCursor {
+  DqWalk wk;
+  int t;
+  DqItem m;
+  __device__ __forceinline__ bool valid(int npairs) const { return wk.valid(npairs); }
+  __device__ __forceinline__ void start(const DqArgs& a, int window, int npairs) {
+    wk.start();
+    t = 0;
+    if (wk.valid(npairs)) m = wk.item(a, window);
+  }
+  __device__ __forceinline__ void next(const DqArgs& a, int window, int npairs) {
     if (++t == m.n) {
       t = 0;
-      w += gridDim.x;
-      if (w < nitems) m = dq_item(a, w, window);
+      wk.next(a);
+      if (wk.valid(npairs)) m = wk.item(a, window);
     }
   }
 };
@@ -1367,7 +1909,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int window = GW ? a.window : -1;
-  const int nitems = a.nqb * a.H * a.B;
+  const int npairs = (a.nqb + 1) / 2 * a.H * a.B;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kDqDsStages; ++i) {
@@ -1404,12 +1946,12 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       // runs kDqDsStages tiles ahead of the tensor core, the K ring kDqKStages.
       constexpr int lag = kDqDsStages - kDqKStages;
       DqCursor cd, ck;
-      cd.start(a, window);
-      ck.start(a, window);
+      cd.start(a, window, npairs);
+      ck.start(a, window, npairs);
       int issued_d = 0, issued_k = 0;
       bool ok = true;
-      for (int u = 0; ok && (cd.valid(nitems) || ck.valid(nitems)); ++u) {
-        if (cd.valid(nitems)) {
+      for (int u = 0; ok && (cd.valid(npairs) || ck.valid(npairs)); ++u) {
+        if (cd.valid(npairs)) {
           const int st = issued_d % kDqDsStages;
           if (!tc::mbar_wait(&ds_empty[st], ((issued_d / kDqDsStages) & 1) ^ 1, abort_flag,
                              a.status)) {
@@ -1421,9 +1963,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             tc::tma_load_3d(smem + st * TILE + c * (TILE / 2), &tds, &ds_full[st],
                             cd.m.qi * BQB + 64 * c, (cd.m.kb_lo + cd.t) * BKV, cd.m.b * a.H + cd.m.h);
           ++issued_d;
-          cd.next(a, window, nitems);
+          cd.next(a, window, npairs);
         }
-        if (u >= lag && ck.valid(nitems)) {
+        if (u >= lag && ck.valid(npairs)) {
           const int st = issued_k % kDqKStages;
           if (!tc::mbar_wait(&k_empty[st], ((issued_k / kDqKStages) & 1) ^ 1, abort_flag,
                              a.status)) {
@@ -1436,7 +1978,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             tc::tma_load_3d(smem + DQ_OFF_K + st * TILE + c * (TILE / 2), &tk, &k_full[st],
                             hk * HD + 64 * c, (ck.m.kb_lo + ck.t) * BKV, ck.m.b);
           ++issued_k;
-          ck.next(a, window, nitems);
+          ck.next(a, window, npairs);
         }
       }
       if (!ok) {
@@ -1453,8 +1995,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       const uint64_t bd = tc::smem_desc_sw128(tc::smem_u32(smem + DQ_OFF_K), TILE / 2, 1024);
       int it = 0, item = 0;
       bool ok = true;
-      for (int w = blockIdx.x; w < nitems && ok; w += gridDim.x, ++item) {
-        const DqItem m = dq_item(a, w, window);
+      DqWalk wk;
+      for (wk.start(); wk.valid(npairs) && ok; wk.next(a), ++item) {
+        const DqItem m = wk.item(a, window);
         const int buf = item & 1;
         // The epilogue of the item two back has read this accumulator.
         if (!tc::mbar_wait(&acc_empty[buf], ((item >> 1) & 1) ^ 1, abort_flag, a.status)) {
@@ -1492,8 +2035,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
     float* dots = reinterpret_cast<float*>(smem + DQ_OFF_DOT);
     int item = 0;
-    for (int w = blockIdx.x; w < nitems; w += gridDim.x, ++item) {
-      const DqItem m = dq_item(a, w, window);
+    DqWalk wk;
+    for (wk.start(); wk.valid(npairs); wk.next(a), ++item) {
+      const DqItem m = wk.item(a, window);
       const int buf = item & 1;
       const uint32_t acc = lane_base + 128 * buf;
       const int q = m.qi * BQB + row;
@@ -1502,18 +2046,27 @@ __global__ void __launch_bounds__(kDqThreads, 1)
       // Everything the row needs besides the accumulator, loaded before it
       // is waited for: the saved normalised q (dims 32 side + [0, 32) and
       // 64 + 32 side + [0, 32)), 1/rms and the 32 pairs' (cos, sin).
+      // 32-byte loads: the q row's halves (the row's address is 32-byte
+      // aligned), and (cos, sin) of four consecutive pairs from the grouped
+      // copy of the table, where a warp's 32 rows read 1 KB at once.
       const __nv_bfloat16* yrow = a.yhat + tok * a.ldy + m.h * HD + 32 * side;
       uint4 yv[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        yv[u] = live ? reinterpret_cast<const uint4*>(yrow)[u] : make_uint4(0u, 0u, 0u, 0u);
-        yv[4 + u] = live ? reinterpret_cast<const uint4*>(yrow + 64)[u] : make_uint4(0u, 0u, 0u, 0u);
+      for (int u = 0; u < 4; u += 2) {
+        uint32_t w0[8], w1[8];
+        tc::ld_global_v8u(yrow + 8 * u, w0);
+        tc::ld_global_v8u(yrow + 64 + 8 * u, w1);
+        yv[u] = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+        yv[u + 1] = make_uint4(w0[4], w0[5], w0[6], w0[7]);
+        yv[4 + u] = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+        yv[5 + u] = make_uint4(w1[4], w1[5], w1[6], w1[7]);
       }
-      const float r = live ? a.rstd_q[tok * a.H + m.h] : 0.f;
-      const float4* cs4 = reinterpret_cast<const float4*>(a.rope_tab + (int64_t)(live ? q : 0) * 64 + 32 * side);
-      float4 cs[16];  // pairs 32 side + 2 i, + 2 i + 1: (cos, sin, cos, sin)
+      const float r = a.rstd_q[tok * a.H + m.h];
+      const float* csg = reinterpret_cast<const float*>(a.rope_tab + (int64_t)a.rope_T * 64) +
+                         ((int64_t)(8 * side) * a.rope_T + (live ? q : 0)) * 8;
+      float cs[8][8];  // pairs 32 side + 4 u + [0, 4): (cos, sin) x 4
 #pragma unroll
-      for (int i = 0; i < 16; ++i) cs[i] = cs4[i];
+      for (int u = 0; u < 8; ++u) tc::ld_global_v8f(csg + (int64_t)u * a.rope_T * 8, cs[u]);
       bool ok = tc::mbar_wait(&acc_full[buf], (item >> 1) & 1, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc::tc_fence_after();
@@ -1556,8 +2109,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         uint32_t lo_[8], hi_[8];
 #pragma unroll
         for (int i = 0; i < 16; i += 2) {
-          const float4 t4 = cs[(16 * c + i) / 2];
-          const float cc[2] = {t4.x, t4.z}, sn[2] = {t4.y, t4.w};
+          const float* t4 = &cs[(16 * c + i) / 4][2 * ((16 * c + i) % 4)];  // pairs i, i + 1 of the chunk
+          const float cc[2] = {t4[0], t4[2]}, sn[2] = {t4[1], t4[3]};
           float o_lo[2], o_hi[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
@@ -1570,13 +2123,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
           hi_[i / 2] = pack_bf16x2(o_hi[0], o_hi[1]);
         }
         if (live) {
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            reinterpret_cast<uint4*>(dst + 16 * c)[u] =
-                make_uint4(lo_[4 * u], lo_[4 * u + 1], lo_[4 * u + 2], lo_[4 * u + 3]);
-            reinterpret_cast<uint4*>(dst + 64 + 16 * c)[u] =
-                make_uint4(hi_[4 * u], hi_[4 * u + 1], hi_[4 * u + 2], hi_[4 * u + 3]);
-          }
+          tc::st_global_v8(dst + 16 * c, lo_[0], lo_[1], lo_[2], lo_[3], lo_[4], lo_[5], lo_[6], lo_[7]);
+          tc::st_global_v8(dst + 64 + 16 * c, hi_[0], hi_[1], hi_[2], hi_[3], hi_[4], hi_[5], hi_[6], hi_[7]);
         }
       }
     }
@@ -1660,19 +2208,19 @@ nc_status attention_fwd(const void* q, const void* k, const void* v, int64_t ld,
 nc_status attention_bwd_tc_ex(const void* q, int64_t ldq, const void* k, const void* v, int64_t ldkv,
                               const void* dout, int64_t ldo, const float* lse, const float* delta,
                               float* dq, void* dk, void* dv, int64_t ldg, int B, int T, int H,
-                              int Hkv, int window, const float2* rope_tab, const float* rstd_k,
-                              void* ds, int64_t ld_ds, int* status, cudaStream_t s,
-                              Profiler* prof) {
+                              int Hkv, int window, const float2* rope_tab, int rope_T,
+                              const float* rstd_k, void* ds, int64_t ld_ds, int* status,
+                              cudaStream_t s, Profiler* prof) {
   static DeviceOnce attr;
   NC_TRY(once_per_device(attr, []() -> nc_status {
-    NC_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc_kernel<false, false>,
+    NC_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc_kernel<false>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdSmem));
-    NC_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc_kernel<true, false>,
+    NC_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc_kernel<true>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdSmem));
-    NC_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc_kernel<false, true>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdSmem));
-    NC_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_tc_kernel<true, true>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdSmem));
+    NC_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_kv_kernel<false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmem));
+    NC_CUDA_TRY(cudaFuncSetAttribute(attn_bwd_kv_kernel<true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmem));
     return NC_OK;
   }));
   const bool sds = ds != nullptr;
@@ -1694,6 +2242,10 @@ nc_status attention_bwd_tc_ex(const void* q, int64_t ldq, const void* k, const v
     if (ld_ds < T || ld_ds % 8 || (reinterpret_cast<uintptr_t>(ds) & 15) ||
         !make_tmap_bf16_3d(&mdq, ds, T, T, (uint64_t)B * H, ld_ds, (int64_t)T * ld_ds, BKV))
       return fail(NC_ERR_INVALID_ARG, "attention_bwd: dS buffer rejected");
+    if (!rope_tab || rope_T < T || !rstd_k)
+      return fail(NC_ERR_INVALID_ARG, "attention_bwd: the store-dS form needs the RoPE table and rstd_k");
+    if (ldg % 16 || ((reinterpret_cast<uintptr_t>(dk) | reinterpret_cast<uintptr_t>(dv)) & 31))
+      return fail(NC_ERR_INVALID_ARG, "attention_bwd: dk / dv rows must be 32-byte aligned");
   } else {
     // dq (fp32, dense [B, T, H * 128]): 32 x 32 boxes, 128-byte swizzle.
     if ((reinterpret_cast<uintptr_t>(dq) & 15) ||
@@ -1717,22 +2269,28 @@ nc_status attention_bwd_tc_ex(const void* q, int64_t ldq, const void* k, const v
   a.ldg = ldg;
   a.status = status;
   a.rope_tab = rope_tab;
+  a.rope_T = rope_T;
   a.rstd_k = rstd_k;
   a.Hkv = Hkv;
+  a.B = B;
   // Five products per (query, key) pair, or four when dQ is left to the
   // query-side kernel.
   const double flops = (sds ? 8.0 : 10.0) * B * H * HD * causal_pairs(T, a.window);
   Probe probe(prof, s, "attn_bwd", flops, 0.0);
   dim3 grid(a.nkb, Hkv, B);  // one CTA per key tile and KV head; it loops over the group
   const bool gw = a.group > 1 || a.window >= 0;
-  if (gw && sds)
-    attn_bwd_tc_kernel<true, true><<<grid, kBwdThreads, kBwdSmem, s>>>(mq, mk, mv, mdo, mdq, a);
-  else if (gw)
-    attn_bwd_tc_kernel<true, false><<<grid, kBwdThreads, kBwdSmem, s>>>(mq, mk, mv, mdo, mdq, a);
-  else if (sds)
-    attn_bwd_tc_kernel<false, true><<<grid, kBwdThreads, kBwdSmem, s>>>(mq, mk, mv, mdo, mdq, a);
-  else
-    attn_bwd_tc_kernel<false, false><<<grid, kBwdThreads, kBwdSmem, s>>>(mq, mk, mv, mdo, mdq, a);
+  if (sds) {
+    // Persistent form: one CTA per SM over the (key tile, KV head, row) items.
+    const unsigned pgrid = (unsigned)std::min<int64_t>((int64_t)(a.nkb + 1) / 2 * Hkv * B, num_sms());
+    if (gw)
+      attn_bwd_kv_kernel<true><<<pgrid, kKvThreads, kKvSmem, s>>>(mq, mk, mv, mdo, mdq, a);
+    else
+      attn_bwd_kv_kernel<false><<<pgrid, kKvThreads, kKvSmem, s>>>(mq, mk, mv, mdo, mdq, a);
+  } else if (gw) {
+    attn_bwd_tc_kernel<true><<<grid, kBwdThreads, kBwdSmem, s>>>(mq, mk, mv, mdo, mdq, a);
+  } else {
+    attn_bwd_tc_kernel<false><<<grid, kBwdThreads, kBwdSmem, s>>>(mq, mk, mv, mdo, mdq, a);
+  }
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }
@@ -1742,13 +2300,13 @@ nc_status attention_bwd_tc(const void* q, const void* k, const void* v, int64_t 
                            float* dq, void* dk, void* dv, int64_t ldg, int B, int T, int H,
                            int* status, cudaStream_t s, Profiler* prof) {
   return attention_bwd_tc_ex(q, ld, k, v, ld, dout, ldo, lse, delta, dq, dk, dv, ldg, B, T, H, H, -1,
-                             nullptr, nullptr, nullptr, 0, status, s, prof);
+                             nullptr, 0, nullptr, nullptr, 0, status, s, prof);
 }
 
 nc_status attention_dq_ex(const void* ds, int64_t ld_ds, const void* k, int64_t ldkv, int B, int T,
                           int H, int Hkv, int window, const void* yhat, int64_t ldy,
-                          const float* rstd_q, const float2* rope_tab, void* out, int64_t ldo,
-                          int* status, cudaStream_t s, Profiler* prof) {
+                          const float* rstd_q, const float2* rope_tab, int rope_T, void* out,
+                          int64_t ldo, int* status, cudaStream_t s, Profiler* prof) {
   static DeviceOnce attr;
   NC_TRY(once_per_device(attr, []() -> nc_status {
     NC_CUDA_TRY(cudaFuncSetAttribute(attn_dq_kernel<false>,
@@ -1758,8 +2316,11 @@ nc_status attention_dq_ex(const void* ds, int64_t ld_ds, const void* k, int64_t 
     return NC_OK;
   }));
   if (B < 1 || T < 1 || H < 1 || Hkv < 1 || H % Hkv || !ds || !k || !yhat || !rstd_q ||
-      !rope_tab || !out)
+      !rope_tab || rope_T < T || !out)
     return fail(NC_ERR_INVALID_ARG, "attention_dq: bad arguments");
+  if (ldy % 16 || ldo % 16 ||
+      ((reinterpret_cast<uintptr_t>(yhat) | reinterpret_cast<uintptr_t>(out)) & 31))
+    return fail(NC_ERR_INVALID_ARG, "attention_dq: q and dq rows must be 32-byte aligned");
   if (ldkv % 8 || ldy % 8 || ldo % 8 || ld_ds < T || ld_ds % 8 ||
       ((reinterpret_cast<uintptr_t>(ds) | reinterpret_cast<uintptr_t>(k) |
         reinterpret_cast<uintptr_t>(yhat) | reinterpret_cast<uintptr_t>(out)) & 15))
@@ -1780,14 +2341,15 @@ nc_status attention_dq_ex(const void* ds, int64_t ld_ds, const void* k, int64_t 
   a.ldy = ldy;
   a.rstd_q = rstd_q;
   a.rope_tab = rope_tab;
+  a.rope_T = rope_T;
   a.out = static_cast<__nv_bfloat16*>(out);
   a.ldo = ldo;
   a.status = status;
   const double flops = 2.0 * B * H * HD * causal_pairs(T, a.window);
   Probe probe(prof, s, "attn_bwd_dq", flops, 0.0);
   // Persistent: one CTA per SM (or per work item when there are fewer).
-  const int nitems = a.nqb * H * B;
-  const unsigned grid = (unsigned)std::min(nitems, num_sms());
+  const int npairs = (a.nqb + 1) / 2 * H * B;
+  const unsigned grid = (unsigned)std::min(npairs, num_sms());
   if (a.group > 1 || a.window >= 0)
     attn_dq_kernel<true><<<grid, kDqThreads, kDqSmem, s>>>(mds, mk, a);
   else

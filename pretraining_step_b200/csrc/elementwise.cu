@@ -113,14 +113,18 @@ __global__ void __launch_bounds__(256) rmsnorm_bwd_kernel(
 }
 
 // ------------------------------------------------------------------ RoPE + QK-norm
-// cos/sin table [T][hd/2]: theta_i(pos) = pos * 10000^(-2i/hd), in double.
+// cos/sin table [T][hd/2]: theta_i(pos) = pos * 10000^(-2i/hd), in double;
+// the same values again, grouped four pairs at a time per position
+// ([hd/8][T][4]), after it.
 __global__ void rope_table_kernel(float2* tab, int T, int hd) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int half = hd / 2;
   if (i >= (int64_t)T * half) return;
   const int pos = (int)(i / half), j = (int)(i % half);
   const double th = (double)pos * pow(10000.0, -2.0 * j / hd);
-  tab[i] = make_float2((float)cos(th), (float)sin(th));
+  const float2 v = make_float2((float)cos(th), (float)sin(th));
+  tab[i] = v;
+  tab[(int64_t)T * half + ((int64_t)(j >> 2) * T + pos) * 4 + (j & 3)] = v;
 }
 
 // ------------------------------------------------------------------ cross-entropy

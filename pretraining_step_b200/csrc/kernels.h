@@ -49,32 +49,31 @@ nc_status attention_bwd_tc(const void* q, const void* k, const void* v, int64_t 
 nc_status attention_fwd_ex(const void* q, int64_t ldq, const void* k, const void* v, int64_t ldkv,
                            void* o, int64_t ldo, float* lse, int B, int T, int H, int Hkv,
                            int window, int* status, cudaStream_t s, Profiler* prof);
-// rope_tab / rstd_k non-null: dk receives the gradient of the k slice before
-// its RoPE + QK-norm (the saved k being their output), i.e. the k-side
-// backward of the q|k|v projection's epilogue is applied in the attention
-// backward's dK epilogue; null: dk is the gradient of the k operand.
 nc_status attention_bwd_ex(const void* q, int64_t ldq, const void* k, const void* v, int64_t ldkv,
                            const void* o, const void* dout, int64_t ldo, const float* lse,
                            float* dq, void* dk, void* dv, int64_t ldg, float* delta, int B, int T,
-                           int H, int Hkv, int window, const float2* rope_tab, const float* rstd_k,
-                           int* status, cudaStream_t s, Profiler* prof);
-// ds non-null: the kernel stores every dS^T tile (bf16 [B*H][T keys][T
-// queries], row stride ld_ds, a multiple of 8 >= T) instead of computing dQ,
-// and dq is not touched; attention_dq_ex then contracts it with K.
+                           int H, int Hkv, int window, int* status, cudaStream_t s, Profiler* prof);
+// ds non-null: the persistent key-side kernel stores every dS^T tile (bf16
+// [B*H][T keys][T queries], row stride ld_ds, a multiple of 8 >= T) instead
+// of computing dQ, dq is not touched, and dK leaves through the k-side RoPE
+// + QK-norm backward (rope_tab: rope_table()'s buffer for rope_T >= T
+// positions; rstd_k non-null; dk, dv 32-byte aligned with ldg a multiple of
+// 16); attention_dq_ex then contracts dS^T with K.
 nc_status attention_bwd_tc_ex(const void* q, int64_t ldq, const void* k, const void* v, int64_t ldkv,
                               const void* dout, int64_t ldo, const float* lse, const float* delta,
                               float* dq, void* dk, void* dv, int64_t ldg, int B, int T, int H,
-                              int Hkv, int window, const float2* rope_tab, const float* rstd_k,
-                              void* ds, int64_t ld_ds, int* status, cudaStream_t s,
-                              Profiler* prof);
+                              int Hkv, int window, const float2* rope_tab, int rope_T,
+                              const float* rstd_k, void* ds, int64_t ld_ds, int* status,
+                              cudaStream_t s, Profiler* prof);
 // dQ = dS K / sqrt(128) from the stored dS^T tiles, through the backward of
 // the q-side RoPE + QK-norm (yhat: the saved normalised q, row stride ldy;
 // rstd_q [B*T, H]), written as bf16 rows of stride ldo (the q slice of the
-// q|k|v gradient).
+// q|k|v gradient; yhat and out 32-byte aligned, ldy and ldo multiples of 16).
+// rope_tab: rope_table()'s buffer for rope_T >= T positions.
 nc_status attention_dq_ex(const void* ds, int64_t ld_ds, const void* k, int64_t ldkv, int B, int T,
                           int H, int Hkv, int window, const void* yhat, int64_t ldy,
-                          const float* rstd_q, const float2* rope_tab, void* out, int64_t ldo,
-                          int* status, cudaStream_t s, Profiler* prof);
+                          const float* rstd_q, const float2* rope_tab, int rope_T, void* out,
+                          int64_t ldo, int* status, cudaStream_t s, Profiler* prof);
 // The model's attention backward: the row sums D, the key-side kernel with
 // the k-side RoPE + QK-norm backward in its dK epilogue and dS^T stored to
 // ds, then the query-side kernel with the q-side backward in its epilogue.
@@ -83,8 +82,9 @@ nc_status attention_bwd_model(const void* q, int64_t ldq, const void* k, const v
                               int64_t ldkv, const void* o, const void* dout, int64_t ldo,
                               const float* lse, float* delta, void* ds, int64_t ld_ds,
                               void* dq_out, void* dk, void* dv, int64_t ldg, int B, int T, int H,
-                              int Hkv, int window, const float2* rope_tab, const float* rstd_q,
-                              const float* rstd_k, int* status, cudaStream_t s, Profiler* prof);
+                              int Hkv, int window, const float2* rope_tab, int rope_T,
+                              const float* rstd_q, const float* rstd_k, int* status, cudaStream_t s,
+                              Profiler* prof);
 
 nc_status embed_gather(const int32_t* tok, int64_t n, const float* E, int V, int d, float* x,
                        int* status, cudaStream_t s, Profiler* prof);
@@ -96,6 +96,10 @@ nc_status rmsnorm_fwd(const float* x, int64_t rows, int d, void* y, float* rstd,
 nc_status rmsnorm_bwd(const void* dh, const void* y, const float* rstd, const float* dres,
                       int64_t rows, int d, float* dx, void* dx_bf16, cudaStream_t s,
                       Profiler* prof);
+// RoPE cos/sin for positions [0, T): tab[pos * hd/2 + i] = (cos, sin) of
+// pos * 10000^(-2i/hd); then, from tab + T * hd/2, the same values grouped
+// for 32-byte loads of four consecutive pairs of one position:
+// [(i / 4) * T + pos] * 4 + i % 4.  tab holds T * hd floats (two float2 per pair).
 nc_status rope_table(float2* tab, int T, int hd, cudaStream_t s);
 nc_status ce_fwd_bwd(void* z, const int32_t* tgt, int64_t n, int V, float* loss_rows,
                      float* loss_out, int* status, cudaStream_t s, Profiler* prof);

@@ -222,7 +222,7 @@ nc_status ensure_rope(nc_params* p, int T) {
   int newT = std::max(T, 2048);
   if (p->rope) cudaFree(p->rope);
   p->rope = nullptr;
-  NC_CUDA_TRY(cudaMalloc(&p->rope, sizeof(float2) * (size_t)newT * (p->hd / 2)));
+  NC_CUDA_TRY(cudaMalloc(&p->rope, 2 * sizeof(float2) * (size_t)newT * (p->hd / 2)));  // two layouts
   NC_TRY(rope_table(p->rope, newT, p->hd, p->stream));
   p->rope_T = newT;
   return NC_OK;
@@ -439,7 +439,7 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
     // a.ds), then the query side (dQ = dS K through the q-side backward).
     NC_TRY(attention_bwd_model(a.qkv[l], Q, a.qkv[l] + d, a.qkv[l] + d + dkv, Q, a.o[l], a.dh, d,
                                a.lse[l], a.delta, a.ds, a.ld_ds, a.dqkv, a.dqkv + d,
-                               a.dqkv + d + dkv, Q, B, T, H, Hkv, p->window[l], p->rope, a.rq[l],
+                               a.dqkv + d + dkv, Q, B, T, H, Hkv, p->window[l], p->rope, p->rope_T, a.rq[l],
                                a.rk[l], p->status, s, pr));
     NC_TRY(proj_dw(p, a.dqkv, Q, Q, a.h1[l], d, d, N, G));
     NC_TRY(proj_dx(p, a.dqkv, N, Q, W, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0));
@@ -1032,8 +1032,7 @@ nc_status nc_op_attention_bwd_ex(const void* q, int64_t ldq, const void* k, cons
   int* st = nullptr;
   NC_TRY(op_status_word(&st));
   return attention_bwd_ex(q, ldq, k, v, ldkv, o, dout, ldo, lse, dq, dk, dv, ldg, delta_scratch, B,
-                          T, H, Hkv, window, nullptr, nullptr, st, static_cast<cudaStream_t>(stream),
-                          nullptr);
+                          T, H, Hkv, window, st, static_cast<cudaStream_t>(stream), nullptr);
 }
 
 size_t nc_newton_schulz_scratch_bytes(int count, int rows, int cols) {
