@@ -1189,9 +1189,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 //   warps 4..11 P^T and dS^T, two threads per key row;
 //   warps 12..15 epilogue, one key row per thread: the row of yhat (the
 //               normalised k, the K operand itself) is copied from shared
-//               memory while the item runs, so K's buffer can take the next
-//               item; at the item's end dV goes out, then dK through
-//               dr = r (g - yhat mean(g yhat)), dk = R(-theta) dr.
+//               memory into registers while the item runs, so K's buffer
+//               can take the next item; at the item's end dV goes out, then
+//               dK through dr = r (g - yhat mean(g yhat)), dk = R(-theta) dr.
 constexpr int kKvThreads = 512;
 constexpr int KV_OFF_TI = B_OFF_BAR;        // [2 stages] (first query, key tile) of the tile
 constexpr int KV_OFF_BAR = KV_OFF_TI + 64;
@@ -1348,8 +1348,7 @@ __global__ void __launch_bounds__(kKvThreads)
       const uint32_t ph = (g >> 1) & 1;
       bool w = true;
       if (c.t == 0) {
-        // K and V of the item, once the previous item's MMAs have read them
-        // and the epilogue has copied its yhat rows.
+        // K and V of the item, once the previous item's MMAs have read them.
         if (lane == 0 && c.n > 0)
           w = tc::mbar_wait(kv_empty, (c.n - 1) & 1, abort_flag, a.status) &&
               tc::mbar_wait(k_copied, (c.n - 1) & 1, abort_flag, a.status);
@@ -1645,35 +1644,40 @@ __global__ void __launch_bounds__(kKvThreads)
     const int qw = warp & 3;
     const int row = qw * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
-    const uint32_t krow = tc::smem_u32(smem + B_OFF_K) + row * 128;
     KvCursor c;
     c.start(a, npairs, group, window);
     for (; c.valid; c.next_item(a, npairs, group, window)) {
       const int n = c.n;
-      // yhat of this key row (dims [8 u, 8 u + 8) in yv[u]) while the item runs.
-      bool ok = tc::mbar_wait(kv_full, n & 1, abort_flag, a.status);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      uint4 yv[16];
-#pragma unroll
-      for (int u = 0; u < 16; ++u)
-        yv[u] = tc::ld_shared_v4(krow + (u >> 3) * (TILE / 2) + (((u & 7) ^ (row & 7)) << 4));
-      tc::mbar_arrive(k_copied);
       const int key = c.m.kb * BKV + row;
       // Keys at or past T (a ragged last tile) take part in the warp-wide
-      // TMEM loads but read and write nothing in global memory.
+      // TMEM loads but write nothing (their global loads read key 0's row).
       const bool live = key < a.T;
       const int64_t tok = (int64_t)c.m.b * a.T + (live ? key : 0);
       const int kcol0 = c.m.hk * HD;
-      const float r = live ? a.rstd_k[tok * a.Hkv + c.m.hk] : 0.f;
+      // yhat of this key row (dims [8 u, 8 u + 8) in yv[u]) from the K tile
+      // in shared memory as soon as it lands, then 1/rms and the first
+      // (cos, sin) groups, all before the item's accumulators are waited for.
+      bool okk = tc::mbar_wait(kv_full, n & 1, abort_flag, a.status);
+      if (!__all_sync(0xffffffffu, okk)) break;
+      uint4 yv[16];
+      {
+        const uint32_t krow = tc::smem_u32(smem + B_OFF_K) + row * 128;
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          yv[u] = tc::ld_shared_v4(krow + (u >> 3) * (TILE / 2) + (((u & 7) ^ (row & 7)) << 4));
+      }
+      tc::mbar_arrive(k_copied);
+      const float r = a.rstd_k[tok * a.Hkv + c.m.hk];
       // (cos, sin) of four consecutive pairs of this key are 32 contiguous
-      // bytes of the grouped table, so a warp's 32 keys read 1 KB at once.
+      // bytes of the grouped table, so a warp's 32 keys read 1 KB at once;
+      // a three-slot ring keeps two groups in flight ahead of their use.
       const float* csg = reinterpret_cast<const float*>(a.rope_tab + (int64_t)a.rope_T * 64) +
                          (int64_t)(live ? key : 0) * 8;
       const int64_t cs_step = (int64_t)a.rope_T * 8;  // floats from one group of 4 pairs to the next
-      float csn0[8], csn1[8];  // pairs [8 j, 8 j + 4) and [8 j + 4, 8 j + 8) of the next chunk j
-      tc::ld_global_v8f(csg, csn0);
-      tc::ld_global_v8f(csg + cs_step, csn1);
-      ok = tc::mbar_wait(dkv_full, n & 1, abort_flag, a.status);
+      float cs0[8], cs1[8], cs2[8];
+      tc::ld_global_v8f(csg, cs0);
+      tc::ld_global_v8f(csg + cs_step, cs1);
+      bool ok = tc::mbar_wait(dkv_full, n & 1, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc::tc_fence_after();
       {
@@ -1725,44 +1729,41 @@ __global__ void __launch_bounds__(kKvThreads)
       }
       const float mean = dot * a.scale / 128.f;
       __nv_bfloat16* dst = a.dk + tok * a.ldg + kcol0;
-      uint32_t lo[8], hi[8];  // two chunks' outputs, stored as 32 bytes each
+      uint32_t lo[8], hi[8];  // four groups' outputs, stored as 32 bytes each
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {  // pairs [8 j, 8 j + 8): dims 8 j + i and 64 + 8 j + i
-        float cs[16];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          cs[u] = csn0[u];
-          cs[8 + u] = csn1[u];
+      for (int j = 0; j < 16; ++j) {  // pairs [4 j, 4 j + 4): dims 4 j + i and 64 + 4 j + i
+        // Ring slot of group j: j % 3; group j + 2 goes into the slot group
+        // j - 1 has just freed.
+        float* cur = (j % 3 == 0) ? cs0 : (j % 3 == 1) ? cs1 : cs2;
+        if (j + 2 < 16) {
+          float* nxt = ((j + 2) % 3 == 0) ? cs0 : ((j + 2) % 3 == 1) ? cs1 : cs2;
+          tc::ld_global_v8f(csg + (j + 2) * cs_step, *reinterpret_cast<float (*)[8]>(nxt));
         }
-        if (j + 1 < 8) {
-          tc::ld_global_v8f(csg + (2 * j + 2) * cs_step, csn0);
-          tc::ld_global_v8f(csg + (2 * j + 3) * cs_step, csn1);
-        }
-        uint32_t g0[8], g1[8];
-        tc::tmem_ld_32x32b_x8(lane_base + TB_DK + 8 * j, g0);
-        tc::tmem_ld_32x32b_x8(lane_base + TB_DK + 64 + 8 * j, g1);
+        uint32_t g0[4], g1[4];
+        tc::tmem_ld_32x32b_x4(lane_base + TB_DK + 4 * j, g0);
+        tc::tmem_ld_32x32b_x4(lane_base + TB_DK + 64 + 4 * j, g1);
         tc::tmem_ld_wait();
-        if (j == 7) {  // dK is read: the MMA warp may overwrite it
+        if (j == 15) {  // dK is read: the MMA warp may overwrite it
           tc::tc_fence_before();
           tc::mbar_arrive(dk_empty);
         }
 #pragma unroll
-        for (int i = 0; i < 8; i += 2) {
+        for (int i = 0; i < 4; i += 2) {
           float o_lo[2], o_hi[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const float cv = cs[2 * (i + e)], sv = cs[2 * (i + e) + 1];
-            const float d0 = r * (__uint_as_float(g0[i + e]) * a.scale - yel2(8 * j + i + e) * mean);
-            const float d1 = r * (__uint_as_float(g1[i + e]) * a.scale - yel2(64 + 8 * j + i + e) * mean);
+            const float cv = cur[2 * (i + e)], sv = cur[2 * (i + e) + 1];
+            const float d0 = r * (__uint_as_float(g0[i + e]) * a.scale - yel2(4 * j + i + e) * mean);
+            const float d1 = r * (__uint_as_float(g1[i + e]) * a.scale - yel2(64 + 4 * j + i + e) * mean);
             o_lo[e] = d0 * cv + d1 * sv;
             o_hi[e] = d1 * cv - d0 * sv;
           }
-          lo[(j & 1) * 4 + i / 2] = pack_bf16x2(o_lo[0], o_lo[1]);
-          hi[(j & 1) * 4 + i / 2] = pack_bf16x2(o_hi[0], o_hi[1]);
+          lo[(j & 3) * 2 + i / 2] = pack_bf16x2(o_lo[0], o_lo[1]);
+          hi[(j & 3) * 2 + i / 2] = pack_bf16x2(o_hi[0], o_hi[1]);
         }
-        if ((j & 1) && live) {
-          tc::st_global_v8(dst + 8 * (j - 1), lo[0], lo[1], lo[2], lo[3], lo[4], lo[5], lo[6], lo[7]);
-          tc::st_global_v8(dst + 64 + 8 * (j - 1), hi[0], hi[1], hi[2], hi[3], hi[4], hi[5], hi[6], hi[7]);
+        if ((j & 3) == 3 && live) {
+          tc::st_global_v8(dst + 4 * (j - 3), lo[0], lo[1], lo[2], lo[3], lo[4], lo[5], lo[6], lo[7]);
+          tc::st_global_v8(dst + 64 + 4 * (j - 3), hi[0], hi[1], hi[2], hi[3], hi[4], hi[5], hi[6], hi[7]);
         }
       }
     }
@@ -2245,7 +2246,7 @@ nc_status attention_bwd_tc_ex(const void* q, int64_t ldq, const void* k, const v
     if (!rope_tab || rope_T < T || !rstd_k)
       return fail(NC_ERR_INVALID_ARG, "attention_bwd: the store-dS form needs the RoPE table and rstd_k");
     if (ldg % 16 || ((reinterpret_cast<uintptr_t>(dk) | reinterpret_cast<uintptr_t>(dv)) & 31))
-      return fail(NC_ERR_INVALID_ARG, "attention_bwd: dk / dv rows must be 32-byte aligned");
+      return fail(NC_ERR_INVALID_ARG, "attention_bwd: dk and dv rows must be 32-byte aligned");
   } else {
     // dq (fp32, dense [B, T, H * 128]): 32 x 32 boxes, 128-byte swizzle.
     if ((reinterpret_cast<uintptr_t>(dq) & 15) ||
