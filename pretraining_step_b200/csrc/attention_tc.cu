@@ -67,6 +67,7 @@ struct FwdArgs {
   int group;   // query heads per KV head (1: one KV head per query head)
   int window;  // query t sees keys [t - window, t]; < 0: every key up to t
   int* status;
+  int B;
 };
 
 // 2^x by the MUFU instruction (ex2.approx, flush-to-zero): the softmax
@@ -359,15 +360,23 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 
-// ------------------------------------------------------------------ forward, two query tiles
-// The plain forward (one KV head per query head, no window) at one CTA per
-// SM: the CTA takes query tiles 2p and 2p + 1 of one (head, batch row) and
-// streams their shared key/value tiles once.  Its two score chains
-// interleave on the tensor pipe, so one tile's softmax runs while the
-// other tile's products execute:
+// ------------------------------------------------------------------ forward, two query tiles, persistent
+// The plain forward (one KV head per query head, no window): one CTA per SM
+// walks work items, each two query tiles (2p, 2p + 1) of one (head, batch
+// row) whose shared key/value tiles it streams once.  The two score chains
+// interleave on the tensor pipe, so one tile's softmax runs while the other
+// tile's products execute:
 //   tensor:  ... PV_a(j)  S_a(j+1)  PV_b(j)  S_b(j+1)  PV_a(j+1) ...
+// Items come in pairs of one (head, row), query-tile pair npairs - 1 - j and
+// then j: their key-tile counts add up to the same total whatever j is, so
+// dealing item pair s to CTA s mod gridDim.x balances the work, and the CTAs
+// working at the same time share a (head, row)'s K and V tiles in L2.  The
+// K/V ring runs on across items, the next item's Q tiles load as soon as the
+// current item's last products that read them are done, and the next item's
+// first scores are computed while the softmax warps still write the current
+// item's output (its first P V product waits for that).
 // 320 threads:
-//   warp 0       TMA: both Q tiles once, then K_j and V_j through two stages
+//   warp 0       TMA: Q_a and Q_b per item, K_j and V_j through two stages
 //                each (a stage is released when both tiles' products that
 //                read it are done);
 //   warp 1       TMEM owner and single-thread MMA issue in the order above;
@@ -375,7 +384,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 //                per query row holding its 128 scores, so the row maximum
 //                needs no exchange between threads; the maximum is raised
 //                only past 2^8 (O rescaled in TMEM then), and P is written as
-//                bf16 over the scores it replaces (key k in column k / 2).
+//                bf16 over the scores it replaces (key k in column k / 2);
+//                at the item's end O / l and lse of the row.
 // TMEM columns: S_a [0,128), S_b [128,256), O_a [256,384), O_b [384,512).
 // The MMAs run in issue order, so S_x(j+1) never overwrites P_x(j) before
 // PV_x(j) has read it, and the commit that publishes S_x(j+1) also covers
@@ -386,6 +396,36 @@ constexpr int PP_OFF_K = 2 * TILE;   // 2 stages
 constexpr int PP_OFF_V = 4 * TILE;   // 2 stages
 constexpr int PP_OFF_BAR = 6 * TILE;
 constexpr int kPPSmem = PP_OFF_BAR + 512;
+
+// This CTA's items in order: item pair s (stride gridDim.x) is query-tile
+// pairs npairs - 1 - j (sub 0) and j (sub 1) of one (head, row).
+struct FwdWalk {
+  int s, sub;
+  __device__ __forceinline__ void start() {
+    s = blockIdx.x;
+    sub = 0;
+  }
+  __device__ __forceinline__ bool valid(int nsuper) const { return s < nsuper; }
+  // Query-tile pair, head and batch row of the current item.
+  __device__ __forceinline__ void item(const FwdArgs& a, int npairs, int& pr, int& h, int& b) const {
+    const int spg = (npairs + 1) / 2;
+    const int grp = s / spg;
+    const int j = s - grp * spg;
+    pr = sub ? j : npairs - 1 - j;
+    h = grp % a.H;
+    b = grp / a.H;
+  }
+  __device__ __forceinline__ void next(int npairs) {
+    const int j = s % ((npairs + 1) / 2);
+    if (sub == 0 && npairs - 1 - j != j) {
+      sub = 1;
+    } else {
+      sub = 0;
+      s += gridDim.x;
+    }
+  }
+};
+
 __global__ void __launch_bounds__(kPPThreads, 1)
     attn_fwd_pp_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const FwdArgs a) {
@@ -396,29 +436,28 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   }
   uint8_t* smem = smem_raw;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PP_OFF_BAR);
-  uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;    // [2]
-  uint64_t* k_empty = bars + 3;   // [2]
-  uint64_t* v_full = bars + 5;    // [2]
-  uint64_t* v_empty = bars + 7;   // [2]
-  uint64_t* s_full = bars + 9;    // [2 tiles]
-  uint64_t* p_full = bars + 11;   // [2 tiles]
-  uint64_t* o_full = bars + 13;   // [2 tiles]
-  uint64_t* drained = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* q_full = bars + 0;    // [2 tiles]
+  uint64_t* q_empty = bars + 2;   // [2 tiles]
+  uint64_t* k_full = bars + 4;    // [2]
+  uint64_t* k_empty = bars + 6;   // [2]
+  uint64_t* v_full = bars + 8;    // [2]
+  uint64_t* v_empty = bars + 10;  // [2]
+  uint64_t* s_full = bars + 12;   // [2 tiles]
+  uint64_t* p_full = bars + 14;   // [2 tiles]
+  uint64_t* o_full = bars + 16;   // [2 tiles]
+  uint64_t* o_empty = bars + 18;  // [2 tiles]
+  uint64_t* drained = bars + 20;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int npairs = (a.nqb + 1) / 2;
-  const int pr = npairs - 1 - (int)blockIdx.x;  // heaviest pairs first
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int qt0 = 2 * pr;                        // tile a; tile b = qt0 + 1 when it exists
-  const bool has_b = qt0 + 1 < a.nqb;
-  const int nkv = has_b ? qt0 + 2 : qt0 + 1;     // key tiles 0 .. the last tile's diagonal
+  const int nsuper = (npairs + 1) / 2 * a.H * a.B;
 
   if (threadIdx.x == 0) {
-    tc::mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&q_full[i], 1);
+      tc::mbar_init(&q_empty[i], 1);
       tc::mbar_init(&k_full[i], 1);
       tc::mbar_init(&k_empty[i], 1);
       tc::mbar_init(&v_full[i], 1);
@@ -426,6 +465,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       tc::mbar_init(&s_full[i], 1);
       tc::mbar_init(&p_full[i], 128);
       tc::mbar_init(&o_full[i], 1);
+      tc::mbar_init(&o_empty[i], 128);
     }
     tc::mbar_init(drained, 1);
     *abort_flag = 0;
@@ -439,38 +479,57 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int col0 = h * HD;
 
   if (warp == 0) {
     if (lane == 0) {
       tc::tma_prefetch_desc(&tq);
       tc::tma_prefetch_desc(&tk);
       tc::tma_prefetch_desc(&tv);
-      tc::mbar_arrive_expect_tx(q_full, has_b ? 2 * TILE : TILE);
-      for (int x = 0; x < (has_b ? 2 : 1); ++x)
-        for (int c = 0; c < 2; ++c)
-          tc::tma_load_3d(smem + PP_OFF_QA + x * TILE + c * (TILE / 2), &tq, q_full, col0 + 64 * c,
-                          (qt0 + x) * BQ, b);
+      int nq[2] = {0, 0};  // loads into each Q slot so far
+      int g = 0;           // K/V tiles loaded so far (ring position)
       int issued_k = 0, issued_v = 0;
       bool ok = true;
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!tc::mbar_wait(&k_empty[st], ph ^ 1, abort_flag, a.status)) { ok = false; break; }
-        tc::mbar_arrive_expect_tx(&k_full[st], TILE);
-        for (int c = 0; c < 2; ++c)
-          tc::tma_load_3d(smem + PP_OFF_K + st * TILE + c * (TILE / 2), &tk, &k_full[st],
-                          col0 + 64 * c, j * BKV, b);
-        ++issued_k;
-        if (!tc::mbar_wait(&v_empty[st], ph ^ 1, abort_flag, a.status)) { ok = false; break; }
-        tc::mbar_arrive_expect_tx(&v_full[st], TILE);
-        for (int c = 0; c < 2; ++c)
-          tc::tma_load_3d(smem + PP_OFF_V + st * TILE + c * (TILE / 2), &tv, &v_full[st],
-                          col0 + 64 * c, j * BKV, b);
-        ++issued_v;
+      FwdWalk w;
+      for (w.start(); w.valid(nsuper) && ok; w.next(npairs)) {
+        int pr, h, b;
+        w.item(a, npairs, pr, h, b);
+        const int qt0 = 2 * pr;
+        const bool has_b = qt0 + 1 < a.nqb;
+        const int nkv = has_b ? qt0 + 2 : qt0 + 1;
+        const int col0 = h * HD;
+        for (int x = 0; x < (has_b ? 2 : 1); ++x) {
+          // The slot is free once the products of the previous item that
+          // read it are done.
+          if (nq[x] > 0 && !tc::mbar_wait(&q_empty[x], (nq[x] - 1) & 1, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
+          tc::mbar_arrive_expect_tx(&q_full[x], TILE);
+          for (int c = 0; c < 2; ++c)
+            tc::tma_load_3d(smem + PP_OFF_QA + x * TILE + c * (TILE / 2), &tq, &q_full[x], col0 + 64 * c,
+                            (qt0 + x) * BQ, b);
+          ++nq[x];
+        }
+        for (int j = 0; j < nkv && ok; ++j, ++g) {
+          const int st = g & 1;
+          const uint32_t ph = (g >> 1) & 1;
+          if (!tc::mbar_wait(&k_empty[st], ph ^ 1, abort_flag, a.status)) { ok = false; break; }
+          tc::mbar_arrive_expect_tx(&k_full[st], TILE);
+          for (int c = 0; c < 2; ++c)
+            tc::tma_load_3d(smem + PP_OFF_K + st * TILE + c * (TILE / 2), &tk, &k_full[st],
+                            col0 + 64 * c, j * BKV, b);
+          ++issued_k;
+          if (!tc::mbar_wait(&v_empty[st], ph ^ 1, abort_flag, a.status)) { ok = false; break; }
+          tc::mbar_arrive_expect_tx(&v_full[st], TILE);
+          for (int c = 0; c < 2; ++c)
+            tc::tma_load_3d(smem + PP_OFF_V + st * TILE + c * (TILE / 2), &tv, &v_full[st],
+                            col0 + 64 * c, j * BKV, b);
+          ++issued_v;
+        }
       }
       if (!ok) {
-        drain_wait(q_full, 0);
+        for (int x = 0; x < 2; ++x)
+          if (nq[x] > 0) drain_wait(&q_full[x], (nq[x] - 1) & 1);
         for (int j = max(0, issued_k - 2); j < issued_k; ++j) drain_wait(&k_full[j & 1], (j >> 1) & 1);
         for (int j = max(0, issued_v - 2); j < issued_v; ++j) drain_wait(&v_full[j & 1], (j >> 1) & 1);
       }
@@ -482,10 +541,10 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       const uint64_t qdesc = tc::smem_desc_sw128(tc::smem_u32(smem + PP_OFF_QA), 16, 1024);
       const uint64_t kdesc = tc::smem_desc_sw128(tc::smem_u32(smem + PP_OFF_K), 16, 1024);
       const uint64_t vdesc = tc::smem_desc_sw128(tc::smem_u32(smem + PP_OFF_V), TILE / 2, 1024);
-      // S_x(j) = Q_x K_j^T into tile x's score columns.
-      auto issue_s = [&](int x, int j) {
+      // S_x = Q_x K^T (K from ring slot ks) into tile x's score columns.
+      auto issue_s = [&](int x, int ks) {
         const uint64_t qd = tc::desc_add(qdesc, x * TILE);
-        const uint64_t kd = tc::desc_add(kdesc, (j & 1) * TILE);
+        const uint64_t kd = tc::desc_add(kdesc, ks * TILE);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (TILE / 2) + (kk & 3) * 32;
@@ -494,71 +553,101 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         }
         tc::umma_commit(&s_full[x]);
       };
-      // O_x += P_x(j) V_j, P from TMEM (key k in column k / 2 of the tile's
-      // score block; 16 keys per MMA).
-      auto issue_pv = [&](int x, int j) {
-        const uint64_t vd = tc::desc_add(vdesc, (j & 1) * TILE);
+      // O_x (+)= P_x V (V from ring slot vs), P from TMEM (key k in column
+      // k / 2 of the tile's score block; 16 keys per MMA).
+      auto issue_pv = [&](int x, int vs, bool acc) {
+        const uint64_t vd = tc::desc_add(vdesc, vs * TILE);
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk)
           tc::umma_bf16_ts(tmem + 256 + 128 * x, tmem + 128 * x + kk * 8,
-                           tc::desc_add(vd, kk * 2048), id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                           tc::desc_add(vd, kk * 2048), id_pv, (acc || kk > 0) ? 1u : 0u);
       };
-      const int last[2] = {qt0, qt0 + 1};  // each tile's last key tile (its diagonal)
-      bool ok = tc::mbar_wait(q_full, 0, abort_flag, a.status) &&
-                tc::mbar_wait(&k_full[0], 0, abort_flag, a.status);
-      if (ok) {
-        tc::tc_fence_after();
-        issue_s(0, 0);
-        if (has_b) issue_s(1, 0);
-        tc::umma_commit(&k_empty[0]);
-      }
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int st = j & 1;
-        if (!tc::mbar_wait(&v_full[st], (j >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
-        bool k_next = false;  // K_{j+1} has landed
-        for (int x = 0; x < (has_b ? 2 : 1); ++x) {
-          if (j > last[x]) continue;
-          if (!tc::mbar_wait(&p_full[x], j & 1, abort_flag, a.status)) { ok = false; break; }
+      int nq[2] = {0, 0}, np[2] = {0, 0}, no[2] = {0, 0};
+      int g = 0;
+      bool ok = true;
+      FwdWalk w;
+      for (w.start(); w.valid(nsuper) && ok; w.next(npairs)) {
+        int pr, h, b;
+        w.item(a, npairs, pr, h, b);
+        const int qt0 = 2 * pr;
+        const bool has_b = qt0 + 1 < a.nqb;
+        const int xs = has_b ? 2 : 1;
+        const int nkv = has_b ? qt0 + 2 : qt0 + 1;
+        const int last[2] = {qt0, qt0 + 1};  // each tile's last key tile (its diagonal)
+        if (!tc::mbar_wait(&k_full[g & 1], (g >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+        for (int x = 0; x < xs && ok; ++x) {
+          ok = tc::mbar_wait(&q_full[x], nq[x] & 1, abort_flag, a.status);
+          ++nq[x];
+          if (!ok) break;
           tc::tc_fence_after();
-          issue_pv(x, j);
-          if (j == last[x]) {
-            tc::umma_commit(&o_full[x]);
-            continue;
-          }
-          if (!k_next) {
-            if (!tc::mbar_wait(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, abort_flag, a.status)) {
+          issue_s(x, g & 1);
+          if (last[x] == 0) tc::umma_commit(&q_empty[x]);  // the item's only scores of tile x
+        }
+        if (!ok) break;
+        tc::umma_commit(&k_empty[g & 1]);
+        for (int j = 0; j < nkv && ok; ++j) {
+          const int st = (g + j) & 1;
+          if (!tc::mbar_wait(&v_full[st], ((g + j) >> 1) & 1, abort_flag, a.status)) { ok = false; break; }
+          bool k_next = false;  // K_{j+1} has landed
+          for (int x = 0; x < xs; ++x) {
+            if (j > last[x]) continue;
+            if (!tc::mbar_wait(&p_full[x], np[x] & 1, abort_flag, a.status)) { ok = false; break; }
+            ++np[x];
+            // The item's first product overwrites O_x: the softmax warps
+            // must have written out the previous item's.
+            if (j == 0 && no[x] > 0 && !tc::mbar_wait(&o_empty[x], (no[x] - 1) & 1, abort_flag, a.status)) {
               ok = false;
               break;
             }
             tc::tc_fence_after();
-            k_next = true;
+            issue_pv(x, st, j > 0);
+            if (j == last[x]) {
+              tc::umma_commit(&o_full[x]);
+              ++no[x];
+              continue;
+            }
+            if (!k_next) {
+              if (!tc::mbar_wait(&k_full[(g + j + 1) & 1], ((g + j + 1) >> 1) & 1, abort_flag, a.status)) {
+                ok = false;
+                break;
+              }
+              tc::tc_fence_after();
+              k_next = true;
+            }
+            issue_s(x, (g + j + 1) & 1);
+            if (j + 1 == last[x]) tc::umma_commit(&q_empty[x]);  // Q_x's last reader
           }
-          issue_s(x, j + 1);
+          if (!ok) break;
+          tc::umma_commit(&v_empty[st]);
+          if (k_next) tc::umma_commit(&k_empty[(g + j + 1) & 1]);
         }
-        if (!ok) break;
-        tc::umma_commit(&v_empty[st]);
-        if (k_next) tc::umma_commit(&k_empty[(j + 1) & 1]);
+        g += nkv;
       }
       tc::umma_commit(drained);
       drain_wait(drained, 0);
     }
-  } else if (warp < 10) {
+  } else {
     // Softmax of tile x: warps 2..5 (x = 0) and 6..9 (x = 1), one thread per
     // query row (a warp may only reach the TMEM lanes of quarter warp % 4).
     const int x = (warp - 2) >> 2;
     const int qw = warp & 3;
     const int row = qw * 32 + lane;
-    if (x == 0 || has_b) {
-      const int qb = qt0 + x;
+    const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
+    const uint32_t s_base = lane_base + 128 * x;
+    const uint32_t o_base = lane_base + 256 + 128 * x;
+    int ns = 0, no = 0;  // score tiles and items of tile x so far
+    bool ok = true;
+    FwdWalk w;
+    for (w.start(); w.valid(nsuper) && ok; w.next(npairs)) {
+      int pr, h, b;
+      w.item(a, npairs, pr, h, b);
+      const int qb = 2 * pr + x;
+      if (qb >= a.nqb) continue;  // no tile b in this item
       const int qi = qb * BQ + row;
       const int key_hi = min(qi, a.T - 1);
-      const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
-      const uint32_t s_base = lane_base + 128 * x;
-      const uint32_t o_base = lane_base + 256 + 128 * x;
       float m_used = -INFINITY, l = 0.f;
-      bool ok = true;
-      for (int j = 0; j <= qb; ++j) {
-        ok = tc::mbar_wait(&s_full[x], j & 1, abort_flag, a.status);
+      for (int j = 0; j <= qb; ++j, ++ns) {
+        ok = tc::mbar_wait(&s_full[x], ns & 1, abort_flag, a.status);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc::tc_fence_after();
         uint32_t r[4][32];
@@ -624,34 +713,36 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         tc::tc_fence_before();
         tc::mbar_arrive(&p_full[x]);
       }
-      if (ok) {
-        ok = tc::mbar_wait(&o_full[x], 0, abort_flag, a.status);
-        ok = __all_sync(0xffffffffu, ok);
-      }
-      if (ok) {
-        tc::tc_fence_after();
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        __nv_bfloat16* orow = a.o + ((int64_t)b * a.T + qi) * a.ldo + col0;
+      if (!ok) break;
+      ok = tc::mbar_wait(&o_full[x], no & 1, abort_flag, a.status);
+      ++no;
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc::tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* orow = a.o + ((int64_t)b * a.T + qi) * a.ldo + h * HD;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tc::tmem_ld_32x32b_x32(o_base + c * 32, o);
-          tc::tmem_ld_wait();
-          if (qi < a.T) {
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tc::tmem_ld_32x32b_x32(o_base + c * 32, o);
+        tc::tmem_ld_wait();
+        if (c == 3) {  // O_x is read: the next item's first product may overwrite it
+          tc::tc_fence_before();
+          tc::mbar_arrive(&o_empty[x]);
+        }
+        if (qi < a.T) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              uint4 v;
-              v.x = pack_bf16x2(__uint_as_float(o[8 * u + 0]) * inv, __uint_as_float(o[8 * u + 1]) * inv);
-              v.y = pack_bf16x2(__uint_as_float(o[8 * u + 2]) * inv, __uint_as_float(o[8 * u + 3]) * inv);
-              v.z = pack_bf16x2(__uint_as_float(o[8 * u + 4]) * inv, __uint_as_float(o[8 * u + 5]) * inv);
-              v.w = pack_bf16x2(__uint_as_float(o[8 * u + 6]) * inv, __uint_as_float(o[8 * u + 7]) * inv);
-              reinterpret_cast<uint4*>(orow + c * 32)[u] = v;
-            }
+          for (int u = 0; u < 4; ++u) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(o[8 * u + 0]) * inv, __uint_as_float(o[8 * u + 1]) * inv);
+            v.y = pack_bf16x2(__uint_as_float(o[8 * u + 2]) * inv, __uint_as_float(o[8 * u + 3]) * inv);
+            v.z = pack_bf16x2(__uint_as_float(o[8 * u + 4]) * inv, __uint_as_float(o[8 * u + 5]) * inv);
+            v.w = pack_bf16x2(__uint_as_float(o[8 * u + 6]) * inv, __uint_as_float(o[8 * u + 7]) * inv);
+            reinterpret_cast<uint4*>(orow + c * 32)[u] = v;
           }
         }
-        if (qi < a.T)
-          a.lse[((int64_t)b * a.H + h) * a.T + qi] = (m_used + log2f(l)) * 0.69314718055994531f;
       }
+      if (qi < a.T)
+        a.lse[((int64_t)b * a.H + h) * a.T + qi] = (m_used + log2f(l)) * 0.69314718055994531f;
     }
   }
   tc::tc_fence_before();
@@ -2186,14 +2277,16 @@ nc_status attention_fwd_ex(const void* q, int64_t ldq, const void* k, const void
   // unbounded, which also keeps the kernels' window sums (up to ~2T) in range.
   a.window = (window < 0 || window >= T - 1) ? -1 : window;
   a.status = status;
+  a.B = B;
   const double flops = 4.0 * B * H * HD * causal_pairs(T, a.window);
   Probe probe(prof, s, "attn_fwd", flops, 0.0);
   if (a.group > 1 || a.window >= 0) {
     dim3 grid(a.nqb, H, B);
     attn_fwd_tc_kernel<true><<<grid, kThreads, kSmem, s>>>(mq, mk, mv, a);
   } else {
-    dim3 grid((a.nqb + 1) / 2, H, B);  // two query tiles per CTA
-    attn_fwd_pp_kernel<<<grid, kPPThreads, kPPSmem, s>>>(mq, mk, mv, a);
+    // Persistent: one CTA per SM over the items (two query tiles each).
+    const int nsuper = ((a.nqb + 1) / 2 + 1) / 2 * H * B;
+    attn_fwd_pp_kernel<<<(unsigned)std::min(nsuper, num_sms()), kPPThreads, kPPSmem, s>>>(mq, mk, mv, a);
   }
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
