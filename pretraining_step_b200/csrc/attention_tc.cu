@@ -680,14 +680,18 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         }
         const float neg_mu = (m_used == -INFINITY) ? 0.f : -m_used;
         l *= alpha;
+        // Arguments two at a time (packed fp32 pairs: one issue slot per two
+        // scores, the same rounding as scalar fma).
+        const float2 sl2v = make_float2(a.sl2, a.sl2), nmu = make_float2(neg_mu, neg_mu);
         float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float p0 = ex2(fmaf(__uint_as_float(r[c][2 * i]), a.sl2, neg_mu));
-            const float p1 = ex2(fmaf(__uint_as_float(r[c][2 * i + 1]), a.sl2, neg_mu));
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(r[c][2 * i]), __uint_as_float(r[c][2 * i + 1])),
+                                        sl2v, nmu);
+            const float p0 = ex2(x.x), p1 = ex2(x.y);
             ls[(2 * i) & 3] += p0;
             ls[(2 * i + 1) & 3] += p1;
             pk[i] = pack_bf16x2(p0, p1);
@@ -699,13 +703,18 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
         // O is idle here: the commit that published S_j also covers P_{j-1} V_{j-1}.
         if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          const float2 al = make_float2(alpha, alpha);
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             uint32_t o[32];
             tc::tmem_ld_32x32b_x32(o_base + c * 32, o);
             tc::tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            for (int i = 0; i < 32; i += 2) {
+              const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), al);
+              o[i] = __float_as_uint(v.x);
+              o[i + 1] = __float_as_uint(v.y);
+            }
             tc::tmem_st_32x32b_x32(o_base + c * 32, o);
           }
         }
@@ -1465,7 +1474,7 @@ __global__ void __launch_bounds__(kKvThreads)
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int q = q0 + lane + 32 * u;
-        lq[lane + 32 * u] = q < a.T ? lse_bh[q] * 1.4426950408889634f : INFINITY;
+        lq[lane + 32 * u] = q < a.T ? -lse_bh[q] * 1.4426950408889634f : -INFINITY;  // negated
       }
       if (lane == 0) {
         reinterpret_cast<int2*>(smem + KV_OFF_TI)[st] = make_int2(q0, c.m.kb);
@@ -1484,7 +1493,7 @@ __global__ void __launch_bounds__(kKvThreads)
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int q = q0 + lane + 32 * u;
-        ldd[lane + 32 * u] = q < a.T ? d_bh[q] : 0.f;
+        ldd[lane + 32 * u] = q < a.T ? -d_bh[q] : 0.f;  // negated
       }
       if (lane == 0) {
         tc::mbar_arrive_expect_tx(&do_full[st], TILE);
@@ -1664,10 +1673,17 @@ __global__ void __launch_bounds__(kKvThreads)
           l[4 * u + 3] = v.w;
         }
         tc::tmem_ld_wait();
-        // Every argument first, then the 32 independent exponentials.
+        // Every argument first (packed fp32 pairs, the same rounding as scalar
+        // fma; l holds -lse log2(e)), then the 32 independent exponentials.
         float p[32];
+        const float2 sl2v = make_float2(a.sl2, a.sl2);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) p[i] = fmaf(__uint_as_float(sv[i]), a.sl2, -l[i]);
+        for (int i = 0; i < 32; i += 2) {
+          const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), sl2v,
+                                      make_float2(l[i], l[i + 1]));
+          p[i] = x.x;
+          p[i + 1] = x.y;
+        }
 #pragma unroll
         for (int i = 0; i < 32; ++i) p[i] = ex2(p[i]);
         if (edge) {
@@ -1713,10 +1729,11 @@ __global__ void __launch_bounds__(kKvThreads)
         uint32_t pd[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float2 p = unpack_bf16x2(pk[cc][i]);
-          const float d0 = p.x * (__uint_as_float(dpv[2 * i]) - dl[2 * i]);
-          const float d1 = p.y * (__uint_as_float(dpv[2 * i + 1]) - dl[2 * i + 1]);
-          pd[i] = pack_bf16x2(d0, d1);
+          // dl holds -D: dS = P (dP - D) as a packed add and multiply.
+          const float2 dd = __fadd2_rn(make_float2(__uint_as_float(dpv[2 * i]), __uint_as_float(dpv[2 * i + 1])),
+                                       make_float2(dl[2 * i], dl[2 * i + 1]));
+          const float2 d = __fmul2_rn(unpack_bf16x2(pk[cc][i]), dd);
+          pd[i] = pack_bf16x2(d.x, d.y);
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
