@@ -78,6 +78,13 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = globaltimer();
   while (!tc::mbar_try_wait(bar, parity))
@@ -664,15 +671,16 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             for (int i = 0; i < 32; ++i)
               if (j * BKV + 32 * c + i > key_hi) r[c][i] = __float_as_uint(-INFINITY);
         }
+        // Row maximum with the three-input max: two scores per instruction.
         float pm[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) pm[u] = -INFINITY;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int i = 0; i < 32; ++i) pm[i & 7] = fmaxf(pm[i & 7], __uint_as_float(r[c][i]));
-        const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                               fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7]))) * a.sl2;
+          for (int i = 0; i < 32; i += 2)
+            pm[(i >> 1) & 7] = fmax3(pm[(i >> 1) & 7], __uint_as_float(r[c][i]), __uint_as_float(r[c][i + 1]));
+        const float mx = fmax3(fmax3(pm[0], pm[1], pm[2]), fmax3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7])) * a.sl2;
         float alpha = 1.f;
         if (mx > m_used + kRescaleThreshold) {
           alpha = ex2(m_used - mx);  // 0 on the first tile
