@@ -91,12 +91,29 @@ struct TileCoord {
 // and a group's A rows, which stay in L2.
 constexpr int kGroupM = 16;
 constexpr int kGroupMinTilesN = 32;
+// Tiles of one (split, batch) plane.  A symmetric output (tiles_m < 0, a
+// square plane of tiles_n x tiles_n tiles) computes only the tiles on or
+// above the diagonal; the epilogue also stores each off-diagonal tile's
+// transpose.
+__device__ __forceinline__ int plane_tiles(const Args& p) {
+  return p.tiles_m >= 0 ? p.tiles_m * p.tiles_n : p.tiles_n * (p.tiles_n + 1) / 2;
+}
+
 __device__ __forceinline__ TileCoord decode(const Args& p, int t) {
   TileCoord c;
-  const int plane = p.tiles_m * p.tiles_n;
+  const int plane = plane_tiles(p);
   const int r = t % plane;
   t /= plane;
-  if (p.tiles_n > kGroupMinTilesN) {
+  if (p.tiles_m < 0) {  // row mb holds column tiles mb .. tiles_n - 1
+    int mb = 0, rem = r, len = p.tiles_n;
+    while (rem >= len) {
+      rem -= len;
+      ++mb;
+      --len;
+    }
+    c.mb = mb;
+    c.nb = mb + rem;
+  } else if (p.tiles_n > kGroupMinTilesN) {
     const int gsize = kGroupM * p.tiles_n;
     const int g = r / gsize;
     const int gm = min(kGroupM, p.tiles_m - g * kGroupM);  // rows in this (possibly last) group
@@ -259,7 +276,8 @@ __device__ __forceinline__ void store_row_chunk(const Args& p, int b, int row, i
 // each store instruction covers whole lines instead of 16 bytes of 32
 // different lines.  Rows past M and columns past N are skipped.
 __device__ __forceinline__ void stage_store_chunk(const Args& p, uint8_t* slot, int lane, bool f32, int b,
-                                                  int row0, int col0, const float (&w)[32]) {
+                                                  int row0, int col0, const float (&w)[32],
+                                                  bool mirror = false) {
   const uint32_t base = tc::smem_u32(slot);
   if (f32) {
     const uint32_t rowa = base + lane * 128;
@@ -314,6 +332,33 @@ __device__ __forceinline__ void stage_store_chunk(const Args& p, uint8_t* slot, 
               d[i] = __ushort_as_bfloat16((unsigned short)h);
             }
         }
+      }
+    }
+    if (mirror) {
+      // The block's transpose at rows col0.., columns row0.. (a symmetric
+      // output's other triangle): lane l gathers 8 block rows of column
+      // it * 8 + l / 4 and stores them as 16 contiguous bytes.
+      const uint16_t* sh = reinterpret_cast<const uint16_t*>(slot);
+      __nv_bfloat16* Dt = (__nv_bfloat16*)p.D + (int64_t)b * p.stride_d + row0;
+#pragma unroll
+      for (int it = 0; it < 4; ++it) {
+        const int cc = it * 8 + (lane >> 2), r0 = (lane & 3) * 8;
+        uint32_t e[4];
+#pragma unroll
+        for (int k = 0; k < 8; k += 2) {
+          const int ra = r0 + k, rb = r0 + k + 1;
+          const uint32_t lo = sh[(ra * 64 + (((cc >> 3) ^ ((ra >> 1) & 3)) << 4)) / 2 + (cc & 7)];
+          const uint32_t hi = sh[(rb * 64 + (((cc >> 3) ^ ((rb >> 1) & 3)) << 4)) / 2 + (cc & 7)];
+          e[k / 2] = lo | (hi << 16);
+        }
+        if (cc < ncol && col0 + cc < p.M && row0 + r0 + 8 <= p.N)
+          *reinterpret_cast<uint4*>(Dt + (int64_t)(col0 + cc) * p.ldd + r0) = make_uint4(e[0], e[1], e[2], e[3]);
+        else if (cc < ncol && col0 + cc < p.M)
+          for (int i = 0; i < 8; ++i)
+            if (row0 + r0 + i < p.N) {
+              const uint32_t h = (e[i >> 1] >> ((i & 1) * 16)) & 0xffffu;
+              Dt[(int64_t)(col0 + cc) * p.ldd + r0 + i] = __ushort_as_bfloat16((unsigned short)h);
+            }
       }
     }
   }
@@ -673,7 +718,8 @@ __device__ __forceinline__ void aux_read_slot(const uint8_t* slot, int lane, boo
 // Aux epilogues of the ring kernel: the output has the aux operand's type, so
 // the finished rows go out through the slot that held the aux rows.
 __device__ __forceinline__ void aux_epilogue_chunk(const Args& p, uint8_t* slot, int lane, bool f32,
-                                                   int b, int row0, int col0, const uint32_t (&r)[32]) {
+                                                   int b, int row0, int col0, const uint32_t (&r)[32],
+                                                   bool mirror) {
   float x[32];
   aux_read_slot(slot, lane, f32, x);
   __syncwarp();  // every lane has read its aux row before any is overwritten
@@ -684,7 +730,7 @@ __device__ __forceinline__ void aux_epilogue_chunk(const Args& p, uint8_t* slot,
     const float a = __uint_as_float(r[j]) * p.alpha;
     w[j] = f32 ? x[j] + a : (relu2_bwd ? 2.f * sqrt_approx(fmaxf(x[j], 0.f)) * a : a + p.beta * x[j]);
   }
-  stage_store_chunk(p, slot, lane, f32, b, row0, col0, w);
+  stage_store_chunk(p, slot, lane, f32, b, row0, col0, w, mirror);
 }
 
 // Plain epilogues (bf16 / fp32 store, ReLU^2) of the pair kernel through the
@@ -742,7 +788,7 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
   const uint32_t tmem_base = *tmem_slot;
 
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-  const int total = p.tiles_m * p.tiles_n * p.split_k * p.batch;  // tiles_m counts 256-row tiles
+  const int total = plane_tiles(p) * p.split_k * p.batch;  // tiles_m counts 256-row tiles
 
   if (warp == 0) {
     if (lane == 0) {
@@ -874,6 +920,7 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
       tc::tc_fence_after();
       const int row = c.mb * 2 * BM + (int)rank * BM + row_in_tile;
       const bool aux = epi_has_aux(p.epi);
+      const bool mirror = p.tiles_m < 0 && c.mb != c.nb;  // symmetric output, off the diagonal
       if constexpr (ROPE) {  // separate instantiation: the other GEMMs carry no RoPE code
         rope_head_epilogue(p, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + half * CH * 32, c.b,
                            row, c.nb * BN + half * CH * 32, ring, lane);
@@ -892,7 +939,7 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
             break;
           }
           if (col0 < p.N)
-            aux_epilogue_chunk(p, ring + slot * slot_bytes, lane, xf32, c.b, row - lane, col0, r);
+            aux_epilogue_chunk(p, ring + slot * slot_bytes, lane, xf32, c.b, row - lane, col0, r, mirror);
           // Every lane is done with the slot: order its accesses before the
           // TMA refill of the same slot with the chunk `slots` ahead.
           tc::fence_proxy_async_smem();
@@ -920,7 +967,7 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
               const float a = __uint_as_float(r[j]) * p.alpha;
               w[j] = p.epi == NC_EPI_RELU2 ? fmaxf(a, 0.f) * fmaxf(a, 0.f) : a;
             }
-            stage_store_chunk(p, ring, lane, f32, c.b, row - lane, col0, w);
+            stage_store_chunk(p, ring, lane, f32, c.b, row - lane, col0, w, mirror);
           }
         }
       } else {
@@ -1045,7 +1092,7 @@ nc_status launch_bn(const nc_gemm_desc& d, int split, int* status, const char* t
 
 template <bool ROPE, bool XR>
 nc_status launch_pair(const nc_gemm_desc& d, int split, int* status, const char* tag,
-                      cudaStream_t s, Profiler* prof) {
+                      cudaStream_t s, Profiler* prof, bool symmetric = false) {
   using C = std::conditional_t<XR, Cfg2X, Cfg2>;
   static DeviceOnce smem_attr;
   NC_TRY(once_per_device(smem_attr, []() -> nc_status {
@@ -1099,7 +1146,12 @@ nc_status launch_pair(const nc_gemm_desc& d, int split, int* status, const char*
     a.rstd_k = d.rstd_k;
   }
   a.status = status;
-  const int64_t total = (int64_t)a.tiles_m * a.tiles_n * a.split_k * a.batch;
+  int64_t plane = (int64_t)a.tiles_m * a.tiles_n;
+  if (symmetric) {  // tiles_m < 0 marks it; the kernel walks the upper triangle
+    plane = (int64_t)a.tiles_n * (a.tiles_n + 1) / 2;
+    a.tiles_m = -a.tiles_n;
+  }
+  const int64_t total = plane * a.split_k * a.batch;
   if (total >= (1ll << 31)) return fail(NC_ERR_INVALID_ARG, "gemm: too many tiles");
   const int pairs = (int)std::min<int64_t>(total, num_sms() / 2);
   cudaLaunchConfig_t cfg = {};
@@ -1114,7 +1166,9 @@ nc_status launch_pair(const nc_gemm_desc& d, int split, int* status, const char*
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const double flops = 2.0 * d.M * (double)d.N * d.K * d.batch;
+  // Algorithmic FLOPs: a symmetric output counts the tiles it computes.
+  const double flops = symmetric ? 2.0 * d.K * d.batch * (double)plane * 256.0 * 256.0
+                                 : 2.0 * d.M * (double)d.N * d.K * d.batch;
   Probe probe(prof, s, tag, flops, 0.0);
   if constexpr (XR)
     NC_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_tc2_aux_kernel, ta, tb, tx, a));
@@ -1187,7 +1241,8 @@ nc_status gemm_launch(const GemmLaunch& g, cudaStream_t s, Profiler* prof) {
   const int waste256 = ((d.N + 255) / 256) * 256 - d.N;
   const int waste128 = ((d.N + 127) / 128) * 128 - d.N;
   // (the RoPE/QK-norm epilogue needs 256-wide tiles: each warp-half is a head)
-  const bool bn256 = rope || (d.N > 128 && waste256 <= waste128);
+  // (a symmetric output walks square 256 x 256 tiles whatever the edge waste)
+  const bool bn256 = rope || g.symmetric || (d.N > 128 && waste256 <= waste128);
   const int bn = bn256 ? 256 : 128;
   const int num_kb = (d.K + BK - 1) / BK;
   const double operand_bytes = 2.0 * ((double)d.M + d.N) * d.K * d.batch;
@@ -1198,6 +1253,10 @@ nc_status gemm_launch(const GemmLaunch& g, cudaStream_t s, Profiler* prof) {
   if (split > num_kb) split = num_kb;
   // 256 x 256 tiles on a CTA pair whenever M spans more than one 128-row
   // tile and 256-wide column tiles fit N; 128 x BN on one CTA otherwise.
+  if (g.symmetric &&
+      (d.M != d.N || !bn256 || d.M <= BM || split != 1 ||
+       (d.epi != NC_EPI_STORE_BF16 && d.epi != NC_EPI_AXPBY_BF16)))
+    return fail(NC_ERR_INVALID_ARG, "gemm: a symmetric output needs M == N > 128, one split and a bf16 epilogue");
   if (bn256 && d.M > BM) {
     if (d.split_k <= 0) {
       const int64_t tiles = (int64_t)((d.M + 2 * BM - 1) / (2 * BM)) * ((d.N + 255) / 256) * d.batch;
@@ -1207,8 +1266,8 @@ nc_status gemm_launch(const GemmLaunch& g, cudaStream_t s, Profiler* prof) {
     // Aux epilogues read the aux operand by TMA (rows and batch strides of
     // 16-byte multiples, which the checks above already imply).
     if (needs_aux && (d.batch == 1 || aligned(d.stride_aux)))
-      return launch_pair<false, true>(d, split, g.status, g.tag, s, prof);
-    return launch_pair<false, false>(d, split, g.status, g.tag, s, prof);
+      return launch_pair<false, true>(d, split, g.status, g.tag, s, prof, g.symmetric);
+    return launch_pair<false, false>(d, split, g.status, g.tag, s, prof, g.symmetric);
   }
   if (rope) return launch_bn<256, true>(d, split, g.status, g.tag, s, prof);
   return bn256 ? launch_bn<256, false>(d, split, g.status, g.tag, s, prof)

@@ -26,6 +26,10 @@ struct GemmLaunch {
   nc_gemm_desc d;
   int* status;             // device status word (may be null)
   const char* tag = "gemm_tc";  // profiler class
+  // The output is symmetric (M == N, e.g. X X^T): only the 256 x 256 tiles on
+  // or above the diagonal are computed, each off-diagonal one also stored
+  // transposed (bf16 store or a*acc + b*aux epilogues, one split, CTA pairs).
+  bool symmetric = false;
 };
 // d.split_k == 0 selects the split automatically (NC_EPI_ACC_F32 only).
 nc_status gemm_launch(const GemmLaunch& g, cudaStream_t s, Profiler* prof);

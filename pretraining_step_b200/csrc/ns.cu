@@ -42,8 +42,9 @@ nc_status newton_schulz_wide(void* x0, int count, int m, int n, int steps, void*
     g.d.B = X; g.d.ldb = n; g.d.stride_b = mn; g.d.b_kmajor = 1;
     g.d.D = A; g.d.ldd = m; g.d.stride_d = mm;
     g.d.epi = NC_EPI_STORE_BF16; g.d.alpha = 1.f; g.d.split_k = 1;
+    g.symmetric = m > 128;  // the upper triangle of tiles, mirrored
     NC_TRY(gemm_launch(g, s, prof));
-    // B = c A A + b A
+    // B = c A A + b A (symmetric too)
     g.d = nc_gemm_desc{};
     g.d.M = m; g.d.N = m; g.d.K = m; g.d.batch = count;
     g.d.A = A; g.d.lda = m; g.d.stride_a = mm; g.d.a_kmajor = 1;
@@ -53,6 +54,7 @@ nc_status newton_schulz_wide(void* x0, int count, int m, int n, int steps, void*
     g.d.epi = NC_EPI_AXPBY_BF16; g.d.alpha = kNsC; g.d.beta = kNsB; g.d.split_k = 1;
     NC_TRY(gemm_launch(g, s, prof));
     // Y = B X + a X
+    g.symmetric = false;
     g.d = nc_gemm_desc{};
     g.d.M = m; g.d.N = n; g.d.K = m; g.d.batch = count;
     g.d.A = Bm; g.d.lda = m; g.d.stride_a = mm; g.d.a_kmajor = 1;

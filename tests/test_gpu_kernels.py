@@ -383,8 +383,13 @@ def test_attention_backward_full_length():
 
 
 # ------------------------------------------------------------------ Newton-Schulz
-@pytest.mark.parametrize("count,rows,cols", [(3, 256, 256), (2, 128, 512), (2, 512, 128)])
+@pytest.mark.parametrize("count,rows,cols", [(3, 256, 256), (2, 128, 512), (2, 512, 128),
+                                             (2, 640, 640), (1, 768, 1536)])
 def test_newton_schulz_op(count, rows, cols):
+    """Five Newton-Schulz steps against the oracle.  From 2 x 2 tiles of 256
+    up, the two symmetric products (X X^T and b A + c A A) compute only the
+    tiles on or above the diagonal and store the others transposed; 640
+    leaves ragged edge tiles on both sides."""
     t = torch()
     X = inputs.normal_stack(70 + rows, count, rows, cols)
     out = t.empty(count, rows, cols, dtype=t.bfloat16, device="cuda")
