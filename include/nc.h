@@ -253,6 +253,18 @@ int* nc_debug_op_status_word(void);
 nc_status nc_op_embed_gather(const int32_t* tokens, int64_t n, const float* E, int vocab, int d,
                              float* x, void* stream);
 
+/* The exponential that the attention backward evaluates on the FMA pipe for
+ * one pair of recomputed probabilities in four (the rest, and the forward,
+ * use the exponential unit):
+ * y[i] ~ 2^x[i] from range reduction x = n + f (n = rint(x)) and a degree-3
+ * minimax polynomial for 2^f on [-1/2, 1/2], relative error at most 7.5e-5,
+ * for x in [-125, 126); below -125 it returns about 2^-125 (the softmax
+ * zeroes masked scores itself).  The softmax is exp(s - max) of the guide's
+ * causal attention (section "1. Modelo GPT"); this entry runs the same
+ * device function over fp32 device arrays x, y of n elements so that its
+ * error can be measured.  NC_ERR_INVALID_ARG for n < 0 or null arrays. */
+nc_status nc_op_exp2_poly(const float* x, float* y, int64_t n, void* stream);
+
 /* Epilogues of the GEMM engine. */
 typedef enum {
   NC_EPI_STORE_BF16 = 0, /* D(bf16) = alpha*acc                               */

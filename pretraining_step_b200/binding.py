@@ -105,6 +105,7 @@ def lib():
         "nc_op_gemm": (ci, [ctypes.POINTER(GemmDesc), vp]),
         "nc_op_rmsnorm": (ci, [vp, i64, ci, vp, vp, vp]),
         "nc_op_embed_gather": (ci, [vp, i64, vp, ci, ci, vp, vp]),
+        "nc_op_exp2_poly": (ci, [vp, vp, i64, vp]),
         "nc_op_sync": (ci, [vp]),
         "nc_debug_op_status_word": (vp, []),
         "nc_op_attention_fwd": (ci, [vp, vp, vp, i64, vp, i64, vp, ci, ci, ci, vp]),
@@ -338,6 +339,12 @@ def embed_gather(tokens, n, E, vocab, d, x, stream=None):
     """x[i] = E[tokens[i]] (fp32 rows, bit for bit); ids out of range are
     clamped and reported by op_sync."""
     _check(lib().nc_op_embed_gather(_ptr(tokens), n, _ptr(E), vocab, d, _ptr(x), _stream(stream)))
+
+
+def exp2_poly(x, y, n, stream=None):
+    """y = 2^x (fp32 device arrays of n elements) by the FMA-pipe exponential
+    of the attention softmax."""
+    _check(lib().nc_op_exp2_poly(_ptr(x), _ptr(y), n, _stream(stream)))
 
 
 def op_sync(stream=None):

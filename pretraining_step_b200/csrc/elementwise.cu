@@ -8,6 +8,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "kernels.h"
+#include "exp2_poly.cuh"
 
 namespace nc {
 namespace {
@@ -559,6 +560,25 @@ nc_status ce_fwd_bwd(void* z, const int32_t* tgt, int64_t n, int V, float* loss_
 nc_status init_normal(float* out, int64_t n, uint64_t key, float stdv, cudaStream_t s) {
   const unsigned grid = (unsigned)std::min<int64_t>(blocks_for(n, 256), 148 * 16);
   init_normal_kernel<<<grid, 256, 0, s>>>(out, n, key, stdv);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+// 2^x through exp2_fma2, two elements per thread (the softmax's FMA-pipe
+// exponential, run on a plain array so that its error can be measured).
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+  const int64_t i = 2 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    const float2 r = exp2_fma2(make_float2(x[i], x[i + 1]));
+    y[i] = r.x;
+    y[i + 1] = r.y;
+  } else if (i < n) {
+    y[i] = exp2_fma2(make_float2(x[i], 0.f)).x;
+  }
+}
+
+nc_status exp2_poly(const float* x, float* y, int64_t n, cudaStream_t s) {
+  exp2_poly_kernel<<<blocks_for((n + 1) / 2, 256), 256, 0, s>>>(x, y, n);
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }

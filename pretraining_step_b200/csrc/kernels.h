@@ -109,6 +109,8 @@ nc_status ce_fwd_bwd(void* z, const int32_t* tgt, int64_t n, int V, float* loss_
                      float* loss_out, int* status, cudaStream_t s, Profiler* prof);
 nc_status init_normal(float* out, int64_t n, uint64_t key, float stdv, cudaStream_t s);
 nc_status f32_to_bf16(const float* in, void* out, int64_t n, cudaStream_t s, Profiler* prof);
+// y[i] = 2^x[i] by exp2_fma2 (exp2_poly.cuh), the softmax's FMA-pipe exponential.
+nc_status exp2_poly(const float* x, float* y, int64_t n, cudaStream_t s);
 // Momentum and per-matrix squared norms over the 6*L block matrices; dkv is
 // the width of wk and wv (d with one KV head per query head).
 nc_status muon_momentum(float* M, const float* G, int L, int d, int dkv, float mu, float* sumsq,

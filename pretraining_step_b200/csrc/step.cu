@@ -975,6 +975,12 @@ nc_status nc_op_embed_gather(const int32_t* tokens, int64_t n, const float* E, i
   return embed_gather(tokens, n, E, vocab, d, x, st, static_cast<cudaStream_t>(stream), nullptr);
 }
 
+nc_status nc_op_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y))) return fail(NC_ERR_INVALID_ARG, "exp2_poly: bad arguments");
+  if (n == 0) return NC_OK;
+  return exp2_poly(x, y, n, static_cast<cudaStream_t>(stream));
+}
+
 nc_status nc_op_sync(void* stream) {
   int* word = nullptr;
   NC_TRY(op_status_word(&word));

@@ -220,6 +220,33 @@ def test_embed_gather_out_of_range_ids_are_clamped_and_reported():
     assert np.array_equal(x.cpu().numpy(), expect)
 
 
+def test_exp2_poly_relative_error():
+    """The softmax's FMA-pipe exponential on the GPU against exact 2^x (fp64):
+    relative error within the polynomial's 7.5e-5 plus fp32 rounding over
+    the softmax's range, integers exact up to the polynomial's value at 0,
+    and arguments below -125 (masked scores: -inf) held near 2^-125."""
+    t = torch()
+    rng = np.random.default_rng(11)
+    x = np.concatenate([np.linspace(-125.0, 20.0, 1 << 20), rng.uniform(-30.0, 1.0, 99_999),
+                        np.arange(-125, 21, dtype=np.float64)]).astype(np.float32)
+    dx = dev_f32(x)
+    y = t.empty_like(dx)
+    nc.exp2_poly(dx, y, x.size)  # odd length: the last thread takes one element
+    t.cuda.synchronize()
+    got = host(y).astype(np.float64)
+    ref = np.exp2(x.astype(np.float64))
+    assert np.max(np.abs(got / ref - 1.0)) < 7.5e-5 + 2e-7
+    special = np.array([-np.inf, -1e30, -126.0, -200.0], dtype=np.float32)
+    ds = dev_f32(special)
+    ys = t.empty_like(ds)
+    nc.exp2_poly(ds, ys, special.size)
+    t.cuda.synchronize()
+    v = host(ys)
+    assert np.all(np.isfinite(v)) and np.all(v > 0) and np.all(v < 2.0 ** -124)
+    with pytest.raises(nc.NcError):
+        nc.exp2_poly(ds, ys, -1)
+
+
 def test_planted_op_status_is_reported_once():
     """An expired bounded wait inside an op (planted here as its status code,
     not produced by a stuck kernel) surfaces as NC_ERR_TIMEOUT at the next
