@@ -644,6 +644,26 @@ def run_op(args):
         flops = 2.0 * M * N * K
         nbytes = 2.0 * (M * K + N * K) + M * N * (4 if f32_out else 2) + \
             (0 if aux is None else aux.numel() * aux.element_size())
+        if args.fp8:
+            # E4M3 operands (both K-major), quantised once before timing.
+            assert ak and bk and K % 16 == 0, "--fp8 needs K-major operands and K a multiple of 16"
+            qa = torch.empty(M * K, device="cuda", dtype=torch.uint8)
+            qb = torch.empty(N * K, device="cuda", dtype=torch.uint8)
+            sc = torch.zeros(2, device="cuda", dtype=torch.float32)
+            scratch = torch.zeros(2, device="cuda", dtype=torch.int32)
+            quant = lambda: nc.fp8_quantize(A, M, K, qa, sc[0:1], scratch[0:1])
+            quant()
+            nc.fp8_quantize(Bm, N, K, qb, sc[1:2], scratch[1:2])
+            torch.cuda.synchronize()
+            ev[0].record()
+            for _ in range(3):
+                quant()
+            ev[1].record()
+            torch.cuda.synchronize()
+            quant_ms = ev[0].elapsed_time(ev[1]) / 3
+            run = lambda: nc.gemm(M, N, K, qa, qb, D, epi=epi, aux=aux,
+                                  split_k=0 if epi == nc.EPI_ACC_F32 else 1, ab_scale=sc)
+            nbytes -= 1.0 * (M * K + N * K)
     else:
         Bb, T_, H = dims
         d = H * 128
@@ -675,9 +695,15 @@ def run_op(args):
     torch.cuda.synchronize()
     ms = ev[0].elapsed_time(ev[1]) / args.steps
     tf = flops / (ms / 1e3) / 1e12
-    print(json.dumps({"op": args.op, "shape": dims, "ms_per_launch": ms, "tflops": tf,
-                      "frac_of_burst_peak": tf / peaks["bf16_tflops"],
-                      "peak_source": peak_kind, "algorithmic_bytes": nbytes}), flush=True)
+    line = {"op": args.op, "shape": dims, "ms_per_launch": ms, "tflops": tf,
+            "frac_of_burst_peak": tf / peaks["bf16_tflops"],
+            "peak_source": peak_kind, "algorithmic_bytes": nbytes}
+    if args.op == "gemm" and args.fp8:
+        # fp8 peak: the measured bf16 burst peak times the nominal fp8 : bf16 ratio (2).
+        line.update({"dtype": "e4m3", "frac_of_burst_peak": tf / (2.0 * peaks["bf16_tflops"]),
+                     "peak_note": "measured bf16 burst x 2 (nominal dense fp8 : bf16 ratio)",
+                     "quantize_a_ms": quant_ms})
+    print(json.dumps(line), flush=True)
     return 0
 
 
@@ -881,6 +907,8 @@ def main():
     ap.add_argument("--vocab", type=int, default=V,
                     help="--op step: vocabulary (smaller only for kernel captures on a small case)")
     ap.add_argument("--shape", default="16384,5120,1280")
+    ap.add_argument("--fp8", action="store_true",
+                    help="--op gemm: E4M3 operands (quantised before timing) with per-tensor scales")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

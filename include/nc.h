@@ -265,6 +265,20 @@ nc_status nc_op_embed_gather(const int32_t* tokens, int64_t n, const float* E, i
  * error can be measured.  NC_ERR_INVALID_ARG for n < 0 or null arrays. */
 nc_status nc_op_exp2_poly(const float* x, float* y, int64_t n, void* stream);
 
+/* E4M3 quantisation of one GEMM operand (the guide's "--fp8" training,
+ * section "1. Modelo GPT", with one dynamic scale per tensor): for x, a
+ * rows x cols matrix of bf16 (x_bf16 != 0) or fp32, row stride ldx,
+ *   s = 448 / max |x|  (fp32; 1 when x is all zero; NaN elements skipped),
+ *   q[r*ldq + c] = E4M3(x[r, c] * s), or q[c*ldq + r] when transpose != 0,
+ * E4M3 the OCP 8-bit format (bias 7, largest 448, subnormals down to 2^-9)
+ * rounded to nearest even and saturated to +-448.  s goes to *scale (device
+ * float), for nc_gemm_desc.ab_scale.  cols and ldx multiples of 8, rows too
+ * when transposing, ldq a multiple of 16 and at least the output row
+ * length; x and q 16-byte aligned; scratch is one device word the call
+ * overwrites.  NC_ERR_INVALID_ARG otherwise. */
+nc_status nc_op_fp8_quantize(const void* x, int x_bf16, int64_t rows, int cols, int64_t ldx, int transpose,
+                             void* q, int64_t ldq, float* scale, void* scratch, void* stream);
+
 /* Epilogues of the GEMM engine. */
 typedef enum {
   NC_EPI_STORE_BF16 = 0, /* D(bf16) = alpha*acc                               */
@@ -318,6 +332,16 @@ typedef struct {
   /* KV heads of the fused projection, 1 <= rope_Hkv <= rope_H; 0 means
    * rope_H (one KV head per query head). */
   int rope_Hkv;
+  /* Operand type: 0 bf16; 1 OCP E4M3 (one byte per element, the guide's
+   * "--fp8" training, section "1. Modelo GPT", here with one dynamic scale
+   * per operand tensor).  E4M3 needs both operands K-major, lda, ldb and
+   * the batch strides multiples of 16, alpha = 1, M > 128, 256-wide column
+   * tiles (N > 128 with no more edge waste than 128-wide ones) and any
+   * epilogue but NC_EPI_AXPBY_BF16; the product is multiplied by
+   * 1 / (ab_scale[0] * ab_scale[1]), the scales nc_op_fp8_quantize wrote
+   * for A and B (two device floats). */
+  int ab_type;
+  const float* ab_scale;
 } nc_gemm_desc;
 nc_status nc_op_gemm(const nc_gemm_desc* desc, void* stream);
 

@@ -46,7 +46,8 @@ class GemmDesc(ctypes.Structure):
                 ("epi", ctypes.c_int), ("alpha", ctypes.c_float), ("beta", ctypes.c_float),
                 ("split_k", ctypes.c_int), ("rope_T", ctypes.c_int), ("rope_H", ctypes.c_int),
                 ("rope_tab", ctypes.c_void_p), ("rstd_q", ctypes.c_void_p),
-                ("rstd_k", ctypes.c_void_p), ("rope_Hkv", ctypes.c_int)]
+                ("rstd_k", ctypes.c_void_p), ("rope_Hkv", ctypes.c_int),
+                ("ab_type", ctypes.c_int), ("ab_scale", ctypes.c_void_p)]
 
 
 class ModelConfig(ctypes.Structure):
@@ -106,6 +107,7 @@ def lib():
         "nc_op_rmsnorm": (ci, [vp, i64, ci, vp, vp, vp]),
         "nc_op_embed_gather": (ci, [vp, i64, vp, ci, ci, vp, vp]),
         "nc_op_exp2_poly": (ci, [vp, vp, i64, vp]),
+        "nc_op_fp8_quantize": (ci, [vp, ci, i64, ci, i64, ci, vp, i64, vp, vp, vp]),
         "nc_op_sync": (ci, [vp]),
         "nc_debug_op_status_word": (vp, []),
         "nc_op_attention_fwd": (ci, [vp, vp, vp, i64, vp, i64, vp, ci, ci, ci, vp]),
@@ -320,7 +322,9 @@ class GPT:
 # ------------------------------------------------------------------ ops
 def gemm(M, N, K, A, B, D, *, lda=None, ldb=None, ldd=None, a_kmajor=True, b_kmajor=True,
          batch=1, stride_a=0, stride_b=0, stride_d=0, epi=EPI_STORE_BF16, aux=None, ldaux=0,
-         stride_aux=0, alpha=1.0, beta=0.0, split_k=1, stream=None):
+         stride_aux=0, alpha=1.0, beta=0.0, split_k=1, ab_scale=None, stream=None):
+    """D = epi(A B^T) on the tensor cores; ab_scale (a device array of the
+    two operands' fp8 scales) selects E4M3 operands (one byte each)."""
     d = GemmDesc()
     d.M, d.N, d.K, d.batch = M, N, K, batch
     d.A, d.B, d.D, d.aux = _ptr(A), _ptr(B), _ptr(D), _ptr(aux)
@@ -332,6 +336,8 @@ def gemm(M, N, K, A, B, D, *, lda=None, ldb=None, ldd=None, a_kmajor=True, b_kma
     d.ldaux = ldaux if ldaux else d.ldd
     d.stride_aux = stride_aux
     d.epi, d.alpha, d.beta, d.split_k = epi, alpha, beta, split_k
+    if ab_scale is not None:
+        d.ab_type, d.ab_scale = 1, _ptr(ab_scale)
     _check(lib().nc_op_gemm(ctypes.byref(d), _stream(stream)))
 
 
@@ -339,6 +345,17 @@ def embed_gather(tokens, n, E, vocab, d, x, stream=None):
     """x[i] = E[tokens[i]] (fp32 rows, bit for bit); ids out of range are
     clamped and reported by op_sync."""
     _check(lib().nc_op_embed_gather(_ptr(tokens), n, _ptr(E), vocab, d, _ptr(x), _stream(stream)))
+
+
+def fp8_quantize(x, rows, cols, q, scale, scratch, *, ldx=None, ldq=None, transpose=False, stream=None):
+    """q = E4M3(x * s), s = 448 / amax(|x|) written to scale[0] (x bf16 or
+    fp32 on the device; q uint8, transposed if asked)."""
+    import torch as _t
+    bf16 = x.dtype == _t.bfloat16
+    ldx = ldx if ldx is not None else cols
+    ldq = ldq if ldq is not None else (rows if transpose else cols)
+    _check(lib().nc_op_fp8_quantize(_ptr(x), int(bf16), rows, cols, ldx, int(bool(transpose)), _ptr(q),
+                                    ldq, _ptr(scale), _ptr(scratch), _stream(stream)))
 
 
 def exp2_poly(x, y, n, stream=None):

@@ -10,6 +10,8 @@
 #include "kernels.h"
 #include "exp2_poly.cuh"
 
+#include <cuda_fp8.h>
+
 namespace nc {
 namespace {
 
@@ -579,6 +581,155 @@ __global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict_
 
 nc_status exp2_poly(const float* x, float* y, int64_t n, cudaStream_t s) {
   exp2_poly_kernel<<<blocks_for((n + 1) / 2, 256), 256, 0, s>>>(x, y, n);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+// ------------------------------------------------------------------ fp8 (E4M3)
+// One dynamic scale per tensor: s = 448 / amax(|x|) (1 when x is all zero),
+// q = E4M3(x * s) rounded to nearest even and saturated to +-448.  x is a
+// rows x cols matrix of bf16 (activations, gradients) or fp32 (weights) with
+// row stride ld; cols a multiple of 8.
+
+__device__ __forceinline__ float fp8_src(const void* x, bool bf16, int64_t i) {
+  return bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(x)[i]) : static_cast<const float*>(x)[i];
+}
+
+// Eight consecutive elements of one row as floats (16- or 32-byte loads).
+__device__ __forceinline__ void fp8_load8(const void* x, bool bf16, int64_t i, float (&v)[8]) {
+  if (bf16) {
+    const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + i);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = unpack_bf16x2(w[j]);
+      v[2 * j] = f.x;
+      v[2 * j + 1] = f.y;
+    }
+  } else {
+    const float4 a = *reinterpret_cast<const float4*>(static_cast<const float*>(x) + i);
+    const float4 b = *reinterpret_cast<const float4*>(static_cast<const float*>(x) + i + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+}
+
+// amax over the matrix into *amax_bits (the bits of a non-negative float, so
+// integer max orders them; zeroed by the caller).  NaN elements are skipped,
+// as fmaxf does.
+__global__ void __launch_bounds__(256) fp8_amax_kernel(const void* __restrict__ x, int bf16, int64_t rows,
+                                                       int cols, int64_t ld, unsigned* amax_bits) {
+  const int cv = cols / 8;
+  const int64_t total = rows * cv;
+  float m = 0.f;
+  for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < total; u += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = u / cv;
+    float v[8];
+    fp8_load8(x, bf16 != 0, r * ld + (u - r * cv) * 8, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
+  }
+  m = warp_max(m);
+  __shared__ float red[8];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int i = 1; i < 8; ++i) m = fmaxf(m, red[i]);
+    atomicMax(amax_bits, __float_as_uint(m));
+  }
+}
+
+__device__ __forceinline__ float fp8_scale_of(const unsigned* amax_bits) {
+  const float amax = __uint_as_float(*amax_bits);
+  return amax > 0.f ? 448.f / amax : 1.f;
+}
+
+// Two floats to two E4M3 bytes (the first in the low byte).
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+  return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+}
+
+// q[r * ldq + c] = E4M3(x[r, c] * s), eight elements per thread.
+__global__ void __launch_bounds__(256) fp8_quant_kernel(const void* __restrict__ x, int bf16, int64_t rows,
+                                                        int cols, int64_t ld, const unsigned* amax_bits,
+                                                        uint8_t* __restrict__ q, int64_t ldq, float* scale) {
+  const float s = fp8_scale_of(amax_bits);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && scale) *scale = s;
+  const int cv = cols / 8;
+  const int64_t total = rows * cv;
+  for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < total; u += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = u / cv;
+    const int64_t c = (u - r * cv) * 8;
+    float v[8];
+    fp8_load8(x, bf16 != 0, r * ld + c, v);
+    uint2 o;
+    o.x = e4m3x2(v[0] * s, v[1] * s) | (e4m3x2(v[2] * s, v[3] * s) << 16);
+    o.y = e4m3x2(v[4] * s, v[5] * s) | (e4m3x2(v[6] * s, v[7] * s) << 16);
+    *reinterpret_cast<uint2*>(q + r * ldq + c) = o;
+  }
+}
+
+// The transpose: q[c * ldq + r] = E4M3(x[r, c] * s), through 64 x 64 tiles in
+// shared memory (rows a multiple of 8 as well).
+__global__ void __launch_bounds__(256) fp8_quant_t_kernel(const void* __restrict__ x, int bf16, int64_t rows,
+                                                          int cols, int64_t ld, const unsigned* amax_bits,
+                                                          uint8_t* __restrict__ q, int64_t ldq, float* scale) {
+  __shared__ uint8_t tile[64][64 + 8];
+  const float s = fp8_scale_of(amax_bits);
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && scale) *scale = s;
+  const int64_t r0 = (int64_t)blockIdx.y * 64;
+  const int c0 = blockIdx.x * 64;
+  // Load: 64 rows x 8 groups of 8 columns, one group per thread per pass.
+  for (int u = threadIdx.x; u < 64 * 8; u += blockDim.x) {
+    const int rr = u >> 3, cg = (u & 7) * 8;
+    const int64_t r = r0 + rr;
+    const int c = c0 + cg;
+    float v[8];
+    if (r < rows && c < cols) {
+      fp8_load8(x, bf16 != 0, r * ld + c, v);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; j += 2) {
+      const uint32_t b = e4m3x2(v[j] * s, v[j + 1] * s);
+      tile[cg + j][rr] = (uint8_t)(b & 0xffu);
+      tile[cg + j + 1][rr] = (uint8_t)(b >> 8);
+    }
+  }
+  __syncthreads();
+  // Store: 64 output rows (columns of x) x 8 groups of 8 bytes.
+  for (int u = threadIdx.x; u < 64 * 8; u += blockDim.x) {
+    const int cc = u >> 3, rg = (u & 7) * 8;
+    const int c = c0 + cc;
+    const int64_t r = r0 + rg;
+    if (c < cols && r < rows) {
+      uint2 o;
+      o.x = (uint32_t)tile[cc][rg] | ((uint32_t)tile[cc][rg + 1] << 8) | ((uint32_t)tile[cc][rg + 2] << 16) |
+            ((uint32_t)tile[cc][rg + 3] << 24);
+      o.y = (uint32_t)tile[cc][rg + 4] | ((uint32_t)tile[cc][rg + 5] << 8) | ((uint32_t)tile[cc][rg + 6] << 16) |
+            ((uint32_t)tile[cc][rg + 7] << 24);
+      *reinterpret_cast<uint2*>(q + (int64_t)c * ldq + r) = o;
+    }
+  }
+}
+
+nc_status fp8_quantize(const void* x, bool bf16, int64_t rows, int cols, int64_t ld, bool transpose,
+                       uint8_t* q, int64_t ldq, float* scale, unsigned* amax_scratch, cudaStream_t s,
+                       Profiler* prof) {
+  Probe probe(prof, s, "fp8_quantize", 0.0, (double)rows * cols * (2.0 * (bf16 ? 2 : 4) + 1.0));
+  NC_CUDA_TRY(cudaMemsetAsync(amax_scratch, 0, sizeof(unsigned), s));
+  const int64_t units = rows * (cols / 8);
+  const unsigned g = (unsigned)std::min<int64_t>((units + 255) / 256, 8LL * num_sms());
+  fp8_amax_kernel<<<g, 256, 0, s>>>(x, bf16 ? 1 : 0, rows, cols, ld, amax_scratch);
+  NC_CUDA_TRY(cudaGetLastError());
+  if (transpose) {
+    dim3 grid((unsigned)((cols + 63) / 64), (unsigned)((rows + 63) / 64));
+    fp8_quant_t_kernel<<<grid, 256, 0, s>>>(x, bf16 ? 1 : 0, rows, cols, ld, amax_scratch, q, ldq, scale);
+  } else {
+    fp8_quant_kernel<<<g, 256, 0, s>>>(x, bf16 ? 1 : 0, rows, cols, ld, amax_scratch, q, ldq, scale);
+  }
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }

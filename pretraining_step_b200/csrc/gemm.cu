@@ -48,9 +48,18 @@ struct Cfg {
 struct Args {
   int M, N, K, batch;
   int tiles_m, tiles_n, split_k, kb_per_split, num_kb;
-  int a_mn, b_mn;
+  int16_t a_mn, b_mn;
+  int16_t fp8;  // E4M3 operands (pair kernel, K-major): 128-element K slices
+  int16_t unused_;
   int epi;
-  float alpha, beta;
+  union {
+    struct {
+      float alpha, beta;
+    };
+    // fp8: the two operands' quantisation scales (device); the epilogue's
+    // alpha becomes 1 / (ab_scale[0] * ab_scale[1]).
+    const float* ab_scale;
+  };
   void* D;
   int64_t ldd;
   // The RoPE/QK-norm epilogue (batch 1, no aux operand) keeps its parameters
@@ -739,7 +748,8 @@ __device__ __forceinline__ bool epi_staged(int epi) {
   return epi == NC_EPI_STORE_BF16 || epi == NC_EPI_RELU2 || epi == NC_EPI_STORE_F32;
 }
 
-template <bool ROPE, bool XR>
+// FP8: E4M3 operands (a stage holds 128 bytes of K per row: 128 elements).
+template <bool ROPE, bool XR, bool FP8>
 __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUtensorMap* tmB,
                                               const CUtensorMap* tmX, const Args& p) {
   using C = std::conditional_t<XR, Cfg2X, Cfg2>;
@@ -811,7 +821,7 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
           if (leader) tc::mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
           uint8_t* a_dst = smem + stage * C::STAGE_BYTES;
           uint8_t* b_dst = a_dst + C::A_BYTES;
-          const int k0 = kb * BK;
+          const int k0 = kb * (FP8 ? 2 * BK : BK);
           if (!p.a_mn) {
             tc::tma_load_3d_pair(a_dst, tmA, &full[stage], k0, m0, c.b);
           } else {
@@ -844,7 +854,7 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
     }
   } else if (warp == 1) {
     if (lane == 0 && leader) {
-      const uint32_t idesc = tc::idesc_bf16_f32(2 * BM, BN, p.a_mn, p.b_mn);
+      const uint32_t idesc = FP8 ? tc::idesc_e4m3_f32(2 * BM, BN) : tc::idesc_bf16_f32(2 * BM, BN, p.a_mn, p.b_mn);
       const uint32_t s0 = tc::smem_u32(smem);
       const uint64_t adesc0 = p.a_mn ? tc::smem_desc_sw128(s0, 8192, 1024) : tc::smem_desc_sw128(s0, 16, 1024);
       const uint64_t bdesc0 = p.b_mn ? tc::smem_desc_sw128(s0 + C::A_BYTES, 8192, 1024)
@@ -871,10 +881,18 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
           tc::tc_fence_after();
           const uint64_t ad = adesc0 + (uint64_t)((stage * C::STAGE_BYTES) >> 4);
           const uint64_t bd = bdesc0 + (uint64_t)((stage * C::STAGE_BYTES) >> 4);
+          // Four MMAs per stage: K = 16 bf16 or K = 32 E4M3 elements, 32 bytes each.
+          if constexpr (FP8) {
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            tc::umma_bf16_ss_pair(d_tmem, tc::desc_add(ad, kk * a_step), tc::desc_add(bd, kk * b_step),
+            for (int kk = 0; kk < BK / 16; ++kk)
+              tc::umma_f8_ss_pair(d_tmem, tc::desc_add(ad, kk * a_step), tc::desc_add(bd, kk * b_step),
                                   idesc, (kb > c.kb0 || kk > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              tc::umma_bf16_ss_pair(d_tmem, tc::desc_add(ad, kk * a_step), tc::desc_add(bd, kk * b_step),
+                                    idesc, (kb > c.kb0 || kk > 0) ? 1u : 0u);
+          }
           tc::umma_commit_pair(&empty[stage]);
           if (++stage == C::STAGES) {
             stage = 0;
@@ -890,6 +908,9 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
       drain_wait(drained, 0);
     }
   } else {
+    // The epilogue, on the kernel's arguments or (FP8) on a copy whose alpha
+    // is the product of the operands' dequantisation factors.
+    auto epilogue = [&](const Args& pe) {
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     constexpr int CH = BN / 32 / 2;
@@ -899,7 +920,7 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
     uint32_t acc_phase = 0;
     // XR: this warp's aux ring; chunk g (counted over this warp's tiles)
     // lives in slot g % slots.  Chunks [g_use, g_use + slots) are in flight.
-    const bool xf32 = p.epi == NC_EPI_RESID_F32;
+    const bool xf32 = pe.epi == NC_EPI_RESID_F32;
     const int slot_bytes = xf32 ? 4096 : 2048;
     const int slots = XR ? Cfg2X::X_WARP_BYTES / slot_bytes : 1;
     const int slot_shift = slots == 4 ? 2 : 1;
@@ -909,20 +930,20 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
     if constexpr (XR) {
       if (lane == 0)
         for (int g = 0; g < slots; ++g)
-          aux_issue<BN, CH>(p, tmX, ring, xfull, slot_bytes, slots, g, pair, npairs, total, (int)rank, q,
+          aux_issue<BN, CH>(pe, tmX, ring, xfull, slot_bytes, slots, g, pair, npairs, total, (int)rank, q,
                             half);
     }
     bool xabort = false;
     for (int t = pair; t < total; t += npairs) {
-      const TileCoord c = decode(p, t);
-      bool ok = tc::mbar_wait(&tfull[acc], acc_phase, abort_flag, p.status);
+      const TileCoord c = decode(pe, t);
+      bool ok = tc::mbar_wait(&tfull[acc], acc_phase, abort_flag, pe.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc::tc_fence_after();
       const int row = c.mb * 2 * BM + (int)rank * BM + row_in_tile;
-      const bool aux = epi_has_aux(p.epi);
-      const bool mirror = p.tiles_m < 0 && c.mb != c.nb;  // symmetric output, off the diagonal
+      const bool aux = epi_has_aux(pe.epi);
+      const bool mirror = pe.tiles_m < 0 && c.mb != c.nb;  // symmetric output, off the diagonal
       if constexpr (ROPE) {  // separate instantiation: the other GEMMs carry no RoPE code
-        rope_head_epilogue(p, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + half * CH * 32, c.b,
+        rope_head_epilogue(pe, tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + half * CH * 32, c.b,
                            row, c.nb * BN + half * CH * 32, ring, lane);
       } else if constexpr (XR) {
 #pragma unroll
@@ -932,27 +953,27 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
           tc::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + ch * 32, r);
           const int col0 = c.nb * BN + ch * 32;
           const int slot = g_use & (slots - 1);
-          const bool got = tc::mbar_wait(&xfull[slot], (g_use >> slot_shift) & 1, abort_flag, p.status);
+          const bool got = tc::mbar_wait(&xfull[slot], (g_use >> slot_shift) & 1, abort_flag, pe.status);
           tc::tmem_ld_wait();
           if (!__all_sync(0xffffffffu, got)) {
             xabort = true;
             break;
           }
-          if (col0 < p.N)
-            aux_epilogue_chunk(p, ring + slot * slot_bytes, lane, xf32, c.b, row - lane, col0, r, mirror);
+          if (col0 < pe.N)
+            aux_epilogue_chunk(pe, ring + slot * slot_bytes, lane, xf32, c.b, row - lane, col0, r, mirror);
           // Every lane is done with the slot: order its accesses before the
           // TMA refill of the same slot with the chunk `slots` ahead.
           tc::fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            aux_issue<BN, CH>(p, tmX, ring, xfull, slot_bytes, slots, g_use + slots, pair, npairs, total,
+            aux_issue<BN, CH>(pe, tmX, ring, xfull, slot_bytes, slots, g_use + slots, pair, npairs, total,
                               (int)rank, q, half);
           }
           ++g_use;
         }
         if (xabort) break;
-      } else if (epi_staged(p.epi)) {
-        const bool f32 = p.epi == NC_EPI_STORE_F32;
+      } else if (epi_staged(pe.epi)) {
+        const bool f32 = pe.epi == NC_EPI_STORE_F32;
 #pragma unroll
         for (int k = 0; k < CH; ++k) {
           const int ch = half * CH + k;
@@ -960,14 +981,14 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
           tc::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + ch * 32, r);
           const int col0 = c.nb * BN + ch * 32;
           tc::tmem_ld_wait();
-          if (col0 < p.N) {
+          if (col0 < pe.N) {
             float w[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-              const float a = __uint_as_float(r[j]) * p.alpha;
-              w[j] = p.epi == NC_EPI_RELU2 ? fmaxf(a, 0.f) * fmaxf(a, 0.f) : a;
+              const float a = __uint_as_float(r[j]) * pe.alpha;
+              w[j] = pe.epi == NC_EPI_RELU2 ? fmaxf(a, 0.f) * fmaxf(a, 0.f) : a;
             }
-            stage_store_chunk(p, ring, lane, f32, c.b, row - lane, col0, w, mirror);
+            stage_store_chunk(pe, ring, lane, f32, c.b, row - lane, col0, w, mirror);
           }
         }
       } else {
@@ -976,7 +997,7 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
       for (int j = 0; j < 32; ++j) xa[j] = xb[j] = 0.f;
       {
         const int col0 = c.nb * BN + half * CH * 32;
-        if (aux && row < p.M && col0 < p.N) load_aux(p, c.b, row, col0, xa);
+        if (aux && row < pe.M && col0 < pe.N) load_aux(pe, c.b, row, col0, xa);
       }
 #pragma unroll
       for (int k = 0; k < CH; ++k) {
@@ -986,13 +1007,13 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
         const int col0 = c.nb * BN + ch * 32;
         float(&cur)[32] = (k & 1) ? xb : xa;
         float(&nxt)[32] = (k & 1) ? xa : xb;
-        if (aux && k + 1 < CH && row < p.M && col0 + 32 < p.N) load_aux(p, c.b, row, col0 + 32, nxt);
+        if (aux && k + 1 < CH && row < pe.M && col0 + 32 < pe.N) load_aux(pe, c.b, row, col0 + 32, nxt);
         tc::tmem_ld_wait();
-        if (row < p.M && col0 < p.N) {
+        if (row < pe.M && col0 < pe.N) {
           float v[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          store_row_chunk(p, c.b, row, col0, v, cur);
+          store_row_chunk(pe, c.b, row, col0, v, cur);
         }
       }
       }
@@ -1008,6 +1029,14 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
       for (int g = g_use; g < g_use + slots; ++g)
         if (pair + (g / CH) * npairs < total) drain_wait(&xfull[g & (slots - 1)], (g >> slot_shift) & 1);
     }
+      };
+    if constexpr (FP8) {
+      Args pe = p;
+      pe.alpha = 1.f / (p.ab_scale[0] * p.ab_scale[1]);
+      epilogue(pe);
+    } else {
+      epilogue(p);
+    }
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -1019,17 +1048,18 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
 }
 
 
-template <bool ROPE>
+template <bool ROPE, bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const Args p) {
-  gemm_tc2_body<ROPE, false>(&tmA, &tmB, nullptr, p);
+  gemm_tc2_body<ROPE, false, FP8>(&tmA, &tmB, nullptr, p);
 }
 
+template <bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc2_aux_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmX, const Args p) {
-  gemm_tc2_body<false, true>(&tmA, &tmB, &tmX, p);
+  gemm_tc2_body<false, true, FP8>(&tmA, &tmB, &tmX, p);
 }
 
 // ------------------------------------------------------------------ host
@@ -1062,6 +1092,8 @@ nc_status launch_bn(const nc_gemm_desc& d, int split, int* status, const char* t
   a.split_k = (a.num_kb + a.kb_per_split - 1) / a.kb_per_split;
   a.a_mn = d.a_kmajor ? 0 : 1;
   a.b_mn = d.b_kmajor ? 0 : 1;
+  a.fp8 = 0;
+  a.unused_ = 0;
   a.epi = d.epi;
   a.alpha = d.alpha;
   a.beta = d.beta;
@@ -1096,12 +1128,17 @@ nc_status launch_pair(const nc_gemm_desc& d, int split, int* status, const char*
   using C = std::conditional_t<XR, Cfg2X, Cfg2>;
   static DeviceOnce smem_attr;
   NC_TRY(once_per_device(smem_attr, []() -> nc_status {
-    if constexpr (XR)
-      NC_CUDA_TRY(cudaFuncSetAttribute(gemm_tc2_aux_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if constexpr (XR) {
+      NC_CUDA_TRY(cudaFuncSetAttribute(gemm_tc2_aux_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM_BYTES));
-    else
-      NC_CUDA_TRY(cudaFuncSetAttribute(gemm_tc2_kernel<ROPE>,
+      NC_CUDA_TRY(cudaFuncSetAttribute(gemm_tc2_aux_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::SMEM_BYTES));
+    } else {
+      NC_CUDA_TRY(cudaFuncSetAttribute(gemm_tc2_kernel<ROPE, false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+      NC_CUDA_TRY(cudaFuncSetAttribute(gemm_tc2_kernel<ROPE, true>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+    }
     return NC_OK;
   }));
   CUtensorMap ta, tb, tx;
@@ -1111,11 +1148,19 @@ nc_status launch_pair(const nc_gemm_desc& d, int split, int* status, const char*
     if (!make_tmap_3d(&tx, d.aux, f32, d.N, d.M, d.batch, d.ldaux, d.stride_aux, 32, 32, f32 ? 128 : 64))
       return fail(NC_ERR_INVALID_ARG, "gemm: cuTensorMapEncodeTiled rejected the aux operand");
   }
-  const bool ok_a = d.a_kmajor ? make_tmap_bf16_3d(&ta, d.A, d.K, d.M, d.batch, d.lda, d.stride_a, BM)
-                               : make_tmap_bf16_3d(&ta, d.A, d.M, d.K, d.batch, d.lda, d.stride_a, 64);
-  const bool ok_b = d.b_kmajor ? make_tmap_bf16_3d(&tb, d.B, d.K, d.N, d.batch, d.ldb, d.stride_b, C::BN / 2)
-                               : make_tmap_bf16_3d(&tb, d.B, d.N, d.K, d.batch, d.ldb, d.stride_b, 64);
+  const bool fp8 = d.ab_type == 1;  // E4M3, both operands K-major (checked by the caller)
+  bool ok_a, ok_b;
+  if (fp8) {
+    ok_a = make_tmap_u8_3d(&ta, d.A, d.K, d.M, d.batch, d.lda, d.stride_a, BM);
+    ok_b = make_tmap_u8_3d(&tb, d.B, d.K, d.N, d.batch, d.ldb, d.stride_b, C::BN / 2);
+  } else {
+    ok_a = d.a_kmajor ? make_tmap_bf16_3d(&ta, d.A, d.K, d.M, d.batch, d.lda, d.stride_a, BM)
+                      : make_tmap_bf16_3d(&ta, d.A, d.M, d.K, d.batch, d.lda, d.stride_a, 64);
+    ok_b = d.b_kmajor ? make_tmap_bf16_3d(&tb, d.B, d.K, d.N, d.batch, d.ldb, d.stride_b, C::BN / 2)
+                      : make_tmap_bf16_3d(&tb, d.B, d.N, d.K, d.batch, d.ldb, d.stride_b, 64);
+  }
   if (!ok_a || !ok_b) return fail(NC_ERR_INVALID_ARG, "gemm: cuTensorMapEncodeTiled rejected an operand");
+  const int bk = fp8 ? 2 * BK : BK;  // K elements per 128-byte stage row
   Args a;
   a.M = d.M;
   a.N = d.N;
@@ -1123,14 +1168,20 @@ nc_status launch_pair(const nc_gemm_desc& d, int split, int* status, const char*
   a.batch = d.batch;
   a.tiles_m = (d.M + 2 * BM - 1) / (2 * BM);
   a.tiles_n = (d.N + C::BN - 1) / C::BN;
-  a.num_kb = (d.K + BK - 1) / BK;
+  a.num_kb = (d.K + bk - 1) / bk;
   a.kb_per_split = (a.num_kb + split - 1) / split;
   a.split_k = (a.num_kb + a.kb_per_split - 1) / a.kb_per_split;
   a.a_mn = d.a_kmajor ? 0 : 1;
   a.b_mn = d.b_kmajor ? 0 : 1;
+  a.fp8 = fp8 ? 1 : 0;
+  a.unused_ = 0;
   a.epi = d.epi;
-  a.alpha = d.alpha;
-  a.beta = d.beta;
+  if (fp8) {
+    a.ab_scale = d.ab_scale;
+  } else {
+    a.alpha = d.alpha;
+    a.beta = d.beta;
+  }
   a.D = d.D;
   a.ldd = d.ldd;
   a.stride_d = d.stride_d;
@@ -1169,11 +1220,19 @@ nc_status launch_pair(const nc_gemm_desc& d, int split, int* status, const char*
   // Algorithmic FLOPs: a symmetric output counts the tiles it computes.
   const double flops = symmetric ? 2.0 * d.K * d.batch * (double)plane * 256.0 * 256.0
                                  : 2.0 * d.M * (double)d.N * d.K * d.batch;
+  (void)bk;
   Probe probe(prof, s, tag, flops, 0.0);
-  if constexpr (XR)
-    NC_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_tc2_aux_kernel, ta, tb, tx, a));
-  else
-    NC_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<ROPE>, ta, tb, a));
+  if constexpr (XR) {
+    if (fp8)
+      NC_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_tc2_aux_kernel<true>, ta, tb, tx, a));
+    else
+      NC_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_tc2_aux_kernel<false>, ta, tb, tx, a));
+  } else {
+    if (fp8)
+      NC_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<ROPE, true>, ta, tb, a));
+    else
+      NC_CUDA_TRY(cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<ROPE, false>, ta, tb, a));
+  }
   return NC_OK;
 }
 
@@ -1215,6 +1274,14 @@ nc_status gemm_launch(const GemmLaunch& g, cudaStream_t s, Profiler* prof) {
   if (d.M < 1 || d.N < 1 || d.K < 1 || d.batch < 1 || !d.A || !d.B || !d.D)
     return fail(NC_ERR_INVALID_ARG, "gemm: empty shape or null operand");
   auto aligned = [](int64_t v) { return v % 8 == 0; };
+  if (d.ab_type != 0 && d.ab_type != 1) return fail(NC_ERR_INVALID_ARG, "gemm: unknown operand type");
+  const bool fp8 = d.ab_type == 1;
+  if (fp8 && (!d.a_kmajor || !d.b_kmajor || d.lda % 16 || d.ldb % 16 ||
+              (d.batch > 1 && (d.stride_a % 16 || d.stride_b % 16)) || !d.ab_scale || d.alpha != 1.f ||
+              d.epi == NC_EPI_AXPBY_BF16 || g.symmetric))
+    return fail(NC_ERR_INVALID_ARG,
+                "gemm: E4M3 operands must be K-major with leading dimensions and batch strides of "
+                "16-byte multiples, scales given, alpha 1 and no alpha*acc + beta*aux epilogue");
   if (!aligned(d.lda) || !aligned(d.ldb) || (d.batch > 1 && (!aligned(d.stride_a) || !aligned(d.stride_b))))
     return fail(NC_ERR_INVALID_ARG, "gemm: leading dimensions and batch strides must be multiples of 8");
   if ((reinterpret_cast<uintptr_t>(d.A) | reinterpret_cast<uintptr_t>(d.B)) & 15)
@@ -1244,8 +1311,8 @@ nc_status gemm_launch(const GemmLaunch& g, cudaStream_t s, Profiler* prof) {
   // (a symmetric output walks square 256 x 256 tiles whatever the edge waste)
   const bool bn256 = rope || g.symmetric || (d.N > 128 && waste256 <= waste128);
   const int bn = bn256 ? 256 : 128;
-  const int num_kb = (d.K + BK - 1) / BK;
-  const double operand_bytes = 2.0 * ((double)d.M + d.N) * d.K * d.batch;
+  const int num_kb = (d.K + (fp8 ? 2 * BK : BK) - 1) / (fp8 ? 2 * BK : BK);
+  const double operand_bytes = (fp8 ? 1.0 : 2.0) * ((double)d.M + d.N) * d.K * d.batch;
   if (split <= 0) {
     const int64_t tiles = (int64_t)((d.M + BM - 1) / BM) * ((d.N + bn - 1) / bn) * d.batch;
     split = auto_split(tiles, num_kb, operand_bytes);
@@ -1269,6 +1336,8 @@ nc_status gemm_launch(const GemmLaunch& g, cudaStream_t s, Profiler* prof) {
       return launch_pair<false, true>(d, split, g.status, g.tag, s, prof, g.symmetric);
     return launch_pair<false, false>(d, split, g.status, g.tag, s, prof, g.symmetric);
   }
+  if (fp8)
+    return fail(NC_ERR_INVALID_ARG, "gemm: E4M3 operands need M > 128 and 256-wide column tiles");
   if (rope) return launch_bn<256, true>(d, split, g.status, g.tag, s, prof);
   return bn256 ? launch_bn<256, false>(d, split, g.status, g.tag, s, prof)
                : launch_bn<128, false>(d, split, g.status, g.tag, s, prof);

@@ -16,6 +16,11 @@ namespace nc {
 bool make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
                        uint64_t batch, int64_t ld, int64_t bstride, uint32_t box_outer);
 
+// The same for 8-bit elements (fp8 operands): box {128, box_outer, 1}, one
+// 128-byte swizzled row of 128 elements per outer index.
+bool make_tmap_u8_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                     uint64_t batch, int64_t ld, int64_t bstride, uint32_t box_outer);
+
 // 3-D TMA tensor map of fp32 (f32) or bf16 elements with an explicit box
 // {box_inner, box_outer, 1} and swizzle span (0, 32, 64 or 128 bytes).
 bool make_tmap_3d(CUtensorMap* m, const void* base, bool f32, uint64_t inner, uint64_t outer,
@@ -109,6 +114,14 @@ nc_status ce_fwd_bwd(void* z, const int32_t* tgt, int64_t n, int V, float* loss_
                      float* loss_out, int* status, cudaStream_t s, Profiler* prof);
 nc_status init_normal(float* out, int64_t n, uint64_t key, float stdv, cudaStream_t s);
 nc_status f32_to_bf16(const float* in, void* out, int64_t n, cudaStream_t s, Profiler* prof);
+// E4M3 quantisation of a rows x cols matrix (bf16, or fp32 when !bf16; row
+// stride ld, cols a multiple of 8, rows too when transposing) with one
+// dynamic scale s = 448 / amax, written to *scale: q[r * ldq + c] (or the
+// transpose, q[c * ldq + r]) = E4M3(x[r, c] * s).  amax_scratch: one device
+// word of scratch.
+nc_status fp8_quantize(const void* x, bool bf16, int64_t rows, int cols, int64_t ld, bool transpose,
+                       uint8_t* q, int64_t ldq, float* scale, unsigned* amax_scratch, cudaStream_t s,
+                       Profiler* prof);
 // y[i] = 2^x[i] by exp2_fma2 (exp2_poly.cuh), the softmax's FMA-pipe exponential.
 nc_status exp2_poly(const float* x, float* y, int64_t n, cudaStream_t s);
 // Momentum and per-matrix squared norms over the 6*L block matrices; dkv is

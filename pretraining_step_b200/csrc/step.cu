@@ -975,6 +975,18 @@ nc_status nc_op_embed_gather(const int32_t* tokens, int64_t n, const float* E, i
   return embed_gather(tokens, n, E, vocab, d, x, st, static_cast<cudaStream_t>(stream), nullptr);
 }
 
+nc_status nc_op_fp8_quantize(const void* x, int x_bf16, int64_t rows, int cols, int64_t ldx, int transpose,
+                             void* q, int64_t ldq, float* scale, void* scratch, void* stream) {
+  if (!x || !q || !scale || !scratch || rows < 1 || cols < 8 || cols % 8 || ldx < cols || ldx % 8 ||
+      (transpose && rows % 8) || ldq % 16 || ldq < (transpose ? rows : (int64_t)cols))
+    return fail(NC_ERR_INVALID_ARG, "fp8_quantize: bad arguments (cols and ldx multiples of 8, rows too "
+                                    "when transposing, ldq a multiple of 16)");
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(q)) & 15)
+    return fail(NC_ERR_INVALID_ARG, "fp8_quantize: x and q must be 16-byte aligned");
+  return fp8_quantize(x, x_bf16 != 0, rows, cols, ldx, transpose != 0, static_cast<uint8_t*>(q), ldq, scale,
+                      static_cast<unsigned*>(scratch), static_cast<cudaStream_t>(stream), nullptr);
+}
+
 nc_status nc_op_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
   if (n < 0 || (n > 0 && (!x || !y))) return fail(NC_ERR_INVALID_ARG, "exp2_poly: bad arguments");
   if (n == 0) return NC_OK;

@@ -44,6 +44,20 @@ bool make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap_u8_3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                     uint64_t batch, int64_t ld, int64_t bstride, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, outer, batch};
+  cuuint64_t strides[2] = {(cuuint64_t)ld, (cuuint64_t)(batch > 1 ? bstride : ld * (int64_t)outer)};
+  cuuint32_t box[3] = {128, box_outer, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool make_tmap_3d(CUtensorMap* m, const void* base, bool f32, uint64_t inner, uint64_t outer,
                   uint64_t batch, int64_t ld, int64_t bstride, uint32_t box_inner, uint32_t box_outer,
                   int swizzle_bytes) {

@@ -247,6 +247,113 @@ def test_exp2_poly_relative_error():
         nc.exp2_poly(ds, ys, -1)
 
 
+# ------------------------------------------------------------------ fp8 (E4M3)
+def _e4m3_decode(q):
+    """Values of E4M3 bytes from the format's definition: sign bit, 4-bit
+    exponent with bias 7, 3-bit mantissa; exponent 0 is subnormal (m * 2^-9);
+    0x7f / 0xff are NaN."""
+    b = np.arange(256)
+    sign = np.where(b & 0x80, -1.0, 1.0)
+    e, m = (b >> 3) & 0xF, b & 7
+    val = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * 2.0 ** (e - 7.0)) * sign
+    val[(b & 0x7F) == 0x7F] = np.nan
+    return val[np.asarray(q, dtype=np.int64)]
+
+
+def _fp8_oracle_q(x, activation):
+    """The oracle's quantised values of x: scale s = oracle.fp8_scale, then
+    E4M3 of the fp32 product x * s (oracle.e4m3_round)."""
+    s = np.float32(oracle.fp8_scale(x, activation=activation))
+    return s, oracle.e4m3_round((np.float32(x) * s).astype(np.float64))
+
+
+@pytest.mark.parametrize("bf16,transpose", [(True, False), (True, True), (False, False), (False, True)])
+def test_fp8_quantize_is_bit_exact(bf16, transpose):
+    t = torch()
+    rows, cols = 80, 208  # ragged against the 64 x 64 transpose tiles
+    x = inputs.bf16_normal(5, (rows, cols)) * 3.0
+    x[3, 7] = 0.0
+    x[10, :8] = [1e-4, -2e-3, 5e-3, 0.3, -7.0, 12.5, -0.0, 0.011]  # subnormal and normal codes
+    x = inputs.round_to_bf16(x.astype(np.float32))  # the same numbers on both paths
+    dx = dev_bf16(x) if bf16 else dev_f32(x)
+    q = t.zeros((cols, rows) if transpose else (rows, cols), dtype=t.uint8, device="cuda")
+    sc = t.zeros(2, dtype=t.float32, device="cuda")
+    scratch = t.zeros(1, dtype=t.int32, device="cuda")
+    nc.fp8_quantize(dx, rows, cols, q, sc, scratch, transpose=transpose)
+    t.cuda.synchronize()
+    s_ref, q_ref = _fp8_oracle_q(x, activation=bf16)
+    assert np.float32(host(sc)[0]) == s_ref
+    got = _e4m3_decode(host(q))
+    assert np.array_equal(got.T if transpose else got, q_ref)
+    # Saturation: the largest magnitude lands on 448 exactly.
+    assert np.nanmax(np.abs(got)) == 448.0
+
+
+@pytest.mark.parametrize("M,N,K,epi", [(512, 768, 640, "f32"), (300, 512, 1000, "f32"),
+                                       (640, 1280, 1280, "bf16"), (384, 256, 256, "resid")])
+def test_fp8_gemm_matches_the_oracle(M, N, K, epi):
+    """y = x W^T on E4M3 operands (x an activation, W a weight), each with its
+    own scale, against the oracle's fp64 product of the same quantised
+    values; ragged M and K included.  The tensor cores sum the exact E4M3
+    products in fp32, so the fp32 output is within 1e-5 (relative Frobenius)
+    and the bf16 output within one bf16 rounding."""
+    t = torch()
+    x = inputs.bf16_normal(11, (M, K))
+    w = (inputs.bf16_normal(12, (N, K)) * K ** -0.5).astype(np.float32)
+    Kp = (K + 15) // 16 * 16
+    qx = t.zeros((M, Kp), dtype=t.uint8, device="cuda")
+    qw = t.zeros((N, Kp), dtype=t.uint8, device="cuda")
+    sc = t.zeros(2, dtype=t.float32, device="cuda")
+    scratch = t.zeros(2, dtype=t.int32, device="cuda")
+    nc.fp8_quantize(dev_bf16(x), M, K, qx, sc[0:1], scratch[0:1], ldq=Kp)
+    nc.fp8_quantize(dev_f32(w), N, K, qw, sc[1:2], scratch[1:2], ldq=Kp)
+    ref = oracle.fp8_matmul_nt(x, w)
+    if epi == "resid":
+        R = inputs.bf16_normal(13, (M, N)).astype(np.float32)
+        D = dev_f32(R)
+        nc.gemm(M, N, K, qx, qw, D, lda=Kp, ldb=Kp, epi=nc.EPI_RESID_F32, aux=D, ab_scale=sc)
+        ref = ref + R
+    else:
+        D = t.zeros(M, N, dtype=t.float32 if epi == "f32" else t.bfloat16, device="cuda")
+        nc.gemm(M, N, K, qx, qw, D, lda=Kp, ldb=Kp,
+                epi=nc.EPI_STORE_F32 if epi == "f32" else nc.EPI_STORE_BF16, ab_scale=sc)
+    t.cuda.synchronize()
+    assert rel_fro(host(D), ref) < (5e-3 if epi == "bf16" else 1e-5)
+
+
+def test_fp8_gemm_weight_gradient_form():
+    """dW = dy^T x (split K, fp32 accumulate) from transposed E4M3 copies of
+    both activations (K = tokens), against the oracle's quantised product."""
+    t = torch()
+    rows, n, k = 1024, 384, 256
+    dy = inputs.bf16_normal(21, (rows, n))
+    x = inputs.bf16_normal(22, (rows, k))
+    qd = t.zeros((n, rows), dtype=t.uint8, device="cuda")
+    qx = t.zeros((k, rows), dtype=t.uint8, device="cuda")
+    sc = t.zeros(2, dtype=t.float32, device="cuda")
+    scratch = t.zeros(2, dtype=t.int32, device="cuda")
+    nc.fp8_quantize(dev_bf16(dy), rows, n, qd, sc[0:1], scratch[0:1], transpose=True)
+    nc.fp8_quantize(dev_bf16(x), rows, k, qx, sc[1:2], scratch[1:2], transpose=True)
+    D = t.zeros(n, k, dtype=t.float32, device="cuda")
+    nc.gemm(n, k, rows, qd, qx, D, epi=nc.EPI_ACC_F32, split_k=0, ab_scale=sc)
+    t.cuda.synchronize()
+    ref = oracle.fp8_matmul_nt(np.ascontiguousarray(dy.T), np.ascontiguousarray(x.T))
+    assert rel_fro(host(D), ref) < 1e-5
+
+
+def test_fp8_gemm_rejects_unsupported_forms():
+    t = torch()
+    q = t.zeros((512, 512), dtype=t.uint8, device="cuda")
+    sc = t.ones(2, dtype=t.float32, device="cuda")
+    D = t.zeros(512, 512, dtype=t.float32, device="cuda")
+    with pytest.raises(nc.NcError):
+        nc.gemm(512, 512, 512, q, q, D, a_kmajor=False, epi=nc.EPI_STORE_F32, ab_scale=sc)
+    with pytest.raises(nc.NcError):
+        nc.gemm(512, 512, 512, q, q, D, epi=nc.EPI_STORE_F32, alpha=2.0, ab_scale=sc)
+    with pytest.raises(nc.NcError):
+        nc.gemm(100, 512, 512, q, q, D, epi=nc.EPI_STORE_F32, ab_scale=sc)  # M <= 128
+
+
 def test_planted_op_status_is_reported_once():
     """An expired bounded wait inside an op (planted here as its status code,
     not produced by a stuck kernel) surfaces as NC_ERR_TIMEOUT at the next
