@@ -851,7 +851,7 @@ def run_step_variant(args, dims, peaks, peak_kind):
     stream = torch.cuda.Stream()
     vocab = args.vocab
     m = nc.GPT(depth, vocab=vocab, seed=1234, all_random=True, stream=stream,
-               n_kv_head=args.kv_heads, window=windows)
+               n_kv_head=args.kv_heads, window=windows, fp8=args.fp8)
     tk, tg = inputs.token_batch(20, Bb, T_, vocab=vocab)
     tok, tgt = torch.from_numpy(tk).cuda(), torch.from_numpy(tg).cuda()
     loss = torch.zeros(1, dtype=torch.float32, device="cuda")
@@ -880,6 +880,7 @@ def run_step_variant(args, dims, peaks, peak_kind):
     fpt = step_flops_per_token(depth, T_, vocab, args.kv_heads, windows)
     print(json.dumps({"op": "step", "depth": depth, "B": Bb, "T": T_, "vocab": vocab,
                       "kv_heads": args.kv_heads, "device_gb_in_use": (total - free) / 1e9,
+                      "gemm_operands": "e4m3 (block projections)" if args.fp8 else "bf16",
                       "device_gb_total": total / 1e9,
                       "windows": windows, "ms_per_step": ms, "tokens_per_s": tok_s,
                       "flops_per_token": fpt, "tflops": tok_s * fpt / 1e12,
@@ -908,7 +909,8 @@ def main():
                     help="--op step: vocabulary (smaller only for kernel captures on a small case)")
     ap.add_argument("--shape", default="16384,5120,1280")
     ap.add_argument("--fp8", action="store_true",
-                    help="--op gemm: E4M3 operands (quantised before timing) with per-tensor scales")
+                    help="--op gemm: E4M3 operands (quantised before timing) with per-tensor "
+                         "scales; --op step: the model's fp8 mode")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -110,6 +110,15 @@ typedef struct {
   int flags;
   int n_kv_head;
   const int32_t* window;
+  /* Non-zero: the guide's "--fp8" training (section "1. Modelo GPT"): every
+   * GEMM of the block projections (q|k|v, o, up, down; forward, input and
+   * weight gradients) runs on E4M3 operands, each operand tensor quantised
+   * whole with its own dynamic scale (nc_op_fp8_quantize; wq|wk|wv as one
+   * tensor, weights from their fp32 masters), the products dequantised in
+   * the GEMM epilogue; lm_head, attention and the norms stay as they are.
+   * Needs d >= 256 (NC_ERR_UNSUPPORTED) and B*T > 128, a multiple of 16
+   * (NC_ERR_INVALID_ARG from the step). */
+  int fp8;
 } nc_model_config;
 nc_status nc_gpt_init_config(const nc_model_config* cfg, nc_params** out);
 void nc_params_free(nc_params* p);

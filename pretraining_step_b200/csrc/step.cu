@@ -91,6 +91,11 @@ struct Acts {
   int64_t ld_ds = 0;  // row stride of ds: T rounded up to a multiple of 8
   float *rf = nullptr, *loss_rows = nullptr, *loss = nullptr, *dx0 = nullptr, *dx1 = nullptr,
         *delta = nullptr;
+  // fp8 mode: E4M3 copies of one GEMM's operands (A; B when it is an
+  // activation; a weight), the pair of scales the GEMM reads, amax scratch.
+  uint8_t *q8a = nullptr, *q8b = nullptr, *q8w = nullptr;
+  float* f8scale = nullptr;
+  unsigned* f8scratch = nullptr;
 };
 
 }  // namespace
@@ -99,6 +104,7 @@ struct Acts {
 struct nc_params {
   int depth = 0, vocab = 0, d = 0, H = 0, hd = 0, F = 0;
   int Hkv = 0, dkv = 0;     // KV heads and the width of k, v (dkv = 128 Hkv)
+  bool fp8 = false;         // block projections on E4M3 operands
   std::vector<int> window;  // per layer: causal left window, -1 = full causal
   cudaStream_t stream = nullptr;
   nc::Profiler* prof = nullptr;
@@ -253,6 +259,8 @@ nc_status ensure_acts(nc_params* p, int B, int T) {
   total += 2 * r(4 * N * d) + 2 * r(2 * N * d) + r(2 * N * F) + r(2 * N * Q) +
            r(4 * N * H);                                     // backward scratch
   total += r(2 * (int64_t)B * H * T * ld_ds);                // attention dS^T tiles
+  const int64_t wmax = std::max(F, Q) * d;                   // largest weight, elements
+  if (p->fp8) total += 2 * r(N * std::max(F, Q)) + r(wmax) + r(8) + r(8);  // E4M3 operands
   void* mem = nullptr;
   cudaError_t e = cudaMalloc(&mem, (size_t)total);
   if (e != cudaSuccess) {
@@ -294,6 +302,13 @@ nc_status ensure_acts(nc_params* p, int B, int T) {
   a.delta = ar.take<float>(N * H);
   a.ld_ds = ld_ds;
   a.ds = ar.take<bf16>((int64_t)B * H * T * ld_ds);
+  if (p->fp8) {
+    a.q8a = ar.take<uint8_t>(N * std::max(F, Q));
+    a.q8b = ar.take<uint8_t>(N * std::max(F, Q));
+    a.q8w = ar.take<uint8_t>(wmax);
+    a.f8scale = ar.take<float>(2);
+    a.f8scratch = ar.take<unsigned>(2);
+  }
   if (ar.used > ar.size) return fail(NC_ERR_CUDA, "activation arena overflow");
   return NC_OK;
 }
@@ -307,10 +322,33 @@ bool is_device_ptr(const void* ptr) {
   return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
 }
 
-// y[M,N] = epi(x[M,K] W[N,K]^T): the forward projection.
+// fp8 mode: the fp32 master of a block matrix from its bf16 copy.
+const float* master_of(const nc_params* p, const bf16* Wb) { return p->blocks + (Wb - p->blocks_b); }
+
+// fp8 mode: quantise one operand to E4M3 (one scale per tensor, into
+// f8scale[slot]): src [rows, cols] with row stride ld, bf16 or fp32, stored
+// K-major as [rows, cols] or, transposed, [cols, rows] (ldq its row length).
+nc_status quant8(nc_params* p, const void* src, bool bf16_src, int64_t rows, int64_t cols, int64_t ld,
+                 bool transpose, uint8_t* q, int slot) {
+  Acts& a = p->act;
+  return fp8_quantize(src, bf16_src, rows, (int)cols, ld, transpose, q, transpose ? rows : cols,
+                      a.f8scale + slot, a.f8scratch + slot, p->stream, p->prof);
+}
+
+// The GEMM of g on the E4M3 operands quantised into A (lda) and B (ldb).
+nc_status gemm8(nc_params* p, GemmLaunch g, const uint8_t* A, int64_t lda, const uint8_t* B, int64_t ldb) {
+  g.d.A = A; g.d.lda = lda; g.d.a_kmajor = 1;
+  g.d.B = B; g.d.ldb = ldb; g.d.b_kmajor = 1;
+  g.d.ab_type = 1;
+  g.d.ab_scale = p->act.f8scale;
+  return gemm_launch(g, p->stream, p->prof);
+}
+
+// y[M,N] = epi(x[M,K] W[N,K]^T): the forward projection.  fp8: a block
+// projection on E4M3 operands (x and W's fp32 master, each quantised whole).
 nc_status proj(nc_params* p, const bf16* x, int64_t M, int64_t K, const bf16* W, int64_t Nout,
                void* D, int64_t ldd, nc_epilogue epi, const void* aux, int64_t ldaux,
-               const char* tag = "gemm_fwd") {
+               const char* tag = "gemm_fwd", bool fp8 = true) {
   GemmLaunch g{};
   g.status = p->status;
   g.tag = tag;
@@ -320,13 +358,19 @@ nc_status proj(nc_params* p, const bf16* x, int64_t M, int64_t K, const bf16* W,
   g.d.D = D; g.d.ldd = ldd;
   g.d.aux = aux; g.d.ldaux = ldaux;
   g.d.epi = epi; g.d.alpha = 1.f; g.d.split_k = 1;
+  if (p->fp8 && fp8) {
+    Acts& a = p->act;
+    NC_TRY(quant8(p, x, true, M, K, K, false, a.q8a, 0));
+    NC_TRY(quant8(p, master_of(p, W), false, Nout, K, K, false, a.q8w, 1));
+    return gemm8(p, g, a.q8a, K, a.q8w, K);
+  }
   return gemm_launch(g, p->stream, p->prof);
 }
 
 // dx[M,N] = epi(dy[M,K] W[K,N]): the input gradient of a projection.
 nc_status proj_dx(nc_params* p, const bf16* dy, int64_t M, int64_t K, const bf16* W, int64_t Nout,
                   void* D, int64_t ldd, nc_epilogue epi, const void* aux, int64_t ldaux,
-                  const char* tag = "gemm_dgrad") {
+                  const char* tag = "gemm_dgrad", bool fp8 = true) {
   GemmLaunch g{};
   g.status = p->status;
   g.tag = tag;
@@ -336,13 +380,19 @@ nc_status proj_dx(nc_params* p, const bf16* dy, int64_t M, int64_t K, const bf16
   g.d.D = D; g.d.ldd = ldd;
   g.d.aux = aux; g.d.ldaux = ldaux;
   g.d.epi = epi; g.d.alpha = 1.f; g.d.split_k = 1;
+  if (p->fp8 && fp8) {  // dy as is; W [K, Nout] transposed to [Nout, K]
+    Acts& a = p->act;
+    NC_TRY(quant8(p, dy, true, M, K, K, false, a.q8a, 0));
+    NC_TRY(quant8(p, master_of(p, W), false, K, Nout, Nout, true, a.q8w, 1));
+    return gemm8(p, g, a.q8a, K, a.q8w, K);
+  }
   return gemm_launch(g, p->stream, p->prof);
 }
 
 // dW[Mo,No] = dy[Ntok,Mo]^T x[Ntok,No] into a zeroed fp32 gradient.
 nc_status proj_dw(nc_params* p, const bf16* dy, int64_t ldy, int64_t Mo, const bf16* x,
                   int64_t ldx, int64_t No, int64_t Ntok, float* dW,
-                  const char* tag = "gemm_wgrad") {
+                  const char* tag = "gemm_wgrad", bool fp8 = true) {
   GemmLaunch g{};
   g.status = p->status;
   g.tag = tag;
@@ -351,6 +401,12 @@ nc_status proj_dw(nc_params* p, const bf16* dy, int64_t ldy, int64_t Mo, const b
   g.d.B = x; g.d.ldb = ldx; g.d.b_kmajor = 0;
   g.d.D = dW; g.d.ldd = No;
   g.d.epi = NC_EPI_ACC_F32; g.d.alpha = 1.f; g.d.split_k = 0;  // automatic split
+  if (p->fp8 && fp8) {  // both transposed to K-major [., Ntok] copies
+    Acts& a = p->act;
+    NC_TRY(quant8(p, dy, true, Ntok, Mo, ldy, true, a.q8a, 0));
+    NC_TRY(quant8(p, x, true, Ntok, No, ldx, true, a.q8b, 1));
+    return gemm8(p, g, a.q8a, Ntok, a.q8b, Ntok);
+  }
   return gemm_launch(g, p->stream, p->prof);
 }
 
@@ -361,6 +417,8 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
   if (p->poisoned) return fail(NC_ERR_TIMEOUT, "handle poisoned by an earlier device timeout");
   if (!tokens || !targets || !g || g->p != p || B < 1 || T < 1 || (int64_t)B * T > (1 << 24))
     return fail(NC_ERR_INVALID_ARG, "fwd_bwd: bad arguments");
+  if (p->fp8 && (((int64_t)B * T) % 16 || (int64_t)B * T <= 128))
+    return fail(NC_ERR_INVALID_ARG, "fwd_bwd: fp8 mode needs B*T > 128 and a multiple of 16");
   NC_TRY(ensure_acts(p, B, T));
   NC_TRY(ensure_rope(p, T));
   Acts& a = p->act;
@@ -400,7 +458,13 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
       g.d.epi = NC_EPI_ROPE_QKNORM; g.d.alpha = 1.f; g.d.split_k = 1;
       g.d.rope_T = T; g.d.rope_H = H; g.d.rope_Hkv = Hkv; g.d.rope_tab = p->rope;
       g.d.rstd_q = a.rq[l]; g.d.rstd_k = a.rk[l];
-      NC_TRY(gemm_launch(g, s, pr));
+      if (p->fp8) {  // wq|wk|wv quantised as one [Q, d] tensor
+        NC_TRY(quant8(p, a.h1[l], true, N, d, d, false, a.q8a, 0));
+        NC_TRY(quant8(p, master_of(p, W), false, Q, d, d, false, a.q8w, 1));
+        NC_TRY(gemm8(p, g, a.q8a, d, a.q8w, d));
+      } else {
+        NC_TRY(gemm_launch(g, s, pr));
+      }
     }
     NC_TRY(attention_fwd_ex(a.qkv[l], Q, a.qkv[l] + d, a.qkv[l] + d + dkv, Q, a.o[l], d,
                             a.lse[l], B, T, H, Hkv, p->window[l], p->status, s, pr));
@@ -411,14 +475,14 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
   }
   NC_TRY(rmsnorm_fwd(a.x[L], N, (int)d, a.hf, a.rf, s, pr));
   NC_TRY(proj(p, a.hf, N, d, p->lm_b, V, a.logits, V, NC_EPI_STORE_BF16, nullptr, 0,
-              "gemm_lmhead"));
+              "gemm_lmhead", false));
   NC_TRY(ce_fwd_bwd(a.logits, tgt, N, V, a.loss_rows, loss_dev ? loss_dev : a.loss, p->status, s,
                     pr));
 
   // ---------------- backward (a.logits now holds dz)
-  NC_TRY(proj_dw(p, a.logits, V, V, a.hf, d, d, N, g->lm, "gemm_lmhead"));
+  NC_TRY(proj_dw(p, a.logits, V, V, a.hf, d, d, N, g->lm, "gemm_lmhead", false));
   NC_TRY(proj_dx(p, a.logits, N, V, p->lm_b, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0,
-                 "gemm_lmhead"));
+                 "gemm_lmhead", false));
   float* dx = a.dx0;
   float* dxn = a.dx1;
   NC_TRY(rmsnorm_bwd(a.dh, a.hf, a.rf, nullptr, N, (int)d, dx, a.dxb, s, pr));
@@ -611,6 +675,11 @@ nc_status nc_gpt_init_config(const nc_model_config* cfg, nc_params** out) {
   p->Hkv = Hkv;
   p->dkv = 128 * Hkv;
   p->F = 4 * p->d;
+  if (cfg->fp8 && p->d < 256) {
+    delete p;
+    return fail(NC_ERR_UNSUPPORTED, "init: fp8 mode needs d >= 256 (depth >= 4)");
+  }
+  p->fp8 = cfg->fp8 != 0;
   p->window.assign(depth, -1);
   if (cfg->window)
     for (int l = 0; l < depth; ++l) p->window[l] = cfg->window[l] < 0 ? -1 : cfg->window[l];
