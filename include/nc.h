@@ -288,6 +288,13 @@ nc_status nc_op_exp2_poly(const float* x, float* y, int64_t n, void* stream);
 nc_status nc_op_fp8_quantize(const void* x, int x_bf16, int64_t rows, int cols, int64_t ldx, int transpose,
                              void* q, int64_t ldq, float* scale, void* scratch, void* stream);
 
+/* The same quantisation of a bf16 matrix into both layouts in one pass:
+ * q[r*cols + c] and qT[c*rows + r] (either may be NULL), the form the fp8
+ * model uses for an operand that feeds a GEMM and, transposed, a weight
+ * gradient.  rows, cols and ldx multiples of 8; pointers 16-byte aligned. */
+nc_status nc_op_fp8_quantize2(const void* x_bf16, int64_t rows, int cols, int64_t ldx, void* q, void* qT,
+                              float* scale, void* scratch, void* stream);
+
 /* Epilogues of the GEMM engine. */
 typedef enum {
   NC_EPI_STORE_BF16 = 0, /* D(bf16) = alpha*acc                               */

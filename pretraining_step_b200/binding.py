@@ -108,6 +108,7 @@ def lib():
         "nc_op_embed_gather": (ci, [vp, i64, vp, ci, ci, vp, vp]),
         "nc_op_exp2_poly": (ci, [vp, vp, i64, vp]),
         "nc_op_fp8_quantize": (ci, [vp, ci, i64, ci, i64, ci, vp, i64, vp, vp, vp]),
+        "nc_op_fp8_quantize2": (ci, [vp, i64, ci, i64, vp, vp, vp, vp, vp]),
         "nc_op_sync": (ci, [vp]),
         "nc_debug_op_status_word": (vp, []),
         "nc_op_attention_fwd": (ci, [vp, vp, vp, i64, vp, i64, vp, ci, ci, ci, vp]),
@@ -356,6 +357,12 @@ def fp8_quantize(x, rows, cols, q, scale, scratch, *, ldx=None, ldq=None, transp
     ldq = ldq if ldq is not None else (rows if transpose else cols)
     _check(lib().nc_op_fp8_quantize(_ptr(x), int(bf16), rows, cols, ldx, int(bool(transpose)), _ptr(q),
                                     ldq, _ptr(scale), _ptr(scratch), _stream(stream)))
+
+
+def fp8_quantize2(x, rows, cols, q, qT, scale, scratch, *, ldx=None, stream=None):
+    """Both layouts of the E4M3 quantisation of a bf16 matrix in one pass."""
+    _check(lib().nc_op_fp8_quantize2(_ptr(x), rows, cols, ldx if ldx is not None else cols, _ptr(q),
+                                     _ptr(qT), _ptr(scale), _ptr(scratch), _stream(stream)))
 
 
 def exp2_poly(x, y, n, stream=None):

@@ -715,6 +715,75 @@ __global__ void __launch_bounds__(256) fp8_quant_t_kernel(const void* __restrict
   }
 }
 
+// Both layouts of a bf16 matrix in one pass: q[r * cols + c] and
+// qT[c * rows + r] (either may be null), through 64 x 128 tiles; rows and
+// cols multiples of 8.  The scale goes to s0 and, when given, s1.
+__global__ void __launch_bounds__(256) fp8_quant2_kernel(const __nv_bfloat16* __restrict__ x, int64_t rows,
+                                                         int cols, int64_t ld, const unsigned* amax_bits,
+                                                         uint8_t* __restrict__ q, uint8_t* __restrict__ qT,
+                                                         float* s0, float* s1) {
+  __shared__ uint8_t tile[128][65];  // [column][row]; the odd row length spreads the byte writes over banks
+  const float s = fp8_scale_of(amax_bits);
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+    if (s0) *s0 = s;
+    if (s1) *s1 = s;
+  }
+  const int64_t r0 = (int64_t)blockIdx.y * 64;
+  const int c0 = blockIdx.x * 128;
+  for (int u = threadIdx.x; u < 64 * 16; u += blockDim.x) {
+    const int rr = u >> 4, cg = (u & 15) * 8;
+    const int64_t r = r0 + rr;
+    const int c = c0 + cg;
+    uint32_t w0 = 0, w1 = 0;
+    if (r < rows && c < cols) {
+      float v[8];
+      fp8_load8(x, true, r * ld + c, v);
+      w0 = e4m3x2(v[0] * s, v[1] * s) | (e4m3x2(v[2] * s, v[3] * s) << 16);
+      w1 = e4m3x2(v[4] * s, v[5] * s) | (e4m3x2(v[6] * s, v[7] * s) << 16);
+      if (q) *reinterpret_cast<uint2*>(q + r * cols + c) = make_uint2(w0, w1);
+    }
+    if (qT) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        tile[cg + j][rr] = (uint8_t)(w0 >> (8 * j));
+        tile[cg + 4 + j][rr] = (uint8_t)(w1 >> (8 * j));
+      }
+    }
+  }
+  if (!qT) return;
+  __syncthreads();
+  for (int u = threadIdx.x; u < 128 * 8; u += blockDim.x) {
+    const int cc = u >> 3, rg = (u & 7) * 8;
+    const int c = c0 + cc;
+    const int64_t r = r0 + rg;
+    if (c < cols && r < rows) {
+      uint32_t o0 = 0, o1 = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        o0 |= (uint32_t)tile[cc][rg + j] << (8 * j);
+        o1 |= (uint32_t)tile[cc][rg + 4 + j] << (8 * j);
+      }
+      *reinterpret_cast<uint2*>(qT + (int64_t)c * rows + r) = make_uint2(o0, o1);
+    }
+  }
+}
+
+nc_status fp8_quantize2(const void* x, int64_t rows, int cols, int64_t ld, uint8_t* q, uint8_t* qT, float* s0,
+                        float* s1, unsigned* amax_scratch, cudaStream_t s, Profiler* prof) {
+  Probe probe(prof, s, "fp8_quantize", 0.0,
+              (double)rows * cols * (2.0 * 2 + (q ? 1.0 : 0.0) + (qT ? 1.0 : 0.0)));
+  NC_CUDA_TRY(cudaMemsetAsync(amax_scratch, 0, sizeof(unsigned), s));
+  const int64_t units = rows * (cols / 8);
+  const unsigned g = (unsigned)std::min<int64_t>((units + 255) / 256, 8LL * num_sms());
+  fp8_amax_kernel<<<g, 256, 0, s>>>(x, 1, rows, cols, ld, amax_scratch);
+  NC_CUDA_TRY(cudaGetLastError());
+  dim3 grid((unsigned)((cols + 127) / 128), (unsigned)((rows + 63) / 64));
+  fp8_quant2_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), rows, cols, ld, amax_scratch, q,
+                                         qT, s0, s1);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
 nc_status fp8_quantize(const void* x, bool bf16, int64_t rows, int cols, int64_t ld, bool transpose,
                        uint8_t* q, int64_t ldq, float* scale, unsigned* amax_scratch, cudaStream_t s,
                        Profiler* prof) {

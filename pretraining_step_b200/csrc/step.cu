@@ -25,6 +25,7 @@
 //   (overwritten in place by their gradient), backward scratch.
 
 #include <algorithm>
+#include <array>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -91,12 +92,21 @@ struct Acts {
   int64_t ld_ds = 0;  // row stride of ds: T rounded up to a multiple of 8
   float *rf = nullptr, *loss_rows = nullptr, *loss = nullptr, *dx0 = nullptr, *dx1 = nullptr,
         *delta = nullptr;
-  // fp8 mode: E4M3 copies of one GEMM's operands (A; B when it is an
-  // activation; a weight), the pair of scales the GEMM reads, amax scratch.
-  uint8_t *q8a = nullptr, *q8b = nullptr, *q8w = nullptr;
-  float* f8scale = nullptr;
+  // fp8 mode: E4M3 copies of the forward activations each layer's
+  // projections read, in both layouts (K-major for the forward GEMM, the
+  // transpose for the weight gradient's): q8f[l][0..7] = h1, h1^T, o, o^T,
+  // h2, h2^T, a, a^T.  q8g / q8gT: the gradient being propagated, both
+  // layouts; q8w: one weight (or its transpose).  f8sc[l][g][2]: the (A, B)
+  // scales of GEMM g of layer l (F8_*); f8scratch: amax scratch.
+  std::vector<std::array<uint8_t*, 8>> q8f;
+  uint8_t *q8g = nullptr, *q8gT = nullptr, *q8w = nullptr;
+  float* f8sc = nullptr;
   unsigned* f8scratch = nullptr;
 };
+
+// The twelve E4M3 GEMMs of a layer in fp8 mode (their scale pairs in f8sc).
+enum { F8_QKV_F, F8_O_F, F8_UP_F, F8_DOWN_F, F8_QKV_D, F8_O_D, F8_UP_D, F8_DOWN_D,
+       F8_QKV_W, F8_O_W, F8_UP_W, F8_DOWN_W, F8_COUNT };
 
 }  // namespace
 }  // namespace nc
@@ -260,7 +270,9 @@ nc_status ensure_acts(nc_params* p, int B, int T) {
            r(4 * N * H);                                     // backward scratch
   total += r(2 * (int64_t)B * H * T * ld_ds);                // attention dS^T tiles
   const int64_t wmax = std::max(F, Q) * d;                   // largest weight, elements
-  if (p->fp8) total += 2 * r(N * std::max(F, Q)) + r(wmax) + r(8) + r(8);  // E4M3 operands
+  if (p->fp8)  // E4M3 operands: saved activations, the propagated gradient, a weight, scales
+    total += L * (6 * r(N * d) + 2 * r(N * F)) + 2 * r(N * std::max(F, Q)) + r(wmax) +
+             r(4 * L * F8_COUNT * 2) + r(4);
   void* mem = nullptr;
   cudaError_t e = cudaMalloc(&mem, (size_t)total);
   if (e != cudaSuccess) {
@@ -303,11 +315,14 @@ nc_status ensure_acts(nc_params* p, int B, int T) {
   a.ld_ds = ld_ds;
   a.ds = ar.take<bf16>((int64_t)B * H * T * ld_ds);
   if (p->fp8) {
-    a.q8a = ar.take<uint8_t>(N * std::max(F, Q));
-    a.q8b = ar.take<uint8_t>(N * std::max(F, Q));
+    a.q8f.resize(L);
+    for (int l = 0; l < L; ++l)
+      for (int j = 0; j < 8; ++j) a.q8f[l][j] = ar.take<uint8_t>(j < 6 ? N * d : N * F);
+    a.q8g = ar.take<uint8_t>(N * std::max(F, Q));
+    a.q8gT = ar.take<uint8_t>(N * std::max(F, Q));
     a.q8w = ar.take<uint8_t>(wmax);
-    a.f8scale = ar.take<float>(2);
-    a.f8scratch = ar.take<unsigned>(2);
+    a.f8sc = ar.take<float>((int64_t)L * F8_COUNT * 2);
+    a.f8scratch = ar.take<unsigned>(1);
   }
   if (ar.used > ar.size) return fail(NC_ERR_CUDA, "activation arena overflow");
   return NC_OK;
@@ -325,30 +340,43 @@ bool is_device_ptr(const void* ptr) {
 // fp8 mode: the fp32 master of a block matrix from its bf16 copy.
 const float* master_of(const nc_params* p, const bf16* Wb) { return p->blocks + (Wb - p->blocks_b); }
 
-// fp8 mode: quantise one operand to E4M3 (one scale per tensor, into
-// f8scale[slot]): src [rows, cols] with row stride ld, bf16 or fp32, stored
-// K-major as [rows, cols] or, transposed, [cols, rows] (ldq its row length).
-nc_status quant8(nc_params* p, const void* src, bool bf16_src, int64_t rows, int64_t cols, int64_t ld,
-                 bool transpose, uint8_t* q, int slot) {
-  Acts& a = p->act;
-  return fp8_quantize(src, bf16_src, rows, (int)cols, ld, transpose, q, transpose ? rows : cols,
-                      a.f8scale + slot, a.f8scratch + slot, p->stream, p->prof);
+// fp8 mode: an activation or gradient (bf16 [rows, cols], row stride ld) to
+// E4M3 in both layouts (either may be null), its scale to s0 (and s1).
+nc_status quant8(nc_params* p, const bf16* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* q,
+                 uint8_t* qT, float* s0, float* s1) {
+  return fp8_quantize2(x, rows, (int)cols, ld, q, qT, s0, s1, p->act.f8scratch, p->stream, p->prof);
 }
 
-// The GEMM of g on the E4M3 operands quantised into A (lda) and B (ldb).
-nc_status gemm8(nc_params* p, GemmLaunch g, const uint8_t* A, int64_t lda, const uint8_t* B, int64_t ldb) {
-  g.d.A = A; g.d.lda = lda; g.d.a_kmajor = 1;
-  g.d.B = B; g.d.ldb = ldb; g.d.b_kmajor = 1;
+// fp8 mode: the fp32 master of a block matrix ([rows, cols]) to E4M3 in
+// p->act.q8w, as is or transposed, its scale to s.
+nc_status quant8w(nc_params* p, const bf16* Wb, int64_t rows, int64_t cols, bool transpose, float* s) {
+  return fp8_quantize(master_of(p, Wb), false, rows, (int)cols, cols, transpose, p->act.q8w,
+                      transpose ? rows : cols, s, p->act.f8scratch, p->stream, p->prof);
+}
+
+// One E4M3 GEMM: D[M, N] = epi(A8[M, K] B8[N, K]^T / (sc[0] sc[1])), both
+// operands K-major; weight gradients (NC_EPI_ACC_F32) split K automatically.
+nc_status gemm8(nc_params* p, int64_t M, int64_t N, int64_t K, const uint8_t* A8, int64_t lda,
+                const uint8_t* B8, int64_t ldb, void* D, int64_t ldd, nc_epilogue epi, const void* aux,
+                int64_t ldaux, const float* sc, const char* tag) {
+  GemmLaunch g{};
+  g.status = p->status;
+  g.tag = tag;
+  g.d.M = (int)M; g.d.N = (int)N; g.d.K = (int)K; g.d.batch = 1;
+  g.d.A = A8; g.d.lda = lda; g.d.a_kmajor = 1;
+  g.d.B = B8; g.d.ldb = ldb; g.d.b_kmajor = 1;
+  g.d.D = D; g.d.ldd = ldd;
+  g.d.aux = aux; g.d.ldaux = ldaux;
+  g.d.epi = epi; g.d.alpha = 1.f; g.d.split_k = epi == NC_EPI_ACC_F32 ? 0 : 1;
   g.d.ab_type = 1;
-  g.d.ab_scale = p->act.f8scale;
+  g.d.ab_scale = sc;
   return gemm_launch(g, p->stream, p->prof);
 }
 
-// y[M,N] = epi(x[M,K] W[N,K]^T): the forward projection.  fp8: a block
-// projection on E4M3 operands (x and W's fp32 master, each quantised whole).
+// y[M,N] = epi(x[M,K] W[N,K]^T): the forward projection.
 nc_status proj(nc_params* p, const bf16* x, int64_t M, int64_t K, const bf16* W, int64_t Nout,
                void* D, int64_t ldd, nc_epilogue epi, const void* aux, int64_t ldaux,
-               const char* tag = "gemm_fwd", bool fp8 = true) {
+               const char* tag = "gemm_fwd") {
   GemmLaunch g{};
   g.status = p->status;
   g.tag = tag;
@@ -358,19 +386,13 @@ nc_status proj(nc_params* p, const bf16* x, int64_t M, int64_t K, const bf16* W,
   g.d.D = D; g.d.ldd = ldd;
   g.d.aux = aux; g.d.ldaux = ldaux;
   g.d.epi = epi; g.d.alpha = 1.f; g.d.split_k = 1;
-  if (p->fp8 && fp8) {
-    Acts& a = p->act;
-    NC_TRY(quant8(p, x, true, M, K, K, false, a.q8a, 0));
-    NC_TRY(quant8(p, master_of(p, W), false, Nout, K, K, false, a.q8w, 1));
-    return gemm8(p, g, a.q8a, K, a.q8w, K);
-  }
   return gemm_launch(g, p->stream, p->prof);
 }
 
 // dx[M,N] = epi(dy[M,K] W[K,N]): the input gradient of a projection.
 nc_status proj_dx(nc_params* p, const bf16* dy, int64_t M, int64_t K, const bf16* W, int64_t Nout,
                   void* D, int64_t ldd, nc_epilogue epi, const void* aux, int64_t ldaux,
-                  const char* tag = "gemm_dgrad", bool fp8 = true) {
+                  const char* tag = "gemm_dgrad") {
   GemmLaunch g{};
   g.status = p->status;
   g.tag = tag;
@@ -380,19 +402,13 @@ nc_status proj_dx(nc_params* p, const bf16* dy, int64_t M, int64_t K, const bf16
   g.d.D = D; g.d.ldd = ldd;
   g.d.aux = aux; g.d.ldaux = ldaux;
   g.d.epi = epi; g.d.alpha = 1.f; g.d.split_k = 1;
-  if (p->fp8 && fp8) {  // dy as is; W [K, Nout] transposed to [Nout, K]
-    Acts& a = p->act;
-    NC_TRY(quant8(p, dy, true, M, K, K, false, a.q8a, 0));
-    NC_TRY(quant8(p, master_of(p, W), false, K, Nout, Nout, true, a.q8w, 1));
-    return gemm8(p, g, a.q8a, K, a.q8w, K);
-  }
   return gemm_launch(g, p->stream, p->prof);
 }
 
 // dW[Mo,No] = dy[Ntok,Mo]^T x[Ntok,No] into a zeroed fp32 gradient.
 nc_status proj_dw(nc_params* p, const bf16* dy, int64_t ldy, int64_t Mo, const bf16* x,
                   int64_t ldx, int64_t No, int64_t Ntok, float* dW,
-                  const char* tag = "gemm_wgrad", bool fp8 = true) {
+                  const char* tag = "gemm_wgrad") {
   GemmLaunch g{};
   g.status = p->status;
   g.tag = tag;
@@ -401,13 +417,58 @@ nc_status proj_dw(nc_params* p, const bf16* dy, int64_t ldy, int64_t Mo, const b
   g.d.B = x; g.d.ldb = ldx; g.d.b_kmajor = 0;
   g.d.D = dW; g.d.ldd = No;
   g.d.epi = NC_EPI_ACC_F32; g.d.alpha = 1.f; g.d.split_k = 0;  // automatic split
-  if (p->fp8 && fp8) {  // both transposed to K-major [., Ntok] copies
-    Acts& a = p->act;
-    NC_TRY(quant8(p, dy, true, Ntok, Mo, ldy, true, a.q8a, 0));
-    NC_TRY(quant8(p, x, true, Ntok, No, ldx, true, a.q8b, 1));
-    return gemm8(p, g, a.q8a, Ntok, a.q8b, Ntok);
-  }
   return gemm_launch(g, p->stream, p->prof);
+}
+
+// The backward of layer l in fp8 mode: the layer's eight GEMMs on E4M3
+// operands (the propagated gradient quantised once per projection in both
+// layouts, the forward activations' transposes saved by the forward, each
+// weight's transpose from its master), the rest as in the bf16 step.  dx:
+// the residual gradient, in and out (through dxn, as the bf16 step's two
+// norm backwards do); a.dxb its bf16 copy.
+nc_status layer_bwd_fp8(nc_params* p, int l, int B, int T, const bf16* W, float* G, float* dx, float* dxn) {
+  Acts& a = p->act;
+  cudaStream_t s = p->stream;
+  Profiler* pr = p->prof;
+  const int H = p->H, Hkv = p->Hkv;
+  const int64_t N = (int64_t)B * T, d = p->d, F = p->F, dkv = p->dkv, Q = qkv_width(p);
+  const int64_t o_wo = mat_offset(p, 3), o_up = mat_offset(p, 4), o_down = mat_offset(p, 5);
+  float* sc = a.f8sc + ((int64_t)l * F8_COUNT) * 2;
+  auto& q = a.q8f[l];
+  // MLP: x_out = xmid + a wdown^T, a = relu(h2 wup^T)^2
+  NC_TRY(quant8(p, a.dxb, N, d, d, a.q8g, a.q8gT, sc + 2 * F8_DOWN_D, sc + 2 * F8_DOWN_W));
+  NC_TRY(gemm8(p, d, F, N, a.q8gT, N, q[7], N, G + o_down, F, NC_EPI_ACC_F32, nullptr, 0, sc + 2 * F8_DOWN_W,
+               "gemm_wgrad"));
+  NC_TRY(quant8w(p, W + o_down, d, F, true, sc + 2 * F8_DOWN_D + 1));
+  NC_TRY(gemm8(p, N, F, d, a.q8g, d, a.q8w, d, a.du, F, NC_EPI_RELU2_BWD, a.a[l], F, sc + 2 * F8_DOWN_D,
+               "gemm_dgrad"));
+  NC_TRY(quant8(p, a.du, N, F, F, a.q8g, a.q8gT, sc + 2 * F8_UP_D, sc + 2 * F8_UP_W));
+  NC_TRY(gemm8(p, F, d, N, a.q8gT, N, q[5], N, G + o_up, d, NC_EPI_ACC_F32, nullptr, 0, sc + 2 * F8_UP_W,
+               "gemm_wgrad"));
+  NC_TRY(quant8w(p, W + o_up, F, d, true, sc + 2 * F8_UP_D + 1));
+  NC_TRY(gemm8(p, N, d, F, a.q8g, F, a.q8w, F, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0, sc + 2 * F8_UP_D,
+               "gemm_dgrad"));
+  NC_TRY(rmsnorm_bwd(a.dh, a.h2[l], a.r2[l], dx, N, (int)d, dxn, a.dxb, s, pr));
+  std::swap(dx, dxn);
+  // Attention: xmid = x + o wo^T
+  NC_TRY(quant8(p, a.dxb, N, d, d, a.q8g, a.q8gT, sc + 2 * F8_O_D, sc + 2 * F8_O_W));
+  NC_TRY(gemm8(p, d, d, N, a.q8gT, N, q[3], N, G + o_wo, d, NC_EPI_ACC_F32, nullptr, 0, sc + 2 * F8_O_W,
+               "gemm_wgrad"));
+  NC_TRY(quant8w(p, W + o_wo, d, d, true, sc + 2 * F8_O_D + 1));
+  NC_TRY(gemm8(p, N, d, d, a.q8g, d, a.q8w, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0, sc + 2 * F8_O_D,
+               "gemm_dgrad"));
+  NC_TRY(attention_bwd_model(a.qkv[l], Q, a.qkv[l] + d, a.qkv[l] + d + dkv, Q, a.o[l], a.dh, d, a.lse[l],
+                             a.delta, a.ds, a.ld_ds, a.dqkv, a.dqkv + d, a.dqkv + d + dkv, Q, B, T, H, Hkv,
+                             p->window[l], p->rope, p->rope_T, a.rq[l], a.rk[l], p->status, s, pr));
+  NC_TRY(quant8(p, a.dqkv, N, Q, Q, a.q8g, a.q8gT, sc + 2 * F8_QKV_D, sc + 2 * F8_QKV_W));
+  NC_TRY(gemm8(p, Q, d, N, a.q8gT, N, q[1], N, G, d, NC_EPI_ACC_F32, nullptr, 0, sc + 2 * F8_QKV_W,
+               "gemm_wgrad"));
+  NC_TRY(quant8w(p, W, Q, d, true, sc + 2 * F8_QKV_D + 1));
+  NC_TRY(gemm8(p, N, d, Q, a.q8g, Q, a.q8w, Q, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0, sc + 2 * F8_QKV_D,
+               "gemm_dgrad"));
+  // Back into the caller's dx (dxn here, after the swap above).
+  NC_TRY(rmsnorm_bwd(a.dh, a.h1[l], a.r1[l], dx, N, (int)d, dxn, a.dxb, s, pr));
+  return NC_OK;
 }
 
 // ids_on_device: the caller has established that tokens and targets are
@@ -458,16 +519,37 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
       g.d.epi = NC_EPI_ROPE_QKNORM; g.d.alpha = 1.f; g.d.split_k = 1;
       g.d.rope_T = T; g.d.rope_H = H; g.d.rope_Hkv = Hkv; g.d.rope_tab = p->rope;
       g.d.rstd_q = a.rq[l]; g.d.rstd_k = a.rk[l];
-      if (p->fp8) {  // wq|wk|wv quantised as one [Q, d] tensor
-        NC_TRY(quant8(p, a.h1[l], true, N, d, d, false, a.q8a, 0));
-        NC_TRY(quant8(p, master_of(p, W), false, Q, d, d, false, a.q8w, 1));
-        NC_TRY(gemm8(p, g, a.q8a, d, a.q8w, d));
-      } else {
-        NC_TRY(gemm_launch(g, s, pr));
+      if (p->fp8) {  // h1 in both layouts (the transpose for the weight gradient); wq|wk|wv as one tensor
+        float* sc = a.f8sc + ((int64_t)l * F8_COUNT) * 2;
+        NC_TRY(quant8(p, a.h1[l], N, d, d, a.q8f[l][0], a.q8f[l][1], sc + 2 * F8_QKV_F, sc + 2 * F8_QKV_W + 1));
+        NC_TRY(quant8w(p, W, Q, d, false, sc + 2 * F8_QKV_F + 1));
+        g.d.A = a.q8f[l][0]; g.d.lda = d;
+        g.d.B = a.q8w; g.d.ldb = d;
+        g.d.ab_type = 1;
+        g.d.ab_scale = sc + 2 * F8_QKV_F;
       }
+      NC_TRY(gemm_launch(g, s, pr));
     }
     NC_TRY(attention_fwd_ex(a.qkv[l], Q, a.qkv[l] + d, a.qkv[l] + d + dkv, Q, a.o[l], d,
                             a.lse[l], B, T, H, Hkv, p->window[l], p->status, s, pr));
+    if (p->fp8) {
+      float* sc = a.f8sc + ((int64_t)l * F8_COUNT) * 2;
+      auto& q = a.q8f[l];
+      NC_TRY(quant8(p, a.o[l], N, d, d, q[2], q[3], sc + 2 * F8_O_F, sc + 2 * F8_O_W + 1));
+      NC_TRY(quant8w(p, W + o_wo, d, d, false, sc + 2 * F8_O_F + 1));
+      NC_TRY(gemm8(p, N, d, d, q[2], d, a.q8w, d, a.xmid[l], d, NC_EPI_RESID_F32, a.x[l], d,
+                   sc + 2 * F8_O_F, "gemm_fwd"));
+      NC_TRY(rmsnorm_fwd(a.xmid[l], N, (int)d, a.h2[l], a.r2[l], s, pr));
+      NC_TRY(quant8(p, a.h2[l], N, d, d, q[4], q[5], sc + 2 * F8_UP_F, sc + 2 * F8_UP_W + 1));
+      NC_TRY(quant8w(p, W + o_up, F, d, false, sc + 2 * F8_UP_F + 1));
+      NC_TRY(gemm8(p, N, F, d, q[4], d, a.q8w, d, a.a[l], F, NC_EPI_RELU2, nullptr, 0, sc + 2 * F8_UP_F,
+                   "gemm_fwd"));
+      NC_TRY(quant8(p, a.a[l], N, F, F, q[6], q[7], sc + 2 * F8_DOWN_F, sc + 2 * F8_DOWN_W + 1));
+      NC_TRY(quant8w(p, W + o_down, d, F, false, sc + 2 * F8_DOWN_F + 1));
+      NC_TRY(gemm8(p, N, d, F, q[6], F, a.q8w, F, a.x[l + 1], d, NC_EPI_RESID_F32, a.xmid[l], d,
+                   sc + 2 * F8_DOWN_F, "gemm_fwd"));
+      continue;
+    }
     NC_TRY(proj(p, a.o[l], N, d, W + o_wo, d, a.xmid[l], d, NC_EPI_RESID_F32, a.x[l], d));
     NC_TRY(rmsnorm_fwd(a.xmid[l], N, (int)d, a.h2[l], a.r2[l], s, pr));
     NC_TRY(proj(p, a.h2[l], N, d, W + o_up, F, a.a[l], F, NC_EPI_RELU2, nullptr, 0));
@@ -475,20 +557,24 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
   }
   NC_TRY(rmsnorm_fwd(a.x[L], N, (int)d, a.hf, a.rf, s, pr));
   NC_TRY(proj(p, a.hf, N, d, p->lm_b, V, a.logits, V, NC_EPI_STORE_BF16, nullptr, 0,
-              "gemm_lmhead", false));
+              "gemm_lmhead"));
   NC_TRY(ce_fwd_bwd(a.logits, tgt, N, V, a.loss_rows, loss_dev ? loss_dev : a.loss, p->status, s,
                     pr));
 
   // ---------------- backward (a.logits now holds dz)
-  NC_TRY(proj_dw(p, a.logits, V, V, a.hf, d, d, N, g->lm, "gemm_lmhead", false));
+  NC_TRY(proj_dw(p, a.logits, V, V, a.hf, d, d, N, g->lm, "gemm_lmhead"));
   NC_TRY(proj_dx(p, a.logits, N, V, p->lm_b, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0,
-                 "gemm_lmhead", false));
+                 "gemm_lmhead"));
   float* dx = a.dx0;
   float* dxn = a.dx1;
   NC_TRY(rmsnorm_bwd(a.dh, a.hf, a.rf, nullptr, N, (int)d, dx, a.dxb, s, pr));
   for (int l = L - 1; l >= 0; --l) {
     const bf16* W = p->blocks_b + l * LS;
     float* G = g->blocks + l * LS;
+    if (p->fp8) {
+      NC_TRY(layer_bwd_fp8(p, l, B, T, W, G, dx, dxn));  // the gradient stays in dx
+      continue;
+    }
     // MLP: x_out = xmid + a wdown^T, a = relu(h2 wup^T)^2
     NC_TRY(proj_dw(p, a.dxb, d, d, a.a[l], F, F, N, G + o_down));
     NC_TRY(proj_dx(p, a.dxb, N, d, W + o_down, F, a.du, F, NC_EPI_RELU2_BWD, a.a[l], F));
@@ -1054,6 +1140,17 @@ nc_status nc_op_fp8_quantize(const void* x, int x_bf16, int64_t rows, int cols, 
     return fail(NC_ERR_INVALID_ARG, "fp8_quantize: x and q must be 16-byte aligned");
   return fp8_quantize(x, x_bf16 != 0, rows, cols, ldx, transpose != 0, static_cast<uint8_t*>(q), ldq, scale,
                       static_cast<unsigned*>(scratch), static_cast<cudaStream_t>(stream), nullptr);
+}
+
+nc_status nc_op_fp8_quantize2(const void* x_bf16, int64_t rows, int cols, int64_t ldx, void* q, void* qT,
+                              float* scale, void* scratch, void* stream) {
+  if (!x_bf16 || (!q && !qT) || !scale || !scratch || rows < 8 || rows % 8 || cols < 8 || cols % 8 ||
+      ldx < cols || ldx % 8)
+    return fail(NC_ERR_INVALID_ARG, "fp8_quantize2: bad arguments (rows, cols and ldx multiples of 8)");
+  if ((reinterpret_cast<uintptr_t>(x_bf16) | reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(qT)) & 15)
+    return fail(NC_ERR_INVALID_ARG, "fp8_quantize2: x, q and qT must be 16-byte aligned");
+  return fp8_quantize2(x_bf16, rows, cols, ldx, static_cast<uint8_t*>(q), static_cast<uint8_t*>(qT), scale,
+                       nullptr, static_cast<unsigned*>(scratch), static_cast<cudaStream_t>(stream), nullptr);
 }
 
 nc_status nc_op_exp2_poly(const float* x, float* y, int64_t n, void* stream) {

@@ -289,6 +289,29 @@ def test_fp8_quantize_is_bit_exact(bf16, transpose):
     assert np.nanmax(np.abs(got)) == 448.0
 
 
+def test_fp8_quantize_both_layouts_in_one_pass():
+    """The one-pass form (both layouts, 64 x 128 tiles, ragged here) gives
+    the single-layout op's bytes and scale, which match the oracle."""
+    t = torch()
+    rows, cols = 200, 328
+    x = inputs.round_to_bf16((inputs.bf16_normal(7, (rows, cols)) * 5.0).astype(np.float32))
+    dx = dev_bf16(x)
+    q = t.zeros((rows, cols), dtype=t.uint8, device="cuda")
+    qT = t.zeros((cols, rows), dtype=t.uint8, device="cuda")
+    q1 = t.zeros((rows, cols + 8), dtype=t.uint8, device="cuda")
+    sc = t.zeros(2, dtype=t.float32, device="cuda")
+    scratch = t.zeros(2, dtype=t.int32, device="cuda")
+    nc.fp8_quantize2(dx, rows, cols, q, qT, sc[0:1], scratch[0:1])
+    nc.fp8_quantize(dx, rows, cols, q1, sc[1:2], scratch[1:2], ldq=cols + 8)
+    t.cuda.synchronize()
+    s = host(sc)
+    assert s[0] == s[1] == np.float32(oracle.fp8_scale(x, activation=True))
+    assert np.array_equal(host(q), host(q1)[:, :cols])
+    assert np.array_equal(host(qT), host(q).T)
+    _, q_ref = _fp8_oracle_q(x, activation=True)
+    assert np.array_equal(_e4m3_decode(host(q)), q_ref)
+
+
 @pytest.mark.parametrize("M,N,K,epi", [(512, 768, 640, "f32"), (300, 512, 1000, "f32"),
                                        (640, 1280, 1280, "bf16"), (384, 256, 256, "resid")])
 def test_fp8_gemm_matches_the_oracle(M, N, K, epi):
