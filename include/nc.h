@@ -358,6 +358,11 @@ typedef struct {
    * for A and B (two device floats). */
   int ab_type;
   const float* ab_scale;
+  /* E4M3 operands, batch 1 and a bf16 epilogue (not the RoPE one) only:
+   * when not NULL, max |D| over the bf16 values stored is folded into
+   * *amax_out with an integer atomic max on the float's bits (the caller
+   * zeroes it first), the amax the output's own fp8 quantisation needs. */
+  unsigned* amax_out;
 } nc_gemm_desc;
 nc_status nc_op_gemm(const nc_gemm_desc* desc, void* stream);
 

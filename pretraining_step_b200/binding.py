@@ -47,7 +47,8 @@ class GemmDesc(ctypes.Structure):
                 ("split_k", ctypes.c_int), ("rope_T", ctypes.c_int), ("rope_H", ctypes.c_int),
                 ("rope_tab", ctypes.c_void_p), ("rstd_q", ctypes.c_void_p),
                 ("rstd_k", ctypes.c_void_p), ("rope_Hkv", ctypes.c_int),
-                ("ab_type", ctypes.c_int), ("ab_scale", ctypes.c_void_p)]
+                ("ab_type", ctypes.c_int), ("ab_scale", ctypes.c_void_p),
+                ("amax_out", ctypes.c_void_p)]
 
 
 class ModelConfig(ctypes.Structure):
@@ -323,7 +324,7 @@ class GPT:
 # ------------------------------------------------------------------ ops
 def gemm(M, N, K, A, B, D, *, lda=None, ldb=None, ldd=None, a_kmajor=True, b_kmajor=True,
          batch=1, stride_a=0, stride_b=0, stride_d=0, epi=EPI_STORE_BF16, aux=None, ldaux=0,
-         stride_aux=0, alpha=1.0, beta=0.0, split_k=1, ab_scale=None, stream=None):
+         stride_aux=0, alpha=1.0, beta=0.0, split_k=1, ab_scale=None, amax_out=None, stream=None):
     """D = epi(A B^T) on the tensor cores; ab_scale (a device array of the
     two operands' fp8 scales) selects E4M3 operands (one byte each)."""
     d = GemmDesc()
@@ -339,6 +340,8 @@ def gemm(M, N, K, A, B, D, *, lda=None, ldb=None, ldd=None, a_kmajor=True, b_kma
     d.epi, d.alpha, d.beta, d.split_k = epi, alpha, beta, split_k
     if ab_scale is not None:
         d.ab_type, d.ab_scale = 1, _ptr(ab_scale)
+    if amax_out is not None:
+        d.amax_out = _ptr(amax_out)
     _check(lib().nc_op_gemm(ctypes.byref(d), _stream(stream)))
 
 

@@ -769,14 +769,16 @@ __global__ void __launch_bounds__(256) fp8_quant2_kernel(const __nv_bfloat16* __
 }
 
 nc_status fp8_quantize2(const void* x, int64_t rows, int cols, int64_t ld, uint8_t* q, uint8_t* qT, float* s0,
-                        float* s1, unsigned* amax_scratch, cudaStream_t s, Profiler* prof) {
+                        float* s1, unsigned* amax_scratch, bool amax_ready, cudaStream_t s, Profiler* prof) {
   Probe probe(prof, s, "fp8_quantize", 0.0,
-              (double)rows * cols * (2.0 * 2 + (q ? 1.0 : 0.0) + (qT ? 1.0 : 0.0)));
-  NC_CUDA_TRY(cudaMemsetAsync(amax_scratch, 0, sizeof(unsigned), s));
-  const int64_t units = rows * (cols / 8);
-  const unsigned g = (unsigned)std::min<int64_t>((units + 255) / 256, 8LL * num_sms());
-  fp8_amax_kernel<<<g, 256, 0, s>>>(x, 1, rows, cols, ld, amax_scratch);
-  NC_CUDA_TRY(cudaGetLastError());
+              (double)rows * cols * ((amax_ready ? 1.0 : 2.0) * 2 + (q ? 1.0 : 0.0) + (qT ? 1.0 : 0.0)));
+  if (!amax_ready) {
+    NC_CUDA_TRY(cudaMemsetAsync(amax_scratch, 0, sizeof(unsigned), s));
+    const int64_t units = rows * (cols / 8);
+    const unsigned g = (unsigned)std::min<int64_t>((units + 255) / 256, 8LL * num_sms());
+    fp8_amax_kernel<<<g, 256, 0, s>>>(x, 1, rows, cols, ld, amax_scratch);
+    NC_CUDA_TRY(cudaGetLastError());
+  }
   dim3 grid((unsigned)((cols + 127) / 128), (unsigned)((rows + 63) / 64));
   fp8_quant2_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), rows, cols, ld, amax_scratch, q,
                                          qT, s0, s1);

@@ -71,6 +71,9 @@ struct Args {
       int rope_T;
       int16_t rope_H, rope_Hkv;  // query heads, KV heads
     };
+    // fp8 kernels with one batch and a bf16 output: where max |output| goes
+    // (the bits of a non-negative float, for integer atomicMax), or null.
+    unsigned* amax_out;
   };
   union {
     const void* aux;
@@ -728,7 +731,7 @@ __device__ __forceinline__ void aux_read_slot(const uint8_t* slot, int lane, boo
 // the finished rows go out through the slot that held the aux rows.
 __device__ __forceinline__ void aux_epilogue_chunk(const Args& p, uint8_t* slot, int lane, bool f32,
                                                    int b, int row0, int col0, const uint32_t (&r)[32],
-                                                   bool mirror) {
+                                                   bool mirror, float& amx) {
   float x[32];
   aux_read_slot(slot, lane, f32, x);
   __syncwarp();  // every lane has read its aux row before any is overwritten
@@ -738,6 +741,7 @@ __device__ __forceinline__ void aux_epilogue_chunk(const Args& p, uint8_t* slot,
   for (int j = 0; j < 32; ++j) {
     const float a = __uint_as_float(r[j]) * p.alpha;
     w[j] = f32 ? x[j] + a : (relu2_bwd ? 2.f * sqrt_approx(fmaxf(x[j], 0.f)) * a : a + p.beta * x[j]);
+    amx = fmaxf(amx, fabsf(w[j]));
   }
   stage_store_chunk(p, slot, lane, f32, b, row0, col0, w, mirror);
 }
@@ -934,6 +938,7 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
                             half);
     }
     bool xabort = false;
+    float amx = 0.f;  // max |output| of this thread's values (fp8 kernels' amax_out)
     for (int t = pair; t < total; t += npairs) {
       const TileCoord c = decode(pe, t);
       bool ok = tc::mbar_wait(&tfull[acc], acc_phase, abort_flag, pe.status);
@@ -960,7 +965,7 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
             break;
           }
           if (col0 < pe.N)
-            aux_epilogue_chunk(pe, ring + slot * slot_bytes, lane, xf32, c.b, row - lane, col0, r, mirror);
+            aux_epilogue_chunk(pe, ring + slot * slot_bytes, lane, xf32, c.b, row - lane, col0, r, mirror, amx);
           // Every lane is done with the slot: order its accesses before the
           // TMA refill of the same slot with the chunk `slots` ahead.
           tc::fence_proxy_async_smem();
@@ -987,6 +992,7 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
             for (int j = 0; j < 32; ++j) {
               const float a = __uint_as_float(r[j]) * pe.alpha;
               w[j] = pe.epi == NC_EPI_RELU2 ? fmaxf(a, 0.f) * fmaxf(a, 0.f) : a;
+              amx = fmaxf(amx, fabsf(w[j]));
             }
             stage_store_chunk(pe, ring, lane, f32, c.b, row - lane, col0, w, mirror);
           }
@@ -1028,6 +1034,14 @@ __device__ __forceinline__ void gemm_tc2_body(const CUtensorMap* tmA, const CUte
       // CTA exits (chunks past the last tile were never requested).
       for (int g = g_use; g < g_use + slots; ++g)
         if (pair + (g / CH) * npairs < total) drain_wait(&xfull[g & (slots - 1)], (g >> slot_shift) & 1);
+    }
+    if constexpr (FP8 && !ROPE) {
+      // The output's amax as the bf16 values stored (rounding is monotonic).
+      if (pe.batch == 1 && pe.amax_out && pe.epi != NC_EPI_STORE_F32 && pe.epi != NC_EPI_RESID_F32 &&
+          pe.epi != NC_EPI_ACC_F32) {
+        amx = warp_max(amx);
+        if (lane == 0) atomicMax(pe.amax_out, __float_as_uint(__bfloat162float(__float2bfloat16_rn(amx))));
+      }
     }
       };
     if constexpr (FP8) {
@@ -1184,7 +1198,8 @@ nc_status launch_pair(const nc_gemm_desc& d, int split, int* status, const char*
   }
   a.D = d.D;
   a.ldd = d.ldd;
-  a.stride_d = d.stride_d;
+  a.stride_d = d.batch > 1 ? d.stride_d : 0;
+  if (fp8 && d.amax_out) a.amax_out = d.amax_out;  // batch 1 (checked by the caller)
   a.aux = d.aux;
   a.ldaux = d.ldaux;
   a.stride_aux = d.stride_aux;
@@ -1276,6 +1291,9 @@ nc_status gemm_launch(const GemmLaunch& g, cudaStream_t s, Profiler* prof) {
   auto aligned = [](int64_t v) { return v % 8 == 0; };
   if (d.ab_type != 0 && d.ab_type != 1) return fail(NC_ERR_INVALID_ARG, "gemm: unknown operand type");
   const bool fp8 = d.ab_type == 1;
+  if (d.amax_out && (!fp8 || d.batch != 1 || d.epi == NC_EPI_ROPE_QKNORM || d.epi == NC_EPI_STORE_F32 ||
+                     d.epi == NC_EPI_RESID_F32 || d.epi == NC_EPI_ACC_F32))
+    return fail(NC_ERR_INVALID_ARG, "gemm: amax_out needs E4M3 operands, one batch and a bf16 epilogue");
   if (fp8 && (!d.a_kmajor || !d.b_kmajor || d.lda % 16 || d.ldb % 16 ||
               (d.batch > 1 && (d.stride_a % 16 || d.stride_b % 16)) || !d.ab_scale || d.alpha != 1.f ||
               d.epi == NC_EPI_AXPBY_BF16 || g.symmetric))

@@ -124,9 +124,10 @@ nc_status fp8_quantize(const void* x, bool bf16, int64_t rows, int cols, int64_t
                        Profiler* prof);
 // The same for a bf16 matrix in both layouts at once (q [rows, cols] and qT
 // [cols, rows], either may be null; rows and cols multiples of 8), the
-// scale written to s0 and, when not null, s1.
+// scale written to s0 and, when not null, s1.  amax_ready: *amax_scratch
+// already holds max |x| (its producer folded it in), so x is read once.
 nc_status fp8_quantize2(const void* x, int64_t rows, int cols, int64_t ld, uint8_t* q, uint8_t* qT, float* s0,
-                        float* s1, unsigned* amax_scratch, cudaStream_t s, Profiler* prof);
+                        float* s1, unsigned* amax_scratch, bool amax_ready, cudaStream_t s, Profiler* prof);
 // y[i] = 2^x[i] by exp2_fma2 (exp2_poly.cuh), the softmax's FMA-pipe exponential.
 nc_status exp2_poly(const float* x, float* y, int64_t n, cudaStream_t s);
 // Momentum and per-matrix squared norms over the 6*L block matrices; dkv is

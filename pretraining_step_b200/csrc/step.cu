@@ -272,7 +272,7 @@ nc_status ensure_acts(nc_params* p, int B, int T) {
   const int64_t wmax = std::max(F, Q) * d;                   // largest weight, elements
   if (p->fp8)  // E4M3 operands: saved activations, the propagated gradient, a weight, scales
     total += L * (6 * r(N * d) + 2 * r(N * F)) + 2 * r(N * std::max(F, Q)) + r(wmax) +
-             r(4 * L * F8_COUNT * 2) + r(4);
+             r(4 * L * F8_COUNT * 2) + r(8);
   void* mem = nullptr;
   cudaError_t e = cudaMalloc(&mem, (size_t)total);
   if (e != cudaSuccess) {
@@ -322,7 +322,7 @@ nc_status ensure_acts(nc_params* p, int B, int T) {
     a.q8gT = ar.take<uint8_t>(N * std::max(F, Q));
     a.q8w = ar.take<uint8_t>(wmax);
     a.f8sc = ar.take<float>((int64_t)L * F8_COUNT * 2);
-    a.f8scratch = ar.take<unsigned>(1);
+    a.f8scratch = ar.take<unsigned>(2);  // [0] amax computed by the quantiser, [1] by a GEMM epilogue
   }
   if (ar.used > ar.size) return fail(NC_ERR_CUDA, "activation arena overflow");
   return NC_OK;
@@ -342,9 +342,12 @@ const float* master_of(const nc_params* p, const bf16* Wb) { return p->blocks + 
 
 // fp8 mode: an activation or gradient (bf16 [rows, cols], row stride ld) to
 // E4M3 in both layouts (either may be null), its scale to s0 (and s1).
+// amax: the word where the tensor's producer folded in max |x| (zeroed
+// before it ran), or null to compute it here.
 nc_status quant8(nc_params* p, const bf16* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* q,
-                 uint8_t* qT, float* s0, float* s1) {
-  return fp8_quantize2(x, rows, (int)cols, ld, q, qT, s0, s1, p->act.f8scratch, p->stream, p->prof);
+                 uint8_t* qT, float* s0, float* s1, unsigned* amax = nullptr) {
+  return fp8_quantize2(x, rows, (int)cols, ld, q, qT, s0, s1, amax ? amax : p->act.f8scratch, amax != nullptr,
+                       p->stream, p->prof);
 }
 
 // fp8 mode: the fp32 master of a block matrix ([rows, cols]) to E4M3 in
@@ -358,7 +361,7 @@ nc_status quant8w(nc_params* p, const bf16* Wb, int64_t rows, int64_t cols, bool
 // operands K-major; weight gradients (NC_EPI_ACC_F32) split K automatically.
 nc_status gemm8(nc_params* p, int64_t M, int64_t N, int64_t K, const uint8_t* A8, int64_t lda,
                 const uint8_t* B8, int64_t ldb, void* D, int64_t ldd, nc_epilogue epi, const void* aux,
-                int64_t ldaux, const float* sc, const char* tag) {
+                int64_t ldaux, const float* sc, const char* tag, unsigned* amax_out = nullptr) {
   GemmLaunch g{};
   g.status = p->status;
   g.tag = tag;
@@ -370,6 +373,8 @@ nc_status gemm8(nc_params* p, int64_t M, int64_t N, int64_t K, const uint8_t* A8
   g.d.epi = epi; g.d.alpha = 1.f; g.d.split_k = epi == NC_EPI_ACC_F32 ? 0 : 1;
   g.d.ab_type = 1;
   g.d.ab_scale = sc;
+  g.d.amax_out = amax_out;
+  if (amax_out) NC_CUDA_TRY(cudaMemsetAsync(amax_out, 0, sizeof(unsigned), p->stream));
   return gemm_launch(g, p->stream, p->prof);
 }
 
@@ -441,8 +446,8 @@ nc_status layer_bwd_fp8(nc_params* p, int l, int B, int T, const bf16* W, float*
                "gemm_wgrad"));
   NC_TRY(quant8w(p, W + o_down, d, F, true, sc + 2 * F8_DOWN_D + 1));
   NC_TRY(gemm8(p, N, F, d, a.q8g, d, a.q8w, d, a.du, F, NC_EPI_RELU2_BWD, a.a[l], F, sc + 2 * F8_DOWN_D,
-               "gemm_dgrad"));
-  NC_TRY(quant8(p, a.du, N, F, F, a.q8g, a.q8gT, sc + 2 * F8_UP_D, sc + 2 * F8_UP_W));
+               "gemm_dgrad", a.f8scratch + 1));
+  NC_TRY(quant8(p, a.du, N, F, F, a.q8g, a.q8gT, sc + 2 * F8_UP_D, sc + 2 * F8_UP_W, a.f8scratch + 1));
   NC_TRY(gemm8(p, F, d, N, a.q8gT, N, q[5], N, G + o_up, d, NC_EPI_ACC_F32, nullptr, 0, sc + 2 * F8_UP_W,
                "gemm_wgrad"));
   NC_TRY(quant8w(p, W + o_up, F, d, true, sc + 2 * F8_UP_D + 1));
@@ -543,8 +548,9 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
       NC_TRY(quant8(p, a.h2[l], N, d, d, q[4], q[5], sc + 2 * F8_UP_F, sc + 2 * F8_UP_W + 1));
       NC_TRY(quant8w(p, W + o_up, F, d, false, sc + 2 * F8_UP_F + 1));
       NC_TRY(gemm8(p, N, F, d, q[4], d, a.q8w, d, a.a[l], F, NC_EPI_RELU2, nullptr, 0, sc + 2 * F8_UP_F,
-                   "gemm_fwd"));
-      NC_TRY(quant8(p, a.a[l], N, F, F, q[6], q[7], sc + 2 * F8_DOWN_F, sc + 2 * F8_DOWN_W + 1));
+                   "gemm_fwd", a.f8scratch + 1));
+      NC_TRY(quant8(p, a.a[l], N, F, F, q[6], q[7], sc + 2 * F8_DOWN_F, sc + 2 * F8_DOWN_W + 1,
+                    a.f8scratch + 1));
       NC_TRY(quant8w(p, W + o_down, d, F, false, sc + 2 * F8_DOWN_F + 1));
       NC_TRY(gemm8(p, N, d, F, q[6], F, a.q8w, F, a.x[l + 1], d, NC_EPI_RESID_F32, a.xmid[l], d,
                    sc + 2 * F8_DOWN_F, "gemm_fwd"));
@@ -1150,7 +1156,7 @@ nc_status nc_op_fp8_quantize2(const void* x_bf16, int64_t rows, int cols, int64_
   if ((reinterpret_cast<uintptr_t>(x_bf16) | reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(qT)) & 15)
     return fail(NC_ERR_INVALID_ARG, "fp8_quantize2: x, q and qT must be 16-byte aligned");
   return fp8_quantize2(x_bf16, rows, cols, ldx, static_cast<uint8_t*>(q), static_cast<uint8_t*>(qT), scale,
-                       nullptr, static_cast<unsigned*>(scratch), static_cast<cudaStream_t>(stream), nullptr);
+                       nullptr, static_cast<unsigned*>(scratch), false, static_cast<cudaStream_t>(stream), nullptr);
 }
 
 nc_status nc_op_exp2_poly(const float* x, float* y, int64_t n, void* stream) {

@@ -364,6 +364,29 @@ def test_fp8_gemm_weight_gradient_form():
     assert rel_fro(host(D), ref) < 1e-5
 
 
+@pytest.mark.parametrize("epi", ["relu2", "relu2_bwd"])
+def test_fp8_gemm_amax_out_is_the_outputs_max(epi):
+    """amax_out receives max |D| over the bf16 values the epilogue stored."""
+    t = torch()
+    M, N, K = 384, 512, 256
+    x = inputs.bf16_normal(31, (M, K))
+    w = inputs.bf16_normal(32, (N, K)) * K ** -0.5
+    qx = t.zeros((M, K), dtype=t.uint8, device="cuda")
+    qw = t.zeros((N, K), dtype=t.uint8, device="cuda")
+    sc = t.zeros(2, dtype=t.float32, device="cuda")
+    scratch = t.zeros(2, dtype=t.int32, device="cuda")
+    nc.fp8_quantize(dev_bf16(x), M, K, qx, sc[0:1], scratch[0:1])
+    nc.fp8_quantize(dev_f32(w), N, K, qw, sc[1:2], scratch[1:2])
+    D = t.zeros(M, N, dtype=t.bfloat16, device="cuda")
+    amax = t.zeros(1, dtype=t.int32, device="cuda")
+    aux = dev_bf16(np.abs(inputs.bf16_normal(33, (M, N)))) if epi == "relu2_bwd" else None
+    nc.gemm(M, N, K, qx, qw, D, epi=nc.EPI_RELU2 if epi == "relu2" else nc.EPI_RELU2_BWD, aux=aux,
+            ab_scale=sc, amax_out=amax)
+    t.cuda.synchronize()
+    got = amax.cpu().numpy().view(np.float32)[0]
+    assert got == np.abs(host(D)).max() > 0
+
+
 def test_fp8_gemm_rejects_unsupported_forms():
     t = torch()
     q = t.zeros((512, 512), dtype=t.uint8, device="cuda")
