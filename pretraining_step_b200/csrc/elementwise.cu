@@ -50,12 +50,31 @@ __global__ void embed_scatter_kernel(const int32_t* __restrict__ tok, int64_t n,
 }
 
 // ------------------------------------------------------------------ RMSNorm
+// max |v| of a block's values (one per thread) into *amax as bf16 bits of a
+// non-negative float (the output's rounding is monotonic, so this is the max
+// of the stored bf16 values); one atomic per block.
+__device__ __forceinline__ void block_amax_bf16(float v, unsigned* amax) {
+  __shared__ float red[32];
+  v = warp_max(v);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int i = 1; i < (int)(blockDim.x >> 5); ++i) v = fmaxf(v, red[i]);
+    atomicMax(amax, __float_as_uint(__bfloat162float(__float2bfloat16_rn(v))));
+  }
+}
+
 // y = x / sqrt(mean(x^2) + eps) as bf16, rstd saved; one warp per row.
+// amax (fp8 mode): max |y| folded in, for the quantisation of y.
 __global__ void rmsnorm_fwd_kernel(const float* __restrict__ x, int64_t rows, int d,
-                                   __nv_bfloat16* __restrict__ y, float* __restrict__ rstd) {
+                                   __nv_bfloat16* __restrict__ y, float* __restrict__ rstd,
+                                   unsigned* amax) {
   const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (r >= rows) return;
+  if (r >= rows) {
+    if (amax) block_amax_bf16(0.f, amax);
+    return;
+  }
   const float4* xr = reinterpret_cast<const float4*>(x + r * d);
   float ss = 0.f;
   for (int i = lane; i < d / 4; i += 32) {
@@ -65,14 +84,17 @@ __global__ void rmsnorm_fwd_kernel(const float* __restrict__ x, int64_t rows, in
   ss = warp_sum(ss);
   const float rs = rsqrtf(ss / d + kNormEps);
   uint2* yr = reinterpret_cast<uint2*>(y + r * d);
+  float am = 0.f;
   for (int i = lane; i < d / 4; i += 32) {
     const float4 v = xr[i];
     uint2 u;
     u.x = pack_bf16x2(v.x * rs, v.y * rs);
     u.y = pack_bf16x2(v.z * rs, v.w * rs);
     yr[i] = u;
+    if (amax) am = fmaxf(am, fmaxf(fmaxf(fabsf(v.x * rs), fabsf(v.y * rs)), fmaxf(fabsf(v.z * rs), fabsf(v.w * rs))));
   }
   if (lane == 0 && rstd) rstd[r] = rs;
+  if (amax) block_amax_bf16(am, amax);
 }
 
 // dx = dres + r * (dh - y * mean(dh * y)) with y = x * r the norm's output,
@@ -82,10 +104,13 @@ __global__ void rmsnorm_fwd_kernel(const float* __restrict__ x, int64_t rows, in
 __global__ void __launch_bounds__(256) rmsnorm_bwd_kernel(
     const __nv_bfloat16* __restrict__ dh, const __nv_bfloat16* __restrict__ y,
     const float* __restrict__ rstd, const float* __restrict__ dres, int64_t rows, int d,
-    float* __restrict__ dx, __nv_bfloat16* __restrict__ dx_bf16) {
+    float* __restrict__ dx, __nv_bfloat16* __restrict__ dx_bf16, unsigned* amax) {
   const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (r >= rows) return;
+  if (r >= rows) {
+    if (amax) block_amax_bf16(0.f, amax);
+    return;
+  }
   const int n4 = d / 4;
   const uint2* gr = reinterpret_cast<const uint2*>(dh + r * d);
   const uint2* yr = reinterpret_cast<const uint2*>(y + r * d);
@@ -101,6 +126,7 @@ __global__ void __launch_bounds__(256) rmsnorm_bwd_kernel(
   const float4* rr = dres ? reinterpret_cast<const float4*>(dres + r * d) : nullptr;
   float4* o = reinterpret_cast<float4*>(dx + r * d);
   uint2* ob = dx_bf16 ? reinterpret_cast<uint2*>(dx_bf16 + r * d) : nullptr;
+  float am = 0.f;
   for (int i = lane; i < n4; i += 32) {
     const uint2 g = gr[i], v = yr[i];
     const float2 g0 = unpack_bf16x2(g.x), g1 = unpack_bf16x2(g.y);
@@ -112,7 +138,9 @@ __global__ void __launch_bounds__(256) rmsnorm_bwd_kernel(
     res.w += rs * (g1.y - y1.y * m);
     o[i] = res;
     if (ob) ob[i] = make_uint2(pack_bf16x2(res.x, res.y), pack_bf16x2(res.z, res.w));
+    if (amax) am = fmaxf(am, fmaxf(fmaxf(fabsf(res.x), fabsf(res.y)), fmaxf(fabsf(res.z), fabsf(res.w))));
   }
+  if (amax) block_amax_bf16(am, amax);
 }
 
 // ------------------------------------------------------------------ RoPE + QK-norm
@@ -515,24 +543,25 @@ nc_status embed_scatter(const int32_t* tok, int64_t n, const float* dx, int V, i
 }
 
 nc_status rmsnorm_fwd(const float* x, int64_t rows, int d, void* y, float* rstd, cudaStream_t s,
-                      Profiler* prof) {
+                      Profiler* prof, unsigned* amax) {
   if (d % 4) return fail(NC_ERR_INVALID_ARG, "rmsnorm: width must be a multiple of 4");
   Probe probe(prof, s, "rmsnorm_fwd", 0.0, rows * (6.0 * d + 4.0));
   rmsnorm_fwd_kernel<<<blocks_for(rows * 32, 256), 256, 0, s>>>(x, rows, d, (__nv_bfloat16*)y,
-                                                                 rstd);
+                                                                 rstd, amax);
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }
 
 nc_status rmsnorm_bwd(const void* dh, const void* y, const float* rstd, const float* dres,
                       int64_t rows, int d, float* dx, void* dx_bf16, cudaStream_t s,
-                      Profiler* prof) {
+                      Profiler* prof, unsigned* amax) {
   if (d % 4) return fail(NC_ERR_UNSUPPORTED, "rmsnorm_bwd: width must be a multiple of 4");
+  if (amax && !dx_bf16) return fail(NC_ERR_INVALID_ARG, "rmsnorm_bwd: amax is of the bf16 copy");
   Probe probe(prof, s, "rmsnorm_bwd", 0.0,
               rows * ((2.0 + 2.0 + (dres ? 4.0 : 0.0) + 4.0 + (dx_bf16 ? 2.0 : 0.0)) * d + 4.0));
   rmsnorm_bwd_kernel<<<blocks_for(rows * 32, 256), 256, 0, s>>>(
       (const __nv_bfloat16*)dh, (const __nv_bfloat16*)y, rstd, dres, rows, d, dx,
-      (__nv_bfloat16*)dx_bf16);
+      (__nv_bfloat16*)dx_bf16, amax);
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;
 }

@@ -99,12 +99,13 @@ nc_status embed_gather(const int32_t* tok, int64_t n, const float* E, int V, int
                        int* status, cudaStream_t s, Profiler* prof);
 nc_status embed_scatter(const int32_t* tok, int64_t n, const float* dx, int V, int d, float* dE,
                         cudaStream_t s, Profiler* prof);
+// amax (fp8 mode; zeroed by the caller): max |y| of the bf16 output folded in.
 nc_status rmsnorm_fwd(const float* x, int64_t rows, int d, void* y, float* rstd, cudaStream_t s,
-                      Profiler* prof);
+                      Profiler* prof, unsigned* amax = nullptr);
 // y: the norm's saved bf16 output (x * rstd as the forward stored it).
 nc_status rmsnorm_bwd(const void* dh, const void* y, const float* rstd, const float* dres,
                       int64_t rows, int d, float* dx, void* dx_bf16, cudaStream_t s,
-                      Profiler* prof);
+                      Profiler* prof, unsigned* amax = nullptr);
 // RoPE cos/sin for positions [0, T): tab[pos * hd/2 + i] = (cos, sin) of
 // pos * 10000^(-2i/hd); then, from tab + T * hd/2, the same values grouped
 // for 32-byte loads of four consecutive pairs of one position:

@@ -357,6 +357,16 @@ nc_status quant8w(nc_params* p, const bf16* Wb, int64_t rows, int64_t cols, bool
                       transpose ? rows : cols, s, p->act.f8scratch, p->stream, p->prof);
 }
 
+// fp8 mode: the word (zeroed here) a norm or GEMM epilogue folds its bf16
+// output's amax into, for that output's quantisation; null in bf16 mode.
+nc_status amax_word(nc_params* p, unsigned** w) {
+  *w = nullptr;
+  if (!p->fp8) return NC_OK;
+  *w = p->act.f8scratch + 1;
+  NC_CUDA_TRY(cudaMemsetAsync(*w, 0, sizeof(unsigned), p->stream));
+  return NC_OK;
+}
+
 // One E4M3 GEMM: D[M, N] = epi(A8[M, K] B8[N, K]^T / (sc[0] sc[1])), both
 // operands K-major; weight gradients (NC_EPI_ACC_F32) split K automatically.
 nc_status gemm8(nc_params* p, int64_t M, int64_t N, int64_t K, const uint8_t* A8, int64_t lda,
@@ -440,8 +450,8 @@ nc_status layer_bwd_fp8(nc_params* p, int l, int B, int T, const bf16* W, float*
   const int64_t o_wo = mat_offset(p, 3), o_up = mat_offset(p, 4), o_down = mat_offset(p, 5);
   float* sc = a.f8sc + ((int64_t)l * F8_COUNT) * 2;
   auto& q = a.q8f[l];
-  // MLP: x_out = xmid + a wdown^T, a = relu(h2 wup^T)^2
-  NC_TRY(quant8(p, a.dxb, N, d, d, a.q8g, a.q8gT, sc + 2 * F8_DOWN_D, sc + 2 * F8_DOWN_W));
+  // MLP: x_out = xmid + a wdown^T, a = relu(h2 wup^T)^2 (dxb's amax from the norm that wrote it)
+  NC_TRY(quant8(p, a.dxb, N, d, d, a.q8g, a.q8gT, sc + 2 * F8_DOWN_D, sc + 2 * F8_DOWN_W, a.f8scratch + 1));
   NC_TRY(gemm8(p, d, F, N, a.q8gT, N, q[7], N, G + o_down, F, NC_EPI_ACC_F32, nullptr, 0, sc + 2 * F8_DOWN_W,
                "gemm_wgrad"));
   NC_TRY(quant8w(p, W + o_down, d, F, true, sc + 2 * F8_DOWN_D + 1));
@@ -453,10 +463,12 @@ nc_status layer_bwd_fp8(nc_params* p, int l, int B, int T, const bf16* W, float*
   NC_TRY(quant8w(p, W + o_up, F, d, true, sc + 2 * F8_UP_D + 1));
   NC_TRY(gemm8(p, N, d, F, a.q8g, F, a.q8w, F, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0, sc + 2 * F8_UP_D,
                "gemm_dgrad"));
-  NC_TRY(rmsnorm_bwd(a.dh, a.h2[l], a.r2[l], dx, N, (int)d, dxn, a.dxb, s, pr));
+  unsigned* am = nullptr;
+  NC_TRY(amax_word(p, &am));
+  NC_TRY(rmsnorm_bwd(a.dh, a.h2[l], a.r2[l], dx, N, (int)d, dxn, a.dxb, s, pr, am));
   std::swap(dx, dxn);
   // Attention: xmid = x + o wo^T
-  NC_TRY(quant8(p, a.dxb, N, d, d, a.q8g, a.q8gT, sc + 2 * F8_O_D, sc + 2 * F8_O_W));
+  NC_TRY(quant8(p, a.dxb, N, d, d, a.q8g, a.q8gT, sc + 2 * F8_O_D, sc + 2 * F8_O_W, am));
   NC_TRY(gemm8(p, d, d, N, a.q8gT, N, q[3], N, G + o_wo, d, NC_EPI_ACC_F32, nullptr, 0, sc + 2 * F8_O_W,
                "gemm_wgrad"));
   NC_TRY(quant8w(p, W + o_wo, d, d, true, sc + 2 * F8_O_D + 1));
@@ -471,8 +483,10 @@ nc_status layer_bwd_fp8(nc_params* p, int l, int B, int T, const bf16* W, float*
   NC_TRY(quant8w(p, W, Q, d, true, sc + 2 * F8_QKV_D + 1));
   NC_TRY(gemm8(p, N, d, Q, a.q8g, Q, a.q8w, Q, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0, sc + 2 * F8_QKV_D,
                "gemm_dgrad"));
-  // Back into the caller's dx (dxn here, after the swap above).
-  NC_TRY(rmsnorm_bwd(a.dh, a.h1[l], a.r1[l], dx, N, (int)d, dxn, a.dxb, s, pr));
+  // Back into the caller's dx (dxn here, after the swap above); its amax
+  // for the next layer's first quantisation.
+  NC_TRY(amax_word(p, &am));
+  NC_TRY(rmsnorm_bwd(a.dh, a.h1[l], a.r1[l], dx, N, (int)d, dxn, a.dxb, s, pr, am));
   return NC_OK;
 }
 
@@ -511,7 +525,9 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
   NC_TRY(embed_gather(tok, N, p->wte, V, (int)d, a.x[0], p->status, s, pr));
   for (int l = 0; l < L; ++l) {
     const bf16* W = p->blocks_b + l * LS;
-    NC_TRY(rmsnorm_fwd(a.x[l], N, (int)d, a.h1[l], a.r1[l], s, pr));
+    unsigned* am = nullptr;
+    NC_TRY(amax_word(p, &am));
+    NC_TRY(rmsnorm_fwd(a.x[l], N, (int)d, a.h1[l], a.r1[l], s, pr, am));
     {
       // q|k|v projection with RoPE + QK-norm fused into the epilogue.
       GemmLaunch g{};
@@ -526,7 +542,8 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
       g.d.rstd_q = a.rq[l]; g.d.rstd_k = a.rk[l];
       if (p->fp8) {  // h1 in both layouts (the transpose for the weight gradient); wq|wk|wv as one tensor
         float* sc = a.f8sc + ((int64_t)l * F8_COUNT) * 2;
-        NC_TRY(quant8(p, a.h1[l], N, d, d, a.q8f[l][0], a.q8f[l][1], sc + 2 * F8_QKV_F, sc + 2 * F8_QKV_W + 1));
+        NC_TRY(quant8(p, a.h1[l], N, d, d, a.q8f[l][0], a.q8f[l][1], sc + 2 * F8_QKV_F, sc + 2 * F8_QKV_W + 1,
+                      am));
         NC_TRY(quant8w(p, W, Q, d, false, sc + 2 * F8_QKV_F + 1));
         g.d.A = a.q8f[l][0]; g.d.lda = d;
         g.d.B = a.q8w; g.d.ldb = d;
@@ -544,8 +561,9 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
       NC_TRY(quant8w(p, W + o_wo, d, d, false, sc + 2 * F8_O_F + 1));
       NC_TRY(gemm8(p, N, d, d, q[2], d, a.q8w, d, a.xmid[l], d, NC_EPI_RESID_F32, a.x[l], d,
                    sc + 2 * F8_O_F, "gemm_fwd"));
-      NC_TRY(rmsnorm_fwd(a.xmid[l], N, (int)d, a.h2[l], a.r2[l], s, pr));
-      NC_TRY(quant8(p, a.h2[l], N, d, d, q[4], q[5], sc + 2 * F8_UP_F, sc + 2 * F8_UP_W + 1));
+      NC_TRY(amax_word(p, &am));
+      NC_TRY(rmsnorm_fwd(a.xmid[l], N, (int)d, a.h2[l], a.r2[l], s, pr, am));
+      NC_TRY(quant8(p, a.h2[l], N, d, d, q[4], q[5], sc + 2 * F8_UP_F, sc + 2 * F8_UP_W + 1, am));
       NC_TRY(quant8w(p, W + o_up, F, d, false, sc + 2 * F8_UP_F + 1));
       NC_TRY(gemm8(p, N, F, d, q[4], d, a.q8w, d, a.a[l], F, NC_EPI_RELU2, nullptr, 0, sc + 2 * F8_UP_F,
                    "gemm_fwd", a.f8scratch + 1));
@@ -573,7 +591,11 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
                  "gemm_lmhead"));
   float* dx = a.dx0;
   float* dxn = a.dx1;
-  NC_TRY(rmsnorm_bwd(a.dh, a.hf, a.rf, nullptr, N, (int)d, dx, a.dxb, s, pr));
+  {
+    unsigned* am = nullptr;  // fp8: dxb's amax for the last layer's first quantisation
+    NC_TRY(amax_word(p, &am));
+    NC_TRY(rmsnorm_bwd(a.dh, a.hf, a.rf, nullptr, N, (int)d, dx, a.dxb, s, pr, am));
+  }
   for (int l = L - 1; l >= 0; --l) {
     const bf16* W = p->blocks_b + l * LS;
     float* G = g->blocks + l * LS;
