@@ -66,13 +66,18 @@ def step_flops_per_token(depth, seq, vocab, n_kv_head=0, windows=None):
     return 6.0 * n_mm + attn
 
 
-def gemm_algorithmic_bytes_by_class(depth=DEPTH, batch=B, seq=T, vocab=V):
+LM_CHUNK = 32768  # tokens per lm_head + cross-entropy chunk (the library's default)
+
+
+def gemm_algorithmic_bytes_by_class(depth=DEPTH, batch=B, seq=T, vocab=V, lm_chunk=LM_CHUNK):
     """Operand and result bytes of every GEMM launch of one step, each operand
     read once and each result written once (bf16 2 B, fp32 4 B; a split-K
     weight gradient counts as one fp32 write), summed per launch class:
-    fwd, dgrad, wgrad (the block projections), lmhead, ns (Newton-Schulz).
-    Returns ({class: bytes}, {class: launches})."""
+    fwd, dgrad, wgrad (the block projections), lmhead (three GEMMs per chunk
+    of lm_chunk tokens, each reading or accumulating W_lm once per chunk),
+    ns (Newton-Schulz).  Returns ({class: bytes}, {class: launches})."""
     d, f, n = 64 * depth, 4 * 64 * depth, batch * seq
+    chunks = -(-n // lm_chunk)
     bf, f4 = 2, 4
     fwd = [
         n * d * bf + 3 * d * d * bf + n * 3 * d * bf,          # q|k|v (+ RoPE / QK-norm)
@@ -92,9 +97,9 @@ def gemm_algorithmic_bytes_by_class(depth=DEPTH, batch=B, seq=T, vocab=V):
         2 * n * d * bf + d * d * f4,                           # dW_o
         n * 3 * d * bf + n * d * bf + 3 * d * d * f4,          # dW_qkv
     ]
-    lm = [n * d * bf + vocab * d * bf + n * vocab * bf,       # logits
-          n * vocab * bf + vocab * d * bf + n * d * bf,       # dh = dz W
-          n * vocab * bf + n * d * bf + vocab * d * f4]       # dW = dz^T h
+    lm = [n * d * bf + chunks * vocab * d * bf + n * vocab * bf,       # logits
+          n * vocab * bf + chunks * vocab * d * bf + n * d * bf,       # dh = dz W
+          n * vocab * bf + n * d * bf + chunks * vocab * d * f4]       # dW += dz^T h
     sq, wide = 4 * depth, 2 * depth                           # Newton-Schulz stacks
     ns = 0
     for cnt, m, k in ((sq, d, d), (wide, d, f)):
@@ -102,7 +107,7 @@ def gemm_algorithmic_bytes_by_class(depth=DEPTH, batch=B, seq=T, vocab=V):
         ns += 5 * ((x + a) + (a + a) + (a + x + x))         # A = X X^T; B = cA^2 + bA; Y = BX + aX
     nbytes = {"fwd": float(depth * sum(fwd)), "dgrad": float(depth * sum(dgrad)),
               "wgrad": float(depth * sum(wgrad)), "lmhead": float(sum(lm)), "ns": float(ns)}
-    launches = {"fwd": 4 * depth, "dgrad": 4 * depth, "wgrad": 4 * depth, "lmhead": 3, "ns": 30}
+    launches = {"fwd": 4 * depth, "dgrad": 4 * depth, "wgrad": 4 * depth, "lmhead": 3 * chunks, "ns": 30}
     return nbytes, launches
 
 

@@ -119,6 +119,16 @@ typedef struct {
    * Needs d >= 256 (NC_ERR_UNSUPPORTED) and B*T > 128, a multiple of 16
    * (NC_ERR_INVALID_ARG from the step). */
   int fp8;
+  /* The untied lm_head (guide, section "1. Modelo GPT") and the softmax
+   * cross-entropy in chunks of this many tokens: each chunk's logits are
+   * computed, turned into their loss rows and, in place, their gradient,
+   * and consumed by the lm_head weight and input gradients before the next
+   * chunk, so only chunk x vocab bf16 logits are held.  0: 32768 tokens (a
+   * 2 GB logits buffer at vocab 32768; at depth 20, B = 32, T = 2048 it ran
+   * about 1 ms faster per step than one 65536-token chunk).  Results do not
+   * depend on it beyond fp32 summation order in the lm_head weight
+   * gradient. */
+  int lm_chunk_tokens;
 } nc_model_config;
 nc_status nc_gpt_init_config(const nc_model_config* cfg, nc_params** out);
 void nc_params_free(nc_params* p);

@@ -54,7 +54,8 @@ class GemmDesc(ctypes.Structure):
 class ModelConfig(ctypes.Structure):
     _fields_ = [("depth", ctypes.c_int), ("vocab", ctypes.c_int), ("seed", ctypes.c_uint64),
                 ("flags", ctypes.c_int), ("n_kv_head", ctypes.c_int),
-                ("window", ctypes.c_void_p), ("fp8", ctypes.c_int)]
+                ("window", ctypes.c_void_p), ("fp8", ctypes.c_int),
+                ("lm_chunk_tokens", ctypes.c_int)]
 
 
 class KernelStat(ctypes.Structure):
@@ -177,11 +178,12 @@ class GPT:
     per layer (negative: full causal)."""
 
     def __init__(self, depth, vocab=32768, seed=0, all_random=False, stream=None, n_kv_head=0,
-                 window=None, fp8=False):
+                 window=None, fp8=False, lm_chunk_tokens=0):
         h = vp()
         cfg = ModelConfig(depth=depth, vocab=vocab, seed=seed,
                           flags=NC_INIT_ALL_RANDOM if all_random else NC_INIT_SPEC,
-                          n_kv_head=n_kv_head, window=None, fp8=int(bool(fp8)))
+                          n_kv_head=n_kv_head, window=None, fp8=int(bool(fp8)),
+                          lm_chunk_tokens=int(lm_chunk_tokens))
         win = None
         if window is not None:
             if len(window) != depth:

@@ -572,17 +572,18 @@ nc_status rope_table(float2* tab, int T, int hd, cudaStream_t s) {
   return NC_OK;
 }
 
-nc_status ce_fwd_bwd(void* z, const int32_t* tgt, int64_t n, int V, float* loss_rows,
-                     float* loss_out, int* status, cudaStream_t s, Profiler* prof) {
+nc_status ce_fwd_bwd(void* z, const int32_t* tgt, int64_t n, int V, float inv_n, float* loss_rows,
+                     int* status, cudaStream_t s, Profiler* prof) {
   if (V % 8 || V > kCeThreads * kCeChunks * 8)
     return fail(NC_ERR_UNSUPPORTED, "cross-entropy: vocab must be a multiple of 8 and <= 32768");
   if (n >= (1ll << 31)) return fail(NC_ERR_INVALID_ARG, "cross-entropy: too many rows");
-  {
-    Probe probe(prof, s, "ce_fwd_bwd", 0.0, n * (4.0 * V + 8.0));
-    ce_fwd_bwd_kernel<<<(unsigned)n, kCeThreads, 0, s>>>((__nv_bfloat16*)z, tgt, V,
-                                                          1.0f / (float)n, loss_rows, status);
-    NC_CUDA_TRY(cudaGetLastError());
-  }
+  Probe probe(prof, s, "ce_fwd_bwd", 0.0, n * (4.0 * V + 8.0));
+  ce_fwd_bwd_kernel<<<(unsigned)n, kCeThreads, 0, s>>>((__nv_bfloat16*)z, tgt, V, inv_n, loss_rows, status);
+  NC_CUDA_TRY(cudaGetLastError());
+  return NC_OK;
+}
+
+nc_status loss_mean(const float* loss_rows, int64_t n, float* loss_out, cudaStream_t s) {
   mean_kernel<<<1, 256, 0, s>>>(loss_rows, n, loss_out);
   NC_CUDA_TRY(cudaGetLastError());
   return NC_OK;

@@ -111,8 +111,13 @@ nc_status rmsnorm_bwd(const void* dh, const void* y, const float* rstd, const fl
 // for 32-byte loads of four consecutive pairs of one position:
 // [(i / 4) * T + pos] * 4 + i % 4.  tab holds T * hd floats (two float2 per pair).
 nc_status rope_table(float2* tab, int T, int hd, cudaStream_t s);
-nc_status ce_fwd_bwd(void* z, const int32_t* tgt, int64_t n, int V, float* loss_rows,
-                     float* loss_out, int* status, cudaStream_t s, Profiler* prof);
+// Softmax cross-entropy of n rows of bf16 logits z [n, V]: loss_rows[i] =
+// lse(z_i) - z_i[tgt_i]; z is overwritten by its gradient (softmax - onehot)
+// * inv_n (inv_n: 1 / the rows of the whole batch when z is one chunk of it).
+nc_status ce_fwd_bwd(void* z, const int32_t* tgt, int64_t n, int V, float inv_n, float* loss_rows,
+                     int* status, cudaStream_t s, Profiler* prof);
+// *loss_out = mean of loss_rows[0, n).
+nc_status loss_mean(const float* loss_rows, int64_t n, float* loss_out, cudaStream_t s);
 nc_status init_normal(float* out, int64_t n, uint64_t key, float stdv, cudaStream_t s);
 nc_status f32_to_bf16(const float* in, void* out, int64_t n, cudaStream_t s, Profiler* prof);
 // E4M3 quantisation of a rows x cols matrix (bf16, or fp32 when !bf16; row

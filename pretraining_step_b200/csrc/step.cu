@@ -115,6 +115,7 @@ struct nc_params {
   int depth = 0, vocab = 0, d = 0, H = 0, hd = 0, F = 0;
   int Hkv = 0, dkv = 0;     // KV heads and the width of k, v (dkv = 128 Hkv)
   bool fp8 = false;         // block projections on E4M3 operands
+  int64_t lm_chunk = 32768;  // tokens per lm_head + cross-entropy chunk
   std::vector<int> window;  // per layer: causal left window, -1 = full causal
   cudaStream_t stream = nullptr;
   nc::Profiler* prof = nullptr;
@@ -264,7 +265,8 @@ nc_status ensure_acts(nc_params* p, int B, int T) {
   total += 2 * L * r(4 * N) + L * r(4 * N * H) + L * r(4 * N * Hkv);  // r1 r2 rq rk
   total += L * r(4 * N * H);                                 // lse [B,H,T]
   total += 2 * L * r(2 * N * d) + L * r(2 * N * Q) + L * r(2 * N * d) + L * r(2 * N * F);
-  total += r(2 * N * d) + r(4 * N) + r(2 * N * V) + r(4 * N) + r(4);  // hf rf logits loss
+  const int64_t NC = std::min<int64_t>(p->lm_chunk, N);  // logits rows held
+  total += r(2 * N * d) + r(4 * N) + r(2 * NC * V) + r(4 * N) + r(4);  // hf rf logits loss
   const int64_t ld_ds = (T + 7) & ~int64_t(7);
   total += 2 * r(4 * N * d) + 2 * r(2 * N * d) + r(2 * N * F) + r(2 * N * Q) +
            r(4 * N * H);                                     // backward scratch
@@ -302,7 +304,7 @@ nc_status ensure_acts(nc_params* p, int B, int T) {
   }
   a.hf = ar.take<bf16>(N * d);
   a.rf = ar.take<float>(N);
-  a.logits = ar.take<bf16>(N * V);
+  a.logits = ar.take<bf16>(NC * V);
   a.loss_rows = ar.take<float>(N);
   a.loss = ar.take<float>(1);
   a.dx0 = ar.take<float>(N * d);
@@ -580,15 +582,23 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
     NC_TRY(proj(p, a.a[l], N, F, W + o_down, d, a.x[l + 1], d, NC_EPI_RESID_F32, a.xmid[l], d));
   }
   NC_TRY(rmsnorm_fwd(a.x[L], N, (int)d, a.hf, a.rf, s, pr));
-  NC_TRY(proj(p, a.hf, N, d, p->lm_b, V, a.logits, V, NC_EPI_STORE_BF16, nullptr, 0,
-              "gemm_lmhead"));
-  NC_TRY(ce_fwd_bwd(a.logits, tgt, N, V, a.loss_rows, loss_dev ? loss_dev : a.loss, p->status, s,
-                    pr));
-
-  // ---------------- backward (a.logits now holds dz)
-  NC_TRY(proj_dw(p, a.logits, V, V, a.hf, d, d, N, g->lm, "gemm_lmhead"));
-  NC_TRY(proj_dx(p, a.logits, N, V, p->lm_b, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0,
-                 "gemm_lmhead"));
+  // lm_head + cross-entropy in chunks of lm_chunk tokens: logits of the
+  // chunk, its loss rows and, in place, its dz
+  // (scaled by 1 / N of the whole batch); then dW_lm += dz^T hf and dh = dz
+  // W_lm for the chunk's rows, so only one chunk's logits are ever held.
+  {
+    const int64_t NC = std::min<int64_t>(p->lm_chunk, N);
+    for (int64_t c0 = 0; c0 < N; c0 += NC) {
+      const int64_t nc = std::min(NC, N - c0);
+      NC_TRY(proj(p, a.hf + c0 * d, nc, d, p->lm_b, V, a.logits, V, NC_EPI_STORE_BF16, nullptr, 0,
+                  "gemm_lmhead"));
+      NC_TRY(ce_fwd_bwd(a.logits, tgt + c0, nc, V, 1.0f / (float)N, a.loss_rows + c0, p->status, s, pr));
+      NC_TRY(proj_dw(p, a.logits, V, V, a.hf + c0 * d, d, d, nc, g->lm, "gemm_lmhead"));
+      NC_TRY(proj_dx(p, a.logits, nc, V, p->lm_b, d, a.dh + c0 * d, d, NC_EPI_STORE_BF16, nullptr, 0,
+                     "gemm_lmhead"));
+    }
+    NC_TRY(loss_mean(a.loss_rows, N, loss_dev ? loss_dev : a.loss, s));
+  }
   float* dx = a.dx0;
   float* dxn = a.dx1;
   {
@@ -794,6 +804,11 @@ nc_status nc_gpt_init_config(const nc_model_config* cfg, nc_params** out) {
     return fail(NC_ERR_UNSUPPORTED, "init: fp8 mode needs d >= 256 (depth >= 4)");
   }
   p->fp8 = cfg->fp8 != 0;
+  if (cfg->lm_chunk_tokens < 0) {
+    delete p;
+    return fail(NC_ERR_INVALID_ARG, "init: lm_chunk_tokens must be >= 0");
+  }
+  p->lm_chunk = cfg->lm_chunk_tokens > 0 ? cfg->lm_chunk_tokens : 32768;
   p->window.assign(depth, -1);
   if (cfg->window)
     for (int l = 0; l < depth; ++l) p->window[l] = cfg->window[l] < 0 ? -1 : cfg->window[l];

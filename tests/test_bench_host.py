@@ -46,12 +46,17 @@ def test_training_flops_per_token_at_three_depths():
 
 
 def test_gemm_byte_model_counts_every_launch_of_the_step():
-    """Twelve GEMMs per layer, three for lm_head and thirty for Newton-Schulz
-    (five iterations of three products on two stacks): 273 at depth 20, with
-    231.1 GB of operands and results."""
+    """Twelve GEMMs per layer, three for lm_head per 32768-token chunk (two
+    chunks of the 65536-token batch) and thirty for Newton-Schulz (five
+    iterations of three products on two stacks): 276 at depth 20, with
+    231.5 GB of operands and results; one chunk less reads W_lm twice and
+    accumulates dW_lm once less (8 B per weight)."""
     total, launches = bench.gemm_algorithmic_bytes_per_step()
-    assert launches == 20 * 12 + 3 + 30 == 273
-    assert abs(total / 1e9 - 231.1) < 0.1
+    assert launches == 20 * 12 + 2 * 3 + 30 == 276
+    assert abs(total / 1e9 - 231.5) < 0.1
+    by1, l1 = bench.gemm_algorithmic_bytes_by_class(lm_chunk=bench.B * bench.T)
+    assert l1["lmhead"] == 3
+    assert total - sum(by1.values()) == bench.V * 64 * bench.DEPTH * 8
     # Doubling the batch doubles every activation term and leaves weights.
     t2, _ = bench.gemm_algorithmic_bytes_per_step(batch=2 * bench.B)
     assert total < t2 < 2 * total

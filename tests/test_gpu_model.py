@@ -71,6 +71,30 @@ def test_fwd_bwd_parity_fp8():
         assert e8 < 0.25 and e8 < ex, (i, names[i], e8, ex)
 
 
+def test_chunked_lm_head_matches_the_oracle_and_the_whole_batch():
+    """lm_head + cross-entropy in chunks of 96 tokens (256 tokens: two whole
+    chunks and a ragged one) against the oracle at the model bars, and
+    against the one-chunk step: the same loss rows (identical loss) and the
+    same gradients up to the lm_head weight gradient's fp32 summation order."""
+    depth, B, T, vocab = 4, 2, 128, 32768
+    P = inputs.random_params(depth, seed=150, vocab=vocab)
+    tok, tgt = inputs.token_batch(151, B, T, vocab=vocab)
+    out = []
+    for chunk in (1 << 30, 96):  # one chunk, then chunks of 96
+        m = _gpt(depth, vocab=vocab, lm_chunk_tokens=chunk)
+        m.load(P)
+        out.append((m.fwd_bwd(tok, tgt), m.grads()))
+        m.close()
+    (l0, G0), (l1, G1) = out
+    assert l1 == l0
+    for g0, g1 in zip(G0, G1):
+        assert rel_fro(g1, g0) < 1e-5
+    lref, Gref, _ = oracle.gpt_fwd_bwd(depth, P, tok, tgt, vocab=vocab)
+    assert abs(l1 - lref) / lref < 2e-3
+    for g, r in zip(G1, Gref):
+        assert rel_fro(g, r) < 3e-2
+
+
 def test_fp8_mode_rejects_small_models_and_batches():
     with pytest.raises(nc.NcError):
         _gpt(2, vocab=512, fp8=True)  # d = 128
