@@ -48,9 +48,7 @@ struct Cfg {
 struct Args {
   int M, N, K, batch;
   int tiles_m, tiles_n, split_k, kb_per_split, num_kb;
-  int16_t a_mn, b_mn;
-  int16_t fp8;  // E4M3 operands (pair kernel, K-major): 128-element K slices
-  int16_t unused_;
+  int a_mn, b_mn;
   int epi;
   union {
     struct {
@@ -1106,8 +1104,6 @@ nc_status launch_bn(const nc_gemm_desc& d, int split, int* status, const char* t
   a.split_k = (a.num_kb + a.kb_per_split - 1) / a.kb_per_split;
   a.a_mn = d.a_kmajor ? 0 : 1;
   a.b_mn = d.b_kmajor ? 0 : 1;
-  a.fp8 = 0;
-  a.unused_ = 0;
   a.epi = d.epi;
   a.alpha = d.alpha;
   a.beta = d.beta;
@@ -1187,10 +1183,8 @@ nc_status launch_pair(const nc_gemm_desc& d, int split, int* status, const char*
   a.split_k = (a.num_kb + a.kb_per_split - 1) / a.kb_per_split;
   a.a_mn = d.a_kmajor ? 0 : 1;
   a.b_mn = d.b_kmajor ? 0 : 1;
-  a.fp8 = fp8 ? 1 : 0;
-  a.unused_ = 0;
   a.epi = d.epi;
-  if (fp8) {
+  if (fp8) {  // the operand type itself is the kernel's FP8 template argument
     a.ab_scale = d.ab_scale;
   } else {
     a.alpha = d.alpha;
