@@ -115,6 +115,11 @@ struct nc_params {
   int depth = 0, vocab = 0, d = 0, H = 0, hd = 0, F = 0;
   int Hkv = 0, dkv = 0;     // KV heads and the width of k, v (dkv = 128 Hkv)
   bool fp8 = false;         // block projections on E4M3 operands
+  // The weight-gradient GEMMs of the bf16 backward run on a second stream
+  // (wg), forked from and joined to the step's stream by events: fork[k]
+  // when the GEMM's inputs are ready, done[k] once it has read them.
+  cudaStream_t wg = nullptr;
+  cudaEvent_t wg_fork[4] = {}, wg_done[4] = {};
   int64_t lm_chunk = 32768;  // tokens per lm_head + cross-entropy chunk
   std::vector<int> window;  // per layer: causal left window, -1 = full causal
   cudaStream_t stream = nullptr;
@@ -425,7 +430,7 @@ nc_status proj_dx(nc_params* p, const bf16* dy, int64_t M, int64_t K, const bf16
 // dW[Mo,No] = dy[Ntok,Mo]^T x[Ntok,No] into a zeroed fp32 gradient.
 nc_status proj_dw(nc_params* p, const bf16* dy, int64_t ldy, int64_t Mo, const bf16* x,
                   int64_t ldx, int64_t No, int64_t Ntok, float* dW,
-                  const char* tag = "gemm_wgrad") {
+                  const char* tag = "gemm_wgrad", cudaStream_t st = nullptr) {
   GemmLaunch g{};
   g.status = p->status;
   g.tag = tag;
@@ -434,7 +439,7 @@ nc_status proj_dw(nc_params* p, const bf16* dy, int64_t ldy, int64_t Mo, const b
   g.d.B = x; g.d.ldb = ldx; g.d.b_kmajor = 0;
   g.d.D = dW; g.d.ldd = No;
   g.d.epi = NC_EPI_ACC_F32; g.d.alpha = 1.f; g.d.split_k = 0;  // automatic split
-  return gemm_launch(g, p->stream, p->prof);
+  return gemm_launch(g, st ? st : p->stream, p->prof);
 }
 
 // The backward of layer l in fp8 mode: the layer's eight GEMMs on E4M3
@@ -613,27 +618,60 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
       NC_TRY(layer_bwd_fp8(p, l, B, T, W, G, dx, dxn));  // the gradient stays in dx
       continue;
     }
+    // Each weight gradient goes to the wg stream as soon as its inputs are
+    // ready; the step's stream waits for it only before it overwrites one
+    // of them (dxb, du, dqkv).  wg work of the previous layer is ordered
+    // before this layer's on wg itself.
+    cudaStream_t w = p->wg;
+    auto fork = [&](int k) -> nc_status {
+      NC_CUDA_TRY(cudaEventRecord(p->wg_fork[k], s));
+      NC_CUDA_TRY(cudaStreamWaitEvent(w, p->wg_fork[k], 0));
+      return NC_OK;
+    };
+    auto done = [&](int k) -> nc_status {
+      NC_CUDA_TRY(cudaEventRecord(p->wg_done[k], w));
+      return NC_OK;
+    };
+    auto wait_done = [&](int k) -> nc_status {
+      NC_CUDA_TRY(cudaStreamWaitEvent(s, p->wg_done[k], 0));
+      return NC_OK;
+    };
     // MLP: x_out = xmid + a wdown^T, a = relu(h2 wup^T)^2
-    NC_TRY(proj_dw(p, a.dxb, d, d, a.a[l], F, F, N, G + o_down));
+    NC_TRY(fork(0));
+    NC_TRY(proj_dw(p, a.dxb, d, d, a.a[l], F, F, N, G + o_down, "gemm_wgrad", w));
+    NC_TRY(done(0));
+    if (l < L - 1) NC_TRY(wait_done(1));  // the previous layer's dW_up has read du
     NC_TRY(proj_dx(p, a.dxb, N, d, W + o_down, F, a.du, F, NC_EPI_RELU2_BWD, a.a[l], F));
-    NC_TRY(proj_dw(p, a.du, F, F, a.h2[l], d, d, N, G + o_up));
+    NC_TRY(fork(1));
+    NC_TRY(proj_dw(p, a.du, F, F, a.h2[l], d, d, N, G + o_up, "gemm_wgrad", w));
+    NC_TRY(done(1));
     NC_TRY(proj_dx(p, a.du, N, F, W + o_up, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0));
+    NC_TRY(wait_done(0));  // dW_down has read dxb
     NC_TRY(rmsnorm_bwd(a.dh, a.h2[l], a.r2[l], dx, N, (int)d, dxn, a.dxb, s, pr));
     std::swap(dx, dxn);
     // Attention: xmid = x + o wo^T
-    NC_TRY(proj_dw(p, a.dxb, d, d, a.o[l], d, d, N, G + o_wo));
+    NC_TRY(fork(2));
+    NC_TRY(proj_dw(p, a.dxb, d, d, a.o[l], d, d, N, G + o_wo, "gemm_wgrad", w));
+    NC_TRY(done(2));
     NC_TRY(proj_dx(p, a.dxb, N, d, W + o_wo, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0));
+    if (l < L - 1) NC_TRY(wait_done(3));  // the previous layer's dW_qkv has read dqkv
     // Key side (dK through the k-side RoPE + QK-norm backward, dV, dS^T to
     // a.ds), then the query side (dQ = dS K through the q-side backward).
     NC_TRY(attention_bwd_model(a.qkv[l], Q, a.qkv[l] + d, a.qkv[l] + d + dkv, Q, a.o[l], a.dh, d,
                                a.lse[l], a.delta, a.ds, a.ld_ds, a.dqkv, a.dqkv + d,
                                a.dqkv + d + dkv, Q, B, T, H, Hkv, p->window[l], p->rope, p->rope_T, a.rq[l],
                                a.rk[l], p->status, s, pr));
-    NC_TRY(proj_dw(p, a.dqkv, Q, Q, a.h1[l], d, d, N, G));
+    NC_TRY(fork(3));
+    NC_TRY(proj_dw(p, a.dqkv, Q, Q, a.h1[l], d, d, N, G, "gemm_wgrad", w));
+    NC_TRY(done(3));
     NC_TRY(proj_dx(p, a.dqkv, N, Q, W, d, a.dh, d, NC_EPI_STORE_BF16, nullptr, 0));
+    NC_TRY(wait_done(2));  // dW_o has read dxb
     NC_TRY(rmsnorm_bwd(a.dh, a.h1[l], a.r1[l], dx, N, (int)d, dxn, a.dxb, s, pr));
     std::swap(dx, dxn);
   }
+  // Every weight gradient is complete before the step's stream goes on (the
+  // optimiser reads them); wg's work is ordered, so its last event covers all.
+  if (!p->fp8) NC_CUDA_TRY(cudaStreamWaitEvent(s, p->wg_done[3], 0));
   NC_TRY(embed_scatter(tok, N, dx, V, (int)d, g->wte, s, pr));
   return NC_OK;
 }
@@ -847,6 +885,12 @@ nc_status nc_gpt_init_config(const nc_model_config* cfg, nc_params** out) {
   if (cudaMallocHost(&p->h_loss, sizeof(float)) != cudaSuccess ||
       cudaMallocHost(&p->h_status, sizeof(int)) != cudaSuccess)
     st = fail(NC_ERR_OOM, "pinned host allocation failed");
+  if (st == NC_OK && cudaStreamCreateWithFlags(&p->wg, cudaStreamNonBlocking) != cudaSuccess)
+    st = fail(NC_ERR_CUDA, "weight-gradient stream creation failed");
+  for (int k = 0; k < 4 && st == NC_OK; ++k)
+    if (cudaEventCreateWithFlags(&p->wg_fork[k], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&p->wg_done[k], cudaEventDisableTiming) != cudaSuccess)
+      st = fail(NC_ERR_CUDA, "weight-gradient event creation failed");
   if (st == NC_OK && cudaMemsetAsync(p->mom, 0, sizeof(float) * be, p->stream) != cudaSuccess)
     st = fail(NC_ERR_CUDA, "momentum clear failed");
   if (st == NC_OK && cudaMemsetAsync(p->status, 0, sizeof(int), p->stream) != cudaSuccess)
@@ -880,6 +924,12 @@ void nc_params_free(nc_params* p) {
   if (p->stream) cudaStreamSynchronize(p->stream);
   else cudaDeviceSynchronize();
   drop_graph(p);
+  if (p->wg) cudaStreamSynchronize(p->wg);
+  for (int k = 0; k < 4; ++k) {
+    if (p->wg_fork[k]) cudaEventDestroy(p->wg_fork[k]);
+    if (p->wg_done[k]) cudaEventDestroy(p->wg_done[k]);
+  }
+  if (p->wg) cudaStreamDestroy(p->wg);
   if (p->act.mem) cudaFree(p->act.mem);
   if (p->rope) cudaFree(p->rope);
   if (p->adam) cudaFree(p->adam);
