@@ -611,6 +611,7 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
     NC_TRY(amax_word(p, &am));
     NC_TRY(rmsnorm_bwd(a.dh, a.hf, a.rf, nullptr, N, (int)d, dx, a.dxb, s, pr, am));
   }
+  const bool two_streams = !p->fp8 && !profiler_enabled(pr);
   for (int l = L - 1; l >= 0; --l) {
     const bf16* W = p->blocks_b + l * LS;
     float* G = g->blocks + l * LS;
@@ -621,18 +622,23 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
     // Each weight gradient goes to the wg stream as soon as its inputs are
     // ready; the step's stream waits for it only before it overwrites one
     // of them (dxb, du, dqkv).  wg work of the previous layer is ordered
-    // before this layer's on wg itself.
-    cudaStream_t w = p->wg;
+    // before this layer's on wg itself.  While the per-launch profiler is
+    // on, everything stays on the step's stream, so that each launch's
+    // events time that launch alone.
+    cudaStream_t w = two_streams ? p->wg : s;
     auto fork = [&](int k) -> nc_status {
+      if (!two_streams) return NC_OK;
       NC_CUDA_TRY(cudaEventRecord(p->wg_fork[k], s));
       NC_CUDA_TRY(cudaStreamWaitEvent(w, p->wg_fork[k], 0));
       return NC_OK;
     };
     auto done = [&](int k) -> nc_status {
+      if (!two_streams) return NC_OK;
       NC_CUDA_TRY(cudaEventRecord(p->wg_done[k], w));
       return NC_OK;
     };
     auto wait_done = [&](int k) -> nc_status {
+      if (!two_streams) return NC_OK;
       NC_CUDA_TRY(cudaStreamWaitEvent(s, p->wg_done[k], 0));
       return NC_OK;
     };
@@ -671,7 +677,7 @@ nc_status fwd_bwd(nc_params* p, const int32_t* tokens, const int32_t* targets, i
   }
   // Every weight gradient is complete before the step's stream goes on (the
   // optimiser reads them); wg's work is ordered, so its last event covers all.
-  if (!p->fp8) NC_CUDA_TRY(cudaStreamWaitEvent(s, p->wg_done[3], 0));
+  if (two_streams) NC_CUDA_TRY(cudaStreamWaitEvent(s, p->wg_done[3], 0));
   NC_TRY(embed_scatter(tok, N, dx, V, (int)d, g->wte, s, pr));
   return NC_OK;
 }
