@@ -1,19 +1,28 @@
 // gemm.cu -- the tcgen05 GEMM engine (sm_100a).
 //
-// One persistent CTA per SM walks a list of 128 x BN output tiles.  Warp
-// roles inside the CTA (192 threads):
-//   warp 0      TMA producer: streams 64-wide K slices of A and B into a
-//               STAGES-deep shared-memory ring (128-byte swizzle), one
-//               mbarrier pair (full / empty) per slot;
-//   warp 1      allocates TMEM; one elected thread issues tcgen05.mma
-//               (M = 128, N = BN, K = 16) into a TMEM accumulator and
-//               releases ring slots and accumulators with tcgen05.commit;
-//   warps 2..5  epilogue: tcgen05.ld the accumulator (each thread owns one
-//               row), apply the fused epilogue, store to global memory.
+// Persistent kernels (one CTA, or one CTA pair, per SM) walk a list of
+// output tiles.  Warp roles inside a CTA (320 threads):
+//   warp 0      TMA producer: streams 128-byte K slices of A and B (64 bf16
+//               or 128 E4M3 elements per row) into a STAGES-deep
+//               shared-memory ring (128-byte swizzle), one mbarrier pair
+//               (full / empty) per slot;
+//   warp 1      allocates TMEM; one elected thread issues tcgen05.mma into a
+//               TMEM accumulator and releases ring slots and accumulators
+//               with tcgen05.commit;
+//   warps 2..9  epilogue: tcgen05.ld the accumulator (a thread owns one row
+//               of its warp's 32-row lane quarter and half of the columns),
+//               apply the fused epilogue, store to global memory through a
+//               per-warp staging slot.
+// gemm_tc_kernel computes 128 x BN tiles on one CTA; gemm_tc2_kernel and
+// gemm_tc2_aux_kernel compute 256 x 256 tiles on a cluster of two CTAs with
+// tcgen05.mma.cta_group::2 (each CTA stages its 128 rows of A and of B, the
+// even CTA issues the MMAs), the aux form reading an epilogue operand
+// through a per-warp TMA ring.  The pair kernels also take E4M3 operands
+// (kind::f8f6f4, both K-major, dequantised by the epilogue's alpha).
 // The accumulator is double-buffered in TMEM (2 x BN columns), so the
 // epilogue of tile i overlaps the main loop of tile i + 1.
-// Operands may be K-major or MN-major (transposed) independently, which
-// covers y = x W^T, dx = dy W and dW = dy^T x without transposes.
+// bf16 operands may be K-major or MN-major (transposed) independently,
+// which covers y = x W^T, dx = dy W and dW = dy^T x without transposes.
 // Every mbarrier wait is bounded (see tc.cuh); a timeout sets the device
 // status word and every role drains and exits.
 
