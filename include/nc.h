@@ -361,8 +361,8 @@ typedef struct {
   /* Operand type: 0 bf16; 1 OCP E4M3 (one byte per element, the guide's
    * "--fp8" training, section "1. Modelo GPT", here with one dynamic scale
    * per operand tensor).  E4M3 needs both operands K-major, lda, ldb and
-   * the batch strides multiples of 16, alpha = 1, M > 128, 256-wide column
-   * tiles (N > 128 with no more edge waste than 128-wide ones) and any
+   * the batch strides multiples of 16, alpha = 1, M > 128, N > 128 (it runs
+   * on 256-wide column tiles, the last one ragged if need be) and any
    * epilogue but NC_EPI_AXPBY_BF16; the product is multiplied by
    * 1 / (ab_scale[0] * ab_scale[1]), the scales nc_op_fp8_quantize wrote
    * for A and B (two device floats). */

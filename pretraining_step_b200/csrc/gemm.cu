@@ -1330,7 +1330,9 @@ nc_status gemm_launch(const GemmLaunch& g, cudaStream_t s, Profiler* prof) {
   const int waste128 = ((d.N + 127) / 128) * 128 - d.N;
   // (the RoPE/QK-norm epilogue needs 256-wide tiles: each warp-half is a head)
   // (a symmetric output walks square 256 x 256 tiles whatever the edge waste)
-  const bool bn256 = rope || g.symmetric || (d.N > 128 && waste256 <= waste128);
+  // (E4M3 operands run only on the 256-wide pair kernel, whatever the edge
+  // waste: d = 1664 at depth 26 leaves half a column tile)
+  const bool bn256 = rope || g.symmetric || (d.N > 128 && (waste256 <= waste128 || fp8));
   const int bn = bn256 ? 256 : 128;
   const int num_kb = (d.K + (fp8 ? 2 * BK : BK) - 1) / (fp8 ? 2 * BK : BK);
   const double operand_bytes = (fp8 ? 1.0 : 2.0) * ((double)d.M + d.N) * d.K * d.batch;
@@ -1358,7 +1360,7 @@ nc_status gemm_launch(const GemmLaunch& g, cudaStream_t s, Profiler* prof) {
     return launch_pair<false, false>(d, split, g.status, g.tag, s, prof, g.symmetric);
   }
   if (fp8)
-    return fail(NC_ERR_INVALID_ARG, "gemm: E4M3 operands need M > 128 and 256-wide column tiles");
+    return fail(NC_ERR_INVALID_ARG, "gemm: E4M3 operands need M > 128 and N > 128");
   if (rope) return launch_bn<256, true>(d, split, g.status, g.tag, s, prof);
   return bn256 ? launch_bn<256, false>(d, split, g.status, g.tag, s, prof)
                : launch_bn<128, false>(d, split, g.status, g.tag, s, prof);

@@ -42,7 +42,8 @@ def test_fwd_bwd_parity(depth, B, T, vocab):
         assert rel_fro(g, r) < 3e-2, (i, names[i], rel_fro(g, r))
 
 
-def test_fwd_bwd_parity_fp8():
+@pytest.mark.parametrize("depth,B,T", [(4, 2, 128), (6, 1, 256)])
+def test_fwd_bwd_parity_fp8(depth, B, T):
     """The fp8 mode (E4M3 block projections, one dynamic scale per operand
     tensor) against the oracle's fp8 model.  Both sides quantise bf16
     activations that differ by rounding, so single elements land on
@@ -52,8 +53,9 @@ def test_fwd_bwd_parity_fp8():
     fp8 and exact models.  Bars: the loss at 2e-3; every gradient closer to
     the oracle's fp8 gradient than to its exact one (the quantisation is
     reproduced, not just tolerated) and within 0.25, far below what a wrong
-    scale, operand or transpose gives (order 1)."""
-    depth, B, T, vocab = 4, 2, 128, 32768
+    scale, operand or transpose gives (order 1).  Depth 6 (d = 384) runs the
+    E4M3 GEMMs on a ragged last column tile."""
+    vocab = 32768
     P = inputs.random_params(depth, seed=140, vocab=vocab)
     tok, tgt = inputs.token_batch(141, B, T, vocab=vocab)
     m = _gpt(depth, vocab=vocab, fp8=True)
