@@ -1330,9 +1330,13 @@ nc_status gemm_launch(const GemmLaunch& g, cudaStream_t s, Profiler* prof) {
   const int waste128 = ((d.N + 127) / 128) * 128 - d.N;
   // (the RoPE/QK-norm epilogue needs 256-wide tiles: each warp-half is a head)
   // (a symmetric output walks square 256 x 256 tiles whatever the edge waste)
-  // (E4M3 operands run only on the 256-wide pair kernel, whatever the edge
-  // waste: d = 1664 at depth 26 leaves half a column tile)
-  const bool bn256 = rope || g.symmetric || (d.N > 128 && (waste256 <= waste128 || fp8));
+  // The 256-wide pair kernel also when its last column tile is ragged, as
+  // long as the padding stays within an eighth of the columns computed
+  // (d = 1664 at depth 26: 128 of 1792): it outruns 128-wide single-CTA
+  // tiles by more than that.  E4M3 operands run only on the pair kernel.
+  const int n256 = ((d.N + 255) / 256) * 256;
+  const bool bn256 = rope || g.symmetric ||
+                     (d.N > 128 && (waste256 <= waste128 || 8 * waste256 <= n256 || fp8));
   const int bn = bn256 ? 256 : 128;
   const int num_kb = (d.K + (fp8 ? 2 * BK : BK) - 1) / (fp8 ? 2 * BK : BK);
   const double operand_bytes = (fp8 ? 1.0 : 2.0) * ((double)d.M + d.N) * d.K * d.batch;
