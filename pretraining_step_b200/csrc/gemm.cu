@@ -1325,7 +1325,7 @@ nc_status gemm_launch(const GemmLaunch& g, cudaStream_t s, Profiler* prof) {
   int split = d.split_k;
   if (split != 1 && d.epi != NC_EPI_ACC_F32)
     return fail(NC_ERR_INVALID_ARG, "gemm: split_k > 1 needs the accumulate epilogue");
-  // N tile: 256 unless 128 wastes less of the last column tile.
+  // N tile: 256 unless 128 wastes less of the last column tile (but see below).
   const int waste256 = ((d.N + 255) / 256) * 256 - d.N;
   const int waste128 = ((d.N + 127) / 128) * 128 - d.N;
   // (the RoPE/QK-norm epilogue needs 256-wide tiles: each warp-half is a head)
